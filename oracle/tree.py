@@ -1,0 +1,126 @@
+"""EAGLE-2 dynamic draft tree, brute force (fp64).
+
+Source: "EAGLE" notes (s1mplewind), EAGLE-2 sections:
+  * "Well-Calibrated Draft Model": the draft confidence of token x is
+    c(x) = exp(logit_x) / sum_i exp(logit_i).
+  * "Expansion of tree": a token's value is its global acceptance
+    V_i = product of the confidences on the path root -> i (rejecting a token
+    cuts its whole subtree); each level keeps the top-k tokens by V and
+    expands each kept token's top-k children.
+  * "Reranking Nodes": after expansion, keep the m tokens with the largest V
+    over all candidates.
+
+Readings the pages leave open, taken here:
+  * m does not count the root; the root is the last accepted token.
+  * Draft rows without a draft model: row 0 is the root's distribution and the
+    node in frontier slot s of level l (1 <= l <= depth-1) owns row
+    1 + (l-1)*k + s.  The frontier slot is the node's rank in that level's
+    selection, ordered by (-logV, candidate id).  R = 1 + (depth-1)*k rows.
+  * Candidate id (gid): level 1 uses gid = r (child rank r of the root);
+    level l >= 2 uses gid = k + (l-2)*k*k + s*k + r, with s the parent's
+    frontier slot and r the child's rank in its row.  Every ordering is by
+    (-logV, gid): ties go to the lower id, so a parent always precedes its child.
+  * V is ranked in log space: logV = sum of log-confidences along the path,
+    i.e. log of the product.  A child's logV is at most its parent's, so the
+    kept set is closed under "parent of".
+  * The top-k children of a row are its k largest raw logits, ties to the
+    lower token id (the same order as by log-confidence).
+  * Output nodes are numbered 1..n in ascending gid (parents before children,
+    siblings in rank order); parent 0 is the root.
+"""
+from __future__ import annotations
+
+from typing import Dict, List
+
+import numpy as np
+
+from .common import logsumexp, near_tie
+
+
+def _row_topk(row: np.ndarray, k: int) -> np.ndarray:
+    """Token ids of the k largest values, ties to the lower id (library sort)."""
+    order = np.lexsort((np.arange(row.shape[0]), -row))
+    return order[:k]
+
+
+def _sort_key(c):
+    return (-c["logV"], c["gid"])
+
+
+def _flag_adjacent(sorted_cands, upto: int, kind: str, level: int, out: list):
+    """Record near-ties between neighbours of a selection (positions < upto+1)."""
+    for i in range(min(upto, len(sorted_cands) - 1)):
+        a, b = sorted_cands[i], sorted_cands[i + 1]
+        if a["parent"] == b["parent"]:
+            # siblings: logV differ only through their raw logits, whose order
+            # (ties to the lower rank, hence lower gid) no rounding can change
+            continue
+        if near_tie(a["logV"], b["logV"]):
+            out.append({"kind": kind, "level": level, "gids": (a["gid"], b["gid"]),
+                        "logV": (a["logV"], b["logV"])})
+
+
+def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
+    """Build one sequence's tree from its R = 1 + (depth-1)*k draft rows (fp64)."""
+    logits = np.asarray(logits, dtype=np.float64)
+    R, V = logits.shape
+    assert depth >= 1 and 1 <= k <= V and m >= 1
+    assert R == 1 + (depth - 1) * k, (R, depth, k)
+
+    row_lse = np.array([logsumexp(logits[r]) for r in range(R)])
+    topk = [_row_topk(logits[r], k) for r in range(R)]
+
+    near_ties: List[dict] = []
+    all_cands: List[dict] = []
+
+    def make(row, r, gid, level, parent):
+        tok = int(topk[row][r])
+        lp = logits[row, tok] - row_lse[row]          # log confidence, <= 0
+        base = 0.0 if parent is None else parent["logV"]
+        return {"gid": gid, "level": level, "token": tok, "logit": logits[row, tok],
+                "lp": lp, "logV": base + lp, "parent": None if parent is None else parent["gid"],
+                "pnode": parent, "slot": -1, "row": -1}
+
+    # level 1: the root's k children
+    level_cands = [make(0, r, r, 1, None) for r in range(k)]
+    all_cands += level_cands
+    for level in range(2, depth + 1):
+        ranked = sorted(level_cands, key=_sort_key)
+        _flag_adjacent(ranked, k, "frontier", level - 1, near_ties)
+        frontier = ranked[:k]
+        nxt = []
+        off = k + (level - 2) * k * k
+        for s, parent in enumerate(frontier):
+            parent["slot"] = s
+            parent["row"] = 1 + (level - 2) * k + s
+            for r in range(k):
+                nxt.append(make(parent["row"], r, off + s * k + r, level, parent))
+        level_cands = nxt
+        all_cands += level_cands
+
+    P = len(all_cands)
+    assert P == k + (depth - 1) * k * k
+    n = min(m, P)
+    ranked = sorted(all_cands, key=_sort_key)
+    _flag_adjacent(ranked[n - 1:], 1, "rerank", 0, near_ties)
+    kept = sorted(ranked[:n], key=lambda c: c["gid"])
+    node_of = {c["gid"]: i + 1 for i, c in enumerate(kept)}
+
+    tokens = np.array([c["token"] for c in kept], dtype=np.int64)
+    parents = np.array([0 if c["parent"] is None else node_of[c["parent"]] for c in kept],
+                       dtype=np.int64)
+    depth_arr = np.array([c["level"] for c in kept], dtype=np.int64)
+    logV = np.array([c["logV"] for c in kept], dtype=np.float64)
+    gid = np.array([c["gid"] for c in kept], dtype=np.int64)
+    draft_row = np.full(n + 1, -1, dtype=np.int64)
+    draft_row[0] = 0
+    for i, c in enumerate(kept):
+        draft_row[i + 1] = c["row"]
+    return {"tokens": tokens, "parents": parents, "depth": depth_arr, "logV": logV,
+            "gid": gid, "draft_row": draft_row, "row_lse": row_lse, "n": n, "P": P,
+            "near_ties": near_ties}
+
+
+def build_trees(logits_b: np.ndarray, depth: int, k: int, m: int) -> List[Dict]:
+    """One tree per sequence of a [B][R][V] fp64 batch."""
+    return [build_tree(logits_b[b], depth, k, m) for b in range(logits_b.shape[0])]
