@@ -1,0 +1,267 @@
+"""ctypes binding of libeagle_tree.so (argument marshalling only).
+
+Every function here checks shapes, allocates outputs / workspaces with torch
+on the tensors' device and calls the C entry point of the same name on the
+current CUDA stream.  All arithmetic happens in the library's kernels.  There
+is no fallback: if the shared library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libeagle_tree.so")
+
+F32, BF16 = 0, 1
+MAX_NODES, MAX_TOPK, MAX_DEPTH, MAX_POOL = 128, 32, 16, 4096
+
+_c_p = ctypes.c_void_p
+_c_i = ctypes.c_int
+_c_ll = ctypes.c_longlong
+_c_sz = ctypes.c_size_t
+_c_f = ctypes.c_float
+
+
+class EagleError(RuntimeError):
+    pass
+
+
+class TreeStruct(ctypes.Structure):
+    _fields_ = [("tokens", _c_p), ("parents", _c_p), ("depth", _c_p), ("logV", _c_p),
+                ("gid", _c_p), ("draft_row", _c_p), ("row_lse", _c_p)]
+
+
+_SIGS = {
+    "eagle_status_string": (ctypes.c_char_p, [_c_i]),
+    "eagle_last_cuda_error": (ctypes.c_char_p, []),
+    "eagle_version": (_c_i, []),
+    "eagle_row_stats_workspace_bytes": (_c_sz, [_c_ll, _c_i, _c_i, _c_i]),
+    "eagle_row_stats": (_c_i, [_c_p, _c_i, _c_ll, _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "eagle_tree_build_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
+    "eagle_tree_build": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
+                                ctypes.POINTER(TreeStruct), ctypes.POINTER(_c_i), _c_p, _c_sz, _c_p]),
+    "eagle_tree_mask": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_p, _c_p, _c_p]),
+    "eagle_tree_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i]),
+    "eagle_tree_attention": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i,
+                                    _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p, _c_sz, _c_p]),
+    "eagle_accept_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
+    "eagle_accept": (_c_i, [_c_p, _c_i, _c_p, _c_i, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i,
+                            _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the shared library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise EagleError(f"{LIB_PATH} is missing: build it with eagle_tree_verification_dynamic_b200.build")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def exported_names():
+    return list(_SIGS)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = lib().eagle_status_string(status).decode()
+        cuda = lib().eagle_last_cuda_error().decode()
+        raise EagleError(f"{what}: {msg}" + (f" ({cuda})" if cuda and status == 7 else ""))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise EagleError(f"unsupported logits dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise EagleError("tensors must be on a CUDA device")
+            if not t.is_contiguous():
+                raise EagleError("tensors must be contiguous")
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns blocks aligned to at least 512 bytes
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- row stats
+def row_stats(logits: torch.Tensor, k: int, want_lse: bool = True):
+    """logits [rows][V] -> (topk_token [rows][k] int32, topk_logit [rows][k] f32, lse [rows] f64)."""
+    _need_cuda(logits)
+    rows, V = logits.reshape(-1, logits.shape[-1]).shape
+    dev = logits.device
+    tok = torch.empty(rows, k, dtype=torch.int32, device=dev)
+    val = torch.empty(rows, k, dtype=torch.float32, device=dev)
+    lse = torch.empty(rows, dtype=torch.float64, device=dev) if want_lse else None
+    dt = _dtype_code(logits)
+    nb = lib().eagle_row_stats_workspace_bytes(rows, V, dt, k)
+    ws = _workspace(nb, dev)
+    _check(lib().eagle_row_stats(_ptr(logits), dt, rows, V, k, _ptr(tok), _ptr(val), _ptr(lse),
+                                 _ptr(ws), nb, _stream(dev)), "eagle_row_stats")
+    return tok, val, lse
+
+
+# --------------------------------------------------------------- tree build
+@dataclass
+class Tree:
+    tokens: torch.Tensor     # [B][n] int32
+    parents: torch.Tensor    # [B][n] int32
+    depth: torch.Tensor      # [B][n] int32
+    logV: torch.Tensor       # [B][n] float32
+    gid: torch.Tensor        # [B][n] int32
+    draft_row: torch.Tensor  # [B][n+1] int32
+    row_lse: torch.Tensor    # [B][R] float64
+    n: int
+
+    def struct(self) -> TreeStruct:
+        return TreeStruct(*[ctypes.c_void_p(t.data_ptr()) for t in
+                            (self.tokens, self.parents, self.depth, self.logV, self.gid,
+                             self.draft_row, self.row_lse)])
+
+
+def pool_size(depth: int, k: int) -> int:
+    return k + (depth - 1) * k * k
+
+
+def alloc_tree(B: int, R: int, depth: int, k: int, m: int, device) -> Tree:
+    n = min(m, pool_size(depth, k))
+    i32 = dict(dtype=torch.int32, device=device)
+    return Tree(tokens=torch.empty(B, n, **i32), parents=torch.empty(B, n, **i32),
+                depth=torch.empty(B, n, **i32), logV=torch.empty(B, n, dtype=torch.float32, device=device),
+                gid=torch.empty(B, n, **i32), draft_row=torch.empty(B, n + 1, **i32),
+                row_lse=torch.empty(B, R, dtype=torch.float64, device=device), n=n)
+
+
+def tree_build_workspace_bytes(B, R, V, dtype_code, k) -> int:
+    return lib().eagle_tree_build_workspace_bytes(B, R, V, dtype_code, k)
+
+
+def tree_build_into(draft_logits: torch.Tensor, depth: int, k: int, m: int, tree: Tree,
+                    ws: torch.Tensor) -> int:
+    B, R, V = draft_logits.shape
+    dt = _dtype_code(draft_logits)
+    st = tree.struct()
+    n_out = _c_i(0)
+    _check(lib().eagle_tree_build(_ptr(draft_logits), dt, B, R, V, depth, k, m, ctypes.byref(st),
+                                  ctypes.byref(n_out), _ptr(ws), ws.numel(), _stream(draft_logits.device)),
+           "eagle_tree_build")
+    return n_out.value
+
+
+def tree_build(draft_logits: torch.Tensor, depth: int, k: int, m: int) -> Tree:
+    """draft_logits [B][R][V] (f32 or bf16) -> Tree."""
+    _need_cuda(draft_logits)
+    B, R, V = draft_logits.shape
+    tree = alloc_tree(B, R, depth, k, m, draft_logits.device)
+    nb = tree_build_workspace_bytes(B, R, V, _dtype_code(draft_logits), k)
+    tree_build_into(draft_logits, depth, k, m, tree, _workspace(nb, draft_logits.device))
+    return tree
+
+
+# ---------------------------------------------------------------- tree mask
+def tree_mask_into(parents, depth, prefix_len, mask, pos):
+    B, n = parents.shape
+    _check(lib().eagle_tree_mask(_ptr(parents), _ptr(depth), _ptr(prefix_len), B, n, _ptr(mask), _ptr(pos),
+                                 _stream(parents.device)), "eagle_tree_mask")
+
+
+def tree_mask(parents: torch.Tensor, depth: Optional[torch.Tensor] = None,
+              prefix_len: Optional[torch.Tensor] = None):
+    """parents [B][n] -> (mask [B][n][2] uint64 as int64, pos [B][n] int32 or None)."""
+    _need_cuda(parents, depth, prefix_len)
+    B, n = parents.shape
+    mask = torch.empty(B, n, 2, dtype=torch.int64, device=parents.device)
+    pos = torch.empty(B, n, dtype=torch.int32, device=parents.device) if depth is not None else None
+    tree_mask_into(parents, depth, prefix_len, mask, pos)
+    return mask, pos
+
+
+# ----------------------------------------------------------- tree attention
+def attention_workspace_bytes(B, n, Hq, Hkv, D, Lmax, window=0) -> int:
+    return lib().eagle_tree_attention_workspace_bytes(B, n, Hq, Hkv, D, Lmax, window)
+
+
+def tree_attention_into(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos, out, ws,
+                        window: int = 0, scale: float = 0.0):
+    B, n, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    _check(lib().eagle_tree_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), Lmax,
+                                      _ptr(k_tree), _ptr(v_tree), _ptr(mask), _ptr(pos), B, n, Hq, Hkv, D,
+                                      window, scale, _ptr(out), _ptr(ws), ws.numel(), _stream(q.device)),
+           "eagle_tree_attention")
+
+
+def tree_attention(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos=None, window: int = 0,
+                   scale: float = 0.0) -> torch.Tensor:
+    """q [B][n][Hq][D] bf16, caches [B][Hkv][Lmax][D] bf16, tree K/V [B][n][Hkv][D] bf16 -> out bf16."""
+    _need_cuda(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos)
+    for t in (q, k_cache, v_cache, k_tree, v_tree):
+        if t.dtype != torch.bfloat16:
+            raise EagleError("attention tensors must be bf16")
+    B, n, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    out = torch.empty_like(q)
+    ws = _workspace(attention_workspace_bytes(B, n, Hq, Hkv, D, Lmax, window), q.device)
+    tree_attention_into(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos, out, ws, window, scale)
+    return out
+
+
+# -------------------------------------------------------------------- accept
+def accept_workspace_bytes(B, n, V, dtype_code) -> int:
+    return lib().eagle_accept_workspace_bytes(B, n, V, dtype_code)
+
+
+def accept_into(target_logits, tokens, parents, draft_row, depth, uniforms, draft_logits, draft_lse,
+                accepted_len, path, bonus, ws):
+    B, n1, V = target_logits.shape
+    n = n1 - 1
+    R = draft_logits.shape[1] if draft_logits is not None else 0
+    ddt = _dtype_code(draft_logits) if draft_logits is not None else 0
+    _check(lib().eagle_accept(_ptr(target_logits), _dtype_code(target_logits), _ptr(draft_logits), ddt,
+                              _ptr(draft_lse), R, _ptr(tokens), _ptr(parents), _ptr(draft_row), _ptr(uniforms),
+                              B, n, V, depth, _ptr(accepted_len), _ptr(path), _ptr(bonus), _ptr(ws), ws.numel(),
+                              _stream(target_logits.device)), "eagle_accept")
+
+
+def accept(target_logits, tokens, parents, draft_row, depth: int, uniforms=None, draft_logits=None,
+           draft_lse=None):
+    """-> (accepted_len [B] int32, path [B][depth] int32, bonus [B] int32)."""
+    _need_cuda(target_logits, tokens, parents, draft_row, uniforms, draft_logits, draft_lse)
+    B, n1, V = target_logits.shape
+    dev = target_logits.device
+    acc = torch.empty(B, dtype=torch.int32, device=dev)
+    path = torch.empty(B, depth, dtype=torch.int32, device=dev)
+    bonus = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = _workspace(accept_workspace_bytes(B, n1 - 1, V, _dtype_code(target_logits)), dev)
+    accept_into(target_logits, tokens, parents, draft_row, depth, uniforms, draft_logits, draft_lse,
+                acc, path, bonus, ws)
+    return acc, path, bonus

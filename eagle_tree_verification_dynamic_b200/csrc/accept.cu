@@ -1,0 +1,331 @@
+// Acceptance walk ("EAGLE" notes, EAGLE-2 "Well-Calibrated Draft Model":
+// acceptance min(1, P_target/P_draft), greedy = argmaxes agree; "Что такое
+// EAGLE-3", section 4 steps 3-4: on rejection the target samples from the
+// adjusted distribution and the longest accepted prefix wins).
+//
+// Target rows first go through the vocabulary sweep (row_stats.cu, k = 1):
+// argmax and log-sum-exp per row.  Then one thread-block cluster per sequence
+// walks its tree.  Every CTA of the cluster evaluates the same scalar
+// decisions from the same data, so they stay in step; the vocabulary-wide
+// quantities a decision needs are computed cooperatively, each CTA on a
+// contiguous slice of the vocabulary, and combined through distributed shared
+// memory in a fixed order (so every CTA sees bit-identical totals):
+//   * after a rejection at node j the current target becomes
+//     max(0, p - q) / Z.  After r rejections it equals
+//     max(0, p - t q) / F(t) with F(t) = sum_x max(0, p(x) - t q(x)),
+//     t_0 = 0 (F = 1), t_{r+1} = t_r + F(t_r); one sweep per rejection gives
+//     F at the new t;
+//   * the bonus token is the smallest x whose cumulative weight exceeds
+//     u_res * total (inverse CDF), found by a prefix scan over the slices.
+#include <cooperative_groups.h>
+
+#include "eagle_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace eagle {
+
+constexpr int kAcceptThreads = 512;
+constexpr int kAcceptWarps = kAcceptThreads / 32;
+
+template <typename T>
+__device__ __forceinline__ float load_logit(const T* p) { return Elem<T>::load(p); }
+
+struct SweepArgs {
+  const void* trow;   // target row j
+  const void* drow;   // draft row draft_row[j] (unused when t == 0)
+  Split2 lse_t, lse_d, t;
+  bool use_q;         // false: weights are p itself
+};
+
+// Weight of token x under the current target: p(x), or max(0, p(x) - t q(x)).
+template <typename T>
+__device__ __forceinline__ float sweep_weight(const SweepArgs& a, int x) {
+  const float p = exp_minus(load_logit(static_cast<const T*>(a.trow) + x), a.lse_t);
+  if (!a.use_q) return p;
+  const float q = exp_minus(load_logit(static_cast<const T*>(a.drow) + x), a.lse_d);
+  return fmaxf(0.f, fmaf(-a.t.lo, q, fmaf(-a.t.hi, q, p)));
+}
+
+struct AcceptSmem {
+  int tok[EAGLE_MAX_NODES];
+  int par[EAGLE_MAX_NODES];
+  int drow[EAGLE_MAX_NODES + 1];
+  double warp_part[kAcceptWarps];
+  double lane_sum[kAcceptThreads];
+  double prefix[kAcceptThreads + 1];
+  double cta_total;
+};
+
+// Deterministic block sum; result valid in every thread.
+__device__ double block_sum(double v, AcceptSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum_d(v);
+  __syncthreads();
+  if (lane == 0) sm.warp_part[warp] = v;
+  __syncthreads();
+  double s = 0.0;
+  for (int w = 0; w < kAcceptWarps; ++w) s += sm.warp_part[w];
+  return s;
+}
+
+// Cluster-wide total of one double per CTA, summed in rank order.
+__device__ double cluster_sum(double cta_value, AcceptSmem& sm, cg::cluster_group& cluster,
+                              double* prefix_of_rank) {
+  if (threadIdx.x == 0) sm.cta_total = cta_value;
+  cluster.sync();
+  const unsigned nb = cluster.num_blocks();
+  const unsigned me = cluster.block_rank();
+  double acc = 0.0;
+  for (unsigned r = 0; r < nb; ++r) {
+    if (r == me && prefix_of_rank) *prefix_of_rank = acc;
+    acc += *cluster.map_shared_rank(&sm.cta_total, r);
+  }
+  cluster.sync();
+  return acc;
+}
+
+template <typename T>
+__device__ double sweep_total(const SweepArgs& a, int V, AcceptSmem& sm, cg::cluster_group& cluster) {
+  const int nt = (int)cluster.num_blocks() * kAcceptThreads;
+  const int gt = (int)cluster.block_rank() * kAcceptThreads + threadIdx.x;
+  const int seg = (V + nt - 1) / nt;
+  const int x0 = min(V, gt * seg), x1 = min(V, x0 + seg);
+  double acc = 0.0;
+  for (int x = x0; x < x1; ++x) acc += (double)sweep_weight<T>(a, x);
+  return cluster_sum(block_sum(acc, sm), sm, cluster, nullptr);
+}
+
+// Inverse CDF over the weights: smallest x with cumsum_x > u * total.  Writes
+// the token to *out from the one thread that owns the crossing; returns the
+// total weight (every thread).
+template <typename T>
+__device__ double sweep_sample(const SweepArgs& a, int V, float u, AcceptSmem& sm,
+                               cg::cluster_group& cluster, int32_t* out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nt = (int)cluster.num_blocks() * kAcceptThreads;
+  const int gt = (int)cluster.block_rank() * kAcceptThreads + tid;
+  (void)lane;
+  const int seg = (V + nt - 1) / nt;
+  const int x0 = min(V, gt * seg), x1 = min(V, x0 + seg);
+  double mine = 0.0;
+  for (int x = x0; x < x1; ++x) mine += (double)sweep_weight<T>(a, x);
+  // Block exclusive prefix of the per-thread sums, summed serially (lane order
+  // within a warp, then warp order) so the prefixes never decrease and the
+  // ownership intervals [prefix[t], prefix[t+1]) tile [0, total) exactly.
+  sm.lane_sum[tid] = mine;
+  __syncthreads();
+  if (lane == 0) {
+    double acc = 0.0;
+    for (int l = 0; l < 32; ++l) { const double v = sm.lane_sum[tid + l]; sm.prefix[tid + l] = acc; acc += v; }
+    sm.warp_part[warp] = acc;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double acc = 0.0;
+    for (int w = 0; w < kAcceptWarps; ++w) { const double v = sm.warp_part[w]; sm.warp_part[w] = acc; acc += v; }
+    sm.prefix[kAcceptThreads] = acc;
+  }
+  __syncthreads();
+  const double excl = sm.prefix[tid];
+  __syncthreads();
+  sm.prefix[tid] = sm.warp_part[warp] + excl;
+  __syncthreads();
+  double my_off = 0.0;
+  const double cta_total = sm.prefix[kAcceptThreads];
+  const double total = cluster_sum(cta_total, sm, cluster, &my_off);
+  if (total > 0.0) {
+    const double thr = (double)u * total;
+    const double start = my_off + sm.prefix[tid];
+    const double end = my_off + sm.prefix[tid + 1];
+    if (start <= thr && thr < end) {
+      double run = 0.0;
+      int pick = -1, last_nz = -1;
+      for (int x = x0; x < x1; ++x) {
+        const float w = sweep_weight<T>(a, x);
+        if (w > 0.f) last_nz = x;
+        run += (double)w;
+        if (my_off + (sm.prefix[tid] + run) > thr) { pick = x; break; }
+      }
+      *out = pick >= 0 ? pick : last_nz;
+    }
+  }
+  return total;
+}
+
+template <typename T>
+__device__ __forceinline__ int argmax_of_row(const ChunkStat* st, const uint64_t* keys, int t_chunks,
+                                             bool want_lse, double* lse) {
+  uint64_t key = 0;
+  warp_finalize_row(st, keys, t_chunks, 1, want_lse, lse, &key);
+  key = __shfl_sync(kFull, key, 0);
+  return key ? key_index(key) : 0;
+}
+
+template <typename T, bool STOCH>
+__global__ void __launch_bounds__(kAcceptThreads)
+accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const double* __restrict__ dlse,
+                   int R, int V, int n, int depth, const ChunkStat* __restrict__ tstats,
+                   const uint64_t* __restrict__ tkeys, int t_chunks, const int32_t* __restrict__ tokens,
+                   const int32_t* __restrict__ parents, const int32_t* __restrict__ draft_row,
+                   const float* __restrict__ uniforms, int32_t* __restrict__ accepted_len,
+                   int32_t* __restrict__ path, int32_t* __restrict__ bonus) {
+  __shared__ AcceptSmem sm;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int b = blockIdx.x / CL;
+  const bool leader = cluster.block_rank() == 0 && threadIdx.x == 0;
+  const int tid = threadIdx.x;
+
+  for (int i = tid; i < n; i += kAcceptThreads) {
+    sm.tok[i] = tokens[(size_t)b * n + i];
+    sm.par[i] = parents[(size_t)b * n + i];
+  }
+  for (int i = tid; i <= n; i += kAcceptThreads) {
+    const int r = draft_row[(size_t)b * (n + 1) + i];
+    sm.drow[i] = (r >= 0 && r < R) ? r : -1;  // an out-of-range row counts as "not expanded"
+  }
+  __syncthreads();
+
+  const size_t trow0 = (size_t)b * (n + 1);
+  auto row_stat = [&](int j) { return tstats + (trow0 + j) * t_chunks; };
+  auto row_keys = [&](int j) { return tkeys + (trow0 + j) * t_chunks; };
+  const float* u_acc = STOCH ? uniforms + (size_t)b * 2 * (n + 1) : nullptr;
+  const float* u_res = STOCH ? u_acc + (n + 1) : nullptr;
+
+  int j = 0, plen = 0;
+  double lse_t = 0.0;
+  int amax = argmax_of_row<T>(row_stat(0), row_keys(0), t_chunks, STOCH, &lse_t);
+  double t = 0.0, F = 1.0;
+  bool rejected_here = false;
+
+  while (plen < depth) {
+    int moved_to = -1;
+    if (!STOCH) {
+      for (int c = 1; c <= n; ++c)
+        if (sm.par[c - 1] == j && sm.tok[c - 1] == amax) { moved_to = c; break; }
+    } else {
+      const int r = sm.drow[j];
+      const T* trow = tgt + (trow0 + j) * (size_t)V;
+      const T* drow = r >= 0 ? dft + ((size_t)b * R + r) * (size_t)V : nullptr;
+      const double lse_d = r >= 0 ? dlse[(size_t)b * R + r] : 0.0;
+      // children of j in node order
+      int c = 1;
+      while (true) {
+        while (c <= n && sm.par[c - 1] != j) ++c;
+        if (c > n || r < 0) break;
+        const int x = sm.tok[c - 1];
+        double ratio = 0.0;  // a token outside the vocabulary is never accepted
+        if (x >= 0 && x < V) {
+          const double px = exp((double)load_logit(trow + x) - lse_t);
+          const double qx = exp((double)load_logit(drow + x) - lse_d);
+          const double rho = t == 0.0 ? px : fmax(0.0, px - t * qx);
+          ratio = rho / (F * qx);
+        }
+        if ((double)u_acc[c] < ratio) { moved_to = c; break; }
+        // rejected: the current target becomes max(0, p - t' q) / F(t')
+        t += F;
+        rejected_here = true;
+        int nc = c + 1;
+        while (nc <= n && sm.par[nc - 1] != j) ++nc;
+        if (nc <= n) {  // another sibling will be tested: need F(t)
+          SweepArgs a;
+          a.trow = trow; a.drow = drow; a.use_q = true;
+          a.lse_t.set(lse_t); a.lse_d.set(lse_d); a.t.set(t);
+          F = sweep_total<T>(a, V, sm, cluster);
+          if (!(F > 0.0)) break;  // p == q left nothing: keep the walk here
+        }
+        c = nc;
+      }
+    }
+    if (moved_to < 0) break;
+    if (leader) path[(size_t)b * depth + plen] = moved_to;
+    ++plen;
+    j = moved_to;
+    t = 0.0;
+    F = 1.0;
+    rejected_here = false;
+    amax = argmax_of_row<T>(row_stat(j), row_keys(j), t_chunks, STOCH, &lse_t);
+  }
+
+  if (leader) {
+    accepted_len[b] = plen;
+    for (int i = plen; i < depth; ++i) path[(size_t)b * depth + i] = -1;
+  }
+  if (!STOCH) {
+    if (leader) bonus[b] = amax;
+    return;
+  }
+  const int r = sm.drow[j];
+  SweepArgs a;
+  a.trow = tgt + (trow0 + j) * (size_t)V;
+  a.drow = r >= 0 ? dft + ((size_t)b * R + r) * (size_t)V : nullptr;
+  a.use_q = rejected_here && r >= 0;
+  a.lse_t.set(lse_t);
+  a.lse_d.set(r >= 0 ? dlse[(size_t)b * R + r] : 0.0);
+  a.t.set(t);
+  const double total = sweep_sample<T>(a, V, u_res[j], sm, cluster, bonus + b);
+  if (!(total > 0.0) && leader) bonus[b] = amax;  // nothing left to sample from
+}
+
+// ------------------------------------------------------------------- host
+size_t accept_ws_bytes(int B, int n, int V, int dtype) {
+  return row_stats_ws_bytes((long long)B * (n + 1), V, dtype_bytes(dtype), 1);
+}
+
+static int accept_cluster_size(int V) {
+  int cl = V / 8192;
+  if (cl < 1) cl = 1;
+  if (cl > 8) cl = 8;
+  return cl;
+}
+
+template <typename T, bool STOCH>
+static cudaError_t launch_walk(const void* tgt, const void* dft, const double* dlse, int R, int V, int n,
+                               int depth, const ChunkStat* st, const uint64_t* keys, int t_chunks,
+                               const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
+                               const float* uniforms, int B, int32_t* acc_len, int32_t* path,
+                               int32_t* bonus, cudaStream_t s) {
+  const int cl = STOCH ? accept_cluster_size(V) : 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(B * cl));
+  cfg.blockDim = dim3(kAcceptThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, accept_walk_kernel<T, STOCH>, static_cast<const T*>(tgt),
+                            static_cast<const T*>(dft), dlse, R, V, n, depth, st, keys, t_chunks, tokens,
+                            parents, draft_row, uniforms, acc_len, path, bonus);
+}
+
+cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,
+                          int R, const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
+                          const float* uniforms, int B, int n, int V, int depth, int32_t* accepted_len,
+                          int32_t* path, int32_t* bonus, void* ws, cudaStream_t s) {
+  const long long rows = (long long)B * (n + 1);
+  const bool stoch = uniforms != nullptr;
+  ChunkStat* st = nullptr;
+  uint64_t* keys = nullptr;
+  row_stats_ws_layout(ws, rows, V, dtype_bytes(tdtype), 1, &st, &keys);
+  cudaError_t e = launch_row_chunk_stats(tgt, tdtype, rows, V, 1, stoch, st, keys, s);
+  if (e != cudaSuccess) return e;
+  const int t_chunks = plan_chunks(rows, V, dtype_bytes(tdtype)).n_chunks;
+  (void)ddtype;  // the draft rows share the target's element type (checked by the caller)
+  if (tdtype == EAGLE_F32)
+    return stoch ? launch_walk<float, true>(tgt, dft, dlse, R, V, n, depth, st, keys, t_chunks, tokens, parents,
+                                            draft_row, uniforms, B, accepted_len, path, bonus, s)
+                 : launch_walk<float, false>(tgt, dft, dlse, R, V, n, depth, st, keys, t_chunks, tokens,
+                                             parents, draft_row, uniforms, B, accepted_len, path, bonus, s);
+  return stoch ? launch_walk<__nv_bfloat16, true>(tgt, dft, dlse, R, V, n, depth, st, keys, t_chunks, tokens,
+                                                  parents, draft_row, uniforms, B, accepted_len, path, bonus, s)
+               : launch_walk<__nv_bfloat16, false>(tgt, dft, dlse, R, V, n, depth, st, keys, t_chunks, tokens,
+                                                   parents, draft_row, uniforms, B, accepted_len, path, bonus, s);
+}
+
+}  // namespace eagle

@@ -1,0 +1,203 @@
+// C-ABI entry points of libeagle_tree: argument validation on the host, then
+// kernel launches on the caller's stream.  Nothing here allocates memory or
+// synchronises the host.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <utility>
+#include <map>
+
+#include "eagle_internal.h"
+
+using namespace eagle;
+
+namespace eagle {
+cudaError_t ensure_smem_limit(const void* kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(kernel, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[key] = bytes;
+  return e;
+}
+}  // namespace eagle
+
+namespace {
+
+thread_local char g_cuda_err[256] = "";
+
+eagle_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return EAGLE_OK;
+  snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return EAGLE_ERR_CUDA;
+}
+
+bool valid_dtype(int d) { return d == EAGLE_F32 || d == EAGLE_BF16; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+eagle_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return EAGLE_OK;
+  if (ws == nullptr || have < need || ((uintptr_t)ws & 255u) != 0) return EAGLE_ERR_WORKSPACE;
+  return EAGLE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* eagle_status_string(int status) {
+  switch (status) {
+    case EAGLE_OK: return "ok";
+    case EAGLE_ERR_NULL: return "null pointer";
+    case EAGLE_ERR_SHAPE: return "invalid shape";
+    case EAGLE_ERR_DTYPE: return "unsupported dtype";
+    case EAGLE_ERR_LIMIT: return "size exceeds a library limit";
+    case EAGLE_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case EAGLE_ERR_ALIGN: return "tensor pointer not 16-byte aligned";
+    case EAGLE_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+const char* eagle_last_cuda_error(void) { return g_cuda_err; }
+
+int eagle_version(void) { return 100; }
+
+// ------------------------------------------------------------------ row stats
+size_t eagle_row_stats_workspace_bytes(long long rows, int V, int dtype, int k) {
+  if (rows <= 0 || V <= 0 || !valid_dtype(dtype) || k < 1) return 0;
+  return row_stats_ws_bytes(rows, V, dtype_bytes(dtype), k);
+}
+
+eagle_status eagle_row_stats(const void* logits, int dtype, long long rows, int V, int k, int32_t* topk_token,
+                             float* topk_logit, double* lse, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (!logits) return EAGLE_ERR_NULL;
+  if (!valid_dtype(dtype)) return EAGLE_ERR_DTYPE;
+  if (rows <= 0 || V <= 0 || k < 1 || rows > 0x7fffffffLL) return EAGLE_ERR_SHAPE;
+  if (k > EAGLE_MAX_TOPK || k > V) return EAGLE_ERR_LIMIT;
+  eagle_status st = check_ws(workspace, workspace_bytes, row_stats_ws_bytes(rows, V, dtype_bytes(dtype), k));
+  if (st != EAGLE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ChunkStat* cs = nullptr;
+  uint64_t* keys = nullptr;
+  row_stats_ws_layout(workspace, rows, V, dtype_bytes(dtype), k, &cs, &keys);
+  st = cuda_status(launch_row_chunk_stats(logits, dtype, rows, V, k, lse != nullptr, cs, keys, s));
+  if (st != EAGLE_OK) return st;
+  const int nc = plan_chunks(rows, V, dtype_bytes(dtype)).n_chunks;
+  return cuda_status(launch_row_stats_finalize(cs, keys, rows, nc, k, topk_token, topk_logit, lse, s));
+}
+
+// ----------------------------------------------------------------- tree build
+size_t eagle_tree_build_workspace_bytes(int B, int R, int V, int dtype, int k) {
+  if (B <= 0 || R <= 0 || V <= 0 || !valid_dtype(dtype) || k < 1) return 0;
+  return row_stats_ws_bytes((long long)B * R, V, dtype_bytes(dtype), k);
+}
+
+eagle_status eagle_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k,
+                              int m, const eagle_tree_t* out, int* n_nodes, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!draft_logits || !out) return EAGLE_ERR_NULL;
+  if (!out->tokens || !out->parents || !out->depth || !out->logV || !out->draft_row || !out->row_lse)
+    return EAGLE_ERR_NULL;
+  if (!valid_dtype(dtype)) return EAGLE_ERR_DTYPE;
+  if (B <= 0 || V <= 0 || depth <= 0 || k <= 0 || m <= 0) return EAGLE_ERR_SHAPE;
+  if (depth > EAGLE_MAX_DEPTH || k > EAGLE_MAX_TOPK || k > V || m > EAGLE_MAX_NODES) return EAGLE_ERR_LIMIT;
+  const long long P = (long long)k + (long long)(depth - 1) * k * k;
+  if (P > EAGLE_MAX_POOL) return EAGLE_ERR_LIMIT;
+  if (R != 1 + (depth - 1) * k) return EAGLE_ERR_SHAPE;
+  eagle_status st =
+      check_ws(workspace, workspace_bytes, row_stats_ws_bytes((long long)B * R, V, dtype_bytes(dtype), k));
+  if (st != EAGLE_OK) return st;
+  const int n = (int)(m < P ? m : P);
+  if (n_nodes) *n_nodes = n;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ChunkStat* cs = nullptr;
+  uint64_t* keys = nullptr;
+  const long long rows = (long long)B * R;
+  row_stats_ws_layout(workspace, rows, V, dtype_bytes(dtype), k, &cs, &keys);
+  st = cuda_status(launch_row_chunk_stats(draft_logits, dtype, rows, V, k, true, cs, keys, s));
+  if (st != EAGLE_OK) return st;
+  const int nc = plan_chunks(rows, V, dtype_bytes(dtype)).n_chunks;
+  return cuda_status(launch_tree_expand(cs, keys, nc, B, R, depth, k, n, *out, s));
+}
+
+// ------------------------------------------------------------------ tree mask
+eagle_status eagle_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len, int B,
+                             int n, uint64_t* mask, int32_t* pos, void* stream) {
+  if (!parents || !mask) return EAGLE_ERR_NULL;
+  if (pos && (!depth || !prefix_len)) return EAGLE_ERR_NULL;
+  if (B <= 0 || n <= 0) return EAGLE_ERR_SHAPE;
+  if (n > EAGLE_MAX_NODES) return EAGLE_ERR_LIMIT;
+  return cuda_status(launch_tree_mask(parents, depth, prefix_len, B, n, mask, pos,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------------- tree attention
+size_t eagle_tree_attention_workspace_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window) {
+  if (B <= 0 || n <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Lmax < 0) return 0;
+  return attention_ws_bytes(B, n, Hq, Hkv, D, Lmax, window);
+}
+
+eagle_status eagle_tree_attention(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* prefix_len, int Lmax, const void* k_tree, const void* v_tree,
+                                  const uint64_t* mask, const int32_t* pos, int B, int n, int Hq, int Hkv, int D,
+                                  int window, float scale, void* out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (!q || !k_tree || !v_tree || !mask || !prefix_len || !out) return EAGLE_ERR_NULL;
+  if (Lmax > 0 && (!k_cache || !v_cache)) return EAGLE_ERR_NULL;
+  if (window > 0 && !pos) return EAGLE_ERR_NULL;
+  if (B <= 0 || n <= 0 || Hq <= 0 || Hkv <= 0 || Lmax < 0 || window < 0) return EAGLE_ERR_SHAPE;
+  if (Hq % Hkv != 0) return EAGLE_ERR_SHAPE;
+  if (D != 64 && D != 128) return EAGLE_ERR_LIMIT;
+  if (n > EAGLE_MAX_NODES) return EAGLE_ERR_LIMIT;
+  if (!aligned16(q) || !aligned16(k_tree) || !aligned16(v_tree) || !aligned16(out) ||
+      (Lmax > 0 && (!aligned16(k_cache) || !aligned16(v_cache))))
+    return EAGLE_ERR_ALIGN;
+  eagle_status st = check_ws(workspace, workspace_bytes, attention_ws_bytes(B, n, Hq, Hkv, D, Lmax, window));
+  if (st != EAGLE_OK) return st;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)D);
+  return cuda_status(launch_tree_attention(q, k_cache, v_cache, prefix_len, Lmax, k_tree, v_tree, mask, pos, B, n,
+                                           Hq, Hkv, D, window, scale, out, workspace,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+// --------------------------------------------------------------------- accept
+size_t eagle_accept_workspace_bytes(int B, int n, int V, int target_dtype) {
+  if (B <= 0 || n <= 0 || V <= 0 || !valid_dtype(target_dtype)) return 0;
+  return accept_ws_bytes(B, n, V, target_dtype);
+}
+
+eagle_status eagle_accept(const void* target_logits, int target_dtype, const void* draft_logits, int draft_dtype,
+                          const double* draft_lse, int R, const int32_t* tokens, const int32_t* parents,
+                          const int32_t* draft_row, const float* uniforms, int B, int n, int V, int depth,
+                          int32_t* accepted_len, int32_t* path, int32_t* bonus, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!target_logits || !tokens || !parents || !draft_row || !accepted_len || !path || !bonus)
+    return EAGLE_ERR_NULL;
+  if (!valid_dtype(target_dtype)) return EAGLE_ERR_DTYPE;
+  const bool stoch = uniforms != nullptr;
+  if (stoch) {
+    if (!draft_logits || !draft_lse) return EAGLE_ERR_NULL;
+    if (!valid_dtype(draft_dtype)) return EAGLE_ERR_DTYPE;
+    if (draft_dtype != target_dtype) return EAGLE_ERR_DTYPE;
+    if (R <= 0) return EAGLE_ERR_SHAPE;
+  }
+  if (B <= 0 || n <= 0 || V <= 0 || depth <= 0) return EAGLE_ERR_SHAPE;
+  if (n > EAGLE_MAX_NODES || depth > EAGLE_MAX_DEPTH) return EAGLE_ERR_LIMIT;
+  if ((long long)B * (n + 1) > 0x7fffffffLL) return EAGLE_ERR_SHAPE;
+  eagle_status st = check_ws(workspace, workspace_bytes, accept_ws_bytes(B, n, V, target_dtype));
+  if (st != EAGLE_OK) return st;
+  return cuda_status(launch_accept(target_logits, target_dtype, draft_logits, draft_dtype, draft_lse, R, tokens,
+                                   parents, draft_row, uniforms, B, n, V, depth, accepted_len, path, bonus,
+                                   workspace, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

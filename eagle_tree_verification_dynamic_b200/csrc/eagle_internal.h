@@ -1,0 +1,66 @@
+// Host-side declarations shared by the translation units of libeagle_tree.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "eagle_tree.h"
+#include "eagle_common.cuh"
+
+namespace eagle {
+
+constexpr int kNumSMs = 148;  // B200
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device), so
+// later launches (including ones under stream capture) only launch.
+cudaError_t ensure_smem_limit(const void* kernel, size_t bytes);
+inline int dtype_bytes(int dtype) { return dtype == EAGLE_F32 ? 4 : 2; }
+
+// ---- row statistics (row_stats.cu)
+struct ChunkPlan {
+  int chunk_elems;
+  int n_chunks;
+};
+ChunkPlan plan_chunks(long long rows, int V, int elem_bytes);
+size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k);
+void row_stats_ws_layout(void* ws, long long rows, int V, int elem_bytes, int k, ChunkStat** stats,
+                         uint64_t** keys);
+cudaError_t launch_row_chunk_stats(const void* x, int dtype, long long rows, int V, int k, bool lse,
+                                   ChunkStat* stats, uint64_t* keys, cudaStream_t s);
+cudaError_t launch_row_stats_finalize(const ChunkStat* stats, const uint64_t* keys, long long rows,
+                                      int n_chunks, int k, int32_t* topk_token, float* topk_logit,
+                                      double* lse, cudaStream_t s);
+
+// ---- tree build (tree_build.cu)
+size_t tree_build_smem_bytes(int R, int k, int P);
+cudaError_t launch_tree_expand(const ChunkStat* stats, const uint64_t* keys, int n_chunks, int B, int R,
+                               int depth, int k, int n, const eagle_tree_t& out, cudaStream_t s);
+
+// ---- tree mask (tree_mask.cu)
+cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len,
+                             int B, int n, uint64_t* mask, int32_t* pos, cudaStream_t s);
+
+// ---- attention (attention.cu)
+struct AttnPlan {
+  int n_splits;   // prefix splits (one more CTA column handles the tree keys)
+  int chunk;      // prefix keys per split
+  int span;       // prefix keys a sequence can see at most (Lmax, or the window)
+};
+AttnPlan plan_attention(int B, int Hkv, int Lmax, int window);
+size_t attention_ws_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window);
+cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen,
+                                  int Lmax, const void* kt, const void* vt, const uint64_t* mask,
+                                  const int32_t* pos, int B, int n, int Hq, int Hkv, int D, int window,
+                                  float scale, void* out, void* ws, cudaStream_t s);
+
+// ---- accept (accept.cu)
+size_t accept_ws_bytes(int B, int n, int V, int dtype);
+cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,
+                          int R, const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
+                          const float* uniforms, int B, int n, int V, int depth, int32_t* accepted_len,
+                          int32_t* path, int32_t* bonus, void* ws, cudaStream_t s);
+
+}  // namespace eagle

@@ -1,0 +1,86 @@
+"""One whole tree-verification step with preallocated buffers.
+
+build (vocabulary sweep + EAGLE-2 expansion/rerank) -> mask -> tree attention
+-> acceptance, enqueued on the current CUDA stream through the C ABI.  All
+buffers and workspaces are allocated once in the constructor, so a step
+allocates nothing and can be captured in a CUDA graph.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+
+
+@dataclass
+class StepShape:
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    Lmax: int
+    depth: int
+    k: int
+    m: int
+    V: int
+    logits_dtype: torch.dtype
+    window: int = 0
+    stochastic: bool = True
+
+    @property
+    def R(self) -> int:
+        return 1 + (self.depth - 1) * self.k
+
+    @property
+    def n(self) -> int:
+        return min(self.m, L.pool_size(self.depth, self.k))
+
+
+class VerifyStep:
+    def __init__(self, shape: StepShape, device=None):
+        self.s = shape
+        dev = torch.device(device or "cuda")
+        self.device = dev
+        s = shape
+        dcode = L.F32 if s.logits_dtype == torch.float32 else L.BF16
+        self.tree = L.alloc_tree(s.B, s.R, s.depth, s.k, s.m, dev)
+        n = self.tree.n
+        self.mask = torch.empty(s.B, n, 2, dtype=torch.int64, device=dev)
+        self.pos = torch.empty(s.B, n, dtype=torch.int32, device=dev)
+        self.out = torch.empty(s.B, n, s.Hq, s.D, dtype=torch.bfloat16, device=dev)
+        self.accepted_len = torch.empty(s.B, dtype=torch.int32, device=dev)
+        self.path = torch.empty(s.B, s.depth, dtype=torch.int32, device=dev)
+        self.bonus = torch.empty(s.B, dtype=torch.int32, device=dev)
+        self.ws_build = L._workspace(L.tree_build_workspace_bytes(s.B, s.R, s.V, dcode, s.k), dev)
+        self.ws_attn = L._workspace(L.attention_workspace_bytes(s.B, n, s.Hq, s.Hkv, s.D, s.Lmax, s.window), dev)
+        self.ws_acc = L._workspace(L.accept_workspace_bytes(s.B, n, s.V, dcode), dev)
+
+    def build(self, draft_logits: torch.Tensor):
+        L.tree_build_into(draft_logits, self.s.depth, self.s.k, self.s.m, self.tree, self.ws_build)
+
+    def mask_(self, prefix_len: torch.Tensor):
+        L.tree_mask_into(self.tree.parents, self.tree.depth, prefix_len, self.mask, self.pos)
+
+    def attention(self, q, k_cache, v_cache, prefix_len, k_tree, v_tree):
+        L.tree_attention_into(q, k_cache, v_cache, prefix_len, k_tree, v_tree, self.mask, self.pos, self.out,
+                              self.ws_attn, self.s.window)
+
+    def accept(self, target_logits, uniforms: Optional[torch.Tensor], draft_logits):
+        if self.s.stochastic:
+            L.accept_into(target_logits, self.tree.tokens, self.tree.parents, self.tree.draft_row, self.s.depth,
+                          uniforms, draft_logits, self.tree.row_lse, self.accepted_len, self.path, self.bonus,
+                          self.ws_acc)
+        else:
+            L.accept_into(target_logits, self.tree.tokens, self.tree.parents, self.tree.draft_row, self.s.depth,
+                          None, None, None, self.accepted_len, self.path, self.bonus, self.ws_acc)
+
+    def __call__(self, inp: dict):
+        """inp: draft_logits, prefix_len, q, k_cache, v_cache, k_tree, v_tree, target_logits, uniforms."""
+        self.build(inp["draft_logits"])
+        self.mask_(inp["prefix_len"])
+        self.attention(inp["q"], inp["k_cache"], inp["v_cache"], inp["prefix_len"], inp["k_tree"], inp["v_tree"])
+        self.accept(inp["target_logits"], inp.get("uniforms"), inp["draft_logits"])
+        return self.accepted_len, self.path, self.bonus

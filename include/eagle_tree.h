@@ -1,0 +1,221 @@
+/*
+ * libeagle_tree -- one EAGLE tree-verification step on NVIDIA B200 (sm_100a).
+ *
+ * The step (as described on three web pages about EAGLE / EAGLE-2 / EAGLE-3 /
+ * EAGLE-4):
+ *   1. build the EAGLE-2 dynamic draft tree from draft logits: confidence
+ *      c(x) = softmax(draft logits)_x, global acceptance V = product of the
+ *      confidences on the root path, per-level top-k expansion, rerank to the
+ *      best m nodes                       ("EAGLE" notes, section EAGLE-2:
+ *      "Well-Calibrated Draft Model", "Expansion of tree", "Reranking Nodes");
+ *   2. per-node ancestor bitmask: a tree token attends to the shared prefix,
+ *      its ancestors and itself, never to siblings or other branches
+ *      ("Технический анализ EAGLE-4", section "Деревья проверки EAGLE-4 и
+ *      утилита управления");
+ *   3. tree-masked attention of the m tree queries over the prefix KV cache
+ *      plus the tree's own keys ("Tree Attention" for verification, "EAGLE"
+ *      notes "3.Verify"; mask semantics as in 2; optional sliding window as in
+ *      the EAGLE-4 drafter, section "Архитектура EAGLE-4");
+ *   4. acceptance: greedy longest path of target argmaxes, or sampling that
+ *      accepts a draft token with probability min(1, p_target/p_draft) and
+ *      resamples from the normalised max(0, p_target - p_draft) ("EAGLE" notes,
+ *      EAGLE-2 "Well-Calibrated Draft Model"; "Что такое EAGLE-3", section 4
+ *      steps 3-4).
+ *
+ * Conventions shared by every entry point
+ *   - All array arguments are DEVICE pointers owned by the caller, unless a
+ *     parameter says otherwise.  Arrays are dense, row-major, in the index
+ *     order written in brackets.  The library allocates nothing; kernels that
+ *     need scratch space take a caller-provided workspace (size from the
+ *     matching *_workspace_bytes function, 256-byte aligned).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work; outputs are valid after the
+ *     stream is synchronised.  No call synchronises the host.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns a non-zero eagle_status and launches nothing.  A
+ *     failed launch returns EAGLE_ERR_CUDA (the CUDA error string is available
+ *     from eagle_last_cuda_error()).
+ *   - Logits are fp32 (EAGLE_F32) or bf16 (EAGLE_BF16, raw 16-bit patterns).
+ *     Rows must hold finite values; at least k values per row must be > -inf
+ *     where a top-k is taken.  Attention tensors (q, K, V) are bf16.
+ *   - Ties: every top-k and argmax orders by value, then by LOWER token id;
+ *     every node ranking orders by log V, then by lower candidate id.
+ *
+ * Tree layout (one tree per sequence b; n = min(m, P) nodes, P the pool size)
+ *   nodes are numbered 1..n, node 0 is the root (the last accepted token, the
+ *   last entry of the prefix KV cache).  Node order = ascending candidate id,
+ *   so a parent always precedes its children and siblings are in confidence
+ *   order.
+ *     tokens   [B][n] int32   token of node i+1
+ *     parents  [B][n] int32   parent node id of node i+1 (0 = root)
+ *     depth    [B][n] int32   1..tree depth
+ *     logV     [B][n] float   log of the global acceptance V of node i+1
+ *     gid      [B][n] int32   candidate id (level-major, see eagle_tree_build)
+ *     draft_row[B][n+1] int32 draft-logit row holding node j's distribution
+ *                             (j = 0 is the root -> row 0), -1 if never expanded
+ *     row_lse  [B][R] double  log-sum-exp of every draft row
+ *     mask     [B][n][2] uint64  bit j%64 of word j/64 set iff node j+1 is node
+ *                             i+1 or one of its ancestors (n <= 128)
+ *     pos      [B][n] int32   position id: prefix_len[b] - 1 + depth
+ */
+#ifndef EAGLE_TREE_H
+#define EAGLE_TREE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EAGLE_API __attribute__((visibility("default")))
+#else
+#define EAGLE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  EAGLE_OK = 0,
+  EAGLE_ERR_NULL = 1,       /* a required pointer is NULL */
+  EAGLE_ERR_SHAPE = 2,      /* a size is non-positive or sizes disagree */
+  EAGLE_ERR_DTYPE = 3,      /* unsupported element type */
+  EAGLE_ERR_LIMIT = 4,      /* a size exceeds a compiled limit below */
+  EAGLE_ERR_WORKSPACE = 5,  /* workspace missing, too small or misaligned */
+  EAGLE_ERR_ALIGN = 6,      /* a tensor pointer is not 16-byte aligned */
+  EAGLE_ERR_CUDA = 7        /* a CUDA launch or runtime call failed */
+} eagle_status;
+
+typedef enum { EAGLE_F32 = 0, EAGLE_BF16 = 1 } eagle_dtype;
+
+#define EAGLE_MAX_NODES 128   /* m (nodes per tree, root excluded) */
+#define EAGLE_MAX_TOPK 32     /* k */
+#define EAGLE_MAX_DEPTH 16    /* tree depth */
+#define EAGLE_MAX_POOL 4096   /* P = k + (depth-1) k^2 candidates per tree */
+#define EAGLE_MASK_WORDS 2    /* uint64 words per mask row */
+
+/* Device pointers of one batch of trees (see "Tree layout" above).  gid may be
+ * NULL when not wanted; the others are required by eagle_tree_build. */
+typedef struct {
+  int32_t* tokens;
+  int32_t* parents;
+  int32_t* depth;
+  float* logV;
+  int32_t* gid;
+  int32_t* draft_row;
+  double* row_lse;
+} eagle_tree_t;
+
+/* Human-readable name of a status code (static string). */
+EAGLE_API const char* eagle_status_string(int status);
+/* Text of the last CUDA error seen by this library in this thread ("" if none). */
+EAGLE_API const char* eagle_last_cuda_error(void);
+/* Library version, major*10000 + minor*100 + patch. */
+EAGLE_API int eagle_version(void);
+
+/* ---------------------------------------------------------------- row stats
+ * Per logit row: the k largest logits (ties to the lower token id) and the
+ * log-sum-exp, i.e. what turns logits into confidences c(x) = exp(l_x - lse)
+ * ("EAGLE" notes, EAGLE-2 "Well-Calibrated Draft Model").
+ *   logits      [rows][V] (dtype)
+ *   topk_token  [rows][k] int32, descending logit (may be NULL)
+ *   topk_logit  [rows][k] float  (may be NULL)
+ *   lse         [rows]    double (may be NULL)
+ * Limits: 1 <= k <= min(V, EAGLE_MAX_TOPK).  Workspace: eagle_row_stats_workspace_bytes. */
+EAGLE_API size_t eagle_row_stats_workspace_bytes(long long rows, int V, int dtype, int k);
+EAGLE_API eagle_status eagle_row_stats(const void* logits, int dtype, long long rows, int V, int k,
+                             int32_t* topk_token, float* topk_logit, double* lse,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------- tree build
+ * EAGLE-2 dynamic tree for B sequences ("EAGLE" notes, EAGLE-2 sections
+ * "Expansion of tree" and "Reranking Nodes").
+ *   draft_logits [B][R][V] (dtype), R = 1 + (depth-1)*k.  Row 0 is the root's
+ *     distribution; the node in frontier slot s of level l (1 <= l < depth)
+ *     owns row 1 + (l-1)*k + s, its children are that row's top-k tokens.
+ *   Level 1 = the root's top-k children.  At each level the frontier is the
+ *   k candidates with the largest log V (= sum of log confidences on the
+ *   path), slot = rank.  Candidate id: gid = r at level 1 and
+ *   gid = k + (l-2)k^2 + s*k + r at level l >= 2 (s = parent's slot, r = child
+ *   rank).  After the last level the n = min(m, P) candidates with the
+ *   largest log V over all levels are kept and numbered by ascending gid.
+ *   out:      device pointers of the tree arrays (all but gid required)
+ *   n_nodes:  HOST pointer, receives n (may be NULL)
+ * Limits: depth <= EAGLE_MAX_DEPTH, k <= EAGLE_MAX_TOPK, k <= V,
+ *         m <= EAGLE_MAX_NODES, P <= EAGLE_MAX_POOL.
+ * Workspace: eagle_tree_build_workspace_bytes. */
+EAGLE_API size_t eagle_tree_build_workspace_bytes(int B, int R, int V, int dtype, int k);
+EAGLE_API eagle_status eagle_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth,
+                              int k, int m, const eagle_tree_t* out, int* n_nodes,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------- tree mask
+ * Ancestor-or-self bitmask and position ids ("Технический анализ EAGLE-4",
+ * "Деревья проверки EAGLE-4 и утилита управления").
+ *   parents [B][n], depth [B][n], prefix_len [B] (int32) -> mask [B][n][2]
+ *   uint64, pos [B][n] int32 (pos may be NULL; prefix_len may be NULL when pos is).
+ * parents must name earlier nodes (0 <= parents[i] <= i); an out-of-range parent
+ * ends that node's walk (its mask then holds the ancestors seen so far).
+ * Limits: n <= EAGLE_MAX_NODES. */
+EAGLE_API eagle_status eagle_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len,
+                             int B, int n, uint64_t* mask, int32_t* pos, void* stream);
+
+/* -------------------------------------------------------- tree attention
+ * out[b][i][h] = softmax_j(q[b][i][h] . key_j * scale) weighted sum of value_j
+ * over the keys node i+1 may see: prefix entries p < prefix_len[b] of KV head
+ * g = h / (Hq/Hkv) (with window W > 0: only p >= pos_i - W + 1) and tree
+ * entries j with mask bit (i, j) set (with a window: pos_j >= pos_i - W + 1).
+ *   q        [B][n][Hq][D]     bf16
+ *   k_cache  [B][Hkv][Lmax][D] bf16, v_cache likewise; entries past
+ *            prefix_len[b] are ignored but must be finite
+ *   prefix_len [B] int32, clamped to [0, Lmax] on the device
+ *   k_tree   [B][n][Hkv][D]    bf16 (keys of the tree tokens), v_tree likewise
+ *   mask     [B][n][2] uint64  (from eagle_tree_mask)
+ *   pos      [B][n] int32      (from eagle_tree_mask; required iff window > 0)
+ *   out      [B][n][Hq][D]     bf16
+ *   scale    softmax scale; <= 0 selects 1/sqrt(D)
+ * Limits: D in {64, 128}, Hq % Hkv == 0, n <= EAGLE_MAX_NODES, all tensor
+ * pointers 16-byte aligned.  Workspace: eagle_tree_attention_workspace_bytes
+ * (split-KV partial outputs). */
+EAGLE_API size_t eagle_tree_attention_workspace_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window);
+EAGLE_API eagle_status eagle_tree_attention(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* prefix_len, int Lmax, const void* k_tree,
+                                  const void* v_tree, const uint64_t* mask, const int32_t* pos,
+                                  int B, int n, int Hq, int Hkv, int D, int window, float scale,
+                                  void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------- accept
+ * Walk each tree from the root ("EAGLE" notes, EAGLE-2 "Well-Calibrated Draft
+ * Model"; "Что такое EAGLE-3", section 4 steps 3-4; EAGLE-4 write-up, section
+ * "Деревья проверки EAGLE-4 и утилита управления").
+ *   target_logits [B][n+1][V] (target_dtype): row j = target distribution
+ *     after node j (row 0 after the root).
+ *   uniforms == NULL -> greedy: t = argmax of the current row (ties to the
+ *     lower id); move to the first child (node order) whose token is t, else
+ *     stop; bonus = t.
+ *   uniforms != NULL -> sampling, uniforms [B][2][n+1] float in [0, 1): row 0
+ *     is u_acc indexed by the tested child's node id, row 1 is u_res indexed
+ *     by the node where the walk stops.  At node j, p = softmax(target row j),
+ *     q = softmax(draft row draft_row[j]).  Children in node order: accept c
+ *     iff u_acc[c] < p(x_c)/q(x_c); on acceptance move to c (fresh p, q); on
+ *     rejection p <- max(0, p - q) / sum(max(0, p - q)), q unchanged.  With no
+ *     child left, stop and draw the bonus from the current p by inverse CDF:
+ *     the smallest token i with cumsum(p)_i > u_res[j] * sum(p).
+ *     draft_logits [B][R][draft_dtype] with draft_lse [B][R] (double, e.g. the
+ *     tree's row_lse) encode q; both are required for sampling, ignored for
+ *     greedy.
+ *   tokens, parents [B][n], draft_row [B][n+1]: the tree.
+ *   accepted_len [B], path [B][depth] (accepted node ids, -1 padded), bonus [B].
+ * Limits: n <= EAGLE_MAX_NODES, depth <= EAGLE_MAX_DEPTH.
+ * Workspace: eagle_accept_workspace_bytes. */
+EAGLE_API size_t eagle_accept_workspace_bytes(int B, int n, int V, int target_dtype);
+EAGLE_API eagle_status eagle_accept(const void* target_logits, int target_dtype, const void* draft_logits,
+                          int draft_dtype, const double* draft_lse, int R, const int32_t* tokens,
+                          const int32_t* parents, const int32_t* draft_row, const float* uniforms,
+                          int B, int n, int V, int depth, int32_t* accepted_len, int32_t* path,
+                          int32_t* bonus, void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EAGLE_TREE_H */

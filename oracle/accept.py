@@ -31,7 +31,10 @@ Readings:
     min(1, p/q)").  Accepting moves to c with a fresh p and q.  Rejecting sets
     p <- max(0, p - q) / sum(max(0, p - q)) and keeps q.  With no child left
     the walk stops at j and the bonus is drawn from the current p by inverse
-    CDF: the smallest token i with cumsum(p)_i > u_res[j] * sum(p).
+    CDF: the smallest token i with cumsum(p)_i > u_res[j] * sum(p).  If a
+    rejection leaves max(0, p - q) identically zero (only possible when
+    p == q, which accepts for every u < 1) the walk stops there and the bonus
+    is the target argmax of that node.
 """
 from __future__ import annotations
 
@@ -97,6 +100,7 @@ def accept_stochastic(target: np.ndarray, draft: np.ndarray, tokens, parents, dr
     u_acc, u_res = uniforms[0], uniforms[1]
     ties: List[dict] = []
     j, path = 0, []
+    degenerate = False
     p = softmax(target[0])
     while True:
         kids = _children(parents, j)
@@ -116,15 +120,21 @@ def accept_stochastic(target: np.ndarray, draft: np.ndarray, tokens, parents, dr
                     moved = True
                     break
                 p_new = _residual(p, q)
-                if p_new is None:  # p == q leaves nothing to resample from (unreachable: u < 1)
+                if p_new is None:
+                    # p == q leaves nothing to resample from; with u < 1 this is
+                    # unreachable (p == q accepts).  Fall back to the target's argmax.
                     ties.append({"kind": "degenerate", "node": c})
-                else:
-                    p = p_new
+                    degenerate = True
+                    break
+                p = p_new
         if not moved:
             break
-    bonus, tie = inverse_cdf(p, float(u_res[j]))
-    if tie:
-        ties.append({"kind": "bonus", "node": j})
+    if degenerate:
+        bonus = int(np.argmax(target[j]))
+    else:
+        bonus, tie = inverse_cdf(p, float(u_res[j]))
+        if tie:
+            ties.append({"kind": "bonus", "node": j})
     assert len(path) <= max_depth
     return {"accepted_len": len(path), "path": path + [-1] * (max_depth - len(path)),
             "bonus": int(bonus), "stop": j, "near_ties": ties}

@@ -1,0 +1,118 @@
+"""The C-ABI library loads and exports every entry point include/*.h declares;
+host-only parts (status strings, workspace sizes, argument validation, which
+returns before anything touches the GPU) behave as documented.  No GPU needed.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import eagle_tree_verification_dynamic_b200 as et
+from eagle_tree_verification_dynamic_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        for m in re.finditer(r"EAGLE_API\s+[\w\s\*]+?\b(eagle_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return et.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared_functions()
+    assert len(declared) >= 12
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(_lib.exported_names())
+
+
+def test_status_strings_and_version(lib):
+    assert lib.eagle_status_string(0) == b"ok"
+    assert lib.eagle_status_string(4) == b"size exceeds a library limit"
+    assert lib.eagle_status_string(99) == b"unknown status"
+    assert lib.eagle_version() >= 100
+
+
+def test_workspace_sizes_are_pure_and_aligned(lib):
+    a = lib.eagle_tree_build_workspace_bytes(4, 41, 128256, 1, 8)
+    assert a > 0 and a % 256 == 0
+    assert a == lib.eagle_tree_build_workspace_bytes(4, 41, 128256, 1, 8)
+    assert lib.eagle_tree_attention_workspace_bytes(1, 60, 32, 32, 128, 2048, 0) > 0
+    assert lib.eagle_accept_workspace_bytes(32, 32, 128256, 1) > 0
+    assert lib.eagle_row_stats_workspace_bytes(0, 10, 0, 1) == 0      # invalid -> 0
+    assert lib.eagle_tree_build_workspace_bytes(1, 5, 1000, 7, 2) == 0  # bad dtype -> 0
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+
+
+def _tree(valid=True):
+    p = FAKE if valid else None
+    return _lib.TreeStruct(p, p, p, p, None, p, p)
+
+
+def test_build_validation(lib):
+    st = _tree()
+    n = ctypes.c_int(0)
+    call = lambda **kw: lib.eagle_tree_build(
+        kw.get("x", FAKE), kw.get("dt", 0), kw.get("B", 1), kw.get("R", 5), kw.get("V", 1000),
+        kw.get("depth", 3), kw.get("k", 2), kw.get("m", 10), ctypes.byref(kw.get("tree", st)),
+        ctypes.byref(n), kw.get("ws", FAKE), kw.get("wsb", 0), None)
+    assert call(x=None) == 1
+    assert call(tree=_tree(False)) == 1
+    assert call(dt=5) == 3
+    assert call(B=0) == 2
+    assert call(R=6) == 2                        # R must be 1 + (depth-1) k
+    assert call(k=33, R=1 + 2 * 33) == 4         # k > EAGLE_MAX_TOPK
+    assert call(m=129) == 4
+    assert call(depth=17, R=1 + 16 * 2) == 4
+    assert call(depth=16, k=32, R=1 + 15 * 32) == 4   # pool > EAGLE_MAX_POOL
+    assert call(k=1001, V=1000, R=1 + 2 * 1001) == 4  # k > V
+    assert call(ws=None, wsb=0) == 5             # workspace required
+    assert call(ws=ctypes.c_void_p(0x1001), wsb=1 << 30) == 5  # misaligned workspace
+
+
+def test_attention_validation(lib):
+    def call(**kw):
+        return lib.eagle_tree_attention(
+            kw.get("q", FAKE), FAKE, FAKE, FAKE, 128, FAKE, FAKE, FAKE, kw.get("pos", None), 1,
+            kw.get("n", 10), kw.get("Hq", 4), kw.get("Hkv", 4), kw.get("D", 64), kw.get("window", 0), 0.0,
+            kw.get("out", FAKE), FAKE, 1 << 30, None)
+    assert call(q=None) == 1
+    assert call(window=16, pos=None) == 1
+    assert call(Hq=6, Hkv=4) == 2
+    assert call(D=96) == 4
+    assert call(n=129) == 4
+    assert call(q=ctypes.c_void_p(0x1008)) == 6   # not 16-byte aligned
+
+
+def test_accept_and_mask_validation(lib):
+    def acc(**kw):
+        return lib.eagle_accept(FAKE, kw.get("dt", 0), kw.get("draft", None), 0, kw.get("lse", None), 5,
+                                FAKE, FAKE, FAKE, kw.get("u", None), 1, kw.get("n", 10), 1000,
+                                kw.get("depth", 3), FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert acc(u=FAKE) == 1                      # sampling needs the draft logits and lse
+    assert acc(u=FAKE, draft=FAKE) == 1
+    assert acc(dt=9) == 3
+    assert acc(n=200) == 4
+    assert acc(depth=0) == 2
+    assert lib.eagle_tree_mask(None, None, None, 1, 10, FAKE, None, None) == 1
+    assert lib.eagle_tree_mask(FAKE, None, None, 1, 129, FAKE, None, None) == 4
+    assert lib.eagle_tree_mask(FAKE, None, None, 1, 10, FAKE, FAKE, None) == 1  # pos needs depth, prefix_len
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(et.EagleError):
+        et.tree_build(torch.zeros(1, 5, 100), 3, 2, 10)

@@ -1,0 +1,131 @@
+"""GPU parity: greedy and sampled acceptance against the oracle's walk.
+
+Both sides receive the oracle's tree and the same target logits, draft logits
+and uniforms.  accepted_len, path and bonus must be bit-exact; a sequence may
+differ only when the oracle flags a near-tie on its walk (u within 1e-6 of an
+acceptance ratio, or an inverse-CDF threshold within 1e-6 of a cumulative sum),
+which is reported.  The GPU also has to preserve the target distribution with
+drafts sampled from q (chi-square over 10^6 seeded trials).
+"""
+import numpy as np
+import pytest
+import torch
+from scipy.stats import chisquare
+
+import eagle_tree_verification_dynamic_b200 as et
+import oracle
+from workloads import gen_draft_logits, gen_uniforms, get_config, make_target_logits
+
+from gpu_helpers import dev, i32, to_dev_logits
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_trees(cfg, stored):
+    x64 = oracle.decode_logits(stored, cfg.logits_dtype)
+    return x64, [oracle.build_tree(x64[b], cfg.depth, cfg.k, cfg.m) for b in range(cfg.B)]
+
+
+def _run_accept(cfg, seed, mode, sigma=None):
+    stored = gen_draft_logits(cfg, seed)
+    x64, trees = _oracle_trees(cfg, stored)
+    draft_row = np.stack([t["draft_row"] for t in trees])
+    tgt = make_target_logits(cfg, seed, stored, draft_row, sigma=sigma)
+    T64 = oracle.decode_logits(tgt, cfg.logits_dtype)
+    tokens = i32(np.stack([t["tokens"] for t in trees]))
+    parents = i32(np.stack([t["parents"] for t in trees]))
+    drow = i32(draft_row)
+    T = to_dev_logits(tgt, cfg.logits_dtype)
+    if mode == "greedy":
+        acc, path, bonus = et.accept(T, tokens, parents, drow, cfg.depth)
+    else:
+        u = gen_uniforms(cfg, seed)
+        lse = torch.from_numpy(np.stack([t["row_lse"] for t in trees])).to(dev())
+        # the draft normalisers come from the GPU's own sweep, as in a real step
+        _, _, lse_gpu = et.row_stats(to_dev_logits(stored, cfg.logits_dtype).reshape(-1, cfg.V), 1)
+        lse_gpu = lse_gpu.reshape(cfg.B, cfg.R)
+        assert torch.allclose(lse_gpu, lse, rtol=0, atol=5e-7)
+        acc, path, bonus = et.accept(T, tokens, parents, drow, cfg.depth, torch.from_numpy(u).to(dev()),
+                                     to_dev_logits(stored, cfg.logits_dtype), lse_gpu)
+    acc, path, bonus = acc.cpu().numpy(), path.cpu().numpy(), bonus.cpu().numpy()
+    reported = 0
+    for b in range(cfg.B):
+        t = trees[b]
+        if mode == "greedy":
+            r = oracle.accept_greedy(T64[b], t["tokens"], t["parents"], cfg.depth)
+        else:
+            r = oracle.accept_stochastic(T64[b], x64[b], t["tokens"], t["parents"], t["draft_row"],
+                                         u[b].astype(np.float64), cfg.depth)
+        same = (int(acc[b]) == r["accepted_len"] and path[b].tolist() == r["path"] and int(bonus[b]) == r["bonus"])
+        if not same:
+            assert r["near_ties"], (f"{cfg.name} seed {seed} seq {b} {mode}: gpu ({acc[b]}, {path[b].tolist()}, "
+                                    f"{bonus[b]}) oracle ({r['accepted_len']}, {r['path']}, {r['bonus']})")
+            reported += 1
+    return acc, reported
+
+
+@pytest.mark.parametrize("name,mode", [("tiny", "greedy"), ("7b", "greedy"), ("7b", "stochastic"),
+                                       ("l3-8b", "stochastic"), ("long", "greedy"), ("serve", "stochastic")])
+def test_accept_configs(name, mode):
+    cfg = get_config(name)
+    for seed in cfg.seeds[:3]:
+        _run_accept(cfg, seed, mode)
+
+
+@pytest.mark.parametrize("mode", ["greedy", "stochastic"])
+def test_accept_7b_all_seeds(mode):
+    cfg = get_config("7b")
+    lens = [int(_run_accept(cfg, s, mode)[0][0]) for s in cfg.seeds]
+    print(f"7b {mode} accepted lengths over seeds: {lens}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "7b"])
+def test_accept_target_equals_draft(name):
+    """sigma = 0: every first child is accepted down to a leaf (closed form)."""
+    cfg = get_config(name)
+    for mode in ("greedy", "stochastic"):
+        acc, _ = _run_accept(cfg, 2, mode, sigma=0.0)
+        assert int(acc[0]) >= 1
+
+
+def test_accept_batch_of_ragged_configs():
+    cfg = get_config("serve", B=12, V=5003, logits_dtype="f32")
+    _run_accept(cfg, 4, "stochastic")
+    _run_accept(cfg, 4, "greedy")
+
+
+def _chi2_gpu(shape: str, trials: int, seed: int) -> float:
+    rng = np.random.default_rng(seed)
+    V = 8
+    p, q, q2 = rng.dirichlet(np.ones(V)), rng.dirichlet(np.ones(V)), rng.dirichlet(np.ones(V))
+    other = rng.dirichlet(np.ones(V))
+    if shape == "star":
+        n, parents, draft_row = 3, [0, 0, 0], [0, -1, -1, -1]
+        draft = np.log(q)[None]
+        target = np.stack([np.log(p)] + [np.log(other)] * 3)
+        toks = np.minimum(np.searchsorted(np.cumsum(q), rng.random((trials, 3)), side="right"), V - 1)
+    else:
+        n, parents, draft_row = 2, [0, 1], [0, 1, -1]
+        draft = np.stack([np.log(q), np.log(q2)])
+        target = np.stack([np.log(p)] + [np.log(other)] * 2)
+        toks = np.stack([np.minimum(np.searchsorted(np.cumsum(q), rng.random(trials), side="right"), V - 1),
+                         np.minimum(np.searchsorted(np.cumsum(q2), rng.random(trials), side="right"), V - 1)], 1)
+    u = rng.random((trials, 2, n + 1)).astype(np.float32)
+    R = draft.shape[0]
+    D = torch.from_numpy(draft.astype(np.float32)).to(dev()).expand(trials, R, V).contiguous()
+    T = torch.from_numpy(target.astype(np.float32)).to(dev()).expand(trials, n + 1, V).contiguous()
+    _, _, lse = et.row_stats(D.reshape(-1, V), 1)
+    acc, path, bonus = et.accept(T, i32(toks), i32(np.tile(parents, (trials, 1))),
+                                 i32(np.tile(draft_row, (trials, 1))), 2, torch.from_numpy(u).to(dev()),
+                                 D, lse.reshape(trials, R))
+    acc, path, bonus = acc.cpu().numpy(), path.cpu().numpy(), bonus.cpu().numpy()
+    first = np.where(acc > 0, toks[np.arange(trials), np.maximum(path[:, 0], 1) - 1], bonus)
+    p32 = np.exp(np.log(p).astype(np.float32).astype(np.float64))
+    p32 /= p32.sum()
+    counts = np.bincount(first, minlength=V)
+    return chisquare(counts, trials * p32).pvalue
+
+
+@pytest.mark.parametrize("shape", ["star", "chain"])
+def test_gpu_sampling_preserves_target_distribution(shape):
+    assert _chi2_gpu(shape, 1_000_000, 40 if shape == "star" else 41) > 1e-3
