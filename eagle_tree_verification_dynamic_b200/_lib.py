@@ -221,7 +221,7 @@ def tree_attention_into(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, p
 
 
 def tree_attention(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos=None, window: int = 0,
-                   scale: float = 0.0) -> torch.Tensor:
+                   scale: float = 0.0, check: bool = True) -> torch.Tensor:
     """q [B][n][Hq][D] bf16, caches [B][Hkv][Lmax][D] bf16, tree K/V [B][n][Hkv][D] bf16 -> out bf16."""
     _need_cuda(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos)
     for t in (q, k_cache, v_cache, k_tree, v_tree):
@@ -232,7 +232,18 @@ def tree_attention(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos=No
     out = torch.empty_like(q)
     ws = _workspace(attention_workspace_bytes(B, n, Hq, Hkv, D, Lmax, window), q.device)
     tree_attention_into(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos, out, ws, window, scale)
+    if check:
+        check_attention_status(ws)
     return out
+
+
+def check_attention_status(ws: torch.Tensor):
+    """Read the device status word the attention kernel keeps in its workspace
+    header (synchronises the stream).  Non-zero means a bounded wait inside the
+    kernel gave up (1) or the shared-memory base was misaligned (2)."""
+    code = int(ws[:4].view(torch.int32).item())
+    if code != 0:
+        raise EagleError(f"eagle_tree_attention: device status {code}")
 
 
 # -------------------------------------------------------------------- accept

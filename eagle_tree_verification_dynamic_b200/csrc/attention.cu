@@ -11,6 +11,8 @@
 //
 // This file is the CUDA-core path (fp32 dot products, online softmax); it
 // serves every shape the library accepts.
+#include <cstdlib>
+
 #include "eagle_internal.h"
 
 namespace eagle {
@@ -169,12 +171,13 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   out[(((size_t)b * n + i) * Hq + h) * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
 }
 
-AttnPlan plan_attention(int B, int Hkv, int Lmax, int window) {
+AttnPlan plan_attention(int B, int n, int Hq, int Hkv, int Lmax, int window) {
   AttnPlan p;
   p.span = window > 0 ? (Lmax < window ? Lmax : window) : Lmax;
   if (p.span < 1) p.span = 1;
-  const int heads = B * Hkv;
-  int splits = (kNumSMs + heads - 1) / heads;
+  // two CTAs per SM: aim for ~2 x 148 CTAs over (row groups x heads x splits)
+  const int heads = B * Hkv * attention_row_groups(n, Hq, Hkv);
+  int splits = (2 * kNumSMs + heads - 1) / heads;
   const int max_splits = (p.span + 63) / 64;
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
@@ -185,38 +188,49 @@ AttnPlan plan_attention(int B, int Hkv, int Lmax, int window) {
   return p;
 }
 
+// workspace: [256 B header: device error word][partial O][partial lse]
 size_t attention_ws_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window) {
-  const AttnPlan p = plan_attention(B, Hkv, Lmax, window);
+  const AttnPlan p = plan_attention(B, n, Hq, Hkv, Lmax, window);
   const size_t slots = (size_t)(p.n_splits + 1) * B * n * Hq;
-  return align_up(slots * D * sizeof(float), 256) + align_up(slots * sizeof(float), 256);
+  return 256 + align_up(slots * D * sizeof(float), 256) + align_up(slots * sizeof(float), 256);
 }
 
-cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen,
-                                  int Lmax, const void* kt, const void* vt, const uint64_t* mask,
-                                  const int32_t* pos, int B, int n, int Hq, int Hkv, int D, int window,
-                                  float scale, void* out, void* ws, cudaStream_t s) {
-  const AttnPlan p = plan_attention(B, Hkv, Lmax, window);
+cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
+                                  const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
+                                  int n, int Hq, int Hkv, int D, int window, float scale, void* out, void* ws,
+                                  cudaStream_t s) {
+  const AttnPlan p = plan_attention(B, n, Hq, Hkv, Lmax, window);
   const size_t slots = (size_t)(p.n_splits + 1) * B * n * Hq;
-  float* part_o = static_cast<float*>(ws);
-  float* part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(slots * D * sizeof(float), 256));
-  const dim3 grid(p.n_splits + 1, Hkv, B);
-  const size_t smem = sizeof(float) * ((size_t)kTileKeys * (2 * D + 1) + (size_t)kAttnWarps * kRowsPerWarp * D);
-  cudaError_t e0 = D == 128 ? ensure_smem_limit((const void*)attn_simt_kernel<128>, smem)
-                            : ensure_smem_limit((const void*)attn_simt_kernel<64>, smem);
-  if (e0 != cudaSuccess) return e0;
+  char* base = static_cast<char*>(ws);
+  int* err = reinterpret_cast<int*>(base);
+  float* part_o = reinterpret_cast<float*>(base + 256);
+  float* part_lse = reinterpret_cast<float*>(base + 256 + align_up(slots * D * sizeof(float), 256));
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
   using bf = __nv_bfloat16;
-  const bf* qq = static_cast<const bf*>(q);
-  const bf* kk = static_cast<const bf*>(kc);
-  const bf* vv = static_cast<const bf*>(vc);
-  const bf* ktt = static_cast<const bf*>(kt);
-  const bf* vtt = static_cast<const bf*>(vt);
-  if (D == 128)
-    attn_simt_kernel<128><<<grid, kAttnThreads, smem, s>>>(qq, kk, vv, plen, Lmax, ktt, vtt, mask, pos, n, Hq,
-                                                        Hkv, window, scale, p.n_splits, p.chunk, part_o, part_lse);
-  else
-    attn_simt_kernel<64><<<grid, kAttnThreads, smem, s>>>(qq, kk, vv, plen, Lmax, ktt, vtt, mask, pos, n, Hq,
-                                                       Hkv, window, scale, p.n_splits, p.chunk, part_o, part_lse);
-  cudaError_t e = cudaGetLastError();
+  static const bool simt = getenv("EAGLE_DEBUG_SIMT_ATTENTION") != nullptr;
+  if (simt) {
+    const dim3 grid(p.n_splits + 1, Hkv, B);
+    const size_t smem =
+        sizeof(float) * ((size_t)kTileKeys * (2 * D + 1) + (size_t)kAttnWarps * kRowsPerWarp * D);
+    e = D == 128 ? ensure_smem_limit((const void*)attn_simt_kernel<128>, smem)
+                 : ensure_smem_limit((const void*)attn_simt_kernel<64>, smem);
+    if (e != cudaSuccess) return e;
+    if (D == 128)
+      attn_simt_kernel<128><<<grid, kAttnThreads, smem, s>>>(
+          static_cast<const bf*>(q), static_cast<const bf*>(kc), static_cast<const bf*>(vc), plen, Lmax,
+          static_cast<const bf*>(kt), static_cast<const bf*>(vt), mask, pos, n, Hq, Hkv, window, scale,
+          p.n_splits, p.chunk, part_o, part_lse);
+    else
+      attn_simt_kernel<64><<<grid, kAttnThreads, smem, s>>>(
+          static_cast<const bf*>(q), static_cast<const bf*>(kc), static_cast<const bf*>(vc), plen, Lmax,
+          static_cast<const bf*>(kt), static_cast<const bf*>(vt), mask, pos, n, Hq, Hkv, window, scale,
+          p.n_splits, p.chunk, part_o, part_lse);
+    e = cudaGetLastError();
+  } else {
+    e = launch_attention_tc(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, D, window, scale, p, part_o,
+                            part_lse, err, s);
+  }
   if (e != cudaSuccess) return e;
   const dim3 cgrid(n * Hq, B);
   if (D == 128)

@@ -1,0 +1,442 @@
+// Tree-masked split-KV attention on the 5th-generation tensor cores
+// ("Tree Attention" verification of the EAGLE notes, "3.Verify"; mask
+// semantics of "Технический анализ EAGLE-4", section "Деревья проверки
+// EAGLE-4 и утилита управления").
+//
+// One CTA = (key split, KV head g, sequence b, group of 128 query rows).  The
+// 128 rows are the (node, head-in-group) pairs of head g, so every K/V tile
+// staged in shared memory serves all tree queries of the GQA group at once.
+//   warp 0      TMA producer: K and V tiles of 64 keys into a 2-stage ring
+//               (128-byte swizzle, no multicast); also allocates TMEM
+//   warp 1      one thread issues tcgen05.mma: S = Q K^T into TMEM, then
+//               O += P V into TMEM (fp32 accumulators, bf16 operands)
+//   warps 2-5   softmax: thread r owns TMEM lane r = query row r; reads its S
+//               row, applies the prefix range / window / tree bitmask, keeps a
+//               running reference max (re-based only when it grows by > 8 in
+//               log2 units, then O and the row sum are rescaled in TMEM),
+//               writes P = 2^(x - m) as bf16 into swizzled shared memory
+// The last split column handles the n tree keys, visible per the ancestor
+// bitmask.  Every CTA writes its normalised partial output and log-sum-exp;
+// attn_combine_kernel merges the splits.
+//
+// Every mbarrier wait is bounded (about 2 s of wall time); a timeout sets an
+// abort flag that ends all roles, records an error word in the workspace
+// header and still frees the TMEM columns before the CTA exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "eagle_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace eagle {
+
+using namespace sm100;
+
+constexpr int kTcThreads = 192;  // 6 warps
+constexpr int kBN = 64;          // keys per tile
+constexpr int kStages = 2;
+constexpr int kRowsPerCta = 128;
+
+template <int D>
+struct TcLayout {
+  static constexpr int kAtoms = D / 64;                 // 128-byte column atoms along D
+  static constexpr int kQBytes = kAtoms * 128 * 128;    // 128 rows
+  static constexpr int kPBytes = 128 * 128;             // 128 rows x 64 keys bf16
+  static constexpr int kKVAtomBytes = kBN * 128;        // 64 keys x 128 B
+  static constexpr int kKBytes = kAtoms * kKVAtomBytes;
+  static constexpr int kStageBytes = 2 * kKBytes;       // K + V
+  static constexpr int kQOff = 0;
+  static constexpr int kPOff = kQOff + kQBytes;
+  static constexpr int kStageOff = kPOff + kPBytes;
+  static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOff + 128;  // + barriers (base is 1024-aligned, checked)
+  static constexpr uint32_t kTmemCols = (64 + D) <= 128 ? 128 : 256;
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColO = 64;
+};
+
+struct TcBars {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t s_full;
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t mma_idle;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(TcBars) <= 128, "barrier block");
+
+struct TcParams {
+  const __nv_bfloat16* q;
+  const int32_t* plen;
+  const uint64_t* mask;
+  const int32_t* pos;
+  float* part_o;
+  float* part_lse;
+  int* err;
+  int Lmax, n, Hq, Hkv, window, n_splits, chunk, row_groups;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 2)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_vt,
+               const TcParams p) {
+  using Lay = TcLayout<D>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  TcBars* bars = reinterpret_cast<TcBars*>(smem + Lay::kBarOff);
+  const uint32_t s_base = smem_u32(smem);
+  if (s_base & 1023u) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicExch(p.err, 2);
+    return;
+  }
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int s = blockIdx.x, g = blockIdx.y;
+  const int b = blockIdx.z / p.row_groups, rg = blockIdx.z % p.row_groups;
+  const int B = gridDim.z / p.row_groups;
+  const int G = p.Hq / p.Hkv;
+  const int rows = p.n * G;
+  const int row0 = rg * kRowsPerCta;
+  const int L = min(max(p.plen[b], 0), p.Lmax);
+  const bool tree = (s == p.n_splits);
+  int k0, k1;
+  if (!tree) {
+    const int lo = p.window > 0 ? max(0, L - p.window + 1) : 0;
+    k0 = lo + s * p.chunk;
+    k1 = min(L, k0 + p.chunk);
+  } else {
+    k0 = 0;
+    k1 = p.n;
+  }
+  const int ntiles = k1 > k0 ? (k1 - k0 + kBN - 1) / kBN : 0;
+
+  // softmax thread -> query row
+  const bool is_soft = warp >= 2;
+  const int quad = warp & 3;
+  const int r_local = quad * 32 + lane;   // TMEM lane = row within the tile
+  const int r_glob = row0 + r_local;
+  const bool row_ok = is_soft && r_glob < rows;
+  const int qi = row_ok ? r_glob / G : 0;
+  const int qh = row_ok ? g * G + r_glob % G : 0;
+
+  if (ntiles == 0) {  // nothing visible in this split: an empty partial
+    if (row_ok) {
+      const size_t slot = (((size_t)s * B + b) * p.n + qi) * p.Hq + qh;
+      for (int d = 0; d < D; ++d) p.part_o[slot * D + d] = 0.f;
+      p.part_lse[slot] = -INFINITY;
+    }
+    return;
+  }
+
+  // ---- set-up: barriers, TMEM, Q tile
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&bars->full[i]), 1);
+      mbar_init(smem_u32(&bars->empty[i]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->p_full), 128);
+    mbar_init(smem_u32(&bars->pv_done), 1);
+    mbar_init(smem_u32(&bars->mma_idle), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_kt);
+    prefetch_tmap(&tm_vt);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&bars->tmem_base), Lay::kTmemCols);
+    tmem_relinquish();
+  }
+  // Q rows (bf16) -> 128-byte swizzled K-major tile
+  for (int e = tid; e < 128 * Lay::kAtoms * 8; e += kTcThreads) {
+    const int r = e / (Lay::kAtoms * 8);
+    const int a = (e / 8) % Lay::kAtoms;
+    const int c = e % 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    const int rr = row0 + r;
+    if (rr < rows) {
+      const int i = rr / G, h = g * G + rr % G;
+      v = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * p.n + i) * p.Hq + h) * D + a * 64 + c * 8);
+    }
+    *reinterpret_cast<uint4*>(smem + Lay::kQOff + a * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < ntiles; ++j) {
+        const int st = j % kStages;
+        if (j >= kStages && !mbar_wait(smem_u32(&bars->empty[st]), ((j / kStages) - 1) & 1, abort)) break;
+        const uint32_t fb = smem_u32(&bars->full[st]);
+        mbar_arrive_expect_tx(fb, Lay::kStageBytes);
+        const uint32_t kdst = s_base + Lay::kStageOff + st * Lay::kStageBytes;
+        const uint32_t vdst = kdst + Lay::kKBytes;
+        const int key0 = k0 + j * kBN;
+        for (int a = 0; a < Lay::kAtoms; ++a) {
+          if (!tree) {
+            const int y = (b * p.Hkv + g) * p.Lmax + key0;
+            tma_load_2d(kdst + a * Lay::kKVAtomBytes, &tm_k, a * 64, y, fb);
+            tma_load_2d(vdst + a * Lay::kKVAtomBytes, &tm_v, a * 64, y, fb);
+          } else {
+            tma_load_3d(kdst + a * Lay::kKVAtomBytes, &tm_kt, a * 64, g, b * p.n + key0, fb);
+            tma_load_3d(vdst + a * Lay::kKVAtomBytes, &tm_vt, a * 64, g, b * p.n + key0, fb);
+          }
+        }
+        ++issued;
+      }
+      // drain: wait until every issued stage has landed before the CTA may exit
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        mbar_wait_drain(smem_u32(&bars->full[j % kStages]), (j / kStages) & 1, 200000000ull);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_qk = idesc_bf16_f32(128, kBN, 0, 0);
+      const uint32_t id_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t t_s = tmem + Lay::kColS, t_o = tmem + Lay::kColO;
+      const uint32_t q_addr = s_base + Lay::kQOff;
+      const uint32_t p_addr = s_base + Lay::kPOff;
+      for (int j = 0; j < ntiles; ++j) {
+        const int st = j % kStages;
+        if (!mbar_wait(smem_u32(&bars->full[st]), (j / kStages) & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t k_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes;
+        const uint32_t v_addr = k_addr + Lay::kKBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 0 + (kk % 4) * 32;
+          const uint64_t da = smem_desc(q_addr + (kk / 4) * 16384 + off, 16, 1024, kSwizzle128B);
+          const uint64_t db = smem_desc(k_addr + (kk / 4) * Lay::kKVAtomBytes + off, 16, 1024, kSwizzle128B);
+          mma_bf16_ss(t_s, da, db, id_qk, kk > 0);
+        }
+        mma_commit(smem_u32(&bars->s_full));
+        if (!mbar_wait(smem_u32(&bars->p_full), j & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t da = smem_desc(p_addr + kk * 32, 16, 1024, kSwizzle128B);
+          const uint64_t db = smem_desc(v_addr + kk * 2048, Lay::kKVAtomBytes, 1024, kSwizzle128B);
+          mma_bf16_ss(t_o, da, db, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&bars->empty[st]));
+        mma_commit(smem_u32(&bars->pv_done));
+      }
+      // every MMA this thread issued has finished before TMEM is released
+      mma_commit(smem_u32(&bars->mma_idle));
+      mbar_wait_drain(smem_u32(&bars->mma_idle), 0, 200000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + Lay::kColS;
+    const uint32_t t_o = tmem + lane_base + Lay::kColO;
+    const int qpos = (row_ok && p.window > 0) ? p.pos[(size_t)b * p.n + qi] : 0;
+    const int win_lo = qpos - p.window + 1;
+    uint64_t mw0 = 0, mw1 = 0;
+    if (row_ok && tree) {
+      mw0 = p.mask[((size_t)b * p.n + qi) * 2];
+      mw1 = p.mask[((size_t)b * p.n + qi) * 2 + 1];
+    }
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    unsigned char* prow = smem + Lay::kPOff + r_local * 128;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full), j & 1, abort))) { ok = false; break; }
+      tc_fence_after();
+      float x[kBN];
+      tmem_ld32(t_s, x);
+      tmem_ld32(t_s + 32, x + 32);
+      tmem_wait_ld();
+      const int key0 = k0 + j * kBN;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        const int kidx = key0 + c;
+        bool vis = row_ok && kidx < k1;
+        if (vis && tree) {
+          vis = ((kidx < 64 ? mw0 >> kidx : mw1 >> (kidx - 64)) & 1ull) != 0;
+          if (vis && p.window > 0) vis = p.pos[(size_t)b * p.n + kidx] >= win_lo;
+        } else if (vis && p.window > 0) {
+          vis = kidx >= win_lo;
+        }
+        x[c] = vis ? x[c] * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[c]);
+      }
+      // PV(j-1) must be complete before P is overwritten or O is rescaled
+      if (j > 0) {
+        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (j - 1) & 1, abort))) { ok = false; break; }
+        tc_fence_after();
+      }
+      const bool rebase = mx > m_used + 8.f;
+      if (__any_sync(kFull, rebase && j > 0 && l > 0.f)) {
+        const float f = (rebase && l > 0.f) ? ex2(m_used - mx) : 1.f;
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float o[32];
+          tmem_ld32(t_o + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) o[t] *= f;
+          tmem_st32(t_o + c0, o);
+        }
+        tmem_wait_st();
+        l *= f;
+      }
+      if (rebase) m_used = mx;
+      float sum = 0.f;
+#pragma unroll
+      for (int c8 = 0; c8 < kBN / 8; ++c8) {
+        uint32_t packed[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float a = x[c8 * 8 + 2 * t] > -INFINITY ? ex2(x[c8 * 8 + 2 * t] - m_used) : 0.f;
+          const float bb = x[c8 * 8 + 2 * t + 1] > -INFINITY ? ex2(x[c8 * 8 + 2 * t + 1] - m_used) : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
+          sum += __low2float(h2) + __high2float(h2);
+          packed[t] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r_local & 7)) << 4)) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
+      l += sum;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->p_full));
+    }
+    // epilogue: normalised partial output and its log-sum-exp
+    if (ok && __all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (ntiles - 1) & 1, abort))) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const size_t slot = (((size_t)s * B + b) * p.n + qi) * p.Hq + qh;
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float o[32];
+        tmem_ld32(t_o + c0, o);
+        tmem_wait_ld();
+        if (row_ok) {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + slot * D + c0);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) dst[t] = make_float4(o[4 * t] * inv, o[4 * t + 1] * inv, o[4 * t + 2] * inv,
+                                                            o[4 * t + 3] * inv);
+        }
+      }
+      if (row_ok) p.part_lse[slot] = l > 0.f ? (m_used + __log2f(l)) * (float)kLn2 : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort && tid == 0) atomicExch(p.err, 1);
+  if (warp == 0) tmem_dealloc(tmem, Lay::kTmemCols);
+}
+
+// ------------------------------------------------------------------- host
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map with a 64-element x 64-row box and 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+              const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int attention_row_groups(int n, int Hq, int Hkv) {
+  const int rows = n * (Hq / Hkv);
+  return (rows + kRowsPerCta - 1) / kRowsPerCta;
+}
+
+template <int D>
+static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
+                             const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
+                             int n, int Hq, int Hkv, int window, float scale, const AttnPlan& plan, float* part_o,
+                             float* part_lse, int* err, cudaStream_t s) {
+  CUtensorMap mk, mv, mkt, mvt;
+  const int Lrows = Lmax > 0 ? Lmax : 1;
+  const void* kbase = Lmax > 0 ? kc : kt;  // any valid address when the cache is empty
+  const void* vbase = Lmax > 0 ? vc : vt;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)B * Hkv * Lrows};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kBN};
+    const cuuint64_t dims0[2] = {(cuuint64_t)D, (cuuint64_t)(Lmax > 0 ? (cuuint64_t)B * Hkv * Lrows : 1)};
+    if (!make_map(&mk, kbase, 2, Lmax > 0 ? dims : dims0, str, box) ||
+        !make_map(&mv, vbase, 2, Lmax > 0 ? dims : dims0, str, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)B * n};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kBN};
+    if (!make_map(&mkt, kt, 3, dims, str, box) || !make_map(&mvt, vt, 3, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  TcParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.plen = plen;
+  p.mask = mask;
+  p.pos = pos;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.err = err;
+  p.Lmax = Lmax;
+  p.n = n;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.window = window;
+  p.n_splits = plan.n_splits;
+  p.chunk = plan.chunk;
+  p.row_groups = attention_row_groups(n, Hq, Hkv);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const size_t smem = TcLayout<D>::kSmemBytes;
+  cudaError_t e = ensure_smem_limit((const void*)attn_tc_kernel<D>, smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(plan.n_splits + 1, Hkv, B * p.row_groups);
+  attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(mk, mv, mkt, mvt, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
+                                const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
+                                int n, int Hq, int Hkv, int D, int window, float scale, const AttnPlan& plan,
+                                float* part_o, float* part_lse, int* err, cudaStream_t s) {
+  if (D == 128)
+    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, plan, part_o,
+                          part_lse, err, s);
+  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, plan, part_o,
+                       part_lse, err, s);
+}
+
+}  // namespace eagle

@@ -43,18 +43,23 @@ cudaError_t launch_tree_expand(const ChunkStat* stats, const uint64_t* keys, int
 cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len,
                              int B, int n, uint64_t* mask, int32_t* pos, cudaStream_t s);
 
-// ---- attention (attention.cu)
+// ---- attention (attention.cu, attention_tc.cu)
 struct AttnPlan {
   int n_splits;   // prefix splits (one more CTA column handles the tree keys)
-  int chunk;      // prefix keys per split
+  int chunk;      // prefix keys per split (multiple of 64)
   int span;       // prefix keys a sequence can see at most (Lmax, or the window)
 };
-AttnPlan plan_attention(int B, int Hkv, int Lmax, int window);
+int attention_row_groups(int n, int Hq, int Hkv);
+AttnPlan plan_attention(int B, int n, int Hq, int Hkv, int Lmax, int window);
 size_t attention_ws_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window);
 cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen,
                                   int Lmax, const void* kt, const void* vt, const uint64_t* mask,
                                   const int32_t* pos, int B, int n, int Hq, int Hkv, int D, int window,
                                   float scale, void* out, void* ws, cudaStream_t s);
+cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
+                                const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
+                                int n, int Hq, int Hkv, int D, int window, float scale, const AttnPlan& plan,
+                                float* part_o, float* part_lse, int* err, cudaStream_t s);
 
 // ---- accept (accept.cu)
 size_t accept_ws_bytes(int B, int n, int V, int dtype);

@@ -95,11 +95,13 @@ row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
         acc = rescale_pow2(acc, e_ref, e_new);
         e_ref = e_new;
       }
-      float part = 0.f;
+      if (e_ref > -INFINITY) {  // until a finite logit arrives every term is exp(-inf) = 0
+        float part = 0.f;
 #pragma unroll
-      for (int i = 0; i < Elem<T>::kPerVec; ++i)
-        if (i < n) part += exp2_scaled(f[i], e_ref);
-      acc += (double)part;
+        for (int i = 0; i < Elem<T>::kPerVec; ++i)
+          if (i < n) part += exp2_scaled(f[i], e_ref);
+        acc += (double)part;
+      }
     }
   };
 
