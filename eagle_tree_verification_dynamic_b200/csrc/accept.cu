@@ -38,13 +38,31 @@ struct SweepArgs {
   bool use_q;         // false: weights are p itself
 };
 
-// Weight of token x under the current target: p(x), or max(0, p(x) - t q(x)).
+constexpr int kSegChunk = 16;
+
+// Weights of tokens base .. base+15 (0 past x1) under the current target:
+// p(x), or max(0, p(x) - t q(x)).  All loads are issued before any use.
 template <typename T>
-__device__ __forceinline__ float sweep_weight(const SweepArgs& a, int x) {
-  const float p = exp_minus(load_logit(static_cast<const T*>(a.trow) + x), a.lse_t);
-  if (!a.use_q) return p;
-  const float q = exp_minus(load_logit(static_cast<const T*>(a.drow) + x), a.lse_d);
-  return fmaxf(0.f, fmaf(-a.t.lo, q, fmaf(-a.t.hi, q, p)));
+__device__ __forceinline__ void sweep_weights(const SweepArgs& a, int base, int x1, float* w) {
+  const T* tr = static_cast<const T*>(a.trow);
+  const T* dr = static_cast<const T*>(a.drow);
+  float lt[kSegChunk], ld[kSegChunk];
+#pragma unroll
+  for (int i = 0; i < kSegChunk; ++i) lt[i] = base + i < x1 ? load_logit(tr + base + i) : -INFINITY;
+  if (a.use_q) {
+#pragma unroll
+    for (int i = 0; i < kSegChunk; ++i) ld[i] = base + i < x1 ? load_logit(dr + base + i) : 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < kSegChunk; ++i) {
+    const float p = exp_minus(lt[i], a.lse_t);
+    if (!a.use_q) {
+      w[i] = p;
+    } else {
+      const float q = exp_minus(ld[i], a.lse_d);
+      w[i] = fmaxf(0.f, fmaf(-a.t.lo, q, fmaf(-a.t.hi, q, p)));
+    }
+  }
 }
 
 struct AcceptSmem {
@@ -92,24 +110,35 @@ __device__ double sweep_total(const SweepArgs& a, int V, AcceptSmem& sm, cg::clu
   const int seg = (V + nt - 1) / nt;
   const int x0 = min(V, gt * seg), x1 = min(V, x0 + seg);
   double acc = 0.0;
-  for (int x = x0; x < x1; ++x) acc += (double)sweep_weight<T>(a, x);
+  for (int base = x0; base < x1; base += kSegChunk) {
+    float w[kSegChunk];
+    sweep_weights<T>(a, base, x1, w);
+#pragma unroll
+    for (int i = 0; i < kSegChunk; ++i) acc += (double)w[i];
+  }
   return cluster_sum(block_sum(acc, sm), sm, cluster, nullptr);
 }
 
 // Inverse CDF over the weights: smallest x with cumsum_x > u * total.  Writes
 // the token to *out from the one thread that owns the crossing; returns the
-// total weight (every thread).
+// total weight (every thread).  Each thread owns a contiguous slice of the
+// vocabulary and sums it in token order, in fp64, element by element; the
+// owner's rescan repeats exactly those additions.
 template <typename T>
 __device__ double sweep_sample(const SweepArgs& a, int V, float u, AcceptSmem& sm,
                                cg::cluster_group& cluster, int32_t* out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nt = (int)cluster.num_blocks() * kAcceptThreads;
   const int gt = (int)cluster.block_rank() * kAcceptThreads + tid;
-  (void)lane;
   const int seg = (V + nt - 1) / nt;
   const int x0 = min(V, gt * seg), x1 = min(V, x0 + seg);
   double mine = 0.0;
-  for (int x = x0; x < x1; ++x) mine += (double)sweep_weight<T>(a, x);
+  for (int base = x0; base < x1; base += kSegChunk) {
+    float w[kSegChunk];
+    sweep_weights<T>(a, base, x1, w);
+#pragma unroll
+    for (int i = 0; i < kSegChunk; ++i) mine += (double)w[i];
+  }
   // Block exclusive prefix of the per-thread sums, summed serially (lane order
   // within a warp, then warp order) so the prefixes never decrease and the
   // ownership intervals [prefix[t], prefix[t+1]) tile [0, total) exactly.
@@ -141,11 +170,16 @@ __device__ double sweep_sample(const SweepArgs& a, int V, float u, AcceptSmem& s
     if (start <= thr && thr < end) {
       double run = 0.0;
       int pick = -1, last_nz = -1;
-      for (int x = x0; x < x1; ++x) {
-        const float w = sweep_weight<T>(a, x);
-        if (w > 0.f) last_nz = x;
-        run += (double)w;
-        if (my_off + (sm.prefix[tid] + run) > thr) { pick = x; break; }
+      for (int base = x0; base < x1 && pick < 0; base += kSegChunk) {
+        float w[kSegChunk];
+        sweep_weights<T>(a, base, x1, w);
+#pragma unroll
+        for (int i = 0; i < kSegChunk; ++i) {
+          if (pick >= 0 || base + i >= x1) continue;
+          if (w[i] > 0.f) last_nz = base + i;
+          run += (double)w[i];
+          if (my_off + (sm.prefix[tid] + run) > thr) pick = base + i;
+        }
       }
       *out = pick >= 0 ? pick : last_nz;
     }

@@ -98,7 +98,7 @@ eagle_status eagle_row_stats(const void* logits, int dtype, long long rows, int 
 // ----------------------------------------------------------------- tree build
 size_t eagle_tree_build_workspace_bytes(int B, int R, int V, int dtype, int k) {
   if (B <= 0 || R <= 0 || V <= 0 || !valid_dtype(dtype) || k < 1) return 0;
-  return row_stats_ws_bytes((long long)B * R, V, dtype_bytes(dtype), k);
+  return tree_build_ws_bytes(B, R, V, dtype_bytes(dtype), k);
 }
 
 eagle_status eagle_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k,
@@ -113,20 +113,12 @@ eagle_status eagle_tree_build(const void* draft_logits, int dtype, int B, int R,
   const long long P = (long long)k + (long long)(depth - 1) * k * k;
   if (P > EAGLE_MAX_POOL) return EAGLE_ERR_LIMIT;
   if (R != 1 + (depth - 1) * k) return EAGLE_ERR_SHAPE;
-  eagle_status st =
-      check_ws(workspace, workspace_bytes, row_stats_ws_bytes((long long)B * R, V, dtype_bytes(dtype), k));
+  eagle_status st = check_ws(workspace, workspace_bytes, tree_build_ws_bytes(B, R, V, dtype_bytes(dtype), k));
   if (st != EAGLE_OK) return st;
   const int n = (int)(m < P ? m : P);
   if (n_nodes) *n_nodes = n;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ChunkStat* cs = nullptr;
-  uint64_t* keys = nullptr;
-  const long long rows = (long long)B * R;
-  row_stats_ws_layout(workspace, rows, V, dtype_bytes(dtype), k, &cs, &keys);
-  st = cuda_status(launch_row_chunk_stats(draft_logits, dtype, rows, V, k, true, cs, keys, s));
-  if (st != EAGLE_OK) return st;
-  const int nc = plan_chunks(rows, V, dtype_bytes(dtype)).n_chunks;
-  return cuda_status(launch_tree_expand(cs, keys, nc, B, R, depth, k, n, *out, s));
+  return cuda_status(launch_tree_build(draft_logits, dtype, B, R, V, depth, k, n, *out, workspace,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 // ------------------------------------------------------------------ tree mask

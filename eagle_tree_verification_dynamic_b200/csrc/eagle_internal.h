@@ -36,8 +36,9 @@ cudaError_t launch_row_stats_finalize(const ChunkStat* stats, const uint64_t* ke
 
 // ---- tree build (tree_build.cu)
 size_t tree_build_smem_bytes(int R, int k, int P);
-cudaError_t launch_tree_expand(const ChunkStat* stats, const uint64_t* keys, int n_chunks, int B, int R,
-                               int depth, int k, int n, const eagle_tree_t& out, cudaStream_t s);
+size_t tree_build_ws_bytes(int B, int R, int V, int elem_bytes, int k);
+cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k, int n,
+                              const eagle_tree_t& out, void* ws, cudaStream_t s);
 
 // ---- tree mask (tree_mask.cu)
 cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len,

@@ -1,10 +1,12 @@
 // EAGLE-2 dynamic draft tree ("EAGLE" notes, EAGLE-2 sections "Expansion of
 // tree" and "Reranking Nodes").  One CTA per sequence:
-//   1. merge the chunk statistics of the sequence's R draft rows into each
-//      row's log-sum-exp and top-k (token, log-confidence lp = logit - lse);
+//   0. (before it, in parallel over all rows) the vocabulary sweep and a
+//      one-warp-per-row merge give each draft row's log-sum-exp and top-k;
+//   1. lp = logit - lse turns the top-k logits into log-confidences;
 //   2. level 1 = the root's k children; for each level up to depth-1, rank the
-//      level's candidates by (log V desc, candidate id asc), the first k form
-//      the frontier (slot = rank, which names the draft row of the node), and
+//      level's candidates by (log V desc, candidate id asc) with a warp bitonic
+//      sort/merge, the first k form the frontier (slot = rank, which names the
+//      draft row of the node), and
 //      their k children each enter the next level with
 //      log V = log V(parent) + lp (log of the product of confidences);
 //   3. a block-wide bitonic sort over all P candidates keeps the best n;
@@ -12,26 +14,36 @@
 //      the tree arrays are written.
 // log V is carried in fp64 so that the rounding of one path sum can only
 // reorder candidates whose values agree to ~1e-15 relative.
-#include <climits>
-
 #include "eagle_internal.h"
 
 namespace eagle {
 
 constexpr int kBuildThreads = 256;
+constexpr int kBuildWarps = kBuildThreads / 32;
+
+// Ranking key of a candidate: the order-preserving bit image of its fp64
+// log V with the lowest 12 mantissa bits replaced by (4095 - id), so that a
+// larger key means a larger log V and, among equal values, a lower id.  Two
+// values that differ only in those 12 bits (relative gap < 2^-40) rank by id.
+__device__ __forceinline__ uint64_t cand_key(double lv, int gid) {
+  uint64_t u = (uint64_t)__double_as_longlong(lv);
+  if (u == 0x8000000000000000ull) u = 0;  // -0 ranks with +0
+  u = (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
+  return (u & ~0xfffull) | (uint64_t)(4095 - gid);
+}
+__device__ __forceinline__ int key_gid(uint64_t key) { return 4095 - (int)(key & 0xfffull); }
 
 struct BuildSmem {
-  double* row_lp;  // [R*k]
-  double* cand_lv; // [P]
-  double* sort_lv; // [Ppow]
-  int* row_tok;    // [R*k]
-  int* cand_tok;   // [P]
-  int* cand_par;   // [P]   parent candidate id, -1 = root
-  int* cand_row;   // [P]   draft row of an expanded candidate, -1 otherwise
-  int* node_of;    // [P]   kept flag, then 1-based node id (0 = dropped)
-  int* sort_gid;   // [Ppow]
-  int* frontier;   // [32]
-  int* scan;       // [kBuildThreads + 1]
+  double* row_lp;    // [R*k] log-confidence of each row's top-k children
+  double* cand_lv;   // [P]   log V
+  uint64_t* sort_k;  // [Ppow]
+  int* row_tok;      // [R*k]
+  int* cand_tok;     // [P]
+  int* cand_par;     // [P]   parent candidate id, -1 = root
+  int* cand_row;     // [P]   draft row of an expanded candidate, -1 otherwise
+  int* node_of;      // [P]   kept flag, then 1-based node id (0 = dropped)
+  int* frontier;     // [32]
+  int* warp_cnt;     // [kBuildWarps]
 };
 
 __host__ __device__ inline int next_pow2(int x) {
@@ -40,17 +52,14 @@ __host__ __device__ inline int next_pow2(int x) {
   return p;
 }
 
-__device__ __forceinline__ bool cand_better(double la, int ga, double lb, int gb) {
-  return la > lb || (la == lb && ga < gb);
-}
-
+// row_tok / row_val: each draft row's top-k tokens and logits (descending),
+// row_lse: each row's log-sum-exp (also the tree's row_lse output).
 __global__ void __launch_bounds__(kBuildThreads)
-tree_expand_kernel(const ChunkStat* __restrict__ stats, const uint64_t* __restrict__ keys,
-                   int n_chunks, int R, int depth, int k, int n, eagle_tree_t out) {
+tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restrict__ row_val_g, int R, int depth,
+                   int k, int n, eagle_tree_t out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = kBuildThreads / 32;
   const int kk = k * k;
   const int P = k + (depth - 1) * kk;
   const int Ppow = next_pow2(P);
@@ -58,51 +67,52 @@ tree_expand_kernel(const ChunkStat* __restrict__ stats, const uint64_t* __restri
   BuildSmem sm;
   {
     unsigned char* p = smem_raw;
-    sm.row_lp = reinterpret_cast<double*>(p);  p += sizeof(double) * R * k;
-    sm.cand_lv = reinterpret_cast<double*>(p); p += sizeof(double) * P;
-    sm.sort_lv = reinterpret_cast<double*>(p); p += sizeof(double) * Ppow;
-    sm.row_tok = reinterpret_cast<int*>(p);    p += sizeof(int) * R * k;
-    sm.cand_tok = reinterpret_cast<int*>(p);   p += sizeof(int) * P;
-    sm.cand_par = reinterpret_cast<int*>(p);   p += sizeof(int) * P;
-    sm.cand_row = reinterpret_cast<int*>(p);   p += sizeof(int) * P;
-    sm.node_of = reinterpret_cast<int*>(p);    p += sizeof(int) * P;
-    sm.sort_gid = reinterpret_cast<int*>(p);   p += sizeof(int) * Ppow;
-    sm.frontier = reinterpret_cast<int*>(p);   p += sizeof(int) * 32;
-    sm.scan = reinterpret_cast<int*>(p);
+    sm.row_lp = reinterpret_cast<double*>(p);    p += sizeof(double) * R * k;
+    sm.cand_lv = reinterpret_cast<double*>(p);   p += sizeof(double) * P;
+    sm.sort_k = reinterpret_cast<uint64_t*>(p);  p += sizeof(uint64_t) * Ppow;
+    sm.row_tok = reinterpret_cast<int*>(p);      p += sizeof(int) * R * k;
+    sm.cand_tok = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
+    sm.cand_par = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
+    sm.cand_row = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
+    sm.node_of = reinterpret_cast<int*>(p);      p += sizeof(int) * P;
+    sm.frontier = reinterpret_cast<int*>(p);     p += sizeof(int) * 32;
+    sm.warp_cnt = reinterpret_cast<int*>(p);
   }
 
-  // 1. per-row log-sum-exp and top-k
-  for (int r = warp; r < R; r += nwarps) {
-    const size_t row = (size_t)b * R + r;
-    double lse = 0.0;
-    uint64_t key = 0;
-    warp_finalize_row(stats + row * n_chunks, keys + row * n_chunks * k, n_chunks, k, true, &lse, &key);
-    if (lane < k) {
-      sm.row_tok[r * k + lane] = key ? key_index(key) : -1;
-      sm.row_lp[r * k + lane] = key ? (double)key_value(key) - lse : -INFINITY;
-    }
-    if (lane == 0) out.row_lse[row] = lse;
+  // 1. each row's children and their log-confidence lp = logit - lse (fp64)
+  for (int e = tid; e < R * k; e += kBuildThreads) {
+    const size_t g = (size_t)b * R * k + e;
+    const int tok = row_tok_g[g];
+    sm.row_tok[e] = tok;
+    sm.row_lp[e] = tok >= 0 ? (double)row_val_g[g] - out.row_lse[(size_t)b * R + e / k] : -INFINITY;
+  }
+  for (int c = tid; c < P; c += kBuildThreads) {
+    sm.cand_row[c] = -1;
+    sm.node_of[c] = 0;
   }
   __syncthreads();
-
-  // 2. level by level
   for (int c = tid; c < k; c += kBuildThreads) {
     sm.cand_lv[c] = sm.row_lp[c];
     sm.cand_tok[c] = sm.row_tok[c];
     sm.cand_par[c] = -1;
-    sm.cand_row[c] = -1;
   }
   __syncthreads();
+
+  // 2. level by level: the k best candidates of the level form the frontier
   for (int level = 1; level < depth; ++level) {
     const int lo = level == 1 ? 0 : k + (level - 2) * kk;
     const int cnt = level == 1 ? k : kk;
-    for (int c = lo + tid; c < lo + cnt; c += kBuildThreads) {
-      const double lv = sm.cand_lv[c];
-      int rank = 0;
-      for (int o = lo; o < lo + cnt; ++o) rank += cand_better(sm.cand_lv[o], o, lv, c) ? 1 : 0;
-      if (rank < k) {
-        sm.frontier[rank] = c;
-        sm.cand_row[c] = 1 + (level - 1) * k + rank;
+    if (warp == 0) {
+      uint64_t list = 0;
+      for (int c0 = 0; c0 < cnt; c0 += 32) {
+        const int c = lo + c0 + lane;
+        const uint64_t key = c0 + lane < cnt ? cand_key(sm.cand_lv[c], c) : 0ull;
+        list = warp_merge_desc(list, warp_sort_desc(key));
+      }
+      if (lane < k) {
+        const int g = key_gid(list);
+        sm.frontier[lane] = g;
+        sm.cand_row[g] = 1 + (level - 1) * k + lane;
       }
     }
     __syncthreads();
@@ -115,50 +125,45 @@ tree_expand_kernel(const ChunkStat* __restrict__ stats, const uint64_t* __restri
       sm.cand_lv[g] = sm.cand_lv[parent] + sm.row_lp[row * k + r];
       sm.cand_tok[g] = sm.row_tok[row * k + r];
       sm.cand_par[g] = parent;
-      sm.cand_row[g] = -1;
     }
     __syncthreads();
   }
 
-  // 3. rerank: bitonic sort of all candidates, best first
-  for (int i = tid; i < Ppow; i += kBuildThreads) {
-    sm.sort_lv[i] = i < P ? sm.cand_lv[i] : -INFINITY;
-    sm.sort_gid[i] = i < P ? i : INT_MAX;
-  }
-  for (int i = tid; i < P; i += kBuildThreads) sm.node_of[i] = 0;
+  // 3. rerank: bitonic sort of all candidate keys, best first; keep n
+  for (int i = tid; i < Ppow; i += kBuildThreads) sm.sort_k[i] = i < P ? cand_key(sm.cand_lv[i], i) : 0ull;
   __syncthreads();
   for (int size = 2; size <= Ppow; size <<= 1) {
     for (int j = size >> 1; j > 0; j >>= 1) {
       for (int i = tid; i < Ppow; i += kBuildThreads) {
         const int o = i ^ j;
         if (o > i) {
+          const uint64_t a = sm.sort_k[i], c = sm.sort_k[o];
           const bool desc = (i & size) == 0;
-          const bool i_better = cand_better(sm.sort_lv[i], sm.sort_gid[i], sm.sort_lv[o], sm.sort_gid[o]);
-          if (desc != i_better) {
-            const double tl = sm.sort_lv[i]; sm.sort_lv[i] = sm.sort_lv[o]; sm.sort_lv[o] = tl;
-            const int tg = sm.sort_gid[i]; sm.sort_gid[i] = sm.sort_gid[o]; sm.sort_gid[o] = tg;
-          }
+          if (desc ? (a < c) : (a > c)) { sm.sort_k[i] = c; sm.sort_k[o] = a; }
         }
       }
       __syncthreads();
     }
   }
-  for (int i = tid; i < n; i += kBuildThreads) sm.node_of[sm.sort_gid[i]] = 1;
+  for (int i = tid; i < n; i += kBuildThreads) sm.node_of[key_gid(sm.sort_k[i])] = 1;
   __syncthreads();
 
-  // 4. renumber kept candidates by ascending id
+  // 4. renumber kept candidates by ascending id (block scan over contiguous ranges)
   const int per = (P + kBuildThreads - 1) / kBuildThreads;
   const int g0 = min(P, tid * per), g1 = min(P, g0 + per);
   int local = 0;
   for (int g = g0; g < g1; ++g) local += sm.node_of[g];
-  sm.scan[tid] = local;
-  __syncthreads();
-  if (tid == 0) {
-    int acc = 0;
-    for (int t = 0; t < kBuildThreads; ++t) { const int v = sm.scan[t]; sm.scan[t] = acc; acc += v; }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
   }
+  if (lane == 31) sm.warp_cnt[warp] = incl;
   __syncthreads();
-  int next = sm.scan[tid];
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += sm.warp_cnt[w];
+  int next = base + incl - local;
   for (int g = g0; g < g1; ++g)
     if (sm.node_of[g]) sm.node_of[g] = ++next;
   __syncthreads();
@@ -180,17 +185,37 @@ tree_expand_kernel(const ChunkStat* __restrict__ stats, const uint64_t* __restri
 
 size_t tree_build_smem_bytes(int R, int k, int P) {
   const int Ppow = next_pow2(P);
-  return sizeof(double) * ((size_t)R * k + P + Ppow) +
-         sizeof(int) * ((size_t)R * k + 4 * (size_t)P + Ppow + 32 + kBuildThreads + 1);
+  return sizeof(double) * ((size_t)R * k + P) + sizeof(uint64_t) * Ppow +
+         sizeof(int) * ((size_t)R * k + 4 * (size_t)P + 32 + kBuildWarps);
 }
 
-cudaError_t launch_tree_expand(const ChunkStat* stats, const uint64_t* keys, int n_chunks, int B, int R,
-                               int depth, int k, int n, const eagle_tree_t& out, cudaStream_t s) {
+// workspace: [chunk stats][chunk keys][row tokens B*R*k int32][row logits B*R*k float]
+size_t tree_build_ws_bytes(int B, int R, int V, int elem_bytes, int k) {
+  const size_t rows = (size_t)B * R;
+  return row_stats_ws_bytes((long long)rows, V, elem_bytes, k) + align_up(rows * k * sizeof(int32_t), 256) +
+         align_up(rows * k * sizeof(float), 256);
+}
+
+cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k, int n,
+                              const eagle_tree_t& out, void* ws, cudaStream_t s) {
+  const long long rows = (long long)B * R;
+  const int eb = dtype_bytes(dtype);
+  ChunkStat* cs = nullptr;
+  uint64_t* keys = nullptr;
+  row_stats_ws_layout(ws, rows, V, eb, k, &cs, &keys);
+  char* tail = static_cast<char*>(ws) + row_stats_ws_bytes(rows, V, eb, k);
+  int32_t* row_tok = reinterpret_cast<int32_t*>(tail);
+  float* row_val = reinterpret_cast<float*>(tail + align_up((size_t)rows * k * sizeof(int32_t), 256));
+  cudaError_t e = launch_row_chunk_stats(draft_logits, dtype, rows, V, k, true, cs, keys, s);
+  if (e != cudaSuccess) return e;
+  const int nc = plan_chunks(rows, V, eb).n_chunks;
+  e = launch_row_stats_finalize(cs, keys, rows, nc, k, row_tok, row_val, out.row_lse, s);
+  if (e != cudaSuccess) return e;
   const int P = k + (depth - 1) * k * k;
   const size_t smem = tree_build_smem_bytes(R, k, P);
-  cudaError_t e = ensure_smem_limit((const void*)tree_expand_kernel, smem);
+  e = ensure_smem_limit((const void*)tree_expand_kernel, smem);
   if (e != cudaSuccess) return e;
-  tree_expand_kernel<<<B, kBuildThreads, smem, s>>>(stats, keys, n_chunks, R, depth, k, n, out);
+  tree_expand_kernel<<<B, kBuildThreads, smem, s>>>(row_tok, row_val, R, depth, k, n, out);
   return cudaGetLastError();
 }
 
