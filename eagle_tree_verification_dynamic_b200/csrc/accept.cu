@@ -7,9 +7,9 @@
 // argmax and log-sum-exp per row.  Then one thread-block cluster per sequence
 // walks its tree.  Every CTA of the cluster evaluates the same scalar
 // decisions from the same data, so they stay in step; the vocabulary-wide
-// quantities a decision needs are computed cooperatively, each CTA on a
-// contiguous slice of the vocabulary, and combined through distributed shared
-// memory in a fixed order (so every CTA sees bit-identical totals):
+// quantities a decision needs are computed cooperatively, each thread on its
+// own contiguous slice of the vocabulary, and combined through distributed
+// shared memory in a fixed order (so every CTA sees bit-identical totals):
 //   * after a rejection at node j the current target becomes
 //     max(0, p - q) / Z.  After r rejections it equals
 //     max(0, p - t q) / F(t) with F(t) = sum_x max(0, p(x) - t q(x)),
@@ -17,6 +17,9 @@
 //     F at the new t;
 //   * the bonus token is the smallest x whose cumulative weight exceeds
 //     u_res * total (inverse CDF), found by a prefix scan over the slices.
+// A thread copies its slice of node j's target row and of its draft row into
+// shared memory on the first sweep at j; later sweeps at j read only that
+// copy (each thread only ever reads its own slice, so no barrier is needed).
 #include <cooperative_groups.h>
 
 #include "eagle_internal.h"
@@ -27,43 +30,21 @@ namespace eagle {
 
 constexpr int kAcceptThreads = 512;
 constexpr int kAcceptWarps = kAcceptThreads / 32;
+constexpr int kCacheBytesPerCta = 64 * 1024;  // both row slices of one CTA
+constexpr int kMaxCluster = 16;
 
 template <typename T>
 __device__ __forceinline__ float load_logit(const T* p) { return Elem<T>::load(p); }
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__host__ __device__ constexpr int slice_max() { return kCacheBytesPerCta / (2 * kAcceptThreads * (int)sizeof(T)); }
 
 struct SweepArgs {
-  const void* trow;   // target row j
-  const void* drow;   // draft row draft_row[j] (unused when t == 0)
   Split2 lse_t, lse_d, t;
-  bool use_q;         // false: weights are p itself
+  bool use_q;  // false: weights are p itself
 };
-
-constexpr int kSegChunk = 16;
-
-// Weights of tokens base .. base+15 (0 past x1) under the current target:
-// p(x), or max(0, p(x) - t q(x)).  All loads are issued before any use.
-template <typename T>
-__device__ __forceinline__ void sweep_weights(const SweepArgs& a, int base, int x1, float* w) {
-  const T* tr = static_cast<const T*>(a.trow);
-  const T* dr = static_cast<const T*>(a.drow);
-  float lt[kSegChunk], ld[kSegChunk];
-#pragma unroll
-  for (int i = 0; i < kSegChunk; ++i) lt[i] = base + i < x1 ? load_logit(tr + base + i) : -INFINITY;
-  if (a.use_q) {
-#pragma unroll
-    for (int i = 0; i < kSegChunk; ++i) ld[i] = base + i < x1 ? load_logit(dr + base + i) : 0.f;
-  }
-#pragma unroll
-  for (int i = 0; i < kSegChunk; ++i) {
-    const float p = exp_minus(lt[i], a.lse_t);
-    if (!a.use_q) {
-      w[i] = p;
-    } else {
-      const float q = exp_minus(ld[i], a.lse_d);
-      w[i] = fmaxf(0.f, fmaf(-a.t.lo, q, fmaf(-a.t.hi, q, p)));
-    }
-  }
-}
 
 struct AcceptSmem {
   int tok[EAGLE_MAX_NODES];
@@ -73,6 +54,38 @@ struct AcceptSmem {
   double lane_sum[kAcceptThreads];
   double prefix[kAcceptThreads + 1];
   double cta_total;
+};
+
+// This thread's slice [x0, x1) of the current rows, cached in shared memory.
+template <typename T>
+struct Slice {
+  T* tc;  // target row slice
+  T* dc;  // draft row slice
+  int x0, x1;
+  int cached_t, cached_d;
+
+  __device__ void load(const T* src, T* dst) const {
+    constexpr int kChunk = 8;
+    for (int b = x0; b < x1; b += kChunk) {
+      T v[kChunk];
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i)
+        if (b + i < x1) v[i] = src[b + i];
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i)
+        if (b + i < x1) dst[b - x0 + i] = v[i];
+    }
+  }
+  __device__ void ensure(const T* trow, int tkey, const T* drow, int dkey) {
+    if (cached_t != tkey) { load(trow, tc); cached_t = tkey; }
+    if (drow && cached_d != dkey) { load(drow, dc); cached_d = dkey; }
+  }
+  __device__ __forceinline__ float weight(const SweepArgs& a, int i) const {
+    const float p = exp_minus(to_f(tc[i]), a.lse_t);
+    if (!a.use_q) return p;
+    const float q = exp_minus(to_f(dc[i]), a.lse_d);
+    return fmaxf(0.f, fmaf(-a.t.lo, q, fmaf(-a.t.hi, q, p)));
+  }
 };
 
 // Deterministic block sum; result valid in every thread.
@@ -104,41 +117,23 @@ __device__ double cluster_sum(double cta_value, AcceptSmem& sm, cg::cluster_grou
 }
 
 template <typename T>
-__device__ double sweep_total(const SweepArgs& a, int V, AcceptSmem& sm, cg::cluster_group& cluster) {
-  const int nt = (int)cluster.num_blocks() * kAcceptThreads;
-  const int gt = (int)cluster.block_rank() * kAcceptThreads + threadIdx.x;
-  const int seg = (V + nt - 1) / nt;
-  const int x0 = min(V, gt * seg), x1 = min(V, x0 + seg);
+__device__ double sweep_total(const Slice<T>& sl, const SweepArgs& a, AcceptSmem& sm, cg::cluster_group& cluster) {
   double acc = 0.0;
-  for (int base = x0; base < x1; base += kSegChunk) {
-    float w[kSegChunk];
-    sweep_weights<T>(a, base, x1, w);
-#pragma unroll
-    for (int i = 0; i < kSegChunk; ++i) acc += (double)w[i];
-  }
+  for (int i = 0; i < sl.x1 - sl.x0; ++i) acc += (double)sl.weight(a, i);
   return cluster_sum(block_sum(acc, sm), sm, cluster, nullptr);
 }
 
 // Inverse CDF over the weights: smallest x with cumsum_x > u * total.  Writes
 // the token to *out from the one thread that owns the crossing; returns the
-// total weight (every thread).  Each thread owns a contiguous slice of the
-// vocabulary and sums it in token order, in fp64, element by element; the
-// owner's rescan repeats exactly those additions.
+// total weight (every thread).  Each thread sums its slice in token order, in
+// fp64, element by element; the owner's rescan repeats exactly those additions.
 template <typename T>
-__device__ double sweep_sample(const SweepArgs& a, int V, float u, AcceptSmem& sm,
+__device__ double sweep_sample(const Slice<T>& sl, const SweepArgs& a, float u, AcceptSmem& sm,
                                cg::cluster_group& cluster, int32_t* out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nt = (int)cluster.num_blocks() * kAcceptThreads;
-  const int gt = (int)cluster.block_rank() * kAcceptThreads + tid;
-  const int seg = (V + nt - 1) / nt;
-  const int x0 = min(V, gt * seg), x1 = min(V, x0 + seg);
+  const int len = sl.x1 - sl.x0;
   double mine = 0.0;
-  for (int base = x0; base < x1; base += kSegChunk) {
-    float w[kSegChunk];
-    sweep_weights<T>(a, base, x1, w);
-#pragma unroll
-    for (int i = 0; i < kSegChunk; ++i) mine += (double)w[i];
-  }
+  for (int i = 0; i < len; ++i) mine += (double)sl.weight(a, i);
   // Block exclusive prefix of the per-thread sums, summed serially (lane order
   // within a warp, then warp order) so the prefixes never decrease and the
   // ownership intervals [prefix[t], prefix[t+1]) tile [0, total) exactly.
@@ -170,16 +165,11 @@ __device__ double sweep_sample(const SweepArgs& a, int V, float u, AcceptSmem& s
     if (start <= thr && thr < end) {
       double run = 0.0;
       int pick = -1, last_nz = -1;
-      for (int base = x0; base < x1 && pick < 0; base += kSegChunk) {
-        float w[kSegChunk];
-        sweep_weights<T>(a, base, x1, w);
-#pragma unroll
-        for (int i = 0; i < kSegChunk; ++i) {
-          if (pick >= 0 || base + i >= x1) continue;
-          if (w[i] > 0.f) last_nz = base + i;
-          run += (double)w[i];
-          if (my_off + (sm.prefix[tid] + run) > thr) pick = base + i;
-        }
+      for (int i = 0; i < len; ++i) {
+        const float w = sl.weight(a, i);
+        if (w > 0.f) last_nz = sl.x0 + i;
+        run += (double)w;
+        if (my_off + (sm.prefix[tid] + run) > thr) { pick = sl.x0 + i; break; }
       }
       *out = pick >= 0 ? pick : last_nz;
     }
@@ -187,7 +177,6 @@ __device__ double sweep_sample(const SweepArgs& a, int V, float u, AcceptSmem& s
   return total;
 }
 
-template <typename T>
 __device__ __forceinline__ int argmax_of_row(const ChunkStat* st, const uint64_t* keys, int t_chunks,
                                              bool want_lse, double* lse) {
   uint64_t key = 0;
@@ -197,14 +186,15 @@ __device__ __forceinline__ int argmax_of_row(const ChunkStat* st, const uint64_t
 }
 
 template <typename T, bool STOCH>
-__global__ void __launch_bounds__(kAcceptThreads)
+__global__ void __launch_bounds__(kAcceptThreads, 2)
 accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const double* __restrict__ dlse,
                    int R, int V, int n, int depth, const ChunkStat* __restrict__ tstats,
                    const uint64_t* __restrict__ tkeys, int t_chunks, const int32_t* __restrict__ tokens,
                    const int32_t* __restrict__ parents, const int32_t* __restrict__ draft_row,
                    const float* __restrict__ uniforms, int32_t* __restrict__ accepted_len,
-                   int32_t* __restrict__ path, int32_t* __restrict__ bonus) {
+                   int32_t* __restrict__ path, int32_t* __restrict__ bonus, int slice) {
   __shared__ AcceptSmem sm;
+  extern __shared__ __align__(16) unsigned char cache_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = (int)cluster.num_blocks();
   const int b = blockIdx.x / CL;
@@ -221,6 +211,18 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   }
   __syncthreads();
 
+  Slice<T> sl;
+  {
+    const int gt = (int)cluster.block_rank() * kAcceptThreads + tid;
+    sl.x0 = min(V, gt * slice);
+    sl.x1 = min(V, sl.x0 + slice);
+    T* base = reinterpret_cast<T*>(cache_raw);
+    sl.tc = base + (size_t)tid * slice;
+    sl.dc = base + (size_t)(kAcceptThreads + tid) * slice;
+    sl.cached_t = -1;
+    sl.cached_d = -1;
+  }
+
   const size_t trow0 = (size_t)b * (n + 1);
   auto row_stat = [&](int j) { return tstats + (trow0 + j) * t_chunks; };
   auto row_keys = [&](int j) { return tkeys + (trow0 + j) * t_chunks; };
@@ -229,7 +231,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
 
   int j = 0, plen = 0;
   double lse_t = 0.0;
-  int amax = argmax_of_row<T>(row_stat(0), row_keys(0), t_chunks, STOCH, &lse_t);
+  int amax = argmax_of_row(row_stat(0), row_keys(0), t_chunks, STOCH, &lse_t);
   double t = 0.0, F = 1.0;
   bool rejected_here = false;
 
@@ -263,10 +265,11 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
         int nc = c + 1;
         while (nc <= n && sm.par[nc - 1] != j) ++nc;
         if (nc <= n) {  // another sibling will be tested: need F(t)
+          sl.ensure(trow, j, drow, r);
           SweepArgs a;
-          a.trow = trow; a.drow = drow; a.use_q = true;
+          a.use_q = true;
           a.lse_t.set(lse_t); a.lse_d.set(lse_d); a.t.set(t);
-          F = sweep_total<T>(a, V, sm, cluster);
+          F = sweep_total<T>(sl, a, sm, cluster);
           if (!(F > 0.0)) break;  // p == q left nothing: keep the walk here
         }
         c = nc;
@@ -279,7 +282,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     t = 0.0;
     F = 1.0;
     rejected_here = false;
-    amax = argmax_of_row<T>(row_stat(j), row_keys(j), t_chunks, STOCH, &lse_t);
+    amax = argmax_of_row(row_stat(j), row_keys(j), t_chunks, STOCH, &lse_t);
   }
 
   if (leader) {
@@ -291,14 +294,14 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     return;
   }
   const int r = sm.drow[j];
+  const bool use_q = rejected_here && r >= 0;
+  sl.ensure(tgt + (trow0 + j) * (size_t)V, j, use_q ? dft + ((size_t)b * R + r) * (size_t)V : nullptr, r);
   SweepArgs a;
-  a.trow = tgt + (trow0 + j) * (size_t)V;
-  a.drow = r >= 0 ? dft + ((size_t)b * R + r) * (size_t)V : nullptr;
-  a.use_q = rejected_here && r >= 0;
+  a.use_q = use_q;
   a.lse_t.set(lse_t);
   a.lse_d.set(r >= 0 ? dlse[(size_t)b * R + r] : 0.0);
   a.t.set(t);
-  const double total = sweep_sample<T>(a, V, u_res[j], sm, cluster, bonus + b);
+  const double total = sweep_sample<T>(sl, a, u_res[j], sm, cluster, bonus + b);
   if (!(total > 0.0) && leader) bonus[b] = amax;  // nothing left to sample from
 }
 
@@ -307,11 +310,9 @@ size_t accept_ws_bytes(int B, int n, int V, int dtype) {
   return row_stats_ws_bytes((long long)B * (n + 1), V, dtype_bytes(dtype), 1);
 }
 
-static int accept_cluster_size(int V) {
-  int cl = V / 8192;
-  if (cl < 1) cl = 1;
-  if (cl > 8) cl = 8;
-  return cl;
+int accept_max_vocab(int dtype) {
+  const int sm = dtype == EAGLE_F32 ? slice_max<float>() : slice_max<__nv_bfloat16>();
+  return kMaxCluster * kAcceptThreads * sm;
 }
 
 template <typename T, bool STOCH>
@@ -320,11 +321,29 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
                                const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                                const float* uniforms, int B, int32_t* acc_len, int32_t* path,
                                int32_t* bonus, cudaStream_t s) {
-  const int cl = STOCH ? accept_cluster_size(V) : 1;
+  int cl = 1, slice = 0;
+  size_t dyn = 0;
+  if (STOCH) {
+    const int per_cta = kAcceptThreads * slice_max<T>();
+    cl = (V + per_cta - 1) / per_cta;
+    if (cl < 1) cl = 1;
+    slice = (V + cl * kAcceptThreads - 1) / (cl * kAcceptThreads);
+    dyn = (size_t)2 * kAcceptThreads * slice * sizeof(T);
+    cudaError_t e = ensure_smem_limit((const void*)accept_walk_kernel<T, STOCH>, dyn + sizeof(AcceptSmem));
+    if (e != cudaSuccess) return e;
+    if (cl > 8) {
+      static bool np_set = false;
+      if (!np_set) {
+        e = cudaFuncSetAttribute(accept_walk_kernel<T, STOCH>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        np_set = true;
+      }
+    }
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(B * cl));
   cfg.blockDim = dim3(kAcceptThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = dyn;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -335,7 +354,7 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, accept_walk_kernel<T, STOCH>, static_cast<const T*>(tgt),
                             static_cast<const T*>(dft), dlse, R, V, n, depth, st, keys, t_chunks, tokens,
-                            parents, draft_row, uniforms, acc_len, path, bonus);
+                            parents, draft_row, uniforms, acc_len, path, bonus, slice);
 }
 
 cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,

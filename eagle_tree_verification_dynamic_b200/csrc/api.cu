@@ -181,6 +181,7 @@ eagle_status eagle_accept(const void* target_logits, int target_dtype, const voi
     if (!valid_dtype(draft_dtype)) return EAGLE_ERR_DTYPE;
     if (draft_dtype != target_dtype) return EAGLE_ERR_DTYPE;
     if (R <= 0) return EAGLE_ERR_SHAPE;
+    if (V > accept_max_vocab(target_dtype)) return EAGLE_ERR_LIMIT;
   }
   if (B <= 0 || n <= 0 || V <= 0 || depth <= 0) return EAGLE_ERR_SHAPE;
   if (n > EAGLE_MAX_NODES || depth > EAGLE_MAX_DEPTH) return EAGLE_ERR_LIMIT;

@@ -151,24 +151,29 @@ attn_simt_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 }
 
 // out[b][i][h][:] = sum_s w_s O_s / sum_s w_s, w_s = exp(lse_s - max lse).
+// The split loops are unrolled so their independent loads are in flight together.
 template <int D>
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                     int S, int B, int n, int Hq, __nv_bfloat16* __restrict__ out) {
   const int ih = blockIdx.x, b = blockIdx.y;
   const int i = ih / Hq, h = ih - i * Hq;
   const int d = threadIdx.x;
+  const size_t stride = (size_t)B * n * Hq;  // between splits
+  const size_t slot0 = ((size_t)b * n + i) * Hq + h;
   float mx = -INFINITY;
-  for (int s = 0; s < S; ++s) mx = fmaxf(mx, part_lse[(((size_t)s * B + b) * n + i) * Hq + h]);
+#pragma unroll 8
+  for (int s = 0; s < S; ++s) mx = fmaxf(mx, part_lse[s * stride + slot0]);
   float num = 0.f, den = 0.f;
   if (mx > -INFINITY) {
+#pragma unroll 8
     for (int s = 0; s < S; ++s) {
-      const size_t slot = (((size_t)s * B + b) * n + i) * Hq + h;
+      const size_t slot = s * stride + slot0;
       const float w = __expf(part_lse[slot] - mx);
       den += w;
       num = fmaf(w, part_o[slot * D + d], num);
     }
   }
-  out[(((size_t)b * n + i) * Hq + h) * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+  out[slot0 * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
 }
 
 AttnPlan plan_attention(int B, int n, int Hq, int Hkv, int Lmax, int window) {

@@ -58,6 +58,7 @@ struct TcLayout {
 };
 
 struct TcBars {
+  uint64_t q_full;
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t s_full;
@@ -78,6 +79,7 @@ struct TcParams {
   float* part_lse;
   int* err;
   int Lmax, n, Hq, Hkv, window, n_splits, chunk, row_groups;
+  int q_by_tma;      // 1: Q rows arrive by TMA (G divides 128), 0: gathered by the threads
   float scale_log2;  // softmax scale * log2(e)
 };
 
@@ -85,7 +87,7 @@ template <int D>
 __global__ void __launch_bounds__(kTcThreads, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_vt,
-               const TcParams p) {
+               const __grid_constant__ CUtensorMap tm_q, const TcParams p) {
   using Lay = TcLayout<D>;
   extern __shared__ __align__(1024) unsigned char smem[];
   TcBars* bars = reinterpret_cast<TcBars*>(smem + Lay::kBarOff);
@@ -135,6 +137,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
   // ---- set-up: barriers, TMEM, Q tile
   if (tid == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&bars->full[i]), 1);
       mbar_init(smem_u32(&bars->empty[i]), 1);
@@ -145,6 +148,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     mbar_init(smem_u32(&bars->mma_idle), 1);
     bars->abort = 0;
     fence_mbar_init();
+    if (p.q_by_tma) {
+      // the 128 query rows of this tile = (node, head-in-group) pairs: a box of
+      // {64 dims, G heads, 128/G nodes} of q viewed as [B*n][Hq][D]
+      const uint32_t qb = smem_u32(&bars->q_full);
+      mbar_arrive_expect_tx(qb, Lay::kQBytes);
+      const int rows_i = kRowsPerCta / G;
+      for (int a = 0; a < Lay::kAtoms; ++a)
+        tma_load_3d(s_base + Lay::kQOff + a * 16384, &tm_q, a * 64, g * G, b * p.n + rg * rows_i, qb);
+    }
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_kt);
@@ -154,20 +166,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     tmem_alloc(smem_u32(&bars->tmem_base), Lay::kTmemCols);
     tmem_relinquish();
   }
-  // Q rows (bf16) -> 128-byte swizzled K-major tile
-  for (int e = tid; e < 128 * Lay::kAtoms * 8; e += kTcThreads) {
-    const int r = e / (Lay::kAtoms * 8);
-    const int a = (e / 8) % Lay::kAtoms;
-    const int c = e % 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    const int rr = row0 + r;
-    if (rr < rows) {
-      const int i = rr / G, h = g * G + rr % G;
-      v = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * p.n + i) * p.Hq + h) * D + a * 64 + c * 8);
+  if (!p.q_by_tma) {
+    // Q rows (bf16) -> 128-byte swizzled K-major tile; all loads issued first
+    constexpr int kVec = 128 * Lay::kAtoms * 8;
+    constexpr int kPer = (kVec + kTcThreads - 1) / kTcThreads;
+    uint4 v[kPer];
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int e = tid + t * kTcThreads;
+      v[t] = make_uint4(0, 0, 0, 0);
+      if (e < kVec) {
+        const int r = e / (Lay::kAtoms * 8), a = (e / 8) % Lay::kAtoms, c = e % 8;
+        const int rr = row0 + r;
+        if (rr < rows) {
+          const int i = rr / G, h = g * G + rr % G;
+          v[t] = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * p.n + i) * p.Hq + h) * D + a * 64 + c * 8);
+        }
+      }
     }
-    *reinterpret_cast<uint4*>(smem + Lay::kQOff + a * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int e = tid + t * kTcThreads;
+      if (e < kVec) {
+        const int r = e / (Lay::kAtoms * 8), a = (e / 8) % Lay::kAtoms, c = e % 8;
+        *reinterpret_cast<uint4*>(smem + Lay::kQOff + a * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) = v[t];
+      }
+    }
+    fence_proxy_async_smem();
   }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -198,7 +224,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         }
         ++issued;
       }
-      // drain: wait until every issued stage has landed before the CTA may exit
+      // drain: wait until every issued copy has landed before the CTA may exit
+      if (p.q_by_tma) mbar_wait_drain(smem_u32(&bars->q_full), 0, 200000000ull);
       for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
         mbar_wait_drain(smem_u32(&bars->full[j % kStages]), (j / kStages) & 1, 200000000ull);
     }
@@ -210,7 +237,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const uint32_t t_s = tmem + Lay::kColS, t_o = tmem + Lay::kColO;
       const uint32_t q_addr = s_base + Lay::kQOff;
       const uint32_t p_addr = s_base + Lay::kPOff;
-      for (int j = 0; j < ntiles; ++j) {
+      const bool q_ok = !p.q_by_tma || mbar_wait(smem_u32(&bars->q_full), 0, abort);
+      for (int j = 0; j < ntiles && q_ok; ++j) {
         const int st = j % kStages;
         if (!mbar_wait(smem_u32(&bars->full[st]), (j / kStages) & 1, abort)) break;
         tc_fence_after();
@@ -403,7 +431,17 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
     if (!make_map(&mkt, kt, 3, dims, str, box) || !make_map(&mvt, vt, 3, dims, str, box))
       return cudaErrorInvalidValue;
   }
+  const int G = Hq / Hkv;
+  CUtensorMap mq;
+  const bool q_tma = (kRowsPerCta % G) == 0;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)B * n};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)(q_tma ? G : 1), (cuuint32_t)(q_tma ? kRowsPerCta / G : 1)};
+    if (!make_map(&mq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
   TcParams p;
+  p.q_by_tma = q_tma ? 1 : 0;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.plen = plen;
   p.mask = mask;
@@ -424,7 +462,7 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
   cudaError_t e = ensure_smem_limit((const void*)attn_tc_kernel<D>, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(plan.n_splits + 1, Hkv, B * p.row_groups);
-  attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(mk, mv, mkt, mvt, p);
+  attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(mk, mv, mkt, mvt, mq, p);
   return cudaGetLastError();
 }
 

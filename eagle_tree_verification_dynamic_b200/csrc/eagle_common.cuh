@@ -159,8 +159,15 @@ __device__ __forceinline__ void warp_finalize_row(const ChunkStat* st, const uin
     s = warp_sum_d(s);
     *lse_out = s > 0.0 ? kLn2 * ((double)e + log2(s)) : -INFINITY;
   }
-  uint64_t list = lane < k ? keys[lane] : 0ull;
-  for (int c = 1; c < n_chunks; ++c) list = warp_merge_desc(list, lane < k ? keys[c * k + lane] : 0ull);
+  uint64_t list = 0ull;
+  for (int c0 = 0; c0 < n_chunks; c0 += 8) {  // 8 chunk lists in flight, then merged
+    uint64_t kv[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) kv[t] = (lane < k && c0 + t < n_chunks) ? keys[(c0 + t) * k + lane] : 0ull;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (c0 + t < n_chunks) list = warp_merge_desc(list, kv[t]);
+  }
   *key_out = list;
 }
 

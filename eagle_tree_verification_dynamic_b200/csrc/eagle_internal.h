@@ -64,6 +64,7 @@ cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, c
 
 // ---- accept (accept.cu)
 size_t accept_ws_bytes(int B, int n, int V, int dtype);
+int accept_max_vocab(int dtype);  // largest V the sampled walk supports
 cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,
                           int R, const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                           const float* uniforms, int B, int n, int V, int depth, int32_t* accepted_len,

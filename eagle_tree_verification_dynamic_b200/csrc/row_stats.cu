@@ -17,7 +17,7 @@ namespace eagle {
 
 constexpr int kStatThreads = 256;
 constexpr int kStatWarps = kStatThreads / 32;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;
 
 struct LaneTop2 {
   float s1, s2;
@@ -168,10 +168,17 @@ row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
   }
   __syncthreads();
 
+  // merge the warps' lists pairwise: 3 rounds for 8 warps
+  for (int step = 1; step < kStatWarps; step <<= 1) {
+    if ((warp & (2 * step - 1)) == 0 && warp + step < kStatWarps) {
+      const uint64_t m = warp_merge_desc(lane < k ? s_keys[warp][lane] : 0ull,
+                                         lane < k ? s_keys[warp + step][lane] : 0ull);
+      if (lane < k) s_keys[warp][lane] = m;
+    }
+    __syncthreads();
+  }
   if (warp == 0) {
-    uint64_t merged = lane < k ? s_keys[0][lane] : 0ull;
-    for (int w = 1; w < kStatWarps; ++w)
-      merged = warp_merge_desc(merged, lane < k ? s_keys[w][lane] : 0ull);
+    const uint64_t merged = lane < k ? s_keys[0][lane] : 0ull;
     const size_t slot = (size_t)row * n_chunks + chunk;
     if (lane < k) keys[slot * k + lane] = merged;
     if (LSE && lane == 0) {

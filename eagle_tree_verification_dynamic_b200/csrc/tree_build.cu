@@ -4,9 +4,9 @@
 //      one-warp-per-row merge give each draft row's log-sum-exp and top-k;
 //   1. lp = logit - lse turns the top-k logits into log-confidences;
 //   2. level 1 = the root's k children; for each level up to depth-1, rank the
-//      level's candidates by (log V desc, candidate id asc) with a warp bitonic
-//      sort/merge, the first k form the frontier (slot = rank, which names the
-//      draft row of the node), and
+//      level's candidates by (log V desc, candidate id asc) (each candidate
+//      counts the larger keys of its level), the first k form the frontier
+//      (slot = rank, which names the draft row of the node), and
 //      their k children each enter the next level with
 //      log V = log V(parent) + lp (log of the product of confidences);
 //   3. a block-wide bitonic sort over all P candidates keeps the best n;
@@ -18,7 +18,7 @@
 
 namespace eagle {
 
-constexpr int kBuildThreads = 256;
+constexpr int kBuildThreads = 1024;
 constexpr int kBuildWarps = kBuildThreads / 32;
 
 // Ranking key of a candidate: the order-preserving bit image of its fp64
@@ -36,7 +36,7 @@ __device__ __forceinline__ int key_gid(uint64_t key) { return 4095 - (int)(key &
 struct BuildSmem {
   double* row_lp;    // [R*k] log-confidence of each row's top-k children
   double* cand_lv;   // [P]   log V
-  uint64_t* sort_k;  // [Ppow]
+  uint64_t* sort_k;  // [max(Ppow, 2*threads)] keys / exchange buffers
   int* row_tok;      // [R*k]
   int* cand_tok;     // [P]
   int* cand_par;     // [P]   parent candidate id, -1 = root
@@ -63,13 +63,14 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   const int kk = k * k;
   const int P = k + (depth - 1) * kk;
   const int Ppow = next_pow2(P);
+  const int nsort = Ppow > 2 * kBuildThreads ? Ppow : 2 * kBuildThreads;
 
   BuildSmem sm;
   {
     unsigned char* p = smem_raw;
     sm.row_lp = reinterpret_cast<double*>(p);    p += sizeof(double) * R * k;
     sm.cand_lv = reinterpret_cast<double*>(p);   p += sizeof(double) * P;
-    sm.sort_k = reinterpret_cast<uint64_t*>(p);  p += sizeof(uint64_t) * Ppow;
+    sm.sort_k = reinterpret_cast<uint64_t*>(p);  p += sizeof(uint64_t) * nsort;
     sm.row_tok = reinterpret_cast<int*>(p);      p += sizeof(int) * R * k;
     sm.cand_tok = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
     sm.cand_par = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
@@ -99,20 +100,20 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   __syncthreads();
 
   // 2. level by level: the k best candidates of the level form the frontier
+  //    (a candidate's rank = how many candidates of its level have a larger key)
   for (int level = 1; level < depth; ++level) {
     const int lo = level == 1 ? 0 : k + (level - 2) * kk;
     const int cnt = level == 1 ? k : kk;
-    if (warp == 0) {
-      uint64_t list = 0;
-      for (int c0 = 0; c0 < cnt; c0 += 32) {
-        const int c = lo + c0 + lane;
-        const uint64_t key = c0 + lane < cnt ? cand_key(sm.cand_lv[c], c) : 0ull;
-        list = warp_merge_desc(list, warp_sort_desc(key));
-      }
-      if (lane < k) {
-        const int g = key_gid(list);
-        sm.frontier[lane] = g;
-        sm.cand_row[g] = 1 + (level - 1) * k + lane;
+    for (int c = tid; c < cnt; c += kBuildThreads) sm.sort_k[c] = cand_key(sm.cand_lv[lo + c], lo + c);
+    __syncthreads();
+    for (int c = tid; c < cnt; c += kBuildThreads) {
+      const uint64_t mine = sm.sort_k[c];
+      int rank = 0;
+#pragma unroll 8
+      for (int o = 0; o < cnt; ++o) rank += sm.sort_k[o] > mine ? 1 : 0;
+      if (rank < k) {
+        sm.frontier[rank] = lo + c;
+        sm.cand_row[lo + c] = 1 + (level - 1) * k + rank;
       }
     }
     __syncthreads();
@@ -129,23 +130,48 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     __syncthreads();
   }
 
-  // 3. rerank: bitonic sort of all candidate keys, best first; keep n
-  for (int i = tid; i < Ppow; i += kBuildThreads) sm.sort_k[i] = i < P ? cand_key(sm.cand_lv[i], i) : 0ull;
-  __syncthreads();
-  for (int size = 2; size <= Ppow; size <<= 1) {
-    for (int j = size >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < Ppow; i += kBuildThreads) {
-        const int o = i ^ j;
-        if (o > i) {
-          const uint64_t a = sm.sort_k[i], c = sm.sort_k[o];
-          const bool desc = (i & size) == 0;
-          if (desc ? (a < c) : (a > c)) { sm.sort_k[i] = c; sm.sort_k[o] = a; }
+  // 3. rerank: bitonic sort of all candidate keys, best first; keep n.  With
+  //    Ppow <= blockDim each thread holds one key: partners closer than 32 are
+  //    exchanged by shuffles, farther ones through a double-buffered array.
+  if (Ppow <= kBuildThreads) {
+    uint64_t key = tid < P ? cand_key(sm.cand_lv[tid], tid) : 0ull;
+    int buf = 0;
+    uint64_t* xbuf[2] = {sm.sort_k, sm.sort_k + kBuildThreads};
+    for (int size = 2; size <= Ppow; size <<= 1) {
+      const bool desc = (tid & size) == 0;
+      for (int j = size >> 1; j > 0; j >>= 1) {
+        uint64_t o;
+        if (j >= 32) {
+          xbuf[buf][tid] = key;
+          __syncthreads();
+          o = xbuf[buf][tid ^ j];
+          buf ^= 1;
+        } else {
+          o = __shfl_xor_sync(kFull, key, j);
         }
+        const bool lower = (tid & j) == 0;
+        key = (lower == desc) ? umax64(key, o) : umin64(key, o);
       }
-      __syncthreads();
     }
+    if (tid < n) sm.node_of[key_gid(key)] = 1;
+  } else {
+    for (int i = tid; i < Ppow; i += kBuildThreads) sm.sort_k[i] = i < P ? cand_key(sm.cand_lv[i], i) : 0ull;
+    __syncthreads();
+    for (int size = 2; size <= Ppow; size <<= 1) {
+      for (int j = size >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < Ppow; i += kBuildThreads) {
+          const int o = i ^ j;
+          if (o > i) {
+            const uint64_t a = sm.sort_k[i], c = sm.sort_k[o];
+            const bool desc = (i & size) == 0;
+            if (desc ? (a < c) : (a > c)) { sm.sort_k[i] = c; sm.sort_k[o] = a; }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int i = tid; i < n; i += kBuildThreads) sm.node_of[key_gid(sm.sort_k[i])] = 1;
   }
-  for (int i = tid; i < n; i += kBuildThreads) sm.node_of[key_gid(sm.sort_k[i])] = 1;
   __syncthreads();
 
   // 4. renumber kept candidates by ascending id (block scan over contiguous ranges)
@@ -185,7 +211,8 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
 
 size_t tree_build_smem_bytes(int R, int k, int P) {
   const int Ppow = next_pow2(P);
-  return sizeof(double) * ((size_t)R * k + P) + sizeof(uint64_t) * Ppow +
+  const int nsort = Ppow > 2 * kBuildThreads ? Ppow : 2 * kBuildThreads;
+  return sizeof(double) * ((size_t)R * k + P) + sizeof(uint64_t) * nsort +
          sizeof(int) * ((size_t)R * k + 4 * (size_t)P + 32 + kBuildWarps);
 }
 

@@ -205,7 +205,8 @@ EAGLE_API eagle_status eagle_tree_attention(const void* q, const void* k_cache, 
  *     greedy.
  *   tokens, parents [B][n], draft_row [B][n+1]: the tree.
  *   accepted_len [B], path [B][depth] (accepted node ids, -1 padded), bonus [B].
- * Limits: n <= EAGLE_MAX_NODES, depth <= EAGLE_MAX_DEPTH.
+ * Limits: n <= EAGLE_MAX_NODES, depth <= EAGLE_MAX_DEPTH; for sampling
+ * V <= 262144 (bf16) or 131072 (fp32).
  * Workspace: eagle_accept_workspace_bytes. */
 EAGLE_API size_t eagle_accept_workspace_bytes(int B, int n, int V, int target_dtype);
 EAGLE_API eagle_status eagle_accept(const void* target_logits, int target_dtype, const void* draft_logits,
