@@ -5,7 +5,8 @@
 //
 // Target rows first go through the vocabulary sweep (row_stats.cu, k = 1):
 // argmax and log-sum-exp per row.  Then one thread-block cluster per sequence
-// walks its tree.  Every CTA of the cluster evaluates the same scalar
+// walks its tree; a prologue stages every per-node value a decision reads
+// (argmax, log-sum-exps, each child's target and draft logit) in shared memory.  Every CTA of the cluster evaluates the same scalar
 // decisions from the same data, so they stay in step; the vocabulary-wide
 // quantities a decision needs are computed cooperatively, each thread on its
 // own contiguous slice of the vocabulary, and combined through distributed
@@ -50,6 +51,11 @@ struct AcceptSmem {
   int tok[EAGLE_MAX_NODES];
   int par[EAGLE_MAX_NODES];
   int drow[EAGLE_MAX_NODES + 1];
+  int amax[EAGLE_MAX_NODES + 1];       // target argmax of row j
+  double lse_t[EAGLE_MAX_NODES + 1];   // target log-sum-exp of row j
+  double lse_d[EAGLE_MAX_NODES + 1];   // log-sum-exp of node j's draft row
+  float tl[EAGLE_MAX_NODES + 1];       // child c: target logit of its token in its parent's row
+  float dl[EAGLE_MAX_NODES + 1];       // child c: draft logit of its token in its parent's draft row
   double warp_part[kAcceptWarps];
   double lane_sum[kAcceptThreads];
   double prefix[kAcceptThreads + 1];
@@ -177,19 +183,11 @@ __device__ double sweep_sample(const Slice<T>& sl, const SweepArgs& a, float u, 
   return total;
 }
 
-__device__ __forceinline__ int argmax_of_row(const ChunkStat* st, const uint64_t* keys, int t_chunks,
-                                             bool want_lse, double* lse) {
-  uint64_t key = 0;
-  warp_finalize_row(st, keys, t_chunks, 1, want_lse, lse, &key);
-  key = __shfl_sync(kFull, key, 0);
-  return key ? key_index(key) : 0;
-}
-
 template <typename T, bool STOCH>
 __global__ void __launch_bounds__(kAcceptThreads, 2)
 accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const double* __restrict__ dlse,
-                   int R, int V, int n, int depth, const ChunkStat* __restrict__ tstats,
-                   const uint64_t* __restrict__ tkeys, int t_chunks, const int32_t* __restrict__ tokens,
+                   int R, int V, int n, int depth, const int32_t* __restrict__ row_amax,
+                   const double* __restrict__ row_lse, const int32_t* __restrict__ tokens,
                    const int32_t* __restrict__ parents, const int32_t* __restrict__ draft_row,
                    const float* __restrict__ uniforms, int32_t* __restrict__ accepted_len,
                    int32_t* __restrict__ path, int32_t* __restrict__ bonus, int slice) {
@@ -201,6 +199,8 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   const bool leader = cluster.block_rank() == 0 && threadIdx.x == 0;
   const int tid = threadIdx.x;
 
+  // ---- prologue: everything the decisions read, in one round of independent loads
+  const size_t trow0 = (size_t)b * (n + 1);
   for (int i = tid; i < n; i += kAcceptThreads) {
     sm.tok[i] = tokens[(size_t)b * n + i];
     sm.par[i] = parents[(size_t)b * n + i];
@@ -208,8 +208,27 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   for (int i = tid; i <= n; i += kAcceptThreads) {
     const int r = draft_row[(size_t)b * (n + 1) + i];
     sm.drow[i] = (r >= 0 && r < R) ? r : -1;  // an out-of-range row counts as "not expanded"
+    sm.amax[i] = row_amax[trow0 + i];
+    if (STOCH) sm.lse_t[i] = row_lse[trow0 + i];
   }
   __syncthreads();
+  if (STOCH) {
+    for (int i = tid; i <= n; i += kAcceptThreads) {
+      const int r = sm.drow[i];
+      sm.lse_d[i] = r >= 0 ? dlse[(size_t)b * R + r] : 0.0;
+      if (i == 0) continue;
+      const int par = sm.par[i - 1], x = sm.tok[i - 1];
+      float tv = -INFINITY, dv = -INFINITY;
+      if (par >= 0 && par <= n && x >= 0 && x < V) {
+        tv = load_logit(tgt + (trow0 + par) * (size_t)V + x);
+        const int pr = draft_row[(size_t)b * (n + 1) + par];
+        if (pr >= 0 && pr < R) dv = load_logit(dft + ((size_t)b * R + pr) * (size_t)V + x);
+      }
+      sm.tl[i] = tv;
+      sm.dl[i] = dv;
+    }
+    __syncthreads();
+  }
 
   Slice<T> sl;
   {
@@ -223,15 +242,12 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     sl.cached_d = -1;
   }
 
-  const size_t trow0 = (size_t)b * (n + 1);
-  auto row_stat = [&](int j) { return tstats + (trow0 + j) * t_chunks; };
-  auto row_keys = [&](int j) { return tkeys + (trow0 + j) * t_chunks; };
   const float* u_acc = STOCH ? uniforms + (size_t)b * 2 * (n + 1) : nullptr;
   const float* u_res = STOCH ? u_acc + (n + 1) : nullptr;
 
   int j = 0, plen = 0;
-  double lse_t = 0.0;
-  int amax = argmax_of_row(row_stat(0), row_keys(0), t_chunks, STOCH, &lse_t);
+  double lse_t = STOCH ? sm.lse_t[0] : 0.0;
+  int amax = sm.amax[0];
   double t = 0.0, F = 1.0;
   bool rejected_here = false;
 
@@ -244,7 +260,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
       const int r = sm.drow[j];
       const T* trow = tgt + (trow0 + j) * (size_t)V;
       const T* drow = r >= 0 ? dft + ((size_t)b * R + r) * (size_t)V : nullptr;
-      const double lse_d = r >= 0 ? dlse[(size_t)b * R + r] : 0.0;
+      const double lse_d = sm.lse_d[j];
       // children of j in node order
       int c = 1;
       while (true) {
@@ -253,8 +269,8 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
         const int x = sm.tok[c - 1];
         double ratio = 0.0;  // a token outside the vocabulary is never accepted
         if (x >= 0 && x < V) {
-          const double px = exp((double)load_logit(trow + x) - lse_t);
-          const double qx = exp((double)load_logit(drow + x) - lse_d);
+          const double px = exp((double)sm.tl[c] - lse_t);
+          const double qx = exp((double)sm.dl[c] - lse_d);
           const double rho = t == 0.0 ? px : fmax(0.0, px - t * qx);
           ratio = rho / (F * qx);
         }
@@ -282,7 +298,8 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     t = 0.0;
     F = 1.0;
     rejected_here = false;
-    amax = argmax_of_row(row_stat(j), row_keys(j), t_chunks, STOCH, &lse_t);
+    amax = sm.amax[j];
+    if (STOCH) lse_t = sm.lse_t[j];
   }
 
   if (leader) {
@@ -299,15 +316,18 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   SweepArgs a;
   a.use_q = use_q;
   a.lse_t.set(lse_t);
-  a.lse_d.set(r >= 0 ? dlse[(size_t)b * R + r] : 0.0);
+  a.lse_d.set(sm.lse_d[j]);
   a.t.set(t);
   const double total = sweep_sample<T>(sl, a, u_res[j], sm, cluster, bonus + b);
   if (!(total > 0.0) && leader) bonus[b] = amax;  // nothing left to sample from
 }
 
 // ------------------------------------------------------------------- host
+// workspace: [row sweep workspace][row argmax rows int32][row lse rows double]
 size_t accept_ws_bytes(int B, int n, int V, int dtype) {
-  return row_stats_ws_bytes((long long)B * (n + 1), V, dtype_bytes(dtype), 1);
+  const long long rows = (long long)B * (n + 1);
+  return row_stats_ws_bytes(rows, V, dtype_bytes(dtype), 1) + align_up((size_t)rows * sizeof(int32_t), 256) +
+         align_up((size_t)rows * sizeof(double), 256);
 }
 
 int accept_max_vocab(int dtype) {
@@ -317,7 +337,7 @@ int accept_max_vocab(int dtype) {
 
 template <typename T, bool STOCH>
 static cudaError_t launch_walk(const void* tgt, const void* dft, const double* dlse, int R, int V, int n,
-                               int depth, const ChunkStat* st, const uint64_t* keys, int t_chunks,
+                               int depth, const int32_t* row_amax, const double* row_lse,
                                const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                                const float* uniforms, int B, int32_t* acc_len, int32_t* path,
                                int32_t* bonus, cudaStream_t s) {
@@ -353,7 +373,7 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, accept_walk_kernel<T, STOCH>, static_cast<const T*>(tgt),
-                            static_cast<const T*>(dft), dlse, R, V, n, depth, st, keys, t_chunks, tokens,
+                            static_cast<const T*>(dft), dlse, R, V, n, depth, row_amax, row_lse, tokens,
                             parents, draft_row, uniforms, acc_len, path, bonus, slice);
 }
 
@@ -363,21 +383,24 @@ cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddty
                           int32_t* path, int32_t* bonus, void* ws, cudaStream_t s) {
   const long long rows = (long long)B * (n + 1);
   const bool stoch = uniforms != nullptr;
-  ChunkStat* st = nullptr;
-  uint64_t* keys = nullptr;
-  row_stats_ws_layout(ws, rows, V, dtype_bytes(tdtype), 1, &st, &keys);
-  cudaError_t e = launch_row_chunk_stats(tgt, tdtype, rows, V, 1, stoch, st, keys, s);
+  char* tail = static_cast<char*>(ws) + row_stats_ws_bytes(rows, V, dtype_bytes(tdtype), 1);
+  int32_t* row_amax = reinterpret_cast<int32_t*>(tail);
+  double* row_lse = reinterpret_cast<double*>(tail + align_up((size_t)rows * sizeof(int32_t), 256));
+  RowOut ro;
+  ro.tok = row_amax;
+  ro.val = nullptr;
+  ro.lse = stoch ? row_lse : nullptr;
+  cudaError_t e = launch_row_stats(tgt, tdtype, rows, V, 1, stoch, ro, ws, s);
   if (e != cudaSuccess) return e;
-  const int t_chunks = plan_chunks(rows, V, dtype_bytes(tdtype)).n_chunks;
   (void)ddtype;  // the draft rows share the target's element type (checked by the caller)
   if (tdtype == EAGLE_F32)
-    return stoch ? launch_walk<float, true>(tgt, dft, dlse, R, V, n, depth, st, keys, t_chunks, tokens, parents,
+    return stoch ? launch_walk<float, true>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens, parents,
                                             draft_row, uniforms, B, accepted_len, path, bonus, s)
-                 : launch_walk<float, false>(tgt, dft, dlse, R, V, n, depth, st, keys, t_chunks, tokens,
+                 : launch_walk<float, false>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
                                              parents, draft_row, uniforms, B, accepted_len, path, bonus, s);
-  return stoch ? launch_walk<__nv_bfloat16, true>(tgt, dft, dlse, R, V, n, depth, st, keys, t_chunks, tokens,
+  return stoch ? launch_walk<__nv_bfloat16, true>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
                                                   parents, draft_row, uniforms, B, accepted_len, path, bonus, s)
-               : launch_walk<__nv_bfloat16, false>(tgt, dft, dlse, R, V, n, depth, st, keys, t_chunks, tokens,
+               : launch_walk<__nv_bfloat16, false>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
                                                    parents, draft_row, uniforms, B, accepted_len, path, bonus, s);
 }
 

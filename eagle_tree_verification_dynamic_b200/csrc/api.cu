@@ -85,14 +85,12 @@ eagle_status eagle_row_stats(const void* logits, int dtype, long long rows, int 
   if (k > EAGLE_MAX_TOPK || k > V) return EAGLE_ERR_LIMIT;
   eagle_status st = check_ws(workspace, workspace_bytes, row_stats_ws_bytes(rows, V, dtype_bytes(dtype), k));
   if (st != EAGLE_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ChunkStat* cs = nullptr;
-  uint64_t* keys = nullptr;
-  row_stats_ws_layout(workspace, rows, V, dtype_bytes(dtype), k, &cs, &keys);
-  st = cuda_status(launch_row_chunk_stats(logits, dtype, rows, V, k, lse != nullptr, cs, keys, s));
-  if (st != EAGLE_OK) return st;
-  const int nc = plan_chunks(rows, V, dtype_bytes(dtype)).n_chunks;
-  return cuda_status(launch_row_stats_finalize(cs, keys, rows, nc, k, topk_token, topk_logit, lse, s));
+  RowOut out;
+  out.tok = topk_token;
+  out.val = topk_logit;
+  out.lse = lse;
+  return cuda_status(launch_row_stats(logits, dtype, rows, V, k, lse != nullptr, out, workspace,
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 // ----------------------------------------------------------------- tree build

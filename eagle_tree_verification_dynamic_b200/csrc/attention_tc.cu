@@ -8,8 +8,10 @@
 // staged in shared memory serves all tree queries of the GQA group at once.
 //   warp 0      TMA producer: K and V tiles of 64 keys into a 2-stage ring
 //               (128-byte swizzle, no multicast); also allocates TMEM
-//   warp 1      one thread issues tcgen05.mma: S = Q K^T into TMEM, then
-//               O += P V into TMEM (fp32 accumulators, bf16 operands)
+//   warp 1      one thread issues tcgen05.mma: S = Q K^T into one of two TMEM
+//               buffers (the next tile's S is computed while this tile's
+//               softmax runs), then O += P V into TMEM (fp32 accumulators,
+//               bf16 operands)
 //   warps 2-5   softmax: thread r owns TMEM lane r = query row r; reads its S
 //               row, applies the prefix range / window / tree bitmask, keeps a
 //               running reference max (re-based only when it grows by > 8 in
@@ -52,16 +54,16 @@ struct TcLayout {
   static constexpr int kStageOff = kPOff + kPBytes;
   static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
   static constexpr int kSmemBytes = kBarOff + 128;  // + barriers (base is 1024-aligned, checked)
-  static constexpr uint32_t kTmemCols = (64 + D) <= 128 ? 128 : 256;
-  static constexpr uint32_t kColS = 0;
-  static constexpr uint32_t kColO = 64;
+  static constexpr uint32_t kTmemCols = 256;  // S double buffer (2 x 64) + O (D)
+  static constexpr uint32_t kColS = 0;        // S buffer b at column 64 * b
+  static constexpr uint32_t kColO = 128;
 };
 
 struct TcBars {
   uint64_t q_full;
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t s_full;
+  uint64_t s_full[2];
   uint64_t p_full;
   uint64_t pv_done;
   uint64_t mma_idle;
@@ -142,7 +144,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       mbar_init(smem_u32(&bars->full[i]), 1);
       mbar_init(smem_u32(&bars->empty[i]), 1);
     }
-    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->s_full[0]), 1);
+    mbar_init(smem_u32(&bars->s_full[1]), 1);
     mbar_init(smem_u32(&bars->p_full), 128);
     mbar_init(smem_u32(&bars->pv_done), 1);
     mbar_init(smem_u32(&bars->mma_idle), 1);
@@ -238,22 +241,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const uint32_t q_addr = s_base + Lay::kQOff;
       const uint32_t p_addr = s_base + Lay::kPOff;
       const bool q_ok = !p.q_by_tma || mbar_wait(smem_u32(&bars->q_full), 0, abort);
-      for (int j = 0; j < ntiles && q_ok; ++j) {
-        const int st = j % kStages;
-        if (!mbar_wait(smem_u32(&bars->full[st]), (j / kStages) & 1, abort)) break;
+      // S = Q K_j^T into S buffer (j & 1)
+      auto issue_qk = [&](int jj) -> bool {
+        const int st = jj % kStages;
+        if (!mbar_wait(smem_u32(&bars->full[st]), (jj / kStages) & 1, abort)) return false;
         tc_fence_after();
         const uint32_t k_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes;
-        const uint32_t v_addr = k_addr + Lay::kKBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * 0 + (kk % 4) * 32;
+          const uint32_t off = (kk % 4) * 32;
           const uint64_t da = smem_desc(q_addr + (kk / 4) * 16384 + off, 16, 1024, kSwizzle128B);
           const uint64_t db = smem_desc(k_addr + (kk / 4) * Lay::kKVAtomBytes + off, 16, 1024, kSwizzle128B);
-          mma_bf16_ss(t_s, da, db, id_qk, kk > 0);
+          mma_bf16_ss(t_s + (uint32_t)((jj & 1) * kBN), da, db, id_qk, kk > 0);
         }
-        mma_commit(smem_u32(&bars->s_full));
-        if (!mbar_wait(smem_u32(&bars->p_full), j & 1, abort)) break;
+        mma_commit(smem_u32(&bars->s_full[jj & 1]));
+        return true;
+      };
+      bool ok = q_ok && issue_qk(0);
+      int next_qk = 1;  // S has two buffers: QK^T runs at most one tile ahead of PV
+      for (int j = 0; j < ntiles && ok; ++j) {
+        // issue whichever is ready first: the next tile's QK^T (its K landed) or
+        // this tile's PV (its P is written)
+        const uint32_t pb = smem_u32(&bars->p_full);
+        uint64_t t0 = 0;
+        for (uint32_t it = 0;; ++it) {
+          if (next_qk < ntiles && next_qk <= j + 1 &&
+              mbar_try_wait(smem_u32(&bars->full[next_qk % kStages]), (next_qk / kStages) & 1)) {
+            if (!issue_qk(next_qk)) { ok = false; break; }
+            ++next_qk;
+          }
+          if (mbar_try_wait(pb, j & 1)) break;
+          if ((it & 15u) == 15u) {
+            if (*abort) { ok = false; break; }
+            const uint64_t now = globaltimer();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > 2000000000ull) { *abort = 1; ok = false; break; }
+          }
+        }
+        if (!ok) break;
         tc_fence_after();
+        const int st = j % kStages;
+        const uint32_t v_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes + Lay::kKBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint64_t da = smem_desc(p_addr + kk * 32, 16, 1024, kSwizzle128B);
@@ -272,6 +300,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t t_s = tmem + lane_base + Lay::kColS;
     const uint32_t t_o = tmem + lane_base + Lay::kColO;
+    // a warp whose 32 rows are all padding only keeps the barrier protocol going
+    const bool warp_live = row0 + quad * 32 < rows;
     const int qpos = (row_ok && p.window > 0) ? p.pos[(size_t)b * p.n + qi] : 0;
     const int win_lo = qpos - p.window + 1;
     uint64_t mw0 = 0, mw1 = 0;
@@ -279,31 +309,42 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       mw0 = p.mask[((size_t)b * p.n + qi) * 2];
       mw1 = p.mask[((size_t)b * p.n + qi) * 2 + 1];
     }
-    float m_used = -INFINITY, l = 0.f;
+    const float sl2 = p.scale_log2;
+    float m_used = -INFINITY, l = 0.f;  // running reference max (scaled, log2 units) and row sum
     bool ok = true;
     unsigned char* prow = smem + Lay::kPOff + r_local * 128;
     for (int j = 0; j < ntiles && ok; ++j) {
-      if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full), j & 1, abort))) { ok = false; break; }
+      if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, abort))) { ok = false; break; }
+      if (!warp_live) {
+        mbar_arrive(smem_u32(&bars->p_full));
+        continue;
+      }
       tc_fence_after();
       float x[kBN];
-      tmem_ld32(t_s, x);
-      tmem_ld32(t_s + 32, x + 32);
+      tmem_ld32(t_s + (uint32_t)((j & 1) * kBN), x);
+      tmem_ld32(t_s + (uint32_t)((j & 1) * kBN + 32), x + 32);
       tmem_wait_ld();
       const int key0 = k0 + j * kBN;
       float mx = -INFINITY;
+      if (tree || p.window > 0 || key0 + kBN > k1) {  // edge tiles: per-key visibility
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        const int kidx = key0 + c;
-        bool vis = row_ok && kidx < k1;
-        if (vis && tree) {
-          vis = ((kidx < 64 ? mw0 >> kidx : mw1 >> (kidx - 64)) & 1ull) != 0;
-          if (vis && p.window > 0) vis = p.pos[(size_t)b * p.n + kidx] >= win_lo;
-        } else if (vis && p.window > 0) {
-          vis = kidx >= win_lo;
+        for (int c = 0; c < kBN; ++c) {
+          const int kidx = key0 + c;
+          bool vis = row_ok && kidx < k1;
+          if (vis && tree) {
+            vis = ((kidx < 64 ? mw0 >> kidx : mw1 >> (kidx - 64)) & 1ull) != 0;
+            if (vis && p.window > 0) vis = p.pos[(size_t)b * p.n + kidx] >= win_lo;
+          } else if (vis && p.window > 0) {
+            vis = kidx >= win_lo;
+          }
+          x[c] = vis ? x[c] : -INFINITY;
+          mx = fmaxf(mx, x[c]);
         }
-        x[c] = vis ? x[c] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
+      } else {  // interior prefix tile: every key visible
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, x[c]);
       }
+      mx *= sl2;  // scale > 0 keeps the order
       // PV(j-1) must be complete before P is overwritten or O is rescaled
       if (j > 0) {
         if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (j - 1) & 1, abort))) { ok = false; break; }
@@ -324,16 +365,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         l *= f;
       }
       if (rebase) m_used = mx;
+      const float neg_m = m_used > -INFINITY ? -m_used : 0.f;  // no visible key yet: every x is -inf
       float sum = 0.f;
 #pragma unroll
       for (int c8 = 0; c8 < kBN / 8; ++c8) {
         uint32_t packed[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const float a = x[c8 * 8 + 2 * t] > -INFINITY ? ex2(x[c8 * 8 + 2 * t] - m_used) : 0.f;
-          const float bb = x[c8 * 8 + 2 * t + 1] > -INFINITY ? ex2(x[c8 * 8 + 2 * t + 1] - m_used) : 0.f;
+          const float a = ex2(fmaf(x[c8 * 8 + 2 * t], sl2, neg_m));
+          const float bb = ex2(fmaf(x[c8 * 8 + 2 * t + 1], sl2, neg_m));
+          sum += a + bb;
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
-          sum += __low2float(h2) + __high2float(h2);
           packed[t] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         *reinterpret_cast<uint4*>(prow + ((c8 ^ (r_local & 7)) << 4)) =
@@ -345,7 +387,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       mbar_arrive(smem_u32(&bars->p_full));
     }
     // epilogue: normalised partial output and its log-sum-exp
-    if (ok && __all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (ntiles - 1) & 1, abort))) {
+    if (ok && warp_live && __all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (ntiles - 1) & 1, abort))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const size_t slot = (((size_t)s * B + b) * p.n + qi) * p.Hq + qh;

@@ -146,31 +146,6 @@ __device__ __forceinline__ float exp_minus(float x, Split2 lse) {
   return exp2f(fmaf(d, kLog2eHi, d * kLog2eLo));
 }
 
-// One warp per row: merge the chunks of a row into (lse, top-k keys).
-__device__ __forceinline__ void warp_finalize_row(const ChunkStat* st, const uint64_t* keys, int n_chunks, int k,
-                                  bool want_lse, double* lse_out, uint64_t* key_out) {
-  const int lane = threadIdx.x & 31;
-  if (want_lse) {
-    LseAccum a;
-    a.init();
-    for (int c = lane; c < n_chunks; c += 32) a.add(st[c].e_ref, st[c].acc);
-    const float e = warp_max_f(a.e);
-    double s = a.s > 0.0 ? rescale_pow2(a.s, a.e, e) : 0.0;
-    s = warp_sum_d(s);
-    *lse_out = s > 0.0 ? kLn2 * ((double)e + log2(s)) : -INFINITY;
-  }
-  uint64_t list = 0ull;
-  for (int c0 = 0; c0 < n_chunks; c0 += 8) {  // 8 chunk lists in flight, then merged
-    uint64_t kv[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) kv[t] = (lane < k && c0 + t < n_chunks) ? keys[(c0 + t) * k + lane] : 0ull;
-#pragma unroll
-    for (int t = 0; t < 8; ++t)
-      if (c0 + t < n_chunks) list = warp_merge_desc(list, kv[t]);
-  }
-  *key_out = list;
-}
-
 // ------------------------------------------------------------------ loading
 template <typename T> struct Elem;
 template <> struct Elem<float> {

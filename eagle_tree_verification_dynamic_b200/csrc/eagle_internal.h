@@ -24,15 +24,16 @@ struct ChunkPlan {
   int chunk_elems;
   int n_chunks;
 };
+// Final per-row outputs of the vocabulary sweep (any pointer may be null).
+struct RowOut {
+  int32_t* tok;  // [rows][k] top-k token ids, descending logit (-1 if the row has fewer)
+  float* val;    // [rows][k] their logits
+  double* lse;   // [rows] log-sum-exp
+};
 ChunkPlan plan_chunks(long long rows, int V, int elem_bytes);
 size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k);
-void row_stats_ws_layout(void* ws, long long rows, int V, int elem_bytes, int k, ChunkStat** stats,
-                         uint64_t** keys);
-cudaError_t launch_row_chunk_stats(const void* x, int dtype, long long rows, int V, int k, bool lse,
-                                   ChunkStat* stats, uint64_t* keys, cudaStream_t s);
-cudaError_t launch_row_stats_finalize(const ChunkStat* stats, const uint64_t* keys, long long rows,
-                                      int n_chunks, int k, int32_t* topk_token, float* topk_logit,
-                                      double* lse, cudaStream_t s);
+cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, int k, bool lse, const RowOut& out,
+                             void* ws, cudaStream_t s);
 
 // ---- tree build (tree_build.cu)
 size_t tree_build_smem_bytes(int R, int k, int P);

@@ -1,16 +1,19 @@
-// Vocabulary sweep over logit rows: per chunk of a row, the top-k tokens by raw
-// logit (ties to the lower token id) and a base-2 scaled partial of
-// sum exp(logit).  The top-k of the draft rows gives the candidate children of
-// a tree node and the log-sum-exp turns logits into draft confidences
-// c(x) = exp(l_x) / sum_i exp(l_i) ("EAGLE" notes, EAGLE-2 "Well-Calibrated
-// Draft Model"); on target rows the same sweep (k = 1) gives the argmax for
-// greedy acceptance and the normaliser of p_target for sampling.
+// Vocabulary sweep over logit rows: the top-k tokens of each row by raw logit
+// (ties to the lower token id) and the row's log-sum-exp.  The top-k of the
+// draft rows gives the candidate children of a tree node and the log-sum-exp
+// turns logits into draft confidences c(x) = exp(l_x) / sum_i exp(l_i)
+// ("EAGLE" notes, EAGLE-2 "Well-Calibrated Draft Model"); on target rows the
+// same sweep (k = 1) gives the argmax for greedy acceptance and the normaliser
+// of p_target for sampling.
 //
 // One CTA owns one (row, chunk).  Threads stream 16-byte vectors (coalesced,
-// L1 no-allocate) and keep, per lane, the two best (value, id) pairs plus a
-// running partial sum; a warp then builds its exact top-k from the lanes'
-// best keys with a bitonic sort, pulling a lane's further elements only when
-// that lane already contributed twice.  Warps merge in shared memory.
+// L1 no-allocate) and keep, per lane, the M best (value, id) pairs in
+// registers plus a base-2 scaled fp64 partial of sum exp(logit).  A warp
+// builds its exact top-k from the lanes' lists with bitonic sort/merge rounds
+// (a lane is rescanned from memory only if all M of its entries made the
+// cut); warps merge pairwise through shared memory.  The CTA that finishes a
+// row's last chunk (an atomic ticket; nobody waits) merges the row's chunks
+// and writes the final per-row outputs.
 #include "eagle_internal.h"
 
 namespace eagle {
@@ -19,18 +22,28 @@ constexpr int kStatThreads = 256;
 constexpr int kStatWarps = kStatThreads / 32;
 constexpr int kUnroll = 8;
 
-struct LaneTop2 {
-  float s1, s2;
-  int i1, i2;
-  __device__ __forceinline__ void init() { s1 = s2 = -INFINITY; i1 = i2 = -1; }
-  // Elements arrive in increasing id; a later equal value never displaces an
-  // earlier one, so among equals the lower id stays ahead.
+// The M largest (value, id) pairs seen by a lane, sorted descending.  Elements
+// arrive in increasing id and only a strictly larger value moves ahead, so
+// among equal values the lower id stays first.
+template <int M>
+struct LaneTop {
+  float s[M];
+  int id[M];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int p = 0; p < M; ++p) { s[p] = -INFINITY; id[p] = -1; }
+  }
   __device__ __forceinline__ void push(float v, int idx) {
-    if (v > s2) {
-      if (v > s1) { s2 = s1; i2 = i1; s1 = v; i1 = idx; }
-      else        { s2 = v; i2 = idx; }
+    if (!(v > s[M - 1])) return;
+#pragma unroll
+    for (int p = 0; p < M; ++p) {
+      if (v > s[p]) {
+        const float tv = s[p]; s[p] = v; v = tv;
+        const int ti = id[p]; id[p] = idx; idx = ti;
+      }
     }
   }
+  __device__ __forceinline__ uint64_t key(int p) const { return id[p] >= 0 ? make_key(s[p], id[p]) : 0ull; }
 };
 
 // Largest key strictly below `last` among this lane's elements of the chunk
@@ -63,10 +76,10 @@ __device__ uint64_t lane_next_below(const T* __restrict__ rp, int c0, int c1, ui
   return best;
 }
 
-template <typename T, bool LSE, bool VEC>
+template <typename T, bool LSE, bool VEC, int M>
 __global__ void __launch_bounds__(kStatThreads)
-row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
-                       ChunkStat* __restrict__ stats, uint64_t* __restrict__ keys) {
+row_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k, ChunkStat* __restrict__ stats,
+                 uint64_t* __restrict__ keys, int* __restrict__ tickets, RowOut out) {
   const long long row = blockIdx.x;
   const int chunk = blockIdx.y, n_chunks = gridDim.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -74,7 +87,7 @@ row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
   const int c0 = chunk * chunk_elems;
   const int c1 = min(V, c0 + chunk_elems);
 
-  LaneTop2 top;
+  LaneTop<M> top;
   top.init();
   float e_ref = -INFINITY;
   double acc = 0.0;
@@ -84,7 +97,7 @@ row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
 #pragma unroll
     for (int i = 1; i < Elem<T>::kPerVec; ++i)
       if (i < n) vmax = fmaxf(vmax, f[i]);
-    if (vmax > top.s2) {
+    if (vmax > top.s[M - 1]) {
 #pragma unroll
       for (int i = 0; i < Elem<T>::kPerVec; ++i)
         if (i < n) top.push(f[i], idx0 + i);
@@ -137,22 +150,33 @@ row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
   __shared__ uint64_t s_keys[kStatWarps][32];
   __shared__ float s_e[kStatWarps];
   __shared__ double s_s[kStatWarps];
+  __shared__ int s_last;
 
-  // ---- warp top-k
-  const uint64_t k1 = top.i1 >= 0 ? make_key(top.s1, top.i1) : 0ull;
+  // ---- warp top-k: lane bests first, then the next entries of the lanes whose
+  // previous entry made the cut
   uint64_t list;
   if (k == 1) {
-    list = warp_max_u64(k1);
+    list = warp_max_u64(top.key(0));
   } else {
-    list = warp_sort_desc(k1);
+    list = warp_sort_desc(top.key(0));
     uint64_t thr = __shfl_sync(kFull, list, k - 1);
-    uint64_t last = top.i2 >= 0 ? make_key(top.s2, top.i2) : 0ull;
-    bool need = last != 0 && last >= thr;
-    while (__any_sync(kFull, need)) {
-      list = warp_merge_desc(list, warp_sort_desc(need ? last : 0ull));
+    bool need = top.key(0) != 0 && top.key(0) >= thr;
+    int r = 1;
+    for (; r < M; ++r) {
+      const uint64_t cand = need ? top.key(r) : 0ull;
+      if (!__any_sync(kFull, cand != 0)) { need = false; break; }
+      list = warp_merge_desc(list, warp_sort_desc(cand));
       thr = __shfl_sync(kFull, list, k - 1);
+      need = cand != 0 && cand >= thr;
+    }
+    // all M entries of some lane made the cut: pull its further elements (rare)
+    uint64_t last = (r == M && need) ? top.key(M - 1) : 0ull;
+    need = last != 0;
+    while (__any_sync(kFull, need)) {
       uint64_t nxt = 0;
-      if (need && last >= thr) nxt = lane_next_below<T, VEC>(rp, c0, c1, last);
+      if (need) nxt = lane_next_below<T, VEC>(rp, c0, c1, last);
+      list = warp_merge_desc(list, warp_sort_desc(nxt));
+      thr = __shfl_sync(kFull, list, k - 1);
       need = nxt != 0 && nxt >= thr;
       last = nxt;
     }
@@ -162,9 +186,9 @@ row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
   // ---- warp partial sums
   if (LSE) {
     const float e = warp_max_f(e_ref);
-    double s = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
-    s = warp_sum_d(s);
-    if (lane == 0) { s_e[warp] = e; s_s[warp] = s; }
+    double sacc = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
+    sacc = warp_sum_d(sacc);
+    if (lane == 0) { s_e[warp] = e; s_s[warp] = sacc; }
   }
   __syncthreads();
 
@@ -177,10 +201,10 @@ row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
     }
     __syncthreads();
   }
+
+  const size_t slot = (size_t)row * n_chunks + chunk;
   if (warp == 0) {
-    const uint64_t merged = lane < k ? s_keys[0][lane] : 0ull;
-    const size_t slot = (size_t)row * n_chunks + chunk;
-    if (lane < k) keys[slot * k + lane] = merged;
+    if (lane < k) keys[slot * k + lane] = s_keys[0][lane];
     if (LSE && lane == 0) {
       LseAccum a;
       a.init();
@@ -192,24 +216,45 @@ row_chunk_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k,
       stats[slot] = cs;
     }
   }
-}
 
-__global__ void row_stats_finalize_kernel(const ChunkStat* __restrict__ stats,
-                                          const uint64_t* __restrict__ keys, long long rows,
-                                          int n_chunks, int k, int32_t* __restrict__ topk_token,
-                                          float* __restrict__ topk_logit, double* __restrict__ lse) {
-  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const int lane = threadIdx.x & 31;
-  double l = 0.0;
-  uint64_t key = 0;
-  warp_finalize_row(stats + row * n_chunks, keys + row * n_chunks * k, n_chunks, k, lse != nullptr,
-                    &l, &key);
-  if (lane < k) {
-    if (topk_token) topk_token[row * k + lane] = key ? key_index(key) : -1;
-    if (topk_logit) topk_logit[row * k + lane] = key ? key_value(key) : -INFINITY;
+  // ---- the CTA that completes the row merges all of its chunks
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(tickets + row, 1) == n_chunks - 1;
+  __syncthreads();
+  if (!s_last || warp != 0) return;
+  __threadfence();
+  const ChunkStat* st = stats + (size_t)row * n_chunks;
+  const uint64_t* kk = keys + (size_t)row * n_chunks * k;
+  double lse = 0.0;
+  if (LSE) {
+    LseAccum a;
+    a.init();
+    for (int c = lane; c < n_chunks; c += 32) {
+      const float e2 = __ldcg(&st[c].e_ref);
+      const double s2 = __ldcg(&st[c].acc);
+      a.add(e2, s2);
+    }
+    const float e = warp_max_f(a.e);
+    double s = a.s > 0.0 ? rescale_pow2(a.s, a.e, e) : 0.0;
+    s = warp_sum_d(s);
+    lse = s > 0.0 ? kLn2 * ((double)e + log2(s)) : -INFINITY;
   }
-  if (lse && lane == 0) lse[row] = l;
+  uint64_t merged = 0ull;
+  for (int c = 0; c < n_chunks; c += 8) {  // 8 chunk lists in flight, then merged
+    uint64_t kv[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      kv[t] = (lane < k && c + t < n_chunks) ? __ldcg(reinterpret_cast<const unsigned long long*>(kk) + (c + t) * k + lane) : 0ull;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (c + t < n_chunks) merged = warp_merge_desc(merged, kv[t]);
+  }
+  if (lane < k) {
+    if (out.tok) out.tok[row * k + lane] = merged ? key_index(merged) : -1;
+    if (out.val) out.val[row * k + lane] = merged ? key_value(merged) : -INFINITY;
+  }
+  if (LSE && out.lse && lane == 0) out.lse[row] = lse;
 }
 
 // ------------------------------------------------------------------- host
@@ -228,52 +273,52 @@ ChunkPlan plan_chunks(long long rows, int V, int elem_bytes) {
   return p;
 }
 
+// workspace: [chunk stats rows*nc][chunk keys rows*nc*k][row tickets rows]
 size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k) {
   const ChunkPlan p = plan_chunks(rows, V, elem_bytes);
   const size_t n = (size_t)rows * p.n_chunks;
-  return align_up(n * sizeof(ChunkStat), 256) + align_up(n * k * sizeof(uint64_t), 256);
+  return align_up(n * sizeof(ChunkStat), 256) + align_up(n * k * sizeof(uint64_t), 256) +
+         align_up((size_t)rows * sizeof(int), 256);
 }
 
-void row_stats_ws_layout(void* ws, long long rows, int V, int elem_bytes, int k, ChunkStat** stats,
-                         uint64_t** keys) {
-  const ChunkPlan p = plan_chunks(rows, V, elem_bytes);
-  const size_t n = (size_t)rows * p.n_chunks;
-  char* base = static_cast<char*>(ws);
-  *stats = reinterpret_cast<ChunkStat*>(base);
-  *keys = reinterpret_cast<uint64_t*>(base + align_up(n * sizeof(ChunkStat), 256));
-}
-
-template <typename T, bool LSE>
-static cudaError_t launch_typed(const void* x, long long rows, int V, int k, const ChunkPlan& p,
-                                bool vec, ChunkStat* stats, uint64_t* keys, cudaStream_t s) {
+template <typename T, bool LSE, int M>
+static void launch_typed(const void* x, long long rows, int V, int k, const ChunkPlan& p, bool vec,
+                         ChunkStat* stats, uint64_t* keys, int* tickets, const RowOut& out, cudaStream_t s) {
   dim3 grid((unsigned)rows, (unsigned)p.n_chunks);
   const T* xp = static_cast<const T*>(x);
   if (vec)
-    row_chunk_stats_kernel<T, LSE, true><<<grid, kStatThreads, 0, s>>>(xp, V, p.chunk_elems, k, stats, keys);
+    row_stats_kernel<T, LSE, true, M><<<grid, kStatThreads, 0, s>>>(xp, V, p.chunk_elems, k, stats, keys, tickets, out);
   else
-    row_chunk_stats_kernel<T, LSE, false><<<grid, kStatThreads, 0, s>>>(xp, V, p.chunk_elems, k, stats, keys);
-  return cudaGetLastError();
+    row_stats_kernel<T, LSE, false, M><<<grid, kStatThreads, 0, s>>>(xp, V, p.chunk_elems, k, stats, keys, tickets, out);
 }
 
-cudaError_t launch_row_chunk_stats(const void* x, int dtype, long long rows, int V, int k, bool lse,
-                                   ChunkStat* stats, uint64_t* keys, cudaStream_t s) {
+template <typename T>
+static void launch_t(const void* x, long long rows, int V, int k, bool lse, const ChunkPlan& p, bool vec,
+                     ChunkStat* stats, uint64_t* keys, int* tickets, const RowOut& out, cudaStream_t s) {
+  if (k == 1) {
+    if (lse) launch_typed<T, true, 1>(x, rows, V, k, p, vec, stats, keys, tickets, out, s);
+    else     launch_typed<T, false, 1>(x, rows, V, k, p, vec, stats, keys, tickets, out, s);
+  } else {
+    if (lse) launch_typed<T, true, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s);
+    else     launch_typed<T, false, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s);
+  }
+}
+
+cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, int k, bool lse, const RowOut& out,
+                             void* ws, cudaStream_t s) {
   const int eb = dtype_bytes(dtype);
   const ChunkPlan p = plan_chunks(rows, V, eb);
+  const size_t n = (size_t)rows * p.n_chunks;
+  char* base = static_cast<char*>(ws);
+  ChunkStat* stats = reinterpret_cast<ChunkStat*>(base);
+  uint64_t* keys = reinterpret_cast<uint64_t*>(base + align_up(n * sizeof(ChunkStat), 256));
+  int* tickets = reinterpret_cast<int*>(base + align_up(n * sizeof(ChunkStat), 256) +
+                                        align_up(n * k * sizeof(uint64_t), 256));
+  cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)rows * sizeof(int), s);
+  if (e != cudaSuccess) return e;
   const bool vec = ((uintptr_t)x % 16 == 0) && (((size_t)V * eb) % 16 == 0);
-  if (dtype == EAGLE_F32)
-    return lse ? launch_typed<float, true>(x, rows, V, k, p, vec, stats, keys, s)
-               : launch_typed<float, false>(x, rows, V, k, p, vec, stats, keys, s);
-  return lse ? launch_typed<__nv_bfloat16, true>(x, rows, V, k, p, vec, stats, keys, s)
-             : launch_typed<__nv_bfloat16, false>(x, rows, V, k, p, vec, stats, keys, s);
-}
-
-cudaError_t launch_row_stats_finalize(const ChunkStat* stats, const uint64_t* keys, long long rows,
-                                      int n_chunks, int k, int32_t* topk_token, float* topk_logit,
-                                      double* lse, cudaStream_t s) {
-  const int warps = 8;
-  const long long blocks = (rows + warps - 1) / warps;
-  row_stats_finalize_kernel<<<(unsigned)blocks, warps * 32, 0, s>>>(stats, keys, rows, n_chunks, k,
-                                                                    topk_token, topk_logit, lse);
+  if (dtype == EAGLE_F32) launch_t<float>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s);
+  else launch_t<__nv_bfloat16>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s);
   return cudaGetLastError();
 }
 

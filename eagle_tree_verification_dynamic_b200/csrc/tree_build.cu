@@ -1,7 +1,7 @@
 // EAGLE-2 dynamic draft tree ("EAGLE" notes, EAGLE-2 sections "Expansion of
 // tree" and "Reranking Nodes").  One CTA per sequence:
-//   0. (before it, in parallel over all rows) the vocabulary sweep and a
-//      one-warp-per-row merge give each draft row's log-sum-exp and top-k;
+//   0. (before it, in parallel over all rows) the vocabulary sweep gives each
+//      draft row's log-sum-exp and top-k;
 //   1. lp = logit - lse turns the top-k logits into log-confidences;
 //   2. level 1 = the root's k children; for each level up to depth-1, rank the
 //      level's candidates by (log V desc, candidate id asc) (each candidate
@@ -227,22 +227,18 @@ cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R,
                               const eagle_tree_t& out, void* ws, cudaStream_t s) {
   const long long rows = (long long)B * R;
   const int eb = dtype_bytes(dtype);
-  ChunkStat* cs = nullptr;
-  uint64_t* keys = nullptr;
-  row_stats_ws_layout(ws, rows, V, eb, k, &cs, &keys);
   char* tail = static_cast<char*>(ws) + row_stats_ws_bytes(rows, V, eb, k);
-  int32_t* row_tok = reinterpret_cast<int32_t*>(tail);
-  float* row_val = reinterpret_cast<float*>(tail + align_up((size_t)rows * k * sizeof(int32_t), 256));
-  cudaError_t e = launch_row_chunk_stats(draft_logits, dtype, rows, V, k, true, cs, keys, s);
-  if (e != cudaSuccess) return e;
-  const int nc = plan_chunks(rows, V, eb).n_chunks;
-  e = launch_row_stats_finalize(cs, keys, rows, nc, k, row_tok, row_val, out.row_lse, s);
+  RowOut ro;
+  ro.tok = reinterpret_cast<int32_t*>(tail);
+  ro.val = reinterpret_cast<float*>(tail + align_up((size_t)rows * k * sizeof(int32_t), 256));
+  ro.lse = out.row_lse;
+  cudaError_t e = launch_row_stats(draft_logits, dtype, rows, V, k, true, ro, ws, s);
   if (e != cudaSuccess) return e;
   const int P = k + (depth - 1) * k * k;
   const size_t smem = tree_build_smem_bytes(R, k, P);
   e = ensure_smem_limit((const void*)tree_expand_kernel, smem);
   if (e != cudaSuccess) return e;
-  tree_expand_kernel<<<B, kBuildThreads, smem, s>>>(row_tok, row_val, R, depth, k, n, out);
+  tree_expand_kernel<<<B, kBuildThreads, smem, s>>>(ro.tok, ro.val, R, depth, k, n, out);
   return cudaGetLastError();
 }
 
