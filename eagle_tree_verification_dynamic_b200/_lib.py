@@ -49,6 +49,8 @@ _SIGS = {
     "eagle_tree_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i]),
     "eagle_tree_attention": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i,
                                     _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p, _c_sz, _c_p]),
+    "eagle_tree_build_noalloc": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
+                                        ctypes.POINTER(TreeStruct), ctypes.POINTER(_c_i), _c_p]),
     "eagle_accept_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
     "eagle_accept": (_c_i, [_c_p, _c_i, _c_p, _c_i, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i,
                             _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),

@@ -215,6 +215,22 @@ EAGLE_API eagle_status eagle_accept(const void* target_logits, int target_dtype,
                           int B, int n, int V, int depth, int32_t* accepted_len, int32_t* path,
                           int32_t* bonus, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ----------------------------------------------------- tree build, no workspace
+ * Not a step of the method (the pages have no counterpart): the same build as
+ * eagle_tree_build for callers that cannot allocate device memory when they
+ * build a tree -- for example a serving loop whose memory pool is sealed after
+ * warm-up, or a plugin interface that hands over only buffers and a stream.
+ * Scratch comes from a fixed 2 MiB array inside the library (held on every GPU
+ * that loads the library until the process exits); nothing is allocated.
+ * Shapes whose eagle_tree_build_workspace_bytes exceeds 2 MiB return
+ * EAGLE_ERR_LIMIT and launch nothing.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and must come before any
+ * stream capture on that device.  All calls share the array: calls whose work
+ * overlaps on the GPU race and must be serialised by the caller. */
+EAGLE_API eagle_status eagle_tree_build_noalloc(const void* draft_logits, int dtype, int B, int R, int V,
+                                                int depth, int k, int m, const eagle_tree_t* out, int* n_nodes,
+                                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif
