@@ -57,9 +57,16 @@ struct AcceptSmem {
   float tl[EAGLE_MAX_NODES + 1];       // child c: target logit of its token in its parent's row
   float dl[EAGLE_MAX_NODES + 1];       // child c: draft logit of its token in its parent's draft row
   double warp_part[kAcceptWarps];
+  double red[2][kAcceptWarps];   // block-reduction slots, alternating by call
   double lane_sum[kAcceptThreads];
   double prefix[kAcceptThreads + 1];
-  double cta_total;
+  double cta_total[2];           // cluster-reduction slots, alternating by call
+};
+
+// Every thread performs the same sequence of reductions, so each keeps its own
+// copy of the slot parities.
+struct Parity {
+  int red = 0, cl = 0;
 };
 
 // This thread's slice [x0, x1) of the current rows, cached in shared memory.
@@ -94,39 +101,46 @@ struct Slice {
   }
 };
 
-// Deterministic block sum; result valid in every thread.
-__device__ double block_sum(double v, AcceptSmem& sm) {
+// Deterministic block sum; result valid in every thread.  One barrier: the
+// per-warp slots alternate between calls, so a slot is rewritten only after
+// every thread has passed the barrier that follows its last read.
+__device__ double block_sum(double v, AcceptSmem& sm, int& parity) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   v = warp_sum_d(v);
-  __syncthreads();
-  if (lane == 0) sm.warp_part[warp] = v;
+  if (lane == 0) sm.red[parity][warp] = v;
   __syncthreads();
   double s = 0.0;
-  for (int w = 0; w < kAcceptWarps; ++w) s += sm.warp_part[w];
+#pragma unroll
+  for (int w = 0; w < kAcceptWarps; ++w) s += sm.red[parity][w];
+  parity ^= 1;
   return s;
 }
 
-// Cluster-wide total of one double per CTA, summed in rank order.
+// Cluster-wide total of one double per CTA, summed in rank order (bit-identical
+// in every CTA).  One cluster barrier per call: the slots alternate between
+// calls; a CTA rewrites a slot only after the next call's barrier, which every
+// CTA reaches only after reading that slot.
 __device__ double cluster_sum(double cta_value, AcceptSmem& sm, cg::cluster_group& cluster,
-                              double* prefix_of_rank) {
-  if (threadIdx.x == 0) sm.cta_total = cta_value;
+                              double* prefix_of_rank, int& parity) {
+  if (threadIdx.x == 0) sm.cta_total[parity] = cta_value;
   cluster.sync();
   const unsigned nb = cluster.num_blocks();
   const unsigned me = cluster.block_rank();
   double acc = 0.0;
   for (unsigned r = 0; r < nb; ++r) {
     if (r == me && prefix_of_rank) *prefix_of_rank = acc;
-    acc += *cluster.map_shared_rank(&sm.cta_total, r);
+    acc += *cluster.map_shared_rank(&sm.cta_total[parity], r);
   }
-  cluster.sync();
+  parity ^= 1;
   return acc;
 }
 
 template <typename T>
-__device__ double sweep_total(const Slice<T>& sl, const SweepArgs& a, AcceptSmem& sm, cg::cluster_group& cluster) {
+__device__ double sweep_total(const Slice<T>& sl, const SweepArgs& a, AcceptSmem& sm, cg::cluster_group& cluster,
+                              Parity& par) {
   double acc = 0.0;
   for (int i = 0; i < sl.x1 - sl.x0; ++i) acc += (double)sl.weight(a, i);
-  return cluster_sum(block_sum(acc, sm), sm, cluster, nullptr);
+  return cluster_sum(block_sum(acc, sm, par.red), sm, cluster, nullptr, par.cl);
 }
 
 // Inverse CDF over the weights: smallest x with cumsum_x > u * total.  Writes
@@ -135,7 +149,7 @@ __device__ double sweep_total(const Slice<T>& sl, const SweepArgs& a, AcceptSmem
 // fp64, element by element; the owner's rescan repeats exactly those additions.
 template <typename T>
 __device__ double sweep_sample(const Slice<T>& sl, const SweepArgs& a, float u, AcceptSmem& sm,
-                               cg::cluster_group& cluster, int32_t* out) {
+                               cg::cluster_group& cluster, int32_t* out, Parity& par) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int len = sl.x1 - sl.x0;
   double mine = 0.0;
@@ -163,7 +177,7 @@ __device__ double sweep_sample(const Slice<T>& sl, const SweepArgs& a, float u, 
   __syncthreads();
   double my_off = 0.0;
   const double cta_total = sm.prefix[kAcceptThreads];
-  const double total = cluster_sum(cta_total, sm, cluster, &my_off);
+  const double total = cluster_sum(cta_total, sm, cluster, &my_off, par.cl);
   if (total > 0.0) {
     const double thr = (double)u * total;
     const double start = my_off + sm.prefix[tid];
@@ -201,6 +215,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
 
   // ---- prologue: everything the decisions read, in one round of independent loads
   const size_t trow0 = (size_t)b * (n + 1);
+  Parity par;
   for (int i = tid; i < n; i += kAcceptThreads) {
     sm.tok[i] = tokens[(size_t)b * n + i];
     sm.par[i] = parents[(size_t)b * n + i];
@@ -285,7 +300,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
           SweepArgs a;
           a.use_q = true;
           a.lse_t.set(lse_t); a.lse_d.set(lse_d); a.t.set(t);
-          F = sweep_total<T>(sl, a, sm, cluster);
+          F = sweep_total<T>(sl, a, sm, cluster, par);
           if (!(F > 0.0)) break;  // p == q left nothing: keep the walk here
         }
         c = nc;
@@ -318,8 +333,9 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   a.lse_t.set(lse_t);
   a.lse_d.set(sm.lse_d[j]);
   a.t.set(t);
-  const double total = sweep_sample<T>(sl, a, u_res[j], sm, cluster, bonus + b);
+  const double total = sweep_sample<T>(sl, a, u_res[j], sm, cluster, bonus + b, par);
   if (!(total > 0.0) && leader) bonus[b] = amax;  // nothing left to sample from
+  cluster.sync();  // no CTA leaves while another may still read its shared memory
 }
 
 // ------------------------------------------------------------------- host

@@ -146,7 +146,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
     mbar_init(smem_u32(&bars->s_full[0]), 1);
     mbar_init(smem_u32(&bars->s_full[1]), 1);
-    mbar_init(smem_u32(&bars->p_full), 128);
+    // only warps holding at least one real query row write P and arrive; a warp
+    // of padding rows never arrives (it could otherwise run a tile ahead and
+    // complete a phase early, since S is double-buffered)
+    const int live_warps = min(4, (rows - row0 + 31) / 32);
+    mbar_init(smem_u32(&bars->p_full), 32 * live_warps);
     mbar_init(smem_u32(&bars->pv_done), 1);
     mbar_init(smem_u32(&bars->mma_idle), 1);
     bars->abort = 0;
@@ -314,11 +318,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     bool ok = true;
     unsigned char* prow = smem + Lay::kPOff + r_local * 128;
     for (int j = 0; j < ntiles && ok; ++j) {
+      if (!warp_live) break;  // padding rows: nothing to compute, nothing to signal
       if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, abort))) { ok = false; break; }
-      if (!warp_live) {
-        mbar_arrive(smem_u32(&bars->p_full));
-        continue;
-      }
       tc_fence_after();
       float x[kBN];
       tmem_ld32(t_s + (uint32_t)((j & 1) * kBN), x);
