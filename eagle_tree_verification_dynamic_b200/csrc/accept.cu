@@ -54,8 +54,8 @@ struct AcceptSmem {
   int amax[EAGLE_MAX_NODES + 1];       // target argmax of row j
   double lse_t[EAGLE_MAX_NODES + 1];   // target log-sum-exp of row j
   double lse_d[EAGLE_MAX_NODES + 1];   // log-sum-exp of node j's draft row
-  float tl[EAGLE_MAX_NODES + 1];       // child c: target logit of its token in its parent's row
-  float dl[EAGLE_MAX_NODES + 1];       // child c: draft logit of its token in its parent's draft row
+  double px[EAGLE_MAX_NODES + 1];      // child c: p(x_c) under its parent's target row
+  double qx[EAGLE_MAX_NODES + 1];      // child c: q(x_c) under its parent's draft row
   double warp_part[kAcceptWarps];
   double red[2][kAcceptWarps];   // block-reduction slots, alternating by call
   double lane_sum[kAcceptThreads];
@@ -138,22 +138,24 @@ __device__ double cluster_sum(double cta_value, AcceptSmem& sm, cg::cluster_grou
 template <typename T>
 __device__ double sweep_total(const Slice<T>& sl, const SweepArgs& a, AcceptSmem& sm, cg::cluster_group& cluster,
                               Parity& par) {
-  double acc = 0.0;
-  for (int i = 0; i < sl.x1 - sl.x0; ++i) acc += (double)sl.weight(a, i);
-  return cluster_sum(block_sum(acc, sm, par.red), sm, cluster, nullptr, par.cl);
+  float acc = 0.f;  // a slice is <= 32 terms: fp32 within it, fp64 across slices
+  for (int i = 0; i < sl.x1 - sl.x0; ++i) acc += sl.weight(a, i);
+  return cluster_sum(block_sum((double)acc, sm, par.red), sm, cluster, nullptr, par.cl);
 }
 
 // Inverse CDF over the weights: smallest x with cumsum_x > u * total.  Writes
 // the token to *out from the one thread that owns the crossing; returns the
-// total weight (every thread).  Each thread sums its slice in token order, in
-// fp64, element by element; the owner's rescan repeats exactly those additions.
+// total weight (every thread).  Each thread sums its slice (<= 32 terms) in
+// token order in fp32; the owner's rescan repeats exactly those additions, so
+// the crossing lies inside the slice whose interval contains the threshold.
 template <typename T>
 __device__ double sweep_sample(const Slice<T>& sl, const SweepArgs& a, float u, AcceptSmem& sm,
                                cg::cluster_group& cluster, int32_t* out, Parity& par) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int len = sl.x1 - sl.x0;
-  double mine = 0.0;
-  for (int i = 0; i < len; ++i) mine += (double)sl.weight(a, i);
+  float mine_f = 0.f;  // fp32 within the slice; the owner's rescan repeats these additions
+  for (int i = 0; i < len; ++i) mine_f += sl.weight(a, i);
+  const double mine = (double)mine_f;
   // Block exclusive prefix of the per-thread sums, summed serially (lane order
   // within a warp, then warp order) so the prefixes never decrease and the
   // ownership intervals [prefix[t], prefix[t+1]) tile [0, total) exactly.
@@ -183,13 +185,13 @@ __device__ double sweep_sample(const Slice<T>& sl, const SweepArgs& a, float u, 
     const double start = my_off + sm.prefix[tid];
     const double end = my_off + sm.prefix[tid + 1];
     if (start <= thr && thr < end) {
-      double run = 0.0;
+      float run = 0.f;
       int pick = -1, last_nz = -1;
       for (int i = 0; i < len; ++i) {
         const float w = sl.weight(a, i);
         if (w > 0.f) last_nz = sl.x0 + i;
-        run += (double)w;
-        if (my_off + (sm.prefix[tid] + run) > thr) { pick = sl.x0 + i; break; }
+        run += w;
+        if (my_off + (sm.prefix[tid] + (double)run) > thr) { pick = sl.x0 + i; break; }
       }
       *out = pick >= 0 ? pick : last_nz;
     }
@@ -231,16 +233,19 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     for (int i = tid; i <= n; i += kAcceptThreads) {
       const int r = sm.drow[i];
       sm.lse_d[i] = r >= 0 ? dlse[(size_t)b * R + r] : 0.0;
-      if (i == 0) continue;
+    }
+    __syncthreads();
+    // one thread per child: p and q of its token under its parent's rows
+    for (int i = tid + 1; i <= n; i += kAcceptThreads) {
       const int par = sm.par[i - 1], x = sm.tok[i - 1];
-      float tv = -INFINITY, dv = -INFINITY;
+      double pv = 0.0, qv = 0.0;
       if (par >= 0 && par <= n && x >= 0 && x < V) {
-        tv = load_logit(tgt + (trow0 + par) * (size_t)V + x);
-        const int pr = draft_row[(size_t)b * (n + 1) + par];
-        if (pr >= 0 && pr < R) dv = load_logit(dft + ((size_t)b * R + pr) * (size_t)V + x);
+        const int pr = sm.drow[par];
+        pv = exp((double)load_logit(tgt + (trow0 + par) * (size_t)V + x) - sm.lse_t[par]);
+        if (pr >= 0) qv = exp((double)load_logit(dft + ((size_t)b * R + pr) * (size_t)V + x) - sm.lse_d[par]);
       }
-      sm.tl[i] = tv;
-      sm.dl[i] = dv;
+      sm.px[i] = pv;
+      sm.qx[i] = qv;
     }
     __syncthreads();
   }
@@ -281,15 +286,11 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
       while (true) {
         while (c <= n && sm.par[c - 1] != j) ++c;
         if (c > n || r < 0) break;
-        const int x = sm.tok[c - 1];
-        double ratio = 0.0;  // a token outside the vocabulary is never accepted
-        if (x >= 0 && x < V) {
-          const double px = exp((double)sm.tl[c] - lse_t);
-          const double qx = exp((double)sm.dl[c] - lse_d);
-          const double rho = t == 0.0 ? px : fmax(0.0, px - t * qx);
-          ratio = rho / (F * qx);
-        }
-        if ((double)u_acc[c] < ratio) { moved_to = c; break; }
+        // accept iff u < rho / (F q), i.e. u F q < rho (q > 0); a token outside
+        // the vocabulary has p = q = 0 and is never accepted
+        const double px = sm.px[c], qx = sm.qx[c];
+        const double rho = t == 0.0 ? px : fmax(0.0, px - t * qx);
+        if (qx > 0.0 && (double)u_acc[c] * (F * qx) < rho) { moved_to = c; break; }
         // rejected: the current target becomes max(0, p - t' q) / F(t')
         t += F;
         rejected_here = true;

@@ -18,12 +18,18 @@
 //               log2 units, then O and the row sum are rescaled in TMEM),
 //               writes P = 2^(x - m) as bf16 into swizzled shared memory
 // The last split column handles the n tree keys, visible per the ancestor
-// bitmask.  Every CTA writes its normalised partial output and log-sum-exp;
-// attn_combine_kernel merges the splits.
+// bitmask.  The splits of one (sequence, KV head, row group) form one thread
+// block cluster: each CTA parks its normalised partial output and log-sum-exp
+// in its own shared memory, then every CTA combines a slice of the rows from
+// all partials through distributed shared memory and writes bf16 output
+// (out = sum_s e^{lse_s - M} O_s / sum_s e^{lse_s - M}).  No partial leaves the
+// chip and no second kernel runs.
 //
 // Every mbarrier wait is bounded (about 2 s of wall time); a timeout sets an
 // abort flag that ends all roles, records an error word in the workspace
-// header and still frees the TMEM columns before the CTA exits.
+// header and still frees the TMEM columns.  No path returns early: every CTA
+// reaches both cluster barriers of the combine.
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -31,6 +37,8 @@
 
 #include "eagle_internal.h"
 #include "sm100_ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace eagle {
 
@@ -77,8 +85,7 @@ struct TcParams {
   const int32_t* plen;
   const uint64_t* mask;
   const int32_t* pos;
-  float* part_o;
-  float* part_lse;
+  __nv_bfloat16* out;
   int* err;
   int Lmax, n, Hq, Hkv, window, n_splits, chunk, row_groups;
   int q_by_tma;      // 1: Q rows arrive by TMA (G divides 128), 0: gathered by the threads
@@ -94,10 +101,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   extern __shared__ __align__(1024) unsigned char smem[];
   TcBars* bars = reinterpret_cast<TcBars*>(smem + Lay::kBarOff);
   const uint32_t s_base = smem_u32(smem);
-  if (s_base & 1023u) {  // the swizzled tiles need 1024-byte alignment
-    if (threadIdx.x == 0) atomicExch(p.err, 2);
-    return;
-  }
+  const bool aligned = (s_base & 1023u) == 0;  // the swizzled tiles need 1024-byte alignment
+  cg::cluster_group cluster = cg::this_cluster();
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int s = blockIdx.x, g = blockIdx.y;
@@ -128,15 +133,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   const int qi = row_ok ? r_glob / G : 0;
   const int qh = row_ok ? g * G + r_glob % G : 0;
 
-  if (ntiles == 0) {  // nothing visible in this split: an empty partial
-    if (row_ok) {
-      const size_t slot = (((size_t)s * B + b) * p.n + qi) * p.Hq + qh;
-      for (int d = 0; d < D; ++d) p.part_o[slot * D + d] = 0.f;
-      p.part_lse[slot] = -INFINITY;
-    }
-    return;
-  }
+  // A CTA with nothing to do (no visible key in its split, or a misaligned
+  // shared-memory base) still takes part in the cluster's combine below.
+  const bool work = aligned && ntiles > 0;
+  if (!aligned && tid == 0) atomicExch(p.err, 2);
+  float m_used = -INFINITY, l = 0.f;  // softmax threads: reference max (scaled, log2) and row sum
+  bool final_ok = false;              // softmax threads: O in TMEM is complete for this row
+  uint32_t tmem = 0;
+  volatile int* abort = &bars->abort;
 
+  if (work) {
   // ---- set-up: barriers, TMEM, Q tile
   if (tid == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
@@ -204,8 +210,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
-  volatile int* abort = &bars->abort;
+  tmem = bars->tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -314,7 +319,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       mw1 = p.mask[((size_t)b * p.n + qi) * 2 + 1];
     }
     const float sl2 = p.scale_log2;
-    float m_used = -INFINITY, l = 0.f;  // running reference max (scaled, log2 units) and row sum
     bool ok = true;
     unsigned char* prow = smem + Lay::kPOff + r_local * 128;
     for (int j = 0; j < ntiles && ok; ++j) {
@@ -387,31 +391,86 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       tc_fence_before();
       mbar_arrive(smem_u32(&bars->p_full));
     }
-    // epilogue: normalised partial output and its log-sum-exp
-    if (ok && warp_live && __all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (ntiles - 1) & 1, abort))) {
-      tc_fence_after();
+    final_ok = ok && warp_live &&
+               __all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (ntiles - 1) & 1, abort));
+  }
+  }  // work
+
+  // ---- park this split's normalised partial (O rows, log-sum-exp) in shared
+  // memory: the K/V stages hold O (row r: D floats, 16-byte chunks XOR-swizzled
+  // by r), the P buffer holds the 128 log-sum-exps.  All TMA copies and MMAs of
+  // this CTA have drained before the barrier below.
+  float* o_part = reinterpret_cast<float*>(smem + Lay::kStageOff);
+  float* lse_part = reinterpret_cast<float*>(smem + Lay::kPOff);
+  constexpr int kChunks = D / 4;  // 16-byte chunks per O row
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp >= 2) {
+    float lse_r = -INFINITY;
+    if (final_ok) {  // warp-uniform
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      const size_t slot = (((size_t)s * B + b) * p.n + qi) * p.Hq + qh;
+      const uint32_t t_o = tmem + ((uint32_t)(quad * 32) << 16) + Lay::kColO;
       for (int c0 = 0; c0 < D; c0 += 32) {
         float o[32];
         tmem_ld32(t_o + c0, o);
         tmem_wait_ld();
-        if (row_ok) {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + slot * D + c0);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) dst[t] = make_float4(o[4 * t] * inv, o[4 * t + 1] * inv, o[4 * t + 2] * inv,
-                                                            o[4 * t + 3] * inv);
+        for (int t = 0; t < 8; ++t) {
+          const int c = (c0 >> 2) + t;
+          *reinterpret_cast<float4*>(o_part + r_local * D + ((c ^ (r_local & (kChunks - 1))) << 2)) =
+              make_float4(o[4 * t] * inv, o[4 * t + 1] * inv, o[4 * t + 2] * inv, o[4 * t + 3] * inv);
         }
       }
-      if (row_ok) p.part_lse[slot] = l > 0.f ? (m_used + __log2f(l)) * (float)kLn2 : -INFINITY;
+      if (row_ok && l > 0.f) lse_r = (m_used + __log2f(l)) * (float)kLn2;
     }
+    lse_part[r_local] = lse_r;
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (*abort && tid == 0) atomicExch(p.err, 1);
-  if (warp == 0) tmem_dealloc(tmem, Lay::kTmemCols);
+  if (work && *abort && tid == 0) atomicExch(p.err, 1);
+  if (work && warp == 0) tmem_dealloc(tmem, Lay::kTmemCols);
+
+  // ---- combine the splits of this (sequence, KV head, row group) across the
+  // cluster: rank cr reduces a slice of the rows, reading every split's
+  // partial through distributed shared memory, and writes bf16 output
+  //   out = sum_s e^{lse_s - M} O_s / sum_s e^{lse_s - M}
+  cluster.sync();
+  {
+    const int CS = (int)cluster.num_blocks(), cr = (int)cluster.block_rank();
+    const int valid = min(kRowsPerCta, rows - row0);
+    const int per = (valid + CS - 1) / CS;
+    const int r_end = min(valid, (cr + 1) * per);
+    constexpr int DPL = D / 32;  // output dims per lane
+    for (int r = cr * per + warp; r < r_end; r += kTcThreads / 32) {
+      const float ls = lane < CS ? *cluster.map_shared_rank(lse_part + r, lane) : -INFINITY;
+      const float M = warp_max_f(ls);
+      const float w = (lane < CS && ls > -INFINITY) ? __expf(ls - M) : 0.f;
+      const float wsum = warp_sum_f(w);
+      float acc[DPL];
+#pragma unroll
+      for (int t = 0; t < DPL; ++t) acc[t] = 0.f;
+      const int c = (lane * DPL) >> 2;  // this lane's 16-byte chunk
+      const int within = (lane * DPL) & 3;
+      const int off = r * D + ((c ^ (r & (kChunks - 1))) << 2) + within;
+      for (int sp = 0; sp < CS; ++sp) {
+        const float ws = __shfl_sync(kFull, w, sp);
+        if (ws == 0.f) continue;
+        const float* src = cluster.map_shared_rank(o_part, sp) + off;
+#pragma unroll
+        for (int t = 0; t < DPL; ++t) acc[t] = fmaf(ws, src[t], acc[t]);
+      }
+      const int rg_row = row0 + r;
+      const int i = rg_row / G, h = g * G + rg_row % G;
+      __nv_bfloat16* dst = p.out + (((size_t)b * p.n + i) * p.Hq + h) * D + lane * DPL;
+      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+      for (int t = 0; t < DPL; t += 2)
+        *reinterpret_cast<__nv_bfloat162*>(dst + t) = __floats2bfloat162_rn(acc[t] * inv, acc[t + 1] * inv);
+    }
+  }
+  cluster.sync();  // no CTA leaves while another may still read its shared memory
 }
 
 // ------------------------------------------------------------------- host
@@ -452,8 +511,8 @@ int attention_row_groups(int n, int Hq, int Hkv) {
 template <int D>
 static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
                              const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
-                             int n, int Hq, int Hkv, int window, float scale, const AttnPlan& plan, float* part_o,
-                             float* part_lse, int* err, cudaStream_t s) {
+                             int n, int Hq, int Hkv, int window, float scale, const AttnPlan& plan, void* out,
+                             int* err, cudaStream_t s) {
   CUtensorMap mk, mv, mkt, mvt;
   const int Lrows = Lmax > 0 ? Lmax : 1;
   const void* kbase = Lmax > 0 ? kc : kt;  // any valid address when the cache is empty
@@ -489,8 +548,7 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
   p.plen = plen;
   p.mask = mask;
   p.pos = pos;
-  p.part_o = part_o;
-  p.part_lse = part_lse;
+  p.out = static_cast<__nv_bfloat16*>(out);
   p.err = err;
   p.Lmax = Lmax;
   p.n = n;
@@ -504,20 +562,37 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
   const size_t smem = TcLayout<D>::kSmemBytes;
   cudaError_t e = ensure_smem_limit((const void*)attn_tc_kernel<D>, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(plan.n_splits + 1, Hkv, B * p.row_groups);
-  attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(mk, mv, mkt, mvt, mq, p);
-  return cudaGetLastError();
+  const int cs = plan.n_splits + 1;  // one cluster = every split of one (sequence, KV head, row group)
+  if (cs > 8) {
+    static bool np_set[2] = {false, false};
+    if (!np_set[D == 128]) {
+      e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+      np_set[D == 128] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, Hkv, B * p.row_groups);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D>, mk, mv, mkt, mvt, mq, p);
 }
 
 cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
                                 const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
                                 int n, int Hq, int Hkv, int D, int window, float scale, const AttnPlan& plan,
-                                float* part_o, float* part_lse, int* err, cudaStream_t s) {
+                                void* out, int* err, cudaStream_t s) {
   if (D == 128)
-    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, plan, part_o,
-                          part_lse, err, s);
-  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, plan, part_o,
-                       part_lse, err, s);
+    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, plan, out, err, s);
+  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, plan, out, err, s);
 }
 
 }  // namespace eagle

@@ -47,7 +47,7 @@ cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* depth, const
 
 // ---- attention (attention.cu, attention_tc.cu)
 struct AttnPlan {
-  int n_splits;   // prefix splits (one more CTA column handles the tree keys)
+  int n_splits;   // prefix splits (one more CTA handles the tree keys); <= 15
   int chunk;      // prefix keys per split (multiple of 64)
   int span;       // prefix keys a sequence can see at most (Lmax, or the window)
 };
@@ -61,7 +61,7 @@ cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc,
 cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
                                 const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
                                 int n, int Hq, int Hkv, int D, int window, float scale, const AttnPlan& plan,
-                                float* part_o, float* part_lse, int* err, cudaStream_t s);
+                                void* out, int* err, cudaStream_t s);
 
 // ---- accept (accept.cu)
 size_t accept_ws_bytes(int B, int n, int V, int dtype);

@@ -175,7 +175,8 @@ EAGLE_API eagle_status eagle_tree_mask(const int32_t* parents, const int32_t* de
  *   scale    softmax scale; <= 0 selects 1/sqrt(D)
  * Limits: D in {64, 128}, Hq % Hkv == 0, n <= EAGLE_MAX_NODES, all tensor
  * pointers 16-byte aligned.  Workspace: eagle_tree_attention_workspace_bytes
- * (split-KV partial outputs). */
+ * (a 256-byte header with the kernel's device status word: 0 = ok, 1 = an
+ * internal wait gave up, 2 = misaligned shared memory). */
 EAGLE_API size_t eagle_tree_attention_workspace_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window);
 EAGLE_API eagle_status eagle_tree_attention(const void* q, const void* k_cache, const void* v_cache,
                                   const int32_t* prefix_len, int Lmax, const void* k_tree,
