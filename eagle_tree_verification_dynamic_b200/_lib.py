@@ -241,8 +241,8 @@ def tree_attention(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos=No
 
 def check_attention_status(ws: torch.Tensor):
     """Read the device status word the attention kernel keeps in its workspace
-    header (synchronises the stream).  Non-zero means a bounded wait inside the
-    kernel gave up (1) or the shared-memory base was misaligned (2)."""
+    header (synchronises the stream).  Non-zero (1) means a bounded wait inside
+    the kernel gave up."""
     code = int(ws[:4].view(torch.int32).item())
     if code != 0:
         raise EagleError(f"eagle_tree_attention: device status {code}")

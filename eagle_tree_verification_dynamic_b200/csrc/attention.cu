@@ -1,42 +1,34 @@
 // Host plan of the tree attention ("Tree Attention" verification of the EAGLE
-// notes, "3.Verify"): how many key splits, and how many keys each, so that
-// about two CTAs per SM are busy; the kernel itself is attention_tc.cu.
+// notes, "3.Verify"): how many CTAs share the tile list, and the workspace that
+// holds the partials of units cut by CTA range boundaries.  The kernels are in
+// attention_tc.cu.
 #include "eagle_internal.h"
 
 namespace eagle {
 
-AttnPlan plan_attention(int B, int n, int Hq, int Hkv, int Lmax, int window) {
-  AttnPlan p;
-  p.span = window > 0 ? (Lmax < window ? Lmax : window) : Lmax;
-  if (p.span < 1) p.span = 1;
-  // two CTAs per SM: aim for ~2 x 148 CTAs over (row groups x heads x splits);
-  // the splits of one head (plus its tree-key split) form one cluster of <= 16
-  const int heads = B * Hkv * attention_row_groups(n, Hq, Hkv);
-  int splits = (2 * kNumSMs + heads - 1) / heads;
-  const int max_splits = (p.span + 63) / 64;
-  if (splits > max_splits) splits = max_splits;
-  if (splits > 15) splits = 15;
-  if (splits < 1) splits = 1;
-  int chunk = (p.span + splits - 1) / splits;
-  chunk = (chunk + 63) / 64 * 64;
-  p.chunk = chunk;
-  p.n_splits = (p.span + chunk - 1) / chunk;
-  return p;
+int attention_row_groups(int n, int Hq, int Hkv) {
+  const int rows = n * (Hq / Hkv);
+  return (rows + kAttnRowsPerUnit - 1) / kAttnRowsPerUnit;
 }
 
-// workspace: a 256-byte header holding the kernel's device status word
-size_t attention_ws_bytes(int, int, int, int, int, int, int) { return 256; }
+int attention_ctas(int B, int n, int Hq, int Hkv, int Lmax, int window) {
+  const long long span = window > 0 ? (Lmax < window ? Lmax : window) : Lmax;
+  const long long tiles_max = (span + kAttnKeysPerTile - 1) / kAttnKeysPerTile + (n + kAttnKeysPerTile - 1) / kAttnKeysPerTile;
+  const long long T_max = (long long)B * Hkv * attention_row_groups(n, Hq, Hkv) * tiles_max;
+  return (int)(T_max < kNumSMs ? T_max : kNumSMs);
+}
 
-cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
-                                  const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
-                                  int n, int Hq, int Hkv, int D, int window, float scale, void* out, void* ws,
-                                  cudaStream_t s) {
-  const AttnPlan p = plan_attention(B, n, Hq, Hkv, Lmax, window);
-  int* err = reinterpret_cast<int*>(ws);
-  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
-  if (e != cudaSuccess) return e;
-  return launch_attention_tc(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, D, window, scale, p, out,
-                             err, s);
+AttnWorkspace attention_ws_layout(int B, int n, int Hq, int Hkv, int D, int Lmax, int window) {
+  AttnWorkspace w;
+  const int C = attention_ctas(B, n, Hq, Hkv, Lmax, window);
+  const size_t U = (size_t)B * Hkv * attention_row_groups(n, Hq, Hkv);
+  const size_t slots = (size_t)C + U;
+  w.status_off = 0;
+  w.cta_status_off = 256;
+  w.part_lse_off = align_up(w.cta_status_off + sizeof(int) * (size_t)C, 256);
+  w.part_o_off = align_up(w.part_lse_off + sizeof(float) * slots * kAttnRowsPerUnit, 256);
+  w.bytes = align_up(w.part_o_off + sizeof(float) * slots * kAttnRowsPerUnit * (size_t)D, 256);
+  return w;
 }
 
 }  // namespace eagle

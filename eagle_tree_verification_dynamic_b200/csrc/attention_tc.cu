@@ -3,33 +3,34 @@
 // semantics of "Технический анализ EAGLE-4", section "Деревья проверки
 // EAGLE-4 и утилита управления").
 //
-// One CTA = (key split, KV head g, sequence b, group of 128 query rows).  The
-// 128 rows are the (node, head-in-group) pairs of head g, so every K/V tile
-// staged in shared memory serves all tree queries of the GQA group at once.
-//   warp 0      TMA producer: K and V tiles of 64 keys into a 2-stage ring
-//               (128-byte swizzle, no multicast); also allocates TMEM
+// Work decomposition.  A unit is (sequence b, KV head g, group rg of 128 query
+// rows); the rows are the (node, head-in-group) pairs of head g, so every K/V
+// tile staged in shared memory serves all tree queries of the GQA group.  A
+// unit's keys are cut into tiles of 64: its visible prefix range first, then
+// its n tree keys.  All tiles of all units form one list (unit-major) that is
+// cut into C equal contiguous ranges, one per CTA, with C <= the SM count and
+// one CTA per SM: every CTA streams the same amount of KV whatever the prefix
+// lengths of a ragged batch.  Each CTA derives the list from prefix_len itself.
+// A unit that lies inside one CTA's range is finished there (bf16 output); a
+// unit cut by range boundaries leaves one normalised partial (O rows and
+// log-sum-exp) per piece, merged by attn_combine_kernel.
+//
+// Roles inside a CTA (192 threads):
+//   warp 0      producer: Q of each unit (TMA box, or a gather when G does not
+//               divide 128) into one of two Q buffers; K and V tiles into a
+//               ring of stages (128-byte swizzle, no multicast); TMEM owner
 //   warp 1      one thread issues tcgen05.mma: S = Q K^T into one of two TMEM
-//               buffers (the next tile's S is computed while this tile's
-//               softmax runs), then O += P V into TMEM (fp32 accumulators,
-//               bf16 operands)
-//   warps 2-5   softmax: thread r owns TMEM lane r = query row r; reads its S
-//               row, applies the prefix range / window / tree bitmask, keeps a
-//               running reference max (re-based only when it grows by > 8 in
-//               log2 units, then O and the row sum are rescaled in TMEM),
-//               writes P = 2^(x - m) as bf16 into swizzled shared memory
-// The last split column handles the n tree keys, visible per the ancestor
-// bitmask.  The splits of one (sequence, KV head, row group) form one thread
-// block cluster: each CTA parks its normalised partial output and log-sum-exp
-// in its own shared memory, then every CTA combines a slice of the rows from
-// all partials through distributed shared memory and writes bf16 output
-// (out = sum_s e^{lse_s - M} O_s / sum_s e^{lse_s - M}).  No partial leaves the
-// chip and no second kernel runs.
+//               S buffers, at most one tile ahead of PV; O += P V into TMEM
+//   warps 2-5   softmax: thread r owns TMEM lane r = query row r; applies the
+//               prefix range / window / tree bitmask, keeps a running reference
+//               max (re-based only when it grows by > 8 in log2 units, then O
+//               and the row sum are rescaled in TMEM), writes P = 2^(x - m) as
+//               bf16 into one of two swizzled P buffers; at the end of a unit's
+//               piece it normalises O and writes the output or the partial
 //
 // Every mbarrier wait is bounded (about 2 s of wall time); a timeout sets an
-// abort flag that ends all roles, records an error word in the workspace
-// header and still frees the TMEM columns.  No path returns early: every CTA
-// reaches both cluster barriers of the combine.
-#include <cooperative_groups.h>
+// abort flag that ends all roles, records a per-CTA status word and still
+// frees the TMEM columns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -38,267 +39,488 @@
 #include "eagle_internal.h"
 #include "sm100_ptx.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace eagle {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 192;  // 6 warps
-constexpr int kBN = 64;          // keys per tile
-constexpr int kStages = 2;
-constexpr int kRowsPerCta = 128;
+constexpr int kTcThreads = 192;   // 6 warps
+constexpr int kBN = kAttnKeysPerTile;
+constexpr int kRowsPerCta = kAttnRowsPerUnit;
+constexpr int kMaxStages = 8;
+constexpr int kSmemOptIn = 232448;  // largest dynamic shared memory a block may opt into on sm_100
+constexpr int kCombineThreads = 128;
 
 template <int D>
 struct TcLayout {
-  static constexpr int kAtoms = D / 64;                 // 128-byte column atoms along D
-  static constexpr int kQBytes = kAtoms * 128 * 128;    // 128 rows
-  static constexpr int kPBytes = 128 * 128;             // 128 rows x 64 keys bf16
-  static constexpr int kKVAtomBytes = kBN * 128;        // 64 keys x 128 B
+  static constexpr int kAtoms = D / 64;               // 128-byte column atoms along D
+  static constexpr int kQBytes = kAtoms * 128 * 128;  // 128 rows
+  static constexpr int kPBytes = 128 * 128;           // 128 rows x 64 keys bf16
+  static constexpr int kKVAtomBytes = kBN * 128;      // 64 keys x 128 B
   static constexpr int kKBytes = kAtoms * kKVAtomBytes;
-  static constexpr int kStageBytes = 2 * kKBytes;       // K + V
-  static constexpr int kQOff = 0;
-  static constexpr int kPOff = kQOff + kQBytes;
-  static constexpr int kStageOff = kPOff + kPBytes;
+  static constexpr int kStageBytes = 2 * kKBytes;     // K + V
+  static constexpr int kBarBytes = 512;
+  static constexpr int kFixed = 2 * kQBytes + 2 * kPBytes + kBarBytes + 1024;  // + base alignment slack
+  static constexpr int kStagesFit = (kSmemOptIn - kFixed) / kStageBytes;
+  static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
+  static constexpr int kQOff = 0;                      // two Q buffers
+  static constexpr int kPOff = 2 * kQBytes;            // two P buffers
+  static constexpr int kStageOff = kPOff + 2 * kPBytes;
   static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
-  static constexpr int kSmemBytes = kBarOff + 128;  // + barriers (base is 1024-aligned, checked)
-  static constexpr uint32_t kTmemCols = 256;  // S double buffer (2 x 64) + O (D)
-  static constexpr uint32_t kColS = 0;        // S buffer b at column 64 * b
+  static constexpr int kSmemBytes = kBarOff + kBarBytes + 1024;
+  static constexpr uint32_t kTmemCols = 256;  // S double buffer (2 x 64) + O (D <= 128)
+  static constexpr uint32_t kColS = 0;        // S buffer i at column 64 * i
   static constexpr uint32_t kColO = 128;
+  static_assert(kStages >= 2, "at least a double-buffered K/V ring");
+  static_assert(kSmemBytes <= kSmemOptIn, "shared memory");
 };
 
 struct TcBars {
-  uint64_t q_full;
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t s_full[2];
-  uint64_t p_full;
-  uint64_t pv_done;
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
   uint64_t mma_idle;
   uint32_t tmem_base;
   int abort;
+  // this CTA's tile range [t0, t1) of the global list, and where it starts
+  int n_tiles;  // t1 - t0
+  int b0, hr0, off0;
 };
-static_assert(sizeof(TcBars) <= 128, "barrier block");
+static_assert(sizeof(TcBars) <= 512, "barrier block");
+
+// ----------------------------------------------------------- tile schedule
+struct AttnGeom {
+  const int32_t* plen;
+  int B, Hkv, RG, n, Lmax, window, C;
+};
+
+__device__ __forceinline__ int geom_len(const AttnGeom& a, int b) {
+  return min(max(__ldg(a.plen + b), 0), a.Lmax);
+}
+// first visible prefix key of a sequence of length L (the window of the
+// shallowest tree node, depth 1, at position L)
+__device__ __forceinline__ int geom_lo(const AttnGeom& a, int L) {
+  return a.window > 0 ? max(0, L - a.window + 1) : 0;
+}
+__device__ __forceinline__ int geom_ptiles(const AttnGeom& a, int L) { return (L - geom_lo(a, L) + kBN - 1) / kBN; }
+__device__ __forceinline__ int geom_tiles(const AttnGeom& a, int b) {
+  return geom_ptiles(a, geom_len(a, b)) + (a.n + kBN - 1) / kBN;
+}
+
+// Whole warp: total tiles of all units, and the first tile of sequence b_end.
+__device__ long long geom_prefix(const AttnGeom& a, int b_end, int lane) {
+  const int HR = a.Hkv * a.RG;
+  long long acc = 0;
+  for (int b = lane; b < b_end; b += 32) acc += (long long)HR * geom_tiles(a, b);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+  return acc;
+}
+
+// Whole warp: the unit (b, hr) holding global tile t and t's offset in it.
+__device__ void geom_locate(const AttnGeom& a, long long t, int lane, int& b_out, int& hr_out, int& off_out) {
+  const int HR = a.Hkv * a.RG;
+  long long base = 0;
+  for (int bc = 0; bc < a.B; bc += 32) {
+    const int b = bc + lane;
+    const int tb = b < a.B ? geom_tiles(a, b) : 0;
+    const long long v = (long long)HR * tb;
+    long long inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(kFull, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const long long exc = inc - v;
+    const bool hit = b < a.B && base + exc <= t && t < base + inc;
+    const unsigned m = __ballot_sync(kFull, hit);
+    if (m) {
+      const int src = __ffs(m) - 1;
+      int bb = 0, hr = 0, off = 0;
+      if (lane == src) {
+        const long long within = t - (base + exc);
+        bb = b;
+        hr = (int)(within / tb);
+        off = (int)(within % tb);
+      }
+      b_out = __shfl_sync(kFull, bb, src);
+      hr_out = __shfl_sync(kFull, hr, src);
+      off_out = __shfl_sync(kFull, off, src);
+      return;
+    }
+    base += __shfl_sync(kFull, inc, 31);
+  }
+  b_out = a.B;
+  hr_out = 0;
+  off_out = 0;
+}
+
+// CTA c holds tiles [c*T/C, (c+1)*T/C); this is the CTA holding tile t.
+__device__ __forceinline__ int cta_of_tile(long long t, long long T, int C) {
+  return (int)(((t + 1) * C - 1) / T);
+}
+// With fewer tiles than CTAs (a ragged batch far below Lmax) some ranges are empty.
+__device__ __forceinline__ bool cta_nonempty(int c, long long T, int C) {
+  return (long long)(c + 1) * T / C > (long long)c * T / C;
+}
+
+// One contiguous piece of a unit inside one CTA's range.
+struct Piece {
+  int b, hr;    // unit = b * HR + hr
+  int tb, te;   // tiles [tb, te) of the unit
+  int ptiles;   // the unit's prefix tiles (tiles >= ptiles are tree tiles)
+  int L, lo;    // prefix length and first visible prefix key
+  bool whole;   // the piece is the entire unit
+};
+
+struct PieceCursor {
+  int b, hr, off, left;
+  __device__ void init(int b0, int hr0, int off0, int n_tiles) {
+    b = b0;
+    hr = hr0;
+    off = off0;
+    left = n_tiles;
+  }
+  __device__ void init(const TcBars* s) { init(s->b0, s->hr0, s->off0, s->n_tiles); }
+  __device__ bool next(const AttnGeom& a, Piece& pc) {
+    if (left <= 0) return false;
+    const int HR = a.Hkv * a.RG;
+    pc.b = b;
+    pc.hr = hr;
+    pc.L = geom_len(a, b);
+    pc.lo = geom_lo(a, pc.L);
+    pc.ptiles = geom_ptiles(a, pc.L);
+    const int tiles = pc.ptiles + (a.n + kBN - 1) / kBN;
+    const int nt = min(tiles - off, left);
+    pc.tb = off;
+    pc.te = off + nt;
+    pc.whole = off == 0 && nt == tiles;
+    left -= nt;
+    off = 0;
+    if (++hr == HR) {
+      hr = 0;
+      ++b;
+    }
+    return true;
+  }
+};
 
 struct TcParams {
   const __nv_bfloat16* q;
-  const int32_t* plen;
   const uint64_t* mask;
   const int32_t* pos;
   __nv_bfloat16* out;
-  int* err;
-  int Lmax, n, Hq, Hkv, window, n_splits, chunk, row_groups;
-  int q_by_tma;      // 1: Q rows arrive by TMA (G divides 128), 0: gathered by the threads
+  float* part_o;    // [C + U][128][D] normalised partial outputs
+  float* part_lse;  // [C + U][128]
+  int* cta_status;  // [C]
+  AttnGeom geo;
+  int Hq;
+  int q_by_tma;      // 1: Q rows arrive by TMA (G divides 128), 0: gathered by the producer warp
   float scale_log2;  // softmax scale * log2(e)
 };
 
+// Loads issued now and consumed later: the K/V stream keeps HBM saturated, so
+// a demand load waits behind it for microseconds; the per-row inputs of a
+// piece are therefore requested a whole piece ahead (the first piece's before
+// the stream starts).
+__device__ __forceinline__ uint64_t ld_early_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.global.nc.u64 %0, [%1];" : "=l"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ int ld_early_s32(const int32_t* p) {
+  int v;
+  asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// What a softmax thread reads besides S for one piece.
+struct RowCtx {
+  uint64_t mw0, mw1;  // ancestor-or-self bitmask of this row's node (pieces with tree tiles)
+  int qpos;           // this row's position (window only)
+  int tpos[4];        // positions of tree keys lane, 32+lane, 64+lane, 96+lane (window and tree tiles)
+};
+
+__device__ __forceinline__ void row_issue(RowCtx& rc, const Piece& pc, const TcParams& p, int r_local, int lane,
+                                          int G) {
+  const AttnGeom& a = p.geo;
+  const int r_glob = (pc.hr % a.RG) * kRowsPerCta + r_local;
+  const bool row_ok = r_glob < a.n * G;
+  const int qi = row_ok ? r_glob / G : 0;
+  const size_t nb = (size_t)pc.b * a.n;
+  const bool has_tree = pc.te > pc.ptiles;
+  rc.mw0 = rc.mw1 = 0;
+  rc.qpos = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) rc.tpos[i] = 0;
+  if (row_ok && has_tree) {
+    rc.mw0 = ld_early_u64(p.mask + (nb + qi) * 2);
+    rc.mw1 = ld_early_u64(p.mask + (nb + qi) * 2 + 1);
+  }
+  if (a.window > 0) {
+    if (row_ok) rc.qpos = ld_early_s32(p.pos + nb + qi);
+    if (has_tree) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (32 * i + lane < a.n) rc.tpos[i] = ld_early_s32(p.pos + nb + 32 * i + lane);
+    }
+  }
+}
+
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 2)
+__global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_vt,
                const __grid_constant__ CUtensorMap tm_q, const TcParams p) {
   using Lay = TcLayout<D>;
-  extern __shared__ __align__(1024) unsigned char smem[];
+  constexpr int S = Lay::kStages;
+  extern __shared__ unsigned char smem_dyn[];
+  // the swizzled tiles need 1024-byte alignment
+  unsigned char* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
   TcBars* bars = reinterpret_cast<TcBars*>(smem + Lay::kBarOff);
   const uint32_t s_base = smem_u32(smem);
-  const bool aligned = (s_base & 1023u) == 0;  // the swizzled tiles need 1024-byte alignment
-  cg::cluster_group cluster = cg::this_cluster();
+  const AttnGeom& a = p.geo;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = blockIdx.x, g = blockIdx.y;
-  const int b = blockIdx.z / p.row_groups, rg = blockIdx.z % p.row_groups;
-  const int B = gridDim.z / p.row_groups;
-  const int G = p.Hq / p.Hkv;
-  const int rows = p.n * G;
-  const int row0 = rg * kRowsPerCta;
-  const int L = min(max(p.plen[b], 0), p.Lmax);
-  const bool tree = (s == p.n_splits);
-  int k0, k1;
-  if (!tree) {
-    const int lo = p.window > 0 ? max(0, L - p.window + 1) : 0;
-    k0 = lo + s * p.chunk;
-    k1 = min(L, k0 + p.chunk);
-  } else {
-    k0 = 0;
-    k1 = p.n;
-  }
-  const int ntiles = k1 > k0 ? (k1 - k0 + kBN - 1) / kBN : 0;
-
-  // softmax thread -> query row
-  const bool is_soft = warp >= 2;
-  const int quad = warp & 3;
-  const int r_local = quad * 32 + lane;   // TMEM lane = row within the tile
-  const int r_glob = row0 + r_local;
-  const bool row_ok = is_soft && r_glob < rows;
-  const int qi = row_ok ? r_glob / G : 0;
-  const int qh = row_ok ? g * G + r_glob % G : 0;
-
-  // A CTA with nothing to do (no visible key in its split, or a misaligned
-  // shared-memory base) still takes part in the cluster's combine below.
-  const bool work = aligned && ntiles > 0;
-  if (!aligned && tid == 0) atomicExch(p.err, 2);
-  float m_used = -INFINITY, l = 0.f;  // softmax threads: reference max (scaled, log2) and row sum
-  bool final_ok = false;              // softmax threads: O in TMEM is complete for this row
-  uint32_t tmem = 0;
+  const int c = blockIdx.x;
+  const int G = p.Hq / a.Hkv;
+  const int rows = a.n * G;
+  const int HR = a.Hkv * a.RG;
   volatile int* abort = &bars->abort;
 
-  if (work) {
-  // ---- set-up: barriers, TMEM, Q tile
   if (tid == 0) {
-    mbar_init(smem_u32(&bars->q_full), 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->q_full[i]), 1);
+      mbar_init(smem_u32(&bars->q_empty[i]), 1);
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      // every softmax thread arrives for every tile, rows or not: a warp can
+      // run at most one tile ahead of P's consumer, and P is double-buffered
+      mbar_init(smem_u32(&bars->p_full[i]), 128);
+      mbar_init(smem_u32(&bars->pv_done[i]), 1);
+    }
+    for (int i = 0; i < S; ++i) {
       mbar_init(smem_u32(&bars->full[i]), 1);
       mbar_init(smem_u32(&bars->empty[i]), 1);
     }
-    mbar_init(smem_u32(&bars->s_full[0]), 1);
-    mbar_init(smem_u32(&bars->s_full[1]), 1);
-    // only warps holding at least one real query row write P and arrive; a warp
-    // of padding rows never arrives (it could otherwise run a tile ahead and
-    // complete a phase early, since S is double-buffered)
-    const int live_warps = min(4, (rows - row0 + 31) / 32);
-    mbar_init(smem_u32(&bars->p_full), 32 * live_warps);
-    mbar_init(smem_u32(&bars->pv_done), 1);
     mbar_init(smem_u32(&bars->mma_idle), 1);
     bars->abort = 0;
     fence_mbar_init();
-    if (p.q_by_tma) {
-      // the 128 query rows of this tile = (node, head-in-group) pairs: a box of
-      // {64 dims, G heads, 128/G nodes} of q viewed as [B*n][Hq][D]
-      const uint32_t qb = smem_u32(&bars->q_full);
-      mbar_arrive_expect_tx(qb, Lay::kQBytes);
-      const int rows_i = kRowsPerCta / G;
-      for (int a = 0; a < Lay::kAtoms; ++a)
-        tma_load_3d(s_base + Lay::kQOff + a * 16384, &tm_q, a * 64, g * G, b * p.n + rg * rows_i, qb);
-    }
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_kt);
     prefetch_tmap(&tm_vt);
+    if (p.q_by_tma) prefetch_tmap(&tm_q);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(&bars->tmem_base), Lay::kTmemCols);
     tmem_relinquish();
   }
-  if (!p.q_by_tma) {
-    // Q rows (bf16) -> 128-byte swizzled K-major tile; all loads issued first
-    constexpr int kVec = 128 * Lay::kAtoms * 8;
-    constexpr int kPer = (kVec + kTcThreads - 1) / kTcThreads;
-    uint4 v[kPer];
-#pragma unroll
-    for (int t = 0; t < kPer; ++t) {
-      const int e = tid + t * kTcThreads;
-      v[t] = make_uint4(0, 0, 0, 0);
-      if (e < kVec) {
-        const int r = e / (Lay::kAtoms * 8), a = (e / 8) % Lay::kAtoms, c = e % 8;
-        const int rr = row0 + r;
-        if (rr < rows) {
-          const int i = rr / G, h = g * G + rr % G;
-          v[t] = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * p.n + i) * p.Hq + h) * D + a * 64 + c * 8);
-        }
-      }
+  // inputs may come from the previous kernel on the stream
+  griddep_wait();
+  // softmax warps: cursor and the first piece's row inputs, requested before
+  // the K/V stream starts
+  PieceCursor scur;
+  Piece spc;
+  RowCtx src;
+  bool s_have = false;
+  const int quad = warp & 3;
+  const int r_local = quad * 32 + lane;  // softmax: TMEM lane = row within the unit's 128
+  if (warp >= 1) {
+    const long long T = geom_prefix(a, a.B, lane);
+    const long long t0 = (long long)c * T / a.C, t1 = (long long)(c + 1) * T / a.C;
+    int b0 = a.B, hr0 = 0, off0 = 0;
+    if (t1 > t0) geom_locate(a, t0, lane, b0, hr0, off0);
+    if (warp == 1 && lane == 0) {
+      bars->n_tiles = (int)(t1 - t0);
+      bars->b0 = b0;
+      bars->hr0 = hr0;
+      bars->off0 = off0;
     }
-#pragma unroll
-    for (int t = 0; t < kPer; ++t) {
-      const int e = tid + t * kTcThreads;
-      if (e < kVec) {
-        const int r = e / (Lay::kAtoms * 8), a = (e / 8) % Lay::kAtoms, c = e % 8;
-        *reinterpret_cast<uint4*>(smem + Lay::kQOff + a * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) = v[t];
-      }
+    if (warp >= 2) {
+      scur.init(b0, hr0, off0, (int)(t1 - t0));
+      s_have = scur.next(a, spc);
+      if (s_have) row_issue(src, spc, p, r_local, lane, G);
     }
-    fence_proxy_async_smem();
   }
+  griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  tmem = bars->tmem_base;
+  const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int issued = 0;
-      for (int j = 0; j < ntiles; ++j) {
-        const int st = j % kStages;
-        if (j >= kStages && !mbar_wait(smem_u32(&bars->empty[st]), ((j / kStages) - 1) & 1, abort)) break;
-        const uint32_t fb = smem_u32(&bars->full[st]);
-        mbar_arrive_expect_tx(fb, Lay::kStageBytes);
-        const uint32_t kdst = s_base + Lay::kStageOff + st * Lay::kStageBytes;
-        const uint32_t vdst = kdst + Lay::kKBytes;
-        const int key0 = k0 + j * kBN;
-        for (int a = 0; a < Lay::kAtoms; ++a) {
-          if (!tree) {
-            const int y = (b * p.Hkv + g) * p.Lmax + key0;
-            tma_load_2d(kdst + a * Lay::kKVAtomBytes, &tm_k, a * 64, y, fb);
-            tma_load_2d(vdst + a * Lay::kKVAtomBytes, &tm_v, a * 64, y, fb);
-          } else {
-            tma_load_3d(kdst + a * Lay::kKVAtomBytes, &tm_kt, a * 64, g, b * p.n + key0, fb);
-            tma_load_3d(vdst + a * Lay::kKVAtomBytes, &tm_vt, a * 64, g, b * p.n + key0, fb);
+    PieceCursor cur;
+    cur.init(bars);
+    Piece pc;
+    int si = 0, jg = 0;  // pieces whose Q was loaded; tiles issued
+    bool ok = true;
+    while (ok && cur.next(a, pc)) {
+      const int qb = si & 1;
+      const int g = pc.hr / a.RG, rg = pc.hr % a.RG;
+      // Q buffer qb was last read by the QK^T of piece si - 2
+      if (si >= 2 && !__all_sync(kFull, mbar_wait(smem_u32(&bars->q_empty[qb]), ((si >> 1) - 1) & 1, abort))) {
+        ok = false;
+        break;
+      }
+      const uint32_t qdst = s_base + Lay::kQOff + qb * Lay::kQBytes;
+      const uint32_t qbar = smem_u32(&bars->q_full[qb]);
+      if (p.q_by_tma) {
+        // the 128 rows = (node, head-in-group) pairs: a box of {64 dims, G
+        // heads, 128/G nodes} of q viewed as [B*n][Hq][D]
+        if (lane == 0) {
+          mbar_arrive_expect_tx(qbar, Lay::kQBytes);
+          const int rows_i = kRowsPerCta / G;
+          for (int at = 0; at < Lay::kAtoms; ++at)
+            tma_load_3d(qdst + at * 16384, &tm_q, at * 64, g * G, pc.b * a.n + rg * rows_i, qbar);
+        }
+      } else {
+        // gather: 16-byte pieces of the 128 rows into the swizzled K-major tile
+        constexpr int kVec = 128 * Lay::kAtoms * 8;
+        constexpr int kBatch = 8;
+        for (int e0 = lane; e0 < kVec; e0 += 32 * kBatch) {
+          uint4 v[kBatch];
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            const int e = e0 + u * 32;
+            v[u] = make_uint4(0, 0, 0, 0);
+            if (e < kVec) {
+              const int r = e / (Lay::kAtoms * 8), at = (e / 8) % Lay::kAtoms, cc = e % 8;
+              const int rr = rg * kRowsPerCta + r;
+              if (rr < rows) {
+                const int i = rr / G, h = g * G + rr % G;
+                v[u] = *reinterpret_cast<const uint4*>(p.q + (((size_t)pc.b * a.n + i) * p.Hq + h) * D + at * 64 +
+                                                       cc * 8);
+              }
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            const int e = e0 + u * 32;
+            if (e < kVec) {
+              const int r = e / (Lay::kAtoms * 8), at = (e / 8) % Lay::kAtoms, cc = e % 8;
+              *reinterpret_cast<uint4*>(smem + Lay::kQOff + qb * Lay::kQBytes + at * 16384 + r * 128 +
+                                        ((cc ^ (r & 7)) << 4)) = v[u];
+            }
           }
         }
-        ++issued;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(qbar);
       }
-      // drain: wait until every issued copy has landed before the CTA may exit
-      if (p.q_by_tma) mbar_wait_drain(smem_u32(&bars->q_full), 0, 200000000ull);
-      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-        mbar_wait_drain(smem_u32(&bars->full[j % kStages]), (j / kStages) & 1, 200000000ull);
+      ++si;
+      if (lane == 0) {
+        for (int t = pc.tb; t < pc.te; ++t) {
+          const int st = jg % S;
+          if (jg >= S && !mbar_wait(smem_u32(&bars->empty[st]), ((jg / S) - 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&bars->full[st]);
+          mbar_arrive_expect_tx(fb, Lay::kStageBytes);
+          const uint32_t kdst = s_base + Lay::kStageOff + st * Lay::kStageBytes;
+          const uint32_t vdst = kdst + Lay::kKBytes;
+          if (t < pc.ptiles) {
+            const int y = (pc.b * a.Hkv + g) * a.Lmax + pc.lo + t * kBN;
+            for (int at = 0; at < Lay::kAtoms; ++at) {
+              tma_load_2d(kdst + at * Lay::kKVAtomBytes, &tm_k, at * 64, y, fb);
+              tma_load_2d(vdst + at * Lay::kKVAtomBytes, &tm_v, at * 64, y, fb);
+            }
+          } else {
+            const int z = pc.b * a.n + (t - pc.ptiles) * kBN;
+            for (int at = 0; at < Lay::kAtoms; ++at) {
+              tma_load_3d(kdst + at * Lay::kKVAtomBytes, &tm_kt, at * 64, g, z, fb);
+              tma_load_3d(vdst + at * Lay::kKVAtomBytes, &tm_vt, at * 64, g, z, fb);
+            }
+          }
+          ++jg;
+        }
+      }
+      ok = __shfl_sync(kFull, ok, 0);
+      jg = __shfl_sync(kFull, jg, 0);
+    }
+    // drain: every issued copy lands before the CTA may exit
+    if (lane == 0) {
+      for (int j = (jg > S ? jg - S : 0); j < jg; ++j)
+        mbar_wait_drain(smem_u32(&bars->full[j % S]), (j / S) & 1, 200000000ull);
+      for (int s2 = (si > 2 ? si - 2 : 0); s2 < si; ++s2)
+        mbar_wait_drain(smem_u32(&bars->q_full[s2 & 1]), (s2 >> 1) & 1, 200000000ull);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(128, kBN, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t t_s = tmem + Lay::kColS, t_o = tmem + Lay::kColO;
-      const uint32_t q_addr = s_base + Lay::kQOff;
-      const uint32_t p_addr = s_base + Lay::kPOff;
-      const bool q_ok = !p.q_by_tma || mbar_wait(smem_u32(&bars->q_full), 0, abort);
-      // S = Q K_j^T into S buffer (j & 1)
-      auto issue_qk = [&](int jj) -> bool {
-        const int st = jj % kStages;
-        if (!mbar_wait(smem_u32(&bars->full[st]), (jj / kStages) & 1, abort)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk % 4) * 32;
-          const uint64_t da = smem_desc(q_addr + (kk / 4) * 16384 + off, 16, 1024, kSwizzle128B);
-          const uint64_t db = smem_desc(k_addr + (kk / 4) * Lay::kKVAtomBytes + off, 16, 1024, kSwizzle128B);
-          mma_bf16_ss(t_s + (uint32_t)((jj & 1) * kBN), da, db, id_qk, kk > 0);
+      const uint32_t t_o = tmem + Lay::kColO;
+      const int total = bars->n_tiles;
+      PieceCursor qc, pcur;
+      qc.init(bars);
+      pcur.init(bars);
+      Piece qp, pp;
+      int q_si = -1, q_rem = 0, jq = 0;  // QK^T cursor: piece, tiles left in it, next tile
+      int p_rem = 0, p_len = 0;          // PV cursor: tiles left in its piece, piece length
+      bool ok = true;
+      for (int jp = 0; jp < total && ok; ++jp) {
+        if (p_rem == 0) {
+          pcur.next(a, pp);
+          p_len = p_rem = pp.te - pp.tb;
         }
-        mma_commit(smem_u32(&bars->s_full[jj & 1]));
-        return true;
-      };
-      bool ok = q_ok && issue_qk(0);
-      int next_qk = 1;  // S has two buffers: QK^T runs at most one tile ahead of PV
-      for (int j = 0; j < ntiles && ok; ++j) {
-        // issue whichever is ready first: the next tile's QK^T (its K landed) or
-        // this tile's PV (its P is written)
-        const uint32_t pb = smem_u32(&bars->p_full);
-        uint64_t t0 = 0;
+        const bool first = p_rem == p_len;  // O restarts at the first tile of a piece
+        // issue whichever is ready first: the next QK^T (its Q and K landed)
+        // or this tile's PV (its P is written)
+        const uint32_t pb = smem_u32(&bars->p_full[jp & 1]);
+        uint64_t tw = 0;
         for (uint32_t it = 0;; ++it) {
-          if (next_qk < ntiles && next_qk <= j + 1 &&
-              mbar_try_wait(smem_u32(&bars->full[next_qk % kStages]), (next_qk / kStages) & 1)) {
-            if (!issue_qk(next_qk)) { ok = false; break; }
-            ++next_qk;
+          if (jq < total && jq <= jp + 1) {
+            if (q_rem == 0) {
+              qc.next(a, qp);
+              ++q_si;
+              q_rem = qp.te - qp.tb;
+            }
+            const int qb = q_si & 1;
+            if (mbar_try_wait(smem_u32(&bars->q_full[qb]), (q_si >> 1) & 1) &&
+                mbar_try_wait(smem_u32(&bars->full[jq % S]), (jq / S) & 1)) {
+              tc_fence_after();
+              const uint32_t q_addr = s_base + Lay::kQOff + qb * Lay::kQBytes;
+              const uint32_t k_addr = s_base + Lay::kStageOff + (jq % S) * Lay::kStageBytes;
+              const uint32_t t_s = tmem + Lay::kColS + (uint32_t)((jq & 1) * kBN);
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk % 4) * 32;
+                const uint64_t da = smem_desc(q_addr + (kk / 4) * 16384 + off, 16, 1024, kSwizzle128B);
+                const uint64_t db = smem_desc(k_addr + (kk / 4) * Lay::kKVAtomBytes + off, 16, 1024, kSwizzle128B);
+                mma_bf16_ss(t_s, da, db, id_qk, kk > 0);
+              }
+              mma_commit(smem_u32(&bars->s_full[jq & 1]));
+              if (--q_rem == 0) mma_commit(smem_u32(&bars->q_empty[qb]));
+              ++jq;
+            }
           }
-          if (mbar_try_wait(pb, j & 1)) break;
+          if (mbar_try_wait(pb, (jp >> 1) & 1)) break;
           if ((it & 15u) == 15u) {
             if (*abort) { ok = false; break; }
             const uint64_t now = globaltimer();
-            if (t0 == 0) t0 = now;
-            else if (now - t0 > 2000000000ull) { *abort = 1; ok = false; break; }
+            if (tw == 0) tw = now;
+            else if (now - tw > 2000000000ull) { *abort = 1; ok = false; break; }
           }
         }
         if (!ok) break;
         tc_fence_after();
-        const int st = j % kStages;
+        const int st = jp % S;
+        const uint32_t p_addr = s_base + Lay::kPOff + (jp & 1) * Lay::kPBytes;
         const uint32_t v_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes + Lay::kKBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint64_t da = smem_desc(p_addr + kk * 32, 16, 1024, kSwizzle128B);
           const uint64_t db = smem_desc(v_addr + kk * 2048, Lay::kKVAtomBytes, 1024, kSwizzle128B);
-          mma_bf16_ss(t_o, da, db, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ss(t_o, da, db, id_pv, (!first || kk > 0) ? 1u : 0u);
         }
         mma_commit(smem_u32(&bars->empty[st]));
-        mma_commit(smem_u32(&bars->pv_done));
+        mma_commit(smem_u32(&bars->pv_done[jp & 1]));
+        --p_rem;
       }
       // every MMA this thread issued has finished before TMEM is released
       mma_commit(smem_u32(&bars->mma_idle));
@@ -309,168 +531,283 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t t_s = tmem + lane_base + Lay::kColS;
     const uint32_t t_o = tmem + lane_base + Lay::kColO;
-    // a warp whose 32 rows are all padding only keeps the barrier protocol going
-    const bool warp_live = row0 + quad * 32 < rows;
-    const int qpos = (row_ok && p.window > 0) ? p.pos[(size_t)b * p.n + qi] : 0;
-    const int win_lo = qpos - p.window + 1;
-    uint64_t mw0 = 0, mw1 = 0;
-    if (row_ok && tree) {
-      mw0 = p.mask[((size_t)b * p.n + qi) * 2];
-      mw1 = p.mask[((size_t)b * p.n + qi) * 2 + 1];
-    }
     const float sl2 = p.scale_log2;
+    Piece pc = spc;
+    RowCtx rc = src;
+    bool have = s_have;
+    int jg = 0;
     bool ok = true;
-    unsigned char* prow = smem + Lay::kPOff + r_local * 128;
-    for (int j = 0; j < ntiles && ok; ++j) {
-      if (!warp_live) break;  // padding rows: nothing to compute, nothing to signal
-      if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, abort))) { ok = false; break; }
-      tc_fence_after();
-      float x[kBN];
-      tmem_ld32(t_s + (uint32_t)((j & 1) * kBN), x);
-      tmem_ld32(t_s + (uint32_t)((j & 1) * kBN + 32), x + 32);
-      tmem_wait_ld();
-      const int key0 = k0 + j * kBN;
-      float mx = -INFINITY;
-      if (tree || p.window > 0 || key0 + kBN > k1) {  // edge tiles: per-key visibility
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          const int kidx = key0 + c;
-          bool vis = row_ok && kidx < k1;
-          if (vis && tree) {
-            vis = ((kidx < 64 ? mw0 >> kidx : mw1 >> (kidx - 64)) & 1ull) != 0;
-            if (vis && p.window > 0) vis = p.pos[(size_t)b * p.n + kidx] >= win_lo;
-          } else if (vis && p.window > 0) {
-            vis = kidx >= win_lo;
-          }
-          x[c] = vis ? x[c] : -INFINITY;
-          mx = fmaxf(mx, x[c]);
+    while (ok && have) {
+      Piece pn;
+      RowCtx rn;
+      const bool have_next = scur.next(a, pn);
+      if (have_next) row_issue(rn, pn, p, r_local, lane, G);  // in flight during this piece
+      const int g = pc.hr / a.RG, rg = pc.hr % a.RG;
+      const int row0 = rg * kRowsPerCta;
+      const int r_glob = row0 + r_local;
+      const bool row_ok = r_glob < rows;
+      const bool warp_live = row0 + quad * 32 < rows;  // a warp of padding rows only keeps the protocol
+      const int qi = row_ok ? r_glob / G : 0;
+      const int qh = row_ok ? g * G + r_glob % G : 0;
+      const int win_lo = rc.qpos - a.window + 1;
+      float m_used = -INFINITY, l = 0.f;  // reference max (scaled, log2) and row sum
+      for (int t = pc.tb; t < pc.te; ++t, ++jg) {
+        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[jg & 1]), (jg >> 1) & 1, abort))) {
+          ok = false;
+          break;
         }
-      } else {  // interior prefix tile: every key visible
+        if (warp_live) {
+          tc_fence_after();
+          float x[kBN];
+          tmem_ld32(t_s + (uint32_t)((jg & 1) * kBN), x);
+          tmem_ld32(t_s + (uint32_t)((jg & 1) * kBN + 32), x + 32);
+          tmem_wait_ld();
+          const bool tree = t >= pc.ptiles;
+          const int key0 = tree ? (t - pc.ptiles) * kBN : pc.lo + t * kBN;
+          const int k1 = tree ? a.n : pc.L;
+          float mx = -INFINITY;
+          if (tree) {  // tree keys: the row's ancestor bitmask (and the window on their positions)
+            const bool hi = key0 >= 64;
+            const uint64_t mw = row_ok ? (hi ? rc.mw1 : rc.mw0) : 0ull;
+            const int tp0 = hi ? rc.tpos[2] : rc.tpos[0], tp1 = hi ? rc.tpos[3] : rc.tpos[1];
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, x[c]);
+            for (int cc = 0; cc < kBN; ++cc) {
+              bool vis = key0 + cc < k1 && ((mw >> cc) & 1ull) != 0;
+              if (a.window > 0) {  // warp-uniform branch; every lane takes part in the shuffle
+                const int kpos = __shfl_sync(kFull, cc < 32 ? tp0 : tp1, cc & 31);
+                vis = vis && kpos >= win_lo;
+              }
+              x[cc] = vis ? x[cc] : -INFINITY;
+              mx = fmaxf(mx, x[cc]);
+            }
+          } else if (a.window > 0 || key0 + kBN > k1) {  // edge prefix tiles: per-key visibility
+#pragma unroll
+            for (int cc = 0; cc < kBN; ++cc) {
+              const int kidx = key0 + cc;
+              const bool vis = row_ok && kidx < k1 && (a.window == 0 || kidx >= win_lo);
+              x[cc] = vis ? x[cc] : -INFINITY;
+              mx = fmaxf(mx, x[cc]);
+            }
+          } else {  // interior prefix tile: every key visible
+#pragma unroll
+            for (int cc = 0; cc < kBN; ++cc) mx = fmaxf(mx, x[cc]);
+          }
+          mx *= sl2;  // scale > 0 keeps the order
+          // P buffer (jg & 1) was last read by PV(jg - 2)
+          if (jg >= 2 &&
+              !__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[jg & 1]), ((jg - 2) >> 1) & 1, abort))) {
+            ok = false;
+            break;
+          }
+          const bool rebase = mx > m_used + 8.f;
+          if (__any_sync(kFull, rebase && t > pc.tb && l > 0.f)) {
+            // O may only be rescaled once PV(jg - 1) has finished accumulating
+            if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[(jg - 1) & 1]), ((jg - 1) >> 1) & 1, abort))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const float f = (rebase && l > 0.f) ? ex2(m_used - mx) : 1.f;
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              float o[32];
+              tmem_ld32(t_o + c0, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int u = 0; u < 32; ++u) o[u] *= f;
+              tmem_st32(t_o + c0, o);
+            }
+            tmem_wait_st();
+            l *= f;
+          }
+          if (rebase) m_used = mx;
+          const float neg_m = m_used > -INFINITY ? -m_used : 0.f;  // no visible key yet: every x is -inf
+          unsigned char* prow = smem + Lay::kPOff + (jg & 1) * Lay::kPBytes + r_local * 128;
+          float sum = 0.f;
+#pragma unroll
+          for (int c8 = 0; c8 < kBN / 8; ++c8) {
+            uint32_t packed[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float e0 = ex2(fmaf(x[c8 * 8 + 2 * u], sl2, neg_m));
+              const float e1 = ex2(fmaf(x[c8 * 8 + 2 * u + 1], sl2, neg_m));
+              sum += e0 + e1;
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+              packed[u] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            *reinterpret_cast<uint4*>(prow + ((c8 ^ (r_local & 7)) << 4)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          }
+          l += sum;
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->p_full[jg & 1]));
       }
-      mx *= sl2;  // scale > 0 keeps the order
-      // PV(j-1) must be complete before P is overwritten or O is rescaled
-      if (j > 0) {
-        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (j - 1) & 1, abort))) { ok = false; break; }
+      if (!ok) break;
+      // ---- end of the piece: normalised O -> bf16 output, or partial + lse
+      if (warp_live) {
+        const int jl = jg - 1;
+        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[jl & 1]), (jl >> 1) & 1, abort))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-      }
-      const bool rebase = mx > m_used + 8.f;
-      if (__any_sync(kFull, rebase && j > 0 && l > 0.f)) {
-        const float f = (rebase && l > 0.f) ? ex2(m_used - mx) : 1.f;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const size_t slot = (size_t)c + (size_t)pc.b * HR + pc.hr;
         for (int c0 = 0; c0 < D; c0 += 32) {
           float o[32];
           tmem_ld32(t_o + c0, o);
           tmem_wait_ld();
+          if (!row_ok) continue;
+          if (pc.whole) {
+            __nv_bfloat16* dst = p.out + (((size_t)pc.b * a.n + qi) * p.Hq + qh) * D + c0;
 #pragma unroll
-          for (int t = 0; t < 32; ++t) o[t] *= f;
-          tmem_st32(t_o + c0, o);
+            for (int u = 0; u < 4; ++u) {
+              uint32_t w[4];
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[u * 8 + 2 * v] * inv, o[u * 8 + 2 * v + 1] * inv);
+                w[v] = *reinterpret_cast<const uint32_t*>(&h2);
+              }
+              *reinterpret_cast<uint4*>(dst + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+            float* dst = p.part_o + (slot * kRowsPerCta + r_local) * D + c0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<float4*>(dst + 4 * u) =
+                  make_float4(o[4 * u] * inv, o[4 * u + 1] * inv, o[4 * u + 2] * inv, o[4 * u + 3] * inv);
+          }
         }
-        tmem_wait_st();
-        l *= f;
+        if (row_ok && !pc.whole)
+          p.part_lse[slot * kRowsPerCta + r_local] = l > 0.f ? (m_used + __log2f(l)) * (float)kLn2 : -INFINITY;
+        tc_fence_before();
       }
-      if (rebase) m_used = mx;
-      const float neg_m = m_used > -INFINITY ? -m_used : 0.f;  // no visible key yet: every x is -inf
-      float sum = 0.f;
-#pragma unroll
-      for (int c8 = 0; c8 < kBN / 8; ++c8) {
-        uint32_t packed[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float a = ex2(fmaf(x[c8 * 8 + 2 * t], sl2, neg_m));
-          const float bb = ex2(fmaf(x[c8 * 8 + 2 * t + 1], sl2, neg_m));
-          sum += a + bb;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
-          packed[t] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r_local & 7)) << 4)) =
-            make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      }
-      l += sum;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&bars->p_full));
+      pc = pn;
+      rc = rn;
+      have = have_next;
     }
-    final_ok = ok && warp_live &&
-               __all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done), (ntiles - 1) & 1, abort));
   }
-  }  // work
 
-  // ---- park this split's normalised partial (O rows, log-sum-exp) in shared
-  // memory: the K/V stages hold O (row r: D floats, 16-byte chunks XOR-swizzled
-  // by r), the P buffer holds the 128 log-sum-exps.  All TMA copies and MMAs of
-  // this CTA have drained before the barrier below.
-  float* o_part = reinterpret_cast<float*>(smem + Lay::kStageOff);
-  float* lse_part = reinterpret_cast<float*>(smem + Lay::kPOff);
-  constexpr int kChunks = D / 4;  // 16-byte chunks per O row
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp >= 2) {
-    float lse_r = -INFINITY;
-    if (final_ok) {  // warp-uniform
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const uint32_t t_o = tmem + ((uint32_t)(quad * 32) << 16) + Lay::kColO;
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float o[32];
-        tmem_ld32(t_o + c0, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int c = (c0 >> 2) + t;
-          *reinterpret_cast<float4*>(o_part + r_local * D + ((c ^ (r_local & (kChunks - 1))) << 2)) =
-              make_float4(o[4 * t] * inv, o[4 * t + 1] * inv, o[4 * t + 2] * inv, o[4 * t + 3] * inv);
-        }
-      }
-      if (row_ok && l > 0.f) lse_r = (m_used + __log2f(l)) * (float)kLn2;
-    }
-    lse_part[r_local] = lse_r;
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (work && *abort && tid == 0) atomicExch(p.err, 1);
-  if (work && warp == 0) tmem_dealloc(tmem, Lay::kTmemCols);
+  if (warp == 0) tmem_dealloc(tmem, Lay::kTmemCols);
+  if (tid == 0) p.cta_status[c] = bars->abort ? 1 : 0;
+}
 
-  // ---- combine the splits of this (sequence, KV head, row group) across the
-  // cluster: rank cr reduces a slice of the rows, reading every split's
-  // partial through distributed shared memory, and writes bf16 output
-  //   out = sum_s e^{lse_s - M} O_s / sum_s e^{lse_s - M}
-  cluster.sync();
-  {
-    const int CS = (int)cluster.num_blocks(), cr = (int)cluster.block_rank();
-    const int valid = min(kRowsPerCta, rows - row0);
-    const int per = (valid + CS - 1) / CS;
-    const int r_end = min(valid, (cr + 1) * per);
-    constexpr int DPL = D / 32;  // output dims per lane
-    for (int r = cr * per + warp; r < r_end; r += kTcThreads / 32) {
-      const float ls = lane < CS ? *cluster.map_shared_rank(lse_part + r, lane) : -INFINITY;
-      const float M = warp_max_f(ls);
-      const float w = (lane < CS && ls > -INFINITY) ? __expf(ls - M) : 0.f;
-      const float wsum = warp_sum_f(w);
-      float acc[DPL];
-#pragma unroll
-      for (int t = 0; t < DPL; ++t) acc[t] = 0.f;
-      const int c = (lane * DPL) >> 2;  // this lane's 16-byte chunk
-      const int within = (lane * DPL) & 3;
-      const int off = r * D + ((c ^ (r & (kChunks - 1))) << 2) + within;
-      for (int sp = 0; sp < CS; ++sp) {
-        const float ws = __shfl_sync(kFull, w, sp);
-        if (ws == 0.f) continue;
-        const float* src = cluster.map_shared_rank(o_part, sp) + off;
-#pragma unroll
-        for (int t = 0; t < DPL; ++t) acc[t] = fmaf(ws, src[t], acc[t]);
-      }
-      const int rg_row = row0 + r;
-      const int i = rg_row / G, h = g * G + rg_row % G;
-      __nv_bfloat16* dst = p.out + (((size_t)b * p.n + i) * p.Hq + h) * D + lane * DPL;
-      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-#pragma unroll
-      for (int t = 0; t < DPL; t += 2)
-        *reinterpret_cast<__nv_bfloat162*>(dst + t) = __floats2bfloat162_rn(acc[t] * inv, acc[t + 1] * inv);
+// Merge the pieces of every unit cut by CTA range boundaries:
+//   out = sum_s e^{lse_s - M} O_s / sum_s e^{lse_s - M}
+// One warp per query row (blockIdx.x = unit, blockIdx.y = group of 4 rows);
+// each lane loads its D/32 dims of every piece's partial in one round of
+// independent L2 reads, up to kCombChunk pieces at a time, merged online.
+// A unit finished inside one CTA is skipped.  Block (0, 0) also folds the
+// per-CTA status words into the workspace header.
+constexpr int kCombineWarps = kCombineThreads / 32;
+constexpr int kCombChunk = 8;
+
+struct CombParams {
+  const float* part_o;
+  const float* part_lse;
+  const int* cta_status;
+  int* status;
+  __nv_bfloat16* out;
+  AttnGeom geo;
+  int Hq;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads)
+attn_combine_kernel(const CombParams p) {
+  const AttnGeom& a = p.geo;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int HR = a.Hkv * a.RG;
+  const int u = blockIdx.x, b = u / HR, hr = u % HR;
+  const int g = hr / a.RG, rg = hr % a.RG;
+  const int G = p.Hq / a.Hkv;
+  __shared__ long long s_T, s_start;
+  __shared__ int s_tiles, s_stat[kCombineWarps];
+  if (warp == 0) {  // the schedule depends only on prefix_len, not on the attention kernel
+    const long long T = geom_prefix(a, a.B, lane);
+    const long long cum = geom_prefix(a, b, lane);
+    const int tiles = geom_tiles(a, b);
+    if (lane == 0) {
+      s_T = T;
+      s_start = cum + (long long)hr * tiles;
+      s_tiles = tiles;
     }
   }
-  cluster.sync();  // no CTA leaves while another may still read its shared memory
+  __syncthreads();
+  griddep_wait();
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    int st = 0;
+    for (int i = tid; i < a.C; i += kCombineThreads) st = max(st, p.cta_status[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) st = max(st, __shfl_xor_sync(kFull, st, o));
+    if (lane == 0) s_stat[warp] = st;
+    __syncthreads();
+    if (tid == 0) {
+      for (int w = 0; w < kCombineWarps; ++w) st = max(st, s_stat[w]);
+      *p.status = st;
+    }
+  }
+  const long long T = s_T, start = s_start;
+  const int c_first = cta_of_tile(start, T, a.C);
+  const int c_last = cta_of_tile(start + s_tiles - 1, T, a.C);
+  const int r = blockIdx.y * kCombineWarps + warp;
+  const int valid = min(kRowsPerCta, a.n * G - rg * kRowsPerCta);
+  if (c_first == c_last || r >= valid) return;
+  const int nseg = c_last - c_first + 1;
+  const size_t slot0 = (size_t)c_first + u;
+  constexpr int DPL = D / 32;  // output dims per lane
+  float M = -INFINITY, wsum = 0.f;
+  float acc[DPL];
+#pragma unroll
+  for (int t = 0; t < DPL; ++t) acc[t] = 0.f;
+  for (int s0 = 0; s0 < nseg; s0 += kCombChunk) {
+    float ls[kCombChunk];
+    float v[kCombChunk][DPL];
+#pragma unroll
+    for (int j = 0; j < kCombChunk; ++j) {
+      // a CTA with an empty range wrote no partial: read the first piece's
+      // (always written, finite) and give it weight 0
+      const int s = s0 + j;
+      const bool live = s < nseg && cta_nonempty(c_first + s, T, a.C);
+      const size_t sl = live ? slot0 + s : slot0;
+      ls[j] = live ? __ldcg(p.part_lse + sl * kRowsPerCta + r) : -INFINITY;
+      const float* src = p.part_o + (sl * kRowsPerCta + r) * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(src));
+        v[j][0] = f.x; v[j][1] = f.y; v[j][2] = f.z; v[j][3] = f.w;
+      } else {
+        const float2 f = __ldcg(reinterpret_cast<const float2*>(src));
+        v[j][0] = f.x; v[j][1] = f.y;
+      }
+    }
+    float mc = M;
+#pragma unroll
+    for (int j = 0; j < kCombChunk; ++j) mc = fmaxf(mc, ls[j]);
+    if (mc == -INFINITY) continue;
+    const float f = M > -INFINITY ? __expf(M - mc) : 0.f;
+    wsum *= f;
+#pragma unroll
+    for (int t = 0; t < DPL; ++t) acc[t] *= f;
+#pragma unroll
+    for (int j = 0; j < kCombChunk; ++j) {
+      const float w = ls[j] > -INFINITY ? __expf(ls[j] - mc) : 0.f;
+      wsum += w;
+#pragma unroll
+      for (int t = 0; t < DPL; ++t) acc[t] = fmaf(w, v[j][t], acc[t]);
+    }
+    M = mc;
+  }
+  const int row = rg * kRowsPerCta + r;
+  const int i = row / G, h = g * G + row % G;
+  __nv_bfloat16* dst = p.out + (((size_t)b * a.n + i) * p.Hq + h) * D + lane * DPL;
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int t = 0; t < DPL; t += 2)
+    *reinterpret_cast<__nv_bfloat162*>(dst + t) = __floats2bfloat162_rn(acc[t] * inv, acc[t + 1] * inv);
 }
 
 // ------------------------------------------------------------------- host
@@ -489,7 +826,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 tensor map with a 64-element x 64-row box and 128-byte swizzle.
+// bf16 tensor map with 128-byte swizzle (box given by the caller).
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
               const cuuint32_t* box) {
   auto fn = encode_fn();
@@ -503,16 +840,10 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
 
 }  // namespace
 
-int attention_row_groups(int n, int Hq, int Hkv) {
-  const int rows = n * (Hq / Hkv);
-  return (rows + kRowsPerCta - 1) / kRowsPerCta;
-}
-
 template <int D>
 static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
                              const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
-                             int n, int Hq, int Hkv, int window, float scale, const AttnPlan& plan, void* out,
-                             int* err, cudaStream_t s) {
+                             int n, int Hq, int Hkv, int window, float scale, void* out, void* ws, cudaStream_t s) {
   CUtensorMap mk, mv, mkt, mvt;
   const int Lrows = Lmax > 0 ? Lmax : 1;
   const void* kbase = Lmax > 0 ? kc : kt;  // any valid address when the cache is empty
@@ -542,57 +873,71 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
     const cuuint32_t box[3] = {64, (cuuint32_t)(q_tma ? G : 1), (cuuint32_t)(q_tma ? kRowsPerCta / G : 1)};
     if (!make_map(&mq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
+  const AttnWorkspace wl = attention_ws_layout(B, n, Hq, Hkv, D, Lmax, window);
+  unsigned char* wsb = static_cast<unsigned char*>(ws);
   TcParams p;
-  p.q_by_tma = q_tma ? 1 : 0;
   p.q = static_cast<const __nv_bfloat16*>(q);
-  p.plen = plen;
   p.mask = mask;
   p.pos = pos;
   p.out = static_cast<__nv_bfloat16*>(out);
-  p.err = err;
-  p.Lmax = Lmax;
-  p.n = n;
+  p.part_o = reinterpret_cast<float*>(wsb + wl.part_o_off);
+  p.part_lse = reinterpret_cast<float*>(wsb + wl.part_lse_off);
+  p.cta_status = reinterpret_cast<int*>(wsb + wl.cta_status_off);
+  p.geo.plen = plen;
+  p.geo.B = B;
+  p.geo.Hkv = Hkv;
+  p.geo.RG = attention_row_groups(n, Hq, Hkv);
+  p.geo.n = n;
+  p.geo.Lmax = Lmax;
+  p.geo.window = window;
+  p.geo.C = attention_ctas(B, n, Hq, Hkv, Lmax, window);
   p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.window = window;
-  p.n_splits = plan.n_splits;
-  p.chunk = plan.chunk;
-  p.row_groups = attention_row_groups(n, Hq, Hkv);
+  p.q_by_tma = q_tma ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = TcLayout<D>::kSmemBytes;
   cudaError_t e = ensure_smem_limit((const void*)attn_tc_kernel<D>, smem);
   if (e != cudaSuccess) return e;
-  const int cs = plan.n_splits + 1;  // one cluster = every split of one (sequence, KV head, row group)
-  if (cs > 8) {
-    static bool np_set[2] = {false, false};
-    if (!np_set[D == 128]) {
-      e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-      np_set[D == 128] = true;
-    }
-  }
+
+  // both kernels may start while their predecessor drains (programmatic
+  // dependent launch); each waits in griddep_wait before reading its inputs
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cs, Hkv, B * p.row_groups);
+  cfg.gridDim = dim3(p.geo.C);
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D>, mk, mv, mkt, mvt, mq, p);
+  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<D>, mk, mv, mkt, mvt, mq, p);
+  if (e != cudaSuccess) return e;
+
+  CombParams cp;
+  cp.part_o = p.part_o;
+  cp.part_lse = p.part_lse;
+  cp.cta_status = p.cta_status;
+  cp.status = reinterpret_cast<int*>(wsb + wl.status_off);
+  cp.out = p.out;
+  cp.geo = p.geo;
+  cp.Hq = Hq;
+  cudaLaunchConfig_t cfg2 = {};
+  cfg2.gridDim = dim3((unsigned)((size_t)B * Hkv * p.geo.RG), kRowsPerCta / kCombineWarps);
+  cfg2.blockDim = dim3(kCombineThreads);
+  cfg2.dynamicSmemBytes = 0;
+  cfg2.stream = s;
+  cfg2.attrs = attr;
+  cfg2.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg2, attn_combine_kernel<D>, cp);
 }
 
-cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
-                                const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
-                                int n, int Hq, int Hkv, int D, int window, float scale, const AttnPlan& plan,
-                                void* out, int* err, cudaStream_t s) {
+cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
+                                  const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
+                                  int n, int Hq, int Hkv, int D, int window, float scale, void* out, void* ws,
+                                  cudaStream_t s) {
   if (D == 128)
-    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, plan, out, err, s);
-  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, plan, out, err, s);
+    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s);
+  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s);
 }
 
 }  // namespace eagle

@@ -45,23 +45,27 @@ cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R,
 cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len,
                              int B, int n, uint64_t* mask, int32_t* pos, cudaStream_t s);
 
-// ---- attention (attention.cu, attention_tc.cu)
-struct AttnPlan {
-  int n_splits;   // prefix splits (one more CTA handles the tree keys); <= 15
-  int chunk;      // prefix keys per split (multiple of 64)
-  int span;       // prefix keys a sequence can see at most (Lmax, or the window)
+// ---- attention (attention.cu: workspace plan; attention_tc.cu: kernels)
+constexpr int kAttnRowsPerUnit = 128;  // query rows per unit (one MMA M)
+constexpr int kAttnKeysPerTile = 64;
+// Workspace of eagle_tree_attention, byte offsets from its (256-aligned) base.
+struct AttnWorkspace {
+  size_t status_off;      // int: the device status word (written by every launch)
+  size_t cta_status_off;  // int [C]: per-CTA status of the main kernel
+  size_t part_lse_off;    // float [C + U][128]: log-sum-exp of each partial
+  size_t part_o_off;      // float [C + U][128][D]: normalised partial outputs
+  size_t bytes;
 };
 int attention_row_groups(int n, int Hq, int Hkv);
-AttnPlan plan_attention(int B, int n, int Hq, int Hkv, int Lmax, int window);
-size_t attention_ws_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window);
+int attention_ctas(int B, int n, int Hq, int Hkv, int Lmax, int window);  // C
+AttnWorkspace attention_ws_layout(int B, int n, int Hq, int Hkv, int D, int Lmax, int window);
+inline size_t attention_ws_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window) {
+  return attention_ws_layout(B, n, Hq, Hkv, D, Lmax, window).bytes;
+}
 cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen,
                                   int Lmax, const void* kt, const void* vt, const uint64_t* mask,
                                   const int32_t* pos, int B, int n, int Hq, int Hkv, int D, int window,
                                   float scale, void* out, void* ws, cudaStream_t s);
-cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
-                                const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
-                                int n, int Hq, int Hkv, int D, int window, float scale, const AttnPlan& plan,
-                                void* out, int* err, cudaStream_t s);
 
 // ---- accept (accept.cu)
 size_t accept_ws_bytes(int B, int n, int V, int dtype);

@@ -44,6 +44,17 @@ struct BuildSmem {
   int* node_of;      // [P]   kept flag, then 1-based node id (0 = dropped)
   int* frontier;     // [32]
   int* warp_cnt;     // [kBuildWarps]
+  int* node_par;     // [EAGLE_MAX_NODES] parent node id of node i+1 (mask fusion)
+  int* node_dep;     // [EAGLE_MAX_NODES]
+};
+
+// Optional fused tree mask: with mask != nullptr the expansion kernel also
+// writes each node's ancestor-or-self bitmask and position id (what
+// eagle_tree_mask computes), saving a launch and a round trip of the tree.
+struct MaskOut {
+  const int32_t* prefix_len;  // [B]
+  uint64_t* mask;             // [B][n][2]
+  int32_t* pos;               // [B][n] (may be null)
 };
 
 __host__ __device__ inline int next_pow2(int x) {
@@ -56,7 +67,7 @@ __host__ __device__ inline int next_pow2(int x) {
 // row_lse: each row's log-sum-exp (also the tree's row_lse output).
 __global__ void __launch_bounds__(kBuildThreads)
 tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restrict__ row_val_g, int R, int depth,
-                   int k, int n, eagle_tree_t out) {
+                   int k, int n, eagle_tree_t out, MaskOut mo) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -77,7 +88,9 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     sm.cand_row = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
     sm.node_of = reinterpret_cast<int*>(p);      p += sizeof(int) * P;
     sm.frontier = reinterpret_cast<int*>(p);     p += sizeof(int) * 32;
-    sm.warp_cnt = reinterpret_cast<int*>(p);
+    sm.warp_cnt = reinterpret_cast<int*>(p);    p += sizeof(int) * kBuildWarps;
+    sm.node_par = reinterpret_cast<int*>(p);     p += sizeof(int) * EAGLE_MAX_NODES;
+    sm.node_dep = reinterpret_cast<int*>(p);
   }
 
   // 1. each row's children and their log-confidence lp = logit - lse (fp64)
@@ -205,15 +218,33 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     out.logV[o] = (float)sm.cand_lv[g];
     if (out.gid) out.gid[o] = g;
     out.draft_row[(size_t)b * (n + 1) + node] = sm.cand_row[g];
+    sm.node_par[node - 1] = par < 0 ? 0 : sm.node_of[par];
+    sm.node_dep[node - 1] = g < k ? 1 : 2 + (g - k) / kk;
   }
   if (tid == 0) out.draft_row[(size_t)b * (n + 1)] = 0;
+  if (mo.mask == nullptr) return;
+  // 5. (fused mask) node i+1 sees itself and its ancestors: walk the parent chain
+  __syncthreads();
+  for (int i = tid; i < n; i += kBuildThreads) {
+    uint64_t w0 = 0, w1 = 0;
+    int node = i + 1;
+    for (int step = 0; step < n && node >= 1; ++step) {
+      const int j = node - 1;
+      if (j < 64) w0 |= 1ull << j; else w1 |= 1ull << (j - 64);
+      node = sm.node_par[j];
+    }
+    const size_t o = (size_t)b * n + i;
+    mo.mask[o * 2] = w0;
+    mo.mask[o * 2 + 1] = w1;
+    if (mo.pos) mo.pos[o] = mo.prefix_len[b] - 1 + sm.node_dep[i];
+  }
 }
 
 size_t tree_build_smem_bytes(int R, int k, int P) {
   const int Ppow = next_pow2(P);
   const int nsort = Ppow > 2 * kBuildThreads ? Ppow : 2 * kBuildThreads;
   return sizeof(double) * ((size_t)R * k + P) + sizeof(uint64_t) * nsort +
-         sizeof(int) * ((size_t)R * k + 4 * (size_t)P + 32 + kBuildWarps);
+         sizeof(int) * ((size_t)R * k + 4 * (size_t)P + 32 + kBuildWarps + 2 * EAGLE_MAX_NODES);
 }
 
 // workspace: [chunk stats][chunk keys][row tokens B*R*k int32][row logits B*R*k float]
@@ -238,7 +269,8 @@ cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R,
   const size_t smem = tree_build_smem_bytes(R, k, P);
   e = ensure_smem_limit((const void*)tree_expand_kernel, smem);
   if (e != cudaSuccess) return e;
-  tree_expand_kernel<<<B, kBuildThreads, smem, s>>>(ro.tok, ro.val, R, depth, k, n, out);
+  MaskOut mo = {nullptr, nullptr, nullptr};
+  tree_expand_kernel<<<B, kBuildThreads, smem, s>>>(ro.tok, ro.val, R, depth, k, n, out, mo);
   return cudaGetLastError();
 }
 

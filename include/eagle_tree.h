@@ -174,9 +174,13 @@ EAGLE_API eagle_status eagle_tree_mask(const int32_t* parents, const int32_t* de
  *   out      [B][n][Hq][D]     bf16
  *   scale    softmax scale; <= 0 selects 1/sqrt(D)
  * Limits: D in {64, 128}, Hq % Hkv == 0, n <= EAGLE_MAX_NODES, all tensor
- * pointers 16-byte aligned.  Workspace: eagle_tree_attention_workspace_bytes
- * (a 256-byte header with the kernel's device status word: 0 = ok, 1 = an
- * internal wait gave up, 2 = misaligned shared memory). */
+ * pointers 16-byte aligned.  Workspace: eagle_tree_attention_workspace_bytes.
+ * It starts with a 256-byte header whose first int is the device status word,
+ * rewritten by every call (0 = ok, 1 = an internal wait gave up); the rest holds
+ * the normalised partial outputs of key ranges split across CTAs (fp32, about
+ * (148 + B*Hkv*ceil(n*Hq/Hkv/128)) * 128 * (D+1) * 4 bytes).  The call launches
+ * two kernels; either may start while its predecessor on the stream drains
+ * (programmatic dependent launch) and waits for it before reading any input. */
 EAGLE_API size_t eagle_tree_attention_workspace_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window);
 EAGLE_API eagle_status eagle_tree_attention(const void* q, const void* k_cache, const void* v_cache,
                                   const int32_t* prefix_len, int Lmax, const void* k_tree,
