@@ -70,33 +70,62 @@ struct Parity {
 };
 
 // This thread's slice [x0, x1) of the current rows, cached in shared memory.
+// Element i of thread t sits at [i * kAcceptThreads + t], so a warp reading
+// its threads' i-th elements touches consecutive words (no bank conflicts).
 template <typename T>
 struct Slice {
+  static constexpr int kVec = 16 / (int)sizeof(T);              // elements per 16-byte load
+  static constexpr int kMaxLoads = slice_max<T>() / kVec;       // 16-byte loads per full slice
   T* tc;  // target row slice
   T* dc;  // draft row slice
   int x0, x1;
+  int slice;    // elements per full slice (a multiple of kVec)
+  bool vec_ok;  // rows 16-byte aligned: full slices load as 16-byte vectors
   int cached_t, cached_d;
 
-  __device__ void load(const T* src, T* dst) const {
-    constexpr int kChunk = 8;
-    for (int b = x0; b < x1; b += kChunk) {
-      T v[kChunk];
+  __device__ __forceinline__ T& at(T* base, int i) const { return base[(size_t)i * kAcceptThreads + threadIdx.x]; }
+
+  // Copy the slices of up to two rows (src may be null), all loads in flight first.
+  __device__ void load2(const T* s0, T* d0, const T* s1, T* d1) const {
+    const int len = x1 - x0;
+    if (vec_ok && len == slice) {
+      uint4 v0[kMaxLoads], v1[kMaxLoads];
 #pragma unroll
-      for (int i = 0; i < kChunk; ++i)
-        if (b + i < x1) v[i] = src[b + i];
+      for (int q = 0; q < kMaxLoads; ++q) {
+        if (q * kVec < len) {
+          if (s0) v0[q] = __ldg(reinterpret_cast<const uint4*>(s0 + x0) + q);
+          if (s1) v1[q] = __ldg(reinterpret_cast<const uint4*>(s1 + x0) + q);
+        }
+      }
 #pragma unroll
-      for (int i = 0; i < kChunk; ++i)
-        if (b + i < x1) dst[b - x0 + i] = v[i];
+      for (int q = 0; q < kMaxLoads; ++q) {
+        if (q * kVec < len) {
+          const T* e0 = reinterpret_cast<const T*>(&v0[q]);
+          const T* e1 = reinterpret_cast<const T*>(&v1[q]);
+#pragma unroll
+          for (int e = 0; e < kVec; ++e) {
+            if (s0) at(d0, q * kVec + e) = e0[e];
+            if (s1) at(d1, q * kVec + e) = e1[e];
+          }
+        }
+      }
+    } else {
+      for (int i = 0; i < len; ++i) {
+        if (s0) at(d0, i) = s0[x0 + i];
+        if (s1) at(d1, i) = s1[x0 + i];
+      }
     }
   }
   __device__ void ensure(const T* trow, int tkey, const T* drow, int dkey) {
-    if (cached_t != tkey) { load(trow, tc); cached_t = tkey; }
-    if (drow && cached_d != dkey) { load(drow, dc); cached_d = dkey; }
+    const bool lt = cached_t != tkey, ld = drow && cached_d != dkey;
+    if (lt || ld) load2(lt ? trow : nullptr, tc, ld ? drow : nullptr, dc);
+    if (lt) cached_t = tkey;
+    if (ld) cached_d = dkey;
   }
   __device__ __forceinline__ float weight(const SweepArgs& a, int i) const {
-    const float p = exp_minus(to_f(tc[i]), a.lse_t);
+    const float p = exp_minus(to_f(at(tc, i)), a.lse_t);
     if (!a.use_q) return p;
-    const float q = exp_minus(to_f(dc[i]), a.lse_d);
+    const float q = exp_minus(to_f(at(dc, i)), a.lse_d);
     return fmaxf(0.f, fmaf(-a.t.lo, q, fmaf(-a.t.hi, q, p)));
   }
 };
@@ -117,19 +146,23 @@ __device__ double block_sum(double v, AcceptSmem& sm, int& parity) {
 }
 
 // Cluster-wide total of one double per CTA, summed in rank order (bit-identical
-// in every CTA).  One cluster barrier per call: the slots alternate between
-// calls; a CTA rewrites a slot only after the next call's barrier, which every
-// CTA reaches only after reading that slot.
+// in every CTA).  Each warp reads the ranks' values once (lane r from rank r)
+// and every thread adds them in rank order from registers.  One cluster barrier
+// per call: the slots alternate between calls; a CTA rewrites a slot only after
+// the next call's barrier, which every CTA reaches only after reading that slot.
 __device__ double cluster_sum(double cta_value, AcceptSmem& sm, cg::cluster_group& cluster,
                               double* prefix_of_rank, int& parity) {
   if (threadIdx.x == 0) sm.cta_total[parity] = cta_value;
   cluster.sync();
   const unsigned nb = cluster.num_blocks();
   const unsigned me = cluster.block_rank();
+  const unsigned lane = threadIdx.x & 31;
+  const double v_lane = lane < nb ? *cluster.map_shared_rank(&sm.cta_total[parity], lane) : 0.0;
   double acc = 0.0;
   for (unsigned r = 0; r < nb; ++r) {
+    const double v = __shfl_sync(kFull, v_lane, r);
     if (r == me && prefix_of_rank) *prefix_of_rank = acc;
-    acc += *cluster.map_shared_rank(&sm.cta_total[parity], r);
+    acc += v;
   }
   parity ^= 1;
   return acc;
@@ -206,7 +239,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
                    const double* __restrict__ row_lse, const int32_t* __restrict__ tokens,
                    const int32_t* __restrict__ parents, const int32_t* __restrict__ draft_row,
                    const float* __restrict__ uniforms, int32_t* __restrict__ accepted_len,
-                   int32_t* __restrict__ path, int32_t* __restrict__ bonus, int slice) {
+                   int32_t* __restrict__ path, int32_t* __restrict__ bonus, int slice, bool vec_ok) {
   __shared__ AcceptSmem sm;
   extern __shared__ __align__(16) unsigned char cache_raw[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -255,9 +288,11 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     const int gt = (int)cluster.block_rank() * kAcceptThreads + tid;
     sl.x0 = min(V, gt * slice);
     sl.x1 = min(V, sl.x0 + slice);
+    sl.slice = slice;
+    sl.vec_ok = vec_ok;
     T* base = reinterpret_cast<T*>(cache_raw);
-    sl.tc = base + (size_t)tid * slice;
-    sl.dc = base + (size_t)(kAcceptThreads + tid) * slice;
+    sl.tc = base;
+    sl.dc = base + (size_t)kAcceptThreads * slice;
     sl.cached_t = -1;
     sl.cached_d = -1;
   }
@@ -360,11 +395,14 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
                                int32_t* bonus, cudaStream_t s) {
   int cl = 1, slice = 0;
   size_t dyn = 0;
+  const bool vec_ok = (((uintptr_t)tgt | (uintptr_t)dft) % 16 == 0) && ((size_t)V * sizeof(T)) % 16 == 0;
   if (STOCH) {
     const int per_cta = kAcceptThreads * slice_max<T>();
     cl = (V + per_cta - 1) / per_cta;
     if (cl < 1) cl = 1;
     slice = (V + cl * kAcceptThreads - 1) / (cl * kAcceptThreads);
+    constexpr int kVec = 16 / (int)sizeof(T);
+    slice = (slice + kVec - 1) / kVec * kVec;  // <= slice_max, itself a multiple of kVec
     dyn = (size_t)2 * kAcceptThreads * slice * sizeof(T);
     cudaError_t e = ensure_smem_limit((const void*)accept_walk_kernel<T, STOCH>, dyn + sizeof(AcceptSmem));
     if (e != cudaSuccess) return e;
@@ -391,7 +429,7 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, accept_walk_kernel<T, STOCH>, static_cast<const T*>(tgt),
                             static_cast<const T*>(dft), dlse, R, V, n, depth, row_amax, row_lse, tokens,
-                            parents, draft_row, uniforms, acc_len, path, bonus, slice);
+                            parents, draft_row, uniforms, acc_len, path, bonus, slice, vec_ok);
 }
 
 cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,

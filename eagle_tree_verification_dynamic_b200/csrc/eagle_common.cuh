@@ -102,10 +102,19 @@ struct ChunkStat {
   double acc;
 };
 
+// 2^z by the hardware approximation (about 2 ulp; results below 2^-126 flush
+// to zero).  Every sum built from it is dominated by terms near 2^0, so a
+// flushed term is far below the fp64 rounding of the sum.
+__device__ __forceinline__ float ex2_ftz(float z) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(z));
+  return y;
+}
+
 __device__ __forceinline__ float exp2_scaled(float x, float e_ref) {
   float z = fmaf(x, kLog2eHi, -e_ref);
   z = fmaf(x, kLog2eLo, z);
-  return exp2f(z);
+  return ex2_ftz(z);
 }
 
 // acc * 2^(from - to) for integer-valued from <= to (exact).
@@ -143,7 +152,7 @@ struct Split2 {
 // subtraction and the base change carried to ~fp32 accuracy of the result.
 __device__ __forceinline__ float exp_minus(float x, Split2 lse) {
   float d = (x - lse.hi) - lse.lo;
-  return exp2f(fmaf(d, kLog2eHi, d * kLog2eLo));
+  return ex2_ftz(fmaf(d, kLog2eHi, d * kLog2eLo));
 }
 
 // ------------------------------------------------------------------ loading
