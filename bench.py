@@ -38,7 +38,12 @@ from workloads import make_target_logits  # noqa: E402
 L2_BYTES = 126 * 2 ** 20
 METRIC = ("tree-verify steps/sec (and achieved KV HBM GB/s of the tree attention) at the 7B shape, "
           "prefix 2048, 60-node tree")
-LAUNCHES_PER_STEP = 7  # row sweep + expand, mask, attention split + combine, target sweep + walk
+LAUNCHES_PER_STEP = 7  # row sweep + expand, mask, attention main + combine, target sweep + walk
+
+# DRAM bytes (read + write) of one launch of the tree attention's main kernel,
+# from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of this
+# kernel version on the named workload; a workload without a capture reports null.
+ATTN_TRAFFIC_BYTES = {"7b": 35116288 + 768}
 
 
 def parse():
@@ -398,7 +403,7 @@ def main():
         "stages": stages,
         "roofline": {"kernel": "tree attention (split-KV + combine)", "bound": "hbm",
                      "achieved": round(attn_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(attn_gbs / hbm_peak, 4), "traffic": None,
+                     "frac": round(attn_gbs / hbm_peak, 4), "traffic": ATTN_TRAFFIC_BYTES.get(cfg.name),
                      "peak_source": f"{peak_src} copy bandwidth (burst)",
                      "algorithmic_bytes": sb["attention"]},
         "step_roofline": {"bytes": sb["step"], "t_min_us": round(sb["step"] / hbm_peak / 1e3, 3),
