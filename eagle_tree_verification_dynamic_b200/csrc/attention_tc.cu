@@ -15,18 +15,22 @@
 // unit cut by range boundaries leaves one normalised partial (O rows and
 // log-sum-exp) per piece, merged by attn_combine_kernel.
 //
-// Roles inside a CTA (192 threads):
+// Roles inside a CTA (320 threads):
 //   warp 0      producer: Q of each unit (TMA box, or a gather when G does not
 //               divide 128) into one of two Q buffers; K and V tiles into a
 //               ring of stages (128-byte swizzle, no multicast); TMEM owner
 //   warp 1      one thread issues tcgen05.mma: S = Q K^T into one of two TMEM
-//               S buffers, at most one tile ahead of PV; O += P V into TMEM
-//   warps 2-5   softmax: thread r owns TMEM lane r = query row r; applies the
-//               prefix range / window / tree bitmask, keeps a running reference
-//               max (re-based only when it grows by > 8 in log2 units, then O
-//               and the row sum are rescaled in TMEM), writes P = 2^(x - m) as
-//               bf16 into one of two swizzled P buffers; at the end of a unit's
-//               piece it normalises O and writes the output or the partial
+//               S buffers, at most one tile ahead of PV; O += P V into TMEM,
+//               each tile's keys 0..31 into O_A and keys 32..63 into O_B
+//   warps 2-9   softmax, two warps per TMEM lane quarter: thread r owns query
+//               row r, one warp the first 32 keys of every tile (and O_A), the
+//               other the last 32 (and O_B).  Each applies the prefix range /
+//               window / tree bitmask, keeps its own running reference max
+//               (re-based only when it grows by > 8 in log2 units, then its O
+//               and row sum are rescaled in TMEM) and writes P = 2^(x - m) as
+//               bf16 into one of two swizzled P buffers.  At the end of a
+//               unit's piece the pair exchanges (max, sum) through shared
+//               memory, merges O_A and O_B, and writes the output or partial
 //
 // Every mbarrier wait is bounded (about 2 s of wall time); a timeout sets an
 // abort flag that ends all roles, records a per-CTA status word and still
@@ -43,13 +47,16 @@ namespace eagle {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 192;   // 6 warps
+constexpr int kTcThreads = 320;   // 10 warps: producer, MMA, 8 softmax
 constexpr int kBN = kAttnKeysPerTile;
 constexpr int kRowsPerCta = kAttnRowsPerUnit;
 constexpr int kMaxStages = 8;
 constexpr int kSmemOptIn = 232448;  // largest dynamic shared memory a block may opt into on sm_100
 constexpr int kCombineThreads = 128;
 
+// Shared memory from the (1024-byte aligned) dynamic base: a 3 KB header
+// (barriers, then each row's (max, sum) exchange between the two softmax
+// warps of a lane quarter), two Q buffers, two P buffers, the K/V ring.
 template <int D>
 struct TcLayout {
   static constexpr int kAtoms = D / 64;               // 128-byte column atoms along D
@@ -58,20 +65,26 @@ struct TcLayout {
   static constexpr int kKVAtomBytes = kBN * 128;      // 64 keys x 128 B
   static constexpr int kKBytes = kAtoms * kKVAtomBytes;
   static constexpr int kStageBytes = 2 * kKBytes;     // K + V
-  static constexpr int kBarBytes = 512;
-  static constexpr int kFixed = 2 * kQBytes + 2 * kPBytes + kBarBytes + 1024;  // + base alignment slack
-  static constexpr int kStagesFit = (kSmemOptIn - kFixed) / kStageBytes;
-  static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
-  static constexpr int kQOff = 0;                      // two Q buffers
-  static constexpr int kPOff = 2 * kQBytes;            // two P buffers
+  static constexpr int kHdrBytes = 3072;
+  static constexpr int kBarOff = 0;
+  static constexpr int kXchOff = 512;                 // float2 [2 halves][128 rows]
+  static constexpr int kQOff = kHdrBytes;             // two Q buffers
+  static constexpr int kPOff = kQOff + 2 * kQBytes;   // two P buffers
   static constexpr int kStageOff = kPOff + 2 * kPBytes;
-  static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
-  static constexpr int kSmemBytes = kBarOff + kBarBytes + 1024;
-  static constexpr uint32_t kTmemCols = 256;  // S double buffer (2 x 64) + O (D <= 128)
-  static constexpr uint32_t kColS = 0;        // S buffer i at column 64 * i
-  static constexpr uint32_t kColO = 128;
+  static constexpr int kStagesFit = (kSmemOptIn - kStageOff) / kStageBytes;
+  static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
+  static constexpr int kSmemBytes = kStageOff + kStages * kStageBytes;
+  // TMEM: S double buffer (2 x 64 columns), then O over each tile's keys
+  // 0..31 (O_A) and over keys 32..63 (O_B): the two softmax warps of a lane
+  // quarter keep independent running maxima and are merged once per piece.
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0;  // S buffer i at column 64 * i
+  static constexpr uint32_t kColOA = 128;
+  static constexpr uint32_t kColOB = 128 + D;
   static_assert(kStages >= 2, "at least a double-buffered K/V ring");
   static_assert(kSmemBytes <= kSmemOptIn, "shared memory");
+  static_assert(kXchOff + 2 * 128 * 8 <= kHdrBytes, "header");
+  static_assert(kColOB + D <= kTmemCols, "TMEM");
 };
 
 struct TcBars {
@@ -83,13 +96,14 @@ struct TcBars {
   uint64_t p_full[2];
   uint64_t pv_done[2];
   uint64_t mma_idle;
+  uint64_t pair[4];  // per lane quarter: both softmax warps wrote their (max, sum)
   uint32_t tmem_base;
   int abort;
   // this CTA's tile range [t0, t1) of the global list, and where it starts
   int n_tiles;  // t1 - t0
   int b0, hr0, off0;
 };
-static_assert(sizeof(TcBars) <= 512, "barrier block");
+static_assert(sizeof(TcBars) <= 512, "barrier block");  // kXchOff
 
 // ----------------------------------------------------------- tile schedule
 struct AttnGeom {
@@ -111,7 +125,7 @@ __device__ __forceinline__ int geom_tiles(const AttnGeom& a, int b) {
 }
 
 // Whole warp: total tiles of all units, and the first tile of sequence b_end.
-__device__ long long geom_prefix(const AttnGeom& a, int b_end, int lane) {
+__device__ __forceinline__ long long geom_prefix(const AttnGeom& a, int b_end, int lane) {
   const int HR = a.Hkv * a.RG;
   long long acc = 0;
   for (int b = lane; b < b_end; b += 32) acc += (long long)HR * geom_tiles(a, b);
@@ -121,7 +135,8 @@ __device__ long long geom_prefix(const AttnGeom& a, int b_end, int lane) {
 }
 
 // Whole warp: the unit (b, hr) holding global tile t and t's offset in it.
-__device__ void geom_locate(const AttnGeom& a, long long t, int lane, int& b_out, int& hr_out, int& off_out) {
+__device__ __forceinline__ void geom_locate(const AttnGeom& a, long long t, int lane, int& b_out, int& hr_out,
+                                            int& off_out) {
   const int HR = a.Hkv * a.RG;
   long long base = 0;
   for (int bc = 0; bc < a.B; bc += 32) {
@@ -178,14 +193,14 @@ struct Piece {
 
 struct PieceCursor {
   int b, hr, off, left;
-  __device__ void init(int b0, int hr0, int off0, int n_tiles) {
+  __device__ __forceinline__ void init(int b0, int hr0, int off0, int n_tiles) {
     b = b0;
     hr = hr0;
     off = off0;
     left = n_tiles;
   }
-  __device__ void init(const TcBars* s) { init(s->b0, s->hr0, s->off0, s->n_tiles); }
-  __device__ bool next(const AttnGeom& a, Piece& pc) {
+  __device__ __forceinline__ void init(const TcBars* s) { init(s->b0, s->hr0, s->off0, s->n_tiles); }
+  __device__ __forceinline__ bool next(const AttnGeom& a, Piece& pc) {
     if (left <= 0) return false;
     const int HR = a.Hkv * a.RG;
     pc.b = b;
@@ -277,15 +292,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_q, const TcParams p) {
   using Lay = TcLayout<D>;
   constexpr int S = Lay::kStages;
-  extern __shared__ unsigned char smem_dyn[];
-  // the swizzled tiles need 1024-byte alignment
-  unsigned char* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
-  TcBars* bars = reinterpret_cast<TcBars*>(smem + Lay::kBarOff);
-  const uint32_t s_base = smem_u32(smem);
+  extern __shared__ __align__(1024) unsigned char smem[];
   const AttnGeom& a = p.geo;
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
+  // The layout fills the opt-in maximum and the swizzled tiles need a
+  // 1024-byte aligned base: with any other base the CTA does nothing and
+  // reports status 2 (the whole CTA leaves here, before any barrier).
+  if ((smem_u32(smem) & 1023u) != 0u) {
+    if (tid == 0) p.cta_status[c] = 2;
+    griddep_wait();
+    griddep_launch_dependents();
+    return;
+  }
+  TcBars* bars = reinterpret_cast<TcBars*>(smem + Lay::kBarOff);
+  const uint32_t s_base = smem_u32(smem);
   const int G = p.Hq / a.Hkv;
   const int rows = a.n * G;
   const int HR = a.Hkv * a.RG;
@@ -296,9 +317,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       mbar_init(smem_u32(&bars->q_full[i]), 1);
       mbar_init(smem_u32(&bars->q_empty[i]), 1);
       mbar_init(smem_u32(&bars->s_full[i]), 1);
-      // every softmax thread arrives for every tile, rows or not: a warp can
-      // run at most one tile ahead of P's consumer, and P is double-buffered
-      mbar_init(smem_u32(&bars->p_full[i]), 128);
+      // every softmax thread (8 warps) arrives for every tile, rows or not: a
+      // warp can run at most one tile ahead of P's consumer, and P is
+      // double-buffered
+      mbar_init(smem_u32(&bars->p_full[i]), 256);
       mbar_init(smem_u32(&bars->pv_done[i]), 1);
     }
     for (int i = 0; i < S; ++i) {
@@ -306,6 +328,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       mbar_init(smem_u32(&bars->empty[i]), 1);
     }
     mbar_init(smem_u32(&bars->mma_idle), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars->pair[i]), 64);
     bars->abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_k);
@@ -342,7 +365,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     if (warp >= 2) {
       scur.init(b0, hr0, off0, (int)(t1 - t0));
       s_have = scur.next(a, spc);
-      if (s_have) row_issue(src, spc, p, r_local, lane, G);
+      if (s_have) {
+        row_issue(src, spc, p, r_local, lane, G);
+        // wait for them here: issued together with the K/V stream they would
+        // queue behind it (a CTA whose range starts at a tree tile stalled
+        // for microseconds on its mask words)
+        uint64_t sink = src.mw0 ^ src.mw1 ^
+                        (uint64_t)(uint32_t)(src.qpos ^ src.tpos[0] ^ src.tpos[1] ^ src.tpos[2] ^ src.tpos[3]);
+        asm volatile("mov.b64 %0, %0;" : "+l"(sink));  // consumes every loaded value
+      }
     }
   }
   griddep_launch_dependents();
@@ -454,7 +485,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(128, kBN, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t t_o = tmem + Lay::kColO;
+      const uint32_t t_oa = tmem + Lay::kColOA, t_ob = tmem + Lay::kColOB;
       const int total = bars->n_tiles;
       PieceCursor qc, pcur;
       qc.init(bars);
@@ -481,8 +512,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
               q_rem = qp.te - qp.tb;
             }
             const int qb = q_si & 1;
-            if (mbar_try_wait(smem_u32(&bars->q_full[qb]), (q_si >> 1) & 1) &&
-                mbar_try_wait(smem_u32(&bars->full[jq % S]), (jq / S) & 1)) {
+            if (mbar_test_wait(smem_u32(&bars->q_full[qb]), (q_si >> 1) & 1) &&
+                mbar_test_wait(smem_u32(&bars->full[jq % S]), (jq / S) & 1)) {
               tc_fence_after();
               const uint32_t q_addr = s_base + Lay::kQOff + qb * Lay::kQBytes;
               const uint32_t k_addr = s_base + Lay::kStageOff + (jq % S) * Lay::kStageBytes;
@@ -499,7 +530,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
               ++jq;
             }
           }
-          if (mbar_try_wait(pb, (jp >> 1) & 1)) break;
+          if (mbar_test_wait(pb, (jp >> 1) & 1)) break;
           if ((it & 15u) == 15u) {
             if (*abort) { ok = false; break; }
             const uint64_t now = globaltimer();
@@ -512,11 +543,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int st = jp % S;
         const uint32_t p_addr = s_base + Lay::kPOff + (jp & 1) * Lay::kPBytes;
         const uint32_t v_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes + Lay::kKBytes;
+        // keys 0..31 of the tile into O_A, keys 32..63 into O_B
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint64_t da = smem_desc(p_addr + kk * 32, 16, 1024, kSwizzle128B);
           const uint64_t db = smem_desc(v_addr + kk * 2048, Lay::kKVAtomBytes, 1024, kSwizzle128B);
-          mma_bf16_ss(t_o, da, db, id_pv, (!first || kk > 0) ? 1u : 0u);
+          mma_bf16_ss(kk < 2 ? t_oa : t_ob, da, db, id_pv, (!first || (kk & 1)) ? 1u : 0u);
         }
         mma_commit(smem_u32(&bars->empty[st]));
         mma_commit(smem_u32(&bars->pv_done[jp & 1]));
@@ -528,14 +560,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------- softmax
+    // warps 2..9: quad = TMEM lane quarter (32 query rows); half = which 32
+    // keys of every tile, and which O accumulator, this warp owns.  The two
+    // halves keep independent running maxima and sums and are merged once
+    // per piece.
+    const int half = (warp - 2) >> 2;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const uint32_t t_s = tmem + lane_base + Lay::kColS;
-    const uint32_t t_o = tmem + lane_base + Lay::kColO;
+    const uint32_t t_s = tmem + lane_base + Lay::kColS + (uint32_t)(half * 32);
+    const uint32_t t_own = tmem + lane_base + (half ? Lay::kColOB : Lay::kColOA);
+    const uint32_t t_oa = tmem + lane_base + Lay::kColOA, t_ob = tmem + lane_base + Lay::kColOB;
+    float2* xch = reinterpret_cast<float2*>(smem + Lay::kXchOff);  // [half][row]
     const float sl2 = p.scale_log2;
     Piece pc = spc;
     RowCtx rc = src;
     bool have = s_have;
-    int jg = 0;
+    int jg = 0, n_epi = 0;
     bool ok = true;
     while (ok && have) {
       Piece pn;
@@ -550,7 +589,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const int qi = row_ok ? r_glob / G : 0;
       const int qh = row_ok ? g * G + r_glob % G : 0;
       const int win_lo = rc.qpos - a.window + 1;
-      float m_used = -INFINITY, l = 0.f;  // reference max (scaled, log2) and row sum
+      float m_used = -INFINITY, l = 0.f;  // reference max (scaled, log2) and row sum of this half
       for (int t = pc.tb; t < pc.te; ++t, ++jg) {
         if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[jg & 1]), (jg >> 1) & 1, abort))) {
           ok = false;
@@ -558,40 +597,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         }
         if (warp_live) {
           tc_fence_after();
-          float x[kBN];
+          float x[32];
           tmem_ld32(t_s + (uint32_t)((jg & 1) * kBN), x);
-          tmem_ld32(t_s + (uint32_t)((jg & 1) * kBN + 32), x + 32);
           tmem_wait_ld();
           const bool tree = t >= pc.ptiles;
-          const int key0 = tree ? (t - pc.ptiles) * kBN : pc.lo + t * kBN;
+          const int key0 = (tree ? (t - pc.ptiles) * kBN : pc.lo + t * kBN) + half * 32;
           const int k1 = tree ? a.n : pc.L;
-          float mx = -INFINITY;
-          if (tree) {  // tree keys: the row's ancestor bitmask (and the window on their positions)
-            const bool hi = key0 >= 64;
-            const uint64_t mw = row_ok ? (hi ? rc.mw1 : rc.mw0) : 0ull;
-            const int tp0 = hi ? rc.tpos[2] : rc.tpos[0], tp1 = hi ? rc.tpos[3] : rc.tpos[1];
+          // visibility of this half's 32 keys as one bit mask, built the same
+          // way on every tile (so the code stays hot in the instruction cache):
+          // keys below the piece's end, then the ancestor bits (tree keys) or
+          // the window's lower bound (prefix keys)
+          const int lim = k1 - key0;
+          uint32_t vm = lim >= 32 ? 0xffffffffu : (lim > 0 ? (1u << lim) - 1u : 0u);
+          const uint64_t mw = key0 >= 64 ? rc.mw1 : rc.mw0;
+          const uint32_t tree_bits = (uint32_t)(mw >> (key0 & 63));
+          const int lo_cut = win_lo - key0;  // prefix keys below it are outside the window
+          const uint32_t win_bits =
+              (a.window == 0 || lo_cut <= 0) ? 0xffffffffu : (lo_cut >= 32 ? 0u : ~((1u << lo_cut) - 1u));
+          vm &= tree ? tree_bits : win_bits;
+          if (!row_ok) vm = 0u;
+          if (tree && a.window > 0) {  // the window on tree keys' positions (rare; warp-uniform)
+            const int grp = key0 >> 5;
+            const int tsel = grp == 0 ? rc.tpos[0] : grp == 1 ? rc.tpos[1] : grp == 2 ? rc.tpos[2] : rc.tpos[3];
 #pragma unroll
-            for (int cc = 0; cc < kBN; ++cc) {
-              bool vis = key0 + cc < k1 && ((mw >> cc) & 1ull) != 0;
-              if (a.window > 0) {  // warp-uniform branch; every lane takes part in the shuffle
-                const int kpos = __shfl_sync(kFull, cc < 32 ? tp0 : tp1, cc & 31);
-                vis = vis && kpos >= win_lo;
-              }
-              x[cc] = vis ? x[cc] : -INFINITY;
-              mx = fmaxf(mx, x[cc]);
+            for (int cc = 0; cc < 32; ++cc) {
+              const int kpos = __shfl_sync(kFull, tsel, cc);  // every lane takes part
+              if (kpos < win_lo) vm &= ~(1u << cc);
             }
-          } else if (a.window > 0 || key0 + kBN > k1) {  // edge prefix tiles: per-key visibility
-#pragma unroll
-            for (int cc = 0; cc < kBN; ++cc) {
-              const int kidx = key0 + cc;
-              const bool vis = row_ok && kidx < k1 && (a.window == 0 || kidx >= win_lo);
-              x[cc] = vis ? x[cc] : -INFINITY;
-              mx = fmaxf(mx, x[cc]);
-            }
-          } else {  // interior prefix tile: every key visible
-#pragma unroll
-            for (int cc = 0; cc < kBN; ++cc) mx = fmaxf(mx, x[cc]);
           }
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) x[cc] = ((vm >> cc) & 1u) ? x[cc] : -INFINITY;
+          float m4[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+          for (int cc = 4; cc < 32; ++cc) m4[cc & 3] = fmaxf(m4[cc & 3], x[cc]);
+          float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           mx *= sl2;  // scale > 0 keeps the order
           // P buffer (jg & 1) was last read by PV(jg - 2)
           if (jg >= 2 &&
@@ -601,20 +640,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           }
           const bool rebase = mx > m_used + 8.f;
           if (__any_sync(kFull, rebase && t > pc.tb && l > 0.f)) {
-            // O may only be rescaled once PV(jg - 1) has finished accumulating
+            // this half's O may only be rescaled once PV(jg - 1) has finished accumulating
             if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[(jg - 1) & 1]), ((jg - 1) >> 1) & 1, abort))) {
               ok = false;
               break;
             }
             tc_fence_after();
             const float f = (rebase && l > 0.f) ? ex2(m_used - mx) : 1.f;
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              float o[32];
-              tmem_ld32(t_o + c0, o);
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              float o[16];
+              tmem_ld16(t_own + c0, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int u = 0; u < 32; ++u) o[u] *= f;
-              tmem_st32(t_o + c0, o);
+              for (int u = 0; u < 16; ++u) o[u] *= f;
+              tmem_st16(t_own + c0, o);
             }
             tmem_wait_st();
             l *= f;
@@ -622,29 +661,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           if (rebase) m_used = mx;
           const float neg_m = m_used > -INFINITY ? -m_used : 0.f;  // no visible key yet: every x is -inf
           unsigned char* prow = smem + Lay::kPOff + (jg & 1) * Lay::kPBytes + r_local * 128;
-          float sum = 0.f;
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c8 = 0; c8 < kBN / 8; ++c8) {
+          for (int c8 = 0; c8 < 4; ++c8) {
             uint32_t packed[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const float e0 = ex2(fmaf(x[c8 * 8 + 2 * u], sl2, neg_m));
               const float e1 = ex2(fmaf(x[c8 * 8 + 2 * u + 1], sl2, neg_m));
-              sum += e0 + e1;
+              s4[u] += e0 + e1;
               const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
               packed[u] = *reinterpret_cast<const uint32_t*>(&h2);
             }
-            *reinterpret_cast<uint4*>(prow + ((c8 ^ (r_local & 7)) << 4)) =
+            const int chunk = half * 4 + c8;  // 16-byte chunk of the 128-byte P row
+            *reinterpret_cast<uint4*>(prow + ((chunk ^ (r_local & 7)) << 4)) =
                 make_uint4(packed[0], packed[1], packed[2], packed[3]);
           }
-          l += sum;
+          l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
           fence_proxy_async_smem();
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->p_full[jg & 1]));
       }
       if (!ok) break;
-      // ---- end of the piece: normalised O -> bf16 output, or partial + lse
+      // ---- end of the piece: merge the two halves' (max, sum), normalise,
+      // write bf16 output or the partial + log-sum-exp.  Each warp of the pair
+      // writes its half of the output columns from both accumulators.
       if (warp_live) {
         const int jl = jg - 1;
         if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[jl & 1]), (jl >> 1) & 1, abort))) {
@@ -652,21 +694,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           break;
         }
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        xch[half * kRowsPerCta + r_local] = make_float2(m_used, l);
+        mbar_arrive(smem_u32(&bars->pair[quad]));
+        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pair[quad]), n_epi & 1, abort))) {
+          ok = false;
+          break;
+        }
+        ++n_epi;
+        const float2 other = xch[(half ^ 1) * kRowsPerCta + r_local];
+        const float ma = half ? other.x : m_used, la = half ? other.y : l;
+        const float mb = half ? m_used : other.x, lb = half ? l : other.y;
+        const float M = fmaxf(ma, mb);
+        const float wa = la > 0.f ? ex2(ma - M) : 0.f;
+        const float wb = lb > 0.f ? ex2(mb - M) : 0.f;
+        const float Ltot = la * wa + lb * wb;
+        const float inv = Ltot > 0.f ? 1.f / Ltot : 0.f;
+        const float fa = wa * inv, fb = wb * inv;
         const size_t slot = (size_t)c + (size_t)pc.b * HR + pc.hr;
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float o[32];
-          tmem_ld32(t_o + c0, o);
+        for (int c0 = half * (D / 2); c0 < (half + 1) * (D / 2); c0 += 16) {  // 16 columns at a time
+          float oa[16], ob[16];
+          tmem_ld16(t_oa + c0, oa);
+          tmem_ld16(t_ob + c0, ob);
           tmem_wait_ld();
           if (!row_ok) continue;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) oa[u] = fmaf(oa[u], fa, ob[u] * fb);
           if (pc.whole) {
             __nv_bfloat16* dst = p.out + (((size_t)pc.b * a.n + qi) * p.Hq + qh) * D + c0;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 2; ++u) {
               uint32_t w[4];
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[u * 8 + 2 * v] * inv, o[u * 8 + 2 * v + 1] * inv);
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(oa[u * 8 + 2 * v], oa[u * 8 + 2 * v + 1]);
                 w[v] = *reinterpret_cast<const uint32_t*>(&h2);
               }
               *reinterpret_cast<uint4*>(dst + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -674,13 +734,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           } else {
             float* dst = p.part_o + (slot * kRowsPerCta + r_local) * D + c0;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<float4*>(dst + 4 * u) =
-                  make_float4(o[4 * u] * inv, o[4 * u + 1] * inv, o[4 * u + 2] * inv, o[4 * u + 3] * inv);
+            for (int u = 0; u < 4; ++u)
+              *reinterpret_cast<float4*>(dst + 4 * u) = make_float4(oa[4 * u], oa[4 * u + 1], oa[4 * u + 2], oa[4 * u + 3]);
           }
         }
-        if (row_ok && !pc.whole)
-          p.part_lse[slot * kRowsPerCta + r_local] = l > 0.f ? (m_used + __log2f(l)) * (float)kLn2 : -INFINITY;
+        if (row_ok && !pc.whole && half == 0)
+          p.part_lse[slot * kRowsPerCta + r_local] = Ltot > 0.f ? (M + __log2f(Ltot)) * (float)kLn2 : -INFINITY;
         tc_fence_before();
       }
       pc = pn;
