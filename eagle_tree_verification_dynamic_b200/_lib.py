@@ -36,6 +36,19 @@ class TreeStruct(ctypes.Structure):
                 ("gid", _c_p), ("draft_row", _c_p), ("row_lse", _c_p)]
 
 
+class StepIn(ctypes.Structure):
+    _fields_ = [("draft_logits", _c_p), ("target_logits", _c_p), ("logits_dtype", _c_i),
+                ("B", _c_i), ("V", _c_i), ("depth", _c_i), ("k", _c_i), ("m", _c_i),
+                ("q", _c_p), ("k_cache", _c_p), ("v_cache", _c_p), ("prefix_len", _c_p), ("Lmax", _c_i),
+                ("k_tree", _c_p), ("v_tree", _c_p), ("Hq", _c_i), ("Hkv", _c_i), ("D", _c_i), ("window", _c_i),
+                ("scale", _c_f), ("uniforms", _c_p)]
+
+
+class StepOut(ctypes.Structure):
+    _fields_ = [("tree", TreeStruct), ("mask", _c_p), ("pos", _c_p), ("attn_out", _c_p),
+                ("accepted_len", _c_p), ("path", _c_p), ("bonus", _c_p)]
+
+
 _SIGS = {
     "eagle_status_string": (ctypes.c_char_p, [_c_i]),
     "eagle_last_cuda_error": (ctypes.c_char_p, []),
@@ -51,6 +64,10 @@ _SIGS = {
                                     _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p, _c_sz, _c_p]),
     "eagle_tree_build_noalloc": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                         ctypes.POINTER(TreeStruct), ctypes.POINTER(_c_i), _c_p]),
+    "eagle_verify_step_workspace_bytes": (_c_sz, [ctypes.POINTER(StepIn)]),
+    "eagle_verify_step_attention_status_offset": (_c_sz, [ctypes.POINTER(StepIn)]),
+    "eagle_verify_step": (_c_i, [ctypes.POINTER(StepIn), ctypes.POINTER(StepOut), ctypes.POINTER(_c_i), _c_p,
+                                 _c_sz, _c_p]),
     "eagle_accept_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
     "eagle_accept": (_c_i, [_c_p, _c_i, _c_p, _c_i, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i,
                             _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
@@ -278,3 +295,37 @@ def accept(target_logits, tokens, parents, draft_row, depth: int, uniforms=None,
     accept_into(target_logits, tokens, parents, draft_row, depth, uniforms, draft_logits, draft_lse,
                 acc, path, bonus, ws)
     return acc, path, bonus
+
+
+# ---------------------------------------------------------------- one step
+def step_in(draft_logits, target_logits, depth, k, m, q, k_cache, v_cache, prefix_len, k_tree, v_tree,
+            uniforms=None, window: int = 0, scale: float = 0.0) -> StepIn:
+    """The C step's inputs: draft_logits [B][R][V] and target_logits [B][n+1][V] (f32 or bf16),
+    q [B][n][Hq][D], caches [B][Hkv][Lmax][D], tree K/V [B][n][Hkv][D] (bf16), prefix_len [B] int32,
+    uniforms [B][2][n+1] f32 or None (greedy)."""
+    B, R, V = draft_logits.shape
+    Hq, D = q.shape[2], q.shape[3]
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    return StepIn(_ptr(draft_logits), _ptr(target_logits), _dtype_code(draft_logits), B, V, depth, k, m,
+                  _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), Lmax, _ptr(k_tree), _ptr(v_tree),
+                  Hq, Hkv, D, window, scale, _ptr(uniforms))
+
+
+def step_workspace_bytes(si: StepIn) -> int:
+    return lib().eagle_verify_step_workspace_bytes(ctypes.byref(si))
+
+
+def step_into(si: StepIn, tree: Tree, mask, pos, attn_out, accepted_len, path, bonus, ws: torch.Tensor,
+              device) -> int:
+    """Enqueue one whole step (build + fused mask, attention, acceptance) on the current stream."""
+    so = StepOut(tree.struct(), _ptr(mask), _ptr(pos), _ptr(attn_out), _ptr(accepted_len), _ptr(path), _ptr(bonus))
+    n_out = _c_i(0)
+    _check(lib().eagle_verify_step(ctypes.byref(si), ctypes.byref(so), ctypes.byref(n_out), _ptr(ws), ws.numel(),
+                                   _stream(device)), "eagle_verify_step")
+    return n_out.value
+
+
+def step_attention_status(si: StepIn, ws: torch.Tensor):
+    """Read the attention's device status word from a step workspace (synchronises)."""
+    off = lib().eagle_verify_step_attention_status_offset(ctypes.byref(si))
+    check_attention_status(ws[off:])

@@ -242,6 +242,8 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
                    int32_t* __restrict__ path, int32_t* __restrict__ bonus, int slice, bool vec_ok) {
   __shared__ AcceptSmem sm;
   extern __shared__ __align__(16) unsigned char cache_raw[];
+  griddep_wait();  // the target row statistics come from the previous kernel
+  griddep_launch_dependents();
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = (int)cluster.num_blocks();
   const int b = blockIdx.x / CL;
@@ -392,7 +394,7 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
                                int depth, const int32_t* row_amax, const double* row_lse,
                                const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                                const float* uniforms, int B, int32_t* acc_len, int32_t* path,
-                               int32_t* bonus, cudaStream_t s) {
+                               int32_t* bonus, cudaStream_t s, bool pdl) {
   int cl = 1, slice = 0;
   size_t dyn = 0;
   const bool vec_ok = (((uintptr_t)tgt | (uintptr_t)dft) % 16 == 0) && ((size_t)V * sizeof(T)) % 16 == 0;
@@ -420,13 +422,15 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
   cfg.blockDim = dim3(kAcceptThreads);
   cfg.dynamicSmemBytes = dyn;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cl;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, accept_walk_kernel<T, STOCH>, static_cast<const T*>(tgt),
                             static_cast<const T*>(dft), dlse, R, V, n, depth, row_amax, row_lse, tokens,
                             parents, draft_row, uniforms, acc_len, path, bonus, slice, vec_ok);
@@ -435,7 +439,7 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
 cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,
                           int R, const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                           const float* uniforms, int B, int n, int V, int depth, int32_t* accepted_len,
-                          int32_t* path, int32_t* bonus, void* ws, cudaStream_t s) {
+                          int32_t* path, int32_t* bonus, void* ws, cudaStream_t s, bool zero_tickets, bool pdl) {
   const long long rows = (long long)B * (n + 1);
   const bool stoch = uniforms != nullptr;
   char* tail = static_cast<char*>(ws) + row_stats_ws_bytes(rows, V, dtype_bytes(tdtype), 1);
@@ -445,18 +449,19 @@ cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddty
   ro.tok = row_amax;
   ro.val = nullptr;
   ro.lse = stoch ? row_lse : nullptr;
-  cudaError_t e = launch_row_stats(tgt, tdtype, rows, V, 1, stoch, ro, ws, s);
+  cudaError_t e = launch_row_stats(tgt, tdtype, rows, V, 1, stoch, ro, ws, s, zero_tickets, pdl);
   if (e != cudaSuccess) return e;
   (void)ddtype;  // the draft rows share the target's element type (checked by the caller)
   if (tdtype == EAGLE_F32)
     return stoch ? launch_walk<float, true>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens, parents,
-                                            draft_row, uniforms, B, accepted_len, path, bonus, s)
+                                            draft_row, uniforms, B, accepted_len, path, bonus, s, pdl)
                  : launch_walk<float, false>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
-                                             parents, draft_row, uniforms, B, accepted_len, path, bonus, s);
+                                             parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl);
   return stoch ? launch_walk<__nv_bfloat16, true>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
-                                                  parents, draft_row, uniforms, B, accepted_len, path, bonus, s)
+                                                  parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl)
                : launch_walk<__nv_bfloat16, false>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
-                                                   parents, draft_row, uniforms, B, accepted_len, path, bonus, s);
+                                                   parents, draft_row, uniforms, B, accepted_len, path, bonus, s,
+                                                   pdl);
 }
 
 }  // namespace eagle

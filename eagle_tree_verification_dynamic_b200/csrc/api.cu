@@ -191,4 +191,105 @@ eagle_status eagle_accept(const void* target_logits, int target_dtype, const voi
                                    workspace, static_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------------ whole step
+}  // extern "C"
+
+namespace {
+
+struct StepLayout {
+  int R, n;
+  size_t build_off, attn_off, acc_off, total;
+};
+
+// Shapes of the step; false for sizes that no call accepts (the step reports which).
+bool step_layout(const eagle_step_in_t* in, StepLayout* L) {
+  if (!in || in->B <= 0 || in->V <= 0 || in->depth <= 0 || in->k <= 0 || in->m <= 0 || !valid_dtype(in->logits_dtype))
+    return false;
+  if (in->depth > EAGLE_MAX_DEPTH || in->k > EAGLE_MAX_TOPK || in->m > EAGLE_MAX_NODES) return false;
+  const long long P = (long long)in->k + (long long)(in->depth - 1) * in->k * in->k;
+  if (P > EAGLE_MAX_POOL) return false;
+  if (in->Hq <= 0 || in->Hkv <= 0 || in->D <= 0 || in->Lmax < 0 || in->window < 0) return false;
+  L->R = 1 + (in->depth - 1) * in->k;
+  L->n = (int)(in->m < P ? in->m : P);
+  const int eb = dtype_bytes(in->logits_dtype);
+  L->build_off = 0;
+  L->attn_off = align_up(tree_build_ws_bytes(in->B, L->R, in->V, eb, in->k), 256);
+  L->acc_off = align_up(L->attn_off + attention_ws_bytes(in->B, L->n, in->Hq, in->Hkv, in->D, in->Lmax, in->window), 256);
+  L->total = align_up(L->acc_off + accept_ws_bytes(in->B, L->n, in->V, in->logits_dtype), 256);
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t eagle_verify_step_workspace_bytes(const eagle_step_in_t* in) {
+  StepLayout L;
+  return step_layout(in, &L) ? L.total : 0;
+}
+
+size_t eagle_verify_step_attention_status_offset(const eagle_step_in_t* in) {
+  StepLayout L;
+  return step_layout(in, &L) ? L.attn_off : 0;
+}
+
+eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t* out, int* n_nodes,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!in || !out) return EAGLE_ERR_NULL;
+  // --- the checks of the four calls, before anything is launched
+  const eagle_tree_t& t = out->tree;
+  if (!in->draft_logits || !in->target_logits || !in->q || !in->k_tree || !in->v_tree || !in->prefix_len)
+    return EAGLE_ERR_NULL;
+  if (!t.tokens || !t.parents || !t.depth || !t.logV || !t.draft_row || !t.row_lse) return EAGLE_ERR_NULL;
+  if (!out->mask || !out->pos || !out->attn_out || !out->accepted_len || !out->path || !out->bonus)
+    return EAGLE_ERR_NULL;
+  if (in->Lmax > 0 && (!in->k_cache || !in->v_cache)) return EAGLE_ERR_NULL;
+  if (!valid_dtype(in->logits_dtype)) return EAGLE_ERR_DTYPE;
+  if (in->B <= 0 || in->V <= 0 || in->depth <= 0 || in->k <= 0 || in->m <= 0) return EAGLE_ERR_SHAPE;
+  if (in->Hq <= 0 || in->Hkv <= 0 || in->Lmax < 0 || in->window < 0 || in->Hq % in->Hkv != 0) return EAGLE_ERR_SHAPE;
+  if (in->depth > EAGLE_MAX_DEPTH || in->k > EAGLE_MAX_TOPK || in->k > in->V || in->m > EAGLE_MAX_NODES)
+    return EAGLE_ERR_LIMIT;
+  if (in->D != 64 && in->D != 128) return EAGLE_ERR_LIMIT;
+  StepLayout L;
+  if (!step_layout(in, &L)) return EAGLE_ERR_LIMIT;
+  if ((long long)in->B * (L.n + 1) > 0x7fffffffLL) return EAGLE_ERR_SHAPE;
+  if (in->uniforms && in->V > accept_max_vocab(in->logits_dtype)) return EAGLE_ERR_LIMIT;
+  if (!aligned16(in->q) || !aligned16(in->k_tree) || !aligned16(in->v_tree) || !aligned16(out->attn_out) ||
+      (in->Lmax > 0 && (!aligned16(in->k_cache) || !aligned16(in->v_cache))))
+    return EAGLE_ERR_ALIGN;
+  eagle_status st = check_ws(workspace, workspace_bytes, L.total);
+  if (st != EAGLE_OK) return st;
+  if (n_nodes) *n_nodes = L.n;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const int eb = dtype_bytes(in->logits_dtype);
+  const int n = L.n;
+  // --- clear both row sweeps' tickets up front; every kernel then chains to
+  // its predecessor with programmatic dependent launch
+  size_t off = 0, bytes = 0;
+  row_stats_tickets_span((long long)in->B * L.R, in->V, eb, in->k, &off, &bytes);
+  cudaError_t e = cudaMemsetAsync(ws + L.build_off + off, 0, bytes, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  row_stats_tickets_span((long long)in->B * (n + 1), in->V, eb, 1, &off, &bytes);
+  e = cudaMemsetAsync(ws + L.acc_off + off, 0, bytes, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  // --- build, with the mask and position ids written by the expansion
+  const MaskOut mo = {in->prefix_len, out->mask, out->pos};
+  e = launch_tree_build(in->draft_logits, in->logits_dtype, in->B, L.R, in->V, in->depth, in->k, n, t,
+                        ws + L.build_off, s, &mo, false, true);
+  if (e != cudaSuccess) return cuda_status(e);
+  // --- tree attention
+  const float scale = in->scale > 0.f ? in->scale : 1.0f / sqrtf((float)in->D);
+  e = launch_tree_attention(in->q, in->k_cache, in->v_cache, in->prefix_len, in->Lmax, in->k_tree, in->v_tree,
+                            out->mask, out->pos, in->B, n, in->Hq, in->Hkv, in->D, in->window, scale, out->attn_out,
+                            ws + L.attn_off, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  // --- acceptance (the draft rows' log-sum-exps are the tree's row_lse)
+  e = launch_accept(in->target_logits, in->logits_dtype, in->draft_logits, in->logits_dtype, t.row_lse, L.R,
+                    t.tokens, t.parents, t.draft_row, in->uniforms, in->B, n, in->V, in->depth, out->accepted_len,
+                    out->path, out->bonus, ws + L.acc_off, s, false, true);
+  return cuda_status(e);
+}
+
 }  // extern "C"

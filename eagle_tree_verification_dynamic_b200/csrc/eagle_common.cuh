@@ -17,6 +17,18 @@ namespace eagle {
 
 constexpr unsigned kFull = 0xffffffffu;
 
+// ------------------------------------------- programmatic dependent launch
+// Every kernel of the library calls griddep_wait() before it touches global
+// memory: launched with programmatic stream serialization it may start while
+// its predecessor on the stream drains, and this blocks until that grid has
+// completed and its memory is visible (a no-op for an ordinary launch).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the grids that depend on this one be scheduled (they still wait in
+// griddep_wait before reading anything this grid writes).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // log2(e) split into an fp32 head and an fp32 tail: x*log2(e) is formed as
 // fma(x, kLog2eHi, x*kLog2eLo) so that the constant's fp32 rounding does not
 // bias every exponent of a row by the same relative amount.

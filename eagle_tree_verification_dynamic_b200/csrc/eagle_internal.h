@@ -14,6 +14,26 @@ constexpr int kNumSMs = 148;  // B200
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launch with an optional programmatic-dependent-launch attribute (the kernel
+// may start while its predecessor drains; it waits in griddep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                 bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device), so
 // later launches (including ones under stream capture) only launch.
 cudaError_t ensure_smem_limit(const void* kernel, size_t bytes);
@@ -32,14 +52,27 @@ struct RowOut {
 };
 ChunkPlan plan_chunks(long long rows, int V, int elem_bytes);
 size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k);
+// zero_tickets: clear the per-row tickets first (else the caller already has);
+// pdl: chain the kernel to its predecessor with programmatic dependent launch.
 cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, int k, bool lse, const RowOut& out,
-                             void* ws, cudaStream_t s);
+                             void* ws, cudaStream_t s, bool zero_tickets = true, bool pdl = false);
+// Byte range of the per-row tickets inside the row-sweep workspace.
+void row_stats_tickets_span(long long rows, int V, int elem_bytes, int k, size_t* off, size_t* bytes);
 
 // ---- tree build (tree_build.cu)
 size_t tree_build_smem_bytes(int R, int k, int P);
 size_t tree_build_ws_bytes(int B, int R, int V, int elem_bytes, int k);
+// Optional fused tree mask: with mask != nullptr the expansion kernel also
+// writes each node's ancestor-or-self bitmask and position id (what
+// eagle_tree_mask computes).
+struct MaskOut {
+  const int32_t* prefix_len;  // [B] (required with pos)
+  uint64_t* mask;             // [B][n][2]
+  int32_t* pos;               // [B][n] (may be null)
+};
 cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k, int n,
-                              const eagle_tree_t& out, void* ws, cudaStream_t s);
+                              const eagle_tree_t& out, void* ws, cudaStream_t s, const MaskOut* mo = nullptr,
+                              bool zero_tickets = true, bool pdl = false);
 
 // ---- tree mask (tree_mask.cu)
 cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len,
@@ -73,6 +106,7 @@ int accept_max_vocab(int dtype);  // largest V the sampled walk supports
 cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,
                           int R, const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                           const float* uniforms, int B, int n, int V, int depth, int32_t* accepted_len,
-                          int32_t* path, int32_t* bonus, void* ws, cudaStream_t s);
+                          int32_t* path, int32_t* bonus, void* ws, cudaStream_t s, bool zero_tickets = true,
+                          bool pdl = false);
 
 }  // namespace eagle

@@ -80,6 +80,7 @@ template <typename T, bool LSE, bool VEC, int M>
 __global__ void __launch_bounds__(kStatThreads)
 row_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k, ChunkStat* __restrict__ stats,
                  uint64_t* __restrict__ keys, int* __restrict__ tickets, RowOut out) {
+  griddep_wait();  // the logits (and this workspace) may belong to the previous kernel
   const long long row = blockIdx.x;
   const int chunk = blockIdx.y, n_chunks = gridDim.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -147,6 +148,7 @@ row_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k, ChunkSt
     }
   }
 
+  griddep_launch_dependents();  // every CTA that reaches here has done its streaming
   __shared__ uint64_t s_keys[kStatWarps][32];
   __shared__ float s_e[kStatWarps];
   __shared__ double s_s[kStatWarps];
@@ -282,30 +284,39 @@ size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k) {
 }
 
 template <typename T, bool LSE, int M>
-static void launch_typed(const void* x, long long rows, int V, int k, const ChunkPlan& p, bool vec,
-                         ChunkStat* stats, uint64_t* keys, int* tickets, const RowOut& out, cudaStream_t s) {
-  dim3 grid((unsigned)rows, (unsigned)p.n_chunks);
+static cudaError_t launch_typed(const void* x, long long rows, int V, int k, const ChunkPlan& p, bool vec,
+                                ChunkStat* stats, uint64_t* keys, int* tickets, const RowOut& out, cudaStream_t s,
+                                bool pdl) {
+  const dim3 grid((unsigned)rows, (unsigned)p.n_chunks);
   const T* xp = static_cast<const T*>(x);
   if (vec)
-    row_stats_kernel<T, LSE, true, M><<<grid, kStatThreads, 0, s>>>(xp, V, p.chunk_elems, k, stats, keys, tickets, out);
-  else
-    row_stats_kernel<T, LSE, false, M><<<grid, kStatThreads, 0, s>>>(xp, V, p.chunk_elems, k, stats, keys, tickets, out);
+    return launch_kernel(row_stats_kernel<T, LSE, true, M>, grid, dim3(kStatThreads), 0, s, pdl, xp, V,
+                         p.chunk_elems, k, stats, keys, tickets, out);
+  return launch_kernel(row_stats_kernel<T, LSE, false, M>, grid, dim3(kStatThreads), 0, s, pdl, xp, V,
+                       p.chunk_elems, k, stats, keys, tickets, out);
 }
 
 template <typename T>
-static void launch_t(const void* x, long long rows, int V, int k, bool lse, const ChunkPlan& p, bool vec,
-                     ChunkStat* stats, uint64_t* keys, int* tickets, const RowOut& out, cudaStream_t s) {
+static cudaError_t launch_t(const void* x, long long rows, int V, int k, bool lse, const ChunkPlan& p, bool vec,
+                            ChunkStat* stats, uint64_t* keys, int* tickets, const RowOut& out, cudaStream_t s,
+                            bool pdl) {
   if (k == 1) {
-    if (lse) launch_typed<T, true, 1>(x, rows, V, k, p, vec, stats, keys, tickets, out, s);
-    else     launch_typed<T, false, 1>(x, rows, V, k, p, vec, stats, keys, tickets, out, s);
-  } else {
-    if (lse) launch_typed<T, true, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s);
-    else     launch_typed<T, false, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s);
+    if (lse) return launch_typed<T, true, 1>(x, rows, V, k, p, vec, stats, keys, tickets, out, s, pdl);
+    return launch_typed<T, false, 1>(x, rows, V, k, p, vec, stats, keys, tickets, out, s, pdl);
   }
+  if (lse) return launch_typed<T, true, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s, pdl);
+  return launch_typed<T, false, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s, pdl);
+}
+
+void row_stats_tickets_span(long long rows, int V, int elem_bytes, int k, size_t* off, size_t* bytes) {
+  const ChunkPlan p = plan_chunks(rows, V, elem_bytes);
+  const size_t n = (size_t)rows * p.n_chunks;
+  *off = align_up(n * sizeof(ChunkStat), 256) + align_up(n * k * sizeof(uint64_t), 256);
+  *bytes = (size_t)rows * sizeof(int);
 }
 
 cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, int k, bool lse, const RowOut& out,
-                             void* ws, cudaStream_t s) {
+                             void* ws, cudaStream_t s, bool zero_tickets, bool pdl) {
   const int eb = dtype_bytes(dtype);
   const ChunkPlan p = plan_chunks(rows, V, eb);
   const size_t n = (size_t)rows * p.n_chunks;
@@ -314,12 +325,13 @@ cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, in
   uint64_t* keys = reinterpret_cast<uint64_t*>(base + align_up(n * sizeof(ChunkStat), 256));
   int* tickets = reinterpret_cast<int*>(base + align_up(n * sizeof(ChunkStat), 256) +
                                         align_up(n * k * sizeof(uint64_t), 256));
-  cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)rows * sizeof(int), s);
-  if (e != cudaSuccess) return e;
+  if (zero_tickets) {
+    cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)rows * sizeof(int), s);
+    if (e != cudaSuccess) return e;
+  }
   const bool vec = ((uintptr_t)x % 16 == 0) && (((size_t)V * eb) % 16 == 0);
-  if (dtype == EAGLE_F32) launch_t<float>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s);
-  else launch_t<__nv_bfloat16>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s);
-  return cudaGetLastError();
+  if (dtype == EAGLE_F32) return launch_t<float>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s, pdl);
+  return launch_t<__nv_bfloat16>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s, pdl);
 }
 
 }  // namespace eagle

@@ -18,17 +18,6 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-// ------------------------------------------- programmatic dependent launch
-// Block until the grids this one depends on have completed and their memory
-// is visible (returns at once for a launch without the programmatic
-// serialization attribute).
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-// Allow the grids that depend on this one to be scheduled; they still wait
-// for this grid's completion in griddep_wait before reading its results.
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

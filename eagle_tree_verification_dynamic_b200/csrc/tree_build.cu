@@ -48,14 +48,6 @@ struct BuildSmem {
   int* node_dep;     // [EAGLE_MAX_NODES]
 };
 
-// Optional fused tree mask: with mask != nullptr the expansion kernel also
-// writes each node's ancestor-or-self bitmask and position id (what
-// eagle_tree_mask computes), saving a launch and a round trip of the tree.
-struct MaskOut {
-  const int32_t* prefix_len;  // [B]
-  uint64_t* mask;             // [B][n][2]
-  int32_t* pos;               // [B][n] (may be null)
-};
 
 __host__ __device__ inline int next_pow2(int x) {
   int p = 1;
@@ -76,6 +68,8 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   const int Ppow = next_pow2(P);
   const int nsort = Ppow > 2 * kBuildThreads ? Ppow : 2 * kBuildThreads;
 
+  griddep_wait();  // the row statistics come from the previous kernel
+  griddep_launch_dependents();
   BuildSmem sm;
   {
     unsigned char* p = smem_raw;
@@ -255,7 +249,8 @@ size_t tree_build_ws_bytes(int B, int R, int V, int elem_bytes, int k) {
 }
 
 cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k, int n,
-                              const eagle_tree_t& out, void* ws, cudaStream_t s) {
+                              const eagle_tree_t& out, void* ws, cudaStream_t s, const MaskOut* mo_in,
+                              bool zero_tickets, bool pdl) {
   const long long rows = (long long)B * R;
   const int eb = dtype_bytes(dtype);
   char* tail = static_cast<char*>(ws) + row_stats_ws_bytes(rows, V, eb, k);
@@ -263,15 +258,15 @@ cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R,
   ro.tok = reinterpret_cast<int32_t*>(tail);
   ro.val = reinterpret_cast<float*>(tail + align_up((size_t)rows * k * sizeof(int32_t), 256));
   ro.lse = out.row_lse;
-  cudaError_t e = launch_row_stats(draft_logits, dtype, rows, V, k, true, ro, ws, s);
+  cudaError_t e = launch_row_stats(draft_logits, dtype, rows, V, k, true, ro, ws, s, zero_tickets, pdl);
   if (e != cudaSuccess) return e;
   const int P = k + (depth - 1) * k * k;
   const size_t smem = tree_build_smem_bytes(R, k, P);
   e = ensure_smem_limit((const void*)tree_expand_kernel, smem);
   if (e != cudaSuccess) return e;
-  MaskOut mo = {nullptr, nullptr, nullptr};
-  tree_expand_kernel<<<B, kBuildThreads, smem, s>>>(ro.tok, ro.val, R, depth, k, n, out, mo);
-  return cudaGetLastError();
+  const MaskOut mo = mo_in ? *mo_in : MaskOut{nullptr, nullptr, nullptr};
+  return launch_kernel(tree_expand_kernel, dim3(B), dim3(kBuildThreads), smem, s, pdl, ro.tok, ro.val, R, depth, k,
+                       n, out, mo);
 }
 
 }  // namespace eagle

@@ -9,6 +9,8 @@ namespace eagle {
 __global__ void tree_mask_kernel(const int32_t* __restrict__ parents, const int32_t* __restrict__ depth,
                                  const int32_t* __restrict__ prefix_len, int B, int n,
                                  uint64_t* __restrict__ mask, int32_t* __restrict__ pos) {
+  griddep_wait();
+  griddep_launch_dependents();
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= (long long)B * n) return;
   const int b = (int)(t / n), i = (int)(t - (long long)b * n);

@@ -1,8 +1,11 @@
 """One whole tree-verification step with preallocated buffers.
 
 build (vocabulary sweep + EAGLE-2 expansion/rerank) -> mask -> tree attention
--> acceptance, enqueued on the current CUDA stream through the C ABI.  All
-buffers and workspaces are allocated once in the constructor, so a step
+-> acceptance, enqueued on the current CUDA stream through the C ABI: either
+as the four calls one after another (``__call__``) or as the single
+``eagle_verify_step`` call (``fused``: the mask fused into the expansion, one
+clearing of the scratch, kernels chained by programmatic dependent launch).
+All buffers and workspaces are allocated once in the constructor, so a step
 allocates nothing and can be captured in a CUDA graph.
 """
 from __future__ import annotations
@@ -57,6 +60,9 @@ class VerifyStep:
         self.ws_build = L._workspace(L.tree_build_workspace_bytes(s.B, s.R, s.V, dcode, s.k), dev)
         self.ws_attn = L._workspace(L.attention_workspace_bytes(s.B, n, s.Hq, s.Hkv, s.D, s.Lmax, s.window), dev)
         self.ws_acc = L._workspace(L.accept_workspace_bytes(s.B, n, s.V, dcode), dev)
+        shape_only = L.StepIn(None, None, dcode, s.B, s.V, s.depth, s.k, s.m, None, None, None, None, s.Lmax, None,
+                              None, s.Hq, s.Hkv, s.D, s.window, 0.0, None)
+        self.ws_step = L._workspace(L.step_workspace_bytes(shape_only), dev)
 
     def build(self, draft_logits: torch.Tensor):
         L.tree_build_into(draft_logits, self.s.depth, self.s.k, self.s.m, self.tree, self.ws_build)
@@ -76,6 +82,21 @@ class VerifyStep:
         else:
             L.accept_into(target_logits, self.tree.tokens, self.tree.parents, self.tree.draft_row, self.s.depth,
                           None, None, None, self.accepted_len, self.path, self.bonus, self.ws_acc)
+
+    def fused(self, inp: dict):
+        """The same step as one eagle_verify_step call (same outputs)."""
+        s = self.s
+        si = L.step_in(inp["draft_logits"], inp["target_logits"], s.depth, s.k, s.m, inp["q"], inp["k_cache"],
+                       inp["v_cache"], inp["prefix_len"], inp["k_tree"], inp["v_tree"],
+                       inp.get("uniforms") if s.stochastic else None, s.window)
+        L.step_into(si, self.tree, self.mask, self.pos, self.out, self.accepted_len, self.path, self.bonus,
+                    self.ws_step, self.device)
+        self._step_in = si
+        return self.accepted_len, self.path, self.bonus
+
+    def fused_attention_status(self):
+        """Raise if the last fused step's attention reported a device status."""
+        L.step_attention_status(self._step_in, self.ws_step)
 
     def __call__(self, inp: dict):
         """inp: draft_logits, prefix_len, q, k_cache, v_cache, k_tree, v_tree, target_logits, uniforms."""

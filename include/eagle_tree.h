@@ -220,6 +220,63 @@ EAGLE_API eagle_status eagle_accept(const void* target_logits, int target_dtype,
                           int B, int n, int V, int depth, int32_t* accepted_len, int32_t* path,
                           int32_t* bonus, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------- one whole step
+ * One verification step in its order: build (eagle_tree_build), mask and
+ * position ids (fused into the build's expansion kernel), tree attention
+ * (eagle_tree_attention) and acceptance (eagle_accept), on one stream.  The
+ * outputs equal those of the four calls made one after another on the same
+ * inputs (the same kernels and the same arithmetic).  The scratch is cleared
+ * once at the start and each kernel may start while its predecessor drains
+ * (programmatic dependent launch): two memsets, seven kernels, no host
+ * synchronisation.
+ *
+ * Inputs (device pointers unless noted; layouts as in the calls above):
+ *   draft_logits [B][R][V] (logits_dtype), R = 1 + (depth-1)*k
+ *   q [B][n][Hq][D], k_cache / v_cache [B][Hkv][Lmax][D], k_tree / v_tree
+ *   [B][n][Hkv][D] (bf16), prefix_len [B] int32, with n = min(m, pool size)
+ *   (the tree size, also written to the HOST int *n_nodes when not NULL)
+ *   target_logits [B][n+1][V] (logits_dtype, the target's rows of the tree)
+ *   uniforms [B][2][n+1] float, or NULL for greedy acceptance
+ * Outputs (caller-allocated, sized by n): the tree arrays (tree.gid may be
+ *   NULL), mask [B][n][2] uint64, pos [B][n] int32, attn_out [B][n][Hq][D]
+ *   bf16, accepted_len [B], path [B][depth], bonus [B] int32.
+ * Limits: those of the four calls.  Workspace: eagle_verify_step_workspace_bytes
+ * (256-byte aligned).  The attention's device status word (0 = ok, 1 = an
+ * internal wait gave up) is the int at byte offset
+ * eagle_verify_step_attention_status_offset of the workspace after the step. */
+typedef struct {
+  const void* draft_logits;
+  const void* target_logits;
+  int logits_dtype;
+  int B, V, depth, k, m;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* prefix_len;
+  int Lmax;
+  const void* k_tree;
+  const void* v_tree;
+  int Hq, Hkv, D, window;
+  float scale;  /* <= 0 selects 1/sqrt(D) */
+  const float* uniforms;
+} eagle_step_in_t;
+
+typedef struct {
+  eagle_tree_t tree;
+  uint64_t* mask;
+  int32_t* pos;
+  void* attn_out;
+  int32_t* accepted_len;
+  int32_t* path;
+  int32_t* bonus;
+} eagle_step_out_t;
+
+/* Both return 0 for an invalid shape (the step itself then reports why). */
+EAGLE_API size_t eagle_verify_step_workspace_bytes(const eagle_step_in_t* in);
+EAGLE_API size_t eagle_verify_step_attention_status_offset(const eagle_step_in_t* in);
+EAGLE_API eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t* out, int* n_nodes,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* ----------------------------------------------------- tree build, no workspace
  * Not a step of the method (the pages have no counterpart): the same build as
  * eagle_tree_build for callers that cannot allocate device memory when they

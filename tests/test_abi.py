@@ -116,3 +116,48 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(et.EagleError):
         et.tree_build(torch.zeros(1, 5, 100), 3, 2, 10)
+
+
+def _step_in(**kw):
+    d = dict(draft_logits=FAKE, target_logits=FAKE, logits_dtype=0, B=1, V=32000, depth=6, k=10, m=60,
+             q=FAKE, k_cache=FAKE, v_cache=FAKE, prefix_len=FAKE, Lmax=2048, k_tree=FAKE, v_tree=FAKE,
+             Hq=32, Hkv=32, D=128, window=0, scale=0.0, uniforms=None)
+    d.update(kw)
+    return _lib.StepIn(*[d[name] for name, _ in _lib.StepIn._fields_])
+
+
+def _step_out(valid=True):
+    p = FAKE if valid else None
+    return _lib.StepOut(_tree(), p, p, p, p, p, p)
+
+
+def test_step_workspace_covers_the_four_calls(lib):
+    si = _step_in()
+    total = lib.eagle_verify_step_workspace_bytes(ctypes.byref(si))
+    assert total > 0 and total % 256 == 0
+    parts = (lib.eagle_tree_build_workspace_bytes(1, 51, 32000, 0, 10)
+             + lib.eagle_tree_attention_workspace_bytes(1, 60, 32, 32, 128, 2048, 0)
+             + lib.eagle_accept_workspace_bytes(1, 60, 32000, 0))
+    assert parts <= total <= parts + 3 * 256
+    off = lib.eagle_verify_step_attention_status_offset(ctypes.byref(si))
+    assert off % 256 == 0 and off >= lib.eagle_tree_build_workspace_bytes(1, 51, 32000, 0, 10)
+    assert lib.eagle_verify_step_workspace_bytes(ctypes.byref(_step_in(D=0))) == 0
+
+
+def test_step_validation(lib):
+    n = ctypes.c_int(0)
+
+    def call(si=None, so=None, ws=FAKE, wsb=1 << 30):
+        si = si or _step_in()
+        so = so or _step_out()
+        return lib.eagle_verify_step(ctypes.byref(si), ctypes.byref(so), ctypes.byref(n), ws, wsb, None)
+    assert lib.eagle_verify_step(None, None, None, FAKE, 0, None) == 1
+    assert call(si=_step_in(q=None)) == 1
+    assert call(so=_step_out(False)) == 1
+    assert call(si=_step_in(logits_dtype=4)) == 3
+    assert call(si=_step_in(Hq=30, Hkv=4)) == 2
+    assert call(si=_step_in(D=96)) == 4
+    assert call(si=_step_in(m=200)) == 4
+    assert call(si=_step_in(q=ctypes.c_void_p(0x1008))) == 6
+    assert call(ws=None, wsb=0) == 5
+    assert n.value == 0  # nothing was reported: every call above failed validation
