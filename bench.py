@@ -204,6 +204,35 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------- multi-rank helpers
+def rank_env():
+    """(world, rank, local_rank) of this process, as torchrun sets them (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def input_seed(rank: int, i: int) -> int:
+    """Seed of input set i on a rank: every rank works on its own sequences."""
+    return 1000 * rank + i
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of a list of floats over all ranks (the slowest rank
+    sets every time); returns the list unchanged when running alone."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(world: int, ms_per_step: float) -> float:
+    """Steps per second of the whole job: every rank completes one step of its
+    own batch per ms_per_step (the max over ranks)."""
+    return world * 1000.0 / ms_per_step
+
+
 # ------------------------------------------------------------------ GPU leg
 def main():
     args = parse()
@@ -216,9 +245,7 @@ def main():
     import eagle_tree_verification_dynamic_b200 as et
     from eagle_tree_verification_dynamic_b200.step import StepShape, VerifyStep
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     if world > 1:
@@ -246,7 +273,7 @@ def main():
     n_sets = min(n_sets, 16)
     sets, hosts, steps = [], [], []
     for i in range(n_sets):
-        seed = 1000 * rank + i
+        seed = input_seed(rank, i)
         stored = gen_draft_logits(cfg, seed)
         plen = gen_prefix_len(cfg, seed)
         q, kc, vc, kt, vt = gen_attention_inputs(cfg, seed, cfg.L)
@@ -372,11 +399,9 @@ def main():
     barrier()
     ms_e2e = e0.elapsed_time(e1) / K
 
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e] + [stage_ms[k] for k in stage_fns], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
-        stage_ms = {k: float(t[2 + i]) for i, k in enumerate(stage_fns)}
+    red = max_over_ranks([ms, ms_e2e] + [stage_ms[k] for k in stage_fns], dist if world > 1 else None, dev)
+    ms, ms_e2e = red[0], red[1]
+    stage_ms = {k: red[2 + i] for i, k in enumerate(stage_fns)}
 
     peaks = {}
     try:
@@ -389,7 +414,7 @@ def main():
 
     sb = step_bytes(cfg, gen_prefix_len(cfg, 0), args.mode)
     attn_gbs = sb["attention"] / (stage_ms["attention"] * 1e-3) / 1e9
-    value = world * 1000.0 / ms
+    value = whole_job_rate(world, ms)
     stages = {k: {"ms": round(v, 5)} for k, v in stage_ms.items()}
     stages["build"]["gbs"] = round(sb["draft"] / (stage_ms["build"] * 1e-3) / 1e9, 1)
     stages["attention"]["gbs"] = round(attn_gbs, 1)
@@ -414,7 +439,7 @@ def main():
                      "algorithmic_bytes": sb["attention"]},
         "step_roofline": {"bytes": sb["step"], "t_min_us": round(sb["step"] / hbm_peak / 1e3, 3),
                           "frac": round(sb["step"] / hbm_peak / 1e3 / (ms * 1e3), 4)},
-        "e2e": {"value": round(world * 1000.0 / ms_e2e, 2), "unit": "steps/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(whole_job_rate(world, ms_e2e), 2), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_STEP * K,
         "clocks": clocks,

@@ -56,6 +56,9 @@ struct AcceptSmem {
   double lse_d[EAGLE_MAX_NODES + 1];   // log-sum-exp of node j's draft row
   double px[EAGLE_MAX_NODES + 1];      // child c: p(x_c) under its parent's target row
   double qx[EAGLE_MAX_NODES + 1];      // child c: q(x_c) under its parent's draft row
+  float u_acc[EAGLE_MAX_NODES + 1];    // the walk's uniforms, staged once
+  float u_res[EAGLE_MAX_NODES + 1];
+  int first_child[EAGLE_MAX_NODES + 1];  // node j's first child in node order (n + 1: none)
   double warp_part[kAcceptWarps];
   double red[2][kAcceptWarps];   // block-reduction slots, alternating by call
   double lane_sum[kAcceptThreads];
@@ -261,7 +264,19 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     const int r = draft_row[(size_t)b * (n + 1) + i];
     sm.drow[i] = (r >= 0 && r < R) ? r : -1;  // an out-of-range row counts as "not expanded"
     sm.amax[i] = row_amax[trow0 + i];
-    if (STOCH) sm.lse_t[i] = row_lse[trow0 + i];
+    if (STOCH) {
+      sm.lse_t[i] = row_lse[trow0 + i];
+      sm.u_acc[i] = uniforms[(size_t)b * 2 * (n + 1) + i];
+      sm.u_res[i] = uniforms[(size_t)b * 2 * (n + 1) + (n + 1) + i];
+    }
+  }
+  __syncthreads();
+  // each node's first child in node order (siblings follow it, in node order)
+  for (int i = tid; i <= n; i += kAcceptThreads) sm.first_child[i] = n + 1;
+  __syncthreads();
+  for (int c = tid + 1; c <= n; c += kAcceptThreads) {
+    const int p = sm.par[c - 1];
+    if (p >= 0 && p <= n) atomicMin(&sm.first_child[p], c);
   }
   __syncthreads();
   if (STOCH) {
@@ -299,8 +314,6 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     sl.cached_d = -1;
   }
 
-  const float* u_acc = STOCH ? uniforms + (size_t)b * 2 * (n + 1) : nullptr;
-  const float* u_res = STOCH ? u_acc + (n + 1) : nullptr;
 
   int j = 0, plen = 0;
   double lse_t = STOCH ? sm.lse_t[0] : 0.0;
@@ -311,7 +324,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   while (plen < depth) {
     int moved_to = -1;
     if (!STOCH) {
-      for (int c = 1; c <= n; ++c)
+      for (int c = sm.first_child[j]; c <= n; ++c)
         if (sm.par[c - 1] == j && sm.tok[c - 1] == amax) { moved_to = c; break; }
     } else {
       const int r = sm.drow[j];
@@ -319,15 +332,14 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
       const T* drow = r >= 0 ? dft + ((size_t)b * R + r) * (size_t)V : nullptr;
       const double lse_d = sm.lse_d[j];
       // children of j in node order
-      int c = 1;
+      int c = sm.first_child[j];
       while (true) {
-        while (c <= n && sm.par[c - 1] != j) ++c;
         if (c > n || r < 0) break;
         // accept iff u < rho / (F q), i.e. u F q < rho (q > 0); a token outside
         // the vocabulary has p = q = 0 and is never accepted
         const double px = sm.px[c], qx = sm.qx[c];
         const double rho = t == 0.0 ? px : fmax(0.0, px - t * qx);
-        if (qx > 0.0 && (double)u_acc[c] * (F * qx) < rho) { moved_to = c; break; }
+        if (qx > 0.0 && (double)sm.u_acc[c] * (F * qx) < rho) { moved_to = c; break; }
         // rejected: the current target becomes max(0, p - t' q) / F(t')
         t += F;
         rejected_here = true;
@@ -371,7 +383,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   a.lse_t.set(lse_t);
   a.lse_d.set(sm.lse_d[j]);
   a.t.set(t);
-  const double total = sweep_sample<T>(sl, a, u_res[j], sm, cluster, bonus + b, par);
+  const double total = sweep_sample<T>(sl, a, sm.u_res[j], sm, cluster, bonus + b, par);
   if (!(total > 0.0) && leader) bonus[b] = amax;  // nothing left to sample from
   cluster.sync();  // no CTA leaves while another may still read its shared memory
 }
