@@ -43,7 +43,7 @@ LAUNCHES_PER_STEP = 6  # one eagle_verify_step: row sweep, expand (+ mask), atte
 # DRAM bytes (read + write) of one launch of the tree attention's main kernel,
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of this
 # kernel version on the named workload; a workload without a capture reports null.
-ATTN_TRAFFIC_BYTES = {"7b": 35116288 + 768}
+ATTN_TRAFFIC_BYTES = {"7b": 35099392 + 13824}
 
 
 def parse():
