@@ -57,7 +57,8 @@ __host__ __device__ inline int next_pow2(int x) {
 
 // row_tok / row_val: each draft row's top-k tokens and logits (descending),
 // row_lse: each row's log-sum-exp (also the tree's row_lse output).
-__global__ void __launch_bounds__(kBuildThreads)
+template <int NT>
+__global__ void __launch_bounds__(NT)
 tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restrict__ row_val_g, int R, int depth,
                    int k, int n, eagle_tree_t out, MaskOut mo) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -66,7 +67,7 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   const int kk = k * k;
   const int P = k + (depth - 1) * kk;
   const int Ppow = next_pow2(P);
-  const int nsort = Ppow > 2 * kBuildThreads ? Ppow : 2 * kBuildThreads;
+  const int nsort = Ppow > 2 * NT ? Ppow : 2 * NT;
 
   griddep_wait();  // the row statistics come from the previous kernel
   griddep_launch_dependents();
@@ -82,24 +83,24 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     sm.cand_row = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
     sm.node_of = reinterpret_cast<int*>(p);      p += sizeof(int) * P;
     sm.frontier = reinterpret_cast<int*>(p);     p += sizeof(int) * 32;
-    sm.warp_cnt = reinterpret_cast<int*>(p);    p += sizeof(int) * kBuildWarps;
+    sm.warp_cnt = reinterpret_cast<int*>(p);    p += sizeof(int) * (NT / 32);
     sm.node_par = reinterpret_cast<int*>(p);     p += sizeof(int) * EAGLE_MAX_NODES;
     sm.node_dep = reinterpret_cast<int*>(p);
   }
 
   // 1. each row's children and their log-confidence lp = logit - lse (fp64)
-  for (int e = tid; e < R * k; e += kBuildThreads) {
+  for (int e = tid; e < R * k; e += NT) {
     const size_t g = (size_t)b * R * k + e;
     const int tok = row_tok_g[g];
     sm.row_tok[e] = tok;
     sm.row_lp[e] = tok >= 0 ? (double)row_val_g[g] - out.row_lse[(size_t)b * R + e / k] : -INFINITY;
   }
-  for (int c = tid; c < P; c += kBuildThreads) {
+  for (int c = tid; c < P; c += NT) {
     sm.cand_row[c] = -1;
     sm.node_of[c] = 0;
   }
   __syncthreads();
-  for (int c = tid; c < k; c += kBuildThreads) {
+  for (int c = tid; c < k; c += NT) {
     sm.cand_lv[c] = sm.row_lp[c];
     sm.cand_tok[c] = sm.row_tok[c];
     sm.cand_par[c] = -1;
@@ -111,9 +112,9 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   for (int level = 1; level < depth; ++level) {
     const int lo = level == 1 ? 0 : k + (level - 2) * kk;
     const int cnt = level == 1 ? k : kk;
-    for (int c = tid; c < cnt; c += kBuildThreads) sm.sort_k[c] = cand_key(sm.cand_lv[lo + c], lo + c);
+    for (int c = tid; c < cnt; c += NT) sm.sort_k[c] = cand_key(sm.cand_lv[lo + c], lo + c);
     __syncthreads();
-    for (int c = tid; c < cnt; c += kBuildThreads) {
+    for (int c = tid; c < cnt; c += NT) {
       const uint64_t mine = sm.sort_k[c];
       int rank = 0;
 #pragma unroll 8
@@ -125,7 +126,7 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     }
     __syncthreads();
     const int lo2 = k + (level - 1) * kk;
-    for (int idx = tid; idx < kk; idx += kBuildThreads) {
+    for (int idx = tid; idx < kk; idx += NT) {
       const int s = idx / k, r = idx - s * k;
       const int parent = sm.frontier[s];
       const int row = 1 + (level - 1) * k + s;
@@ -140,18 +141,18 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   // 3. rerank: bitonic sort of all candidate keys, best first; keep n.  With
   //    Ppow <= blockDim each thread holds one key: partners closer than 32 are
   //    exchanged by shuffles, farther ones through a double-buffered array.
-  if (Ppow <= kBuildThreads) {
+  if (Ppow <= NT) {
     uint64_t key = tid < P ? cand_key(sm.cand_lv[tid], tid) : 0ull;
     int buf = 0;
-    uint64_t* xbuf[2] = {sm.sort_k, sm.sort_k + kBuildThreads};
     for (int size = 2; size <= Ppow; size <<= 1) {
       const bool desc = (tid & size) == 0;
       for (int j = size >> 1; j > 0; j >>= 1) {
         uint64_t o;
         if (j >= 32) {
-          xbuf[buf][tid] = key;
+          uint64_t* xb = sm.sort_k + buf * NT;  // double-buffered exchange array
+          xb[tid] = key;
           __syncthreads();
-          o = xbuf[buf][tid ^ j];
+          o = xb[tid ^ j];
           buf ^= 1;
         } else {
           o = __shfl_xor_sync(kFull, key, j);
@@ -162,11 +163,11 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     }
     if (tid < n) sm.node_of[key_gid(key)] = 1;
   } else {
-    for (int i = tid; i < Ppow; i += kBuildThreads) sm.sort_k[i] = i < P ? cand_key(sm.cand_lv[i], i) : 0ull;
+    for (int i = tid; i < Ppow; i += NT) sm.sort_k[i] = i < P ? cand_key(sm.cand_lv[i], i) : 0ull;
     __syncthreads();
     for (int size = 2; size <= Ppow; size <<= 1) {
       for (int j = size >> 1; j > 0; j >>= 1) {
-        for (int i = tid; i < Ppow; i += kBuildThreads) {
+        for (int i = tid; i < Ppow; i += NT) {
           const int o = i ^ j;
           if (o > i) {
             const uint64_t a = sm.sort_k[i], c = sm.sort_k[o];
@@ -177,12 +178,12 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
         __syncthreads();
       }
     }
-    for (int i = tid; i < n; i += kBuildThreads) sm.node_of[key_gid(sm.sort_k[i])] = 1;
+    for (int i = tid; i < n; i += NT) sm.node_of[key_gid(sm.sort_k[i])] = 1;
   }
   __syncthreads();
 
   // 4. renumber kept candidates by ascending id (block scan over contiguous ranges)
-  const int per = (P + kBuildThreads - 1) / kBuildThreads;
+  const int per = (P + NT - 1) / NT;
   const int g0 = min(P, tid * per), g1 = min(P, g0 + per);
   int local = 0;
   for (int g = g0; g < g1; ++g) local += sm.node_of[g];
@@ -201,7 +202,7 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     if (sm.node_of[g]) sm.node_of[g] = ++next;
   __syncthreads();
 
-  for (int g = tid; g < P; g += kBuildThreads) {
+  for (int g = tid; g < P; g += NT) {
     const int node = sm.node_of[g];
     if (!node) continue;
     const size_t o = (size_t)b * n + (node - 1);
@@ -219,7 +220,7 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   if (mo.mask == nullptr) return;
   // 5. (fused mask) node i+1 sees itself and its ancestors: walk the parent chain
   __syncthreads();
-  for (int i = tid; i < n; i += kBuildThreads) {
+  for (int i = tid; i < n; i += NT) {
     uint64_t w0 = 0, w1 = 0;
     int node = i + 1;
     for (int step = 0; step < n && node >= 1; ++step) {
@@ -234,11 +235,16 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   }
 }
 
+// Block size of the expansion: 512 threads while the rerank's keys fit one per
+// thread (block barriers cost less with fewer warps), else 1024.
+static int build_threads(int P) { return next_pow2(P) <= 512 ? 512 : kBuildThreads; }
+
 size_t tree_build_smem_bytes(int R, int k, int P) {
+  const int nt = build_threads(P);
   const int Ppow = next_pow2(P);
-  const int nsort = Ppow > 2 * kBuildThreads ? Ppow : 2 * kBuildThreads;
+  const int nsort = Ppow > 2 * nt ? Ppow : 2 * nt;
   return sizeof(double) * ((size_t)R * k + P) + sizeof(uint64_t) * nsort +
-         sizeof(int) * ((size_t)R * k + 4 * (size_t)P + 32 + kBuildWarps + 2 * EAGLE_MAX_NODES);
+         sizeof(int) * ((size_t)R * k + 4 * (size_t)P + 32 + nt / 32 + 2 * EAGLE_MAX_NODES);
 }
 
 // workspace: [chunk stats][chunk keys][row tokens B*R*k int32][row logits B*R*k float]
@@ -262,11 +268,17 @@ cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R,
   if (e != cudaSuccess) return e;
   const int P = k + (depth - 1) * k * k;
   const size_t smem = tree_build_smem_bytes(R, k, P);
-  e = ensure_smem_limit((const void*)tree_expand_kernel, smem);
-  if (e != cudaSuccess) return e;
   const MaskOut mo = mo_in ? *mo_in : MaskOut{nullptr, nullptr, nullptr};
-  return launch_kernel(tree_expand_kernel, dim3(B), dim3(kBuildThreads), smem, s, pdl, ro.tok, ro.val, R, depth, k,
-                       n, out, mo);
+  if (build_threads(P) == 512) {
+    e = ensure_smem_limit((const void*)tree_expand_kernel<512>, smem);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(tree_expand_kernel<512>, dim3(B), dim3(512), smem, s, pdl, ro.tok, ro.val, R, depth, k,
+                         n, out, mo);
+  }
+  e = ensure_smem_limit((const void*)tree_expand_kernel<kBuildThreads>, smem);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(tree_expand_kernel<kBuildThreads>, dim3(B), dim3(kBuildThreads), smem, s, pdl, ro.tok, ro.val,
+                       R, depth, k, n, out, mo);
 }
 
 }  // namespace eagle
