@@ -235,9 +235,13 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   }
 }
 
-// Block size of the expansion: 512 threads while the rerank's keys fit one per
-// thread (block barriers cost less with fewer warps), else 1024.
-static int build_threads(int P) { return next_pow2(P) <= 512 ? 512 : kBuildThreads; }
+// Block size of the expansion: the rerank's key count rounded to a power of
+// two (one key per thread; block barriers cost less with fewer warps),
+// between 128 and 1024 threads.
+static int build_threads(int P) {
+  const int p = next_pow2(P);
+  return p < 128 ? 128 : (p > kBuildThreads ? kBuildThreads : p);
+}
 
 size_t tree_build_smem_bytes(int R, int k, int P) {
   const int nt = build_threads(P);
@@ -269,16 +273,17 @@ cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R,
   const int P = k + (depth - 1) * k * k;
   const size_t smem = tree_build_smem_bytes(R, k, P);
   const MaskOut mo = mo_in ? *mo_in : MaskOut{nullptr, nullptr, nullptr};
-  if (build_threads(P) == 512) {
-    e = ensure_smem_limit((const void*)tree_expand_kernel<512>, smem);
-    if (e != cudaSuccess) return e;
-    return launch_kernel(tree_expand_kernel<512>, dim3(B), dim3(512), smem, s, pdl, ro.tok, ro.val, R, depth, k,
-                         n, out, mo);
+  auto go = [&](auto kernel, int nt) -> cudaError_t {
+    cudaError_t e2 = ensure_smem_limit((const void*)kernel, smem);
+    if (e2 != cudaSuccess) return e2;
+    return launch_kernel(kernel, dim3(B), dim3(nt), smem, s, pdl, ro.tok, ro.val, R, depth, k, n, out, mo);
+  };
+  switch (build_threads(P)) {
+    case 128: return go(tree_expand_kernel<128>, 128);
+    case 256: return go(tree_expand_kernel<256>, 256);
+    case 512: return go(tree_expand_kernel<512>, 512);
+    default: return go(tree_expand_kernel<kBuildThreads>, kBuildThreads);
   }
-  e = ensure_smem_limit((const void*)tree_expand_kernel<kBuildThreads>, smem);
-  if (e != cudaSuccess) return e;
-  return launch_kernel(tree_expand_kernel<kBuildThreads>, dim3(B), dim3(kBuildThreads), smem, s, pdl, ro.tok, ro.val,
-                       R, depth, k, n, out, mo);
 }
 
 }  // namespace eagle
