@@ -22,6 +22,9 @@ Everything is plain numpy in fp64, written step by step from the pages:
                 resampling (EAGLE-2 "Well-Calibrated Draft Model" formula;
                 aivaro.ru EAGLE-3 answer, section 4 steps 3-4; EAGLE-4
                 write-up, same section as the mask).
+* ``kv``        after acceptance: the accepted path's keys and values are
+                appended to the prefix cache, the rejected ones dropped (EAGLE-4
+                write-up, same section).
 
 Pins (tests/test_oracle_*.py) tie each function to something other than
 itself: hand-worked fixtures, closed forms, library routines on special cases,
@@ -34,3 +37,4 @@ from .tree import build_tree, build_trees  # noqa: F401
 from .mask import ancestor_mask, pack_mask, positions  # noqa: F401
 from .attention import tree_attention, tree_attention_rows  # noqa: F401
 from .accept import accept_greedy, accept_stochastic, inverse_cdf  # noqa: F401
+from .kv import compact_kv  # noqa: F401
