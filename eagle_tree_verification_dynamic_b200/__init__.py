@@ -16,8 +16,13 @@ from ._lib import (  # noqa: F401
     alloc_tree,
     attention_workspace_bytes,
     exported_names,
+    kv_compact,
+    kv_compact_into,
     lib,
     pool_size,
+    step_in,
+    step_into,
+    step_workspace_bytes,
     row_stats,
     tree_attention,
     tree_attention_into,

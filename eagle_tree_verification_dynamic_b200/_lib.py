@@ -68,6 +68,8 @@ _SIGS = {
     "eagle_verify_step_attention_status_offset": (_c_sz, [ctypes.POINTER(StepIn)]),
     "eagle_verify_step": (_c_i, [ctypes.POINTER(StepIn), ctypes.POINTER(StepOut), ctypes.POINTER(_c_i), _c_p,
                                  _c_sz, _c_p]),
+    "eagle_kv_compact": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
+                                _c_p]),
     "eagle_accept_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
     "eagle_accept": (_c_i, [_c_p, _c_i, _c_p, _c_i, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i,
                             _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
@@ -329,3 +331,22 @@ def step_attention_status(si: StepIn, ws: torch.Tensor):
     """Read the attention's device status word from a step workspace (synchronises)."""
     off = lib().eagle_verify_step_attention_status_offset(ctypes.byref(si))
     check_attention_status(ws[off:])
+
+
+# ------------------------------------------------------- KV-cache compaction
+def kv_compact_into(k_tree, v_tree, path, accepted_len, prefix_len, k_cache, v_cache, new_prefix_len):
+    """Append the accepted path's tree keys/values to the caches (in place); new lengths into new_prefix_len."""
+    B, n, Hkv, D = k_tree.shape
+    Lmax, depth = k_cache.shape[2], path.shape[1]
+    _check(lib().eagle_kv_compact(_ptr(k_tree), _ptr(v_tree), _ptr(path), _ptr(accepted_len), _ptr(prefix_len),
+                                  _ptr(k_cache), _ptr(v_cache), _ptr(new_prefix_len), B, n, Hkv, D, Lmax, depth,
+                                  _stream(k_tree.device)), "eagle_kv_compact")
+
+
+def kv_compact(k_tree, v_tree, path, accepted_len, prefix_len, k_cache, v_cache) -> torch.Tensor:
+    """k_tree / v_tree [B][n][Hkv][D] bf16, path [B][depth], accepted_len [B], prefix_len [B] int32,
+    caches [B][Hkv][Lmax][D] bf16 (updated in place) -> new prefix lengths [B] int32."""
+    _need_cuda(k_tree, v_tree, path, accepted_len, prefix_len, k_cache, v_cache)
+    new_len = torch.empty_like(prefix_len)
+    kv_compact_into(k_tree, v_tree, path, accepted_len, prefix_len, k_cache, v_cache, new_len)
+    return new_len

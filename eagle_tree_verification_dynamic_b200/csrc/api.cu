@@ -191,6 +191,21 @@ eagle_status eagle_accept(const void* target_logits, int target_dtype, const voi
                                    workspace, static_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------ KV-cache compaction
+eagle_status eagle_kv_compact(const void* k_tree, const void* v_tree, const int32_t* path,
+                              const int32_t* accepted_len, const int32_t* prefix_len, void* k_cache, void* v_cache,
+                              int32_t* new_prefix_len, int B, int n, int Hkv, int D, int Lmax, int depth,
+                              void* stream) {
+  if (!k_tree || !v_tree || !path || !accepted_len || !prefix_len || !k_cache || !v_cache || !new_prefix_len)
+    return EAGLE_ERR_NULL;
+  if (B <= 0 || n <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0 || depth <= 0) return EAGLE_ERR_SHAPE;
+  if (D % 8 != 0 || new_prefix_len == prefix_len) return EAGLE_ERR_SHAPE;
+  if (n > EAGLE_MAX_NODES || depth > EAGLE_MAX_DEPTH || B > 65535) return EAGLE_ERR_LIMIT;
+  if (!aligned16(k_tree) || !aligned16(v_tree) || !aligned16(k_cache) || !aligned16(v_cache)) return EAGLE_ERR_ALIGN;
+  return cuda_status(launch_kv_compact(k_tree, v_tree, path, accepted_len, prefix_len, k_cache, v_cache,
+                                       new_prefix_len, B, n, Hkv, D, Lmax, depth, static_cast<cudaStream_t>(stream)));
+}
+
 // ------------------------------------------------------------ whole step
 }  // extern "C"
 

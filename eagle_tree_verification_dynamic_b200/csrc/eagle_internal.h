@@ -100,6 +100,11 @@ cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc,
                                   const int32_t* pos, int B, int n, int Hq, int Hkv, int D, int window,
                                   float scale, void* out, void* ws, cudaStream_t s);
 
+// ---- KV-cache compaction after acceptance (kv_compact.cu)
+cudaError_t launch_kv_compact(const void* k_tree, const void* v_tree, const int32_t* path, const int32_t* accepted_len,
+                              const int32_t* prefix_len, void* k_cache, void* v_cache, int32_t* new_len, int B, int n,
+                              int Hkv, int D, int Lmax, int depth, cudaStream_t s);
+
 // ---- accept (accept.cu)
 size_t accept_ws_bytes(int B, int n, int V, int dtype);
 int accept_max_vocab(int dtype);  // largest V the sampled walk supports

@@ -220,6 +220,28 @@ EAGLE_API eagle_status eagle_accept(const void* target_logits, int target_dtype,
                           int B, int n, int V, int depth, int32_t* accepted_len, int32_t* path,
                           int32_t* bonus, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------- KV-cache compaction
+ * After acceptance ("Технический анализ EAGLE-4", section "Деревья проверки
+ * EAGLE-4 и утилита управления": the accepted continuation is kept, the
+ * rejected KV-cache entries are freed): the keys and values that the
+ * verification pass computed for the accepted nodes are appended to each
+ * sequence's prefix cache in path order, the i-th accepted node (depth i+1)
+ * at position prefix_len[b] + i, which is its position id; rejected nodes are
+ * not copied (the bonus token has no key or value yet).
+ *   k_tree, v_tree [B][n][Hkv][D] bf16 (the tree's keys and values)
+ *   path [B][depth], accepted_len [B] (from eagle_accept; node ids 1..n)
+ *   prefix_len [B] (clamped to [0, Lmax])
+ *   k_cache, v_cache [B][Hkv][Lmax][D] bf16, updated in place
+ *   new_prefix_len [B] int32 (must not be prefix_len itself): prefix_len plus
+ *     the entries copied.  The copy ends at the first path entry that is not a
+ *     node id in 1..n or whose position would reach Lmax.
+ * Limits: n <= EAGLE_MAX_NODES, depth <= EAGLE_MAX_DEPTH, B <= 65535, D % 8 ==
+ * 0, tensor pointers 16-byte aligned.  No workspace. */
+EAGLE_API eagle_status eagle_kv_compact(const void* k_tree, const void* v_tree, const int32_t* path,
+                                        const int32_t* accepted_len, const int32_t* prefix_len, void* k_cache,
+                                        void* v_cache, int32_t* new_prefix_len, int B, int n, int Hkv, int D,
+                                        int Lmax, int depth, void* stream);
+
 /* ---------------------------------------------------------- one whole step
  * One verification step in its order: build (eagle_tree_build), mask and
  * position ids (fused into the build's expansion kernel), tree attention

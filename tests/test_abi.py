@@ -161,3 +161,16 @@ def test_step_validation(lib):
     assert call(si=_step_in(q=ctypes.c_void_p(0x1008))) == 6
     assert call(ws=None, wsb=0) == 5
     assert n.value == 0  # nothing was reported: every call above failed validation
+
+
+def test_kv_compact_validation(lib):
+    def call(**kw):
+        return lib.eagle_kv_compact(kw.get("kt", FAKE), FAKE, FAKE, FAKE, kw.get("plen", FAKE), FAKE, FAKE,
+                                    kw.get("out", ctypes.c_void_p(0x2000)), 1, kw.get("n", 10), 8,
+                                    kw.get("D", 128), 2048, kw.get("depth", 6), None)
+    assert call(kt=None) == 1
+    assert call(D=100) == 2                                   # D % 8 != 0
+    assert call(plen=ctypes.c_void_p(0x2000)) == 2           # in-place length update is refused
+    assert call(n=129) == 4
+    assert call(depth=17) == 4
+    assert call(kt=ctypes.c_void_p(0x1008)) == 6
