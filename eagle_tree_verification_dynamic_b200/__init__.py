@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     F32,
     EagleError,
     Tree,
+    TreeGrower,
     accept,
     accept_into,
     accept_workspace_bytes,

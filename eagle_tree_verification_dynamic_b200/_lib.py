@@ -68,6 +68,11 @@ _SIGS = {
     "eagle_verify_step_attention_status_offset": (_c_sz, [ctypes.POINTER(StepIn)]),
     "eagle_verify_step": (_c_i, [ctypes.POINTER(StepIn), ctypes.POINTER(StepOut), ctypes.POINTER(_c_i), _c_p,
                                  _c_sz, _c_p]),
+    "eagle_tree_grow_state_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
+    "eagle_tree_grow_begin": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p, _c_p]),
+    "eagle_tree_grow_level": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p, _c_p]),
+    "eagle_tree_grow_finish": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, ctypes.POINTER(TreeStruct),
+                                      ctypes.POINTER(_c_i), _c_p]),
     "eagle_kv_compact": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                 _c_p]),
     "eagle_accept_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
@@ -350,3 +355,41 @@ def kv_compact(k_tree, v_tree, path, accepted_len, prefix_len, k_cache, v_cache)
     new_len = torch.empty_like(prefix_len)
     kv_compact_into(k_tree, v_tree, path, accepted_len, prefix_len, k_cache, v_cache, new_len)
     return new_len
+
+
+# ---------------------------------------------------- tree grown per level
+class TreeGrower:
+    """The build one level at a time: begin(root rows [B][V]) and level(rows [B][k][V], level) each return the
+    new frontier (tokens [B][k], parent slots [B][k]); finish(m) returns the Tree (equal to tree_build on the
+    same rows)."""
+
+    def __init__(self, B: int, V: int, depth: int, k: int, dtype: torch.dtype, device):
+        self.B, self.V, self.depth, self.k = B, V, depth, k
+        self.dt = F32 if dtype == torch.float32 else BF16
+        self.device = torch.device(device)
+        nb = lib().eagle_tree_grow_state_bytes(B, V, self.dt, depth, k)
+        self.state = _workspace(nb, self.device)
+        self.ftok = torch.empty(B, k, dtype=torch.int32, device=self.device)
+        self.fpar = torch.empty(B, k, dtype=torch.int32, device=self.device)
+
+    def begin(self, root_logits: torch.Tensor):
+        _check(lib().eagle_tree_grow_begin(_ptr(root_logits), self.dt, self.B, self.V, self.depth, self.k,
+                                           _ptr(self.state), self.state.numel(), _ptr(self.ftok), _ptr(self.fpar),
+                                           _stream(self.device)), "eagle_tree_grow_begin")
+        return self.ftok, self.fpar
+
+    def level(self, level_logits: torch.Tensor, level: int):
+        _check(lib().eagle_tree_grow_level(_ptr(level_logits), self.dt, self.B, self.V, self.depth, self.k, level,
+                                           _ptr(self.state), self.state.numel(), _ptr(self.ftok), _ptr(self.fpar),
+                                           _stream(self.device)), "eagle_tree_grow_level")
+        return self.ftok, self.fpar
+
+    def finish(self, m: int) -> Tree:
+        R = 1 + (self.depth - 1) * self.k
+        tree = alloc_tree(self.B, R, self.depth, self.k, m, self.device)
+        st = tree.struct()
+        n_out = _c_i(0)
+        _check(lib().eagle_tree_grow_finish(self.dt, self.B, self.V, self.depth, self.k, m, _ptr(self.state),
+                                            self.state.numel(), ctypes.byref(st), ctypes.byref(n_out),
+                                            _stream(self.device)), "eagle_tree_grow_finish")
+        return tree

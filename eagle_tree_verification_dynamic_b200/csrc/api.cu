@@ -32,6 +32,13 @@ cudaError_t ensure_smem_limit(const void* kernel, size_t bytes) {
 namespace {
 
 thread_local char g_cuda_err[256] = "";
+eagle_status cuda_status(cudaError_t e);
+
+}  // namespace
+
+eagle_status eagle::report_cuda(cudaError_t e) { return cuda_status(e); }
+
+namespace {
 
 eagle_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return EAGLE_OK;

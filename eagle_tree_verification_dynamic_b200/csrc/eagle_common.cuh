@@ -105,6 +105,18 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
+// Ranking key of a candidate: the order-preserving bit image of its fp64
+// log V with the lowest 12 mantissa bits replaced by (4095 - id), so that a
+// larger key means a larger log V and, among equal values, a lower id.  Two
+// values that differ only in those 12 bits (relative gap < 2^-40) rank by id.
+__device__ __forceinline__ uint64_t cand_key(double lv, int gid) {
+  uint64_t u = (uint64_t)__double_as_longlong(lv);
+  if (u == 0x8000000000000000ull) u = 0;  // -0 ranks with +0
+  u = (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
+  return (u & ~0xfffull) | (uint64_t)(4095 - gid);
+}
+__device__ __forceinline__ int key_gid(uint64_t key) { return 4095 - (int)(key & 0xfffull); }
+
 // ------------------------------------------------------- scaled exp partials
 // Partial sum of one chunk: acc = sum 2^(x*log2e - e_ref), e_ref an integer
 // (as float; -inf when the chunk held no finite term).

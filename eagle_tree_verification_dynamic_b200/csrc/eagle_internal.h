@@ -51,11 +51,16 @@ struct RowOut {
   double* lse;   // [rows] log-sum-exp
 };
 ChunkPlan plan_chunks(long long rows, int V, int elem_bytes);
-size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k);
+// plan_rows > 0: cut rows into chunks as a sweep of plan_rows rows would (the
+// chunking fixes the order of the log-sum-exp's fp64 partial sums).
+size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k, long long plan_rows = 0);
 // zero_tickets: clear the per-row tickets first (else the caller already has);
 // pdl: chain the kernel to its predecessor with programmatic dependent launch.
 cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, int k, bool lse, const RowOut& out,
-                             void* ws, cudaStream_t s, bool zero_tickets = true, bool pdl = false);
+                             void* ws, cudaStream_t s, bool zero_tickets = true, bool pdl = false,
+                             long long plan_rows = 0);
+// CUDA error -> status, recording the error text for eagle_last_cuda_error.
+eagle_status report_cuda(cudaError_t e);
 // Byte range of the per-row tickets inside the row-sweep workspace.
 void row_stats_tickets_span(long long rows, int V, int elem_bytes, int k, size_t* off, size_t* bytes);
 
@@ -73,6 +78,11 @@ struct MaskOut {
 cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k, int n,
                               const eagle_tree_t& out, void* ws, cudaStream_t s, const MaskOut* mo = nullptr,
                               bool zero_tickets = true, bool pdl = false);
+
+// The expansion / rerank alone, from each row's top-k tokens and logits
+// [B][R][k] and out.row_lse [B][R] (the build's second kernel).
+cudaError_t launch_tree_expand(const int32_t* row_tok, const float* row_val, int B, int R, int depth, int k, int n,
+                               const eagle_tree_t& out, const MaskOut* mo, bool pdl, cudaStream_t s);
 
 // ---- tree mask (tree_mask.cu)
 cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len,

@@ -276,8 +276,8 @@ ChunkPlan plan_chunks(long long rows, int V, int elem_bytes) {
 }
 
 // workspace: [chunk stats rows*nc][chunk keys rows*nc*k][row tickets rows]
-size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k) {
-  const ChunkPlan p = plan_chunks(rows, V, elem_bytes);
+size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k, long long plan_rows) {
+  const ChunkPlan p = plan_chunks(plan_rows > 0 ? plan_rows : rows, V, elem_bytes);
   const size_t n = (size_t)rows * p.n_chunks;
   return align_up(n * sizeof(ChunkStat), 256) + align_up(n * k * sizeof(uint64_t), 256) +
          align_up((size_t)rows * sizeof(int), 256);
@@ -316,9 +316,9 @@ void row_stats_tickets_span(long long rows, int V, int elem_bytes, int k, size_t
 }
 
 cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, int k, bool lse, const RowOut& out,
-                             void* ws, cudaStream_t s, bool zero_tickets, bool pdl) {
+                             void* ws, cudaStream_t s, bool zero_tickets, bool pdl, long long plan_rows) {
   const int eb = dtype_bytes(dtype);
-  const ChunkPlan p = plan_chunks(rows, V, eb);
+  const ChunkPlan p = plan_chunks(plan_rows > 0 ? plan_rows : rows, V, eb);
   const size_t n = (size_t)rows * p.n_chunks;
   char* base = static_cast<char*>(ws);
   ChunkStat* stats = reinterpret_cast<ChunkStat*>(base);

@@ -21,18 +21,6 @@ namespace eagle {
 constexpr int kBuildThreads = 1024;
 constexpr int kBuildWarps = kBuildThreads / 32;
 
-// Ranking key of a candidate: the order-preserving bit image of its fp64
-// log V with the lowest 12 mantissa bits replaced by (4095 - id), so that a
-// larger key means a larger log V and, among equal values, a lower id.  Two
-// values that differ only in those 12 bits (relative gap < 2^-40) rank by id.
-__device__ __forceinline__ uint64_t cand_key(double lv, int gid) {
-  uint64_t u = (uint64_t)__double_as_longlong(lv);
-  if (u == 0x8000000000000000ull) u = 0;  // -0 ranks with +0
-  u = (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
-  return (u & ~0xfffull) | (uint64_t)(4095 - gid);
-}
-__device__ __forceinline__ int key_gid(uint64_t key) { return 4095 - (int)(key & 0xfffull); }
-
 struct BuildSmem {
   double* row_lp;    // [R*k] log-confidence of each row's top-k children
   double* cand_lv;   // [P]   log V
@@ -258,6 +246,24 @@ size_t tree_build_ws_bytes(int B, int R, int V, int elem_bytes, int k) {
          align_up(rows * k * sizeof(float), 256);
 }
 
+cudaError_t launch_tree_expand(const int32_t* row_tok, const float* row_val, int B, int R, int depth, int k, int n,
+                               const eagle_tree_t& out, const MaskOut* mo_in, bool pdl, cudaStream_t s) {
+  const int P = k + (depth - 1) * k * k;
+  const size_t smem = tree_build_smem_bytes(R, k, P);
+  const MaskOut mo = mo_in ? *mo_in : MaskOut{nullptr, nullptr, nullptr};
+  auto go = [&](auto kernel, int nt) -> cudaError_t {
+    cudaError_t e2 = ensure_smem_limit((const void*)kernel, smem);
+    if (e2 != cudaSuccess) return e2;
+    return launch_kernel(kernel, dim3(B), dim3(nt), smem, s, pdl, row_tok, row_val, R, depth, k, n, out, mo);
+  };
+  switch (build_threads(P)) {
+    case 128: return go(tree_expand_kernel<128>, 128);
+    case 256: return go(tree_expand_kernel<256>, 256);
+    case 512: return go(tree_expand_kernel<512>, 512);
+    default: return go(tree_expand_kernel<kBuildThreads>, kBuildThreads);
+  }
+}
+
 cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k, int n,
                               const eagle_tree_t& out, void* ws, cudaStream_t s, const MaskOut* mo_in,
                               bool zero_tickets, bool pdl) {
@@ -270,20 +276,7 @@ cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R,
   ro.lse = out.row_lse;
   cudaError_t e = launch_row_stats(draft_logits, dtype, rows, V, k, true, ro, ws, s, zero_tickets, pdl);
   if (e != cudaSuccess) return e;
-  const int P = k + (depth - 1) * k * k;
-  const size_t smem = tree_build_smem_bytes(R, k, P);
-  const MaskOut mo = mo_in ? *mo_in : MaskOut{nullptr, nullptr, nullptr};
-  auto go = [&](auto kernel, int nt) -> cudaError_t {
-    cudaError_t e2 = ensure_smem_limit((const void*)kernel, smem);
-    if (e2 != cudaSuccess) return e2;
-    return launch_kernel(kernel, dim3(B), dim3(nt), smem, s, pdl, ro.tok, ro.val, R, depth, k, n, out, mo);
-  };
-  switch (build_threads(P)) {
-    case 128: return go(tree_expand_kernel<128>, 128);
-    case 256: return go(tree_expand_kernel<256>, 256);
-    case 512: return go(tree_expand_kernel<512>, 512);
-    default: return go(tree_expand_kernel<kBuildThreads>, kBuildThreads);
-  }
+  return launch_tree_expand(ro.tok, ro.val, B, R, depth, k, n, out, mo_in, pdl, s);
 }
 
 }  // namespace eagle

@@ -220,6 +220,36 @@ EAGLE_API eagle_status eagle_accept(const void* target_logits, int target_dtype,
                           int B, int n, int V, int depth, int32_t* accepted_len, int32_t* path,
                           int32_t* bonus, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------- tree grown one level at a time
+ * The build of eagle_tree_build for a draft model that produces each level's
+ * distributions only once it knows the frontier ("EAGLE" notes, EAGLE-2
+ * "Expansion of tree", "Reranking Nodes").  On one stream:
+ *   eagle_tree_grow_begin(root_logits [B][V])      row 0; writes the level-1
+ *     frontier: frontier_tokens [B][k] (slot order), frontier_parents [B][k]
+ *     (-1: the root);
+ *   eagle_tree_grow_level(level_logits [B][k][V], level = 2..depth): row s is
+ *     the distribution after frontier slot s of the previous level (draft row
+ *     1 + (level-2)k + s of eagle_tree_build); writes the level's frontier
+ *     (tokens, and each one's parent as a slot of the previous frontier) while
+ *     level < depth;
+ *   eagle_tree_grow_finish(m, out): the tree, equal bit for bit to
+ *     eagle_tree_build on the same rows (same kernels, same fp64 log V, the
+ *     rows' log-sum-exps summed in the same order).
+ * frontier pointers may be NULL.  state: eagle_tree_grow_state_bytes bytes,
+ * 256-byte aligned, kept by the caller from begin to finish (it holds every
+ * row's top-k and log-sum-exp and the frontier's log V).  Limits: those of
+ * eagle_tree_build. */
+EAGLE_API size_t eagle_tree_grow_state_bytes(int B, int V, int dtype, int depth, int k);
+EAGLE_API eagle_status eagle_tree_grow_begin(const void* root_logits, int dtype, int B, int V, int depth, int k,
+                                             void* state, size_t state_bytes, int32_t* frontier_tokens,
+                                             int32_t* frontier_parents, void* stream);
+EAGLE_API eagle_status eagle_tree_grow_level(const void* level_logits, int dtype, int B, int V, int depth, int k,
+                                             int level, void* state, size_t state_bytes, int32_t* frontier_tokens,
+                                             int32_t* frontier_parents, void* stream);
+EAGLE_API eagle_status eagle_tree_grow_finish(int dtype, int B, int V, int depth, int k, int m, void* state,
+                                              size_t state_bytes, const eagle_tree_t* out, int* n_nodes,
+                                              void* stream);
+
 /* ------------------------------------------------- KV-cache compaction
  * After acceptance ("Технический анализ EAGLE-4", section "Деревья проверки
  * EAGLE-4 и утилита управления": the accepted continuation is kept, the

@@ -84,10 +84,14 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
     # level 1: the root's k children
     level_cands = [make(0, r, r, 1, None) for r in range(k)]
     all_cands += level_cands
+    frontiers: List[dict] = []    # per expanded level: the k tokens by slot and their parents' slots
     for level in range(2, depth + 1):
         ranked = sorted(level_cands, key=_sort_key)
         _flag_adjacent(ranked, k, "frontier", level - 1, near_ties)
         frontier = ranked[:k]
+        frontiers.append({"tokens": np.array([c["token"] for c in frontier], dtype=np.int64),
+                          "parent_slot": np.array([-1 if c["pnode"] is None else c["pnode"]["slot"]
+                                                   for c in frontier], dtype=np.int64)})
         nxt = []
         off = k + (level - 2) * k * k
         for s, parent in enumerate(frontier):
@@ -118,7 +122,7 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
         draft_row[i + 1] = c["row"]
     return {"tokens": tokens, "parents": parents, "depth": depth_arr, "logV": logV,
             "gid": gid, "draft_row": draft_row, "row_lse": row_lse, "n": n, "P": P,
-            "near_ties": near_ties}
+            "frontiers": frontiers, "near_ties": near_ties}
 
 
 def build_trees(logits_b: np.ndarray, depth: int, k: int, m: int) -> List[Dict]:

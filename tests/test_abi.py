@@ -174,3 +174,23 @@ def test_kv_compact_validation(lib):
     assert call(n=129) == 4
     assert call(depth=17) == 4
     assert call(kt=ctypes.c_void_p(0x1008)) == 6
+
+
+def test_tree_grow_validation(lib):
+    nb = lib.eagle_tree_grow_state_bytes(2, 32000, 0, 6, 10)
+    assert nb > 0 and nb % 256 == 0
+    assert lib.eagle_tree_grow_state_bytes(2, 32000, 5, 6, 10) == 0
+    begin = lambda **kw: lib.eagle_tree_grow_begin(kw.get("x", FAKE), kw.get("dt", 0), 2, 32000, kw.get("depth", 6),
+                                                   kw.get("k", 10), kw.get("st", FAKE), kw.get("nb", nb), None, None,
+                                                   None)
+    assert begin(x=None) == 1
+    assert begin(dt=3) == 3
+    assert begin(k=33) == 4
+    assert begin(nb=nb - 1) == 5
+    assert begin(st=ctypes.c_void_p(0x1010)) == 5              # state not 256-byte aligned
+    lvl = lambda level: lib.eagle_tree_grow_level(FAKE, 0, 2, 32000, 6, 10, level, FAKE, nb, None, None, None)
+    assert lvl(1) == 2 and lvl(7) == 2
+    n = ctypes.c_int(0)
+    assert lib.eagle_tree_grow_finish(0, 2, 32000, 6, 10, 60, FAKE, nb, None, ctypes.byref(n), None) == 1
+    assert lib.eagle_tree_grow_finish(0, 2, 32000, 6, 10, 129, FAKE, nb, ctypes.byref(_tree()), ctypes.byref(n),
+                                      None) == 4

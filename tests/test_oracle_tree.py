@@ -167,3 +167,36 @@ def test_confident_draft_grows_deeper():
     sharp[:, 0] += 12.0
     assert oracle.build_tree(sharp, depth, k, m)["depth"].max() == depth
     assert oracle.build_tree(flat, depth, k, m)["depth"].max() <= 2
+
+
+def test_frontiers_brute_force():
+    """Each expanded level's frontier, by brute force: enumerate every root path
+    of that depth from the rows' softmax (children of the previous frontier
+    only), rank by the product of confidences, ties to the lower candidate id."""
+    cfg = get_config("tiny", V=40, depth=4, k=3, B=1, logits_dtype="f32")
+    x = gen_draft_logits(cfg, 11)[0].astype(np.float64)
+    k = cfg.k
+    t = oracle.build_tree(x, cfg.depth, k, 10**6)
+    p = softmax(x, axis=1)
+    # level 1: the root's children by probability, ties to the lower token
+    order = sorted(range(x.shape[1]), key=lambda v: (-p[0, v], v))[:k]
+    front = [(p[0, v], r, v) for r, v in enumerate(order)]          # (V, gid, token)
+    for level in range(1, cfg.depth):
+        ranked = sorted(front, key=lambda c: (-c[0], c[1]))[:k]
+        got = t["frontiers"][level - 1]
+        assert got["tokens"].tolist() == [c[2] for c in ranked]
+        if level == 1:
+            assert got["parent_slot"].tolist() == [-1] * k
+        else:
+            assert got["parent_slot"].tolist() == [(c[1] - k - (level - 2) * k * k) // k for c in ranked]
+        nxt = []
+        for s, (v, _, _) in enumerate(ranked):
+            row = 1 + (level - 1) * k + s
+            kids = sorted(range(x.shape[1]), key=lambda u: (-p[row, u], u))[:k]
+            nxt += [(v * p[row, u], k + (level - 1) * k * k + s * k + r, u) for r, u in enumerate(kids)]
+        front = nxt
+    # with every candidate kept, frontier slot s of level l is the node owning row 1 + (l-1)k + s
+    for level, f in enumerate(t["frontiers"], start=1):
+        for s, tok in enumerate(f["tokens"]):
+            node = int(np.nonzero(t["draft_row"][1:] == 1 + (level - 1) * k + s)[0][0])
+            assert t["tokens"][node] == tok and t["depth"][node] == level
