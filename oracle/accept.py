@@ -35,6 +35,12 @@ Readings:
     rejection leaves max(0, p - q) identically zero (only possible when
     p == q, which accepts for every u < 1) the walk stops there and the bonus
     is the target argmax of that node.
+  * Sampling without replacement (the pages are silent; the counterpart of the
+    rule above for siblings that are distinct tokens, as the top-k children of
+    a draft row always are): a rejected child's token can no longer be drawn,
+    so after the residual step q <- q with q(x_c) = 0, renormalised.  Accept,
+    residual and bonus are otherwise as above; with one child per node the two
+    rules coincide.
 """
 from __future__ import annotations
 
@@ -91,8 +97,16 @@ def accept_greedy(target: np.ndarray, tokens, parents, max_depth: int) -> Dict:
             "bonus": bonus, "stop": j, "near_ties": []}
 
 
+def _without(q: np.ndarray, x: int):
+    """q with token x removed and the rest renormalised.  None when nothing is left."""
+    q = q.copy()
+    q[x] = 0.0
+    S = q.sum()
+    return q / S if S > 0.0 else None
+
+
 def accept_stochastic(target: np.ndarray, draft: np.ndarray, tokens, parents, draft_row,
-                      uniforms: np.ndarray, max_depth: int) -> Dict:
+                      uniforms: np.ndarray, max_depth: int, without_replacement: bool = False) -> Dict:
     target = np.asarray(target, dtype=np.float64)
     draft = np.asarray(draft, dtype=np.float64)
     tokens = np.asarray(tokens)
@@ -127,6 +141,12 @@ def accept_stochastic(target: np.ndarray, draft: np.ndarray, tokens, parents, dr
                     degenerate = True
                     break
                 p = p_new
+                if without_replacement:
+                    q = _without(q, x)
+                    if q is None:
+                        ties.append({"kind": "degenerate", "node": c})
+                        degenerate = True
+                        break
         if not moved:
             break
     if degenerate:

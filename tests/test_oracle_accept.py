@@ -121,6 +121,76 @@ def test_sigma0_closed_forms(name):
     assert s["bonus"] == int(np.searchsorted(c, u[1, leaf] * c[-1], side="right"))
 
 
+@pytest.mark.parametrize("case", [0, 1])
+@pytest.mark.parametrize("rule", ["with_replacement", "without_replacement"])
+def test_handworked_without_replacement(golden_dir, case, rule):
+    with open(os.path.join(golden_dir, "accept_without_replacement_handworked.json")) as f:
+        fx = json.load(f)
+    c = fx["cases"][case]
+    r = oracle.accept_stochastic(np.log(np.array(fx["target_probs"])), np.log(np.array(fx["draft_probs"])),
+                                 fx["tokens"], fx["parents"], fx["draft_row"], np.array([c["u_acc"], c["u_res"]]),
+                                 2, without_replacement=rule == "without_replacement")
+    assert (r["accepted_len"], r["path"], r["bonus"]) == tuple(c[rule][f] for f in ("accepted_len", "path", "bonus"))
+
+
+def test_one_child_per_node_rules_coincide():
+    """With a single child per node nothing is drawn after a rejection, so both rules agree."""
+    cfg = get_config("tiny", k=1, depth=4, m=3, V=50, B=1, logits_dtype="f32")
+    draft = oracle.decode_logits(gen_draft_logits(cfg, 4), "f32")[0]
+    t = oracle.build_tree(draft, cfg.depth, cfg.k, cfg.m)
+    target = make_target_logits(cfg, 4, gen_draft_logits(cfg, 4), t["draft_row"][None])[0].astype(np.float64)
+    for s in range(40):
+        u = gen_uniforms(cfg, s)[0].astype(np.float64)
+        a = oracle.accept_stochastic(target, draft, t["tokens"], t["parents"], t["draft_row"], u, cfg.depth)
+        b = oracle.accept_stochastic(target, draft, t["tokens"], t["parents"], t["draft_row"], u, cfg.depth,
+                                     without_replacement=True)
+        assert (a["accepted_len"], a["path"], a["bonus"]) == (b["accepted_len"], b["path"], b["bonus"])
+
+
+def _draw_without_replacement(rng, q, count):
+    """`count` distinct tokens, each drawn from q restricted to the tokens not drawn yet."""
+    w = q.copy()
+    out = []
+    for _ in range(count):
+        c = np.cumsum(w)
+        x = min(int(np.searchsorted(c, rng.random() * c[-1], side="right")), q.shape[0] - 1)
+        out.append(x)
+        w[x] = 0.0
+    return np.array(out)
+
+
+def _chi2_first_token_distinct(trials, seed, rule_without):
+    """First emitted token over `trials` walks of a star of 3 distinct siblings
+    drawn without replacement from q; the walk uses the rule given."""
+    rng = np.random.default_rng(seed)
+    V = 8
+    p = rng.dirichlet(np.ones(V))
+    q = rng.dirichlet(np.ones(V) * 0.5)
+    other = np.log(rng.dirichlet(np.ones(V)))
+    parents = np.array([0, 0, 0])
+    draft_row = np.array([0, -1, -1, -1])
+    draft = np.log(q)[None]
+    target = np.stack([np.log(p), other, other, other])
+    counts = np.zeros(V, dtype=np.int64)
+    for _ in range(trials):
+        toks = _draw_without_replacement(rng, q, 3)
+        u = rng.random((2, 4)).astype(np.float32).astype(np.float64)
+        r = oracle.accept_stochastic(target, draft, toks, parents, draft_row, u, 1, without_replacement=rule_without)
+        counts[int(toks[r["path"][0] - 1]) if r["accepted_len"] else r["bonus"]] += 1
+    return chisquare(counts, trials * p).pvalue
+
+
+@pytest.mark.slow
+def test_sampling_without_replacement_preserves_target_distribution():
+    assert _chi2_first_token_distinct(1_000_000, 33, True) > 1e-3
+
+
+def test_with_replacement_rule_on_distinct_drafts_is_caught():
+    """The with-replacement residual chain applied to siblings drawn without
+    replacement is biased; the same test must see it."""
+    assert _chi2_first_token_distinct(200_000, 34, False) < 1e-6
+
+
 def _chi2_first_token(trials, shape, seed):
     """First emitted token over `trials` walks with drafts sampled from q."""
     rng = np.random.default_rng(seed)
