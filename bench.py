@@ -9,7 +9,7 @@ input sets whose total size exceeds twice the L2 cache are rotated between
 steps, so every step reads its KV cache and logits from HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
-                    [--mode stochastic|greedy] [--impl ours|reference]
+                    [--mode stochastic|stochastic-wor|greedy] [--impl ours|reference]
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own replica of
 the workload (the step has no cross-sequence exchange); the job value is the
@@ -52,7 +52,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="7b")
-    ap.add_argument("--mode", default="stochastic", choices=["stochastic", "greedy"])
+    ap.add_argument("--mode", default="stochastic", choices=["stochastic", "stochastic-wor", "greedy"],
+                    help="acceptance: sampled (rejected siblings' tokens kept in q, or removed: -wor) or greedy")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -73,7 +74,7 @@ def step_bytes(cfg, plen, mode):
     target = cfg.B * (cfg.m + 1) * cfg.V * eb
     kv = sum(2 * cfg.Hkv * min(int(p), cfg.window or int(p)) * cfg.D * 2 for p in plen)
     attn_other = cfg.B * cfg.m * (2 * cfg.Hq + 2 * cfg.Hkv) * cfg.D * 2  # q, out, tree K, tree V
-    accept = target + (draft if mode == "stochastic" else 0)
+    accept = target + (draft if mode.startswith("stochastic") else 0)
     return {"draft": draft, "attention": kv + attn_other, "kv": kv, "accept": accept,
             "step": draft + kv + attn_other + accept}
 
@@ -153,9 +154,9 @@ def oracle_step(cfg, seed, mode):
         oracle.pack_mask(oracle.ancestor_mask(t["parents"]))
         oracle.tree_attention(dec(q[b]), dec(kc[b]), dec(vc[b]), int(plen[b]), dec(kt[b]), dec(vt[b]),
                               t["parents"], t["depth"], window=cfg.window)
-        if mode == "stochastic":
+        if mode.startswith("stochastic"):
             oracle.accept_stochastic(tgt[b], x[b], t["tokens"], t["parents"], t["draft_row"],
-                                     u[b].astype(np.float64), cfg.depth)
+                                     u[b].astype(np.float64), cfg.depth, without_replacement=mode == "stochastic-wor")
         else:
             oracle.accept_greedy(tgt[b], t["tokens"], t["parents"], cfg.depth)
     return t_build + (time.perf_counter() - t1)
@@ -253,7 +254,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     cfg = get_config(args.config)
-    stoch = args.mode == "stochastic"
+    stoch = args.mode.startswith("stochastic")
     tdt = torch.float32 if cfg.logits_dtype == "f32" else torch.bfloat16
 
     def to_logits(a):
@@ -265,7 +266,8 @@ def main():
         return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
 
     shape = StepShape(B=cfg.B, Hq=cfg.Hq, Hkv=cfg.Hkv, D=cfg.D, Lmax=cfg.L, depth=cfg.depth, k=cfg.k, m=cfg.m,
-                      V=cfg.V, logits_dtype=tdt, window=cfg.window, stochastic=stoch)
+                      V=cfg.V, logits_dtype=tdt, window=cfg.window, stochastic=stoch,
+                      without_replacement=args.mode == "stochastic-wor")
 
     # input sets: enough distinct sets that their bytes exceed 2x L2
     sb0 = step_bytes(cfg, gen_prefix_len(cfg, 0), args.mode)

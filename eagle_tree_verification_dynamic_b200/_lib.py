@@ -41,7 +41,7 @@ class StepIn(ctypes.Structure):
                 ("B", _c_i), ("V", _c_i), ("depth", _c_i), ("k", _c_i), ("m", _c_i),
                 ("q", _c_p), ("k_cache", _c_p), ("v_cache", _c_p), ("prefix_len", _c_p), ("Lmax", _c_i),
                 ("k_tree", _c_p), ("v_tree", _c_p), ("Hq", _c_i), ("Hkv", _c_i), ("D", _c_i), ("window", _c_i),
-                ("scale", _c_f), ("uniforms", _c_p)]
+                ("scale", _c_f), ("uniforms", _c_p), ("sampling_rule", _c_i)]
 
 
 class StepOut(ctypes.Structure):
@@ -76,6 +76,8 @@ _SIGS = {
     "eagle_kv_compact": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                 _c_p]),
     "eagle_accept_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
+    "eagle_accept_with_rule": (_c_i, [_c_p, _c_i, _c_p, _c_i, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i,
+                                      _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "eagle_accept": (_c_i, [_c_p, _c_i, _c_p, _c_i, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i,
                             _c_i, _c_i, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
 }
@@ -277,21 +279,27 @@ def accept_workspace_bytes(B, n, V, dtype_code) -> int:
     return lib().eagle_accept_workspace_bytes(B, n, V, dtype_code)
 
 
+SAMPLE_WITH_REPLACEMENT, SAMPLE_WITHOUT_REPLACEMENT = 0, 1
+
+
 def accept_into(target_logits, tokens, parents, draft_row, depth, uniforms, draft_logits, draft_lse,
-                accepted_len, path, bonus, ws):
+                accepted_len, path, bonus, ws, without_replacement: bool = False):
     B, n1, V = target_logits.shape
     n = n1 - 1
     R = draft_logits.shape[1] if draft_logits is not None else 0
     ddt = _dtype_code(draft_logits) if draft_logits is not None else 0
-    _check(lib().eagle_accept(_ptr(target_logits), _dtype_code(target_logits), _ptr(draft_logits), ddt,
-                              _ptr(draft_lse), R, _ptr(tokens), _ptr(parents), _ptr(draft_row), _ptr(uniforms),
-                              B, n, V, depth, _ptr(accepted_len), _ptr(path), _ptr(bonus), _ptr(ws), ws.numel(),
-                              _stream(target_logits.device)), "eagle_accept")
+    rule = SAMPLE_WITHOUT_REPLACEMENT if without_replacement else SAMPLE_WITH_REPLACEMENT
+    _check(lib().eagle_accept_with_rule(_ptr(target_logits), _dtype_code(target_logits), _ptr(draft_logits), ddt,
+                                        _ptr(draft_lse), R, _ptr(tokens), _ptr(parents), _ptr(draft_row),
+                                        _ptr(uniforms), rule, B, n, V, depth, _ptr(accepted_len), _ptr(path),
+                                        _ptr(bonus), _ptr(ws), ws.numel(), _stream(target_logits.device)),
+           "eagle_accept_with_rule")
 
 
 def accept(target_logits, tokens, parents, draft_row, depth: int, uniforms=None, draft_logits=None,
-           draft_lse=None):
-    """-> (accepted_len [B] int32, path [B][depth] int32, bonus [B] int32)."""
+           draft_lse=None, without_replacement: bool = False):
+    """-> (accepted_len [B] int32, path [B][depth] int32, bonus [B] int32).  without_replacement: after a
+    sampled child is rejected its token leaves the draft distribution (q renormalised)."""
     _need_cuda(target_logits, tokens, parents, draft_row, uniforms, draft_logits, draft_lse)
     B, n1, V = target_logits.shape
     dev = target_logits.device
@@ -300,13 +308,13 @@ def accept(target_logits, tokens, parents, draft_row, depth: int, uniforms=None,
     bonus = torch.empty(B, dtype=torch.int32, device=dev)
     ws = _workspace(accept_workspace_bytes(B, n1 - 1, V, _dtype_code(target_logits)), dev)
     accept_into(target_logits, tokens, parents, draft_row, depth, uniforms, draft_logits, draft_lse,
-                acc, path, bonus, ws)
+                acc, path, bonus, ws, without_replacement)
     return acc, path, bonus
 
 
 # ---------------------------------------------------------------- one step
 def step_in(draft_logits, target_logits, depth, k, m, q, k_cache, v_cache, prefix_len, k_tree, v_tree,
-            uniforms=None, window: int = 0, scale: float = 0.0) -> StepIn:
+            uniforms=None, window: int = 0, scale: float = 0.0, without_replacement: bool = False) -> StepIn:
     """The C step's inputs: draft_logits [B][R][V] and target_logits [B][n+1][V] (f32 or bf16),
     q [B][n][Hq][D], caches [B][Hkv][Lmax][D], tree K/V [B][n][Hkv][D] (bf16), prefix_len [B] int32,
     uniforms [B][2][n+1] f32 or None (greedy)."""
@@ -315,7 +323,8 @@ def step_in(draft_logits, target_logits, depth, k, m, q, k_cache, v_cache, prefi
     Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
     return StepIn(_ptr(draft_logits), _ptr(target_logits), _dtype_code(draft_logits), B, V, depth, k, m,
                   _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), Lmax, _ptr(k_tree), _ptr(v_tree),
-                  Hq, Hkv, D, window, scale, _ptr(uniforms))
+                  Hq, Hkv, D, window, scale, _ptr(uniforms),
+                  SAMPLE_WITHOUT_REPLACEMENT if without_replacement else SAMPLE_WITH_REPLACEMENT)
 
 
 def step_workspace_bytes(si: StepIn) -> int:

@@ -16,6 +16,11 @@
 //     max(0, p - t q) / F(t) with F(t) = sum_x max(0, p(x) - t q(x)),
 //     t_0 = 0 (F = 1), t_{r+1} = t_r + F(t_r); one sweep per rejection gives
 //     F at the new t;
+//   * sampling without replacement also removes each rejected token from q
+//     and renormalises it.  With S = the draft mass not yet rejected at j, the
+//     current target is still max(0, p - t q) / F(t) (q the unchanged draft
+//     row), the ratio gains a factor S and the update becomes
+//     t_{r+1} = t_r + F(t_r) / S_r; with replacement S stays 1;
 //   * the bonus token is the smallest x whose cumulative weight exceeds
 //     u_res * total (inverse CDF), found by a prefix scan over the slices.
 // A thread copies its slice of node j's target row and of its draft row into
@@ -242,7 +247,8 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
                    const double* __restrict__ row_lse, const int32_t* __restrict__ tokens,
                    const int32_t* __restrict__ parents, const int32_t* __restrict__ draft_row,
                    const float* __restrict__ uniforms, int32_t* __restrict__ accepted_len,
-                   int32_t* __restrict__ path, int32_t* __restrict__ bonus, int slice, bool vec_ok) {
+                   int32_t* __restrict__ path, int32_t* __restrict__ bonus, int slice, bool vec_ok,
+                   bool without_replacement) {
   __shared__ AcceptSmem sm;
   extern __shared__ __align__(16) unsigned char cache_raw[];
   griddep_wait();  // the target row statistics come from the previous kernel
@@ -318,8 +324,8 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   int j = 0, plen = 0;
   double lse_t = STOCH ? sm.lse_t[0] : 0.0;
   int amax = sm.amax[0];
-  double t = 0.0, F = 1.0;
-  bool rejected_here = false;
+  double t = 0.0, F = 1.0, S = 1.0;  // S: draft mass not yet rejected at j (1 with replacement)
+  bool rejected_here = false, degenerate = false;
 
   while (plen < depth) {
     int moved_to = -1;
@@ -335,14 +341,18 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
       int c = sm.first_child[j];
       while (true) {
         if (c > n || r < 0) break;
-        // accept iff u < rho / (F q), i.e. u F q < rho (q > 0); a token outside
-        // the vocabulary has p = q = 0 and is never accepted
+        // accept iff u < S rho / (F q), i.e. u F q < S rho (q > 0); a token
+        // outside the vocabulary has p = q = 0 and is never accepted
         const double px = sm.px[c], qx = sm.qx[c];
         const double rho = t == 0.0 ? px : fmax(0.0, px - t * qx);
-        if (qx > 0.0 && (double)sm.u_acc[c] * (F * qx) < rho) { moved_to = c; break; }
+        if (qx > 0.0 && (double)sm.u_acc[c] * (F * qx) < S * rho) { moved_to = c; break; }
         // rejected: the current target becomes max(0, p - t' q) / F(t')
-        t += F;
+        t += F / S;
         rejected_here = true;
+        if (without_replacement) {
+          S -= qx;
+          if (!(S > 0.0)) { degenerate = true; break; }  // q has nothing left to draw from
+        }
         int nc = c + 1;
         while (nc <= n && sm.par[nc - 1] != j) ++nc;
         if (nc <= n) {  // another sibling will be tested: need F(t)
@@ -362,6 +372,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     j = moved_to;
     t = 0.0;
     F = 1.0;
+    S = 1.0;
     rejected_here = false;
     amax = sm.amax[j];
     if (STOCH) lse_t = sm.lse_t[j];
@@ -373,6 +384,11 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   }
   if (!STOCH) {
     if (leader) bonus[b] = amax;
+    return;
+  }
+  if (degenerate) {
+    if (leader) bonus[b] = amax;
+    cluster.sync();
     return;
   }
   const int r = sm.drow[j];
@@ -406,7 +422,7 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
                                int depth, const int32_t* row_amax, const double* row_lse,
                                const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                                const float* uniforms, int B, int32_t* acc_len, int32_t* path,
-                               int32_t* bonus, cudaStream_t s, bool pdl) {
+                               int32_t* bonus, cudaStream_t s, bool pdl, bool without_replacement) {
   int cl = 1, slice = 0;
   size_t dyn = 0;
   const bool vec_ok = (((uintptr_t)tgt | (uintptr_t)dft) % 16 == 0) && ((size_t)V * sizeof(T)) % 16 == 0;
@@ -445,13 +461,15 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
   cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, accept_walk_kernel<T, STOCH>, static_cast<const T*>(tgt),
                             static_cast<const T*>(dft), dlse, R, V, n, depth, row_amax, row_lse, tokens,
-                            parents, draft_row, uniforms, acc_len, path, bonus, slice, vec_ok);
+                            parents, draft_row, uniforms, acc_len, path, bonus, slice, vec_ok,
+                            without_replacement);
 }
 
 cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,
                           int R, const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                           const float* uniforms, int B, int n, int V, int depth, int32_t* accepted_len,
-                          int32_t* path, int32_t* bonus, void* ws, cudaStream_t s, bool zero_tickets, bool pdl) {
+                          int32_t* path, int32_t* bonus, void* ws, cudaStream_t s, bool zero_tickets, bool pdl,
+                          bool without_replacement) {
   const long long rows = (long long)B * (n + 1);
   const bool stoch = uniforms != nullptr;
   char* tail = static_cast<char*>(ws) + row_stats_ws_bytes(rows, V, dtype_bytes(tdtype), 1);
@@ -466,14 +484,16 @@ cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddty
   (void)ddtype;  // the draft rows share the target's element type (checked by the caller)
   if (tdtype == EAGLE_F32)
     return stoch ? launch_walk<float, true>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens, parents,
-                                            draft_row, uniforms, B, accepted_len, path, bonus, s, pdl)
+                                            draft_row, uniforms, B, accepted_len, path, bonus, s, pdl,
+                                            without_replacement)
                  : launch_walk<float, false>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
-                                             parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl);
+                                             parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl, false);
   return stoch ? launch_walk<__nv_bfloat16, true>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
-                                                  parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl)
+                                                  parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl,
+                                                  without_replacement)
                : launch_walk<__nv_bfloat16, false>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
                                                    parents, draft_row, uniforms, B, accepted_len, path, bonus, s,
-                                                   pdl);
+                                                   pdl, false);
 }
 
 }  // namespace eagle

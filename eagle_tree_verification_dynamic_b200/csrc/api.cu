@@ -177,6 +177,19 @@ eagle_status eagle_accept(const void* target_logits, int target_dtype, const voi
                           const int32_t* draft_row, const float* uniforms, int B, int n, int V, int depth,
                           int32_t* accepted_len, int32_t* path, int32_t* bonus, void* workspace,
                           size_t workspace_bytes, void* stream) {
+  return eagle_accept_with_rule(target_logits, target_dtype, draft_logits, draft_dtype, draft_lse, R, tokens, parents,
+                                draft_row, uniforms, EAGLE_SAMPLE_WITH_REPLACEMENT, B, n, V, depth, accepted_len,
+                                path, bonus, workspace, workspace_bytes, stream);
+}
+
+eagle_status eagle_accept_with_rule(const void* target_logits, int target_dtype, const void* draft_logits,
+                                    int draft_dtype, const double* draft_lse, int R, const int32_t* tokens,
+                                    const int32_t* parents, const int32_t* draft_row, const float* uniforms,
+                                    int sampling_rule, int B, int n, int V, int depth, int32_t* accepted_len,
+                                    int32_t* path, int32_t* bonus, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  if (sampling_rule != EAGLE_SAMPLE_WITH_REPLACEMENT && sampling_rule != EAGLE_SAMPLE_WITHOUT_REPLACEMENT)
+    return EAGLE_ERR_SHAPE;
   if (!target_logits || !tokens || !parents || !draft_row || !accepted_len || !path || !bonus)
     return EAGLE_ERR_NULL;
   if (!valid_dtype(target_dtype)) return EAGLE_ERR_DTYPE;
@@ -195,7 +208,8 @@ eagle_status eagle_accept(const void* target_logits, int target_dtype, const voi
   if (st != EAGLE_OK) return st;
   return cuda_status(launch_accept(target_logits, target_dtype, draft_logits, draft_dtype, draft_lse, R, tokens,
                                    parents, draft_row, uniforms, B, n, V, depth, accepted_len, path, bonus,
-                                   workspace, static_cast<cudaStream_t>(stream)));
+                                   workspace, static_cast<cudaStream_t>(stream), true, false,
+                                   sampling_rule == EAGLE_SAMPLE_WITHOUT_REPLACEMENT));
 }
 
 // ------------------------------------------------------ KV-cache compaction
@@ -276,6 +290,8 @@ eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t
   if (!step_layout(in, &L)) return EAGLE_ERR_LIMIT;
   if ((long long)in->B * (L.n + 1) > 0x7fffffffLL) return EAGLE_ERR_SHAPE;
   if (in->uniforms && in->V > accept_max_vocab(in->logits_dtype)) return EAGLE_ERR_LIMIT;
+  if (in->sampling_rule != EAGLE_SAMPLE_WITH_REPLACEMENT && in->sampling_rule != EAGLE_SAMPLE_WITHOUT_REPLACEMENT)
+    return EAGLE_ERR_SHAPE;
   if (!aligned16(in->q) || !aligned16(in->k_tree) || !aligned16(in->v_tree) || !aligned16(out->attn_out) ||
       (in->Lmax > 0 && (!aligned16(in->k_cache) || !aligned16(in->v_cache))))
     return EAGLE_ERR_ALIGN;
@@ -310,7 +326,8 @@ eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t
   // --- acceptance (the draft rows' log-sum-exps are the tree's row_lse)
   e = launch_accept(in->target_logits, in->logits_dtype, in->draft_logits, in->logits_dtype, t.row_lse, L.R,
                     t.tokens, t.parents, t.draft_row, in->uniforms, in->B, n, in->V, in->depth, out->accepted_len,
-                    out->path, out->bonus, ws + L.acc_off, s, false, true);
+                    out->path, out->bonus, ws + L.acc_off, s, false, true,
+                    in->sampling_rule == EAGLE_SAMPLE_WITHOUT_REPLACEMENT);
   return cuda_status(e);
 }
 

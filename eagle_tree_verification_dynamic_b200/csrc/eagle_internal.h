@@ -122,6 +122,6 @@ cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddty
                           int R, const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                           const float* uniforms, int B, int n, int V, int depth, int32_t* accepted_len,
                           int32_t* path, int32_t* bonus, void* ws, cudaStream_t s, bool zero_tickets = true,
-                          bool pdl = false);
+                          bool pdl = false, bool without_replacement = false);
 
 }  // namespace eagle

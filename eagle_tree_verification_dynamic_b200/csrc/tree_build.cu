@@ -18,8 +18,7 @@
 
 namespace eagle {
 
-constexpr int kBuildThreads = 1024;
-constexpr int kBuildWarps = kBuildThreads / 32;
+constexpr int kBuildThreads = 1024;  // the largest expansion block
 
 struct BuildSmem {
   double* row_lp;    // [R*k] log-confidence of each row's top-k children
@@ -31,7 +30,7 @@ struct BuildSmem {
   int* cand_row;     // [P]   draft row of an expanded candidate, -1 otherwise
   int* node_of;      // [P]   kept flag, then 1-based node id (0 = dropped)
   int* frontier;     // [32]
-  int* warp_cnt;     // [kBuildWarps]
+  int* warp_cnt;     // [NT / 32]
   int* node_par;     // [EAGLE_MAX_NODES] parent node id of node i+1 (mask fusion)
   int* node_dep;     // [EAGLE_MAX_NODES]
 };

@@ -32,6 +32,7 @@ class StepShape:
     logits_dtype: torch.dtype
     window: int = 0
     stochastic: bool = True
+    without_replacement: bool = False   # sampled acceptance: a rejected child's token leaves q
 
     @property
     def R(self) -> int:
@@ -61,7 +62,7 @@ class VerifyStep:
         self.ws_attn = L._workspace(L.attention_workspace_bytes(s.B, n, s.Hq, s.Hkv, s.D, s.Lmax, s.window), dev)
         self.ws_acc = L._workspace(L.accept_workspace_bytes(s.B, n, s.V, dcode), dev)
         shape_only = L.StepIn(None, None, dcode, s.B, s.V, s.depth, s.k, s.m, None, None, None, None, s.Lmax, None,
-                              None, s.Hq, s.Hkv, s.D, s.window, 0.0, None)
+                              None, s.Hq, s.Hkv, s.D, s.window, 0.0, None, 0)
         self.ws_step = L._workspace(L.step_workspace_bytes(shape_only), dev)
 
     def build(self, draft_logits: torch.Tensor):
@@ -78,7 +79,7 @@ class VerifyStep:
         if self.s.stochastic:
             L.accept_into(target_logits, self.tree.tokens, self.tree.parents, self.tree.draft_row, self.s.depth,
                           uniforms, draft_logits, self.tree.row_lse, self.accepted_len, self.path, self.bonus,
-                          self.ws_acc)
+                          self.ws_acc, self.s.without_replacement)
         else:
             L.accept_into(target_logits, self.tree.tokens, self.tree.parents, self.tree.draft_row, self.s.depth,
                           None, None, None, self.accepted_len, self.path, self.bonus, self.ws_acc)
@@ -88,7 +89,8 @@ class VerifyStep:
         s = self.s
         si = L.step_in(inp["draft_logits"], inp["target_logits"], s.depth, s.k, s.m, inp["q"], inp["k_cache"],
                        inp["v_cache"], inp["prefix_len"], inp["k_tree"], inp["v_tree"],
-                       inp.get("uniforms") if s.stochastic else None, s.window)
+                       inp.get("uniforms") if s.stochastic else None, s.window,
+                       without_replacement=s.without_replacement)
         L.step_into(si, self.tree, self.mask, self.pos, self.out, self.accepted_len, self.path, self.bonus,
                     self.ws_step, self.device)
         self._step_in = si

@@ -214,6 +214,27 @@ EAGLE_API eagle_status eagle_tree_attention(const void* q, const void* k_cache, 
  * V <= 262144 (bf16) or 131072 (fp32).
  * Workspace: eagle_accept_workspace_bytes. */
 EAGLE_API size_t eagle_accept_workspace_bytes(int B, int n, int V, int target_dtype);
+
+/* How q changes when a sampled child is rejected (the pages do not say):
+ *   EAGLE_SAMPLE_WITH_REPLACEMENT: q is kept (eagle_accept);
+ *   EAGLE_SAMPLE_WITHOUT_REPLACEMENT: for siblings drafted without replacement
+ *     (distinct tokens, as top-k children always are): after the residual step
+ *     the rejected token is removed from q and q renormalised,
+ *     q <- q with q(x_c) = 0, divided by its remaining sum.
+ *     With one child per node both rules give the same walk.  If nothing is
+ *     left in q the walk stops at that node and the bonus is the target argmax. */
+enum { EAGLE_SAMPLE_WITH_REPLACEMENT = 0, EAGLE_SAMPLE_WITHOUT_REPLACEMENT = 1 };
+
+/* eagle_accept with the sampling rule chosen (ignored for greedy, uniforms ==
+ * NULL); any other rule value returns EAGLE_ERR_SHAPE.  Arguments otherwise as
+ * in eagle_accept. */
+EAGLE_API eagle_status eagle_accept_with_rule(const void* target_logits, int target_dtype, const void* draft_logits,
+                                              int draft_dtype, const double* draft_lse, int R,
+                                              const int32_t* tokens, const int32_t* parents,
+                                              const int32_t* draft_row, const float* uniforms, int sampling_rule,
+                                              int B, int n, int V, int depth, int32_t* accepted_len,
+                                              int32_t* path, int32_t* bonus, void* workspace,
+                                              size_t workspace_bytes, void* stream);
 EAGLE_API eagle_status eagle_accept(const void* target_logits, int target_dtype, const void* draft_logits,
                           int draft_dtype, const double* draft_lse, int R, const int32_t* tokens,
                           const int32_t* parents, const int32_t* draft_row, const float* uniforms,
@@ -289,6 +310,8 @@ EAGLE_API eagle_status eagle_kv_compact(const void* k_tree, const void* v_tree, 
  *   (the tree size, also written to the HOST int *n_nodes when not NULL)
  *   target_logits [B][n+1][V] (logits_dtype, the target's rows of the tree)
  *   uniforms [B][2][n+1] float, or NULL for greedy acceptance
+ *   sampling_rule: EAGLE_SAMPLE_WITH_REPLACEMENT or _WITHOUT_REPLACEMENT (as
+ *   in eagle_accept_with_rule; ignored for greedy)
  * Outputs (caller-allocated, sized by n): the tree arrays (tree.gid may be
  *   NULL), mask [B][n][2] uint64, pos [B][n] int32, attn_out [B][n][Hq][D]
  *   bf16, accepted_len [B], path [B][depth], bonus [B] int32.
@@ -311,6 +334,7 @@ typedef struct {
   int Hq, Hkv, D, window;
   float scale;  /* <= 0 selects 1/sqrt(D) */
   const float* uniforms;
+  int sampling_rule;  /* EAGLE_SAMPLE_WITH_REPLACEMENT or _WITHOUT_REPLACEMENT (sampled acceptance) */
 } eagle_step_in_t;
 
 typedef struct {

@@ -107,6 +107,11 @@ def test_accept_and_mask_validation(lib):
     assert acc(dt=9) == 3
     assert acc(n=200) == 4
     assert acc(depth=0) == 2
+    rule = lambda r: lib.eagle_accept_with_rule(FAKE, 0, FAKE, 0, FAKE, 5, FAKE, FAKE, FAKE, FAKE, r, 1, 10, 1000, 3,
+                                                FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert rule(2) == 2 and rule(-1) == 2
+    assert lib.eagle_accept_with_rule(FAKE, 0, None, 0, None, 5, FAKE, FAKE, FAKE, FAKE, 1, 1, 10, 1000, 3,
+                                      FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == 1
     assert lib.eagle_tree_mask(None, None, None, 1, 10, FAKE, None, None) == 1
     assert lib.eagle_tree_mask(FAKE, None, None, 1, 129, FAKE, None, None) == 4
     assert lib.eagle_tree_mask(FAKE, None, None, 1, 10, FAKE, FAKE, None) == 1  # pos needs depth, prefix_len
@@ -121,7 +126,7 @@ def test_binding_refuses_cpu_tensors():
 def _step_in(**kw):
     d = dict(draft_logits=FAKE, target_logits=FAKE, logits_dtype=0, B=1, V=32000, depth=6, k=10, m=60,
              q=FAKE, k_cache=FAKE, v_cache=FAKE, prefix_len=FAKE, Lmax=2048, k_tree=FAKE, v_tree=FAKE,
-             Hq=32, Hkv=32, D=128, window=0, scale=0.0, uniforms=None)
+             Hq=32, Hkv=32, D=128, window=0, scale=0.0, uniforms=None, sampling_rule=0)
     d.update(kw)
     return _lib.StepIn(*[d[name] for name, _ in _lib.StepIn._fields_])
 
@@ -160,6 +165,7 @@ def test_step_validation(lib):
     assert call(si=_step_in(m=200)) == 4
     assert call(si=_step_in(q=ctypes.c_void_p(0x1008))) == 6
     assert call(ws=None, wsb=0) == 5
+    assert call(si=_step_in(sampling_rule=2)) == 2
     assert n.value == 0  # nothing was reported: every call above failed validation
 
 

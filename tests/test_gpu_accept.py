@@ -26,7 +26,7 @@ def _oracle_trees(cfg, stored):
     return x64, [oracle.build_tree(x64[b], cfg.depth, cfg.k, cfg.m) for b in range(cfg.B)]
 
 
-def _run_accept(cfg, seed, mode, sigma=None):
+def _run_accept(cfg, seed, mode, sigma=None, without_replacement=False):
     stored = gen_draft_logits(cfg, seed)
     x64, trees = _oracle_trees(cfg, stored)
     draft_row = np.stack([t["draft_row"] for t in trees])
@@ -46,7 +46,8 @@ def _run_accept(cfg, seed, mode, sigma=None):
         lse_gpu = lse_gpu.reshape(cfg.B, cfg.R)
         assert torch.allclose(lse_gpu, lse, rtol=0, atol=5e-7)
         acc, path, bonus = et.accept(T, tokens, parents, drow, cfg.depth, torch.from_numpy(u).to(dev()),
-                                     to_dev_logits(stored, cfg.logits_dtype), lse_gpu)
+                                     to_dev_logits(stored, cfg.logits_dtype), lse_gpu,
+                                     without_replacement=without_replacement)
     acc, path, bonus = acc.cpu().numpy(), path.cpu().numpy(), bonus.cpu().numpy()
     reported = 0
     for b in range(cfg.B):
@@ -55,7 +56,7 @@ def _run_accept(cfg, seed, mode, sigma=None):
             r = oracle.accept_greedy(T64[b], t["tokens"], t["parents"], cfg.depth)
         else:
             r = oracle.accept_stochastic(T64[b], x64[b], t["tokens"], t["parents"], t["draft_row"],
-                                         u[b].astype(np.float64), cfg.depth)
+                                         u[b].astype(np.float64), cfg.depth, without_replacement)
         same = (int(acc[b]) == r["accepted_len"] and path[b].tolist() == r["path"] and int(bonus[b]) == r["bonus"])
         if not same:
             assert r["near_ties"], (f"{cfg.name} seed {seed} seq {b} {mode}: gpu ({acc[b]}, {path[b].tolist()}, "
@@ -92,6 +93,52 @@ def test_accept_batch_of_ragged_configs():
     cfg = get_config("serve", B=12, V=5003, logits_dtype="f32")
     _run_accept(cfg, 4, "stochastic")
     _run_accept(cfg, 4, "greedy")
+
+
+@pytest.mark.parametrize("name", ["tiny", "7b", "l3-8b", "serve"])
+def test_accept_without_replacement_configs(name):
+    cfg = get_config(name)
+    for seed in cfg.seeds[:3]:
+        _run_accept(cfg, seed, "stochastic", without_replacement=True)
+
+
+def test_accept_without_replacement_ragged_and_more_seeds():
+    _run_accept(get_config("serve", B=12, V=5003, logits_dtype="f32"), 4, "stochastic", without_replacement=True)
+    cfg = get_config("7b")
+    lens = [int(_run_accept(cfg, s, "stochastic", without_replacement=True)[0][0]) for s in cfg.seeds]
+    print(f"7b sampled without replacement, accepted lengths over seeds: {lens}")
+
+
+def _chi2_gpu_distinct(trials: int, seed: int, without_replacement: bool) -> float:
+    """A star of 3 distinct siblings drawn without replacement from q; first emitted token vs p."""
+    rng = np.random.default_rng(seed)
+    V = 8
+    p, q = rng.dirichlet(np.ones(V)), rng.dirichlet(np.ones(V) * 0.5)
+    q32 = np.exp(np.log(q).astype(np.float32).astype(np.float64))
+    q32 /= q32.sum()
+    # Gumbel top-3 of log q: a draw without replacement, in draw order
+    g = np.log(q32)[None, :] - np.log(-np.log(rng.random((trials, V))))
+    toks = np.argsort(-g, axis=1)[:, :3]
+    other = rng.dirichlet(np.ones(V))
+    target = np.stack([np.log(p)] + [np.log(other)] * 3)
+    u = rng.random((trials, 2, 4)).astype(np.float32)
+    D = torch.from_numpy(np.log(q)[None].astype(np.float32)).to(dev()).expand(trials, 1, V).contiguous()
+    T = torch.from_numpy(target.astype(np.float32)).to(dev()).expand(trials, 4, V).contiguous()
+    _, _, lse = et.row_stats(D.reshape(-1, V), 1)
+    acc, path, bonus = et.accept(T, i32(toks), i32(np.zeros((trials, 3))), i32(np.tile([0, -1, -1, -1], (trials, 1))),
+                                 1, torch.from_numpy(u).to(dev()), D, lse.reshape(trials, 1),
+                                 without_replacement=without_replacement)
+    acc, path, bonus = acc.cpu().numpy(), path.cpu().numpy(), bonus.cpu().numpy()
+    first = np.where(acc > 0, toks[np.arange(trials), np.maximum(path[:, 0], 1) - 1], bonus)
+    p32 = np.exp(np.log(p).astype(np.float32).astype(np.float64))
+    p32 /= p32.sum()
+    return chisquare(np.bincount(first, minlength=V), trials * p32).pvalue
+
+
+def test_gpu_sampling_without_replacement_preserves_target_distribution():
+    assert _chi2_gpu_distinct(1_000_000, 42, True) > 1e-3
+    # the with-replacement rule on the same kind of draws is biased, and the test sees it
+    assert _chi2_gpu_distinct(200_000, 43, False) < 1e-6
 
 
 def _chi2_gpu(shape: str, trials: int, seed: int) -> float:

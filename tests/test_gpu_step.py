@@ -44,7 +44,8 @@ def _run_both(name, mode, seed=0):
     dev = torch.device("cuda")
     w, inp, tdt, logits = _inputs(cfg, seed, dev)
     shape = StepShape(B=cfg.B, Hq=cfg.Hq, Hkv=cfg.Hkv, D=cfg.D, Lmax=cfg.L, depth=cfg.depth, k=cfg.k, m=cfg.m,
-                      V=cfg.V, logits_dtype=tdt, window=cfg.window, stochastic=(mode == "stochastic"))
+                      V=cfg.V, logits_dtype=tdt, window=cfg.window, stochastic=mode.startswith("stochastic"),
+                      without_replacement=(mode == "stochastic-wor"))
     sep, one = VerifyStep(shape, dev), VerifyStep(shape, dev)
     sep.build(inp["draft_logits"])
     torch.cuda.synchronize()
@@ -58,6 +59,7 @@ def _run_both(name, mode, seed=0):
 
 @pytest.mark.parametrize("name,mode", [("tiny", "greedy"), ("tiny", "stochastic"), ("7b", "stochastic"),
                                        ("7b", "greedy"), ("l3-8b", "stochastic"), ("serve", "stochastic"),
+                                       ("7b", "stochastic-wor"), ("serve", "stochastic-wor"),
                                        ("long-window", "greedy")])
 def test_step_equals_the_separate_calls(name, mode):
     cfg, w, inp, sep, one = _run_both(name, mode)
