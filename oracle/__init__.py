@@ -12,6 +12,9 @@ Everything is plain numpy in fp64, written step by step from the pages:
                 root path, per-level top-k expansion, rerank to the best m
                 ("s1mplewind eagle" notes, EAGLE-2: "Well-Calibrated Draft Model",
                 "Expansion of tree", "Reranking Nodes").
+* ``static_tree`` EAGLE-1's fixed tree: a template of parents and sibling
+                ranks filled from each parent's top tokens ("EAGLE" notes,
+                "1. EAGLE pipeline / Draft Model").
 * ``mask``      tree attention mask: a node sees the shared prefix, its
                 ancestors and itself ("Технический анализ EAGLE-4", section
                 "Деревья проверки EAGLE-4 и утилита управления").
@@ -34,6 +37,7 @@ through special cases that reduce to library attention (causal, decode, MHA).
 """
 from .common import decode_logits, logsumexp, softmax, near_tie  # noqa: F401
 from .tree import build_tree, build_trees  # noqa: F401
+from .static_tree import build_static_tree, template_rows  # noqa: F401
 from .mask import ancestor_mask, pack_mask, positions  # noqa: F401
 from .attention import tree_attention, tree_attention_rows  # noqa: F401
 from .accept import accept_greedy, accept_stochastic, inverse_cdf  # noqa: F401
