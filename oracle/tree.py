@@ -85,10 +85,12 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
     level_cands = [make(0, r, r, 1, None) for r in range(k)]
     all_cands += level_cands
     frontiers: List[dict] = []    # per expanded level: the k tokens by slot and their parents' slots
+    gains: List[float] = []       # per level: sum of V over its k best candidates
     for level in range(2, depth + 1):
         ranked = sorted(level_cands, key=_sort_key)
         _flag_adjacent(ranked, k, "frontier", level - 1, near_ties)
         frontier = ranked[:k]
+        gains.append(float(sum(np.exp(c["logV"]) for c in frontier)))
         frontiers.append({"tokens": np.array([c["token"] for c in frontier], dtype=np.int64),
                           "parent_slot": np.array([-1 if c["pnode"] is None else c["pnode"]["slot"]
                                                    for c in frontier], dtype=np.int64)})
@@ -102,6 +104,7 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
         level_cands = nxt
         all_cands += level_cands
 
+    gains.append(float(sum(np.exp(c["logV"]) for c in sorted(level_cands, key=_sort_key)[:k])))
     P = len(all_cands)
     assert P == k + (depth - 1) * k * k
     n = min(m, P)
@@ -122,7 +125,7 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
         draft_row[i + 1] = c["row"]
     return {"tokens": tokens, "parents": parents, "depth": depth_arr, "logV": logV,
             "gid": gid, "draft_row": draft_row, "row_lse": row_lse, "n": n, "P": P,
-            "frontiers": frontiers, "near_ties": near_ties}
+            "frontiers": frontiers, "gains": np.array(gains), "near_ties": near_ties}
 
 
 def build_trees(logits_b: np.ndarray, depth: int, k: int, m: int) -> List[Dict]:
