@@ -18,6 +18,8 @@ from ._lib import (  # noqa: F401
     attention_workspace_bytes,
     exported_names,
     kv_compact,
+    static_tree_build,
+    static_tree_rows,
     kv_compact_into,
     lib,
     pool_size,

@@ -44,6 +44,10 @@ class StepIn(ctypes.Structure):
                 ("scale", _c_f), ("uniforms", _c_p), ("sampling_rule", _c_i)]
 
 
+class CostTableStruct(ctypes.Structure):
+    _fields_ = [("nB", _c_i), ("nL", _c_i), ("nN", _c_i), ("B", _c_p), ("L", _c_p), ("N", _c_p), ("us", _c_p)]
+
+
 class StepOut(ctypes.Structure):
     _fields_ = [("tree", TreeStruct), ("mask", _c_p), ("pos", _c_p), ("attn_out", _c_p),
                 ("accepted_len", _c_p), ("path", _c_p), ("bonus", _c_p)]
@@ -71,8 +75,18 @@ _SIGS = {
     "eagle_tree_grow_state_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
     "eagle_tree_grow_begin": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p, _c_p]),
     "eagle_tree_grow_level": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p, _c_p]),
-    "eagle_tree_grow_finish": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, ctypes.POINTER(TreeStruct),
-                                      ctypes.POINTER(_c_i), _c_p]),
+    "eagle_tree_grow_gains": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p]),
+    "eagle_tree_grow_finish": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz,
+                                      ctypes.POINTER(TreeStruct), ctypes.POINTER(_c_i), _c_p]),
+    "eagle_static_tree_rows": (_c_i, [_c_p, _c_p, _c_i]),
+    "eagle_static_tree_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_p, _c_p, _c_i]),
+    "eagle_static_tree_build": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_i, ctypes.POINTER(TreeStruct),
+                                       _c_p, _c_sz, _c_p]),
+    "eagle_cost_at": (ctypes.c_double, [ctypes.POINTER(CostTableStruct), ctypes.c_double, ctypes.c_double,
+                                        ctypes.c_double]),
+    "eagle_size_keep_level": (_c_i, [ctypes.POINTER(CostTableStruct), ctypes.c_double, ctypes.c_double, _c_i, _c_i,
+                                     _c_p, _c_i, ctypes.c_double, ctypes.POINTER(_c_i),
+                                     ctypes.POINTER(ctypes.c_double)]),
     "eagle_kv_compact": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                 _c_p]),
     "eagle_accept_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
@@ -369,8 +383,9 @@ def kv_compact(k_tree, v_tree, path, accepted_len, prefix_len, k_cache, v_cache)
 # ---------------------------------------------------- tree grown per level
 class TreeGrower:
     """The build one level at a time: begin(root rows [B][V]) and level(rows [B][k][V], level) each return the
-    new frontier (tokens [B][k], parent slots [B][k]); finish(m) returns the Tree (equal to tree_build on the
-    same rows)."""
+    new frontier (tokens [B][k], parent slots [B][k]); gains() the last level's per-sequence gain [B] (device,
+    float64); finish(m, levels) returns the Tree over the first `levels` levels (equal to tree_build of that
+    depth on the same rows)."""
 
     def __init__(self, B: int, V: int, depth: int, k: int, dtype: torch.dtype, device):
         self.B, self.V, self.depth, self.k = B, V, depth, k
@@ -380,6 +395,7 @@ class TreeGrower:
         self.state = _workspace(nb, self.device)
         self.ftok = torch.empty(B, k, dtype=torch.int32, device=self.device)
         self.fpar = torch.empty(B, k, dtype=torch.int32, device=self.device)
+        self.gain = torch.empty(B, dtype=torch.float64, device=self.device)
 
     def begin(self, root_logits: torch.Tensor):
         _check(lib().eagle_tree_grow_begin(_ptr(root_logits), self.dt, self.B, self.V, self.depth, self.k,
@@ -393,12 +409,59 @@ class TreeGrower:
                                            _stream(self.device)), "eagle_tree_grow_level")
         return self.ftok, self.fpar
 
-    def finish(self, m: int) -> Tree:
+    def gains(self) -> torch.Tensor:
+        _check(lib().eagle_tree_grow_gains(self.dt, self.B, self.V, self.depth, self.k, _ptr(self.state),
+                                           self.state.numel(), _ptr(self.gain), _stream(self.device)),
+               "eagle_tree_grow_gains")
+        return self.gain
+
+    def finish(self, m: int, levels: Optional[int] = None) -> Tree:
+        levels = self.depth if levels is None else levels
         R = 1 + (self.depth - 1) * self.k
-        tree = alloc_tree(self.B, R, self.depth, self.k, m, self.device)
+        tree = alloc_tree(self.B, R, levels, self.k, m, self.device)
         st = tree.struct()
         n_out = _c_i(0)
-        _check(lib().eagle_tree_grow_finish(self.dt, self.B, self.V, self.depth, self.k, m, _ptr(self.state),
-                                            self.state.numel(), ctypes.byref(st), ctypes.byref(n_out),
-                                            _stream(self.device)), "eagle_tree_grow_finish")
+        _check(lib().eagle_tree_grow_finish(self.dt, self.B, self.V, self.depth, self.k, levels, m,
+                                            _ptr(self.state), self.state.numel(), ctypes.byref(st),
+                                            ctypes.byref(n_out), _stream(self.device)), "eagle_tree_grow_finish")
         return tree
+
+
+# --------------------------------------------------------------- static tree
+def _template(parents, ranks):
+    p = (ctypes.c_int32 * len(parents))(*[int(v) for v in parents])
+    r = (ctypes.c_int32 * len(ranks))(*[int(v) for v in ranks])
+    if len(parents) != len(ranks):
+        raise EagleError("static tree: parents and ranks differ in length")
+    return p, r
+
+
+def static_tree_rows(parents, ranks) -> int:
+    """Number of draft rows R the template needs (row 0 = root, then each node with a child)."""
+    p, r = _template(parents, ranks)
+    R = lib().eagle_static_tree_rows(p, r, len(parents))
+    if R < 0:
+        raise EagleError("static tree: invalid template")
+    return R
+
+
+def static_tree_build(draft_logits: torch.Tensor, parents, ranks) -> Tree:
+    """EAGLE-1 fixed tree: draft_logits [B][R][V] (R = static_tree_rows), template parents/ranks
+    (host sequences, node i+1 at index i) -> Tree with n = len(parents) nodes in template order."""
+    _need_cuda(draft_logits)
+    B, R, V = draft_logits.shape
+    n = len(parents)
+    p, r = _template(parents, ranks)
+    dev = draft_logits.device
+    dt = _dtype_code(draft_logits)
+    i32 = dict(dtype=torch.int32, device=dev)
+    tree = Tree(tokens=torch.empty(B, n, **i32), parents=torch.empty(B, n, **i32), depth=torch.empty(B, n, **i32),
+                logV=torch.empty(B, n, dtype=torch.float32, device=dev), gid=torch.empty(B, n, **i32),
+                draft_row=torch.empty(B, n + 1, **i32), row_lse=torch.empty(B, R, dtype=torch.float64, device=dev),
+                n=n)
+    nb = lib().eagle_static_tree_workspace_bytes(B, V, dt, p, r, n)
+    ws = _workspace(max(nb, 256), dev)
+    st = tree.struct()
+    _check(lib().eagle_static_tree_build(_ptr(draft_logits), dt, B, R, V, p, r, n, ctypes.byref(st), _ptr(ws),
+                                         ws.numel(), _stream(dev)), "eagle_static_tree_build")
+    return tree

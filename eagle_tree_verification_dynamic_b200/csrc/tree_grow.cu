@@ -8,8 +8,12 @@
 //           their top-k children form the next level's k^2 candidates,
 //           log V = log V(parent) + log c(child); the k best (log V, then lower
 //           candidate id) form the next frontier
-//   finish  the expansion / rerank kernel of eagle_tree_build on every row so
-//           far: the m best candidates of all levels, numbered by ascending id
+//   finish  the expansion / rerank kernel of eagle_tree_build on the rows of
+//           the levels grown: the m best candidates, numbered by ascending id
+//   gains   per sequence, the sum of V = exp(log V) over the last level's k
+//           best candidates: the expected number of tokens those candidates
+//           add (EAGLE-4 write-up, harness: the gain in cumulative
+//           probability that a level brings)
 //
 // The state keeps each row's top-k tokens and logits and its log-sum-exp in
 // the layout the one-shot build uses, plus the frontier's log V, so the tree
@@ -22,7 +26,7 @@ namespace eagle {
 namespace {
 
 struct GrowLayout {
-  size_t row_tok, row_val, row_lse, front_lv, lvl_tok, lvl_val, lvl_lse, row_ws, total;
+  size_t row_tok, row_val, row_lse, front_lv, gain, lvl_tok, lvl_val, lvl_lse, row_ws, total;
 };
 
 GrowLayout grow_layout(int B, int V, int dtype, int depth, int k) {
@@ -34,6 +38,7 @@ GrowLayout grow_layout(int B, int V, int dtype, int depth, int k) {
   g.row_val = o;  o = align_up(o + sizeof(float) * B * R * k, 256);
   g.row_lse = o;  o = align_up(o + sizeof(double) * B * R, 256);
   g.front_lv = o; o = align_up(o + sizeof(double) * B * k, 256);
+  g.gain = o;     o = align_up(o + sizeof(double) * B, 256);
   g.lvl_tok = o;  o = align_up(o + sizeof(int32_t) * lvl_rows * k, 256);
   g.lvl_val = o;  o = align_up(o + sizeof(float) * lvl_rows * k, 256);
   g.lvl_lse = o;  o = align_up(o + sizeof(double) * lvl_rows, 256);
@@ -46,20 +51,21 @@ GrowLayout grow_layout(int B, int V, int dtype, int depth, int k) {
 constexpr int kGrowThreads = 1024;
 
 // One CTA per sequence: file the swept rows of this level into the row arrays,
-// then (unless this is the last level) pick the next frontier.
+// then pick the level's k best candidates (the next frontier) and their gain.
 //   level 1: rows = {0}, candidates = the root's k children (gid = r)
 //   level l: rows = 1 + (l-2)k + s, candidates gid = k + (l-2)k^2 + s k + r
 __global__ void __launch_bounds__(kGrowThreads)
 tree_grow_kernel(const int32_t* __restrict__ lvl_tok, const float* __restrict__ lvl_val,
                  const double* __restrict__ lvl_lse, int32_t* __restrict__ row_tok, float* __restrict__ row_val,
-                 double* __restrict__ row_lse, double* __restrict__ front_lv, int32_t* __restrict__ front_tok,
-                 int32_t* __restrict__ front_par, int R, int k, int level, int want_frontier) {
+                 double* __restrict__ row_lse, double* __restrict__ front_lv, double* __restrict__ gain,
+                 int32_t* __restrict__ front_tok, int32_t* __restrict__ front_par, int R, int k, int level) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ double s_lv[32 * 32];
   __shared__ int s_tok[32 * 32];
   __shared__ uint64_t s_key[32 * 32];
   __shared__ double s_flv[32];
+  __shared__ double s_best[32];
   const int b = blockIdx.x, tid = threadIdx.x;
   const int nrows = level == 1 ? 1 : k;
   const int r0 = level == 1 ? 0 : 1 + (level - 2) * k;
@@ -72,7 +78,6 @@ tree_grow_kernel(const int32_t* __restrict__ lvl_tok, const float* __restrict__ 
     row_val[dst] = lvl_val[src];
   }
   for (int rr = tid; rr < nrows; rr += kGrowThreads) row_lse[(size_t)b * R + r0 + rr] = lvl_lse[(size_t)b * nrows + rr];
-  if (!want_frontier) return;
   // 2. the level's candidates: log V = log V(parent) + (logit - lse), as the one-shot build forms it
   for (int s = tid; s < k; s += kGrowThreads) s_flv[s] = level == 1 ? 0.0 : front_lv[(size_t)b * k + s];
   __syncthreads();
@@ -95,10 +100,18 @@ tree_grow_kernel(const int32_t* __restrict__ lvl_tok, const float* __restrict__ 
     int rank = 0;
     for (int o = 0; o < cnt; ++o) rank += s_key[o] > mine ? 1 : 0;
     if (rank < k) {
-      front_lv[(size_t)b * k + rank] = s_lv[c];
+      s_best[rank] = s_lv[c];
       if (front_tok) front_tok[(size_t)b * k + rank] = s_tok[c];
       if (front_par) front_par[(size_t)b * k + rank] = level == 1 ? -1 : c / k;
     }
+  }
+  __syncthreads();
+  // s_flv (the previous frontier) is read above; the new one replaces it only now
+  for (int s = tid; s < k; s += kGrowThreads) front_lv[(size_t)b * k + s] = s_best[s];
+  if (tid == 0) {
+    double g = 0.0;  // in rank order
+    for (int s = 0; s < k; ++s) g += exp(s_best[s]);
+    gain[b] = g;
   }
 }
 
@@ -126,11 +139,11 @@ cudaError_t grow_step(const void* logits, int dtype, int B, int V, int depth, in
   cudaError_t e = launch_row_stats(logits, dtype, (long long)B * nrows, V, k, true, ro, st + g.row_ws, s, true, false,
                                    (long long)B * R);
   if (e != cudaSuccess) return e;
-  const int want = level < depth ? 1 : 0;
   return launch_kernel(tree_grow_kernel, dim3(B), dim3(kGrowThreads), 0, s, true, ro.tok, ro.val,
                        (const double*)ro.lse, reinterpret_cast<int32_t*>(st + g.row_tok),
                        reinterpret_cast<float*>(st + g.row_val), reinterpret_cast<double*>(st + g.row_lse),
-                       reinterpret_cast<double*>(st + g.front_lv), ftok, fpar, R, k, level, want);
+                       reinterpret_cast<double*>(st + g.front_lv), reinterpret_cast<double*>(st + g.gain), ftok,
+                       fpar, R, k, level);
 }
 
 eagle_status cuda_st(cudaError_t e) { return report_cuda(e); }
@@ -169,16 +182,26 @@ EAGLE_API eagle_status eagle_tree_grow_level(const void* level_logits, int dtype
                            static_cast<cudaStream_t>(stream)));
 }
 
-EAGLE_API eagle_status eagle_tree_grow_finish(int dtype, int B, int V, int depth, int k, int m, void* state,
-                                              size_t state_bytes, const eagle_tree_t* out, int* n_nodes,
-                                              void* stream) {
+EAGLE_API eagle_status eagle_tree_grow_gains(int dtype, int B, int V, int depth, int k, void* state,
+                                             size_t state_bytes, double* gains, void* stream) {
+  if (!gains) return EAGLE_ERR_NULL;
+  const eagle_status st = grow_check(dtype, B, V, depth, k, state, state_bytes);
+  if (st != EAGLE_OK) return st;
+  const GrowLayout g = grow_layout(B, V, dtype, depth, k);
+  return cuda_st(cudaMemcpyAsync(gains, static_cast<char*>(state) + g.gain, sizeof(double) * B,
+                                 cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+}
+
+EAGLE_API eagle_status eagle_tree_grow_finish(int dtype, int B, int V, int depth, int k, int levels, int m,
+                                              void* state, size_t state_bytes, const eagle_tree_t* out,
+                                              int* n_nodes, void* stream) {
   if (!out || !out->tokens || !out->parents || !out->depth || !out->logV || !out->draft_row || !out->row_lse)
     return EAGLE_ERR_NULL;
   const eagle_status st = grow_check(dtype, B, V, depth, k, state, state_bytes);
   if (st != EAGLE_OK) return st;
-  if (m <= 0) return EAGLE_ERR_SHAPE;
+  if (m <= 0 || levels < 1 || levels > depth) return EAGLE_ERR_SHAPE;
   if (m > EAGLE_MAX_NODES) return EAGLE_ERR_LIMIT;
-  const long long P = (long long)k + (long long)(depth - 1) * k * k;
+  const long long P = (long long)k + (long long)(levels - 1) * k * k;
   const int n = (int)(m < P ? m : P);
   if (n_nodes) *n_nodes = n;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -189,8 +212,8 @@ EAGLE_API eagle_status eagle_tree_grow_finish(int dtype, int B, int V, int depth
   cudaError_t e = cudaMemcpyAsync(out->row_lse, stp + g.row_lse, sizeof(double) * B * R, cudaMemcpyDeviceToDevice, s);
   if (e != cudaSuccess) return cuda_st(e);
   return cuda_st(launch_tree_expand(reinterpret_cast<const int32_t*>(stp + g.row_tok),
-                                    reinterpret_cast<const float*>(stp + g.row_val), B, R, depth, k, n, *out, nullptr,
-                                    false, s));
+                                    reinterpret_cast<const float*>(stp + g.row_val), B, R, levels, k, n, *out,
+                                    nullptr, false, s));
 }
 
 }  // extern "C"

@@ -1,0 +1,104 @@
+"""Cost-aware tree sizing: the EAGLE-4 harness's level-by-level decision
+(EAGLE-4 write-up, "Деревья проверки EAGLE-4 и утилита управления").
+
+A CostTable holds verification latencies measured on the GPU against batch
+size, context length and candidates per sequence (``calibrate.py`` measures
+this library's share of verification).  ``grow_sized`` drafts a tree level by
+level with a TreeGrower, asks the library after each level whether the level's
+gain in cumulative probability is worth its marginal cost, stops drafting at
+the first level that is not, and builds the tree of the levels kept.  The
+decision itself is the library's (``eagle_size_keep_level``); this module only
+marshals the table and drives the loop.
+"""
+from __future__ import annotations
+
+import ctypes
+import json
+from dataclasses import dataclass
+from typing import Callable, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from . import _lib as L
+
+
+@dataclass
+class CostTable:
+    """us[len(B)][len(L)][len(N)]: verification latency at each grid point (ascending grids)."""
+    B: np.ndarray
+    L: np.ndarray
+    N: np.ndarray
+    us: np.ndarray
+    unit: str = "us"
+
+    def __post_init__(self):
+        self.B, self.L, self.N = (np.ascontiguousarray(a, dtype=np.float64) for a in (self.B, self.L, self.N))
+        self.us = np.ascontiguousarray(self.us, dtype=np.float64)
+        if self.us.shape != (self.B.size, self.L.size, self.N.size):
+            raise ValueError(f"cost table: us has shape {self.us.shape}, grids give "
+                             f"{(self.B.size, self.L.size, self.N.size)}")
+
+    def struct(self) -> L.CostTableStruct:
+        p = lambda a: ctypes.c_void_p(a.ctypes.data)
+        return L.CostTableStruct(self.B.size, self.L.size, self.N.size, p(self.B), p(self.L), p(self.N), p(self.us))
+
+    def at(self, B: float, L_: float, N: float) -> float:
+        return float(L.lib().eagle_cost_at(ctypes.byref(self.struct()), B, L_, N))
+
+    def keep_level(self, B: float, L_: float, k: int, level: int, gains: Sequence[float],
+                   threshold: float) -> Tuple[bool, float]:
+        g = np.ascontiguousarray(np.asarray(gains, dtype=np.float64).reshape(-1))
+        keep, ratio = ctypes.c_int(0), ctypes.c_double(0.0)
+        L._check(L.lib().eagle_size_keep_level(ctypes.byref(self.struct()), B, L_, k, level,
+                                                   ctypes.c_void_p(g.ctypes.data), g.size, threshold,
+                                                   ctypes.byref(keep), ctypes.byref(ratio)),
+                 "eagle_size_keep_level")
+        return bool(keep.value), float(ratio.value)
+
+    def to_json(self, path: str, **meta):
+        with open(path, "w") as f:
+            json.dump({"B": self.B.tolist(), "L": self.L.tolist(), "N": self.N.tolist(), "us": self.us.tolist(),
+                       "unit": self.unit, **meta}, f, indent=1)
+
+    @classmethod
+    def from_json(cls, path: str) -> "CostTable":
+        with open(path) as f:
+            d = json.load(f)
+        return cls(np.array(d["B"]), np.array(d["L"]), np.array(d["N"]), np.array(d["us"]), d.get("unit", "us"))
+
+
+@dataclass
+class SizedTree:
+    tree: Optional[L.Tree]     # None when no level was worth verifying
+    levels_kept: int
+    levels_drafted: int
+    ratios: list               # each drafted level's gain / marginal cost
+
+
+def grow_sized(grower: L.TreeGrower, root_logits: torch.Tensor,
+               draft_fn: Callable[[int, torch.Tensor, torch.Tensor], torch.Tensor], table: CostTable,
+               context_len: float, threshold: float) -> SizedTree:
+    """Draft level by level while each level pays for itself.
+
+    draft_fn(level, frontier_tokens [B][k], frontier_parents [B][k]) -> that level's rows [B][k][V] on the
+    device (the draft model's distributions after each frontier node).  After each level the per-sequence
+    gains are read back (one small device-to-host copy: the host decides whether to run the draft model
+    again) and the library's decision applied.  The tree keeps m = k x (levels kept) candidates, the best
+    by V over every level drafted."""
+    B, k = grower.B, grower.k
+    tok, par = grower.begin(root_logits)
+    kept, drafted, ratios = 0, 0, []
+    for level in range(1, grower.depth + 1):
+        if level > 1:
+            tok, par = grower.level(draft_fn(level, tok, par), level)
+        drafted = level
+        keep, ratio = table.keep_level(B, context_len, k, level, grower.gains().cpu().numpy(), threshold)
+        ratios.append(ratio)
+        if not keep:
+            break
+        kept = level
+    if kept == 0:
+        return SizedTree(None, 0, drafted, ratios)
+    m = min(k * kept, L.MAX_NODES)
+    return SizedTree(grower.finish(m, levels=drafted), kept, drafted, ratios)

@@ -250,12 +250,20 @@ EAGLE_API eagle_status eagle_accept(const void* target_logits, int target_dtype,
  *     (-1: the root);
  *   eagle_tree_grow_level(level_logits [B][k][V], level = 2..depth): row s is
  *     the distribution after frontier slot s of the previous level (draft row
- *     1 + (level-2)k + s of eagle_tree_build); writes the level's frontier
- *     (tokens, and each one's parent as a slot of the previous frontier) while
- *     level < depth;
- *   eagle_tree_grow_finish(m, out): the tree, equal bit for bit to
- *     eagle_tree_build on the same rows (same kernels, same fp64 log V, the
- *     rows' log-sum-exps summed in the same order).
+ *     1 + (level-2)k + s of eagle_tree_build); writes the level's k best
+ *     candidates, the next frontier (tokens, and each one's parent as a slot
+ *     of the previous frontier);
+ *   eagle_tree_grow_gains(gains [B] double, device): after begin or a level,
+ *     per sequence the sum of V = exp(log V) over that level's k best
+ *     candidates, the expected number of tokens they add (the gain a
+ *     cost-aware harness weighs against the level's cost; EAGLE-4 write-up,
+ *     "Деревья проверки EAGLE-4 и утилита управления");
+ *   eagle_tree_grow_finish(levels, m, out): the tree over the first `levels`
+ *     levels grown (1 <= levels <= depth; n = min(m, k + (levels-1)k^2)),
+ *     equal bit for bit to eagle_tree_build with that depth on the same rows
+ *     (same kernels, same fp64 log V, the rows' log-sum-exps summed in the
+ *     same order).  out->row_lse is [B][R] with R = 1 + (depth-1)k; rows of
+ *     levels not grown are undefined.
  * frontier pointers may be NULL.  state: eagle_tree_grow_state_bytes bytes,
  * 256-byte aligned, kept by the caller from begin to finish (it holds every
  * row's top-k and log-sum-exp and the frontier's log V).  Limits: those of
@@ -267,9 +275,69 @@ EAGLE_API eagle_status eagle_tree_grow_begin(const void* root_logits, int dtype,
 EAGLE_API eagle_status eagle_tree_grow_level(const void* level_logits, int dtype, int B, int V, int depth, int k,
                                              int level, void* state, size_t state_bytes, int32_t* frontier_tokens,
                                              int32_t* frontier_parents, void* stream);
-EAGLE_API eagle_status eagle_tree_grow_finish(int dtype, int B, int V, int depth, int k, int m, void* state,
-                                              size_t state_bytes, const eagle_tree_t* out, int* n_nodes,
-                                              void* stream);
+EAGLE_API eagle_status eagle_tree_grow_gains(int dtype, int B, int V, int depth, int k, void* state,
+                                             size_t state_bytes, double* gains, void* stream);
+EAGLE_API eagle_status eagle_tree_grow_finish(int dtype, int B, int V, int depth, int k, int levels, int m,
+                                              void* state, size_t state_bytes, const eagle_tree_t* out,
+                                              int* n_nodes, void* stream);
+
+/* ------------------------------------------------- cost-aware tree sizing
+ * EAGLE-4 write-up, "Деревья проверки EAGLE-4 и утилита управления": a table
+ * of verification latency against batch size, context length and candidates
+ * per sequence, measured once on the GPU; at each draft level the gain in
+ * cumulative probability over the level's marginal cost against a threshold.
+ * Host functions (no device access, no stream):
+ *   table: ascending grids B[nB], L[nL], N[nN] (N = candidates verified per
+ *     sequence) and latencies us[nB][nL][nN] (any time unit), all finite,
+ *     host memory owned by the caller.  Cost between grid points:
+ *     multilinear interpolation; outside the grid the end segments are
+ *     extended; an axis with one point is constant.
+ *   eagle_cost_at: the interpolated cost, NaN for an invalid table.
+ *   eagle_size_keep_level: level l (1-based) grows the verified set from
+ *     (l-1)k to lk candidates per sequence; ratio = sum(gains[0..nb)) /
+ *     (C(B, L, lk) - C(B, L, (l-1)k)), infinite when the cost does not grow;
+ *     *keep = ratio >= threshold.  gains: HOST [nb], the level's per-sequence
+ *     gains (eagle_tree_grow_gains).  A harness drafts level l + 1 only while
+ *     level l is kept, and verifies m = k x (levels kept) candidates.
+ *     ratio may be NULL.  Errors: EAGLE_ERR_NULL, EAGLE_ERR_SHAPE (invalid
+ *     table or arguments). */
+typedef struct {
+  int nB, nL, nN;
+  const double* B;
+  const double* L;
+  const double* N;
+  const double* us; /* [nB][nL][nN] */
+} eagle_cost_table_t;
+EAGLE_API double eagle_cost_at(const eagle_cost_table_t* table, double B, double L, double N);
+EAGLE_API eagle_status eagle_size_keep_level(const eagle_cost_table_t* table, double B, double L, int k, int level,
+                                             const double* gains, int nb, double threshold, int* keep,
+                                             double* ratio);
+
+/* -------------------------------------------------------- static tree
+ * EAGLE-1's fixed draft tree ("EAGLE" notes, "1. EAGLE pipeline / Draft
+ * Model"): one template for every step; node i's token is the rank-r_i token
+ * of its parent's draft row (by logit, ties to the lower token id).
+ *   parents [n], ranks [n]: HOST arrays, the template.  parents[i] is the
+ *     parent of node i+1: 0 for the root, else a node id <= i (a parent comes
+ *     first).  ranks[i] in [0, EAGLE_MAX_TOPK); siblings have distinct ranks.
+ *     n <= EAGLE_MAX_NODES.  The template is copied into the launch
+ *     parameters: the arrays may be freed when the call returns.
+ *   draft_logits [B][R][V] (dtype): row 0 is the root's; every node with a
+ *     child owns a row, numbered 1, 2, ... in node order;
+ *     R = eagle_static_tree_rows(parents, ranks, n).
+ *   out: as for eagle_tree_build, with n nodes per sequence in template order;
+ *     gid (optional) = the node's template index i; row_lse [B][R].
+ * An invalid template returns EAGLE_ERR_SHAPE (eagle_static_tree_rows: -1),
+ * a largest rank >= V EAGLE_ERR_LIMIT.  Two launches: the vocabulary sweep
+ * (k = largest rank + 1) and the fill kernel.
+ * Workspace: eagle_static_tree_workspace_bytes (0 for an invalid template). */
+EAGLE_API int eagle_static_tree_rows(const int32_t* parents, const int32_t* ranks, int n);
+EAGLE_API size_t eagle_static_tree_workspace_bytes(int B, int V, int dtype, const int32_t* parents,
+                                                   const int32_t* ranks, int n);
+EAGLE_API eagle_status eagle_static_tree_build(const void* draft_logits, int dtype, int B, int R, int V,
+                                               const int32_t* parents, const int32_t* ranks, int n,
+                                               const eagle_tree_t* out, void* workspace, size_t workspace_bytes,
+                                               void* stream);
 
 /* ------------------------------------------------- KV-cache compaction
  * After acceptance ("Технический анализ EAGLE-4", section "Деревья проверки

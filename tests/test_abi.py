@@ -197,6 +197,31 @@ def test_tree_grow_validation(lib):
     lvl = lambda level: lib.eagle_tree_grow_level(FAKE, 0, 2, 32000, 6, 10, level, FAKE, nb, None, None, None)
     assert lvl(1) == 2 and lvl(7) == 2
     n = ctypes.c_int(0)
-    assert lib.eagle_tree_grow_finish(0, 2, 32000, 6, 10, 60, FAKE, nb, None, ctypes.byref(n), None) == 1
-    assert lib.eagle_tree_grow_finish(0, 2, 32000, 6, 10, 129, FAKE, nb, ctypes.byref(_tree()), ctypes.byref(n),
-                                      None) == 4
+    fin = lambda levels, m, t: lib.eagle_tree_grow_finish(0, 2, 32000, 6, 10, levels, m, FAKE, nb, t,
+                                                         ctypes.byref(n), None)
+    assert fin(6, 60, None) == 1
+    assert fin(6, 129, ctypes.byref(_tree())) == 4
+    assert fin(0, 60, ctypes.byref(_tree())) == 2 and fin(7, 60, ctypes.byref(_tree())) == 2
+    assert lib.eagle_tree_grow_gains(0, 2, 32000, 6, 10, FAKE, nb, None, None) == 1
+
+
+def test_static_tree_validation(lib):
+    arr = lambda v: (ctypes.c_int32 * len(v))(*v)
+    par, rk = arr([0, 0, 1, 1, 3]), arr([0, 1, 0, 1, 0])
+    assert lib.eagle_static_tree_rows(par, rk, 5) == 3
+    assert lib.eagle_static_tree_rows(arr([0, 2]), arr([0, 0]), 2) == -1      # parent after its child
+    assert lib.eagle_static_tree_rows(arr([0, 0]), arr([1, 1]), 2) == -1      # two siblings, one rank
+    assert lib.eagle_static_tree_rows(arr([0]), arr([32]), 1) == -1           # rank beyond the top-k limit
+    assert lib.eagle_static_tree_rows(par, rk, 0) == -1
+    nb = lib.eagle_static_tree_workspace_bytes(4, 1000, 1, par, rk, 5)
+    assert nb > 0 and nb % 256 == 0
+    assert lib.eagle_static_tree_workspace_bytes(4, 1000, 1, arr([0, 2]), arr([0, 0]), 2) == 0
+    t = _tree()
+    build = lambda **kw: lib.eagle_static_tree_build(kw.get("x", FAKE), 0, 4, kw.get("R", 3), kw.get("V", 1000),
+                                                     kw.get("par", par), rk, 5, ctypes.byref(t), FAKE,
+                                                     kw.get("nb", nb), None)
+    assert build(x=None) == 1
+    assert build(R=4) == 2
+    assert build(par=arr([0, 0, 1, 1, 5])) == 2
+    assert build(V=1) == 4                                                     # rank 1 needs two tokens
+    assert build(nb=nb - 1) == 5
