@@ -1,7 +1,8 @@
 """GPU parity: EAGLE-1 static tree (eagle_static_tree_build) against the oracle.
 
-Tokens, parents, depth, draft rows and node ids bit-exact; log V within 2e-6
-(stored as fp32), row log-sum-exp within 5e-7.  Templates: the hand-worked
+Tokens, parents, depth, draft rows and node ids bit-exact; log V within
+depth x 5e-7 (one row log-sum-exp per level) plus the fp32 store's half ulp,
+row log-sum-exp within 5e-7.  Templates: the hand-worked
 one, the full k-ary tree of depth 2, kept dynamic trees re-read as templates
 (the shapes EAGLE-2 produces), a long rank-0 chain and a 128-node template;
 then a whole step on a static tree (mask, attention, sampled acceptance)
@@ -33,7 +34,10 @@ def _check(x_stored, dtype, parents, ranks):
         ref = oracle.build_static_tree(x64[b], parents, ranks)
         for f in ("tokens", "parents", "depth", "draft_row", "gid"):
             assert getattr(tree, f)[b].cpu().numpy().tolist() == ref[f].tolist(), (b, f)
-        np.testing.assert_allclose(tree.logV[b].cpu().numpy(), ref["logV"], rtol=0, atol=2e-6)
+        # each row log-sum-exp on the path is within 5e-7 of fp64, and the fp32
+        # store rounds by half an ulp of |log V|
+        bound = ref["depth"] * 5e-7 + np.abs(ref["logV"]) * 2.0 ** -24 + 1e-7
+        assert np.all(np.abs(tree.logV[b].cpu().numpy() - ref["logV"]) <= bound), b
         np.testing.assert_allclose(tree.row_lse[b].cpu().numpy(), ref["row_lse"], rtol=0, atol=5e-7)
         refs.append(ref)
     return tree, refs
