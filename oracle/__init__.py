@@ -25,6 +25,8 @@ Everything is plain numpy in fp64, written step by step from the pages:
                 resampling (EAGLE-2 "Well-Calibrated Draft Model" formula;
                 aivaro.ru EAGLE-3 answer, section 4 steps 3-4; EAGLE-4
                 write-up, same section as the mask).
+* ``paged``     the prefix cache as pages of a shared pool named by a block
+                table: gather, and compaction into pages.
 * ``sizing``    cost-aware tree sizing: a measured latency table, each
                 level's gain in cumulative probability over its marginal cost
                 against a threshold (EAGLE-4 write-up, same section).
@@ -45,4 +47,5 @@ from .mask import ancestor_mask, pack_mask, positions  # noqa: F401
 from .attention import tree_attention, tree_attention_rows  # noqa: F401
 from .accept import accept_greedy, accept_stochastic, inverse_cdf  # noqa: F401
 from .kv import compact_kv  # noqa: F401
+from .paged import compact_kv_paged, gather_pages  # noqa: F401
 from .sizing import cost_at, keep_level, level_ratio, levels_kept  # noqa: F401
