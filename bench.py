@@ -10,6 +10,7 @@ steps, so every step reads its KV cache and logits from HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
                     [--mode stochastic|stochastic-wor|greedy] [--impl ours|reference]
+                    [--paged PAGE_SIZE]
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own replica of
 the workload (the step has no cross-sequence exchange); the job value is the
@@ -57,6 +58,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
+                    help="prefix cache as a shuffled pool of pages of this many keys (16, 32 or a multiple of 64)")
     return ap.parse_args()
 
 
@@ -77,6 +80,23 @@ def step_bytes(cfg, plen, mode):
     accept = target + (draft if mode.startswith("stochastic") else 0)
     return {"draft": draft, "attention": kv + attn_other, "kv": kv, "accept": accept,
             "step": draft + kv + attn_other + accept}
+
+
+def page_caches(torch, kc, vc, ps: int, room: int, seed: int):
+    """Dense caches [B][Hkv][L][D] -> pools [num_pages][Hkv][ps][D] whose pages (every sequence's, with room
+    for `room` more keys) are shuffled through the pool, and the block table [B][pages_per_seq]."""
+    B, Hkv, L, D = kc.shape
+    pps = (L + room + ps - 1) // ps
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(B * pps, generator=g).to(kc.device)
+    pools = []
+    for c in (kc, vc):
+        pad = torch.zeros(B, Hkv, pps * ps, D, dtype=c.dtype, device=c.device)
+        pad[:, :, :L] = c
+        pool = torch.empty(B * pps, Hkv, ps, D, dtype=c.dtype, device=c.device)
+        pool[perm] = pad.view(B, Hkv, pps, ps, D).permute(0, 2, 1, 3, 4).reshape(B * pps, Hkv, ps, D)
+        pools.append(pool)
+    return pools[0], pools[1], perm.view(B, pps).to(torch.int32).contiguous()
 
 
 # ----------------------------------------------------------------- clocks
@@ -265,9 +285,11 @@ def main():
     def to_bf16(a):
         return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
 
-    shape = StepShape(B=cfg.B, Hq=cfg.Hq, Hkv=cfg.Hkv, D=cfg.D, Lmax=cfg.L, depth=cfg.depth, k=cfg.k, m=cfg.m,
-                      V=cfg.V, logits_dtype=tdt, window=cfg.window, stochastic=stoch,
-                      without_replacement=args.mode == "stochastic-wor")
+    ps = args.paged
+    pps = (cfg.L + cfg.depth + ps - 1) // ps if ps else 0
+    shape = StepShape(B=cfg.B, Hq=cfg.Hq, Hkv=cfg.Hkv, D=cfg.D, Lmax=pps * ps if ps else cfg.L, depth=cfg.depth,
+                      k=cfg.k, m=cfg.m, V=cfg.V, logits_dtype=tdt, window=cfg.window, stochastic=stoch,
+                      without_replacement=args.mode == "stochastic-wor", paged=ps > 0)
 
     # input sets: enough distinct sets that their bytes exceed 2x L2
     sb0 = step_bytes(cfg, gen_prefix_len(cfg, 0), args.mode)
@@ -282,6 +304,9 @@ def main():
         inp = {"draft_logits": to_logits(stored), "prefix_len": torch.from_numpy(plen).to(dev),
                "q": to_bf16(q), "k_cache": to_bf16(kc), "v_cache": to_bf16(vc), "k_tree": to_bf16(kt),
                "v_tree": to_bf16(vt), "uniforms": torch.from_numpy(gen_uniforms(cfg, seed)).to(dev)}
+        if ps:
+            inp["k_cache"], inp["v_cache"], inp["block_table"] = page_caches(torch, inp["k_cache"], inp["v_cache"],
+                                                                             ps, cfg.depth, seed)
         st = VerifyStep(shape, dev)
         st.build(inp["draft_logits"])
         torch.cuda.synchronize()
@@ -289,7 +314,8 @@ def main():
         inp["target_logits"] = to_logits(tgt)
         sets.append(inp)
         steps.append(st)
-        hosts.append({k: v.cpu().pin_memory() for k, v in inp.items() if k not in ("k_cache", "v_cache")})
+        hosts.append({k: v.cpu().pin_memory() for k, v in inp.items()
+                      if k not in ("k_cache", "v_cache", "block_table")})
     set_bytes = sum(sum(t.numel() * t.element_size() for t in s.values()) for s in sets)
 
     stream = torch.cuda.Stream(dev)
@@ -375,10 +401,16 @@ def main():
     # copies of its caches with room past the prefix (the workloads fill theirs)
     def room(t):
         return torch.cat([t, torch.zeros_like(t[:, :, :cfg.depth])], dim=2).contiguous()
-    cc = [(room(inp["k_cache"]), room(inp["v_cache"]), torch.empty_like(inp["prefix_len"])) for inp in sets]
-    comp_graphs = [capture(lambda st=st, inp=inp, c=c: et.kv_compact_into(
-        inp["k_tree"], inp["v_tree"], st.path, st.accepted_len, inp["prefix_len"], c[0], c[1], c[2]))
-        for st, inp, c in zip(steps, sets, cc)]
+    if ps:  # the pools already hold a page past each prefix
+        cc = [(inp["k_cache"].clone(), inp["v_cache"].clone(), torch.empty_like(inp["prefix_len"])) for inp in sets]
+        comp_graphs = [capture(lambda st=st, inp=inp, c=c: et.kv_compact_paged_into(
+            inp["k_tree"], inp["v_tree"], st.path, st.accepted_len, inp["prefix_len"], c[0], c[1],
+            inp["block_table"], c[2])) for st, inp, c in zip(steps, sets, cc)]
+    else:
+        cc = [(room(inp["k_cache"]), room(inp["v_cache"]), torch.empty_like(inp["prefix_len"])) for inp in sets]
+        comp_graphs = [capture(lambda st=st, inp=inp, c=c: et.kv_compact_into(
+            inp["k_tree"], inp["v_tree"], st.path, st.accepted_len, inp["prefix_len"], c[0], c[1], c[2]))
+            for st, inp, c in zip(steps, sets, cc)]
     compact_ms = timed(comp_graphs, K, W)
     torch.cuda.synchronize()
     acc_now = [int(st.accepted_len.sum()) for st in steps]
@@ -445,7 +477,7 @@ def main():
         "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 attention (fp32 accumulate), " + cfg.logits_dtype + " logits",
         "data": "synthetic (seeded; no weights or datasets)",
-        "config": {"workload": workload_desc(cfg, args.mode),
+        "config": {"workload": workload_desc(cfg, args.mode) + (f", paged KV cache ({ps}-key pages)" if ps else ""),
                    "l2": f"{n_sets} rotating input sets, {set_bytes / 2**20:.0f} MiB > 2x L2",
                    "graph": f"each step one eagle_verify_step call, as one CUDA graph ({launch_mode[0]})",
                    "parallelism": f"replicas x{world}"},

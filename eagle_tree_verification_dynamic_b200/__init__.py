@@ -18,6 +18,10 @@ from ._lib import (  # noqa: F401
     attention_workspace_bytes,
     exported_names,
     kv_compact,
+    kv_compact_paged,
+    kv_compact_paged_into,
+    tree_attention_paged,
+    tree_attention_paged_into,
     static_tree_build,
     static_tree_rows,
     kv_compact_into,

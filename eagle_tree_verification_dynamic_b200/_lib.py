@@ -41,7 +41,8 @@ class StepIn(ctypes.Structure):
                 ("B", _c_i), ("V", _c_i), ("depth", _c_i), ("k", _c_i), ("m", _c_i),
                 ("q", _c_p), ("k_cache", _c_p), ("v_cache", _c_p), ("prefix_len", _c_p), ("Lmax", _c_i),
                 ("k_tree", _c_p), ("v_tree", _c_p), ("Hq", _c_i), ("Hkv", _c_i), ("D", _c_i), ("window", _c_i),
-                ("scale", _c_f), ("uniforms", _c_p), ("sampling_rule", _c_i)]
+                ("scale", _c_f), ("uniforms", _c_p), ("sampling_rule", _c_i),
+                ("block_table", _c_p), ("page_size", _c_i), ("pages_per_seq", _c_i), ("num_pages", _c_i)]
 
 
 class CostTableStruct(ctypes.Structure):
@@ -87,6 +88,10 @@ _SIGS = {
     "eagle_size_keep_level": (_c_i, [ctypes.POINTER(CostTableStruct), ctypes.c_double, ctypes.c_double, _c_i, _c_i,
                                      _c_p, _c_i, ctypes.c_double, ctypes.POINTER(_c_i),
                                      ctypes.POINTER(ctypes.c_double)]),
+    "eagle_tree_attention_paged": (_c_i, [_c_p, _c_p, _c_p, _c_i, _c_i, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                          _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p, _c_sz, _c_p]),
+    "eagle_kv_compact_paged": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_p, _c_i, _c_p, _c_i,
+                                      _c_i, _c_i, _c_i, _c_i, _c_p]),
     "eagle_kv_compact": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                 _c_p]),
     "eagle_accept_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i]),
@@ -281,11 +286,57 @@ def tree_attention(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos=No
 
 def check_attention_status(ws: torch.Tensor):
     """Read the device status word the attention kernel keeps in its workspace
-    header (synchronises the stream).  Non-zero (1) means a bounded wait inside
-    the kernel gave up."""
+    header (synchronises the stream).  1: a bounded wait inside the kernel gave
+    up; 3: a paged cache named a page outside its pool for a key in use."""
     code = int(ws[:4].view(torch.int32).item())
     if code != 0:
         raise EagleError(f"eagle_tree_attention: device status {code}")
+
+
+# ------------------------------------------------------- paged prefix cache
+def tree_attention_paged_into(q, k_pages, v_pages, block_table, prefix_len, k_tree, v_tree, mask, pos, out, ws,
+                              window: int = 0, scale: float = 0.0):
+    """k_pages / v_pages [num_pages][Hkv][page_size][D] bf16, block_table [B][pages_per_seq] int32."""
+    B, n, Hq, D = q.shape
+    num_pages, Hkv, ps = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    _check(lib().eagle_tree_attention_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), num_pages, ps, _ptr(block_table),
+                                            block_table.shape[1], _ptr(prefix_len), _ptr(k_tree), _ptr(v_tree),
+                                            _ptr(mask), _ptr(pos), B, n, Hq, Hkv, D, window, scale, _ptr(out),
+                                            _ptr(ws), ws.numel(), _stream(q.device)), "eagle_tree_attention_paged")
+
+
+def tree_attention_paged(q, k_pages, v_pages, block_table, prefix_len, k_tree, v_tree, mask, pos=None,
+                         window: int = 0, scale: float = 0.0, check: bool = True) -> torch.Tensor:
+    """Tree attention over a paged prefix cache -> out [B][n][Hq][D] bf16 (raises on a device status when
+    check, e.g. a page id outside the pool for a key in use)."""
+    _need_cuda(q, k_pages, v_pages, block_table, prefix_len, k_tree, v_tree, mask, pos)
+    B, n, Hq, D = q.shape
+    Hkv, ps = k_pages.shape[1], k_pages.shape[2]
+    out = torch.empty_like(q)
+    ws = _workspace(attention_workspace_bytes(B, n, Hq, Hkv, D, block_table.shape[1] * ps, window), q.device)
+    tree_attention_paged_into(q, k_pages, v_pages, block_table, prefix_len, k_tree, v_tree, mask, pos, out, ws,
+                              window, scale)
+    if check:
+        check_attention_status(ws)
+    return out
+
+
+def kv_compact_paged_into(k_tree, v_tree, path, accepted_len, prefix_len, k_pages, v_pages, block_table,
+                          new_prefix_len):
+    """kv_compact into a paged cache (pools updated in place); new lengths into new_prefix_len."""
+    B, n, Hkv, D = k_tree.shape
+    _check(lib().eagle_kv_compact_paged(_ptr(k_tree), _ptr(v_tree), _ptr(path), _ptr(accepted_len), _ptr(prefix_len),
+                                        _ptr(k_pages), _ptr(v_pages), k_pages.shape[0], k_pages.shape[2],
+                                        _ptr(block_table), block_table.shape[1], _ptr(new_prefix_len), B, n, Hkv, D,
+                                        path.shape[1], _stream(k_tree.device)), "eagle_kv_compact_paged")
+
+
+def kv_compact_paged(k_tree, v_tree, path, accepted_len, prefix_len, k_pages, v_pages, block_table) -> torch.Tensor:
+    """kv_compact into a paged cache (pools updated in place) -> new prefix lengths [B] int32."""
+    _need_cuda(k_tree, v_tree, path, accepted_len, prefix_len, k_pages, v_pages, block_table)
+    new_len = torch.empty_like(prefix_len)
+    kv_compact_paged_into(k_tree, v_tree, path, accepted_len, prefix_len, k_pages, v_pages, block_table, new_len)
+    return new_len
 
 
 # -------------------------------------------------------------------- accept
@@ -328,17 +379,20 @@ def accept(target_logits, tokens, parents, draft_row, depth: int, uniforms=None,
 
 # ---------------------------------------------------------------- one step
 def step_in(draft_logits, target_logits, depth, k, m, q, k_cache, v_cache, prefix_len, k_tree, v_tree,
-            uniforms=None, window: int = 0, scale: float = 0.0, without_replacement: bool = False) -> StepIn:
+            uniforms=None, window: int = 0, scale: float = 0.0, without_replacement: bool = False,
+            block_table=None) -> StepIn:
     """The C step's inputs: draft_logits [B][R][V] and target_logits [B][n+1][V] (f32 or bf16),
     q [B][n][Hq][D], caches [B][Hkv][Lmax][D], tree K/V [B][n][Hkv][D] (bf16), prefix_len [B] int32,
     uniforms [B][2][n+1] f32 or None (greedy)."""
     B, R, V = draft_logits.shape
     Hq, D = q.shape[2], q.shape[3]
     Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    paged = (_ptr(block_table), k_cache.shape[2], block_table.shape[1], k_cache.shape[0]) if block_table is not None \
+        else (None, 0, 0, 0)
     return StepIn(_ptr(draft_logits), _ptr(target_logits), _dtype_code(draft_logits), B, V, depth, k, m,
-                  _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), Lmax, _ptr(k_tree), _ptr(v_tree),
-                  Hq, Hkv, D, window, scale, _ptr(uniforms),
-                  SAMPLE_WITHOUT_REPLACEMENT if without_replacement else SAMPLE_WITH_REPLACEMENT)
+                  _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), 0 if block_table is not None else Lmax,
+                  _ptr(k_tree), _ptr(v_tree), Hq, Hkv, D, window, scale, _ptr(uniforms),
+                  SAMPLE_WITHOUT_REPLACEMENT if without_replacement else SAMPLE_WITH_REPLACEMENT, *paged)
 
 
 def step_workspace_bytes(si: StepIn) -> int:

@@ -13,8 +13,9 @@ tokens to these numbers.  N = 0 costs nothing (there is nothing to verify).
         [--B 1,4,16,32] [--L 1024,4096,16384] [--N 0,8,16,32,64,96,128] \
         [--Hq 32 --Hkv 8 --D 128 --V 128256 --dtype bf16]
 
-Inputs are random device tensors; the L2 cache is flushed before every timed
-repetition and the median of the repetitions is kept.
+Inputs are random device tensors; the three calls are captured in one CUDA
+graph (device time, without the host's per-call overhead), the L2 cache is
+flushed before every timed replay and the median of the replays is kept.
 """
 from __future__ import annotations
 
@@ -73,17 +74,25 @@ def measure_point(B: int, Lctx: int, n: int, Hq: int, Hkv: int, D: int, V: int, 
         L.tree_attention_into(q, kc, vc, plen, kt, vt, mask, pos, out, ws_a)
         L.accept_into(target, tokens, parents, draft_row, max_depth, None, None, None, acc, path, bonus, ws_c)
 
-    for _ in range(3):
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):  # sets the kernels' attributes before capture
+            verify()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
         verify()
     times = []
-    for _ in range(reps):
-        flush.add_(1)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        verify()
-        b.record()
-        b.synchronize()
-        times.append(a.elapsed_time(b) * 1000.0)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            flush.add_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b) * 1000.0)
+    del graph
     return statistics.median(times)
 
 
@@ -114,7 +123,7 @@ def main():
     a = ap.parse_args()
     dtype = torch.bfloat16 if a.dtype == "bf16" else torch.float32
     t = calibrate(_ints(a.B), _ints(a.L), _ints(a.N), a.Hq, a.Hkv, a.D, a.V, dtype, a.reps)
-    t.to_json(a.out, what="mask + tree attention + greedy acceptance, median microseconds, L2 flushed",
+    t.to_json(a.out, what="mask + tree attention + greedy acceptance as one CUDA graph, median microseconds, L2 flushed",
               Hq=a.Hq, Hkv=a.Hkv, D=a.D, V=a.V, dtype=a.dtype, gpu=torch.cuda.get_device_name())
     print(f"wrote {a.out}: {t.us.size} points, {t.us.min():.1f}..{t.us.max():.1f} us")
 

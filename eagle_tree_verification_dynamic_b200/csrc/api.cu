@@ -166,6 +166,70 @@ eagle_status eagle_tree_attention(const void* q, const void* k_cache, const void
                                            static_cast<cudaStream_t>(stream)));
 }
 
+}  // extern "C"
+
+namespace {
+
+// A paged prefix cache's description: page_size 16, 32 or a multiple of 64;
+// every row index of the pools and every capacity fits in an int.
+eagle_status check_paged(const int32_t* block_table, int page_size, int pages_per_seq, int num_pages, int Hkv) {
+  if (!block_table) return EAGLE_ERR_NULL;
+  if (page_size <= 0 || pages_per_seq <= 0 || num_pages <= 0 || Hkv <= 0) return EAGLE_ERR_SHAPE;
+  if (!(page_size == 16 || page_size == 32 || page_size % 64 == 0)) return EAGLE_ERR_SHAPE;
+  if ((long long)num_pages * Hkv * page_size > 0x7fffffffLL) return EAGLE_ERR_LIMIT;
+  if ((long long)pages_per_seq * page_size > (1LL << 30)) return EAGLE_ERR_LIMIT;
+  return EAGLE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+eagle_status eagle_tree_attention_paged(const void* q, const void* k_pages, const void* v_pages, int num_pages,
+                                        int page_size, const int32_t* block_table, int pages_per_seq,
+                                        const int32_t* prefix_len, const void* k_tree, const void* v_tree,
+                                        const uint64_t* mask, const int32_t* pos, int B, int n, int Hq, int Hkv,
+                                        int D, int window, float scale, void* out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (!q || !k_pages || !v_pages || !k_tree || !v_tree || !mask || !prefix_len || !out) return EAGLE_ERR_NULL;
+  if (window > 0 && !pos) return EAGLE_ERR_NULL;
+  eagle_status st = check_paged(block_table, page_size, pages_per_seq, num_pages, Hkv);
+  if (st != EAGLE_OK) return st;
+  if (B <= 0 || n <= 0 || Hq <= 0 || window < 0 || Hq % Hkv != 0) return EAGLE_ERR_SHAPE;
+  if (D != 64 && D != 128) return EAGLE_ERR_LIMIT;
+  if (n > EAGLE_MAX_NODES) return EAGLE_ERR_LIMIT;
+  if (!aligned16(q) || !aligned16(k_tree) || !aligned16(v_tree) || !aligned16(out) || !aligned16(k_pages) ||
+      !aligned16(v_pages))
+    return EAGLE_ERR_ALIGN;
+  const int cap = pages_per_seq * page_size;
+  st = check_ws(workspace, workspace_bytes, attention_ws_bytes(B, n, Hq, Hkv, D, cap, window));
+  if (st != EAGLE_OK) return st;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)D);
+  const PagedKV pg = {block_table, page_size, pages_per_seq, num_pages};
+  return cuda_status(launch_tree_attention(q, k_pages, v_pages, prefix_len, cap, k_tree, v_tree, mask, pos, B, n,
+                                           Hq, Hkv, D, window, scale, out, workspace,
+                                           static_cast<cudaStream_t>(stream), &pg));
+}
+
+eagle_status eagle_kv_compact_paged(const void* k_tree, const void* v_tree, const int32_t* path,
+                                    const int32_t* accepted_len, const int32_t* prefix_len, void* k_pages,
+                                    void* v_pages, int num_pages, int page_size, const int32_t* block_table,
+                                    int pages_per_seq, int32_t* new_prefix_len, int B, int n, int Hkv, int D,
+                                    int depth, void* stream) {
+  if (!k_tree || !v_tree || !path || !accepted_len || !prefix_len || !k_pages || !v_pages || !new_prefix_len)
+    return EAGLE_ERR_NULL;
+  eagle_status st = check_paged(block_table, page_size, pages_per_seq, num_pages, Hkv);
+  if (st != EAGLE_OK) return st;
+  if (B <= 0 || n <= 0 || D <= 0 || depth <= 0) return EAGLE_ERR_SHAPE;
+  if (D % 8 != 0 || new_prefix_len == prefix_len) return EAGLE_ERR_SHAPE;
+  if (n > EAGLE_MAX_NODES || depth > EAGLE_MAX_DEPTH || B > 65535) return EAGLE_ERR_LIMIT;
+  if (!aligned16(k_tree) || !aligned16(v_tree) || !aligned16(k_pages) || !aligned16(v_pages)) return EAGLE_ERR_ALIGN;
+  const PagedKV pg = {block_table, page_size, pages_per_seq, num_pages};
+  return cuda_status(launch_kv_compact(k_tree, v_tree, path, accepted_len, prefix_len, k_pages, v_pages,
+                                       new_prefix_len, B, n, Hkv, D, pages_per_seq * page_size, depth,
+                                       static_cast<cudaStream_t>(stream), &pg));
+}
+
 // --------------------------------------------------------------------- accept
 size_t eagle_accept_workspace_bytes(int B, int n, int V, int target_dtype) {
   if (B <= 0 || n <= 0 || V <= 0 || !valid_dtype(target_dtype)) return 0;
@@ -245,12 +309,17 @@ bool step_layout(const eagle_step_in_t* in, StepLayout* L) {
   const long long P = (long long)in->k + (long long)(in->depth - 1) * in->k * in->k;
   if (P > EAGLE_MAX_POOL) return false;
   if (in->Hq <= 0 || in->Hkv <= 0 || in->D <= 0 || in->Lmax < 0 || in->window < 0) return false;
+  if (in->block_table && (in->page_size <= 0 || in->pages_per_seq <= 0 ||
+                          (long long)in->pages_per_seq * in->page_size > (1LL << 30)))
+    return false;
+  // a paged cache holds up to pages_per_seq * page_size keys per sequence
+  const int cap = in->block_table ? in->pages_per_seq * in->page_size : in->Lmax;
   L->R = 1 + (in->depth - 1) * in->k;
   L->n = (int)(in->m < P ? in->m : P);
   const int eb = dtype_bytes(in->logits_dtype);
   L->build_off = 0;
   L->attn_off = align_up(tree_build_ws_bytes(in->B, L->R, in->V, eb, in->k), 256);
-  L->acc_off = align_up(L->attn_off + attention_ws_bytes(in->B, L->n, in->Hq, in->Hkv, in->D, in->Lmax, in->window), 256);
+  L->acc_off = align_up(L->attn_off + attention_ws_bytes(in->B, L->n, in->Hq, in->Hkv, in->D, cap, in->window), 256);
   L->total = align_up(L->acc_off + accept_ws_bytes(in->B, L->n, in->V, in->logits_dtype), 256);
   return true;
 }
@@ -279,7 +348,12 @@ eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t
   if (!t.tokens || !t.parents || !t.depth || !t.logV || !t.draft_row || !t.row_lse) return EAGLE_ERR_NULL;
   if (!out->mask || !out->pos || !out->attn_out || !out->accepted_len || !out->path || !out->bonus)
     return EAGLE_ERR_NULL;
-  if (in->Lmax > 0 && (!in->k_cache || !in->v_cache)) return EAGLE_ERR_NULL;
+  const bool paged = in->block_table != nullptr;
+  if ((paged || in->Lmax > 0) && (!in->k_cache || !in->v_cache)) return EAGLE_ERR_NULL;
+  if (paged) {
+    const eagle_status ps = check_paged(in->block_table, in->page_size, in->pages_per_seq, in->num_pages, in->Hkv);
+    if (ps != EAGLE_OK) return ps;
+  }
   if (!valid_dtype(in->logits_dtype)) return EAGLE_ERR_DTYPE;
   if (in->B <= 0 || in->V <= 0 || in->depth <= 0 || in->k <= 0 || in->m <= 0) return EAGLE_ERR_SHAPE;
   if (in->Hq <= 0 || in->Hkv <= 0 || in->Lmax < 0 || in->window < 0 || in->Hq % in->Hkv != 0) return EAGLE_ERR_SHAPE;
@@ -293,7 +367,7 @@ eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t
   if (in->sampling_rule != EAGLE_SAMPLE_WITH_REPLACEMENT && in->sampling_rule != EAGLE_SAMPLE_WITHOUT_REPLACEMENT)
     return EAGLE_ERR_SHAPE;
   if (!aligned16(in->q) || !aligned16(in->k_tree) || !aligned16(in->v_tree) || !aligned16(out->attn_out) ||
-      (in->Lmax > 0 && (!aligned16(in->k_cache) || !aligned16(in->v_cache))))
+      ((paged || in->Lmax > 0) && (!aligned16(in->k_cache) || !aligned16(in->v_cache))))
     return EAGLE_ERR_ALIGN;
   eagle_status st = check_ws(workspace, workspace_bytes, L.total);
   if (st != EAGLE_OK) return st;
@@ -319,9 +393,10 @@ eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t
   if (e != cudaSuccess) return cuda_status(e);
   // --- tree attention
   const float scale = in->scale > 0.f ? in->scale : 1.0f / sqrtf((float)in->D);
+  const PagedKV pg = {in->block_table, in->page_size, in->pages_per_seq, in->num_pages};
   e = launch_tree_attention(in->q, in->k_cache, in->v_cache, in->prefix_len, in->Lmax, in->k_tree, in->v_tree,
                             out->mask, out->pos, in->B, n, in->Hq, in->Hkv, in->D, in->window, scale, out->attn_out,
-                            ws + L.attn_off, s);
+                            ws + L.attn_off, s, paged ? &pg : nullptr);
   if (e != cudaSuccess) return cuda_status(e);
   // --- acceptance (the draft rows' log-sum-exps are the tree's row_lse)
   e = launch_accept(in->target_logits, in->logits_dtype, in->draft_logits, in->logits_dtype, t.row_lse, L.R,

@@ -99,6 +99,7 @@ struct TcBars {
   uint64_t pair[4];  // per lane quarter: both softmax warps wrote their (max, sum)
   uint32_t tmem_base;
   int abort;
+  int bad_page;  // a key inside the sequence sat on a page id outside the pool
   // this CTA's tile range [t0, t1) of the global list, and where it starts
   int n_tiles;  // t1 - t0
   int b0, hr0, off0;
@@ -109,6 +110,7 @@ static_assert(sizeof(TcBars) <= 512, "barrier block");  // kXchOff
 struct AttnGeom {
   const int32_t* plen;
   int B, Hkv, RG, n, Lmax, window, C;
+  int lo_align;  // the first prefix tile starts at a multiple of this (64 for a paged cache, else 1)
 };
 
 __device__ __forceinline__ int geom_len(const AttnGeom& a, int b) {
@@ -117,7 +119,8 @@ __device__ __forceinline__ int geom_len(const AttnGeom& a, int b) {
 // first visible prefix key of a sequence of length L (the window of the
 // shallowest tree node, depth 1, at position L)
 __device__ __forceinline__ int geom_lo(const AttnGeom& a, int L) {
-  return a.window > 0 ? max(0, L - a.window + 1) : 0;
+  const int lo = a.window > 0 ? max(0, L - a.window + 1) : 0;
+  return lo - lo % a.lo_align;  // keys below the window start are masked row by row
 }
 __device__ __forceinline__ int geom_ptiles(const AttnGeom& a, int L) { return (L - geom_lo(a, L) + kBN - 1) / kBN; }
 __device__ __forceinline__ int geom_tiles(const AttnGeom& a, int b) {
@@ -235,6 +238,10 @@ struct TcParams {
   int Hq;
   int q_by_tma;      // 1: Q rows arrive by TMA (G divides 128), 0: gathered by the producer warp
   float scale_log2;  // softmax scale * log2(e)
+  // paged prefix cache (block_table != null): pools [num_pages][Hkv][page_size][D],
+  // block_table [B][pages_per_seq] page ids
+  const int32_t* block_table;
+  int page_size, pages_per_seq, num_pages;
 };
 
 // Loads issued now and consumed later: the K/V stream keeps HBM saturated, so
@@ -285,6 +292,85 @@ __device__ __forceinline__ void row_issue(RowCtx& rc, const Piece& pc, const TcP
   }
 }
 
+// Block-table entry idx of a sequence (-1 past the table's width).
+__device__ __forceinline__ int table_entry(const int32_t* bt, int idx, int width) {
+  return idx < width ? ld_early_s32(bt + idx) : -1;
+}
+
+// Producer for a paged prefix cache: the K/V tiles of one piece.  A prefix
+// tile's 64 keys (starting at a multiple of 64) arrive as boxes of
+// min(page_size, 64) keys, each from the page the sequence's block table
+// names.  The whole warp walks the tiles (lane 0 waits and issues) and reads
+// the table 32 entries per coalesced load; the next 32 are requested as soon
+// as the current ones are first used, so only a piece's first lookup waits on
+// memory.  A page id outside the pool turns into a box past the end, which
+// reads zeros; if a key inside the sequence sat there, the CTA reports it.
+// Returns false when a wait gave up.
+template <int D>
+__device__ bool produce_paged(const TcParams& p, const AttnGeom& a, const Piece& pc, int g, uint32_t s_base,
+                              TcBars* bars, volatile int* abort, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                              const CUtensorMap* tm_kt, const CUtensorMap* tm_vt, int lane, int& jg) {
+  using Lay = TcLayout<D>;
+  constexpr int S = Lay::kStages;
+  const int ps = p.page_size;
+  const int sub = ps < kBN ? ps : kBN;  // keys per box
+  const int nsub = kBN / sub;           // boxes per tile: 1, 2 or 4
+  const int32_t* bt = p.block_table + (size_t)pc.b * p.pages_per_seq;
+  const int past_end = p.num_pages * a.Hkv * ps;  // first row past the pools (the host keeps it in int range)
+  int c0 = -64, cur = -1, nxt = -1;               // table chunk [c0, c0 + 32): lane l holds entry c0 + l
+  for (int t = pc.tb; t < pc.te; ++t) {
+    const int st = jg % S;
+    bool w = true;
+    if (lane == 0 && jg >= S) w = mbar_wait(smem_u32(&bars->empty[st]), ((jg / S) - 1) & 1, abort);
+    if (!__shfl_sync(kFull, w, 0)) return false;
+    const uint32_t fb = smem_u32(&bars->full[st]);
+    const uint32_t kdst = s_base + Lay::kStageOff + st * Lay::kStageBytes;
+    const uint32_t vdst = kdst + Lay::kKBytes;
+    if (t < pc.ptiles) {
+      const int key0 = pc.lo + t * kBN;
+      const int e0 = key0 / ps;  // the tile's first entry; its nsub entries share e0's chunk
+      const int base = e0 & ~31;
+      if (base != c0) {  // warp-uniform
+        cur = base == c0 + 32 ? nxt : table_entry(bt, base + lane, p.pages_per_seq);
+        c0 = base;
+        nxt = table_entry(bt, c0 + 32 + lane, p.pages_per_seq);
+      }
+      int row[4];
+      bool bad = false;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int page = __shfl_sync(kFull, cur, (e0 - c0 + j) & 31);  // every lane takes part
+        const int kj = key0 + j * sub;
+        const bool valid = page >= 0 && page < p.num_pages;
+        if (j < nsub && !valid && kj < pc.L) bad = true;
+        row[j] = valid ? (page * a.Hkv + g) * ps + kj % ps : past_end;
+      }
+      if (lane == 0) {
+        if (bad) bars->bad_page = 1;
+        mbar_arrive_expect_tx(fb, Lay::kStageBytes);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (j < nsub) {
+            for (int at = 0; at < Lay::kAtoms; ++at) {
+              tma_load_2d(kdst + at * Lay::kKVAtomBytes + j * sub * 128, tm_k, at * 64, row[j], fb);
+              tma_load_2d(vdst + at * Lay::kKVAtomBytes + j * sub * 128, tm_v, at * 64, row[j], fb);
+            }
+          }
+        }
+      }
+    } else if (lane == 0) {
+      mbar_arrive_expect_tx(fb, Lay::kStageBytes);
+      const int z = pc.b * a.n + (t - pc.ptiles) * kBN;
+      for (int at = 0; at < Lay::kAtoms; ++at) {
+        tma_load_3d(kdst + at * Lay::kKVAtomBytes, tm_kt, at * 64, g, z, fb);
+        tma_load_3d(vdst + at * Lay::kKVAtomBytes, tm_vt, at * 64, g, z, fb);
+      }
+    }
+    ++jg;
+  }
+  return true;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -330,6 +416,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     mbar_init(smem_u32(&bars->mma_idle), 1);
     for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars->pair[i]), 64);
     bars->abort = 0;
+    bars->bad_page = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -443,7 +530,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         if (lane == 0) mbar_arrive(qbar);
       }
       ++si;
-      if (lane == 0) {
+      if (p.block_table != nullptr) {
+        ok = produce_paged<D>(p, a, pc, g, s_base, bars, abort, &tm_k, &tm_v, &tm_kt, &tm_vt, lane, jg);
+      } else if (lane == 0) {
         for (int t = pc.tb; t < pc.te; ++t) {
           const int st = jg % S;
           if (jg >= S && !mbar_wait(smem_u32(&bars->empty[st]), ((jg / S) - 1) & 1, abort)) {
@@ -752,7 +841,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, Lay::kTmemCols);
-  if (tid == 0) p.cta_status[c] = bars->abort ? 1 : 0;
+  if (tid == 0) p.cta_status[c] = bars->abort ? 1 : (bars->bad_page ? 3 : 0);
 }
 
 // Merge the pieces of every unit cut by CTA range boundaries:
@@ -902,12 +991,21 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
 template <int D>
 static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
                              const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
-                             int n, int Hq, int Hkv, int window, float scale, void* out, void* ws, cudaStream_t s) {
+                             int n, int Hq, int Hkv, int window, float scale, void* out, void* ws, cudaStream_t s,
+                             const PagedKV* pg) {
   CUtensorMap mk, mv, mkt, mvt;
+  const bool paged = pg != nullptr && pg->block_table != nullptr;
+  if (paged) Lmax = pg->pages_per_seq * pg->page_size;  // a sequence's capacity
   const int Lrows = Lmax > 0 ? Lmax : 1;
   const void* kbase = Lmax > 0 ? kc : kt;  // any valid address when the cache is empty
   const void* vbase = Lmax > 0 ? vc : vt;
-  {
+  if (paged) {
+    // pools [num_pages][Hkv][page_size][D] as rows of D; a box is min(page_size, 64) keys
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pg->num_pages * Hkv * pg->page_size};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)(pg->page_size < kBN ? pg->page_size : kBN)};
+    if (!make_map(&mk, kc, 2, dims, str, box) || !make_map(&mv, vc, 2, dims, str, box)) return cudaErrorInvalidValue;
+  } else {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)B * Hkv * Lrows};
     const cuuint64_t str[1] = {(cuuint64_t)D * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)kBN};
@@ -950,7 +1048,12 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
   p.geo.Lmax = Lmax;
   p.geo.window = window;
   p.geo.C = attention_ctas(B, n, Hq, Hkv, Lmax, window);
+  p.geo.lo_align = paged ? kBN : 1;
   p.Hq = Hq;
+  p.block_table = paged ? pg->block_table : nullptr;
+  p.page_size = paged ? pg->page_size : 0;
+  p.pages_per_seq = paged ? pg->pages_per_seq : 0;
+  p.num_pages = paged ? pg->num_pages : 0;
   p.q_by_tma = q_tma ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = TcLayout<D>::kSmemBytes;
@@ -993,10 +1096,10 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
 cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
                                   const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
                                   int n, int Hq, int Hkv, int D, int window, float scale, void* out, void* ws,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, const PagedKV* pg) {
   if (D == 128)
-    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s);
-  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s);
+    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s, pg);
+  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s, pg);
 }
 
 }  // namespace eagle

@@ -105,15 +105,23 @@ AttnWorkspace attention_ws_layout(int B, int n, int Hq, int Hkv, int D, int Lmax
 inline size_t attention_ws_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window) {
   return attention_ws_layout(B, n, Hq, Hkv, D, Lmax, window).bytes;
 }
+// A paged prefix cache: pools [num_pages][Hkv][page_size][D], block_table
+// [B][pages_per_seq] page ids; page_size is 16, 32 or a multiple of 64.
+struct PagedKV {
+  const int32_t* block_table;
+  int page_size, pages_per_seq, num_pages;
+};
+// pg == nullptr: dense caches [B][Hkv][Lmax][D]; else kc / vc are the pools
+// and a sequence holds up to pages_per_seq * page_size keys (Lmax unused).
 cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen,
                                   int Lmax, const void* kt, const void* vt, const uint64_t* mask,
                                   const int32_t* pos, int B, int n, int Hq, int Hkv, int D, int window,
-                                  float scale, void* out, void* ws, cudaStream_t s);
+                                  float scale, void* out, void* ws, cudaStream_t s, const PagedKV* pg = nullptr);
 
 // ---- KV-cache compaction after acceptance (kv_compact.cu)
 cudaError_t launch_kv_compact(const void* k_tree, const void* v_tree, const int32_t* path, const int32_t* accepted_len,
                               const int32_t* prefix_len, void* k_cache, void* v_cache, int32_t* new_len, int B, int n,
-                              int Hkv, int D, int Lmax, int depth, cudaStream_t s);
+                              int Hkv, int D, int Lmax, int depth, cudaStream_t s, const PagedKV* pg = nullptr);
 
 // ---- accept (accept.cu)
 size_t accept_ws_bytes(int B, int n, int V, int dtype);

@@ -33,6 +33,7 @@ class StepShape:
     window: int = 0
     stochastic: bool = True
     without_replacement: bool = False   # sampled acceptance: a rejected child's token leaves q
+    paged: bool = False                 # prefix cache as page pools + block table (Lmax = pages_per_seq x page_size)
 
     @property
     def R(self) -> int:
@@ -71,9 +72,13 @@ class VerifyStep:
     def mask_(self, prefix_len: torch.Tensor):
         L.tree_mask_into(self.tree.parents, self.tree.depth, prefix_len, self.mask, self.pos)
 
-    def attention(self, q, k_cache, v_cache, prefix_len, k_tree, v_tree):
-        L.tree_attention_into(q, k_cache, v_cache, prefix_len, k_tree, v_tree, self.mask, self.pos, self.out,
-                              self.ws_attn, self.s.window)
+    def attention(self, q, k_cache, v_cache, prefix_len, k_tree, v_tree, block_table=None):
+        if self.s.paged:
+            L.tree_attention_paged_into(q, k_cache, v_cache, block_table, prefix_len, k_tree, v_tree, self.mask,
+                                        self.pos, self.out, self.ws_attn, self.s.window)
+        else:
+            L.tree_attention_into(q, k_cache, v_cache, prefix_len, k_tree, v_tree, self.mask, self.pos, self.out,
+                                  self.ws_attn, self.s.window)
 
     def accept(self, target_logits, uniforms: Optional[torch.Tensor], draft_logits):
         if self.s.stochastic:
@@ -90,7 +95,8 @@ class VerifyStep:
         si = L.step_in(inp["draft_logits"], inp["target_logits"], s.depth, s.k, s.m, inp["q"], inp["k_cache"],
                        inp["v_cache"], inp["prefix_len"], inp["k_tree"], inp["v_tree"],
                        inp.get("uniforms") if s.stochastic else None, s.window,
-                       without_replacement=s.without_replacement)
+                       without_replacement=s.without_replacement,
+                       block_table=inp["block_table"] if s.paged else None)
         L.step_into(si, self.tree, self.mask, self.pos, self.out, self.accepted_len, self.path, self.bonus,
                     self.ws_step, self.device)
         self._step_in = si
@@ -104,6 +110,7 @@ class VerifyStep:
         """inp: draft_logits, prefix_len, q, k_cache, v_cache, k_tree, v_tree, target_logits, uniforms."""
         self.build(inp["draft_logits"])
         self.mask_(inp["prefix_len"])
-        self.attention(inp["q"], inp["k_cache"], inp["v_cache"], inp["prefix_len"], inp["k_tree"], inp["v_tree"])
+        self.attention(inp["q"], inp["k_cache"], inp["v_cache"], inp["prefix_len"], inp["k_tree"], inp["v_tree"],
+                       inp.get("block_table"))
         self.accept(inp["target_logits"], inp.get("uniforms"), inp["draft_logits"])
         return self.accepted_len, self.path, self.bonus

@@ -176,7 +176,8 @@ EAGLE_API eagle_status eagle_tree_mask(const int32_t* parents, const int32_t* de
  * Limits: D in {64, 128}, Hq % Hkv == 0, n <= EAGLE_MAX_NODES, all tensor
  * pointers 16-byte aligned.  Workspace: eagle_tree_attention_workspace_bytes.
  * It starts with a 256-byte header whose first int is the device status word,
- * rewritten by every call (0 = ok, 1 = an internal wait gave up); the rest holds
+ * rewritten by every call (0 = ok, 1 = an internal wait gave up, 3 = a paged
+ * cache named a page outside its pool for a key in use); the rest holds
  * the normalised partial outputs of key ranges split across CTAs (fp32, about
  * (148 + B*Hkv*ceil(n*Hq/Hkv/128)) * 128 * (D+1) * 4 bytes).  The call launches
  * two kernels; either may start while its predecessor on the stream drains
@@ -187,6 +188,32 @@ EAGLE_API eagle_status eagle_tree_attention(const void* q, const void* k_cache, 
                                   const void* v_tree, const uint64_t* mask, const int32_t* pos,
                                   int B, int n, int Hq, int Hkv, int D, int window, float scale,
                                   void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------- paged prefix cache
+ * eagle_tree_attention over a paged prefix cache, for batches whose prefixes
+ * differ in length: the cache is a pool of pages instead of one [Lmax] slab
+ * per sequence.
+ *   k_pages, v_pages [num_pages][Hkv][page_size][D] bf16 (16-byte aligned);
+ *   block_table [B][pages_per_seq] int32 device: sequence b's key at position
+ *     p sits at offset p % page_size of page block_table[b][p / page_size];
+ *     entries past a sequence's length are not read for it (any value).
+ *   page_size: 16, 32 or a multiple of 64; num_pages * Hkv * page_size < 2^31.
+ *   A sequence holds up to pages_per_seq * page_size keys (prefix_len is
+ *   clamped to that); pass that product as Lmax to
+ *   eagle_tree_attention_workspace_bytes.
+ * Everything else (q, tree K/V, mask, pos, window, scale, out, workspace) as
+ * in eagle_tree_attention, with the same result up to the order of
+ * floating-point sums (identical without a window).  A page id outside
+ * [0, num_pages) for a key below prefix_len reads zeros and sets device
+ * status 3 in the workspace header (see eagle_tree_attention).  Host errors:
+ * EAGLE_ERR_NULL, EAGLE_ERR_SHAPE (page_size), EAGLE_ERR_LIMIT, EAGLE_ERR_ALIGN,
+ * EAGLE_ERR_WORKSPACE. */
+EAGLE_API eagle_status eagle_tree_attention_paged(const void* q, const void* k_pages, const void* v_pages,
+                                                  int num_pages, int page_size, const int32_t* block_table,
+                                                  int pages_per_seq, const int32_t* prefix_len, const void* k_tree,
+                                                  const void* v_tree, const uint64_t* mask, const int32_t* pos,
+                                                  int B, int n, int Hq, int Hkv, int D, int window, float scale,
+                                                  void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ----------------------------------------------------------------- accept
  * Walk each tree from the root ("EAGLE" notes, EAGLE-2 "Well-Calibrated Draft
@@ -360,6 +387,17 @@ EAGLE_API eagle_status eagle_kv_compact(const void* k_tree, const void* v_tree, 
                                         const int32_t* accepted_len, const int32_t* prefix_len, void* k_cache,
                                         void* v_cache, int32_t* new_prefix_len, int B, int n, int Hkv, int D,
                                         int Lmax, int depth, void* stream);
+/* The same into a paged cache (layout as for eagle_tree_attention_paged):
+ * position p goes to offset p % page_size of page block_table[b][p /
+ * page_size]; a sequence holds up to pages_per_seq * page_size keys, and the
+ * copy also ends at a position whose page id lies outside [0, num_pages) (a
+ * page not allocated yet). */
+EAGLE_API eagle_status eagle_kv_compact_paged(const void* k_tree, const void* v_tree, const int32_t* path,
+                                              const int32_t* accepted_len, const int32_t* prefix_len, void* k_pages,
+                                              void* v_pages, int num_pages, int page_size,
+                                              const int32_t* block_table, int pages_per_seq,
+                                              int32_t* new_prefix_len, int B, int n, int Hkv, int D, int depth,
+                                              void* stream);
 
 /* ---------------------------------------------------------- one whole step
  * One verification step in its order: build (eagle_tree_build), mask and
@@ -384,8 +422,8 @@ EAGLE_API eagle_status eagle_kv_compact(const void* k_tree, const void* v_tree, 
  *   NULL), mask [B][n][2] uint64, pos [B][n] int32, attn_out [B][n][Hq][D]
  *   bf16, accepted_len [B], path [B][depth], bonus [B] int32.
  * Limits: those of the four calls.  Workspace: eagle_verify_step_workspace_bytes
- * (256-byte aligned).  The attention's device status word (0 = ok, 1 = an
- * internal wait gave up) is the int at byte offset
+ * (256-byte aligned).  The attention's device status word (as for
+ * eagle_tree_attention) is the int at byte offset
  * eagle_verify_step_attention_status_offset of the workspace after the step. */
 typedef struct {
   const void* draft_logits;
@@ -403,6 +441,10 @@ typedef struct {
   float scale;  /* <= 0 selects 1/sqrt(D) */
   const float* uniforms;
   int sampling_rule;  /* EAGLE_SAMPLE_WITH_REPLACEMENT or _WITHOUT_REPLACEMENT (sampled acceptance) */
+  /* paged prefix cache (block_table != NULL): k_cache / v_cache are the page
+   * pools and Lmax is unused, as in eagle_tree_attention_paged */
+  const int32_t* block_table;
+  int page_size, pages_per_seq, num_pages;
 } eagle_step_in_t;
 
 typedef struct {

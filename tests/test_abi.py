@@ -126,7 +126,8 @@ def test_binding_refuses_cpu_tensors():
 def _step_in(**kw):
     d = dict(draft_logits=FAKE, target_logits=FAKE, logits_dtype=0, B=1, V=32000, depth=6, k=10, m=60,
              q=FAKE, k_cache=FAKE, v_cache=FAKE, prefix_len=FAKE, Lmax=2048, k_tree=FAKE, v_tree=FAKE,
-             Hq=32, Hkv=32, D=128, window=0, scale=0.0, uniforms=None, sampling_rule=0)
+             Hq=32, Hkv=32, D=128, window=0, scale=0.0, uniforms=None, sampling_rule=0, block_table=None,
+             page_size=0, pages_per_seq=0, num_pages=0)
     d.update(kw)
     return _lib.StepIn(*[d[name] for name, _ in _lib.StepIn._fields_])
 
@@ -166,6 +167,11 @@ def test_step_validation(lib):
     assert call(si=_step_in(q=ctypes.c_void_p(0x1008))) == 6
     assert call(ws=None, wsb=0) == 5
     assert call(si=_step_in(sampling_rule=2)) == 2
+    assert call(si=_step_in(block_table=FAKE, page_size=48, pages_per_seq=40, num_pages=100)) == 2
+    assert call(si=_step_in(block_table=FAKE, page_size=64, pages_per_seq=40, num_pages=100), ws=None, wsb=0) == 5
+    paged = lib.eagle_verify_step_workspace_bytes(ctypes.byref(_step_in(block_table=FAKE, page_size=64,
+                                                                         pages_per_seq=32, num_pages=100, Lmax=0)))
+    assert paged == lib.eagle_verify_step_workspace_bytes(ctypes.byref(_step_in(Lmax=2048)))
     assert n.value == 0  # nothing was reported: every call above failed validation
 
 
@@ -225,3 +231,24 @@ def test_static_tree_validation(lib):
     assert build(par=arr([0, 0, 1, 1, 5])) == 2
     assert build(V=1) == 4                                                     # rank 1 needs two tokens
     assert build(nb=nb - 1) == 5
+
+
+def test_paged_validation(lib):
+    FAKE2 = ctypes.c_void_p(0x2000)
+    def att(**kw):
+        d = dict(num_pages=100, ps=64, bt=FAKE, pps=8, B=2, n=10, Hq=32, Hkv=8, D=128, window=0, ws=FAKE,
+                 nb=1 << 30)
+        d.update(kw)
+        return lib.eagle_tree_attention_paged(FAKE, FAKE, FAKE, d["num_pages"], d["ps"], d["bt"], d["pps"], FAKE, FAKE,
+                                              FAKE, FAKE, FAKE, d["B"], d["n"], d["Hq"], d["Hkv"], d["D"], d["window"],
+                                              0.0, FAKE, d["ws"], d["nb"], None)
+    assert att(bt=None) == 1
+    assert att(ps=48) == 2 and att(ps=8) == 2 and att(ps=0) == 2
+    assert att(ps=192, nb=16) == 5                # a multiple of 64 passes; the short workspace stops the call
+    assert att(num_pages=1 << 20, ps=4096) == 4   # pool rows past int range
+    assert att(D=96) == 4
+    assert att(ws=None, nb=0) == 5
+    comp = lambda **kw: lib.eagle_kv_compact_paged(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("np", 100),
+                                                   kw.get("ps", 16), kw.get("bt", FAKE), 8, kw.get("nl", FAKE2), 2,
+                                                   10, 8, 128, 6, None)
+    assert comp(bt=None) == 1 and comp(ps=24) == 2 and comp(nl=FAKE) == 2   # new lengths aliasing prefix_len
