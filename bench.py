@@ -44,7 +44,7 @@ LAUNCHES_PER_STEP = 6  # one eagle_verify_step: row sweep, expand (+ mask), atte
 # DRAM bytes (read + write) of one launch of the tree attention's main kernel,
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of this
 # kernel version on the named workload; a workload without a capture reports null.
-ATTN_TRAFFIC_BYTES = {"7b": 35099392 + 13824}
+ATTN_TRAFFIC_BYTES = {"7b": 35108352 + 0}
 
 
 def parse():
@@ -361,7 +361,7 @@ def main():
         "build": lambda st, inp: st.build(inp["draft_logits"]),
         "mask": lambda st, inp: st.mask_(inp["prefix_len"]),
         "attention": lambda st, inp: st.attention(inp["q"], inp["k_cache"], inp["v_cache"], inp["prefix_len"],
-                                                  inp["k_tree"], inp["v_tree"]),
+                                                  inp["k_tree"], inp["v_tree"], inp.get("block_table")),
         "accept": lambda st, inp: st.accept(inp["target_logits"], inp["uniforms"], inp["draft_logits"]),
     }
     stage_graphs = {name: [capture(lambda st=st, inp=inp, f=f: f(st, inp)) for st, inp in zip(steps, sets)]

@@ -14,6 +14,7 @@ from __future__ import annotations
 
 import ctypes
 import json
+import os
 from dataclasses import dataclass
 from typing import Callable, Optional, Sequence, Tuple
 
@@ -66,6 +67,17 @@ class CostTable:
         with open(path) as f:
             d = json.load(f)
         return cls(np.array(d["B"]), np.array(d["L"]), np.array(d["N"]), np.array(d["us"]), d.get("unit", "us"))
+
+
+# Measured on a B200 by calibrate.py (mask + tree attention + greedy acceptance as one CUDA graph, L2 flushed):
+# Hq 32, Hkv 8, D 128, V 128256 bf16; B in {1, 4, 16, 32}, L in {1024, 4096, 16384}, N up to 128.
+DEFAULT_TABLE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "data",
+                             "cost_b200_hq32_hkv8_d128_v128256_bf16.json")
+
+
+def default_table() -> CostTable:
+    """The cost table measured on a B200 for the 32/8-head, D 128, 128k-vocabulary shape."""
+    return CostTable.from_json(DEFAULT_TABLE)
 
 
 @dataclass

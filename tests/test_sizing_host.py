@@ -99,3 +99,14 @@ def test_harness_stops_at_the_first_level_that_does_not_pay():
     fg = _FakeGrower(gains)
     r = grow_sized(fg, None, lambda *a: None, table, 150, 0.5)
     assert (r.levels_kept, r.levels_drafted, r.tree) == (0, 1, None)
+
+
+def test_the_shipped_b200_table():
+    from eagle_tree_verification_dynamic_b200.sizing import default_table
+    t = default_table()
+    assert t.us.shape == (t.B.size, t.L.size, t.N.size) and np.all(np.isfinite(t.us))
+    for i, j, l in [(0, 0, 1), (3, 2, 6), (1, 1, 3)]:
+        assert t.at(t.B[i], t.L[j], t.N[l]) == pytest.approx(t.us[i, j, l], rel=1e-12)
+    assert np.all(t.us[:, :, 0] == 0.0) and np.all(t.us[:, :, 1:] > 0.0)
+    # verification grows with the batch's work: the largest grid point costs the most
+    assert t.us[-1, -1, -1] == t.us.max()
