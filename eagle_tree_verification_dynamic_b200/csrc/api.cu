@@ -75,7 +75,7 @@ const char* eagle_status_string(int status) {
 
 const char* eagle_last_cuda_error(void) { return g_cuda_err; }
 
-int eagle_version(void) { return 100; }
+int eagle_version(void) { return 200; }  // 0.2.0: eagle_step_in_t gained the sampling rule and paged-cache fields
 
 // ------------------------------------------------------------------ row stats
 size_t eagle_row_stats_workspace_bytes(long long rows, int V, int dtype, int k) {
