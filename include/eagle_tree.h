@@ -21,6 +21,13 @@
  *      resamples from the normalised max(0, p_target - p_draft) ("EAGLE" notes,
  *      EAGLE-2 "Well-Calibrated Draft Model"; "Что такое EAGLE-3", section 4
  *      steps 3-4).
+ * Around it: the whole step as one call (eagle_verify_step); the tree grown
+ * one level at a time for a draft model in the loop (eagle_tree_grow_*), with
+ * the EAGLE-4 harness's cost-aware sizing (eagle_cost_at,
+ * eagle_size_keep_level); EAGLE-1's static tree (eagle_static_tree_build);
+ * sampling without replacement (eagle_accept_with_rule); a paged prefix cache
+ * (eagle_tree_attention_paged); and the accepted path's keys and values into
+ * the cache (eagle_kv_compact, _paged).
  *
  * Conventions shared by every entry point
  *   - All array arguments are DEVICE pointers owned by the caller, unless a
@@ -34,7 +41,10 @@
  *   - Arguments are validated on the host before anything is launched; an
  *     invalid call returns a non-zero eagle_status and launches nothing.  A
  *     failed launch returns EAGLE_ERR_CUDA (the CUDA error string is available
- *     from eagle_last_cuda_error()).
+ *     from eagle_last_cuda_error()).  What the host cannot see (device data
+ *     such as a paged cache's page ids, or a wait inside a kernel that gave
+ *     up) is reported through a device status word in the workspace (see
+ *     eagle_tree_attention); no kernel traps.
  *   - Logits are fp32 (EAGLE_F32) or bf16 (EAGLE_BF16, raw 16-bit patterns).
  *     Rows must hold finite values; at least k values per row must be > -inf
  *     where a top-k is taken.  Attention tensors (q, K, V) are bf16.
