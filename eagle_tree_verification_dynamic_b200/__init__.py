@@ -41,6 +41,7 @@ from ._lib import (  # noqa: F401
     lib,
     pool_size,
     row_stats,
+    static_template_from_paths,
     static_tree_build,
     static_tree_rows,
     step_in,

@@ -490,6 +490,25 @@ def _template(parents, ranks):
     return p, r
 
 
+def static_template_from_paths(paths):
+    """A static tree written as rank paths -> (parents, ranks) in template order.
+
+    Each path lists sibling ranks from the root: (0,) is the root's likeliest child, (0, 1) that child's
+    second likeliest, and so on.  Every prefix of a path must itself be a path.  Nodes are numbered by
+    (depth, path), so a parent precedes its children and siblings follow their rank."""
+    keyed = sorted({tuple(int(r) for r in p) for p in paths}, key=lambda p: (len(p), p))
+    if not keyed or any(len(p) == 0 for p in keyed):
+        raise EagleError("static tree: empty path")
+    node_of = {p: i + 1 for i, p in enumerate(keyed)}
+    parents, ranks = [], []
+    for p in keyed:
+        if len(p) > 1 and p[:-1] not in node_of:
+            raise EagleError(f"static tree: path {p} has no parent path {p[:-1]}")
+        parents.append(0 if len(p) == 1 else node_of[p[:-1]])
+        ranks.append(p[-1])
+    return parents, ranks
+
+
 def static_tree_rows(parents, ranks) -> int:
     """Number of draft rows R the template needs (row 0 = root, then each node with a child)."""
     p, r = _template(parents, ranks)

@@ -88,3 +88,22 @@ def test_token_relabelling():
     b = oracle.build_static_tree(y, parents, ranks)
     assert b["tokens"].tolist() == perm[a["tokens"]].tolist()
     np.testing.assert_allclose(b["logV"], a["logV"], rtol=0, atol=1e-12)
+
+
+def test_rank_paths_to_template():
+    """The binding's rank-path helper (host code) gives the template whose
+    static tree, on rows from the oracle's dynamic depth-2 tree, is that tree."""
+    import eagle_tree_verification_dynamic_b200 as et
+    k = 3
+    paths = [(s, r) for s in range(k) for r in range(k)] + [(r,) for r in range(k)]
+    parents, ranks = et.static_template_from_paths(paths)
+    assert parents == [0] * k + [1 + s for s in range(k) for _ in range(k)]
+    assert ranks == list(range(k)) + [r for _ in range(k) for r in range(k)]
+    cfg = get_config("tiny", depth=2, k=k, m=k + k * k, V=60, B=1, logits_dtype="f32")
+    x = oracle.decode_logits(gen_draft_logits(cfg, 9), "f32")[0]
+    st = oracle.build_static_tree(x, parents, ranks)
+    dyn = oracle.build_tree(x, 2, k, k + k * k)
+    assert st["tokens"].tolist() == dyn["tokens"].tolist()
+    with pytest.raises(et.EagleError):
+        et.static_template_from_paths([(0,), (1, 0)])          # (1,) is missing
+    assert et.static_template_from_paths([(0, 0), (0,), (0, 0, 2)]) == ([0, 1, 2], [0, 0, 2])
