@@ -247,6 +247,9 @@ EAGLE_API eagle_status eagle_tree_attention_paged(const void* q, const void* k_p
  *     greedy.
  *   tokens, parents [B][n], draft_row [B][n+1]: the tree.
  *   accepted_len [B], path [B][depth] (accepted node ids, -1 padded), bonus [B].
+ * The uniforms are device data and are not checked: outside [0, 1) the walk
+ * still ends, but the bonus token of a sequence whose u_res is >= 1 or NaN is
+ * unspecified (it may be left unwritten).
  * Limits: n <= EAGLE_MAX_NODES, depth <= EAGLE_MAX_DEPTH; for sampling
  * V <= 262144 (bf16) or 131072 (fp32).
  * Workspace: eagle_accept_workspace_bytes. */

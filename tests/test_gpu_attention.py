@@ -69,6 +69,25 @@ def test_attention_ragged_batch_and_empty_prefix():
     _run(B, n, 8, 2, 128, 300, plen, 0, seed=3, parents_b=[t[0] for t in trees], depth_b=[t[1] for t in trees])
 
 
+def test_prefix_lengths_outside_the_cache_are_clamped():
+    """prefix_len is device data the host cannot check: the kernel clamps it to
+    [0, Lmax], so -7 behaves as 0 and Lmax + 50 as Lmax, bit for bit."""
+    rng = np.random.default_rng(5)
+    B, n, Lmax = 3, 12, 200
+    trees = [_random_tree(rng, n, 4) for _ in range(B)]
+    par, dep = np.stack([t[0] for t in trees]), np.stack([t[1] for t in trees])
+    cfg = get_config("tiny", B=B, m=n, Hq=8, Hkv=2, D=128, L=Lmax)
+    q, kc, vc, kt, vt = (to_dev_bf16(a) for a in gen_attention_inputs(cfg, 4, Lmax))
+
+    def run(plen):
+        pl = i32(np.array(plen, dtype=np.int32))
+        mask, pos = et.tree_mask(i32(par), i32(dep), pl)
+        return et.tree_attention(q, kc, vc, pl, kt, vt, mask, pos)
+    a, b = run([-7, Lmax + 50, Lmax]), run([0, Lmax, Lmax])
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_attention_chain_equals_causal():
     n, L = 16, 500
     par = np.arange(n)
