@@ -27,6 +27,24 @@ cudaError_t ensure_smem_limit(const void* kernel, size_t bytes) {
   if (e == cudaSuccess) done[key] = bytes;
   return e;
 }
+
+int device_sm_count() {
+  constexpr int kMaxDev = 64;
+  static int cached[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();  // clear the error a GPU-less host leaves behind
+    return 148;
+  }
+  if (cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  cached[dev] = n;  // a racing writer stores the same value
+  return n;
+}
 }  // namespace eagle
 
 namespace {

@@ -15,7 +15,8 @@ int attention_ctas(int B, int n, int Hq, int Hkv, int Lmax, int window) {
   const long long span = window > 0 ? (Lmax < window ? Lmax : window) : Lmax;
   const long long tiles_max = (span + kAttnKeysPerTile - 1) / kAttnKeysPerTile + (n + kAttnKeysPerTile - 1) / kAttnKeysPerTile;
   const long long T_max = (long long)B * Hkv * attention_row_groups(n, Hq, Hkv) * tiles_max;
-  return (int)(T_max < kNumSMs ? T_max : kNumSMs);
+  const int sms = device_sm_count();
+  return (int)(T_max < sms ? T_max : sms);
 }
 
 AttnWorkspace attention_ws_layout(int B, int n, int Hq, int Hkv, int D, int Lmax, int window) {

@@ -29,9 +29,12 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// log2(e) split into an fp32 head and an fp32 tail: x*log2(e) is formed as
-// fma(x, kLog2eHi, x*kLog2eLo) so that the constant's fp32 rounding does not
-// bias every exponent of a row by the same relative amount.
+// log2(e) as an unevaluated sum of two fp32 numbers (the head is log2(e)
+// rounded to fp32, the tail is the remainder rounded to fp32: the double-float
+// representation of a constant used in Dekker's and Cody-Waite's techniques),
+// good to about 48 bits.  x*log2(e) is formed as fma(x, kLog2eHi, x*kLog2eLo)
+// so that the head's fp32 rounding does not bias every exponent of a row by
+// the same relative amount.
 constexpr float kLog2eHi = 1.4426950216293335f;
 constexpr float kLog2eLo = 1.925963033500011e-08f;
 constexpr double kLn2 = 0.69314718055994530942;

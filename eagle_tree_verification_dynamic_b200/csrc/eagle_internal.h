@@ -10,7 +10,12 @@
 
 namespace eagle {
 
-constexpr int kNumSMs = 148;  // B200
+// Streaming multiprocessors of the current device (cudaDevAttrMultiProcessorCount,
+// read once per device); 148, a B200's count, when no device can be queried
+// (host-only sizing on a machine without a GPU).  Grids and workspaces that
+// scale with the SM count use it, so a workspace sized on one device is
+// checked against the same count when the call launches.
+int device_sm_count();
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

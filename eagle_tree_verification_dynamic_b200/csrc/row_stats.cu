@@ -262,7 +262,7 @@ row_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k, ChunkSt
 // ------------------------------------------------------------------- host
 ChunkPlan plan_chunks(long long rows, int V, int elem_bytes) {
   const int per_vec = 16 / elem_bytes;
-  const long long target = 4LL * kNumSMs;
+  const long long target = 4LL * device_sm_count();
   long long want = rows > 0 ? (target + rows - 1) / rows : 1;
   const long long max_chunks = V / 4096 > 1 ? V / 4096 : 1;
   if (want < 1) want = 1;

@@ -13,10 +13,17 @@
 // stand-in, not device memory), so on the first call on each device, with that
 // device current, its device address is looked up with cudaGetSymbolAddress
 // and cached.  That first call on a device should therefore be made before any
-// stream capture begins.  Calls share the one array: two calls whose work
-// overlaps on the GPU (different streams, or different host threads) race on
-// it and must be serialised by the caller.  The build kernels write every
-// scratch byte before reading it, so nothing needs clearing between calls.
+// stream capture begins.  The cached address lives as long as the process's
+// context on that device: after cudaDeviceReset (or anything else that tears
+// the primary context down) the library's module is loaded again elsewhere and
+// the cached address is stale, so a process that resets a device must be
+// restarted before it calls this entry point again.  Calls share the one
+// array: two calls whose work overlaps on the GPU (different streams, or
+// different host threads) race on it and must be serialised by the caller.
+// What must start at zero is cleared on the caller's stream at every call: the
+// per-row tickets of the vocabulary sweep are reset with cudaMemsetAsync
+// before its kernel runs; every other scratch byte is written before it is
+// read.
 #include <mutex>
 
 #include "eagle_internal.h"

@@ -486,7 +486,9 @@ EAGLE_API eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_
  * Shapes whose eagle_tree_build_workspace_bytes exceeds 2 MiB return
  * EAGLE_ERR_LIMIT and launch nothing.  The first call on a device looks up the
  * array's device address (cudaGetSymbolAddress) and must come before any
- * stream capture on that device.  All calls share the array: calls whose work
+ * stream capture on that device; the address is cached for the life of the
+ * process, so a process that resets the device (cudaDeviceReset) must restart
+ * before calling this again.  All calls share the array: calls whose work
  * overlaps on the GPU race and must be serialised by the caller. */
 EAGLE_API eagle_status eagle_tree_build_noalloc(const void* draft_logits, int dtype, int B, int R, int V,
                                                 int depth, int k, int m, const eagle_tree_t* out, int* n_nodes,

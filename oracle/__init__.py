@@ -45,7 +45,7 @@ from .tree import build_tree, build_trees  # noqa: F401
 from .static_tree import build_static_tree, template_rows  # noqa: F401
 from .mask import ancestor_mask, pack_mask, positions  # noqa: F401
 from .attention import tree_attention, tree_attention_rows  # noqa: F401
-from .accept import accept_greedy, accept_stochastic, inverse_cdf  # noqa: F401
+from .accept import accept_greedy, accept_stochastic, inverse_cdf, inverse_cdf_band  # noqa: F401
 from .kv import compact_kv  # noqa: F401
 from .paged import compact_kv_paged, gather_pages  # noqa: F401
 from .sizing import cost_at, keep_level, level_ratio, levels_kept  # noqa: F401

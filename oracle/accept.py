@@ -79,6 +79,20 @@ def inverse_cdf(weights: np.ndarray, u: float):
     return i, tie
 
 
+def inverse_cdf_band(weights: np.ndarray, u: float, rel: float = 1e-6) -> List[int]:
+    """Every index the inverse CDF returns for some threshold within rel * sum
+    of u * sum: the smallest i with cumsum_i > t, for t in that band.  These
+    are the results a draw near a cumulative-sum boundary may give once the
+    sums are rounded differently."""
+    c = np.cumsum(np.asarray(weights, dtype=np.float64))
+    Z = c[-1]
+    last = c.shape[0] - 1
+    lo = min(int(np.searchsorted(c, u * Z - rel * Z, side="right")), last)
+    hi = min(int(np.searchsorted(c, u * Z + rel * Z, side="right")), last)
+    w = np.diff(np.concatenate([[0.0], c]))
+    return [lo] + [i for i in range(lo + 1, hi + 1) if w[i] > 0.0]
+
+
 def accept_greedy(target: np.ndarray, tokens, parents, max_depth: int) -> Dict:
     target = np.asarray(target, dtype=np.float64)
     tokens = np.asarray(tokens)
@@ -106,7 +120,10 @@ def _without(q: np.ndarray, x: int):
 
 
 def accept_stochastic(target: np.ndarray, draft: np.ndarray, tokens, parents, draft_row,
-                      uniforms: np.ndarray, max_depth: int, without_replacement: bool = False) -> Dict:
+                      uniforms: np.ndarray, max_depth: int, without_replacement: bool = False,
+                      flip=()) -> Dict:
+    """`flip`: node ids whose accept test is decided the other way (for checking
+    a result downstream of a flagged near-tie); empty for the plain walk."""
     target = np.asarray(target, dtype=np.float64)
     draft = np.asarray(draft, dtype=np.float64)
     tokens = np.asarray(tokens)
@@ -127,7 +144,7 @@ def accept_stochastic(target: np.ndarray, draft: np.ndarray, tokens, parents, dr
                 u = float(u_acc[c])
                 if near_tie(u, ratio):
                     ties.append({"kind": "accept", "node": c, "u": u, "ratio": ratio})
-                if u < ratio:
+                if (u < ratio) != (c in flip):
                     path.append(c)
                     j = c
                     p = softmax(target[c])
@@ -154,7 +171,7 @@ def accept_stochastic(target: np.ndarray, draft: np.ndarray, tokens, parents, dr
     else:
         bonus, tie = inverse_cdf(p, float(u_res[j]))
         if tie:
-            ties.append({"kind": "bonus", "node": j})
+            ties.append({"kind": "bonus", "node": j, "alternatives": inverse_cdf_band(p, float(u_res[j]))})
     assert len(path) <= max_depth
     return {"accepted_len": len(path), "path": path + [-1] * (max_depth - len(path)),
             "bonus": int(bonus), "stop": j, "near_ties": ties}

@@ -43,9 +43,11 @@ def _softmax_rows(s: np.ndarray) -> np.ndarray:
 
 
 def tree_attention(q, k_cache, v_cache, L: int, k_tree, v_tree, parents, depth,
-                   window: int = 0, scale: Optional[float] = None) -> np.ndarray:
+                   window: int = 0, scale: Optional[float] = None, return_weights: bool = False):
     """One sequence.  q [n][Hq][D]; k_cache, v_cache [Hkv][>=L][D];
-    k_tree, v_tree [n][Hkv][D]; all fp64.  Returns out [n][Hq][D] fp64."""
+    k_tree, v_tree [n][Hkv][D]; all fp64.  Returns out [n][Hq][D] fp64, and with
+    return_weights also the softmax weights [n][Hq][L+n] over (prefix keys,
+    tree keys) that produced it."""
     q = np.asarray(q, dtype=np.float64)
     n, Hq, D = q.shape
     Hkv = k_cache.shape[0]
@@ -53,31 +55,38 @@ def tree_attention(q, k_cache, v_cache, L: int, k_tree, v_tree, parents, depth,
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     vis = _visible(L, parents, depth, window)
     out = np.empty((n, Hq, D), dtype=np.float64)
+    weights = np.empty((n, Hq, L + n), dtype=np.float64) if return_weights else None
     for h in range(Hq):
         g = h // G
         keys = np.concatenate([k_cache[g, :L], k_tree[:, g]], axis=0).astype(np.float64)
         vals = np.concatenate([v_cache[g, :L], v_tree[:, g]], axis=0).astype(np.float64)
         s = (q[:, h] @ keys.T) * scale
         s = np.where(vis, s, -np.inf)
-        out[:, h] = _softmax_rows(s) @ vals
-    return out
+        p = _softmax_rows(s)
+        out[:, h] = p @ vals
+        if return_weights:
+            weights[:, h] = p
+    return (out, weights) if return_weights else out
 
 
 def tree_attention_rows(q, k_cache, v_cache, L: int, k_tree, v_tree, parents, depth,
                         rows: Iterable[Tuple[int, int]], window: int = 0,
-                        scale: Optional[float] = None) -> np.ndarray:
-    """The same, for selected (node index i, head h) pairs only -> [len(rows)][D]."""
+                        scale: Optional[float] = None, return_weights: bool = False):
+    """The same, for selected (node index i, head h) pairs only -> [len(rows)][D]
+    (and with return_weights the weights [len(rows)][L+n])."""
     n, Hq, D = q.shape
     Hkv = k_cache.shape[0]
     G = Hq // Hkv
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     vis = _visible(L, parents, depth, window)
-    res = []
+    res, ws = [], []
     for i, h in rows:
         g = h // G
         keys = np.concatenate([k_cache[g, :L], k_tree[:, g]], axis=0).astype(np.float64)
         vals = np.concatenate([v_cache[g, :L], v_tree[:, g]], axis=0).astype(np.float64)
         s = (keys @ np.asarray(q[i, h], dtype=np.float64)) * scale
         s = np.where(vis[i], s, -np.inf)
-        res.append(_softmax_rows(s[None])[0] @ vals)
-    return np.array(res)
+        p = _softmax_rows(s[None])[0]
+        res.append(p @ vals)
+        ws.append(p)
+    return (np.array(res), np.array(ws)) if return_weights else np.array(res)

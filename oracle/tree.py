@@ -48,7 +48,11 @@ def _sort_key(c):
 
 
 def _flag_adjacent(sorted_cands, upto: int, kind: str, level: int, out: list):
-    """Record near-ties between neighbours of a selection (positions < upto+1)."""
+    """Record near-ties between neighbours of a selection (positions < upto+1).
+
+    Each record names the decision: (kind, level) and the two candidate ids in
+    the order this run ranked them, so that the same selection can be re-run
+    with the pair the other way round (see `_apply_flips`)."""
     for i in range(min(upto, len(sorted_cands) - 1)):
         a, b = sorted_cands[i], sorted_cands[i + 1]
         if a["parent"] == b["parent"]:
@@ -60,8 +64,30 @@ def _flag_adjacent(sorted_cands, upto: int, kind: str, level: int, out: list):
                         "logV": (a["logV"], b["logV"])})
 
 
-def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
-    """Build one sequence's tree from its R = 1 + (depth-1)*k draft rows (fp64)."""
+def _apply_flips(ranked, kind: str, level: int, flip) -> list:
+    """Resolve flagged near-ties the other way: for every record of `flip` that
+    names this selection (kind, level) and whose two candidates are neighbours
+    here in the recorded order, swap them.  A ranking within the near-tie band
+    is decided by rounding, so either order is a correct result; the tests use
+    this to tell a difference downstream of a flagged decision (allowed) from
+    any other difference (a failure)."""
+    for f in flip:
+        if f["kind"] != kind or f["level"] != level:
+            continue
+        a, b = f["gids"]
+        for i in range(len(ranked) - 1):
+            if ranked[i]["gid"] == a and ranked[i + 1]["gid"] == b:
+                if ranked[i + 1]["parent"] != a:  # a child never ranks above its parent
+                    ranked[i], ranked[i + 1] = ranked[i + 1], ranked[i]
+                break
+    return ranked
+
+
+def build_tree(logits: np.ndarray, depth: int, k: int, m: int, flip=()) -> Dict:
+    """Build one sequence's tree from its R = 1 + (depth-1)*k draft rows (fp64).
+
+    `flip`: near-tie records (as returned in "near_ties") to resolve the other
+    way; empty for the plain build."""
     logits = np.asarray(logits, dtype=np.float64)
     R, V = logits.shape
     assert depth >= 1 and 1 <= k <= V and m >= 1
@@ -87,7 +113,7 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
     frontiers: List[dict] = []    # per expanded level: the k tokens by slot and their parents' slots
     gains: List[float] = []       # per level: sum of V over its k best candidates
     for level in range(2, depth + 1):
-        ranked = sorted(level_cands, key=_sort_key)
+        ranked = _apply_flips(sorted(level_cands, key=_sort_key), "frontier", level - 1, flip)
         _flag_adjacent(ranked, k, "frontier", level - 1, near_ties)
         frontier = ranked[:k]
         gains.append(float(sum(np.exp(c["logV"]) for c in frontier)))
@@ -108,7 +134,7 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int) -> Dict:
     P = len(all_cands)
     assert P == k + (depth - 1) * k * k
     n = min(m, P)
-    ranked = sorted(all_cands, key=_sort_key)
+    ranked = _apply_flips(sorted(all_cands, key=_sort_key), "rerank", 0, flip)
     _flag_adjacent(ranked[n - 1:], 1, "rerank", 0, near_ties)
     kept = sorted(ranked[:n], key=lambda c: c["gid"])
     node_of = {c["gid"]: i + 1 for i, c in enumerate(kept)}

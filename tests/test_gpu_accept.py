@@ -2,9 +2,10 @@
 
 Both sides receive the oracle's tree and the same target logits, draft logits
 and uniforms.  accepted_len, path and bonus must be bit-exact; a sequence may
-differ only when the oracle flags a near-tie on its walk (u within 1e-6 of an
-acceptance ratio, or an inverse-CDF threshold within 1e-6 of a cumulative sum),
-which is reported.  The GPU also has to preserve the target distribution with
+differ only as the oracle's walk does when a decision it flags as a near-tie
+(u within 1e-6 of an acceptance ratio, or an inverse-CDF threshold within 1e-6
+of a cumulative sum) goes the other way (tests/parity.py); at most one such
+sequence is allowed per test.  The GPU also has to preserve the target distribution with
 drafts sampled from q (chi-square over 10^6 seeded trials).
 """
 import numpy as np
@@ -17,6 +18,7 @@ import oracle
 from workloads import gen_draft_logits, gen_uniforms, get_config, make_target_logits
 
 from gpu_helpers import dev, i32, to_dev_logits
+from parity import walk_match
 
 pytestmark = pytest.mark.gpu
 
@@ -54,14 +56,18 @@ def _run_accept(cfg, seed, mode, sigma=None, without_replacement=False):
         t = trees[b]
         if mode == "greedy":
             r = oracle.accept_greedy(T64[b], t["tokens"], t["parents"], cfg.depth)
+            rewalk = None
         else:
-            r = oracle.accept_stochastic(T64[b], x64[b], t["tokens"], t["parents"], t["draft_row"],
-                                         u[b].astype(np.float64), cfg.depth, without_replacement)
-        same = (int(acc[b]) == r["accepted_len"] and path[b].tolist() == r["path"] and int(bonus[b]) == r["bonus"])
-        if not same:
-            assert r["near_ties"], (f"{cfg.name} seed {seed} seq {b} {mode}: gpu ({acc[b]}, {path[b].tolist()}, "
-                                    f"{bonus[b]}) oracle ({r['accepted_len']}, {r['path']}, {r['bonus']})")
-            reported += 1
+            ub = u[b].astype(np.float64)
+            r = oracle.accept_stochastic(T64[b], x64[b], t["tokens"], t["parents"], t["draft_row"], ub, cfg.depth,
+                                         without_replacement)
+            rewalk = lambda nodes, b=b, t=t, ub=ub: oracle.accept_stochastic(
+                T64[b], x64[b], t["tokens"], t["parents"], t["draft_row"], ub, cfg.depth, without_replacement,
+                flip=nodes)
+        e = walk_match((acc[b], path[b].tolist(), bonus[b]), r, rewalk)
+        if e:
+            print(f"{cfg.name} seed {seed} seq {b} {mode}: matched with a flagged near-tie flipped")
+        reported += e
     return acc, reported
 
 
@@ -69,15 +75,15 @@ def _run_accept(cfg, seed, mode, sigma=None, without_replacement=False):
                                        ("l3-8b", "stochastic"), ("long", "greedy"), ("serve", "stochastic")])
 def test_accept_configs(name, mode):
     cfg = get_config(name)
-    for seed in cfg.seeds[:3]:
-        _run_accept(cfg, seed, mode)
+    assert sum(_run_accept(cfg, seed, mode)[1] for seed in cfg.seeds[:3]) <= 1
 
 
 @pytest.mark.parametrize("mode", ["greedy", "stochastic"])
 def test_accept_7b_all_seeds(mode):
     cfg = get_config("7b")
-    lens = [int(_run_accept(cfg, s, mode)[0][0]) for s in cfg.seeds]
-    print(f"7b {mode} accepted lengths over seeds: {lens}")
+    runs = [_run_accept(cfg, s, mode) for s in cfg.seeds]
+    assert sum(r[1] for r in runs) <= 1
+    print(f"7b {mode} accepted lengths over seeds: {[int(r[0][0]) for r in runs]}")
 
 
 @pytest.mark.parametrize("name", ["tiny", "7b"])
@@ -85,28 +91,28 @@ def test_accept_target_equals_draft(name):
     """sigma = 0: every first child is accepted down to a leaf (closed form)."""
     cfg = get_config(name)
     for mode in ("greedy", "stochastic"):
-        acc, _ = _run_accept(cfg, 2, mode, sigma=0.0)
-        assert int(acc[0]) >= 1
+        acc, excused = _run_accept(cfg, 2, mode, sigma=0.0)
+        assert int(acc[0]) >= 1 and excused <= 1
 
 
 def test_accept_batch_of_ragged_configs():
     cfg = get_config("serve", B=12, V=5003, logits_dtype="f32")
-    _run_accept(cfg, 4, "stochastic")
-    _run_accept(cfg, 4, "greedy")
+    assert _run_accept(cfg, 4, "stochastic")[1] + _run_accept(cfg, 4, "greedy")[1] <= 1
 
 
 @pytest.mark.parametrize("name", ["tiny", "7b", "l3-8b", "serve"])
 def test_accept_without_replacement_configs(name):
     cfg = get_config(name)
-    for seed in cfg.seeds[:3]:
-        _run_accept(cfg, seed, "stochastic", without_replacement=True)
+    assert sum(_run_accept(cfg, seed, "stochastic", without_replacement=True)[1] for seed in cfg.seeds[:3]) <= 1
 
 
 def test_accept_without_replacement_ragged_and_more_seeds():
-    _run_accept(get_config("serve", B=12, V=5003, logits_dtype="f32"), 4, "stochastic", without_replacement=True)
+    assert _run_accept(get_config("serve", B=12, V=5003, logits_dtype="f32"), 4, "stochastic",
+                       without_replacement=True)[1] <= 1
     cfg = get_config("7b")
-    lens = [int(_run_accept(cfg, s, "stochastic", without_replacement=True)[0][0]) for s in cfg.seeds]
-    print(f"7b sampled without replacement, accepted lengths over seeds: {lens}")
+    runs = [_run_accept(cfg, s, "stochastic", without_replacement=True) for s in cfg.seeds]
+    assert sum(r[1] for r in runs) <= 1
+    print(f"7b sampled without replacement, accepted lengths over seeds: {[int(r[0][0]) for r in runs]}")
 
 
 def _chi2_gpu_distinct(trials: int, seed: int, without_replacement: bool) -> float:

@@ -14,7 +14,7 @@ import eagle_tree_verification_dynamic_b200 as et
 import oracle
 from workloads import gen_attention_inputs, gen_draft_logits, gen_prefix_len, get_config
 
-from gpu_helpers import check_attention, dec, i32, to_dev_bf16, to_dev_logits, tree_of
+from gpu_helpers import attention_ref, check_attention, dec, i32, to_dev_bf16, to_dev_logits, tree_of
 
 pytestmark = pytest.mark.gpu
 
@@ -39,9 +39,9 @@ def _run(B, n, Hq, Hkv, D, Lmax, plen, window, seed, parents_b, depth_b):
                             to_dev_bf16(vt), mask, pos, window=window)
     out = out.float().cpu().numpy()
     for b in range(B):
-        ref = oracle.tree_attention(dec(q[b]), dec(kc[b]), dec(vc[b]), int(plen[b]), dec(kt[b]), dec(vt[b]),
-                                    par[b], dep[b], window=window)
-        check_attention(out[b], ref)
+        ref, s = attention_ref(dec(q[b]), dec(kc[b]), dec(vc[b]), int(plen[b]), dec(kt[b]), dec(vt[b]),
+                               par[b], dep[b], window=window)
+        check_attention(out[b], ref, s)
 
 
 @pytest.mark.parametrize("B,n,Hq,Hkv,D,Lmax,window", [
@@ -111,7 +111,7 @@ def test_attention_full_size_sampled(name):
         t = tree_of(tree, b)
         rows = [(int(i), int(h)) for i, h in zip(rng.integers(0, cfg.m, 12), rng.integers(0, cfg.Hq, 12))]
         rows += [(cfg.m - 1, cfg.Hq - 1), (0, 0)]
-        ref = oracle.tree_attention_rows(dec(q[b]), dec(kc[b]), dec(vc[b]), int(plen[b]), dec(kt[b]),
-                                         dec(vt[b]), t["parents"], t["depth"], rows, window=cfg.window)
+        ref, s = attention_ref(dec(q[b]), dec(kc[b]), dec(vc[b]), int(plen[b]), dec(kt[b]), dec(vt[b]),
+                               t["parents"], t["depth"], window=cfg.window, rows=rows)
         got = np.array([out[b, i, h] for i, h in rows])
-        check_attention(got, ref)
+        check_attention(got, ref, s)

@@ -21,7 +21,7 @@ from workloads import gen_attention_inputs, gen_draft_logits, gen_prefix_len, ge
 
 from workloads.gen import bf16_bits_from_f32
 
-from gpu_helpers import check_attention, dec, i32, to_dev_bf16, to_dev_logits
+from gpu_helpers import attention_ref, check_attention, dec, i32, to_dev_bf16, to_dev_logits
 
 pytestmark = pytest.mark.gpu
 
@@ -82,9 +82,9 @@ def test_paged_window_against_the_oracle(ps):
         par, dep = tree.parents[b].cpu().numpy(), tree.depth[b].cpu().numpy()
         rows = [(int(i), int(h)) for i, h in zip(rng.integers(0, tree.n, 10), rng.integers(0, cfg.Hq, 10))]
         rows += [(0, 0), (tree.n - 1, cfg.Hq - 1)]
-        ref = oracle.tree_attention_rows(dec(qh[b]), dec(kch[b]), dec(vch[b]), int(plen[b]), dec(kth[b]), dec(vth[b]),
-                                         par, dep, rows, window=cfg.window)
-        check_attention(np.array([out[b, i, h] for i, h in rows]), ref)
+        ref, s = attention_ref(dec(qh[b]), dec(kch[b]), dec(vch[b]), int(plen[b]), dec(kth[b]), dec(vth[b]),
+                               par, dep, window=cfg.window, rows=rows)
+        check_attention(np.array([out[b, i, h] for i, h in rows]), ref, s)
 
 
 def test_missing_page_reports_status_3():

@@ -14,7 +14,8 @@ import oracle
 from eagle_tree_verification_dynamic_b200.sizing import CostTable, grow_sized
 from workloads import gen_draft_logits, get_config
 
-from gpu_helpers import to_dev_logits, tree_of, trees_equal
+from gpu_helpers import to_dev_logits, tree_of
+from parity import tree_match
 
 pytestmark = pytest.mark.gpu
 
@@ -68,9 +69,11 @@ def test_sized_growth_matches_the_oracle(name, threshold):
         return
     m = min(k * kept, 128)
     R = 1 + (drafted - 1) * k
+    excused = 0
     for b in range(cfg.B):
         ref = oracle.build_tree(x64[b][:R], drafted, k, m)
         got = tree_of(r.tree, b)
         got["row_lse"] = got["row_lse"][:R]
-        assert trees_equal(got, ref) or ref["near_ties"], (name, threshold, b)
+        excused += tree_match(got, ref, lambda fl, b=b: oracle.build_tree(x64[b][:R], drafted, k, m, flip=fl))[0]
         np.testing.assert_allclose(got["row_lse"], ref["row_lse"], rtol=0, atol=5e-7)
+    assert excused <= 1, (name, threshold)

@@ -16,7 +16,8 @@ import oracle
 from eagle_tree_verification_dynamic_b200.step import StepShape, VerifyStep
 from workloads import get_config, make_target_logits, make_workload
 
-from gpu_helpers import check_attention, dec
+from parity import walk_match
+from gpu_helpers import attention_ref, check_attention, dec
 
 pytestmark = pytest.mark.gpu
 
@@ -81,13 +82,11 @@ def test_step_matches_the_oracle_on_the_tiny_workload():
     np.testing.assert_array_equal(one.mask[0].cpu().numpy().view(np.uint64),
                                   oracle.pack_mask(oracle.ancestor_mask(ref["parents"])))
     np.testing.assert_array_equal(one.pos[0].cpu().numpy(), oracle.positions(ref["depth"], int(w.prefix_len[0])))
-    ref_out = oracle.tree_attention(dec(w.q[0]), dec(w.k_cache[0]), dec(w.v_cache[0]), int(w.prefix_len[0]),
-                                    dec(w.k_tree[0]), dec(w.v_tree[0]), ref["parents"], ref["depth"])
-    check_attention(one.out[0].float().cpu().numpy(), ref_out)
+    ref_out, s = attention_ref(dec(w.q[0]), dec(w.k_cache[0]), dec(w.v_cache[0]), int(w.prefix_len[0]),
+                               dec(w.k_tree[0]), dec(w.v_tree[0]), ref["parents"], ref["depth"])
+    check_attention(one.out[0].float().cpu().numpy(), ref_out, s)
     tgt = oracle.decode_logits(make_target_logits(cfg, 0, w.draft_logits, ref["draft_row"][None]),
                                cfg.logits_dtype)[0]
-    s = oracle.accept_stochastic(tgt, x, ref["tokens"], ref["parents"], ref["draft_row"],
-                                 w.uniforms[0].astype(np.float64), cfg.depth)
-    if not s["near_ties"]:
-        assert int(one.accepted_len[0]) == s["accepted_len"]
-        assert int(one.bonus[0]) == s["bonus"]
+    walk = lambda nodes=(): oracle.accept_stochastic(tgt, x, ref["tokens"], ref["parents"], ref["draft_row"],
+                                                     w.uniforms[0].astype(np.float64), cfg.depth, flip=set(nodes))
+    walk_match((one.accepted_len[0], one.path[0].cpu().numpy().tolist(), one.bonus[0]), walk(), walk)

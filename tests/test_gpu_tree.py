@@ -2,9 +2,9 @@
 tree mask, against the oracle on the same seeded inputs.
 
 Tokens, parents, depth, draft rows, candidate ids and mask bits must be
-bit-exact.  A tree may differ only downstream of a decision the oracle flags as
-a near-tie (two log V within 1e-6 relative); such a case is reported, not
-failed.  Float outputs: log-sum-exp within 5e-7 absolute (fp32 exponentials,
+bit-exact.  A tree may differ only as the oracle's tree does when a decision it
+flags as a near-tie (two log V within 1e-6 relative) is resolved the other way
+(tests/parity.py); at most one such case is allowed per test.  Float outputs: log-sum-exp within 5e-7 absolute (fp32 exponentials,
 fp64 sums), log V within 2e-6 absolute (stored as fp32).
 """
 import numpy as np
@@ -17,6 +17,7 @@ from workloads import CONFIGS, gen_draft_logits, get_config, gen_prefix_len
 from workloads.gen import bf16_bits_from_f32
 
 from gpu_helpers import dev, i32, to_dev_logits, tree_of, trees_equal
+from parity import tree_match
 
 pytestmark = pytest.mark.gpu
 
@@ -61,18 +62,20 @@ def test_row_stats_unaligned_rows_and_neg_inf():
 
 
 def _check_trees(cfg, seed, gpu_tree, stored):
+    """Number of sequences whose tree matched only with a flagged near-tie flipped (at most 1)."""
     x64 = oracle.decode_logits(stored, cfg.logits_dtype)
-    reported = []
+    excused = 0
     for b in range(cfg.B):
         ref = oracle.build_tree(x64[b], cfg.depth, cfg.k, cfg.m)
         got = tree_of(gpu_tree, b)
         np.testing.assert_allclose(got["row_lse"], ref["row_lse"], rtol=0, atol=5e-7)
-        if not trees_equal(got, ref):
-            assert ref["near_ties"], f"{cfg.name} seed {seed} seq {b}: tree differs with no near-tie"
-            reported.append((b, ref["near_ties"]))
-            continue
-        np.testing.assert_allclose(got["logV"], ref["logV"], rtol=0, atol=2e-6)
-    return reported
+        e, matched = tree_match(got, ref, lambda fl, b=b: oracle.build_tree(x64[b], cfg.depth, cfg.k, cfg.m, flip=fl))
+        if e:
+            print(f"{cfg.name} seed {seed} seq {b}: matched with a flagged near-tie flipped")
+        excused += e
+        np.testing.assert_allclose(got["logV"], matched["logV"], rtol=0, atol=2e-6)
+    assert excused <= 1, f"{excused} sequences needed a flipped near-tie"
+    return excused
 
 
 @pytest.mark.parametrize("name", ["tiny", "7b", "l3-8b", "long", "serve"])
@@ -81,9 +84,7 @@ def test_tree_build_configs_seed0(name):
     stored = gen_draft_logits(cfg, 0)
     tree = et.tree_build(to_dev_logits(stored, cfg.logits_dtype), cfg.depth, cfg.k, cfg.m)
     torch.cuda.synchronize()
-    rep = _check_trees(cfg, 0, tree, stored)
-    if rep:
-        print(f"near-tie mismatches reported: {rep}")
+    _check_trees(cfg, 0, tree, stored)
 
 
 @pytest.mark.parametrize("name", ["7b", "l3-8b"])
