@@ -32,7 +32,9 @@ from ._lib import (  # noqa: F401
     accept_into,
     accept_workspace_bytes,
     alloc_tree,
+    attention_wait_probe,
     attention_workspace_bytes,
+    check_attention_status,
     exported_names,
     kv_compact,
     kv_compact_into,

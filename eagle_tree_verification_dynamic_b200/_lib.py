@@ -67,6 +67,7 @@ _SIGS = {
     "eagle_tree_attention_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i]),
     "eagle_tree_attention": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i,
                                     _c_i, _c_i, _c_i, _c_i, _c_f, _c_p, _c_p, _c_sz, _c_p]),
+    "eagle_debug_attention_wait_probe": (None, [ctypes.c_ulonglong]),
     "eagle_tree_build_noalloc": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                         ctypes.POINTER(TreeStruct), ctypes.POINTER(_c_i), _c_p]),
     "eagle_verify_step_workspace_bytes": (_c_sz, [ctypes.POINTER(StepIn)]),
@@ -161,6 +162,19 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 
 
 # ---------------------------------------------------------------- row stats
+def row_stats_workspace_bytes(rows: int, V: int, dtype_code: int, k: int) -> int:
+    return lib().eagle_row_stats_workspace_bytes(rows, V, dtype_code, k)
+
+
+def row_stats_into(logits: torch.Tensor, k: int, tok: torch.Tensor, val: torch.Tensor, lse, ws: torch.Tensor):
+    """The vocabulary sweep into preallocated outputs (tok [rows][k] int32, val [rows][k] f32, lse [rows] f64
+    or None) and workspace."""
+    rows, V = logits.reshape(-1, logits.shape[-1]).shape
+    dt = _dtype_code(logits)
+    _check(lib().eagle_row_stats(_ptr(logits), dt, rows, V, k, _ptr(tok), _ptr(val), _ptr(lse), _ptr(ws),
+                                 ws.numel(), _stream(logits.device)), "eagle_row_stats")
+
+
 def row_stats(logits: torch.Tensor, k: int, want_lse: bool = True):
     """logits [rows][V] -> (topk_token [rows][k] int32, topk_logit [rows][k] f32, lse [rows] f64)."""
     _need_cuda(logits)
@@ -282,6 +296,12 @@ def tree_attention(q, k_cache, v_cache, prefix_len, k_tree, v_tree, mask, pos=No
     if check:
         check_attention_status(ws)
     return out
+
+
+def attention_wait_probe(limit_ns: int):
+    """Diagnostics: make every following attention launch take its abort path
+    after a bounded wait of limit_ns that nothing completes (0 turns it off)."""
+    lib().eagle_debug_attention_wait_probe(int(limit_ns))
 
 
 def check_attention_status(ws: torch.Tensor):

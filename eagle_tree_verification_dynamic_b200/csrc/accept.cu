@@ -273,7 +273,10 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     if (STOCH) {
       sm.lse_t[i] = row_lse[trow0 + i];
       sm.u_acc[i] = uniforms[(size_t)b * 2 * (n + 1) + i];
-      sm.u_res[i] = uniforms[(size_t)b * 2 * (n + 1) + (n + 1) + i];
+      // the residual draw needs u in [0, 1): a NaN or negative u reads as 0 and
+      // u >= 1 as the largest float below 1, so the bonus is always written
+      const float ur = uniforms[(size_t)b * 2 * (n + 1) + (n + 1) + i];
+      sm.u_res[i] = ur >= 0.f ? fminf(ur, 0x1.fffffep-1f) : 0.f;
     }
   }
   __syncthreads();

@@ -2,9 +2,17 @@
 // notes, "3.Verify"): how many CTAs share the tile list, and the workspace that
 // holds the partials of units cut by CTA range boundaries.  The kernels are in
 // attention_tc.cu.
+#include <atomic>
+
 #include "eagle_internal.h"
 
 namespace eagle {
+
+namespace {
+std::atomic<unsigned long long> g_probe_ns{0};
+}  // namespace
+
+unsigned long long attention_wait_probe_ns() { return g_probe_ns.load(std::memory_order_relaxed); }
 
 int attention_row_groups(int n, int Hq, int Hkv) {
   const int rows = n * (Hq / Hkv);
@@ -33,3 +41,7 @@ AttnWorkspace attention_ws_layout(int B, int n, int Hq, int Hkv, int D, int Lmax
 }
 
 }  // namespace eagle
+
+extern "C" EAGLE_API void eagle_debug_attention_wait_probe(unsigned long long limit_ns) {
+  eagle::g_probe_ns.store(limit_ns, std::memory_order_relaxed);
+}

@@ -97,6 +97,7 @@ struct TcBars {
   uint64_t pv_done[2];
   uint64_t mma_idle;
   uint64_t pair[4];  // per lane quarter: both softmax warps wrote their (max, sum)
+  uint64_t never;    // nothing arrives here: the wait probe's barrier
   uint32_t tmem_base;
   int abort;
   int bad_page;  // a key inside the sequence sat on a page id outside the pool
@@ -242,6 +243,9 @@ struct TcParams {
   // block_table [B][pages_per_seq] page ids
   const int32_t* block_table;
   int page_size, pages_per_seq, num_pages;
+  // > 0: every softmax warp first waits this long (ns) on a barrier nothing
+  // completes, so the CTA takes its abort path (eagle_debug_attention_wait_probe)
+  unsigned long long probe_ns;
 };
 
 // Loads issued now and consumed later: the K/V stream keeps HBM saturated, so
@@ -415,6 +419,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
     mbar_init(smem_u32(&bars->mma_idle), 1);
     for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars->pair[i]), 64);
+    mbar_init(smem_u32(&bars->never), 1);
     bars->abort = 0;
     bars->bad_page = 0;
     fence_mbar_init();
@@ -665,6 +670,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     bool have = s_have;
     int jg = 0, n_epi = 0;
     bool ok = true;
+    // the wait probe: a bounded wait that runs out, then the same abort path as
+    // any wait that gives up (the other roles see the flag and drain)
+    if (p.probe_ns != 0ull && !__all_sync(kFull, mbar_wait(smem_u32(&bars->never), 0, abort, p.probe_ns))) ok = false;
     while (ok && have) {
       Piece pn;
       RowCtx rn;
@@ -1056,6 +1064,7 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
   p.num_pages = paged ? pg->num_pages : 0;
   p.q_by_tma = q_tma ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.probe_ns = attention_wait_probe_ns();
   const size_t smem = TcLayout<D>::kSmemBytes;
   cudaError_t e = ensure_smem_limit((const void*)attn_tc_kernel<D>, smem);
   if (e != cudaSuccess) return e;

@@ -105,6 +105,9 @@ struct AttnWorkspace {
   size_t bytes;
 };
 int attention_row_groups(int n, int Hq, int Hkv);
+// The wait probe's limit for the next attention launches (0: off); see
+// eagle_debug_attention_wait_probe.
+unsigned long long attention_wait_probe_ns();
 int attention_ctas(int B, int n, int Hq, int Hkv, int Lmax, int window);  // C
 AttnWorkspace attention_ws_layout(int B, int n, int Hq, int Hkv, int D, int Lmax, int window);
 inline size_t attention_ws_bytes(int B, int n, int Hq, int Hkv, int D, int Lmax, int window) {

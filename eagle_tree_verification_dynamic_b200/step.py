@@ -65,6 +65,25 @@ class VerifyStep:
         shape_only = L.StepIn(None, None, dcode, s.B, s.V, s.depth, s.k, s.m, None, None, None, None, s.Lmax, None,
                               None, s.Hq, s.Hkv, s.D, s.window, 0.0, None, 0)
         self.ws_step = L._workspace(L.step_workspace_bytes(shape_only), dev)
+        # the two vocabulary sweeps on their own (for timing them apart from the
+        # expansion and the walk): draft rows top-k + lse, target rows argmax + lse
+        rows_d, rows_t = s.B * s.R, s.B * (n + 1)
+        self.sw_tok = torch.empty(rows_d, s.k, dtype=torch.int32, device=dev)
+        self.sw_val = torch.empty(rows_d, s.k, dtype=torch.float32, device=dev)
+        self.sw_lse = torch.empty(rows_d, dtype=torch.float64, device=dev)
+        self.sw_amax = torch.empty(rows_t, 1, dtype=torch.int32, device=dev)
+        self.sw_max = torch.empty(rows_t, 1, dtype=torch.float32, device=dev)
+        self.sw_lse_t = torch.empty(rows_t, dtype=torch.float64, device=dev)
+        self.ws_sweep_d = L._workspace(L.row_stats_workspace_bytes(rows_d, s.V, dcode, s.k), dev)
+        self.ws_sweep_t = L._workspace(L.row_stats_workspace_bytes(rows_t, s.V, dcode, 1), dev)
+
+    def draft_sweep(self, draft_logits: torch.Tensor):
+        """The build's vocabulary sweep alone: top-k and log-sum-exp of every draft row."""
+        L.row_stats_into(draft_logits, self.s.k, self.sw_tok, self.sw_val, self.sw_lse, self.ws_sweep_d)
+
+    def accept_sweep(self, target_logits: torch.Tensor):
+        """The acceptance's target sweep alone: argmax and log-sum-exp of every target row."""
+        L.row_stats_into(target_logits, 1, self.sw_amax, self.sw_max, self.sw_lse_t, self.ws_sweep_t)
 
     def build(self, draft_logits: torch.Tensor):
         L.tree_build_into(draft_logits, self.s.depth, self.s.k, self.s.m, self.tree, self.ws_build)

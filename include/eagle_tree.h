@@ -247,9 +247,10 @@ EAGLE_API eagle_status eagle_tree_attention_paged(const void* q, const void* k_p
  *     greedy.
  *   tokens, parents [B][n], draft_row [B][n+1]: the tree.
  *   accepted_len [B], path [B][depth] (accepted node ids, -1 padded), bonus [B].
- * The uniforms are device data and are not checked: outside [0, 1) the walk
- * still ends, but the bonus token of a sequence whose u_res is >= 1 or NaN is
- * unspecified (it may be left unwritten).
+ * The uniforms are device data and are not checked on the host.  The walk
+ * reads a u_res that is NaN or negative as 0 and one >= 1 as the largest float
+ * below 1 (1 - 2^-24), so every sequence gets a bonus token; a u_acc outside
+ * [0, 1) is used as given (NaN rejects).
  * Limits: n <= EAGLE_MAX_NODES, depth <= EAGLE_MAX_DEPTH; for sampling
  * V <= 262144 (bf16) or 131072 (fp32).
  * Workspace: eagle_accept_workspace_bytes. */
@@ -475,6 +476,19 @@ EAGLE_API size_t eagle_verify_step_workspace_bytes(const eagle_step_in_t* in);
 EAGLE_API size_t eagle_verify_step_attention_status_offset(const eagle_step_in_t* in);
 EAGLE_API eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t* out, int* n_nodes,
                                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------ diagnostics
+ * Not a step of the method: a probe of the attention kernel's failure path.
+ * With limit_ns > 0, every attention launch that follows (eagle_tree_attention,
+ * _paged and the attention of eagle_verify_step) makes each softmax warp first
+ * wait limit_ns on a barrier that nothing completes.  The wait gives up, and
+ * the CTA takes the same path as any bounded wait that runs out: it sets its
+ * abort flag, the other roles stop, every TMA copy and MMA in flight is drained,
+ * TMEM is freed, and the workspace's status word reads 1 (the output is then
+ * undefined).  limit_ns = 0 turns the probe off.  Process-wide; calls that race
+ * with launches on other threads see either setting.  For tests of error
+ * handling: nothing faults, traps or hangs. */
+EAGLE_API void eagle_debug_attention_wait_probe(unsigned long long limit_ns);
 
 /* ----------------------------------------------------- tree build, no workspace
  * Not a step of the method (the pages have no counterpart): the same build as

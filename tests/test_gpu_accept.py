@@ -182,3 +182,32 @@ def _chi2_gpu(shape: str, trials: int, seed: int) -> float:
 @pytest.mark.parametrize("shape", ["star", "chain"])
 def test_gpu_sampling_preserves_target_distribution(shape):
     assert _chi2_gpu(shape, 1_000_000, 40 if shape == "star" else 41) > 1e-3
+
+
+def test_residual_uniform_outside_the_unit_interval_is_clamped():
+    """u_res = 1.0 draws as 1 - 2^-24 and NaN (or a negative u) as 0, bit for bit,
+    so the bonus token is always a token of the vocabulary."""
+    cfg = get_config("7b", B=4)
+    stored = gen_draft_logits(cfg, 6)
+    x64, trees = _oracle_trees(cfg, stored)
+    draft_row = np.stack([t["draft_row"] for t in trees])
+    tgt = make_target_logits(cfg, 6, stored, draft_row)
+    args = (to_dev_logits(tgt, cfg.logits_dtype), i32(np.stack([t["tokens"] for t in trees])),
+            i32(np.stack([t["parents"] for t in trees])), i32(draft_row), cfg.depth)
+    D = to_dev_logits(stored, cfg.logits_dtype)
+    _, _, lse = et.row_stats(D.reshape(-1, cfg.V), 1)
+    lse = lse.reshape(cfg.B, cfg.R)
+    u = gen_uniforms(cfg, 6)
+
+    def run(ures):
+        uu = u.copy()
+        uu[:, 1, :] = ures  # every node's residual uniform, wherever the walk stops
+        acc, path, bonus = et.accept(*args, torch.from_numpy(uu).to(dev()), D, lse)
+        return acc.cpu().numpy(), bonus.cpu().numpy()
+
+    for bad, same in ((np.float32(1.0), np.float32(1.0 - 2.0 ** -24)), (np.float32(7.5), np.float32(1.0 - 2.0 ** -24)),
+                      (np.float32(np.nan), np.float32(0.0)), (np.float32(-0.25), np.float32(0.0))):
+        acc_b, bonus_b = run(bad)
+        acc_s, bonus_s = run(same)
+        assert (acc_b == acc_s).all() and (bonus_b == bonus_s).all(), (bad, bonus_b, bonus_s)
+        assert ((bonus_b >= 0) & (bonus_b < cfg.V)).all()

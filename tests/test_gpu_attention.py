@@ -52,6 +52,9 @@ def _run(B, n, Hq, Hkv, D, Lmax, plen, window, seed, parents_b, depth_b):
     (1, 100, 2, 2, 128, 96, 0),     # n > 64 uses the second mask word
     (1, 20, 8, 4, 128, 2000, 300),  # sliding window
     (2, 9, 4, 4, 64, 50, 8),        # window shorter than the tree depth
+    (1, 37, 12, 2, 128, 700, 0),    # G = 6 does not divide 128: the producer warp gathers Q; 2 row groups
+    (2, 60, 40, 8, 128, 500, 0),    # G = 5, three row groups per KV head, the last one ragged
+    (1, 21, 6, 2, 64, 300, 40),     # G = 3 at D = 64, with a window
 ])
 def test_attention_small(B, n, Hq, Hkv, D, Lmax, window):
     rng = np.random.default_rng(n * 7 + Lmax)
@@ -115,3 +118,29 @@ def test_attention_full_size_sampled(name):
                                t["parents"], t["depth"], window=cfg.window, rows=rows)
         got = np.array([out[b, i, h] for i, h in rows])
         check_attention(got, ref, s)
+
+
+def test_a_wait_that_runs_out_reports_status_1_and_the_next_call_is_clean():
+    """The failure path of the bounded waits: with the wait probe on, every CTA's
+    softmax warps wait 1 ms on a barrier nothing completes, give up, and the CTA
+    aborts (the other roles stop, copies and MMAs in flight drain, TMEM is
+    freed); the status word reads 1.  With the probe off again the same call
+    returns status 0 and the same output as before, bit for bit."""
+    rng = np.random.default_rng(31)
+    B, n, Hq, Hkv, D, Lmax = 2, 30, 8, 2, 128, 1500
+    trees = [_random_tree(rng, n, 5) for _ in range(B)]
+    par, dep = np.stack([t[0] for t in trees]), np.stack([t[1] for t in trees])
+    cfg = get_config("tiny", B=B, m=n, Hq=Hq, Hkv=Hkv, D=D, L=Lmax)
+    q, kc, vc, kt, vt = (to_dev_bf16(a) for a in gen_attention_inputs(cfg, 12, Lmax))
+    plen = i32(np.array([Lmax, Lmax - 77], dtype=np.int32))
+    mask, pos = et.tree_mask(i32(par), i32(dep), plen)
+    good = et.tree_attention(q, kc, vc, plen, kt, vt, mask, pos)
+    try:
+        et.attention_wait_probe(1_000_000)
+        with pytest.raises(et.EagleError, match="device status 1"):
+            et.tree_attention(q, kc, vc, plen, kt, vt, mask, pos)
+    finally:
+        et.attention_wait_probe(0)
+    again = et.tree_attention(q, kc, vc, plen, kt, vt, mask, pos)
+    torch.cuda.synchronize()
+    assert torch.equal(again.view(torch.int16), good.view(torch.int16))
