@@ -78,6 +78,13 @@ _SIGS = {
     "eagle_tree_grow_begin": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p, _c_p]),
     "eagle_tree_grow_level": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p, _c_p]),
     "eagle_tree_grow_gains": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p]),
+    "eagle_tree_grow_level_width": (_c_i, [_c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p,
+                                           _c_p, _c_p]),
+    "eagle_tree_grow_frontier_logv": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz, _c_p, _c_p]),
+    "eagle_tree_grow_finish_widths": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_sz,
+                                             ctypes.POINTER(TreeStruct), ctypes.POINTER(_c_i), _c_p]),
+    "eagle_size_level_width": (_c_i, [ctypes.POINTER(CostTableStruct), ctypes.c_double, ctypes.c_double, _c_i, _c_p,
+                                      _c_i, _c_i, ctypes.c_double, ctypes.POINTER(_c_i), _c_p]),
     "eagle_tree_grow_finish": (_c_i, [_c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_sz,
                                       ctypes.POINTER(TreeStruct), ctypes.POINTER(_c_i), _c_p]),
     "eagle_static_tree_rows": (_c_i, [_c_p, _c_p, _c_i]),
@@ -470,6 +477,7 @@ class TreeGrower:
         self.ftok = torch.empty(B, k, dtype=torch.int32, device=self.device)
         self.fpar = torch.empty(B, k, dtype=torch.int32, device=self.device)
         self.gain = torch.empty(B, dtype=torch.float64, device=self.device)
+        self.flogv = torch.empty(B, k, dtype=torch.float64, device=self.device)
 
     def begin(self, root_logits: torch.Tensor):
         _check(lib().eagle_tree_grow_begin(_ptr(root_logits), self.dt, self.B, self.V, self.depth, self.k,
@@ -482,6 +490,34 @@ class TreeGrower:
                                            _ptr(self.state), self.state.numel(), _ptr(self.ftok), _ptr(self.fpar),
                                            _stream(self.device)), "eagle_tree_grow_level")
         return self.ftok, self.fpar
+
+    def level_width(self, level_logits: torch.Tensor, level: int, width: int):
+        """A level drafted from the first `width` frontier slots only: level_logits [B][width][V]."""
+        _check(lib().eagle_tree_grow_level_width(_ptr(level_logits), self.dt, self.B, self.V, self.depth, self.k,
+                                                 level, width, _ptr(self.state), self.state.numel(), _ptr(self.ftok),
+                                                 _ptr(self.fpar), _stream(self.device)), "eagle_tree_grow_level_width")
+        return self.ftok, self.fpar
+
+    def frontier_logv(self) -> torch.Tensor:
+        """The last level's k best candidates per sequence, log V in rank order [B][k] (device, float64)."""
+        _check(lib().eagle_tree_grow_frontier_logv(self.dt, self.B, self.V, self.depth, self.k, _ptr(self.state),
+                                                   self.state.numel(), _ptr(self.flogv), _stream(self.device)),
+               "eagle_tree_grow_frontier_logv")
+        return self.flogv
+
+    def finish_widths(self, widths) -> Tree:
+        """The tree keeping the widths[l-1] best candidates of each level l drafted."""
+        levels = len(widths)
+        w = (ctypes.c_int * levels)(*[int(x) for x in widths])
+        R = 1 + (self.depth - 1) * self.k
+        tree = alloc_tree(self.B, R, levels, self.k, max(1, sum(int(x) for x in widths)), self.device)
+        st = tree.struct()
+        n_out = _c_i(0)
+        _check(lib().eagle_tree_grow_finish_widths(self.dt, self.B, self.V, self.depth, self.k, levels, w,
+                                                   _ptr(self.state), self.state.numel(), ctypes.byref(st),
+                                                   ctypes.byref(n_out), _stream(self.device)),
+               "eagle_tree_grow_finish_widths")
+        return tree
 
     def gains(self) -> torch.Tensor:
         _check(lib().eagle_tree_grow_gains(self.dt, self.B, self.V, self.depth, self.k, _ptr(self.state),

@@ -80,8 +80,14 @@ struct Parity {
 // This thread's slice [x0, x1) of the current rows, cached in shared memory.
 // Element i of thread t sits at [i * kAcceptThreads + t], so a warp reading
 // its threads' i-th elements touches consecutive words (no bank conflicts).
+// With fp32 logits the cache holds the probabilities p = exp(l - lse_t) and
+// q = exp(l - lse_d) themselves (same size as the logits), computed once when
+// a row is loaded, so every later sweep at that node costs two FMAs and a max
+// per token; with bf16 logits it holds the logits (half the bytes) and each
+// sweep recomputes the exponentials.
 template <typename T>
 struct Slice {
+  static constexpr bool kProbs = sizeof(T) == 4;
   static constexpr int kVec = 16 / (int)sizeof(T);              // elements per 16-byte load
   static constexpr int kMaxLoads = slice_max<T>() / kVec;       // 16-byte loads per full slice
   T* tc;  // target row slice
@@ -93,8 +99,13 @@ struct Slice {
 
   __device__ __forceinline__ T& at(T* base, int i) const { return base[(size_t)i * kAcceptThreads + threadIdx.x]; }
 
-  // Copy the slices of up to two rows (src may be null), all loads in flight first.
-  __device__ void load2(const T* s0, T* d0, const T* s1, T* d1) const {
+  __device__ __forceinline__ T stored(T v, Split2 lse) const {
+    if constexpr (kProbs) return exp_minus(to_f(v), lse);
+    return v;
+  }
+  // Copy the slices of up to two rows (src may be null), all loads in flight
+  // first; with kProbs each element is stored as its probability under lse0 / lse1.
+  __device__ void load2(const T* s0, T* d0, Split2 lse0, const T* s1, T* d1, Split2 lse1) const {
     const int len = x1 - x0;
     if (vec_ok && len == slice) {
       uint4 v0[kMaxLoads], v1[kMaxLoads];
@@ -112,28 +123,35 @@ struct Slice {
           const T* e1 = reinterpret_cast<const T*>(&v1[q]);
 #pragma unroll
           for (int e = 0; e < kVec; ++e) {
-            if (s0) at(d0, q * kVec + e) = e0[e];
-            if (s1) at(d1, q * kVec + e) = e1[e];
+            if (s0) at(d0, q * kVec + e) = stored(e0[e], lse0);
+            if (s1) at(d1, q * kVec + e) = stored(e1[e], lse1);
           }
         }
       }
     } else {
       for (int i = 0; i < len; ++i) {
-        if (s0) at(d0, i) = s0[x0 + i];
-        if (s1) at(d1, i) = s1[x0 + i];
+        if (s0) at(d0, i) = stored(s0[x0 + i], lse0);
+        if (s1) at(d1, i) = stored(s1[x0 + i], lse1);
       }
     }
   }
-  __device__ void ensure(const T* trow, int tkey, const T* drow, int dkey) {
+  // tkey / dkey name the rows (target row j, draft row r), lse_t / lse_d their normalisers.
+  __device__ void ensure(const T* trow, int tkey, Split2 lse_t, const T* drow, int dkey, Split2 lse_d) {
     const bool lt = cached_t != tkey, ld = drow && cached_d != dkey;
-    if (lt || ld) load2(lt ? trow : nullptr, tc, ld ? drow : nullptr, dc);
+    if (lt || ld) load2(lt ? trow : nullptr, tc, lse_t, ld ? drow : nullptr, dc, lse_d);
     if (lt) cached_t = tkey;
     if (ld) cached_d = dkey;
   }
   __device__ __forceinline__ float weight(const SweepArgs& a, int i) const {
-    const float p = exp_minus(to_f(at(tc, i)), a.lse_t);
+    float p, q = 0.f;
+    if constexpr (kProbs) {
+      p = to_f(at(tc, i));
+      if (a.use_q) q = to_f(at(dc, i));
+    } else {
+      p = exp_minus(to_f(at(tc, i)), a.lse_t);
+      if (a.use_q) q = exp_minus(to_f(at(dc, i)), a.lse_d);
+    }
     if (!a.use_q) return p;
-    const float q = exp_minus(to_f(at(dc, i)), a.lse_d);
     return fmaxf(0.f, fmaf(-a.t.lo, q, fmaf(-a.t.hi, q, p)));
   }
 };
@@ -359,10 +377,10 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
         int nc = c + 1;
         while (nc <= n && sm.par[nc - 1] != j) ++nc;
         if (nc <= n) {  // another sibling will be tested: need F(t)
-          sl.ensure(trow, j, drow, r);
           SweepArgs a;
           a.use_q = true;
           a.lse_t.set(lse_t); a.lse_d.set(lse_d); a.t.set(t);
+          sl.ensure(trow, j, a.lse_t, drow, r, a.lse_d);
           F = sweep_total<T>(sl, a, sm, cluster, par);
           if (!(F > 0.0)) break;  // p == q left nothing: keep the walk here
         }
@@ -396,12 +414,13 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   }
   const int r = sm.drow[j];
   const bool use_q = rejected_here && r >= 0;
-  sl.ensure(tgt + (trow0 + j) * (size_t)V, j, use_q ? dft + ((size_t)b * R + r) * (size_t)V : nullptr, r);
   SweepArgs a;
   a.use_q = use_q;
   a.lse_t.set(lse_t);
   a.lse_d.set(sm.lse_d[j]);
   a.t.set(t);
+  sl.ensure(tgt + (trow0 + j) * (size_t)V, j, a.lse_t, use_q ? dft + ((size_t)b * R + r) * (size_t)V : nullptr, r,
+            a.lse_d);
   const double total = sweep_sample<T>(sl, a, sm.u_res[j], sm, cluster, bonus + b, par);
   if (!(total > 0.0) && leader) bonus[b] = amax;  // nothing left to sample from
   cluster.sync();  // no CTA leaves while another may still read its shared memory

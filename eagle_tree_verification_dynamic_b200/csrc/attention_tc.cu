@@ -50,18 +50,17 @@ using namespace sm100;
 constexpr int kTcThreads = 320;   // 10 warps: producer, MMA, 8 softmax
 constexpr int kBN = kAttnKeysPerTile;
 constexpr int kRowsPerCta = kAttnRowsPerUnit;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
 constexpr int kSmemOptIn = 232448;  // largest dynamic shared memory a block may opt into on sm_100
 constexpr int kCombineThreads = 128;
 
 // Shared memory from the (1024-byte aligned) dynamic base: a 3 KB header
 // (barriers, then each row's (max, sum) exchange between the two softmax
-// warps of a lane quarter), two Q buffers, two P buffers, the K/V ring.
+// warps of a lane quarter), two Q buffers, the K/V ring (P lives in TMEM).
 template <int D>
 struct TcLayout {
   static constexpr int kAtoms = D / 64;               // 128-byte column atoms along D
   static constexpr int kQBytes = kAtoms * 128 * 128;  // 128 rows
-  static constexpr int kPBytes = 128 * 128;           // 128 rows x 64 keys bf16
   static constexpr int kKVAtomBytes = kBN * 128;      // 64 keys x 128 B
   static constexpr int kKBytes = kAtoms * kKVAtomBytes;
   static constexpr int kStageBytes = 2 * kKBytes;     // K + V
@@ -69,14 +68,16 @@ struct TcLayout {
   static constexpr int kBarOff = 0;
   static constexpr int kXchOff = 512;                 // float2 [2 halves][128 rows]
   static constexpr int kQOff = kHdrBytes;             // two Q buffers
-  static constexpr int kPOff = kQOff + 2 * kQBytes;   // two P buffers
-  static constexpr int kStageOff = kPOff + 2 * kPBytes;
+  static constexpr int kStageOff = kQOff + 2 * kQBytes;
   static constexpr int kStagesFit = (kSmemOptIn - kStageOff) / kStageBytes;
   static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
   static constexpr int kSmemBytes = kStageOff + kStages * kStageBytes;
   // TMEM: S double buffer (2 x 64 columns), then O over each tile's keys
   // 0..31 (O_A) and over keys 32..63 (O_B): the two softmax warps of a lane
   // quarter keep independent running maxima and are merged once per piece.
+  // P (bf16, two keys per column) overwrites the S it came from: keys 0..31
+  // at the buffer's columns 0..15, keys 32..63 at columns 32..47, each inside
+  // the columns of S its own warp has already read.
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0;  // S buffer i at column 64 * i
   static constexpr uint32_t kColOA = 128;
@@ -635,14 +636,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         if (!ok) break;
         tc_fence_after();
         const int st = jp % S;
-        const uint32_t p_addr = s_base + Lay::kPOff + (jp & 1) * Lay::kPBytes;
+        const uint32_t p_tmem = tmem + Lay::kColS + (uint32_t)((jp & 1) * kBN);
         const uint32_t v_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes + Lay::kKBytes;
-        // keys 0..31 of the tile into O_A, keys 32..63 into O_B
+        // keys 0..31 of the tile into O_A, keys 32..63 into O_B; P from TMEM
+        // (16 keys = 8 columns per MMA)
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t da = smem_desc(p_addr + kk * 32, 16, 1024, kSwizzle128B);
+          const uint32_t a_col = (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8);
           const uint64_t db = smem_desc(v_addr + kk * 2048, Lay::kKVAtomBytes, 1024, kSwizzle128B);
-          mma_bf16_ss(kk < 2 ? t_oa : t_ob, da, db, id_pv, (!first || (kk & 1)) ? 1u : 0u);
+          mma_bf16_ts(kk < 2 ? t_oa : t_ob, p_tmem + a_col, db, id_pv, (!first || (kk & 1)) ? 1u : 0u);
         }
         mma_commit(smem_u32(&bars->empty[st]));
         mma_commit(smem_u32(&bars->pv_done[jp & 1]));
@@ -729,12 +731,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           for (int cc = 4; cc < 32; ++cc) m4[cc & 3] = fmaxf(m4[cc & 3], x[cc]);
           float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           mx *= sl2;  // scale > 0 keeps the order
-          // P buffer (jg & 1) was last read by PV(jg - 2)
-          if (jg >= 2 &&
-              !__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[jg & 1]), ((jg - 2) >> 1) & 1, abort))) {
-            ok = false;
-            break;
-          }
+          // (P of this tile replaces S(jg) in TMEM: PV(jg - 2), the last reader of
+          // those columns, completed before QK^T(jg), whose commit s_full waited on)
           const bool rebase = mx > m_used + 8.f;
           if (__any_sync(kFull, rebase && t > pc.tb && l > 0.f)) {
             // this half's O may only be rescaled once PV(jg - 1) has finished accumulating
@@ -757,25 +755,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           }
           if (rebase) m_used = mx;
           const float neg_m = m_used > -INFINITY ? -m_used : 0.f;  // no visible key yet: every x is -inf
-          unsigned char* prow = smem + Lay::kPOff + (jg & 1) * Lay::kPBytes + r_local * 128;
           float s4[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t packed[16];
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            uint32_t packed[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float e0 = ex2(fmaf(x[c8 * 8 + 2 * u], sl2, neg_m));
-              const float e1 = ex2(fmaf(x[c8 * 8 + 2 * u + 1], sl2, neg_m));
-              s4[u] += e0 + e1;
-              const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-              packed[u] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            const int chunk = half * 4 + c8;  // 16-byte chunk of the 128-byte P row
-            *reinterpret_cast<uint4*>(prow + ((chunk ^ (r_local & 7)) << 4)) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          for (int c2 = 0; c2 < 16; ++c2) {
+            const float e0 = ex2(fmaf(x[2 * c2], sl2, neg_m));
+            const float e1 = ex2(fmaf(x[2 * c2 + 1], sl2, neg_m));
+            s4[c2 & 3] += e0 + e1;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+            packed[c2] = *reinterpret_cast<const uint32_t*>(&h2);
           }
           l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
-          fence_proxy_async_smem();
+          tmem_st16u(t_s + (uint32_t)((jg & 1) * kBN), packed);  // P over this half's first 16 S columns
+          tmem_wait_st();
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&bars->p_full[jg & 1]));

@@ -86,8 +86,11 @@ cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R,
 
 // The expansion / rerank alone, from each row's top-k tokens and logits
 // [B][R][k] and out.row_lse [B][R] (the build's second kernel).
+// widths (host, depth entries, or null): keep the widths[l-1] best candidates
+// of each level l instead of the n best over all levels (n = their sum).
 cudaError_t launch_tree_expand(const int32_t* row_tok, const float* row_val, int B, int R, int depth, int k, int n,
-                               const eagle_tree_t& out, const MaskOut* mo, bool pdl, cudaStream_t s);
+                               const eagle_tree_t& out, const MaskOut* mo, bool pdl, cudaStream_t s,
+                               const int* widths = nullptr);
 
 // ---- tree mask (tree_mask.cu)
 cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* depth, const int32_t* prefix_len,

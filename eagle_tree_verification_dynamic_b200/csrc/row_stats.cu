@@ -6,15 +6,22 @@
 // same sweep (k = 1) gives the argmax for greedy acceptance and the normaliser
 // of p_target for sampling.
 //
-// One CTA owns one (row, chunk).  Threads stream 16-byte vectors (coalesced,
-// L1 no-allocate) and keep, per lane, the M best (value, id) pairs in
-// registers plus a base-2 scaled fp64 partial of sum exp(logit).  A warp
-// builds its exact top-k from the lanes' lists with bitonic sort/merge rounds
-// (a lane is rescanned from memory only if all M of its entries made the
-// cut); warps merge pairwise through shared memory.  The CTA that finishes a
-// row's last chunk (an atomic ticket; nobody waits) merges the row's chunks
-// and writes the final per-row outputs.
+// Rows whose bytes are 16-byte aligned (the usual case) go through
+// row_sweep_kernel: every row is cut into fixed 16 KB chunks, all chunks of all
+// rows form one list, and a persistent grid (three CTAs per SM) takes
+// contiguous ranges of it.  In each CTA one producer thread streams its chunks
+// into a four-stage shared-memory ring with untiled bulk copies (TMA, no
+// multicast) while eight consumer warps read them: per lane the M best
+// (value, id) pairs in registers, and per chunk a base-2 scaled fp64 partial of
+// sum exp(logit) reduced in a fixed order (so a row's log-sum-exp does not
+// depend on the grid).  At the end of each row segment the warps build the
+// segment's exact top-k from the lanes' lists (bitonic sort/merge rounds; a
+// lane is rescanned from memory only if all M of its entries made the cut),
+// and the CTA that completes a row (an atomic ticket; nobody waits) merges the
+// row's chunks and writes the final per-row outputs.  Other rows use
+// row_stats_kernel, one CTA per (row, chunk) with scalar loads.
 #include "eagle_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace eagle {
 
@@ -259,6 +266,275 @@ row_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k, ChunkSt
   if (LSE && out.lse && lane == 0) out.lse[row] = lse;
 }
 
+// ------------------------------------------------------ chunked TMA sweep
+constexpr int kSwConsumerWarps = 8;
+constexpr int kSwConsumers = kSwConsumerWarps * 32;
+constexpr int kSwThreads = kSwConsumers + 32;  // + one producer warp
+constexpr int kSwChunkBytes = 16384;           // one ring stage = one chunk
+constexpr int kSwStages = 4;
+constexpr int kSwCtasPerSm = 3;
+
+struct SwShared {
+  uint64_t full[kSwStages];
+  uint64_t empty[kSwStages];
+  uint64_t keys[kSwConsumerWarps][32];
+  float e[2][kSwConsumerWarps];  // per-chunk warp partials, double-buffered by chunk parity
+  double s[2][kSwConsumerWarps];
+  int abort;
+  int last;
+};
+constexpr size_t kSwSmemBytes = (size_t)kSwStages * kSwChunkBytes + sizeof(SwShared);
+
+struct SweepArgs {
+  const unsigned char* x;  // row r starts at x + r * row_bytes (16-byte aligned)
+  long long nchunks;       // rows * ncpr
+  int V, k, ncpr, chunk_elems, row_bytes;
+  ChunkStat* stats;  // [rows * ncpr]: log-sum-exp partial of every chunk
+  uint64_t* keys;    // [rows * ncpr][k]: a segment's top-k sits in its last chunk's slot, zeros elsewhere
+  int* tickets;      // [rows]
+  int* status;       // set to 1 when a wait gave up (the outputs are then undefined)
+  RowOut out;
+};
+
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSwConsumers) : "memory"); }
+
+// Largest key strictly below `last` among this consumer thread's elements of
+// the chunks [c0, c1] of a row (the main sweep's element assignment; -inf and
+// NaN never qualify), read from global memory.
+template <typename T>
+__device__ uint64_t seg_next_below(const SweepArgs& a, long long row, int c0, int c1, uint64_t last) {
+  constexpr int N = Elem<T>::kPerVec;
+  uint64_t best = 0;
+  const unsigned char* rp = a.x + (size_t)row * a.row_bytes;
+  for (int c = c0; c <= c1; ++c) {
+    const int off = c * kSwChunkBytes;
+    const int nvec = min(kSwChunkBytes, a.row_bytes - off) / 16;
+    const uint4* vp = reinterpret_cast<const uint4*>(rp + off);
+    for (int v = threadIdx.x; v < nvec; v += kSwConsumers) {
+      float f[N];
+      Elem<T>::unpack(__ldg(vp + v), f);
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        if (!(f[i] > -INFINITY)) continue;
+        const uint64_t key = make_key(f[i], c * a.chunk_elems + v * N + i);
+        if (key < last && key > best) best = key;
+      }
+    }
+  }
+  return best;
+}
+
+template <typename T, int M>
+__global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(SweepArgs a) {
+  using namespace sm100;
+  constexpr int N = Elem<T>::kPerVec;
+  constexpr int S = kSwStages;
+  extern __shared__ __align__(1024) unsigned char sw_smem[];
+  SwShared& sh = *reinterpret_cast<SwShared*>(sw_smem + (size_t)S * kSwChunkBytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long C = gridDim.x;
+  const long long g0 = (long long)blockIdx.x * a.nchunks / C;
+  const long long g1 = (long long)(blockIdx.x + 1) * a.nchunks / C;
+  const int nj = (int)(g1 - g0);
+  volatile int* abort = &sh.abort;
+  const uint32_t ring = smem_u32(sw_smem);
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&sh.full[i]), 1);
+      mbar_init(smem_u32(&sh.empty[i]), kSwConsumerWarps);
+    }
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();  // the logits (and this workspace) may belong to the previous kernel
+
+  if (warp == kSwConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int j = 0;
+      for (; j < nj; ++j) {
+        const int st = j % S;
+        if (j >= S && !mbar_wait(smem_u32(&sh.empty[st]), ((j / S) - 1) & 1, abort)) break;
+        if (*abort) break;
+        const long long g = g0 + j;
+        const long long row = g / a.ncpr;
+        const int off = (int)(g - row * a.ncpr) * kSwChunkBytes;
+        const int bytes = min(kSwChunkBytes, a.row_bytes - off);
+        const uint32_t fb = smem_u32(&sh.full[st]);
+        mbar_arrive_expect_tx(fb, (uint32_t)bytes);
+        bulk_load(ring + st * kSwChunkBytes, a.x + (size_t)row * a.row_bytes + off, (uint32_t)bytes, fb);
+      }
+      // every copy issued lands before the CTA may exit
+      for (int d = (j > S ? j - S : 0); d < j; ++d) mbar_wait_drain(smem_u32(&sh.full[d % S]), (d / S) & 1, 200000000ull);
+      if (*abort) atomicExch(a.status, 1);
+    }
+    griddep_launch_dependents();
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  LaneTop<M> top;
+  top.init();
+  float e_ref = -INFINITY;
+  double acc = 0.0;
+  long long seg_row = -1;
+  int seg_c0 = 0;
+
+  // end of a row segment [seg_c0, c_last] of row seg_row: its top-k into the
+  // last chunk's slot (zeros into the others), then the row's ticket
+  auto finish_segment = [&](int c_last) {
+    const int k = a.k;
+    uint64_t list;
+    if (k == 1) {
+      list = warp_max_u64(top.key(0));
+    } else {
+      list = warp_sort_desc(top.key(0));
+      uint64_t thr = __shfl_sync(kFull, list, k - 1);
+      bool need = top.key(0) != 0 && top.key(0) >= thr;
+      int r = 1;
+      for (; r < M; ++r) {
+        const uint64_t cand = need ? top.key(r) : 0ull;
+        if (!__any_sync(kFull, cand != 0)) { need = false; break; }
+        list = warp_merge_desc(list, warp_sort_desc(cand));
+        thr = __shfl_sync(kFull, list, k - 1);
+        need = cand != 0 && cand >= thr;
+      }
+      // all M entries of some lane made the cut: pull its further elements (rare)
+      uint64_t last = (r == M && need) ? top.key(M - 1) : 0ull;
+      need = last != 0;
+      while (__any_sync(kFull, need)) {
+        uint64_t nxt = 0;
+        if (need) nxt = seg_next_below<T>(a, seg_row, seg_c0, c_last, last);
+        list = warp_merge_desc(list, warp_sort_desc(nxt));
+        thr = __shfl_sync(kFull, list, k - 1);
+        need = nxt != 0 && nxt >= thr;
+        last = nxt;
+      }
+    }
+    if (lane < k) sh.keys[warp][lane] = list;
+    consumer_sync();
+    for (int step = 1; step < kSwConsumerWarps; step <<= 1) {  // pairwise merges: 3 rounds
+      if ((warp & (2 * step - 1)) == 0 && warp + step < kSwConsumerWarps) {
+        const uint64_t m = warp_merge_desc(lane < k ? sh.keys[warp][lane] : 0ull,
+                                           lane < k ? sh.keys[warp + step][lane] : 0ull);
+        if (lane < k) sh.keys[warp][lane] = m;
+      }
+      consumer_sync();
+    }
+    const size_t slot0 = (size_t)seg_row * a.ncpr;
+    if (warp == 0 && lane < k) a.keys[(slot0 + c_last) * k + lane] = sh.keys[0][lane];
+    for (int e = tid; e < (c_last - seg_c0) * k; e += kSwConsumers) a.keys[(slot0 + seg_c0) * k + e] = 0ull;
+    __threadfence();
+    consumer_sync();
+    if (tid == 0) {
+      const int nseg = c_last - seg_c0 + 1;
+      sh.last = atomicAdd(a.tickets + seg_row, nseg) + nseg == a.ncpr;
+    }
+    consumer_sync();
+    if (sh.last && warp == 0) {
+      // ---- this CTA completed the row: merge all of its chunks (fixed order)
+      __threadfence();
+      const ChunkStat* st = a.stats + slot0;
+      const uint64_t* kk = a.keys + slot0 * k;
+      double lse = 0.0;
+      LseAccum la;
+      la.init();
+      for (int c = lane; c < a.ncpr; c += 32) la.add(__ldcg(&st[c].e_ref), __ldcg(&st[c].acc));
+      const float e = warp_max_f(la.e);
+      double sum = la.s > 0.0 ? rescale_pow2(la.s, la.e, e) : 0.0;
+      sum = warp_sum_d(sum);
+      lse = sum > 0.0 ? kLn2 * ((double)e + log2(sum)) : -INFINITY;
+      uint64_t merged = 0ull;
+      for (int c = 0; c < a.ncpr; c += 8) {  // 8 chunk lists in flight, then merged
+        uint64_t kv[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          kv[t] = (lane < k && c + t < a.ncpr)
+                      ? __ldcg(reinterpret_cast<const unsigned long long*>(kk) + (size_t)(c + t) * k + lane)
+                      : 0ull;
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          if (c + t < a.ncpr) merged = warp_merge_desc(merged, kv[t]);
+      }
+      if (lane < k) {
+        if (a.out.tok) a.out.tok[seg_row * k + lane] = merged ? key_index(merged) : -1;
+        if (a.out.val) a.out.val[seg_row * k + lane] = merged ? key_value(merged) : -INFINITY;
+      }
+      if (a.out.lse && lane == 0) a.out.lse[seg_row] = lse;
+    }
+  };
+
+  for (int j = 0; j < nj; ++j) {
+    const long long g = g0 + j;
+    const long long row = g / a.ncpr;
+    const int c = (int)(g - row * a.ncpr);
+    if (row != seg_row) {
+      if (seg_row >= 0) finish_segment(c == 0 ? a.ncpr - 1 : c - 1);
+      seg_row = row;
+      seg_c0 = c;
+      top.init();
+    }
+    const int st = j % S;
+    // a wait that gives up leaves the data undefined but keeps every warp on
+    // the same barriers (the status word reports it)
+    mbar_wait(smem_u32(&sh.full[st]), (j / S) & 1, abort);
+    const int nvec = min(kSwChunkBytes, a.row_bytes - c * kSwChunkBytes) / 16;
+    const uint4* sp = reinterpret_cast<const uint4*>(sw_smem + st * kSwChunkBytes);
+    const int idx_base = c * a.chunk_elems;
+    for (int v = tid; v < nvec; v += kSwConsumers) {
+      float f[N];
+      Elem<T>::unpack(sp[v], f);
+      float vmax = f[0];
+#pragma unroll
+      for (int i = 1; i < N; ++i) vmax = fmaxf(vmax, f[i]);
+      if (vmax > top.s[M - 1]) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) top.push(f[i], idx_base + v * N + i);
+      }
+      if (vmax * kLog2eHi > e_ref) {  // a new reference exponent (rare)
+        const float e_new = ceilf(vmax * kLog2eHi);
+        acc = rescale_pow2(acc, e_ref, e_new);
+        e_ref = e_new;
+      }
+      if (e_ref > -INFINITY) {  // until a finite logit arrives every term is exp(-inf) = 0
+        float part = 0.f;
+#pragma unroll
+        for (int i = 0; i < N; ++i) part += exp2_scaled(f[i], e_ref);
+        acc += (double)part;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&sh.empty[st]));
+    // this chunk's log-sum-exp partial: lanes, then warps, in a fixed order
+    {
+      const float e = warp_max_f(e_ref);
+      double sum = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
+      sum = warp_sum_d(sum);
+      if (lane == 0) {
+        sh.e[j & 1][warp] = e;
+        sh.s[j & 1][warp] = sum;
+      }
+    }
+    consumer_sync();
+    if (tid == 0) {
+      LseAccum la;
+      la.init();
+      for (int w = 0; w < kSwConsumerWarps; ++w) la.add(sh.e[j & 1][w], sh.s[j & 1][w]);
+      ChunkStat cs;
+      cs.e_ref = la.e;
+      cs.pad = 0;
+      cs.acc = la.s;
+      a.stats[g] = cs;
+    }
+    e_ref = -INFINITY;
+    acc = 0.0;
+  }
+  griddep_launch_dependents();
+  if (seg_row >= 0) finish_segment((int)(g1 - 1 - seg_row * a.ncpr));
+  if (tid == 0 && *abort) atomicExch(a.status, 1);
+}
+
 // ------------------------------------------------------------------- host
 ChunkPlan plan_chunks(long long rows, int V, int elem_bytes) {
   const int per_vec = 16 / elem_bytes;
@@ -275,12 +551,34 @@ ChunkPlan plan_chunks(long long rows, int V, int elem_bytes) {
   return p;
 }
 
-// workspace: [chunk stats rows*nc][chunk keys rows*nc*k][row tickets rows]
-size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k, long long plan_rows) {
+namespace {
+
+// Chunks per row of the TMA sweep (fixed 16 KB chunks: independent of the row count).
+int sweep_chunks_per_row(int V, int elem_bytes) {
+  return (int)(((long long)V * elem_bytes + kSwChunkBytes - 1) / kSwChunkBytes);
+}
+
+// workspace: [chunk stats rows*nc][chunk keys rows*nc*k][row tickets rows + status word]
+// with nc the larger chunk count of the two kernels, so either one fits.
+struct RsLayout {
+  size_t keys_off, tickets_off, status_off, bytes;
+};
+RsLayout rs_layout(long long rows, int V, int elem_bytes, int k, long long plan_rows) {
   const ChunkPlan p = plan_chunks(plan_rows > 0 ? plan_rows : rows, V, elem_bytes);
-  const size_t n = (size_t)rows * p.n_chunks;
-  return align_up(n * sizeof(ChunkStat), 256) + align_up(n * k * sizeof(uint64_t), 256) +
-         align_up((size_t)rows * sizeof(int), 256);
+  const int nc_sw = sweep_chunks_per_row(V, elem_bytes);
+  const size_t n = (size_t)rows * (size_t)(p.n_chunks > nc_sw ? p.n_chunks : nc_sw);
+  RsLayout l;
+  l.keys_off = align_up(n * sizeof(ChunkStat), 256);
+  l.tickets_off = l.keys_off + align_up(n * k * sizeof(uint64_t), 256);
+  l.status_off = l.tickets_off + (size_t)rows * sizeof(int);
+  l.bytes = align_up(l.status_off + sizeof(int), 256);
+  return l;
+}
+
+}  // namespace
+
+size_t row_stats_ws_bytes(long long rows, int V, int elem_bytes, int k, long long plan_rows) {
+  return rs_layout(rows, V, elem_bytes, k, plan_rows).bytes;
 }
 
 template <typename T, bool LSE, int M>
@@ -308,28 +606,54 @@ static cudaError_t launch_t(const void* x, long long rows, int V, int k, bool ls
   return launch_typed<T, false, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s, pdl);
 }
 
+template <typename T, int M>
+static cudaError_t launch_sweep(const SweepArgs& a, cudaStream_t s, bool pdl) {
+  cudaError_t e = ensure_smem_limit((const void*)row_sweep_kernel<T, M>, kSwSmemBytes);
+  if (e != cudaSuccess) return e;
+  long long C = (long long)device_sm_count() * kSwCtasPerSm;
+  if (C > a.nchunks) C = a.nchunks;
+  return launch_kernel(row_sweep_kernel<T, M>, dim3((unsigned)C), dim3(kSwThreads), kSwSmemBytes, s, pdl, a);
+}
+
 void row_stats_tickets_span(long long rows, int V, int elem_bytes, int k, size_t* off, size_t* bytes) {
-  const ChunkPlan p = plan_chunks(rows, V, elem_bytes);
-  const size_t n = (size_t)rows * p.n_chunks;
-  *off = align_up(n * sizeof(ChunkStat), 256) + align_up(n * k * sizeof(uint64_t), 256);
-  *bytes = (size_t)rows * sizeof(int);
+  const RsLayout l = rs_layout(rows, V, elem_bytes, k, 0);
+  *off = l.tickets_off;
+  *bytes = (size_t)rows * sizeof(int) + sizeof(int);  // the tickets and the status word
 }
 
 cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, int k, bool lse, const RowOut& out,
                              void* ws, cudaStream_t s, bool zero_tickets, bool pdl, long long plan_rows) {
   const int eb = dtype_bytes(dtype);
-  const ChunkPlan p = plan_chunks(plan_rows > 0 ? plan_rows : rows, V, eb);
-  const size_t n = (size_t)rows * p.n_chunks;
+  const RsLayout l = rs_layout(rows, V, eb, k, plan_rows);
   char* base = static_cast<char*>(ws);
   ChunkStat* stats = reinterpret_cast<ChunkStat*>(base);
-  uint64_t* keys = reinterpret_cast<uint64_t*>(base + align_up(n * sizeof(ChunkStat), 256));
-  int* tickets = reinterpret_cast<int*>(base + align_up(n * sizeof(ChunkStat), 256) +
-                                        align_up(n * k * sizeof(uint64_t), 256));
+  uint64_t* keys = reinterpret_cast<uint64_t*>(base + l.keys_off);
+  int* tickets = reinterpret_cast<int*>(base + l.tickets_off);
   if (zero_tickets) {
-    cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)rows * sizeof(int), s);
+    cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)rows * sizeof(int) + sizeof(int), s);
     if (e != cudaSuccess) return e;
   }
   const bool vec = ((uintptr_t)x % 16 == 0) && (((size_t)V * eb) % 16 == 0);
+  if (vec && (size_t)V * eb <= 0x7fffffffu) {
+    // the chunked TMA sweep computes the log-sum-exp always (lse == false only drops the output)
+    SweepArgs a;
+    a.x = static_cast<const unsigned char*>(x);
+    a.ncpr = sweep_chunks_per_row(V, eb);
+    a.nchunks = rows * a.ncpr;
+    a.V = V;
+    a.k = k;
+    a.chunk_elems = kSwChunkBytes / eb;
+    a.row_bytes = V * eb;
+    a.stats = stats;
+    a.keys = keys;
+    a.tickets = tickets;
+    a.status = reinterpret_cast<int*>(base + l.status_off);
+    a.out = out;
+    if (!lse) a.out.lse = nullptr;
+    if (dtype == EAGLE_F32) return k == 1 ? launch_sweep<float, 1>(a, s, pdl) : launch_sweep<float, 4>(a, s, pdl);
+    return k == 1 ? launch_sweep<__nv_bfloat16, 1>(a, s, pdl) : launch_sweep<__nv_bfloat16, 4>(a, s, pdl);
+  }
+  const ChunkPlan p = plan_chunks(plan_rows > 0 ? plan_rows : rows, V, eb);
   if (dtype == EAGLE_F32) return launch_t<float>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s, pdl);
   return launch_t<__nv_bfloat16>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s, pdl);
 }

@@ -11,7 +11,13 @@
 //   level l  grows the verified set from (l-1)k to lk candidates per
 //            sequence; ratio = (sum of the batch's gains) / (C(lk) - C((l-1)k))
 //            in tokens per unit of cost (infinite when the cost does not
-//            grow); the level is kept iff ratio >= threshold.
+//            grow); the level is kept iff ratio >= threshold;
+//   width    (widening or deepening) the level's candidates one at a time in
+//            descending V, the j-th best of every sequence together: gain =
+//            sum over the batch of its V, marginal cost C(n + j) - C(n + j - 1)
+//            with n candidates per sequence chosen before this level; taken
+//            while gain > 0 and gain / cost >= threshold (a cost that does not
+//            grow passes); the number taken is the level's width.
 #include <cmath>
 
 #include "eagle_internal.h"
@@ -85,6 +91,30 @@ EAGLE_API eagle_status eagle_size_keep_level(const eagle_cost_table_t* table, do
   const double r = dc <= 0.0 ? INFINITY : g / dc;
   if (ratio) *ratio = r;
   *keep = r >= threshold ? 1 : 0;
+  return EAGLE_OK;
+}
+
+EAGLE_API eagle_status eagle_size_level_width(const eagle_cost_table_t* table, double B, double L, int n_before,
+                                             const double* logv, int k, int nb, double threshold, int* width,
+                                             double* ratios) {
+  if (!table || !logv || !width) return EAGLE_ERR_NULL;
+  if (!valid_table(table)) return EAGLE_ERR_SHAPE;
+  if (k <= 0 || nb <= 0 || n_before < 0 || !std::isfinite(B) || !std::isfinite(L) || std::isnan(threshold))
+    return EAGLE_ERR_SHAPE;
+  int w = 0;
+  for (int j = 0; j < k; ++j) {
+    double g = 0.0;
+    for (int b = 0; b < nb; ++b) g += std::exp(logv[(size_t)b * k + j]);  // V = 0 for log V = -inf
+    const double dc = cost(table, B, L, (double)(n_before + j + 1)) - cost(table, B, L, (double)(n_before + j));
+    const double r = dc <= 0.0 ? INFINITY : g / dc;
+    if (ratios) ratios[j] = r;
+    if (!(g > 0.0 && r >= threshold)) {
+      for (int i = j + 1; ratios && i < k; ++i) ratios[i] = NAN;  // not examined
+      break;
+    }
+    w = j + 1;
+  }
+  *width = w;
   return EAGLE_OK;
 }
 

@@ -3,13 +3,15 @@
 //   0. (before it, in parallel over all rows) the vocabulary sweep gives each
 //      draft row's log-sum-exp and top-k;
 //   1. lp = logit - lse turns the top-k logits into log-confidences;
-//   2. level 1 = the root's k children; for each level up to depth-1, rank the
-//      level's candidates by (log V desc, candidate id asc) (each candidate
-//      counts the larger keys of its level), the first k form the frontier
-//      (slot = rank, which names the draft row of the node), and
-//      their k children each enter the next level with
+//   2. level 1 = the root's k children; for each level, every candidate counts
+//      the larger (log V desc, candidate id asc) keys of its level: that count
+//      is its rank, which places it in the level's sorted list, and the first
+//      k ranks form the frontier (slot = rank, which names the draft row of
+//      the node); their k children each enter the next level with
 //      log V = log V(parent) + lp (log of the product of confidences);
-//   3. a block-wide bitonic sort over all P candidates keeps the best n;
+//   3. rerank: a candidate's rank among all P is its rank in its own level
+//      plus, for every other level, the number of larger keys there (a binary
+//      search in that level's sorted list); the n with rank < n are kept;
 //   4. a prefix count renumbers the kept candidates 1..n by ascending id and
 //      the tree arrays are written.
 // log V is carried in fp64 so that the rounding of one path sum can only
@@ -18,12 +20,14 @@
 
 namespace eagle {
 
-constexpr int kBuildThreads = 1024;  // the largest expansion block
+constexpr int kBuildThreads = 256;  // the largest expansion block
 
 struct BuildSmem {
   double* row_lp;    // [R*k] log-confidence of each row's top-k children
   double* cand_lv;   // [P]   log V
-  uint64_t* sort_k;  // [max(Ppow, 2*threads)] keys / exchange buffers
+  uint64_t* keys;    // [P]   ranking key of candidate g
+  uint64_t* sorted;  // [P]   each level's keys in rank order, at the level's id range
+  int* lrank;        // [P]   rank of candidate g within its level
   int* row_tok;      // [R*k]
   int* cand_tok;     // [P]
   int* cand_par;     // [P]   parent candidate id, -1 = root
@@ -36,25 +40,23 @@ struct BuildSmem {
 };
 
 
-__host__ __device__ inline int next_pow2(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
+// Per-level widths of the cost-aware harness (on = 0: keep the best n overall).
+struct LevelWidths {
+  int w[EAGLE_MAX_DEPTH];
+  int on;
+};
 
 // row_tok / row_val: each draft row's top-k tokens and logits (descending),
 // row_lse: each row's log-sum-exp (also the tree's row_lse output).
 template <int NT>
 __global__ void __launch_bounds__(NT)
 tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restrict__ row_val_g, int R, int depth,
-                   int k, int n, eagle_tree_t out, MaskOut mo) {
+                   int k, int n, eagle_tree_t out, MaskOut mo, LevelWidths lw) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kk = k * k;
   const int P = k + (depth - 1) * kk;
-  const int Ppow = next_pow2(P);
-  const int nsort = Ppow > 2 * NT ? Ppow : 2 * NT;
 
   griddep_wait();  // the row statistics come from the previous kernel
   griddep_launch_dependents();
@@ -63,14 +65,16 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     unsigned char* p = smem_raw;
     sm.row_lp = reinterpret_cast<double*>(p);    p += sizeof(double) * R * k;
     sm.cand_lv = reinterpret_cast<double*>(p);   p += sizeof(double) * P;
-    sm.sort_k = reinterpret_cast<uint64_t*>(p);  p += sizeof(uint64_t) * nsort;
+    sm.keys = reinterpret_cast<uint64_t*>(p);    p += sizeof(uint64_t) * P;
+    sm.sorted = reinterpret_cast<uint64_t*>(p);  p += sizeof(uint64_t) * P;
+    sm.lrank = reinterpret_cast<int*>(p);        p += sizeof(int) * P;
     sm.row_tok = reinterpret_cast<int*>(p);      p += sizeof(int) * R * k;
     sm.cand_tok = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
     sm.cand_par = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
     sm.cand_row = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
     sm.node_of = reinterpret_cast<int*>(p);      p += sizeof(int) * P;
     sm.frontier = reinterpret_cast<int*>(p);     p += sizeof(int) * 32;
-    sm.warp_cnt = reinterpret_cast<int*>(p);    p += sizeof(int) * (NT / 32);
+    sm.warp_cnt = reinterpret_cast<int*>(p);     p += sizeof(int) * (NT / 32);
     sm.node_par = reinterpret_cast<int*>(p);     p += sizeof(int) * EAGLE_MAX_NODES;
     sm.node_dep = reinterpret_cast<int*>(p);
   }
@@ -82,90 +86,75 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     sm.row_tok[e] = tok;
     sm.row_lp[e] = tok >= 0 ? (double)row_val_g[g] - out.row_lse[(size_t)b * R + e / k] : -INFINITY;
   }
+  __syncthreads();
   for (int c = tid; c < P; c += NT) {
     sm.cand_row[c] = -1;
-    sm.node_of[c] = 0;
-  }
-  __syncthreads();
-  for (int c = tid; c < k; c += NT) {
-    sm.cand_lv[c] = sm.row_lp[c];
-    sm.cand_tok[c] = sm.row_tok[c];
-    sm.cand_par[c] = -1;
+    if (c < k) {  // level 1: the root's children
+      sm.cand_lv[c] = sm.row_lp[c];
+      sm.cand_tok[c] = sm.row_tok[c];
+      sm.cand_par[c] = -1;
+      sm.keys[c] = cand_key(sm.row_lp[c], c);
+    }
   }
   __syncthreads();
 
-  // 2. level by level: the k best candidates of the level form the frontier
-  //    (a candidate's rank = how many candidates of its level have a larger key)
-  for (int level = 1; level < depth; ++level) {
+  // 2. level by level: a candidate's rank = how many keys of its level are
+  //    larger; it files the key into the level's sorted list, and the first k
+  //    ranks form the frontier whose children make the next level
+  for (int level = 1; level <= depth; ++level) {
     const int lo = level == 1 ? 0 : k + (level - 2) * kk;
     const int cnt = level == 1 ? k : kk;
-    for (int c = tid; c < cnt; c += NT) sm.sort_k[c] = cand_key(sm.cand_lv[lo + c], lo + c);
-    __syncthreads();
     for (int c = tid; c < cnt; c += NT) {
-      const uint64_t mine = sm.sort_k[c];
+      const uint64_t mine = sm.keys[lo + c];
       int rank = 0;
 #pragma unroll 8
-      for (int o = 0; o < cnt; ++o) rank += sm.sort_k[o] > mine ? 1 : 0;
-      if (rank < k) {
+      for (int o = 0; o < cnt; ++o) rank += sm.keys[lo + o] > mine ? 1 : 0;
+      sm.sorted[lo + rank] = mine;
+      sm.lrank[lo + c] = rank;
+      if (level < depth && rank < k) {
         sm.frontier[rank] = lo + c;
         sm.cand_row[lo + c] = 1 + (level - 1) * k + rank;
       }
     }
     __syncthreads();
+    if (level == depth) break;
     const int lo2 = k + (level - 1) * kk;
     for (int idx = tid; idx < kk; idx += NT) {
       const int s = idx / k, r = idx - s * k;
       const int parent = sm.frontier[s];
       const int row = 1 + (level - 1) * k + s;
       const int g = lo2 + idx;
-      sm.cand_lv[g] = sm.cand_lv[parent] + sm.row_lp[row * k + r];
+      const double lv = sm.cand_lv[parent] + sm.row_lp[row * k + r];
+      sm.cand_lv[g] = lv;
       sm.cand_tok[g] = sm.row_tok[row * k + r];
       sm.cand_par[g] = parent;
+      sm.keys[g] = cand_key(lv, g);
     }
     __syncthreads();
   }
 
-  // 3. rerank: bitonic sort of all candidate keys, best first; keep n.  With
-  //    Ppow <= blockDim each thread holds one key: partners closer than 32 are
-  //    exchanged by shuffles, farther ones through a double-buffered array.
-  if (Ppow <= NT) {
-    uint64_t key = tid < P ? cand_key(sm.cand_lv[tid], tid) : 0ull;
-    int buf = 0;
-    for (int size = 2; size <= Ppow; size <<= 1) {
-      const bool desc = (tid & size) == 0;
-      for (int j = size >> 1; j > 0; j >>= 1) {
-        uint64_t o;
-        if (j >= 32) {
-          uint64_t* xb = sm.sort_k + buf * NT;  // double-buffered exchange array
-          xb[tid] = key;
-          __syncthreads();
-          o = xb[tid ^ j];
-          buf ^= 1;
-        } else {
-          o = __shfl_xor_sync(kFull, key, j);
-        }
-        const bool lower = (tid & j) == 0;
-        key = (lower == desc) ? umax64(key, o) : umin64(key, o);
-      }
+  // 3. rerank: rank among all P = rank in its own level + the larger keys of
+  //    every other level (binary search in that level's descending list);
+  //    with per-level widths, the level's rank against its width
+  for (int g = tid; g < P; g += NT) {
+    const uint64_t x = sm.keys[g];
+    const int own = g < k ? 1 : 2 + (g - k) / kk;
+    int rank = sm.lrank[g];
+    if (lw.on) {
+      sm.node_of[g] = rank < lw.w[own - 1] ? 1 : 0;
+      continue;
     }
-    if (tid < n) sm.node_of[key_gid(key)] = 1;
-  } else {
-    for (int i = tid; i < Ppow; i += NT) sm.sort_k[i] = i < P ? cand_key(sm.cand_lv[i], i) : 0ull;
-    __syncthreads();
-    for (int size = 2; size <= Ppow; size <<= 1) {
-      for (int j = size >> 1; j > 0; j >>= 1) {
-        for (int i = tid; i < Ppow; i += NT) {
-          const int o = i ^ j;
-          if (o > i) {
-            const uint64_t a = sm.sort_k[i], c = sm.sort_k[o];
-            const bool desc = (i & size) == 0;
-            if (desc ? (a < c) : (a > c)) { sm.sort_k[i] = c; sm.sort_k[o] = a; }
-          }
-        }
-        __syncthreads();
+    for (int level = 1; level <= depth && rank < n; ++level) {
+      if (level == own) continue;
+      const int lo = level == 1 ? 0 : k + (level - 2) * kk;
+      int a = 0, z = level == 1 ? k : kk;
+      while (a < z) {  // first position whose key is below x
+        const int mid = (a + z) >> 1;
+        if (sm.sorted[lo + mid] > x) a = mid + 1; else z = mid;
       }
+      rank += a;
     }
-    for (int i = tid; i < n; i += NT) sm.node_of[key_gid(sm.sort_k[i])] = 1;
+    sm.node_of[g] = rank < n ? 1 : 0;
   }
   __syncthreads();
 
@@ -222,20 +211,15 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   }
 }
 
-// Block size of the expansion: the rerank's key count rounded to a power of
-// two (one key per thread; block barriers cost less with fewer warps),
-// between 128 and 1024 threads.
-static int build_threads(int P) {
-  const int p = next_pow2(P);
-  return p < 128 ? 128 : (p > kBuildThreads ? kBuildThreads : p);
-}
+// Block size of the expansion: 128 threads for pools up to 128 candidates,
+// else 256 (the work is in per-level loops; block barriers cost less with
+// fewer warps).
+static int build_threads(int P) { return P <= 128 ? 128 : kBuildThreads; }
 
 size_t tree_build_smem_bytes(int R, int k, int P) {
   const int nt = build_threads(P);
-  const int Ppow = next_pow2(P);
-  const int nsort = Ppow > 2 * nt ? Ppow : 2 * nt;
-  return sizeof(double) * ((size_t)R * k + P) + sizeof(uint64_t) * nsort +
-         sizeof(int) * ((size_t)R * k + 4 * (size_t)P + 32 + nt / 32 + 2 * EAGLE_MAX_NODES);
+  return sizeof(double) * ((size_t)R * k + P) + 2 * sizeof(uint64_t) * P +
+         sizeof(int) * ((size_t)R * k + 5 * (size_t)P + 32 + nt / 32 + 2 * EAGLE_MAX_NODES);
 }
 
 // workspace: [chunk stats][chunk keys][row tokens B*R*k int32][row logits B*R*k float]
@@ -246,21 +230,21 @@ size_t tree_build_ws_bytes(int B, int R, int V, int elem_bytes, int k) {
 }
 
 cudaError_t launch_tree_expand(const int32_t* row_tok, const float* row_val, int B, int R, int depth, int k, int n,
-                               const eagle_tree_t& out, const MaskOut* mo_in, bool pdl, cudaStream_t s) {
+                               const eagle_tree_t& out, const MaskOut* mo_in, bool pdl, cudaStream_t s,
+                               const int* widths) {
   const int P = k + (depth - 1) * k * k;
   const size_t smem = tree_build_smem_bytes(R, k, P);
   const MaskOut mo = mo_in ? *mo_in : MaskOut{nullptr, nullptr, nullptr};
+  LevelWidths lw = {};
+  lw.on = widths != nullptr;
+  for (int l = 0; widths && l < depth; ++l) lw.w[l] = widths[l];
   auto go = [&](auto kernel, int nt) -> cudaError_t {
     cudaError_t e2 = ensure_smem_limit((const void*)kernel, smem);
     if (e2 != cudaSuccess) return e2;
-    return launch_kernel(kernel, dim3(B), dim3(nt), smem, s, pdl, row_tok, row_val, R, depth, k, n, out, mo);
+    return launch_kernel(kernel, dim3(B), dim3(nt), smem, s, pdl, row_tok, row_val, R, depth, k, n, out, mo, lw);
   };
-  switch (build_threads(P)) {
-    case 128: return go(tree_expand_kernel<128>, 128);
-    case 256: return go(tree_expand_kernel<256>, 256);
-    case 512: return go(tree_expand_kernel<512>, 512);
-    default: return go(tree_expand_kernel<kBuildThreads>, kBuildThreads);
-  }
+  if (build_threads(P) == 128) return go(tree_expand_kernel<128>, 128);
+  return go(tree_expand_kernel<kBuildThreads>, kBuildThreads);
 }
 
 cudaError_t launch_tree_build(const void* draft_logits, int dtype, int B, int R, int V, int depth, int k, int n,

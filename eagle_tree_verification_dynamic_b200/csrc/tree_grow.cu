@@ -14,6 +14,11 @@
 //           best candidates: the expected number of tokens those candidates
 //           add (EAGLE-4 write-up, harness: the gain in cumulative
 //           probability that a level brings)
+//   widths  (the harness widening or deepening) a level may be drafted from
+//           the first w frontier slots only: the caller passes w rows per
+//           sequence, the other slots count as rows of -inf (no children);
+//           frontier_logv reads the last level's k best log V in rank order,
+//           and finish_widths keeps the w_l best candidates of each level.
 //
 // The state keeps each row's top-k tokens and logits and its log-sum-exp in
 // the layout the one-shot build uses, plus the frontier's log V, so the tree
@@ -58,7 +63,8 @@ __global__ void __launch_bounds__(kGrowThreads)
 tree_grow_kernel(const int32_t* __restrict__ lvl_tok, const float* __restrict__ lvl_val,
                  const double* __restrict__ lvl_lse, int32_t* __restrict__ row_tok, float* __restrict__ row_val,
                  double* __restrict__ row_lse, double* __restrict__ front_lv, double* __restrict__ gain,
-                 int32_t* __restrict__ front_tok, int32_t* __restrict__ front_par, int R, int k, int level) {
+                 int32_t* __restrict__ front_tok, int32_t* __restrict__ front_par, int R, int k, int level,
+                 int width) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ double s_lv[32 * 32];
@@ -67,17 +73,19 @@ tree_grow_kernel(const int32_t* __restrict__ lvl_tok, const float* __restrict__ 
   __shared__ double s_flv[32];
   __shared__ double s_best[32];
   const int b = blockIdx.x, tid = threadIdx.x;
-  const int nrows = level == 1 ? 1 : k;
+  const int nrows = level == 1 ? 1 : k;      // the level's slots
+  const int nin = level == 1 ? 1 : width;    // rows swept: the first nin slots; the rest have no children
   const int r0 = level == 1 ? 0 : 1 + (level - 2) * k;
   // 1. this level's rows into the per-sequence row arrays
   for (int e = tid; e < nrows * k; e += kGrowThreads) {
     const int rr = e / k, j = e - rr * k;
-    const size_t src = ((size_t)b * nrows + rr) * k + j;
+    const size_t src = ((size_t)b * nin + rr) * k + j;
     const size_t dst = ((size_t)b * R + r0 + rr) * k + j;
-    row_tok[dst] = lvl_tok[src];
-    row_val[dst] = lvl_val[src];
+    row_tok[dst] = rr < nin ? lvl_tok[src] : -1;
+    row_val[dst] = rr < nin ? lvl_val[src] : -INFINITY;
   }
-  for (int rr = tid; rr < nrows; rr += kGrowThreads) row_lse[(size_t)b * R + r0 + rr] = lvl_lse[(size_t)b * nrows + rr];
+  for (int rr = tid; rr < nrows; rr += kGrowThreads)
+    row_lse[(size_t)b * R + r0 + rr] = rr < nin ? lvl_lse[(size_t)b * nin + rr] : -INFINITY;
   // 2. the level's candidates: log V = log V(parent) + (logit - lse), as the one-shot build forms it
   for (int s = tid; s < k; s += kGrowThreads) s_flv[s] = level == 1 ? 0.0 : front_lv[(size_t)b * k + s];
   __syncthreads();
@@ -85,9 +93,9 @@ tree_grow_kernel(const int32_t* __restrict__ lvl_tok, const float* __restrict__ 
   const int gid0 = level == 1 ? 0 : k + (level - 2) * k * k;
   for (int c = tid; c < cnt; c += kGrowThreads) {
     const int s = c / k;
-    const size_t src = ((size_t)b * nrows + s) * k + (c - s * k);
-    const int tok = lvl_tok[src];
-    const double lp = tok >= 0 ? (double)lvl_val[src] - lvl_lse[(size_t)b * nrows + s] : -INFINITY;
+    const size_t src = ((size_t)b * nin + s) * k + (c - s * k);
+    const int tok = s < nin ? lvl_tok[src] : -1;
+    const double lp = tok >= 0 ? (double)lvl_val[src] - lvl_lse[(size_t)b * nin + s] : -INFINITY;
     const double lv = level == 1 ? lp : s_flv[s] + lp;
     s_lv[c] = lv;
     s_tok[c] = tok;
@@ -125,12 +133,13 @@ eagle_status grow_check(int dtype, int B, int V, int depth, int k, void* state, 
   return EAGLE_OK;
 }
 
-// Sweep nrows rows per sequence and file them (and pick the frontier).
-cudaError_t grow_step(const void* logits, int dtype, int B, int V, int depth, int k, int level, void* state,
-                      int32_t* ftok, int32_t* fpar, cudaStream_t s) {
+// Sweep the level's rows (1 at the root, else `width` per sequence) and file
+// them (and pick the frontier).
+cudaError_t grow_step(const void* logits, int dtype, int B, int V, int depth, int k, int level, int width,
+                      void* state, int32_t* ftok, int32_t* fpar, cudaStream_t s) {
   const GrowLayout g = grow_layout(B, V, dtype, depth, k);
   char* st = static_cast<char*>(state);
-  const int nrows = level == 1 ? 1 : k;
+  const int nrows = level == 1 ? 1 : width;
   RowOut ro;
   ro.tok = reinterpret_cast<int32_t*>(st + g.lvl_tok);
   ro.val = reinterpret_cast<float*>(st + g.lvl_val);
@@ -143,7 +152,7 @@ cudaError_t grow_step(const void* logits, int dtype, int B, int V, int depth, in
                        (const double*)ro.lse, reinterpret_cast<int32_t*>(st + g.row_tok),
                        reinterpret_cast<float*>(st + g.row_val), reinterpret_cast<double*>(st + g.row_lse),
                        reinterpret_cast<double*>(st + g.front_lv), reinterpret_cast<double*>(st + g.gain), ftok,
-                       fpar, R, k, level);
+                       fpar, R, k, level, width);
 }
 
 eagle_status cuda_st(cudaError_t e) { return report_cuda(e); }
@@ -167,7 +176,7 @@ EAGLE_API eagle_status eagle_tree_grow_begin(const void* root_logits, int dtype,
   if (!root_logits) return EAGLE_ERR_NULL;
   const eagle_status st = grow_check(dtype, B, V, depth, k, state, state_bytes);
   if (st != EAGLE_OK) return st;
-  return cuda_st(grow_step(root_logits, dtype, B, V, depth, k, 1, state, frontier_tokens, frontier_parents,
+  return cuda_st(grow_step(root_logits, dtype, B, V, depth, k, 1, 1, state, frontier_tokens, frontier_parents,
                            static_cast<cudaStream_t>(stream)));
 }
 
@@ -178,8 +187,30 @@ EAGLE_API eagle_status eagle_tree_grow_level(const void* level_logits, int dtype
   const eagle_status st = grow_check(dtype, B, V, depth, k, state, state_bytes);
   if (st != EAGLE_OK) return st;
   if (level < 2 || level > depth) return EAGLE_ERR_SHAPE;
-  return cuda_st(grow_step(level_logits, dtype, B, V, depth, k, level, state, frontier_tokens, frontier_parents,
+  return cuda_st(grow_step(level_logits, dtype, B, V, depth, k, level, k, state, frontier_tokens, frontier_parents,
                            static_cast<cudaStream_t>(stream)));
+}
+
+EAGLE_API eagle_status eagle_tree_grow_level_width(const void* level_logits, int dtype, int B, int V, int depth,
+                                                   int k, int level, int width, void* state, size_t state_bytes,
+                                                   int32_t* frontier_tokens, int32_t* frontier_parents,
+                                                   void* stream) {
+  if (!level_logits) return EAGLE_ERR_NULL;
+  const eagle_status st = grow_check(dtype, B, V, depth, k, state, state_bytes);
+  if (st != EAGLE_OK) return st;
+  if (level < 2 || level > depth || width < 1 || width > k) return EAGLE_ERR_SHAPE;
+  return cuda_st(grow_step(level_logits, dtype, B, V, depth, k, level, width, state, frontier_tokens,
+                           frontier_parents, static_cast<cudaStream_t>(stream)));
+}
+
+EAGLE_API eagle_status eagle_tree_grow_frontier_logv(int dtype, int B, int V, int depth, int k, void* state,
+                                                     size_t state_bytes, double* logv, void* stream) {
+  if (!logv) return EAGLE_ERR_NULL;
+  const eagle_status st = grow_check(dtype, B, V, depth, k, state, state_bytes);
+  if (st != EAGLE_OK) return st;
+  const GrowLayout g = grow_layout(B, V, dtype, depth, k);
+  return cuda_st(cudaMemcpyAsync(logv, static_cast<char*>(state) + g.front_lv, sizeof(double) * B * k,
+                                 cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
 }
 
 EAGLE_API eagle_status eagle_tree_grow_gains(int dtype, int B, int V, int depth, int k, void* state,
@@ -214,6 +245,35 @@ EAGLE_API eagle_status eagle_tree_grow_finish(int dtype, int B, int V, int depth
   return cuda_st(launch_tree_expand(reinterpret_cast<const int32_t*>(stp + g.row_tok),
                                     reinterpret_cast<const float*>(stp + g.row_val), B, R, levels, k, n, *out,
                                     nullptr, false, s));
+}
+
+EAGLE_API eagle_status eagle_tree_grow_finish_widths(int dtype, int B, int V, int depth, int k, int levels,
+                                                     const int* widths, void* state, size_t state_bytes,
+                                                     const eagle_tree_t* out, int* n_nodes, void* stream) {
+  if (!widths || !out || !out->tokens || !out->parents || !out->depth || !out->logV || !out->draft_row ||
+      !out->row_lse)
+    return EAGLE_ERR_NULL;
+  const eagle_status st = grow_check(dtype, B, V, depth, k, state, state_bytes);
+  if (st != EAGLE_OK) return st;
+  if (levels < 1 || levels > depth) return EAGLE_ERR_SHAPE;
+  int n = 0;
+  for (int l = 0; l < levels; ++l) {
+    // level 1 has k candidates; a deeper level's come from the w_{l-1} nodes chosen above it
+    const int avail = l == 0 ? k : widths[l - 1] * k;
+    if (widths[l] < 1 || widths[l] > k || widths[l] > avail) return EAGLE_ERR_SHAPE;
+    n += widths[l];
+  }
+  if (n > EAGLE_MAX_NODES) return EAGLE_ERR_LIMIT;
+  if (n_nodes) *n_nodes = n;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const GrowLayout g = grow_layout(B, V, dtype, depth, k);
+  char* stp = static_cast<char*>(state);
+  const int R = 1 + (depth - 1) * k;
+  cudaError_t e = cudaMemcpyAsync(out->row_lse, stp + g.row_lse, sizeof(double) * B * R, cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return cuda_st(e);
+  return cuda_st(launch_tree_expand(reinterpret_cast<const int32_t*>(stp + g.row_tok),
+                                    reinterpret_cast<const float*>(stp + g.row_val), B, R, levels, k, n, *out,
+                                    nullptr, false, s, widths));
 }
 
 }  // extern "C"

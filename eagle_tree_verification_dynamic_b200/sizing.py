@@ -57,6 +57,18 @@ class CostTable:
                  "eagle_size_keep_level")
         return bool(keep.value), float(ratio.value)
 
+    def level_width(self, B: float, L_: float, n_before: int, logv, threshold: float) -> Tuple[int, np.ndarray]:
+        """Width of a level (eagle_size_level_width): logv [nb][k] each sequence's k best log V, descending."""
+        lv = np.ascontiguousarray(np.asarray(logv, dtype=np.float64))
+        nb, k = lv.shape
+        width = ctypes.c_int(0)
+        ratios = np.zeros(k, dtype=np.float64)
+        L._check(L.lib().eagle_size_level_width(ctypes.byref(self.struct()), B, L_, int(n_before),
+                                                    ctypes.c_void_p(lv.ctypes.data), k, nb, threshold,
+                                                    ctypes.byref(width), ctypes.c_void_p(ratios.ctypes.data)),
+                 "eagle_size_level_width")
+        return int(width.value), ratios
+
     def to_json(self, path: str, **meta):
         with open(path, "w") as f:
             json.dump({"B": self.B.tolist(), "L": self.L.tolist(), "N": self.N.tolist(), "us": self.us.tolist(),
@@ -114,3 +126,38 @@ def grow_sized(grower: L.TreeGrower, root_logits: torch.Tensor,
         return SizedTree(None, 0, drafted, ratios)
     m = min(k * kept, L.MAX_NODES)
     return SizedTree(grower.finish(m, levels=drafted), kept, drafted, ratios)
+
+
+@dataclass
+class WidthTree:
+    tree: Optional[L.Tree]     # None when not even the first candidate was worth verifying
+    widths: list               # candidates kept per level (each level drafted from the previous width)
+    ratios: list               # per level drafted: each examined candidate's gain / marginal cost
+
+
+def grow_widths(grower: L.TreeGrower, root_logits: torch.Tensor,
+                draft_fn: Callable[[int, torch.Tensor, torch.Tensor, int], torch.Tensor], table: CostTable,
+                context_len: float, threshold: float) -> WidthTree:
+    """Widen or deepen while each candidate pays for itself.
+
+    After each level the level's k best log V per sequence are read back (one small device-to-host copy)
+    and the library chooses the level's width; the next level is drafted from that many frontier slots:
+    draft_fn(level, frontier_tokens [B][k], frontier_parents [B][k], width) -> rows [B][width][V] (the draft
+    model runs on the chosen nodes only).  Drafting stops at a width of 0 or at the grower's depth; the
+    tree keeps each level's chosen candidates (at most MAX_NODES in all)."""
+    B = grower.B
+    tok, par = grower.begin(root_logits)
+    widths, ratios, n = [], [], 0
+    for level in range(1, grower.depth + 1):
+        if level > 1:
+            tok, par = grower.level_width(draft_fn(level, tok, par, widths[-1]), level, widths[-1])
+        w, r = table.level_width(B, context_len, n, grower.frontier_logv().cpu().numpy(), threshold)
+        ratios.append(r)
+        w = min(w, L.MAX_NODES - n)
+        if w == 0:
+            break
+        widths.append(w)
+        n += w
+    if not widths:
+        return WidthTree(None, [], ratios)
+    return WidthTree(grower.finish_widths(widths), widths, ratios)

@@ -321,6 +321,32 @@ EAGLE_API eagle_status eagle_tree_grow_gains(int dtype, int B, int V, int depth,
 EAGLE_API eagle_status eagle_tree_grow_finish(int dtype, int B, int V, int depth, int k, int levels, int m,
                                               void* state, size_t state_bytes, const eagle_tree_t* out,
                                               int* n_nodes, void* stream);
+/* Widening or deepening (EAGLE-4 write-up, same section as the sizing below:
+ * the harness widens or deepens the tree while gain over marginal cost stays
+ * above a threshold, with no fixed top-k):
+ *   eagle_tree_grow_level_width: as eagle_tree_grow_level, but the level is
+ *     drafted from the first `width` frontier slots only (1 <= width <= k):
+ *     level_logits is [B][width][V]; the other slots count as rows of -inf,
+ *     whose candidates have V = 0 (token -1) and are never chosen.
+ *   eagle_tree_grow_frontier_logv (logv [B][k] double, device): after begin
+ *     or a level, each sequence's k best candidates of that level, log V in
+ *     rank order (-inf for a candidate of V = 0); the input of
+ *     eagle_size_level_width.
+ *   eagle_tree_grow_finish_widths (widths HOST [levels]): the tree keeping
+ *     the widths[l-1] best candidates of each level l, n = their sum nodes,
+ *     numbered by ascending candidate id; requires 1 <= widths[0] <= k and
+ *     1 <= widths[l] <= min(k, widths[l-1] k), level l + 1 having been drafted
+ *     from widths[l-1] slots.  Errors: EAGLE_ERR_SHAPE for widths outside
+ *     those bounds, EAGLE_ERR_LIMIT for n > EAGLE_MAX_NODES. */
+EAGLE_API eagle_status eagle_tree_grow_level_width(const void* level_logits, int dtype, int B, int V, int depth,
+                                                   int k, int level, int width, void* state, size_t state_bytes,
+                                                   int32_t* frontier_tokens, int32_t* frontier_parents,
+                                                   void* stream);
+EAGLE_API eagle_status eagle_tree_grow_frontier_logv(int dtype, int B, int V, int depth, int k, void* state,
+                                                     size_t state_bytes, double* logv, void* stream);
+EAGLE_API eagle_status eagle_tree_grow_finish_widths(int dtype, int B, int V, int depth, int k, int levels,
+                                                     const int* widths, void* state, size_t state_bytes,
+                                                     const eagle_tree_t* out, int* n_nodes, void* stream);
 
 /* ------------------------------------------------- cost-aware tree sizing
  * EAGLE-4 write-up, "Деревья проверки EAGLE-4 и утилита управления": a table
@@ -353,6 +379,20 @@ EAGLE_API double eagle_cost_at(const eagle_cost_table_t* table, double B, double
 EAGLE_API eagle_status eagle_size_keep_level(const eagle_cost_table_t* table, double B, double L, int k, int level,
                                              const double* gains, int nb, double threshold, int* keep,
                                              double* ratio);
+/* eagle_size_level_width: the width of one level when the harness widens or
+ * deepens.  logv: HOST [nb][k], each sequence's k best candidates of the
+ * level, log V in descending order (eagle_tree_grow_frontier_logv);
+ * n_before: candidates per sequence chosen at the earlier levels.  The j-th
+ * best of every sequence is taken together, in order: gain = sum over the
+ * batch of its V = exp(log V), marginal cost C(B, L, n_before + j) -
+ * C(B, L, n_before + j - 1); taken while gain > 0 and gain / cost >=
+ * threshold (infinite when the cost does not grow); the first that fails ends
+ * the level.  *width = the number taken (0: stop drafting).  ratios (HOST [k]
+ * or NULL): each examined candidate's ratio, NaN past the first failure.
+ * Errors: EAGLE_ERR_NULL, EAGLE_ERR_SHAPE. */
+EAGLE_API eagle_status eagle_size_level_width(const eagle_cost_table_t* table, double B, double L, int n_before,
+                                              const double* logv, int k, int nb, double threshold, int* width,
+                                              double* ratios);
 
 /* -------------------------------------------------------- static tree
  * EAGLE-1's fixed draft tree ("EAGLE" notes, "1. EAGLE pipeline / Draft

@@ -48,4 +48,4 @@ from .attention import tree_attention, tree_attention_rows  # noqa: F401
 from .accept import accept_greedy, accept_stochastic, inverse_cdf, inverse_cdf_band  # noqa: F401
 from .kv import compact_kv  # noqa: F401
 from .paged import compact_kv_paged, gather_pages  # noqa: F401
-from .sizing import cost_at, keep_level, level_ratio, levels_kept  # noqa: F401
+from .sizing import cost_at, keep_level, level_ratio, level_width, levels_kept  # noqa: F401

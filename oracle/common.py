@@ -24,6 +24,8 @@ def logsumexp(row: np.ndarray) -> float:
     """log sum_i exp(row_i) in fp64, shifted by the maximum."""
     row = np.asarray(row, dtype=np.float64)
     mx = row.max()
+    if mx == -np.inf:  # every term is exp(-inf) = 0: log 0
+        return -np.inf
     return float(mx + np.log(np.exp(row - mx).sum()))
 
 

@@ -24,6 +24,20 @@ Readings the pages leave open, taken here:
     With no level kept there is nothing to verify.
   * For a batch of mixed context lengths the caller passes one L (e.g. the
     mean).
+  * Widening or deepening (the same passage: the harness "widens or deepens
+    the tree while the ratio stays above the threshold", giving a wide, deep
+    tree at batch 1 and a narrow tree or a chain at large batch, with no fixed
+    top-k): at level l the level's candidates are taken one at a time in
+    descending V, the j-th best of every sequence together.  With N
+    candidates per sequence already chosen, the j-th adds the batch gain
+    sum_b V_b,(j) at the marginal cost C(B, L, N + 1) - C(B, L, N); it is taken
+    while its gain is positive and gain / cost >= threshold (a cost that does
+    not grow always passes), and the first one that fails ends the level.  The
+    level's width w_l is the number taken; w_l = 0 stops drafting.  The next
+    level is drafted from the w_l chosen nodes only, and the tree verifies,
+    level by level, the w_l best of each level (closed under "parent of",
+    since each level's candidates are children of the previous level's
+    chosen nodes).
 """
 from __future__ import annotations
 
@@ -81,3 +95,23 @@ def levels_kept(table, B: float, L: float, k: int, gains_by_level: Sequence[Sequ
             break
         kept = level
     return kept
+
+
+def level_width(table, B: float, L: float, n_before: int, values_by_seq: Sequence[Sequence[float]],
+                threshold: float):
+    """(width, ratios): how many of a level's candidates to verify.  values_by_seq[b] holds sequence b's
+    candidate values V of this level in descending order (one list per sequence, equal lengths);
+    n_before = candidates per sequence chosen at earlier levels.  ratios[j] is the j-th candidate's batch
+    gain over its marginal cost, for the candidates examined."""
+    Bs, Ls, Ns, us = table
+    vals = np.asarray(values_by_seq, dtype=np.float64)
+    width, ratios = 0, []
+    for j in range(vals.shape[1]):
+        g = float(np.sum(vals[:, j]))
+        dc = cost_at(Bs, Ls, Ns, us, B, L, n_before + j + 1) - cost_at(Bs, Ls, Ns, us, B, L, n_before + j)
+        r = np.inf if dc <= 0.0 else g / dc
+        ratios.append(r)
+        if not (g > 0.0 and r >= threshold):
+            break
+        width = j + 1
+    return width, ratios

@@ -27,6 +27,13 @@ Readings the pages leave open, taken here:
     lower token id (the same order as by log-confidence).
   * Output nodes are numbered 1..n in ascending gid (parents before children,
     siblings in rank order); parent 0 is the root.
+  * A logit of -inf has confidence 0 and is no child: a row with fewer than k
+    finite logits fills its remaining children with token -1 and log V = -inf
+    (a row of -inf marks a frontier node the caller chose not to draft from).
+  * With per-level widths (the cost-aware harness's widening, see
+    oracle.sizing): instead of the best m over all levels, the tree keeps the
+    w_l best candidates of each level l (by the same ordering), for the levels
+    given.
 """
 from __future__ import annotations
 
@@ -38,9 +45,10 @@ from .common import logsumexp, near_tie
 
 
 def _row_topk(row: np.ndarray, k: int) -> np.ndarray:
-    """Token ids of the k largest values, ties to the lower id (library sort)."""
-    order = np.lexsort((np.arange(row.shape[0]), -row))
-    return order[:k]
+    """Token ids of the k largest values, ties to the lower id (library sort);
+    -1 in place of a logit of -inf."""
+    order = np.lexsort((np.arange(row.shape[0]), -row))[:k]
+    return np.where(np.isneginf(row[order]), -1, order)
 
 
 def _sort_key(c):
@@ -83,11 +91,12 @@ def _apply_flips(ranked, kind: str, level: int, flip) -> list:
     return ranked
 
 
-def build_tree(logits: np.ndarray, depth: int, k: int, m: int, flip=()) -> Dict:
+def build_tree(logits: np.ndarray, depth: int, k: int, m: int, flip=(), widths=None) -> Dict:
     """Build one sequence's tree from its R = 1 + (depth-1)*k draft rows (fp64).
 
     `flip`: near-tie records (as returned in "near_ties") to resolve the other
-    way; empty for the plain build."""
+    way; empty for the plain build.  `widths`: per-level widths w_1.. (at most
+    depth of them) to keep the w_l best of each level instead of the best m."""
     logits = np.asarray(logits, dtype=np.float64)
     R, V = logits.shape
     assert depth >= 1 and 1 <= k <= V and m >= 1
@@ -101,7 +110,7 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int, flip=()) -> Dict:
 
     def make(row, r, gid, level, parent):
         tok = int(topk[row][r])
-        lp = logits[row, tok] - row_lse[row]          # log confidence, <= 0
+        lp = logits[row, tok] - row_lse[row] if tok >= 0 else -np.inf  # log confidence, <= 0
         base = 0.0 if parent is None else parent["logV"]
         return {"gid": gid, "level": level, "token": tok, "logit": logits[row, tok],
                 "lp": lp, "logV": base + lp, "parent": None if parent is None else parent["gid"],
@@ -112,11 +121,13 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int, flip=()) -> Dict:
     all_cands += level_cands
     frontiers: List[dict] = []    # per expanded level: the k tokens by slot and their parents' slots
     gains: List[float] = []       # per level: sum of V over its k best candidates
+    level_logv: List[np.ndarray] = []  # per level: log V of its k best candidates, in rank order
     for level in range(2, depth + 1):
         ranked = _apply_flips(sorted(level_cands, key=_sort_key), "frontier", level - 1, flip)
         _flag_adjacent(ranked, k, "frontier", level - 1, near_ties)
         frontier = ranked[:k]
         gains.append(float(sum(np.exp(c["logV"]) for c in frontier)))
+        level_logv.append(np.array([c["logV"] for c in frontier]))
         frontiers.append({"tokens": np.array([c["token"] for c in frontier], dtype=np.int64),
                           "parent_slot": np.array([-1 if c["pnode"] is None else c["pnode"]["slot"]
                                                    for c in frontier], dtype=np.int64)})
@@ -130,13 +141,28 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int, flip=()) -> Dict:
         level_cands = nxt
         all_cands += level_cands
 
-    gains.append(float(sum(np.exp(c["logV"]) for c in sorted(level_cands, key=_sort_key)[:k])))
+    last = sorted(level_cands, key=_sort_key)[:k]
+    gains.append(float(sum(np.exp(c["logV"]) for c in last)))
+    level_logv.append(np.array([c["logV"] for c in last]))
     P = len(all_cands)
     assert P == k + (depth - 1) * k * k
-    n = min(m, P)
-    ranked = _apply_flips(sorted(all_cands, key=_sort_key), "rerank", 0, flip)
-    _flag_adjacent(ranked[n - 1:], 1, "rerank", 0, near_ties)
-    kept = sorted(ranked[:n], key=lambda c: c["gid"])
+    if widths is None:
+        n = min(m, P)
+        ranked = _apply_flips(sorted(all_cands, key=_sort_key), "rerank", 0, flip)
+        _flag_adjacent(ranked[n - 1:], 1, "rerank", 0, near_ties)
+        kept = sorted(ranked[:n], key=lambda c: c["gid"])
+    else:
+        assert 1 <= len(widths) <= depth
+        chosen = []
+        for level, w in enumerate(widths, start=1):
+            ranked = _apply_flips(sorted([c for c in all_cands if c["level"] == level], key=_sort_key), "width",
+                                  level, flip)
+            assert 0 <= w <= len(ranked)
+            if 0 < w < len(ranked):
+                _flag_adjacent(ranked[w - 1:], 1, "width", level, near_ties)
+            chosen += ranked[:w]
+        kept = sorted(chosen, key=lambda c: c["gid"])
+        n = len(kept)
     node_of = {c["gid"]: i + 1 for i, c in enumerate(kept)}
 
     tokens = np.array([c["token"] for c in kept], dtype=np.int64)
@@ -151,7 +177,7 @@ def build_tree(logits: np.ndarray, depth: int, k: int, m: int, flip=()) -> Dict:
         draft_row[i + 1] = c["row"]
     return {"tokens": tokens, "parents": parents, "depth": depth_arr, "logV": logV,
             "gid": gid, "draft_row": draft_row, "row_lse": row_lse, "n": n, "P": P,
-            "frontiers": frontiers, "gains": np.array(gains), "near_ties": near_ties}
+            "frontiers": frontiers, "gains": np.array(gains), "level_logv": level_logv, "near_ties": near_ties}
 
 
 def build_trees(logits_b: np.ndarray, depth: int, k: int, m: int) -> List[Dict]:
