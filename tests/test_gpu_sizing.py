@@ -77,3 +77,43 @@ def test_sized_growth_matches_the_oracle(name, threshold):
         excused += tree_match(got, ref, lambda fl, b=b: oracle.build_tree(x64[b][:R], drafted, k, m, flip=fl))[0]
         np.testing.assert_allclose(got["row_lse"], ref["row_lse"], rtol=0, atol=5e-7)
     assert excused <= 1, (name, threshold)
+
+
+@pytest.mark.parametrize("B,threshold", [(1, 0.5), (32, 0.5), (8, 0.3), (32, 0.05)])
+def test_widening_harness_matches_the_oracle(B, threshold):
+    """grow_widths (the library's width decision between draft levels, each level drafted from the chosen
+    nodes only) against the same harness on the oracle: the widths level by level and the tree of the
+    chosen candidates.  At batch 1 on the saturating table every level keeps its full width; at batch 32
+    with threshold 0.5 the tree is a chain."""
+    from eagle_tree_verification_dynamic_b200.sizing import grow_widths
+    from sizing_helpers import _masked, confident_draft, oracle_grow_widths, saturating_table
+
+    cfg, stored = confident_draft()
+    stored = stored[:B]
+    x64 = oracle.decode_logits(stored, "f32")
+    table = CostTable(*saturating_table())
+    xd = torch.from_numpy(stored).cuda()
+    g = et.TreeGrower(B, cfg.V, cfg.depth, cfg.k, torch.float32, "cuda")
+
+    def draft_fn(level, tok, par, width):  # the rows the draft model gives the chosen frontier slots
+        r0 = 1 + (level - 2) * cfg.k
+        return xd[:, r0:r0 + width].contiguous()
+
+    res = grow_widths(g, xd[:, 0].contiguous(), draft_fn, table, 2048, threshold)
+    torch.cuda.synchronize()
+    want_w, trees = oracle_grow_widths(list(x64), cfg.depth, cfg.k, (table.B, table.L, table.N, table.us), 2048,
+                                       threshold)
+    assert res.widths == want_w
+    if B == 1:
+        assert want_w == [cfg.k] * cfg.depth
+    if B == 32 and threshold == 0.5:
+        assert want_w == [1] * cfg.depth
+    R = 1 + (len(want_w) - 1) * cfg.k
+    excused = 0
+    for b in range(B):
+        rows = _masked(x64[b][:R], cfg.k, want_w)
+        e, ref = tree_match(tree_of(res.tree, b), trees[b],
+                            lambda fl, rows=rows: oracle.build_tree(rows, len(want_w), cfg.k, 1, widths=want_w,
+                                                                    flip=fl))
+        excused += e
+    assert excused <= 1

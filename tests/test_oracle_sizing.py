@@ -17,6 +17,7 @@ import pytest
 from scipy.special import softmax
 
 import oracle
+from sizing_helpers import confident_draft, oracle_grow_widths, saturating_table
 from workloads import gen_draft_logits, get_config
 
 
@@ -95,3 +96,39 @@ def test_larger_batches_keep_fewer_levels():
         kept.append(oracle.levels_kept(table, B, 2048, cfg.k, gl, 0.5))
     assert kept[0] == cfg.depth and kept[-1] < kept[0]
     assert all(a >= b for a, b in zip(kept, kept[1:])), kept
+
+
+# ------------------------------------------------------- widening or deepening
+def test_level_width_handworked():
+    # cost 10 + 2N: every candidate costs 2 per step at any B, L
+    table = ([1, 2], [100, 200], [0, 100], np.array([[[10.0, 210.0]] * 2] * 2))
+    vals = [[0.9, 0.5, 0.2, 0.0], [0.7, 0.3, 0.1, 0.0]]   # batch gains 1.6, 0.8, 0.3, 0 -> ratios .8, .4, .15, 0
+    assert oracle.level_width(table, 2, 150, 0, vals, 0.1)[0] == 3
+    assert oracle.level_width(table, 2, 150, 0, vals, 0.4)[0] == 2
+    assert oracle.level_width(table, 2, 150, 0, vals, 0.5)[0] == 1
+    assert oracle.level_width(table, 2, 150, 0, vals, 0.9)[0] == 0
+    assert oracle.level_width(table, 2, 150, 0, vals, 0.0)[0] == 3       # a candidate of V = 0 is never taken
+    w, r = oracle.level_width(table, 2, 150, 5, vals, 0.1)
+    np.testing.assert_allclose(r[:3], [0.8, 0.4, 0.15])
+
+
+def test_level_width_flat_cost_takes_every_positive_candidate():
+    # every candidate count on the grid: the cost difference is exactly 0 (an infinite ratio)
+    table = ([1, 64], [128, 65536], list(range(40)), np.full((2, 2, 40), 40.0))
+    assert oracle.level_width(table, 1, 128, 17, [[0.3, 1e-9, 1e-30, 0.0]], 1e6)[0] == 3
+
+
+def test_batch_one_grows_wide_and_deep_large_batch_a_chain():
+    """The harness's two ends: at batch 1 the cost does not grow with the tree, so every level keeps its
+    full width; at batch 32 each further candidate costs 0.5 * 32 per step, which only each level's best
+    candidate pays for (a chain)."""
+    cfg, stored = confident_draft()
+    x = oracle.decode_logits(stored, "f32")
+    table = saturating_table()
+    w1, t1 = oracle_grow_widths([x[0]], cfg.depth, cfg.k, table, 2048, 0.5)
+    assert w1 == [cfg.k] * cfg.depth
+    assert t1[0]["n"] == cfg.k * cfg.depth
+    w32, t32 = oracle_grow_widths(list(x), cfg.depth, cfg.k, table, 2048, 0.5)
+    assert w32 == [1] * cfg.depth, w32
+    for t in t32:  # a chain: node i's parent is node i - 1
+        assert t["parents"].tolist() == list(range(len(w32)))

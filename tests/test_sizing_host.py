@@ -110,3 +110,29 @@ def test_the_shipped_b200_table():
     assert np.all(t.us[:, :, 0] == 0.0) and np.all(t.us[:, :, 1:] > 0.0)
     # verification grows with the batch's work: the largest grid point costs the most
     assert t.us[-1, -1, -1] == t.us.max()
+
+
+def test_level_widths_match_the_oracle():
+    rng = np.random.default_rng(5)
+    checked = 0
+    for _ in range(300):
+        t = _random_table(rng)
+        B, L, k = int(rng.integers(1, 33)), float(rng.uniform(100, 30000)), int(rng.integers(1, 11))
+        n_before = int(rng.integers(0, 40))
+        v = np.sort(rng.uniform(0, 1, size=(B, k)) ** 3, axis=1)[:, ::-1]
+        v[:, k - int(rng.integers(0, k)):] = 0.0 if rng.random() < 0.3 else v[:, k - 1:k].min()
+        with np.errstate(divide="ignore"):
+            logv = np.log(v)  # -inf for V = 0
+        thr = float(rng.uniform(0, 0.05))
+        w, ratios = t.level_width(B, L, n_before, logv, thr)
+        want_w, want_r = oracle.level_width((t.B, t.L, t.N, t.us), B, L, n_before, np.exp(logv), thr)
+        near = any(abs(r - thr) <= 1e-9 * max(1.0, abs(thr)) for r in want_r if np.isfinite(r))
+        if not near:
+            assert w == want_w
+            checked += 1
+        for j, r in enumerate(want_r):
+            if np.isinf(r):
+                assert np.isinf(ratios[j])
+            else:
+                assert ratios[j] == pytest.approx(r, rel=1e-12, abs=1e-300)
+    assert checked > 250
