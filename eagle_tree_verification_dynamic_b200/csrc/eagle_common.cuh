@@ -144,10 +144,17 @@ __device__ __forceinline__ float exp2_scaled(float x, float e_ref) {
   return ex2_ftz(z);
 }
 
-// acc * 2^(from - to) for integer-valued from <= to (exact).
+// acc * 2^(from - to) for integer-valued from <= to (exact; the same rounding
+// as ldexp when the result is subnormal).  For d = from - to >= -1022 the
+// power of two is assembled from its exponent bits (d + 1.5 * 2^23 holds the
+// integer d in its low mantissa bits); below that ldexp handles it.
 __device__ __forceinline__ double rescale_pow2(double acc, float from, float to) {
-  const float d = fmaxf(from - to, -1100.0f);
-  return ldexp(acc, (int)d);
+  const float d = from - to;
+  if (d >= -1022.0f) {
+    const int di = __float_as_int(d + 12582912.0f) - 0x4B400000;
+    return acc * __longlong_as_double((long long)(1023 + di) << 52);
+  }
+  return ldexp(acc, (int)fmaxf(d, -1100.0f));
 }
 
 // Merge (e_ref, acc) pairs; returns the natural-log total (fp64).

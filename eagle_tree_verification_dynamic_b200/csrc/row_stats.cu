@@ -267,23 +267,19 @@ row_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k, ChunkSt
 }
 
 // ------------------------------------------------------ chunked TMA sweep
-constexpr int kSwConsumerWarps = 8;
-constexpr int kSwConsumers = kSwConsumerWarps * 32;
-constexpr int kSwThreads = kSwConsumers + 32;  // + one producer warp
-constexpr int kSwChunkBytes = 16384;           // one ring stage = one chunk
-constexpr int kSwStages = 4;
-constexpr int kSwCtasPerSm = 3;
+constexpr int kSwWarps = 8;                 // warps per CTA, each streaming its own chunks
+constexpr int kSwThreads = kSwWarps * 32;
+constexpr int kSwChunkBytes = 4096;         // one chunk = one warp step: 8 16-byte vectors per lane
+constexpr int kSwVecPerLane = kSwChunkBytes / 16 / 32;
+constexpr int kSwStages = 3;                // each warp's private ring
+constexpr int kSwCtasPerSm = 2;
+constexpr int kSwMinChunksPerWarp = 4;      // fewer, longer warp ranges: fewer top-k segments per row
 
 struct SwShared {
-  uint64_t full[kSwStages];
-  uint64_t empty[kSwStages];
-  uint64_t keys[kSwConsumerWarps][32];
-  float e[2][kSwConsumerWarps];  // per-chunk warp partials, double-buffered by chunk parity
-  double s[2][kSwConsumerWarps];
+  uint64_t full[kSwWarps][kSwStages];
   int abort;
-  int last;
 };
-constexpr size_t kSwSmemBytes = (size_t)kSwStages * kSwChunkBytes + sizeof(SwShared);
+constexpr size_t kSwSmemBytes = (size_t)kSwWarps * kSwStages * kSwChunkBytes + sizeof(SwShared);
 
 struct SweepArgs {
   const unsigned char* x;  // row r starts at x + r * row_bytes (16-byte aligned)
@@ -296,21 +292,20 @@ struct SweepArgs {
   RowOut out;
 };
 
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSwConsumers) : "memory"); }
-
-// Largest key strictly below `last` among this consumer thread's elements of
-// the chunks [c0, c1] of a row (the main sweep's element assignment; -inf and
-// NaN never qualify), read from global memory.
+// Largest key strictly below `last` among this lane's elements of the chunks
+// [c0, c1] of a row (the main sweep's element assignment; -inf and NaN never
+// qualify), read from global memory.
 template <typename T>
 __device__ uint64_t seg_next_below(const SweepArgs& a, long long row, int c0, int c1, uint64_t last) {
   constexpr int N = Elem<T>::kPerVec;
+  const int lane = threadIdx.x & 31;
   uint64_t best = 0;
   const unsigned char* rp = a.x + (size_t)row * a.row_bytes;
   for (int c = c0; c <= c1; ++c) {
     const int off = c * kSwChunkBytes;
     const int nvec = min(kSwChunkBytes, a.row_bytes - off) / 16;
     const uint4* vp = reinterpret_cast<const uint4*>(rp + off);
-    for (int v = threadIdx.x; v < nvec; v += kSwConsumers) {
+    for (int v = lane; v < nvec; v += 32) {
       float f[N];
       Elem<T>::unpack(__ldg(vp + v), f);
 #pragma unroll
@@ -324,64 +319,59 @@ __device__ uint64_t seg_next_below(const SweepArgs& a, long long row, int c0, in
   return best;
 }
 
+// Every warp works alone: its contiguous range of the chunk list streams
+// through a private three-stage ring (lane 0 issues the bulk copies), each
+// chunk's log-sum-exp partial is a warp reduction written by lane 0, and at
+// the end of each row segment the warp writes the segment's top-k and takes
+// the row's ticket; the warp completing a row merges it.  No block barrier.
 template <typename T, int M>
 __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(SweepArgs a) {
   using namespace sm100;
   constexpr int N = Elem<T>::kPerVec;
   constexpr int S = kSwStages;
   extern __shared__ __align__(1024) unsigned char sw_smem[];
-  SwShared& sh = *reinterpret_cast<SwShared*>(sw_smem + (size_t)S * kSwChunkBytes);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long C = gridDim.x;
-  const long long g0 = (long long)blockIdx.x * a.nchunks / C;
-  const long long g1 = (long long)(blockIdx.x + 1) * a.nchunks / C;
+  SwShared& sh = *reinterpret_cast<SwShared*>(sw_smem + (size_t)kSwWarps * S * kSwChunkBytes);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long W = (long long)gridDim.x * kSwWarps;
+  const long long gw = (long long)blockIdx.x * kSwWarps + warp;
+  const long long g0 = gw * a.nchunks / W, g1 = (gw + 1) * a.nchunks / W;
   const int nj = (int)(g1 - g0);
+  const uint32_t ring = smem_u32(sw_smem + (size_t)warp * S * kSwChunkBytes);
+  const unsigned char* ringp = sw_smem + (size_t)warp * S * kSwChunkBytes;
   volatile int* abort = &sh.abort;
-  const uint32_t ring = smem_u32(sw_smem);
-  if (tid == 0) {
-    for (int i = 0; i < S; ++i) {
-      mbar_init(smem_u32(&sh.full[i]), 1);
-      mbar_init(smem_u32(&sh.empty[i]), kSwConsumerWarps);
-    }
-    sh.abort = 0;
+  if (threadIdx.x == 0) sh.abort = 0;
+  if (lane == 0) {
+    for (int i = 0; i < S; ++i) mbar_init(smem_u32(&sh.full[warp][i]), 1);
     fence_mbar_init();
   }
   __syncthreads();
   griddep_wait();  // the logits (and this workspace) may belong to the previous kernel
 
-  if (warp == kSwConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int j = 0;
-      for (; j < nj; ++j) {
-        const int st = j % S;
-        if (j >= S && !mbar_wait(smem_u32(&sh.empty[st]), ((j / S) - 1) & 1, abort)) break;
-        if (*abort) break;
-        const long long g = g0 + j;
-        const long long row = g / a.ncpr;
-        const int off = (int)(g - row * a.ncpr) * kSwChunkBytes;
-        const int bytes = min(kSwChunkBytes, a.row_bytes - off);
-        const uint32_t fb = smem_u32(&sh.full[st]);
-        mbar_arrive_expect_tx(fb, (uint32_t)bytes);
-        bulk_load(ring + st * kSwChunkBytes, a.x + (size_t)row * a.row_bytes + off, (uint32_t)bytes, fb);
-      }
-      // every copy issued lands before the CTA may exit
-      for (int d = (j > S ? j - S : 0); d < j; ++d) mbar_wait_drain(smem_u32(&sh.full[d % S]), (d / S) & 1, 200000000ull);
-      if (*abort) atomicExch(a.status, 1);
-    }
-    griddep_launch_dependents();
-    return;
-  }
+  // chunk j of this warp: row and chunk-of-row, advanced without divisions
+  long long row = g0 / a.ncpr;
+  int c = (int)(g0 - row * a.ncpr);
+  int issued = 0;
+  long long irow = row;
+  int ic = c;
+  auto issue_next = [&]() {  // lane 0
+    const int off = ic * kSwChunkBytes;
+    const int bytes = min(kSwChunkBytes, a.row_bytes - off);
+    const int st = issued % S;
+    const uint32_t fb = smem_u32(&sh.full[warp][st]);
+    mbar_arrive_expect_tx(fb, (uint32_t)bytes);
+    bulk_load(ring + st * kSwChunkBytes, a.x + (size_t)irow * a.row_bytes + off, (uint32_t)bytes, fb);
+    ++issued;
+    if (++ic == a.ncpr) { ic = 0; ++irow; }
+  };
+  if (lane == 0)
+    while (issued < nj && issued < S) issue_next();
 
-  // -------------------------------------------------------------- consumers
   LaneTop<M> top;
   top.init();
-  float e_ref = -INFINITY;
-  double acc = 0.0;
-  long long seg_row = -1;
-  int seg_c0 = 0;
+  long long seg_row = row;
+  int seg_c0 = c;
 
-  // end of a row segment [seg_c0, c_last] of row seg_row: its top-k into the
+  // end of the segment [seg_c0, c_last] of row seg_row: its top-k into the
   // last chunk's slot (zeros into the others), then the row's ticket
   auto finish_segment = [&](int c_last) {
     const int k = a.k;
@@ -412,85 +402,73 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
         last = nxt;
       }
     }
-    if (lane < k) sh.keys[warp][lane] = list;
-    consumer_sync();
-    for (int step = 1; step < kSwConsumerWarps; step <<= 1) {  // pairwise merges: 3 rounds
-      if ((warp & (2 * step - 1)) == 0 && warp + step < kSwConsumerWarps) {
-        const uint64_t m = warp_merge_desc(lane < k ? sh.keys[warp][lane] : 0ull,
-                                           lane < k ? sh.keys[warp + step][lane] : 0ull);
-        if (lane < k) sh.keys[warp][lane] = m;
-      }
-      consumer_sync();
-    }
     const size_t slot0 = (size_t)seg_row * a.ncpr;
-    if (warp == 0 && lane < k) a.keys[(slot0 + c_last) * k + lane] = sh.keys[0][lane];
-    for (int e = tid; e < (c_last - seg_c0) * k; e += kSwConsumers) a.keys[(slot0 + seg_c0) * k + e] = 0ull;
+    if (lane < k) a.keys[(slot0 + c_last) * k + lane] = list;
+    for (int e = lane; e < (c_last - seg_c0) * k; e += 32) a.keys[(slot0 + seg_c0) * k + e] = 0ull;
     __threadfence();
-    consumer_sync();
-    if (tid == 0) {
+    __syncwarp();
+    int last_one = 0;
+    if (lane == 0) {
       const int nseg = c_last - seg_c0 + 1;
-      sh.last = atomicAdd(a.tickets + seg_row, nseg) + nseg == a.ncpr;
+      last_one = atomicAdd(a.tickets + seg_row, nseg) + nseg == a.ncpr;
     }
-    consumer_sync();
-    if (sh.last && warp == 0) {
-      // ---- this CTA completed the row: merge all of its chunks (fixed order)
-      __threadfence();
-      const ChunkStat* st = a.stats + slot0;
-      const uint64_t* kk = a.keys + slot0 * k;
-      double lse = 0.0;
-      LseAccum la;
-      la.init();
-      for (int c = lane; c < a.ncpr; c += 32) la.add(__ldcg(&st[c].e_ref), __ldcg(&st[c].acc));
-      const float e = warp_max_f(la.e);
-      double sum = la.s > 0.0 ? rescale_pow2(la.s, la.e, e) : 0.0;
-      sum = warp_sum_d(sum);
-      lse = sum > 0.0 ? kLn2 * ((double)e + log2(sum)) : -INFINITY;
-      uint64_t merged = 0ull;
-      for (int c = 0; c < a.ncpr; c += 8) {  // 8 chunk lists in flight, then merged
-        uint64_t kv[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          kv[t] = (lane < k && c + t < a.ncpr)
-                      ? __ldcg(reinterpret_cast<const unsigned long long*>(kk) + (size_t)(c + t) * k + lane)
-                      : 0ull;
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          if (c + t < a.ncpr) merged = warp_merge_desc(merged, kv[t]);
+    if (!__shfl_sync(kFull, last_one, 0)) return;
+    // ---- this warp completed the row: merge all of its chunks (fixed order)
+    __threadfence();
+    const ChunkStat* st = a.stats + slot0;
+    const uint64_t* kk = a.keys + slot0 * k;
+    LseAccum la;
+    la.init();
+    for (int cc = lane; cc < a.ncpr; cc += 32) la.add(__ldcg(&st[cc].e_ref), __ldcg(&st[cc].acc));
+    const float e = warp_max_f(la.e);
+    double sum = la.s > 0.0 ? rescale_pow2(la.s, la.e, e) : 0.0;
+    sum = warp_sum_d(sum);
+    const double lse = sum > 0.0 ? kLn2 * ((double)e + log2(sum)) : -INFINITY;
+    uint64_t merged = 0ull;
+    const unsigned long long* kq = reinterpret_cast<const unsigned long long*>(kk);
+    for (int c0 = 0; c0 < a.ncpr; c0 += 32) {  // only the slots holding a segment's list
+      const bool full_slot = c0 + lane < a.ncpr && __ldcg(kq + (size_t)(c0 + lane) * k) != 0ull;
+      unsigned m = __ballot_sync(kFull, full_slot);
+      while (m) {
+        const int s2 = c0 + __ffs(m) - 1;
+        m &= m - 1;
+        merged = warp_merge_desc(merged, lane < k ? __ldcg(kq + (size_t)s2 * k + lane) : 0ull);
       }
-      if (lane < k) {
-        if (a.out.tok) a.out.tok[seg_row * k + lane] = merged ? key_index(merged) : -1;
-        if (a.out.val) a.out.val[seg_row * k + lane] = merged ? key_value(merged) : -INFINITY;
-      }
-      if (a.out.lse && lane == 0) a.out.lse[seg_row] = lse;
     }
+    if (lane < k) {
+      if (a.out.tok) a.out.tok[seg_row * k + lane] = merged ? key_index(merged) : -1;
+      if (a.out.val) a.out.val[seg_row * k + lane] = merged ? key_value(merged) : -INFINITY;
+    }
+    if (a.out.lse && lane == 0) a.out.lse[seg_row] = lse;
   };
 
   for (int j = 0; j < nj; ++j) {
-    const long long g = g0 + j;
-    const long long row = g / a.ncpr;
-    const int c = (int)(g - row * a.ncpr);
-    if (row != seg_row) {
-      if (seg_row >= 0) finish_segment(c == 0 ? a.ncpr - 1 : c - 1);
+    if (row != seg_row) {  // the range crossed into the next row (at its chunk 0)
+      finish_segment(a.ncpr - 1);
       seg_row = row;
       seg_c0 = c;
       top.init();
     }
     const int st = j % S;
-    // a wait that gives up leaves the data undefined but keeps every warp on
-    // the same barriers (the status word reports it)
-    mbar_wait(smem_u32(&sh.full[st]), (j / S) & 1, abort);
+    // a wait that gives up leaves the data undefined (the status word reports it)
+    mbar_wait(smem_u32(&sh.full[warp][st]), (j / S) & 1, abort);
     const int nvec = min(kSwChunkBytes, a.row_bytes - c * kSwChunkBytes) / 16;
-    const uint4* sp = reinterpret_cast<const uint4*>(sw_smem + st * kSwChunkBytes);
+    const uint4* sp = reinterpret_cast<const uint4*>(ringp + st * kSwChunkBytes);
     const int idx_base = c * a.chunk_elems;
-    for (int v = tid; v < nvec; v += kSwConsumers) {
+    float e_ref = -INFINITY;
+    double acc = 0.0;
+#pragma unroll 2
+    for (int i = 0; i < kSwVecPerLane; ++i) {
+      const int v = lane + 32 * i;
+      if (v >= nvec) break;
       float f[N];
       Elem<T>::unpack(sp[v], f);
       float vmax = f[0];
 #pragma unroll
-      for (int i = 1; i < N; ++i) vmax = fmaxf(vmax, f[i]);
+      for (int q = 1; q < N; ++q) vmax = fmaxf(vmax, f[q]);
       if (vmax > top.s[M - 1]) {
 #pragma unroll
-        for (int i = 0; i < N; ++i) top.push(f[i], idx_base + v * N + i);
+        for (int q = 0; q < N; ++q) top.push(f[q], idx_base + v * N + q);
       }
       if (vmax * kLog2eHi > e_ref) {  // a new reference exponent (rare)
         const float e_new = ceilf(vmax * kLog2eHi);
@@ -500,39 +478,36 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
       if (e_ref > -INFINITY) {  // until a finite logit arrives every term is exp(-inf) = 0
         float part = 0.f;
 #pragma unroll
-        for (int i = 0; i < N; ++i) part += exp2_scaled(f[i], e_ref);
+        for (int q = 0; q < N; ++q) part += exp2_scaled(f[q], e_ref);
         acc += (double)part;
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&sh.empty[st]));
-    // this chunk's log-sum-exp partial: lanes, then warps, in a fixed order
-    {
-      const float e = warp_max_f(e_ref);
-      double sum = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
-      sum = warp_sum_d(sum);
-      if (lane == 0) {
-        sh.e[j & 1][warp] = e;
-        sh.s[j & 1][warp] = sum;
-      }
-    }
-    consumer_sync();
-    if (tid == 0) {
-      LseAccum la;
-      la.init();
-      for (int w = 0; w < kSwConsumerWarps; ++w) la.add(sh.e[j & 1][w], sh.s[j & 1][w]);
+    // this chunk's log-sum-exp partial: a fixed lane order
+    const float e = warp_max_f(e_ref);
+    double sum = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
+    sum = warp_sum_d(sum);
+    if (lane == 0) {
       ChunkStat cs;
-      cs.e_ref = la.e;
+      cs.e_ref = e;
       cs.pad = 0;
-      cs.acc = la.s;
-      a.stats[g] = cs;
+      cs.acc = sum;
+      a.stats[(size_t)row * a.ncpr + c] = cs;
     }
-    e_ref = -INFINITY;
-    acc = 0.0;
+    __syncwarp();
+    if (lane == 0 && issued < nj && !*abort) {
+      fence_proxy_async_smem();  // this stage's reads come before the copy that overwrites it
+      issue_next();
+    }
+    if (++c == a.ncpr) { c = 0; ++row; }
   }
   griddep_launch_dependents();
-  if (seg_row >= 0) finish_segment((int)(g1 - 1 - seg_row * a.ncpr));
-  if (tid == 0 && *abort) atomicExch(a.status, 1);
+  if (nj > 0) finish_segment(c == 0 ? a.ncpr - 1 : c - 1);
+  if (lane == 0) {
+    // every copy issued lands before the CTA may exit
+    for (int d = issued > S ? issued - S : 0; d < issued; ++d)
+      mbar_wait_drain(smem_u32(&sh.full[warp][d % S]), (d / S) & 1, 200000000ull);
+    if (*abort) atomicExch(a.status, 1);
+  }
 }
 
 // ------------------------------------------------------------------- host
@@ -611,7 +586,9 @@ static cudaError_t launch_sweep(const SweepArgs& a, cudaStream_t s, bool pdl) {
   cudaError_t e = ensure_smem_limit((const void*)row_sweep_kernel<T, M>, kSwSmemBytes);
   if (e != cudaSuccess) return e;
   long long C = (long long)device_sm_count() * kSwCtasPerSm;
-  if (C > a.nchunks) C = a.nchunks;
+  const long long want = (a.nchunks + (long long)kSwWarps * kSwMinChunksPerWarp - 1) /
+                         ((long long)kSwWarps * kSwMinChunksPerWarp);
+  if (C > want) C = want;
   return launch_kernel(row_sweep_kernel<T, M>, dim3((unsigned)C), dim3(kSwThreads), kSwSmemBytes, s, pdl, a);
 }
 
