@@ -72,16 +72,18 @@ struct TcLayout {
   static constexpr int kStagesFit = (kSmemOptIn - kStageOff) / kStageBytes;
   static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
   static constexpr int kSmemBytes = kStageOff + kStages * kStageBytes;
-  // TMEM: S double buffer (2 x 64 columns), then O over each tile's keys
-  // 0..31 (O_A) and over keys 32..63 (O_B): the two softmax warps of a lane
-  // quarter keep independent running maxima and are merged once per piece.
+  // TMEM: three S buffers (64 columns each: QK^T may run two tiles ahead of
+  // PV, so the softmax warps find the next S ready), then O over each tile's
+  // keys 0..31 (O_A) and over keys 32..63 (O_B): the two softmax warps of a
+  // lane quarter keep independent running maxima and are merged once per piece.
   // P (bf16, two keys per column) overwrites the S it came from: keys 0..31
   // at the buffer's columns 0..15, keys 32..63 at columns 32..47, each inside
   // the columns of S its own warp has already read.
   static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kSBufs = 3;
   static constexpr uint32_t kColS = 0;  // S buffer i at column 64 * i
-  static constexpr uint32_t kColOA = 128;
-  static constexpr uint32_t kColOB = 128 + D;
+  static constexpr uint32_t kColOA = kSBufs * 64;
+  static constexpr uint32_t kColOB = kSBufs * 64 + D;
   static_assert(kStages >= 2, "at least a double-buffered K/V ring");
   static_assert(kSmemBytes <= kSmemOptIn, "shared memory");
   static_assert(kXchOff + 2 * 128 * 8 <= kHdrBytes, "header");
@@ -93,9 +95,9 @@ struct TcBars {
   uint64_t q_empty[2];
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  uint64_t s_full[3];
+  uint64_t p_full[3][2];  // per S buffer, per half of the tile's keys (the four warps writing that half)
+  uint64_t pv_done[3];
   uint64_t mma_idle;
   uint64_t pair[4];  // per lane quarter: both softmax warps wrote their (max, sum)
   uint64_t never;    // nothing arrives here: the wait probe's barrier
@@ -407,11 +409,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->q_full[i]), 1);
       mbar_init(smem_u32(&bars->q_empty[i]), 1);
+    }
+    for (int i = 0; i < 3; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
-      // every softmax thread (8 warps) arrives for every tile, rows or not: a
-      // warp can run at most one tile ahead of P's consumer, and P is
-      // double-buffered
-      mbar_init(smem_u32(&bars->p_full[i]), 256);
+      // every softmax thread of a half (4 warps) arrives for every tile, rows
+      // or not; S(j) is written only after PV(j - 3) was issued, so a phase
+      // completes before the next one on the same barrier begins
+      mbar_init(smem_u32(&bars->p_full[i][0]), 128);
+      mbar_init(smem_u32(&bars->p_full[i][1]), 128);
       mbar_init(smem_u32(&bars->pv_done[i]), 1);
     }
     for (int i = 0; i < S; ++i) {
@@ -458,15 +463,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     if (warp >= 2) {
       scur.init(b0, hr0, off0, (int)(t1 - t0));
       s_have = scur.next(a, spc);
-      if (s_have) {
-        row_issue(src, spc, p, r_local, lane, G);
-        // wait for them here: issued together with the K/V stream they would
-        // queue behind it (a CTA whose range starts at a tree tile stalled
-        // for microseconds on its mask words)
-        uint64_t sink = src.mw0 ^ src.mw1 ^
-                        (uint64_t)(uint32_t)(src.qpos ^ src.tpos[0] ^ src.tpos[1] ^ src.tpos[2] ^ src.tpos[3]);
-        asm volatile("mov.b64 %0, %0;" : "+l"(sink));  // consumes every loaded value
-      }
+      // issued before the block barrier, so ahead of the first K/V copies,
+      // and consumed only at the piece's first tile: the producer does not
+      // wait for them (a load issued behind the K/V stream waits microseconds)
+      if (s_have) row_issue(src, spc, p, r_local, lane, G);
     }
   }
   griddep_launch_dependents();
@@ -595,12 +595,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           p_len = p_rem = pp.te - pp.tb;
         }
         const bool first = p_rem == p_len;  // O restarts at the first tile of a piece
-        // issue whichever is ready first: the next QK^T (its Q and K landed)
-        // or this tile's PV (its P is written)
-        const uint32_t pb = smem_u32(&bars->p_full[jp & 1]);
+        // issue whatever is ready: the next QK^T (its Q and K landed; at most
+        // two tiles ahead), and this tile's PV per half of its keys (that
+        // half's P is written)
+        const int pbuf = jp % 3;
+        const uint32_t ppar = (uint32_t)(jp / 3) & 1u;
+        const int st = jp % S;
+        const uint32_t p_tmem = tmem + Lay::kColS + (uint32_t)(pbuf * kBN);
+        const uint32_t v_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes + Lay::kKBytes;
+        bool done_h[2] = {false, false};
         uint64_t tw = 0;
         for (uint32_t it = 0;; ++it) {
-          if (jq < total && jq <= jp + 1) {
+          if (jq < total && jq <= jp + 2) {
             if (q_rem == 0) {
               qc.next(a, qp);
               ++q_si;
@@ -612,7 +618,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
               tc_fence_after();
               const uint32_t q_addr = s_base + Lay::kQOff + qb * Lay::kQBytes;
               const uint32_t k_addr = s_base + Lay::kStageOff + (jq % S) * Lay::kStageBytes;
-              const uint32_t t_s = tmem + Lay::kColS + (uint32_t)((jq & 1) * kBN);
+              const uint32_t t_s = tmem + Lay::kColS + (uint32_t)((jq % 3) * kBN);
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = (kk % 4) * 32;
@@ -620,12 +626,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                 const uint64_t db = smem_desc(k_addr + (kk / 4) * Lay::kKVAtomBytes + off, 16, 1024, kSwizzle128B);
                 mma_bf16_ss(t_s, da, db, id_qk, kk > 0);
               }
-              mma_commit(smem_u32(&bars->s_full[jq & 1]));
+              mma_commit(smem_u32(&bars->s_full[jq % 3]));
               if (--q_rem == 0) mma_commit(smem_u32(&bars->q_empty[qb]));
               ++jq;
             }
           }
-          if (mbar_test_wait(pb, (jp >> 1) & 1)) break;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (!done_h[h] && mbar_test_wait(smem_u32(&bars->p_full[pbuf][h]), ppar)) {
+              tc_fence_after();
+              // keys 32h..32h+31 of the tile into O_A (h = 0) or O_B (h = 1); P
+              // from TMEM, 16 keys = 8 columns per MMA
+#pragma unroll
+              for (int kk = 2 * h; kk < 2 * h + 2; ++kk) {
+                const uint32_t a_col = (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8);
+                const uint64_t db = smem_desc(v_addr + kk * 2048, Lay::kKVAtomBytes, 1024, kSwizzle128B);
+                mma_bf16_ts(h ? t_ob : t_oa, p_tmem + a_col, db, id_pv, (!first || (kk & 1)) ? 1u : 0u);
+              }
+              done_h[h] = true;
+            }
+          }
+          if (done_h[0] && done_h[1]) break;
           if ((it & 15u) == 15u) {
             if (*abort) { ok = false; break; }
             const uint64_t now = globaltimer();
@@ -634,20 +655,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           }
         }
         if (!ok) break;
-        tc_fence_after();
-        const int st = jp % S;
-        const uint32_t p_tmem = tmem + Lay::kColS + (uint32_t)((jp & 1) * kBN);
-        const uint32_t v_addr = s_base + Lay::kStageOff + st * Lay::kStageBytes + Lay::kKBytes;
-        // keys 0..31 of the tile into O_A, keys 32..63 into O_B; P from TMEM
-        // (16 keys = 8 columns per MMA)
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t a_col = (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8);
-          const uint64_t db = smem_desc(v_addr + kk * 2048, Lay::kKVAtomBytes, 1024, kSwizzle128B);
-          mma_bf16_ts(kk < 2 ? t_oa : t_ob, p_tmem + a_col, db, id_pv, (!first || (kk & 1)) ? 1u : 0u);
-        }
         mma_commit(smem_u32(&bars->empty[st]));
-        mma_commit(smem_u32(&bars->pv_done[jp & 1]));
+        mma_commit(smem_u32(&bars->pv_done[pbuf]));
         --p_rem;
       }
       // every MMA this thread issued has finished before TMEM is released
@@ -690,14 +699,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const int win_lo = rc.qpos - a.window + 1;
       float m_used = -INFINITY, l = 0.f;  // reference max (scaled, log2) and row sum of this half
       for (int t = pc.tb; t < pc.te; ++t, ++jg) {
-        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[jg & 1]), (jg >> 1) & 1, abort))) {
+        const int sbuf = jg % 3;
+        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[sbuf]), (uint32_t)(jg / 3) & 1u, abort))) {
           ok = false;
           break;
         }
         if (warp_live) {
           tc_fence_after();
           float x[32];
-          tmem_ld32(t_s + (uint32_t)((jg & 1) * kBN), x);
+          tmem_ld32(t_s + (uint32_t)(sbuf * kBN), x);
           tmem_wait_ld();
           const bool tree = t >= pc.ptiles;
           const int key0 = (tree ? (t - pc.ptiles) * kBN : pc.lo + t * kBN) + half * 32;
@@ -724,19 +734,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
               if (kpos < win_lo) vm &= ~(1u << cc);
             }
           }
+          if (__any_sync(kFull, vm != 0xffffffffu)) {  // most prefix tiles see every key
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) x[cc] = ((vm >> cc) & 1u) ? x[cc] : -INFINITY;
-          float m4[4] = {x[0], x[1], x[2], x[3]};
+            for (int cc = 0; cc < 32; ++cc) x[cc] = ((vm >> cc) & 1u) ? x[cc] : -INFINITY;
+          }
+          float m4[4] = {fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8]),
+                         fmax3(x[9], x[10], x[11])};
 #pragma unroll
-          for (int cc = 4; cc < 32; ++cc) m4[cc & 3] = fmaxf(m4[cc & 3], x[cc]);
-          float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          for (int cc = 12; cc < 28; cc += 8) {
+            m4[0] = fmax3(m4[0], x[cc], x[cc + 1]);
+            m4[1] = fmax3(m4[1], x[cc + 2], x[cc + 3]);
+            m4[2] = fmax3(m4[2], x[cc + 4], x[cc + 5]);
+            m4[3] = fmax3(m4[3], x[cc + 6], x[cc + 7]);
+          }
+          float mx = fmax3(fmax3(m4[0], m4[1], m4[2]), fmax3(m4[3], x[28], x[29]), fmaxf(x[30], x[31]));
           mx *= sl2;  // scale > 0 keeps the order
           // (P of this tile replaces S(jg) in TMEM: PV(jg - 2), the last reader of
           // those columns, completed before QK^T(jg), whose commit s_full waited on)
           const bool rebase = mx > m_used + 8.f;
           if (__any_sync(kFull, rebase && t > pc.tb && l > 0.f)) {
             // this half's O may only be rescaled once PV(jg - 1) has finished accumulating
-            if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[(jg - 1) & 1]), ((jg - 1) >> 1) & 1, abort))) {
+            if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[(jg - 1) % 3]), (uint32_t)((jg - 1) / 3) & 1u,
+                                             abort))) {
               ok = false;
               break;
             }
@@ -755,22 +774,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           }
           if (rebase) m_used = mx;
           const float neg_m = m_used > -INFINITY ? -m_used : 0.f;  // no visible key yet: every x is -inf
-          float s4[4] = {0.f, 0.f, 0.f, 0.f};
+          float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
           uint32_t packed[16];
+          const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
           for (int c2 = 0; c2 < 16; ++c2) {
-            const float e0 = ex2(fmaf(x[2 * c2], sl2, neg_m));
-            const float e1 = ex2(fmaf(x[2 * c2 + 1], sl2, neg_m));
-            s4[c2 & 3] += e0 + e1;
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+            const float2 z = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), sl2x2, nm2);
+            const float2 e = make_float2(ex2(z.x), ex2(z.y));
+            s2[c2 & 1] = fadd2(s2[c2 & 1], e);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e.x, e.y);
             packed[c2] = *reinterpret_cast<const uint32_t*>(&h2);
           }
-          l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
-          tmem_st16u(t_s + (uint32_t)((jg & 1) * kBN), packed);  // P over this half's first 16 S columns
+          const float2 st2 = fadd2(s2[0], s2[1]);
+          l += st2.x + st2.y;
+          tmem_st16u(t_s + (uint32_t)(sbuf * kBN), packed);  // P over this half's first 16 S columns
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->p_full[jg & 1]));
+        mbar_arrive(smem_u32(&bars->p_full[sbuf][half]));
       }
       if (!ok) break;
       // ---- end of the piece: merge the two halves' (max, sum), normalise,
@@ -778,7 +799,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       // writes its half of the output columns from both accumulators.
       if (warp_live) {
         const int jl = jg - 1;
-        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[jl & 1]), (jl >> 1) & 1, abort))) {
+        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->pv_done[jl % 3]), (uint32_t)(jl / 3) & 1u, abort))) {
           ok = false;
           break;
         }

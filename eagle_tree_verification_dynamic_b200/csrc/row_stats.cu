@@ -29,9 +29,11 @@ constexpr int kStatThreads = 256;
 constexpr int kStatWarps = kStatThreads / 32;
 constexpr int kUnroll = 8;
 
-// The M largest (value, id) pairs seen by a lane, sorted descending.  Elements
-// arrive in increasing id and only a strictly larger value moves ahead, so
-// among equal values the lower id stays first.
+// The M largest (value, id) pairs seen by a lane, sorted by (value desc, id
+// asc).  Elements arrive in increasing id, so a new element goes behind any
+// equal value; an element it displaces is carried down and goes ahead of an
+// equal value with a higher id (it arrived earlier), which keeps the list in
+// key order.
 template <int M>
 struct LaneTop {
   float s[M];
@@ -44,7 +46,7 @@ struct LaneTop {
     if (!(v > s[M - 1])) return;
 #pragma unroll
     for (int p = 0; p < M; ++p) {
-      if (v > s[p]) {
+      if (v > s[p] || (v == s[p] && idx < id[p])) {
         const float tv = s[p]; s[p] = v; v = tv;
         const int ti = id[p]; id[p] = idx; idx = ti;
       }
