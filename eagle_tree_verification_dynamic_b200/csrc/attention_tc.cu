@@ -582,6 +582,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const uint32_t id_pv = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t t_oa = tmem + Lay::kColOA, t_ob = tmem + Lay::kColOB;
       const int total = bars->n_tiles;
+      // one throw-away MMA while the first tiles are in flight (the first
+      // MMA of a CTA was measured to take ~3 us longer than the next ones):
+      // it reads the second Q buffer and the last K/V stage, whatever they
+      // hold, into the third S buffer, which QK^T(2) overwrites (in order)
+      if (total > 0) {
+        const uint64_t da = smem_desc(s_base + Lay::kQOff + Lay::kQBytes, 16, 1024, kSwizzle128B);
+        const uint64_t db = smem_desc(s_base + Lay::kStageOff + (S - 1) * Lay::kStageBytes, 16, 1024, kSwizzle128B);
+        mma_bf16_ss(tmem + Lay::kColS + 2u * kBN, da, db, id_qk, 0u);
+      }
       PieceCursor qc, pcur;
       qc.init(bars);
       pcur.init(bars);
@@ -633,7 +642,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (!done_h[h] && mbar_test_wait(smem_u32(&bars->p_full[pbuf][h]), ppar)) {
+            // the first half still missing is waited for with a short sleep
+            // (the MMA warp shares its scheduler with two softmax warps, whose
+            // issue slots a spinning poll would take); the other is only tested
+            const uint32_t pbar = smem_u32(&bars->p_full[pbuf][h]);
+            const bool waited = (h == 0 || done_h[0]) ? mbar_try_wait_hint(pbar, ppar, 200u) : mbar_test_wait(pbar, ppar);
+            if (!done_h[h] && waited) {
               tc_fence_after();
               // keys 32h..32h+31 of the tile into O_A (h = 0) or O_B (h = 1); P
               // from TMEM, 16 keys = 8 columns per MMA

@@ -273,8 +273,8 @@ constexpr int kSwWarps = 8;                 // warps per CTA, each streaming its
 constexpr int kSwThreads = kSwWarps * 32;
 constexpr int kSwChunkBytes = 4096;         // one chunk = one warp step: 8 16-byte vectors per lane
 constexpr int kSwVecPerLane = kSwChunkBytes / 16 / 32;
-constexpr int kSwStages = 3;                // each warp's private ring
-constexpr int kSwCtasPerSm = 2;
+constexpr int kSwStages = 2;                // each warp's private ring
+constexpr int kSwCtasPerSm = 3;
 constexpr int kSwMinChunksPerWarp = 4;      // fewer, longer warp ranges: fewer top-k segments per row
 
 struct SwShared {
@@ -294,39 +294,67 @@ struct SweepArgs {
   RowOut out;
 };
 
-// Largest key strictly below `last` among this lane's elements of the chunks
-// [c0, c1] of a row (the main sweep's element assignment; -inf and NaN never
-// qualify), read from global memory.
+// Merge into the warp's sorted list (lane i: the i-th best key, 0 = none) the
+// keys of this lane's elements of one chunk in shared memory (vector
+// v = lane + 32 i, element q) that are above lo (or equal to it, with incl),
+// for the lanes with `mine` set.  Each lane offers its qualifiers best first,
+// one per round, and stops at the first that misses the list's k-th key; a
+// lane with more than four qualifiers whose fourth made the cut reads its
+// elements again below that one.  Whole warp.
 template <typename T>
-__device__ uint64_t seg_next_below(const SweepArgs& a, long long row, int c0, int c1, uint64_t last) {
+__device__ __forceinline__ uint64_t merge_chunk(uint64_t list, int k, const uint4* sp, int nvec, int idx_base,
+                                                uint64_t lo, bool incl, bool mine) {
   constexpr int N = Elem<T>::kPerVec;
   const int lane = threadIdx.x & 31;
-  uint64_t best = 0;
-  const unsigned char* rp = a.x + (size_t)row * a.row_bytes;
-  for (int c = c0; c <= c1; ++c) {
-    const int off = c * kSwChunkBytes;
-    const int nvec = min(kSwChunkBytes, a.row_bytes - off) / 16;
-    const uint4* vp = reinterpret_cast<const uint4*>(rp + off);
-    for (int v = lane; v < nvec; v += 32) {
-      float f[N];
-      Elem<T>::unpack(__ldg(vp + v), f);
+  uint64_t last = ~0ull;  // this lane's keys at or above `last` are merged already
+  bool more = mine;
+  while (__any_sync(kFull, more)) {
+    uint64_t best[4] = {0ull, 0ull, 0ull, 0ull};
+    int cnt = 0;
+    if (more) {
+      for (int i = 0; i < kSwVecPerLane; ++i) {
+        const int v = lane + 32 * i;
+        if (v >= nvec) break;
+        float e[N];
+        Elem<T>::unpack(sp[v], e);
 #pragma unroll
-      for (int i = 0; i < N; ++i) {
-        if (!(f[i] > -INFINITY)) continue;
-        const uint64_t key = make_key(f[i], c * a.chunk_elems + v * N + i);
-        if (key < last && key > best) best = key;
+        for (int q = 0; q < N; ++q) {
+          if (!(e[q] > -INFINITY)) continue;
+          uint64_t x = make_key(e[q], idx_base + v * N + q);
+          if (!(x < last && (x > lo || (incl && x == lo)))) continue;
+          ++cnt;
+#pragma unroll
+          for (int p = 0; p < 4; ++p)  // keys are unique: a plain sorted insertion
+            if (x > best[p]) { const uint64_t t = best[p]; best[p] = x; x = t; }
+        }
       }
     }
+    bool offer = cnt > 0;
+    int r = 0;
+    for (; r < 4; ++r) {
+      const uint64_t cand = (offer && r < cnt) ? best[r] : 0ull;
+      if (!__any_sync(kFull, cand != 0)) break;
+      list = warp_merge_desc(list, warp_sort_desc(cand));
+      const uint64_t kth = __shfl_sync(kFull, list, k - 1);
+      offer = cand != 0 && (kth == 0 || cand >= kth);
+    }
+    more = offer && r == 4 && cnt > 4;
+    if (more) last = best[3];
   }
-  return best;
+  return list;
 }
 
 // Every warp works alone: its contiguous range of the chunk list streams
-// through a private three-stage ring (lane 0 issues the bulk copies), each
-// chunk's log-sum-exp partial is a warp reduction written by lane 0, and at
-// the end of each row segment the warp writes the segment's top-k and takes
-// the row's ticket; the warp completing a row merges it.  No block barrier.
-template <typename T, int M>
+// through a private two-stage ring (lane 0 issues the bulk copies), each
+// chunk's log-sum-exp partial is a warp reduction written by lane 0, and the
+// warp keeps the running top-k of its row segment as a sorted list across its
+// lanes: the main pass only compares each vector's maximum with the list's
+// k-th value, and the few elements above it are read again from the chunk in
+// shared memory and merged (while the list holds fewer than k keys, a chunk's
+// candidates are the elements at or above the k-th largest lane maximum).
+// At the end of a row segment the warp writes its list and takes the row's
+// ticket; the warp that completes a row merges it.  No block barrier.
+template <typename T>
 __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(SweepArgs a) {
   using namespace sm100;
   constexpr int N = Elem<T>::kPerVec;
@@ -334,6 +362,7 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
   extern __shared__ __align__(1024) unsigned char sw_smem[];
   SwShared& sh = *reinterpret_cast<SwShared*>(sw_smem + (size_t)kSwWarps * S * kSwChunkBytes);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int k = a.k;
   const long long W = (long long)gridDim.x * kSwWarps;
   const long long gw = (long long)blockIdx.x * kSwWarps + warp;
   const long long g0 = gw * a.nchunks / W, g1 = (gw + 1) * a.nchunks / W;
@@ -368,42 +397,14 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
   if (lane == 0)
     while (issued < nj && issued < S) issue_next();
 
-  LaneTop<M> top;
-  top.init();
+  uint64_t list = 0ull;  // the segment's running top-k (lane i: the i-th best key)
+  float thr_v = -INFINITY;  // the value of its k-th key (-inf while it holds fewer than k)
   long long seg_row = row;
   int seg_c0 = c;
 
   // end of the segment [seg_c0, c_last] of row seg_row: its top-k into the
   // last chunk's slot (zeros into the others), then the row's ticket
   auto finish_segment = [&](int c_last) {
-    const int k = a.k;
-    uint64_t list;
-    if (k == 1) {
-      list = warp_max_u64(top.key(0));
-    } else {
-      list = warp_sort_desc(top.key(0));
-      uint64_t thr = __shfl_sync(kFull, list, k - 1);
-      bool need = top.key(0) != 0 && top.key(0) >= thr;
-      int r = 1;
-      for (; r < M; ++r) {
-        const uint64_t cand = need ? top.key(r) : 0ull;
-        if (!__any_sync(kFull, cand != 0)) { need = false; break; }
-        list = warp_merge_desc(list, warp_sort_desc(cand));
-        thr = __shfl_sync(kFull, list, k - 1);
-        need = cand != 0 && cand >= thr;
-      }
-      // all M entries of some lane made the cut: pull its further elements (rare)
-      uint64_t last = (r == M && need) ? top.key(M - 1) : 0ull;
-      need = last != 0;
-      while (__any_sync(kFull, need)) {
-        uint64_t nxt = 0;
-        if (need) nxt = seg_next_below<T>(a, seg_row, seg_c0, c_last, last);
-        list = warp_merge_desc(list, warp_sort_desc(nxt));
-        thr = __shfl_sync(kFull, list, k - 1);
-        need = nxt != 0 && nxt >= thr;
-        last = nxt;
-      }
-    }
     const size_t slot0 = (size_t)seg_row * a.ncpr;
     if (lane < k) a.keys[(slot0 + c_last) * k + lane] = list;
     for (int e = lane; e < (c_last - seg_c0) * k; e += 32) a.keys[(slot0 + seg_c0) * k + e] = 0ull;
@@ -449,7 +450,8 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
       finish_segment(a.ncpr - 1);
       seg_row = row;
       seg_c0 = c;
-      top.init();
+      list = 0ull;
+      thr_v = -INFINITY;
     }
     const int st = j % S;
     // a wait that gives up leaves the data undefined (the status word reports it)
@@ -459,41 +461,65 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     const int idx_base = c * a.chunk_elems;
     float e_ref = -INFINITY;
     double acc = 0.0;
-#pragma unroll 2
+    float lane_max = -INFINITY;
+    bool flag = false;
+    const float2 hi2 = make_float2(kLog2eHi, kLog2eHi), lo2 = make_float2(kLog2eLo, kLog2eLo);
+#pragma unroll 4
     for (int i = 0; i < kSwVecPerLane; ++i) {
       const int v = lane + 32 * i;
       if (v >= nvec) break;
       float f[N];
       Elem<T>::unpack(sp[v], f);
-      float vmax = f[0];
-#pragma unroll
-      for (int q = 1; q < N; ++q) vmax = fmaxf(vmax, f[q]);
-      if (vmax > top.s[M - 1]) {
-#pragma unroll
-        for (int q = 0; q < N; ++q) top.push(f[q], idx_base + v * N + q);
-      }
+      float vmax;
+      if constexpr (N == 8) vmax = fmax3(fmax3(f[0], f[1], f[2]), fmax3(f[3], f[4], f[5]), fmaxf(f[6], f[7]));
+      else vmax = fmaxf(fmax3(f[0], f[1], f[2]), f[3]);
+      flag |= vmax > thr_v;
+      lane_max = fmaxf(lane_max, vmax);
       if (vmax * kLog2eHi > e_ref) {  // a new reference exponent (rare)
         const float e_new = ceilf(vmax * kLog2eHi);
         acc = rescale_pow2(acc, e_ref, e_new);
         e_ref = e_new;
       }
       if (e_ref > -INFINITY) {  // until a finite logit arrives every term is exp(-inf) = 0
-        float part = 0.f;
+        // 2^(x log2(e) - e_ref), the product formed with log2(e) as a head/tail pair
+        const float2 ne = make_float2(-e_ref, -e_ref);
+        float2 part = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q = 0; q < N; ++q) part += exp2_scaled(f[q], e_ref);
-        acc += (double)part;
+        for (int q = 0; q < N; q += 2) {
+          const float2 xq = make_float2(f[q], f[q + 1]);
+          const float2 z = ffma2(xq, lo2, ffma2(xq, hi2, ne));
+          part = fadd2(part, make_float2(ex2_ftz(z.x), ex2_ftz(z.y)));
+        }
+        acc += (double)(part.x + part.y);
       }
     }
     // this chunk's log-sum-exp partial: a fixed lane order
-    const float e = warp_max_f(e_ref);
-    double sum = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
-    sum = warp_sum_d(sum);
-    if (lane == 0) {
-      ChunkStat cs;
-      cs.e_ref = e;
-      cs.pad = 0;
-      cs.acc = sum;
-      a.stats[(size_t)row * a.ncpr + c] = cs;
+    {
+      const float e = warp_max_f(e_ref);
+      double sum = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
+      sum = warp_sum_d(sum);
+      if (lane == 0) {
+        ChunkStat cs;
+        cs.e_ref = e;
+        cs.pad = 0;
+        cs.acc = sum;
+        a.stats[(size_t)row * a.ncpr + c] = cs;
+      }
+    }
+    // the segment's top-k: merge this chunk's elements above the threshold
+    const uint64_t kth = __shfl_sync(kFull, list, k - 1);
+    if (kth == 0ull) {
+      // fewer than k keys so far: the chunk's top k are at or above the k-th
+      // largest lane maximum (k lanes hold an element that large)
+      const uint64_t mk = warp_sort_desc(((uint64_t)order_bits(lane_max) << 32) | (uint32_t)lane);
+      const float lo_v = order_value((uint32_t)(__shfl_sync(kFull, mk, k - 1) >> 32));
+      list = merge_chunk<T>(list, k, sp, nvec, idx_base, (uint64_t)order_bits(lo_v) << 32, true, lane_max >= lo_v);
+    } else if (__any_sync(kFull, flag)) {
+      list = merge_chunk<T>(list, k, sp, nvec, idx_base, kth, false, flag);
+    }
+    {
+      const uint64_t k2 = __shfl_sync(kFull, list, k - 1);
+      thr_v = k2 ? key_value(k2) : -INFINITY;
     }
     __syncwarp();
     if (lane == 0 && issued < nj && !*abort) {
@@ -583,15 +609,15 @@ static cudaError_t launch_t(const void* x, long long rows, int V, int k, bool ls
   return launch_typed<T, false, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s, pdl);
 }
 
-template <typename T, int M>
+template <typename T>
 static cudaError_t launch_sweep(const SweepArgs& a, cudaStream_t s, bool pdl) {
-  cudaError_t e = ensure_smem_limit((const void*)row_sweep_kernel<T, M>, kSwSmemBytes);
+  cudaError_t e = ensure_smem_limit((const void*)row_sweep_kernel<T>, kSwSmemBytes);
   if (e != cudaSuccess) return e;
   long long C = (long long)device_sm_count() * kSwCtasPerSm;
   const long long want = (a.nchunks + (long long)kSwWarps * kSwMinChunksPerWarp - 1) /
                          ((long long)kSwWarps * kSwMinChunksPerWarp);
   if (C > want) C = want;
-  return launch_kernel(row_sweep_kernel<T, M>, dim3((unsigned)C), dim3(kSwThreads), kSwSmemBytes, s, pdl, a);
+  return launch_kernel(row_sweep_kernel<T>, dim3((unsigned)C), dim3(kSwThreads), kSwSmemBytes, s, pdl, a);
 }
 
 void row_stats_tickets_span(long long rows, int V, int elem_bytes, int k, size_t* off, size_t* bytes) {
@@ -629,8 +655,8 @@ cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, in
     a.status = reinterpret_cast<int*>(base + l.status_off);
     a.out = out;
     if (!lse) a.out.lse = nullptr;
-    if (dtype == EAGLE_F32) return k == 1 ? launch_sweep<float, 1>(a, s, pdl) : launch_sweep<float, 4>(a, s, pdl);
-    return k == 1 ? launch_sweep<__nv_bfloat16, 1>(a, s, pdl) : launch_sweep<__nv_bfloat16, 4>(a, s, pdl);
+    if (dtype == EAGLE_F32) return launch_sweep<float>(a, s, pdl);
+    return launch_sweep<__nv_bfloat16>(a, s, pdl);
   }
   const ChunkPlan p = plan_chunks(plan_rows > 0 ? plan_rows : rows, V, eb);
   if (dtype == EAGLE_F32) return launch_t<float>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s, pdl);

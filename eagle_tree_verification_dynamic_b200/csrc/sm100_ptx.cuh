@@ -43,6 +43,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Potentially blocking test with a suspend-time hint: the thread may sleep up
+// to about hint_ns waiting for the phase (freeing its issue slots for the other
+// warps of its scheduler) before the call returns false.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Non-blocking test (never suspends the thread): for loops that poll several
 // barriers and must react to whichever completes first.
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
