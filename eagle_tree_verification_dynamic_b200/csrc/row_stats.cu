@@ -7,19 +7,21 @@
 // of p_target for sampling.
 //
 // Rows whose bytes are 16-byte aligned (the usual case) go through
-// row_sweep_kernel: every row is cut into fixed 16 KB chunks, all chunks of all
-// rows form one list, and a persistent grid (three CTAs per SM) takes
-// contiguous ranges of it.  In each CTA one producer thread streams its chunks
-// into a four-stage shared-memory ring with untiled bulk copies (TMA, no
-// multicast) while eight consumer warps read them: per lane the M best
-// (value, id) pairs in registers, and per chunk a base-2 scaled fp64 partial of
-// sum exp(logit) reduced in a fixed order (so a row's log-sum-exp does not
-// depend on the grid).  At the end of each row segment the warps build the
-// segment's exact top-k from the lanes' lists (bitonic sort/merge rounds; a
-// lane is rescanned from memory only if all M of its entries made the cut),
-// and the CTA that completes a row (an atomic ticket; nobody waits) merges the
-// row's chunks and writes the final per-row outputs.  Other rows use
-// row_stats_kernel, one CTA per (row, chunk) with scalar loads.
+// row_sweep_kernel: every row is cut into fixed 4 KB chunks, all chunks of all
+// rows form one list, and each warp of a persistent grid (up to three CTAs of
+// eight warps per SM) takes a contiguous range of it and streams it through
+// its own two-stage shared-memory ring (untiled bulk copies, no multicast).
+// Per chunk a base-2 scaled fp64 partial of sum exp(logit), reduced over the
+// warp in a fixed order, goes to the chunk's slot (so a row's log-sum-exp does
+// not depend on the grid).  The top-k of the warp's row segment: for k = 1
+// each lane keeps its best (value, id) key; for k > 1 the warp buffers the
+// keys above a threshold and selects by rank when the buffer fills, which
+// raises the threshold, so almost every vector is dismissed by one compare of
+// its maximum.  At a segment's end the warp writes its list into the
+// segment's last chunk slot and takes the row's ticket; the warp that
+// completes a row (nobody waits) merges the row's slots and writes the
+// per-row outputs.  Other rows use row_stats_kernel, one CTA per (row, chunk)
+// with scalar loads.
 #include "eagle_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -275,10 +277,13 @@ constexpr int kSwChunkBytes = 4096;         // one chunk = one warp step: 8 16-b
 constexpr int kSwVecPerLane = kSwChunkBytes / 16 / 32;
 constexpr int kSwStages = 2;                // each warp's private ring
 constexpr int kSwCtasPerSm = 3;
-constexpr int kSwMinChunksPerWarp = 4;      // fewer, longer warp ranges: fewer top-k segments per row
+constexpr int kSwCap = 64;                  // candidate keys a warp buffers before it selects
+
+static_assert(kSwCap >= 32 + EAGLE_MAX_TOPK, "after a select one more round of 32 offers must fit");
 
 struct SwShared {
   uint64_t full[kSwWarps][kSwStages];
+  uint64_t cand[kSwWarps][kSwCap];
   int abort;
 };
 constexpr size_t kSwSmemBytes = (size_t)kSwWarps * kSwStages * kSwChunkBytes + sizeof(SwShared);
@@ -294,67 +299,81 @@ struct SweepArgs {
   RowOut out;
 };
 
-// Merge into the warp's sorted list (lane i: the i-th best key, 0 = none) the
-// keys of this lane's elements of one chunk in shared memory (vector
-// v = lane + 32 i, element q) that are above lo (or equal to it, with incl),
-// for the lanes with `mine` set.  Each lane offers its qualifiers best first,
-// one per round, and stops at the first that misses the list's k-th key; a
-// lane with more than four qualifiers whose fourth made the cut reads its
-// elements again below that one.  Whole warp.
-template <typename T>
-__device__ __forceinline__ uint64_t merge_chunk(uint64_t list, int k, const uint4* sp, int nvec, int idx_base,
-                                                uint64_t lo, bool incl, bool mine) {
-  constexpr int N = Elem<T>::kPerVec;
+// The k-th largest of the lanes' values (ties broken by lane), in every lane.
+__device__ __forceinline__ float warp_kth_largest(float v, int k) {
   const int lane = threadIdx.x & 31;
-  uint64_t last = ~0ull;  // this lane's keys at or above `last` are merged already
-  bool more = mine;
-  while (__any_sync(kFull, more)) {
-    uint64_t best[4] = {0ull, 0ull, 0ull, 0ull};
-    int cnt = 0;
-    if (more) {
-      for (int i = 0; i < kSwVecPerLane; ++i) {
-        const int v = lane + 32 * i;
-        if (v >= nvec) break;
-        float e[N];
-        Elem<T>::unpack(sp[v], e);
+  const uint32_t mine = order_bits(v);
+  int rank = 0;
 #pragma unroll
-        for (int q = 0; q < N; ++q) {
-          if (!(e[q] > -INFINITY)) continue;
-          uint64_t x = make_key(e[q], idx_base + v * N + q);
-          if (!(x < last && (x > lo || (incl && x == lo)))) continue;
-          ++cnt;
-#pragma unroll
-          for (int p = 0; p < 4; ++p)  // keys are unique: a plain sorted insertion
-            if (x > best[p]) { const uint64_t t = best[p]; best[p] = x; x = t; }
-        }
-      }
-    }
-    bool offer = cnt > 0;
-    int r = 0;
-    for (; r < 4; ++r) {
-      const uint64_t cand = (offer && r < cnt) ? best[r] : 0ull;
-      if (!__any_sync(kFull, cand != 0)) break;
-      list = warp_merge_desc(list, warp_sort_desc(cand));
-      const uint64_t kth = __shfl_sync(kFull, list, k - 1);
-      offer = cand != 0 && (kth == 0 || cand >= kth);
-    }
-    more = offer && r == 4 && cnt > 4;
-    if (more) last = best[3];
+  for (int d = 1; d < 32; ++d) {
+    const int src = (lane + d) & 31;
+    const uint32_t o = __shfl_sync(kFull, mine, src);
+    rank += (o > mine || (o == mine && src < lane)) ? 1 : 0;
   }
-  return list;
+  const unsigned m = __ballot_sync(kFull, rank == k - 1);  // ranks are a permutation of 0..31
+  return __shfl_sync(kFull, v, __ffs(m) - 1);
 }
 
+// A warp's candidate keys in shared memory.  Invariant: every key offered
+// that is above tau is in buf[0, cnt).  select() sorts the buffer by rank
+// (the number of larger keys; keys are unique), keeps the best k and, once it
+// holds k, raises tau to the k-th.  cnt and tau are warp-uniform.
+struct CandBuf {
+  uint64_t* buf;
+  int cnt;
+  uint64_t tau;
+
+  __device__ __forceinline__ void select(int k) {
+    constexpr int R = kSwCap / 32;
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    uint64_t mine[R];
+    int rank[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = lane + 32 * r;
+      mine[r] = i < cnt ? buf[i] : 0ull;
+      rank[r] = 0;
+    }
+    for (int j = 0; j < cnt; ++j) {
+      const uint64_t o = buf[j];  // the same word in every lane: a broadcast
+#pragma unroll
+      for (int r = 0; r < R; ++r) rank[r] += o > mine[r] ? 1 : 0;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (lane + 32 * r < cnt && rank[r] < k) buf[rank[r]] = mine[r];
+    __syncwarp();
+    if (cnt >= k) {
+      cnt = k;
+      tau = buf[k - 1];
+    }
+  }
+  // Whole warp; each lane offers one key (0: none).
+  __device__ __forceinline__ void offer(uint64_t key, int k) {
+    const int lane = threadIdx.x & 31;
+    const bool has = key > tau;
+    const unsigned m = __ballot_sync(kFull, has);
+    if (m == 0u) return;
+    if (has) buf[cnt + __popc(m & ((1u << lane) - 1u))] = key;
+    cnt += __popc(m);
+    if (cnt > kSwCap - 32) select(k);
+  }
+};
+
 // Every warp works alone: its contiguous range of the chunk list streams
-// through a private two-stage ring (lane 0 issues the bulk copies), each
-// chunk's log-sum-exp partial is a warp reduction written by lane 0, and the
-// warp keeps the running top-k of its row segment as a sorted list across its
-// lanes: the main pass only compares each vector's maximum with the list's
-// k-th value, and the few elements above it are read again from the chunk in
-// shared memory and merged (while the list holds fewer than k keys, a chunk's
-// candidates are the elements at or above the k-th largest lane maximum).
-// At the end of a row segment the warp writes its list and takes the row's
-// ticket; the warp that completes a row merges it.  No block barrier.
-template <typename T>
+// through a private two-stage ring (lane 0 issues the bulk copies) and each
+// chunk's log-sum-exp partial is a warp reduction written by lane 0.  The
+// running top-k of the warp's row segment: with k = 1 each lane keeps its best
+// key and the warp takes the maximum at the segment's end; with k > 1 the warp
+// buffers candidate keys above a threshold (from the first chunk, the k-th
+// largest lane maximum: k elements reach it) and selects by rank whenever the
+// buffer fills, which raises the threshold to the k-th key; a vector whose
+// maximum is below the threshold is never looked at again.  At the end of a
+// row segment the warp writes its list and takes the row's ticket; the warp
+// that completes a row merges it.  No block barrier.
+template <typename T, bool K1>
 __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(SweepArgs a) {
   using namespace sm100;
   constexpr int N = Elem<T>::kPerVec;
@@ -362,7 +381,7 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
   extern __shared__ __align__(1024) unsigned char sw_smem[];
   SwShared& sh = *reinterpret_cast<SwShared*>(sw_smem + (size_t)kSwWarps * S * kSwChunkBytes);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int k = a.k;
+  const int k = K1 ? 1 : a.k;
   const long long W = (long long)gridDim.x * kSwWarps;
   const long long gw = (long long)blockIdx.x * kSwWarps + warp;
   const long long g0 = gw * a.nchunks / W, g1 = (gw + 1) * a.nchunks / W;
@@ -397,8 +416,13 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
   if (lane == 0)
     while (issued < nj && issued < S) issue_next();
 
-  uint64_t list = 0ull;  // the segment's running top-k (lane i: the i-th best key)
-  float thr_v = -INFINITY;  // the value of its k-th key (-inf while it holds fewer than k)
+  uint64_t best = 0ull;      // k = 1: this lane's best key of the segment
+  float best_v = -INFINITY;  // and its value
+  CandBuf cb;                // k > 1: the warp's candidates of the segment
+  cb.buf = sh.cand[warp];
+  cb.cnt = 0;
+  cb.tau = 0ull;
+  bool fresh = true;  // k > 1: the segment has no threshold yet
   long long seg_row = row;
   int seg_c0 = c;
 
@@ -406,8 +430,15 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
   // last chunk's slot (zeros into the others), then the row's ticket
   auto finish_segment = [&](int c_last) {
     const size_t slot0 = (size_t)seg_row * a.ncpr;
-    if (lane < k) a.keys[(slot0 + c_last) * k + lane] = list;
-    for (int e = lane; e < (c_last - seg_c0) * k; e += 32) a.keys[(slot0 + seg_c0) * k + e] = 0ull;
+    if constexpr (K1) {
+      const uint64_t w = warp_max_u64(best);
+      if (lane == 0) a.keys[slot0 + c_last] = w;
+      for (int e = lane; e < c_last - seg_c0; e += 32) a.keys[slot0 + seg_c0 + e] = 0ull;
+    } else {
+      cb.select(k);
+      if (lane < k) a.keys[(slot0 + c_last) * k + lane] = lane < cb.cnt ? cb.buf[lane] : 0ull;
+      for (int e = lane; e < (c_last - seg_c0) * k; e += 32) a.keys[(slot0 + seg_c0) * k + e] = 0ull;
+    }
     __threadfence();
     __syncwarp();
     int last_one = 0;
@@ -419,7 +450,7 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     // ---- this warp completed the row: merge all of its chunks (fixed order)
     __threadfence();
     const ChunkStat* st = a.stats + slot0;
-    const uint64_t* kk = a.keys + slot0 * k;
+    const unsigned long long* kq = reinterpret_cast<const unsigned long long*>(a.keys + slot0 * k);
     LseAccum la;
     la.init();
     for (int cc = lane; cc < a.ncpr; cc += 32) la.add(__ldcg(&st[cc].e_ref), __ldcg(&st[cc].acc));
@@ -427,20 +458,57 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     double sum = la.s > 0.0 ? rescale_pow2(la.s, la.e, e) : 0.0;
     sum = warp_sum_d(sum);
     const double lse = sum > 0.0 ? kLn2 * ((double)e + log2(sum)) : -INFINITY;
-    uint64_t merged = 0ull;
-    const unsigned long long* kq = reinterpret_cast<const unsigned long long*>(kk);
-    for (int c0 = 0; c0 < a.ncpr; c0 += 32) {  // only the slots holding a segment's list
-      const bool full_slot = c0 + lane < a.ncpr && __ldcg(kq + (size_t)(c0 + lane) * k) != 0ull;
-      unsigned m = __ballot_sync(kFull, full_slot);
-      while (m) {
-        const int s2 = c0 + __ffs(m) - 1;
-        m &= m - 1;
-        merged = warp_merge_desc(merged, lane < k ? __ldcg(kq + (size_t)s2 * k + lane) : 0ull);
+    if constexpr (K1) {
+      uint64_t m = 0ull;
+      for (int c0 = 0; c0 < a.ncpr; c0 += 128) {  // four slots a lane in flight
+        uint64_t v[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int i = c0 + lane + 32 * t;
+          v[t] = i < a.ncpr ? __ldcg(kq + i) : 0ull;
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) m = umax64(m, v[t]);
       }
-    }
-    if (lane < k) {
-      if (a.out.tok) a.out.tok[seg_row * k + lane] = merged ? key_index(merged) : -1;
-      if (a.out.val) a.out.val[seg_row * k + lane] = merged ? key_value(merged) : -INFINITY;
+      m = warp_max_u64(m);
+      if (lane == 0) {
+        if (a.out.tok) a.out.tok[seg_row] = m ? key_index(m) : -1;
+        if (a.out.val) a.out.val[seg_row] = m ? key_value(m) : -INFINITY;
+      }
+    } else {
+      // a segment list of k keys bounds the row's k-th key from below: only
+      // keys at or above the best such bound can make the cut
+      uint64_t tk = 0ull;
+      for (int c0 = 0; c0 < a.ncpr; c0 += 128) {
+        uint64_t v[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int i = c0 + lane + 32 * t;
+          v[t] = i < a.ncpr ? __ldcg(kq + (size_t)i * k + (k - 1)) : 0ull;
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) tk = umax64(tk, v[t]);
+      }
+      tk = warp_max_u64(tk);
+      cb.cnt = 0;
+      cb.tau = tk ? tk - 1ull : 0ull;
+      const int total = a.ncpr * k;
+      for (int e0 = 0; e0 < total; e0 += 128) {
+        uint64_t v[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int i = e0 + lane + 32 * t;
+          v[t] = i < total ? __ldcg(kq + i) : 0ull;
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) cb.offer(v[t], k);
+      }
+      cb.select(k);
+      if (lane < k) {
+        const uint64_t m = lane < cb.cnt ? cb.buf[lane] : 0ull;
+        if (a.out.tok) a.out.tok[seg_row * k + lane] = m ? key_index(m) : -1;
+        if (a.out.val) a.out.val[seg_row * k + lane] = m ? key_value(m) : -INFINITY;
+      }
     }
     if (a.out.lse && lane == 0) a.out.lse[seg_row] = lse;
   };
@@ -450,8 +518,11 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
       finish_segment(a.ncpr - 1);
       seg_row = row;
       seg_c0 = c;
-      list = 0ull;
-      thr_v = -INFINITY;
+      best = 0ull;
+      best_v = -INFINITY;
+      cb.cnt = 0;
+      cb.tau = 0ull;
+      fresh = true;
     }
     const int st = j % S;
     // a wait that gives up leaves the data undefined (the status word reports it)
@@ -462,19 +533,28 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     float e_ref = -INFINITY;
     double acc = 0.0;
     float lane_max = -INFINITY;
-    bool flag = false;
+    float vmx[kSwVecPerLane];
     const float2 hi2 = make_float2(kLog2eHi, kLog2eHi), lo2 = make_float2(kLog2eLo, kLog2eLo);
-#pragma unroll 4
+#pragma unroll
     for (int i = 0; i < kSwVecPerLane; ++i) {
       const int v = lane + 32 * i;
-      if (v >= nvec) break;
+      vmx[i] = -INFINITY;
+      if (v >= nvec) continue;
       float f[N];
       Elem<T>::unpack(sp[v], f);
       float vmax;
       if constexpr (N == 8) vmax = fmax3(fmax3(f[0], f[1], f[2]), fmax3(f[3], f[4], f[5]), fmaxf(f[6], f[7]));
       else vmax = fmaxf(fmax3(f[0], f[1], f[2]), f[3]);
-      flag |= vmax > thr_v;
+      vmx[i] = vmax;
       lane_max = fmaxf(lane_max, vmax);
+      if constexpr (K1) {
+        if (vmax >= best_v) {  // rare once the lane holds a large value
+#pragma unroll
+          for (int q = 0; q < N; ++q)
+            if (f[q] > -INFINITY) best = umax64(best, make_key(f[q], idx_base + v * N + q));
+          best_v = best ? key_value(best) : -INFINITY;
+        }
+      }
       if (vmax * kLog2eHi > e_ref) {  // a new reference exponent (rare)
         const float e_new = ceilf(vmax * kLog2eHi);
         acc = rescale_pow2(acc, e_ref, e_new);
@@ -506,20 +586,50 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
         a.stats[(size_t)row * a.ncpr + c] = cs;
       }
     }
-    // the segment's top-k: merge this chunk's elements above the threshold
-    const uint64_t kth = __shfl_sync(kFull, list, k - 1);
-    if (kth == 0ull) {
-      // fewer than k keys so far: the chunk's top k are at or above the k-th
-      // largest lane maximum (k lanes hold an element that large)
-      const uint64_t mk = warp_sort_desc(((uint64_t)order_bits(lane_max) << 32) | (uint32_t)lane);
-      const float lo_v = order_value((uint32_t)(__shfl_sync(kFull, mk, k - 1) >> 32));
-      list = merge_chunk<T>(list, k, sp, nvec, idx_base, (uint64_t)order_bits(lo_v) << 32, true, lane_max >= lo_v);
-    } else if (__any_sync(kFull, flag)) {
-      list = merge_chunk<T>(list, k, sp, nvec, idx_base, kth, false, flag);
-    }
-    {
-      const uint64_t k2 = __shfl_sync(kFull, list, k - 1);
-      thr_v = k2 ? key_value(k2) : -INFINITY;
+    if constexpr (!K1) {
+      if (fresh) {
+        // k lanes hold an element at or above the k-th largest lane maximum
+        const float t0 = warp_kth_largest(lane_max, k);
+        cb.tau = t0 > -INFINITY ? ((uint64_t)order_bits(t0) << 32) - 1ull : 0ull;
+        fresh = false;
+      }
+      // offer this lane's elements above tau, one per lane and round, from
+      // the vectors whose maximum reaches tau's value
+      const float tv = cb.tau ? key_value(cb.tau) : -INFINITY;
+      uint32_t fl = 0u;
+#pragma unroll
+      for (int i = 0; i < kSwVecPerLane; ++i)
+        if (lane + 32 * i < nvec && vmx[i] >= tv) fl |= 1u << i;
+      int cq = 0;  // next element of the lowest flagged vector
+      for (;;) {
+        uint64_t key = 0ull;
+        while (fl != 0u) {
+          const int i = __ffs(fl) - 1;
+          const int v = lane + 32 * i;
+          float f[N];
+          Elem<T>::unpack(sp[v], f);
+          int nq = N;
+#pragma unroll
+          for (int q = 0; q < N; ++q) {
+            if (key == 0ull && q >= cq && f[q] > -INFINITY) {
+              const uint64_t x = make_key(f[q], idx_base + v * N + q);
+              if (x > cb.tau) {
+                key = x;
+                nq = q + 1;
+              }
+            }
+          }
+          if (key != 0ull && nq < N) {
+            cq = nq;
+            break;
+          }
+          fl &= fl - 1u;
+          cq = 0;
+          if (key != 0ull) break;
+        }
+        if (!__any_sync(kFull, key != 0ull)) break;
+        cb.offer(key, k);
+      }
     }
     __syncwarp();
     if (lane == 0 && issued < nj && !*abort) {
@@ -609,15 +719,15 @@ static cudaError_t launch_t(const void* x, long long rows, int V, int k, bool ls
   return launch_typed<T, false, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s, pdl);
 }
 
-template <typename T>
+template <typename T, bool K1>
 static cudaError_t launch_sweep(const SweepArgs& a, cudaStream_t s, bool pdl) {
-  cudaError_t e = ensure_smem_limit((const void*)row_sweep_kernel<T>, kSwSmemBytes);
+  cudaError_t e = ensure_smem_limit((const void*)row_sweep_kernel<T, K1>, kSwSmemBytes);
   if (e != cudaSuccess) return e;
+  // at most three CTAs per SM, and no more warps than chunks
   long long C = (long long)device_sm_count() * kSwCtasPerSm;
-  const long long want = (a.nchunks + (long long)kSwWarps * kSwMinChunksPerWarp - 1) /
-                         ((long long)kSwWarps * kSwMinChunksPerWarp);
+  const long long want = (a.nchunks + kSwWarps - 1) / kSwWarps;
   if (C > want) C = want;
-  return launch_kernel(row_sweep_kernel<T>, dim3((unsigned)C), dim3(kSwThreads), kSwSmemBytes, s, pdl, a);
+  return launch_kernel(row_sweep_kernel<T, K1>, dim3((unsigned)C), dim3(kSwThreads), kSwSmemBytes, s, pdl, a);
 }
 
 void row_stats_tickets_span(long long rows, int V, int elem_bytes, int k, size_t* off, size_t* bytes) {
@@ -655,8 +765,8 @@ cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, in
     a.status = reinterpret_cast<int*>(base + l.status_off);
     a.out = out;
     if (!lse) a.out.lse = nullptr;
-    if (dtype == EAGLE_F32) return launch_sweep<float>(a, s, pdl);
-    return launch_sweep<__nv_bfloat16>(a, s, pdl);
+    if (dtype == EAGLE_F32) return k == 1 ? launch_sweep<float, true>(a, s, pdl) : launch_sweep<float, false>(a, s, pdl);
+    return k == 1 ? launch_sweep<__nv_bfloat16, true>(a, s, pdl) : launch_sweep<__nv_bfloat16, false>(a, s, pdl);
   }
   const ChunkPlan p = plan_chunks(plan_rows > 0 ? plan_rows : rows, V, eb);
   if (dtype == EAGLE_F32) return launch_t<float>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s, pdl);
