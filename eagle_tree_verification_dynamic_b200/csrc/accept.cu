@@ -135,6 +135,23 @@ struct Slice {
       }
     }
   }
+  // A full, 16-byte aligned slice of row src: its loads (issue) and, once
+  // they land, the cached copy (store).  Used to request a row early.
+  __device__ __forceinline__ void issue(const T* src, uint4* v) const {
+#pragma unroll
+    for (int q = 0; q < kMaxLoads; ++q)
+      if (q * kVec < slice) v[q] = __ldg(reinterpret_cast<const uint4*>(src + x0) + q);
+  }
+  __device__ __forceinline__ void store(const uint4* v, T* d, Split2 lse) const {
+#pragma unroll
+    for (int q = 0; q < kMaxLoads; ++q) {
+      if (q * kVec < slice) {
+        const T* e = reinterpret_cast<const T*>(&v[q]);
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) at(d, q * kVec + u) = stored(e[u], lse);
+      }
+    }
+  }
   // tkey / dkey name the rows (target row j, draft row r), lse_t / lse_d their normalisers.
   __device__ void ensure(const T* trow, int tkey, Split2 lse_t, const T* drow, int dkey, Split2 lse_d) {
     const bool lt = cached_t != tkey, ld = drow && cached_d != dkey;
@@ -277,56 +294,6 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   const bool leader = cluster.block_rank() == 0 && threadIdx.x == 0;
   const int tid = threadIdx.x;
 
-  // ---- prologue: everything the decisions read, in one round of independent loads
-  const size_t trow0 = (size_t)b * (n + 1);
-  Parity par;
-  for (int i = tid; i < n; i += kAcceptThreads) {
-    sm.tok[i] = tokens[(size_t)b * n + i];
-    sm.par[i] = parents[(size_t)b * n + i];
-  }
-  for (int i = tid; i <= n; i += kAcceptThreads) {
-    const int r = draft_row[(size_t)b * (n + 1) + i];
-    sm.drow[i] = (r >= 0 && r < R) ? r : -1;  // an out-of-range row counts as "not expanded"
-    sm.amax[i] = row_amax[trow0 + i];
-    if (STOCH) {
-      sm.lse_t[i] = row_lse[trow0 + i];
-      sm.u_acc[i] = uniforms[(size_t)b * 2 * (n + 1) + i];
-      // the residual draw needs u in [0, 1): a NaN or negative u reads as 0 and
-      // u >= 1 as the largest float below 1, so the bonus is always written
-      const float ur = uniforms[(size_t)b * 2 * (n + 1) + (n + 1) + i];
-      sm.u_res[i] = ur >= 0.f ? fminf(ur, 0x1.fffffep-1f) : 0.f;
-    }
-  }
-  __syncthreads();
-  // each node's first child in node order (siblings follow it, in node order)
-  for (int i = tid; i <= n; i += kAcceptThreads) sm.first_child[i] = n + 1;
-  __syncthreads();
-  for (int c = tid + 1; c <= n; c += kAcceptThreads) {
-    const int p = sm.par[c - 1];
-    if (p >= 0 && p <= n) atomicMin(&sm.first_child[p], c);
-  }
-  __syncthreads();
-  if (STOCH) {
-    for (int i = tid; i <= n; i += kAcceptThreads) {
-      const int r = sm.drow[i];
-      sm.lse_d[i] = r >= 0 ? dlse[(size_t)b * R + r] : 0.0;
-    }
-    __syncthreads();
-    // one thread per child: p and q of its token under its parent's rows
-    for (int i = tid + 1; i <= n; i += kAcceptThreads) {
-      const int par = sm.par[i - 1], x = sm.tok[i - 1];
-      double pv = 0.0, qv = 0.0;
-      if (par >= 0 && par <= n && x >= 0 && x < V) {
-        const int pr = sm.drow[par];
-        pv = exp((double)load_logit(tgt + (trow0 + par) * (size_t)V + x) - sm.lse_t[par]);
-        if (pr >= 0) qv = exp((double)load_logit(dft + ((size_t)b * R + pr) * (size_t)V + x) - sm.lse_d[par]);
-      }
-      sm.px[i] = pv;
-      sm.qx[i] = qv;
-    }
-    __syncthreads();
-  }
-
   Slice<T> sl;
   {
     const int gt = (int)cluster.block_rank() * kAcceptThreads + tid;
@@ -341,6 +308,107 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     sl.cached_d = -1;
   }
 
+  // ---- prologue: every value a decision reads, staged in shared memory.
+  // Thread i stages node i and child c = i + 1 (n < kAcceptThreads) in three
+  // rounds of dependent loads: the child's parent and token; the parent's
+  // rows, log-sum-exp and the token's target logit; the token's draft logit.
+  // The root's row slices (read by the first sweep of any walk that rejects
+  // at the root) are requested with the first two rounds.
+  static_assert(EAGLE_MAX_NODES < kAcceptThreads, "one node and one child per thread");
+  const size_t trow0 = (size_t)b * (n + 1);
+  Parity par;
+  for (int i = tid; i <= n; i += kAcceptThreads) sm.first_child[i] = n + 1;
+  const int c_me = tid + 1;
+  int cpar = -1, ctok = -1;
+  if (c_me <= n) {
+    cpar = parents[(size_t)b * n + c_me - 1];
+    ctok = tokens[(size_t)b * n + c_me - 1];
+  }
+  int nd_r = -1, nd_amax = 0;
+  double nd_lse = 0.0;
+  float nd_ua = 0.f, nd_ur = 0.f;
+  if (tid <= n) {
+    const int r = draft_row[trow0 + tid];
+    nd_r = (r >= 0 && r < R) ? r : -1;  // an out-of-range row counts as "not expanded"
+    nd_amax = row_amax[trow0 + tid];
+    if (STOCH) {
+      nd_lse = row_lse[trow0 + tid];
+      nd_ua = uniforms[(size_t)b * 2 * (n + 1) + tid];
+      nd_ur = uniforms[(size_t)b * 2 * (n + 1) + (n + 1) + tid];
+    }
+  }
+  constexpr int kML = Slice<T>::kMaxLoads;
+  uint4 pre_t[kML], pre_d[kML];
+  const bool pre = STOCH && sl.vec_ok && sl.x1 - sl.x0 == sl.slice;
+  double lse_t0 = 0.0, lse_d0 = 0.0;
+  int r0 = -1;
+  if (pre) {
+    lse_t0 = row_lse[trow0];
+    const int r = draft_row[trow0];
+    r0 = (r >= 0 && r < R) ? r : -1;
+    sl.issue(tgt + trow0 * (size_t)V, pre_t);
+  }
+  // round 2
+  const bool cvalid = c_me <= n && cpar >= 0 && cpar <= n && ctok >= 0 && ctok < V;
+  double p_logit = 0.0, p_lse = 0.0, nd_lse_d = 0.0;
+  int p_row = -1;
+  if (STOCH) {
+    if (cvalid) {
+      p_logit = (double)load_logit(tgt + (trow0 + cpar) * (size_t)V + ctok);
+      p_lse = row_lse[trow0 + cpar];
+      const int r = draft_row[trow0 + cpar];
+      p_row = (r >= 0 && r < R) ? r : -1;
+    }
+    if (tid <= n && nd_r >= 0) nd_lse_d = dlse[(size_t)b * R + nd_r];
+    if (pre && r0 >= 0) {
+      lse_d0 = dlse[(size_t)b * R + r0];
+      sl.issue(dft + ((size_t)b * R + r0) * (size_t)V, pre_d);
+    }
+  }
+  if (pre) {  // the target slice landed with round 1
+    Split2 l2;
+    l2.set(lse_t0);
+    sl.store(pre_t, sl.tc, l2);
+    sl.cached_t = 0;
+  }
+  // round 3
+  double q_logit = 0.0, q_lse = 0.0;
+  if (STOCH && cvalid && p_row >= 0) {
+    q_logit = (double)load_logit(dft + ((size_t)b * R + p_row) * (size_t)V + ctok);
+    q_lse = dlse[(size_t)b * R + p_row];
+  }
+  if (pre && r0 >= 0) {  // the draft slice landed with round 2
+    Split2 l2;
+    l2.set(lse_d0);
+    sl.store(pre_d, sl.dc, l2);
+    sl.cached_d = r0;
+  }
+  if (c_me <= n) {
+    sm.tok[c_me - 1] = ctok;
+    sm.par[c_me - 1] = cpar;
+  }
+  if (tid <= n) {
+    sm.drow[tid] = nd_r;
+    sm.amax[tid] = nd_amax;
+    if (STOCH) {
+      sm.lse_t[tid] = nd_lse;
+      sm.lse_d[tid] = nd_r >= 0 ? nd_lse_d : 0.0;
+      sm.u_acc[tid] = nd_ua;
+      // the residual draw needs u in [0, 1): a NaN or negative u reads as 0 and
+      // u >= 1 as the largest float below 1, so the bonus is always written
+      sm.u_res[tid] = nd_ur >= 0.f ? fminf(nd_ur, 0x1.fffffep-1f) : 0.f;
+    }
+  }
+  if (STOCH && c_me <= n) {
+    // p and q of the child's token under its parent's rows; a token outside
+    // the vocabulary has p = q = 0
+    sm.px[c_me] = cvalid ? exp(p_logit - p_lse) : 0.0;
+    sm.qx[c_me] = (cvalid && p_row >= 0) ? exp(q_logit - q_lse) : 0.0;
+  }
+  __syncthreads();  // first_child's initial values and the node arrays
+  // each node's first child in node order (siblings follow it, in node order)
+  if (c_me <= n && cpar >= 0 && cpar <= n) atomicMin(&sm.first_child[cpar], c_me);
+  __syncthreads();
 
   int j = 0, plen = 0;
   double lse_t = STOCH ? sm.lse_t[0] : 0.0;

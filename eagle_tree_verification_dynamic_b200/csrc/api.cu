@@ -414,7 +414,7 @@ eagle_status eagle_verify_step(const eagle_step_in_t* in, const eagle_step_out_t
   const PagedKV pg = {in->block_table, in->page_size, in->pages_per_seq, in->num_pages};
   e = launch_tree_attention(in->q, in->k_cache, in->v_cache, in->prefix_len, in->Lmax, in->k_tree, in->v_tree,
                             out->mask, out->pos, in->B, n, in->Hq, in->Hkv, in->D, in->window, scale, out->attn_out,
-                            ws + L.attn_off, s, paged ? &pg : nullptr);
+                            ws + L.attn_off, s, paged ? &pg : nullptr, /*early=*/true);
   if (e != cudaSuccess) return cuda_status(e);
   // --- acceptance (the draft rows' log-sum-exps are the tree's row_lse)
   e = launch_accept(in->target_logits, in->logits_dtype, in->draft_logits, in->logits_dtype, t.row_lse, L.R,

@@ -249,6 +249,11 @@ struct TcParams {
   // > 0: every softmax warp first waits this long (ns) on a barrier nothing
   // completes, so the CTA takes its abort path (eagle_debug_attention_wait_probe)
   unsigned long long probe_ns;
+  // 1: everything but mask and pos was written before the previous kernel on
+  // the stream started (the fused step, where that kernel is the expansion),
+  // so Q, the prefix and tree K/V and prefix_len are read at once and only the
+  // softmax warps wait for the previous kernel (for mask and pos)
+  int early;
 };
 
 // Loads issued now and consumed later: the K/V stream keeps HBM saturated, so
@@ -439,8 +444,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     tmem_alloc(smem_u32(&bars->tmem_base), Lay::kTmemCols);
     tmem_relinquish();
   }
-  // inputs may come from the previous kernel on the stream
-  griddep_wait();
+  // inputs may come from the previous kernel on the stream (with p.early only
+  // mask and pos do, and the softmax warps wait for them after the barrier)
+  if (!p.early) griddep_wait();
   // softmax warps: cursor and the first piece's row inputs, requested before
   // the K/V stream starts
   PieceCursor scur;
@@ -466,10 +472,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       // issued before the block barrier, so ahead of the first K/V copies,
       // and consumed only at the piece's first tile: the producer does not
       // wait for them (a load issued behind the K/V stream waits microseconds)
-      if (s_have) row_issue(src, spc, p, r_local, lane, G);
+      if (s_have && !p.early) row_issue(src, spc, p, r_local, lane, G);
     }
   }
-  griddep_launch_dependents();
+  // a thread lets the next kernel start only after its own griddep_wait, so
+  // that kernel's early reads never see work older than this kernel's
+  // predecessor unfinished
+  if (!p.early) griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -568,6 +577,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       ok = __shfl_sync(kFull, ok, 0);
       jg = __shfl_sync(kFull, jg, 0);
     }
+    if (p.early) {
+      griddep_wait();
+      griddep_launch_dependents();
+    }
     // drain: every issued copy lands before the CTA may exit
     if (lane == 0) {
       for (int j = (jg > S ? jg - S : 0); j < jg; ++j)
@@ -577,6 +590,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
+    if (p.early) {
+      griddep_wait();
+      griddep_launch_dependents();
+    }
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(128, kBN, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(128, D, 0, 1);
@@ -690,6 +707,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     const uint32_t t_oa = tmem + lane_base + Lay::kColOA, t_ob = tmem + lane_base + Lay::kColOB;
     float2* xch = reinterpret_cast<float2*>(smem + Lay::kXchOff);  // [half][row]
     const float sl2 = p.scale_log2;
+    if (p.early) {
+      griddep_wait();  // mask and pos come from the previous kernel
+      griddep_launch_dependents();
+      if (s_have) row_issue(src, spc, p, r_local, lane, G);
+    }
     Piece pc = spc;
     RowCtx rc = src;
     bool have = s_have;
@@ -1027,7 +1049,7 @@ template <int D>
 static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
                              const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
                              int n, int Hq, int Hkv, int window, float scale, void* out, void* ws, cudaStream_t s,
-                             const PagedKV* pg) {
+                             const PagedKV* pg, bool early) {
   CUtensorMap mk, mv, mkt, mvt;
   const bool paged = pg != nullptr && pg->block_table != nullptr;
   if (paged) Lmax = pg->pages_per_seq * pg->page_size;  // a sequence's capacity
@@ -1092,6 +1114,7 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
   p.q_by_tma = q_tma ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.probe_ns = attention_wait_probe_ns();
+  p.early = early ? 1 : 0;
   const size_t smem = TcLayout<D>::kSmemBytes;
   cudaError_t e = ensure_smem_limit((const void*)attn_tc_kernel<D>, smem);
   if (e != cudaSuccess) return e;
@@ -1132,10 +1155,11 @@ static cudaError_t launch_tc(const void* q, const void* kc, const void* vc, cons
 cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen, int Lmax,
                                   const void* kt, const void* vt, const uint64_t* mask, const int32_t* pos, int B,
                                   int n, int Hq, int Hkv, int D, int window, float scale, void* out, void* ws,
-                                  cudaStream_t s, const PagedKV* pg) {
+                                  cudaStream_t s, const PagedKV* pg, bool early) {
   if (D == 128)
-    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s, pg);
-  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s, pg);
+    return launch_tc<128>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s, pg,
+                          early);
+  return launch_tc<64>(q, kc, vc, plen, Lmax, kt, vt, mask, pos, B, n, Hq, Hkv, window, scale, out, ws, s, pg, early);
 }
 
 }  // namespace eagle

@@ -198,6 +198,11 @@ template <> struct Elem<float> {
     f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
   }
   __device__ static __forceinline__ float load(const float* p) { return __ldg(p); }
+  // the largest element of a vector (NaN ignored, as fmaxf does)
+  __device__ static __forceinline__ float vec_max(const uint4& u) {
+    return fmaxf(fmaxf(__uint_as_float(u.x), __uint_as_float(u.y)), fmaxf(__uint_as_float(u.z), __uint_as_float(u.w)));
+  }
+  __device__ static __forceinline__ uint4 neg_inf_vec() { return make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u); }
 };
 template <> struct Elem<__nv_bfloat16> {
   static constexpr int kPerVec = 8;
@@ -211,6 +216,16 @@ template <> struct Elem<__nv_bfloat16> {
     const unsigned short s = __ldg(reinterpret_cast<const unsigned short*>(p));
     return __uint_as_float(((uint32_t)s) << 16);
   }
+  // the largest element of a vector: packed bf16x2 maxima (a NaN operand
+  // yields the other one), then the larger half
+  __device__ static __forceinline__ float vec_max(const uint4& u) {
+    uint32_t m01, m23, m;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m01) : "r"(u.x), "r"(u.y));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m23) : "r"(u.z), "r"(u.w));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(m01), "r"(m23));
+    return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xffff0000u));
+  }
+  __device__ static __forceinline__ uint4 neg_inf_vec() { return make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u); }
 };
 
 // Streaming 16-byte load that does not keep the line in L1.

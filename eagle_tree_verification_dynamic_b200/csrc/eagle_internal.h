@@ -124,10 +124,14 @@ struct PagedKV {
 };
 // pg == nullptr: dense caches [B][Hkv][Lmax][D]; else kc / vc are the pools
 // and a sequence holds up to pages_per_seq * page_size keys (Lmax unused).
+// early: every input except mask and pos was complete before the previous
+// kernel on the stream started, so the K/V stream begins before that kernel
+// ends (only the fused step, whose previous kernel is the expansion, sets it).
 cudaError_t launch_tree_attention(const void* q, const void* kc, const void* vc, const int32_t* plen,
                                   int Lmax, const void* kt, const void* vt, const uint64_t* mask,
                                   const int32_t* pos, int B, int n, int Hq, int Hkv, int D, int window,
-                                  float scale, void* out, void* ws, cudaStream_t s, const PagedKV* pg = nullptr);
+                                  float scale, void* out, void* ws, cudaStream_t s, const PagedKV* pg = nullptr,
+                                  bool early = false);
 
 // ---- KV-cache compaction after acceptance (kv_compact.cu)
 cudaError_t launch_kv_compact(const void* k_tree, const void* v_tree, const int32_t* path, const int32_t* accepted_len,

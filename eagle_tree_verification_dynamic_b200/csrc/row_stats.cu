@@ -447,61 +447,76 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
       last_one = atomicAdd(a.tickets + seg_row, nseg) + nseg == a.ncpr;
     }
     if (!__shfl_sync(kFull, last_one, 0)) return;
-    // ---- this warp completed the row: merge all of its chunks (fixed order)
+    // ---- this warp completed the row: merge its slots.  The chunk partials,
+    // the segment lists' k-th keys and the first 256 slot keys are requested
+    // together (one round of L2 reads for most rows).
     __threadfence();
     const ChunkStat* st = a.stats + slot0;
     const unsigned long long* kq = reinterpret_cast<const unsigned long long*>(a.keys + slot0 * k);
+    const int total = a.ncpr * k;
+    uint64_t kv[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int i = lane + 32 * t;
+      kv[t] = i < total ? __ldcg(kq + i) : 0ull;
+    }
+    uint64_t tk = 0ull;  // k > 1: the best segment list's k-th key bounds the row's from below
+    if constexpr (!K1) {
+      uint64_t v[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int i = lane + 32 * t;
+        v[t] = i < a.ncpr ? __ldcg(kq + (size_t)i * k + (k - 1)) : 0ull;
+      }
+      for (int i0 = 128 + lane; i0 < a.ncpr; i0 += 32) tk = umax64(tk, __ldcg(kq + (size_t)i0 * k + (k - 1)));
+#pragma unroll
+      for (int t = 0; t < 4; ++t) tk = umax64(tk, v[t]);
+    }
     LseAccum la;
     la.init();
-    for (int cc = lane; cc < a.ncpr; cc += 32) la.add(__ldcg(&st[cc].e_ref), __ldcg(&st[cc].acc));
+    for (int c0 = 0; c0 < a.ncpr; c0 += 64) {  // lane l adds chunks l, l + 32, ... in order
+      const int i0 = c0 + lane, i1 = c0 + 32 + lane;
+      float e0 = -INFINITY, e1 = -INFINITY;
+      double s0 = 0.0, s1 = 0.0;
+      if (i0 < a.ncpr) {
+        e0 = __ldcg(&st[i0].e_ref);
+        s0 = __ldcg(&st[i0].acc);
+      }
+      if (i1 < a.ncpr) {
+        e1 = __ldcg(&st[i1].e_ref);
+        s1 = __ldcg(&st[i1].acc);
+      }
+      la.add(e0, s0);
+      la.add(e1, s1);
+    }
     const float e = warp_max_f(la.e);
     double sum = la.s > 0.0 ? rescale_pow2(la.s, la.e, e) : 0.0;
     sum = warp_sum_d(sum);
     const double lse = sum > 0.0 ? kLn2 * ((double)e + log2(sum)) : -INFINITY;
     if constexpr (K1) {
       uint64_t m = 0ull;
-      for (int c0 = 0; c0 < a.ncpr; c0 += 128) {  // four slots a lane in flight
-        uint64_t v[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int i = c0 + lane + 32 * t;
-          v[t] = i < a.ncpr ? __ldcg(kq + i) : 0ull;
-        }
-#pragma unroll
-        for (int t = 0; t < 4; ++t) m = umax64(m, v[t]);
-      }
+      for (int t = 0; t < 8; ++t) m = umax64(m, kv[t]);
+      for (int i0 = 256 + lane; i0 < total; i0 += 32) m = umax64(m, __ldcg(kq + i0));
       m = warp_max_u64(m);
       if (lane == 0) {
         if (a.out.tok) a.out.tok[seg_row] = m ? key_index(m) : -1;
         if (a.out.val) a.out.val[seg_row] = m ? key_value(m) : -INFINITY;
       }
     } else {
-      // a segment list of k keys bounds the row's k-th key from below: only
-      // keys at or above the best such bound can make the cut
-      uint64_t tk = 0ull;
-      for (int c0 = 0; c0 < a.ncpr; c0 += 128) {
-        uint64_t v[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int i = c0 + lane + 32 * t;
-          v[t] = i < a.ncpr ? __ldcg(kq + (size_t)i * k + (k - 1)) : 0ull;
-        }
-#pragma unroll
-        for (int t = 0; t < 4; ++t) tk = umax64(tk, v[t]);
-      }
       tk = warp_max_u64(tk);
       cb.cnt = 0;
-      cb.tau = tk ? tk - 1ull : 0ull;
-      const int total = a.ncpr * k;
-      for (int e0 = 0; e0 < total; e0 += 128) {
-        uint64_t v[4];
+      cb.tau = tk ? tk - 1ull : 0ull;  // keys at or above tk
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
+      for (int t = 0; t < 8; ++t) cb.offer(kv[t], k);
+      for (int e0 = 256; e0 < total; e0 += 256) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
           const int i = e0 + lane + 32 * t;
-          v[t] = i < total ? __ldcg(kq + i) : 0ull;
+          kv[t] = i < total ? __ldcg(kq + i) : 0ull;
         }
 #pragma unroll
-        for (int t = 0; t < 4; ++t) cb.offer(v[t], k);
+        for (int t = 0; t < 8; ++t) cb.offer(kv[t], k);
       }
       cb.select(k);
       if (lane < k) {
@@ -530,39 +545,45 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     const int nvec = min(kSwChunkBytes, a.row_bytes - c * kSwChunkBytes) / 16;
     const uint4* sp = reinterpret_cast<const uint4*>(ringp + st * kSwChunkBytes);
     const int idx_base = c * a.chunk_elems;
-    float e_ref = -INFINITY;
-    double acc = 0.0;
-    float lane_max = -INFINITY;
+    // pass 1: the lane's vectors into registers (past the chunk's end: -inf),
+    // their maxima and the lane maximum
+    uint4 raw[kSwVecPerLane];
     float vmx[kSwVecPerLane];
-    const float2 hi2 = make_float2(kLog2eHi, kLog2eHi), lo2 = make_float2(kLog2eLo, kLog2eLo);
+    float lane_max = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kSwVecPerLane; ++i) {
       const int v = lane + 32 * i;
-      vmx[i] = -INFINITY;
-      if (v >= nvec) continue;
-      float f[N];
-      Elem<T>::unpack(sp[v], f);
-      float vmax;
-      if constexpr (N == 8) vmax = fmax3(fmax3(f[0], f[1], f[2]), fmax3(f[3], f[4], f[5]), fmaxf(f[6], f[7]));
-      else vmax = fmaxf(fmax3(f[0], f[1], f[2]), f[3]);
-      vmx[i] = vmax;
-      lane_max = fmaxf(lane_max, vmax);
-      if constexpr (K1) {
-        if (vmax >= best_v) {  // rare once the lane holds a large value
+      raw[i] = v < nvec ? sp[v] : Elem<T>::neg_inf_vec();
+      vmx[i] = Elem<T>::vec_max(raw[i]);
+      lane_max = fmaxf(lane_max, vmx[i]);
+    }
+    if constexpr (K1) {
+      if (lane_max >= best_v) {  // rare once the lane holds a large value
 #pragma unroll
-          for (int q = 0; q < N; ++q)
-            if (f[q] > -INFINITY) best = umax64(best, make_key(f[q], idx_base + v * N + q));
-          best_v = best ? key_value(best) : -INFINITY;
+        for (int i = 0; i < kSwVecPerLane; ++i) {
+          if (vmx[i] >= best_v) {
+            float f[N];
+            Elem<T>::unpack(raw[i], f);
+#pragma unroll
+            for (int q = 0; q < N; ++q)
+              if (f[q] > -INFINITY) best = umax64(best, make_key(f[q], idx_base + (lane + 32 * i) * N + q));
+          }
         }
+        best_v = best ? key_value(best) : -INFINITY;
       }
-      if (vmax * kLog2eHi > e_ref) {  // a new reference exponent (rare)
-        const float e_new = ceilf(vmax * kLog2eHi);
-        acc = rescale_pow2(acc, e_ref, e_new);
-        e_ref = e_new;
-      }
-      if (e_ref > -INFINITY) {  // until a finite logit arrives every term is exp(-inf) = 0
-        // 2^(x log2(e) - e_ref), the product formed with log2(e) as a head/tail pair
-        const float2 ne = make_float2(-e_ref, -e_ref);
+    }
+    // pass 2: sum of 2^(x log2(e) - e_ref) with one reference exponent for
+    // the lane's chunk (every term <= 1; the product x log2(e) formed with
+    // log2(e) as a head/tail pair), each vector's terms in fp32, fp64 across
+    const float e_ref = lane_max > -INFINITY ? ceilf(lane_max * kLog2eHi) : -INFINITY;
+    double acc = 0.0;
+    if (e_ref > -INFINITY) {  // else every term is exp(-inf) = 0
+      const float2 hi2 = make_float2(kLog2eHi, kLog2eHi), lo2 = make_float2(kLog2eLo, kLog2eLo);
+      const float2 ne = make_float2(-e_ref, -e_ref);
+#pragma unroll
+      for (int i = 0; i < kSwVecPerLane; ++i) {
+        float f[N];
+        Elem<T>::unpack(raw[i], f);
         float2 part = make_float2(0.f, 0.f);
 #pragma unroll
         for (int q = 0; q < N; q += 2) {

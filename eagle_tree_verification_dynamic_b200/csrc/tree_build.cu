@@ -27,7 +27,6 @@ struct BuildSmem {
   double* cand_lv;   // [P]   log V
   uint64_t* keys;    // [P]   ranking key of candidate g
   uint64_t* sorted;  // [P]   each level's keys in rank order, at the level's id range
-  int* lrank;        // [P]   rank of candidate g within its level
   int* row_tok;      // [R*k]
   int* cand_tok;     // [P]
   int* cand_par;     // [P]   parent candidate id, -1 = root
@@ -67,7 +66,6 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     sm.cand_lv = reinterpret_cast<double*>(p);   p += sizeof(double) * P;
     sm.keys = reinterpret_cast<uint64_t*>(p);    p += sizeof(uint64_t) * P;
     sm.sorted = reinterpret_cast<uint64_t*>(p);  p += sizeof(uint64_t) * P;
-    sm.lrank = reinterpret_cast<int*>(p);        p += sizeof(int) * P;
     sm.row_tok = reinterpret_cast<int*>(p);      p += sizeof(int) * R * k;
     sm.cand_tok = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
     sm.cand_par = reinterpret_cast<int*>(p);     p += sizeof(int) * P;
@@ -104,16 +102,24 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   for (int level = 1; level <= depth; ++level) {
     const int lo = level == 1 ? 0 : k + (level - 2) * kk;
     const int cnt = level == 1 ? k : kk;
-    for (int c = tid; c < cnt; c += NT) {
-      const uint64_t mine = sm.keys[lo + c];
+    // tpc adjacent lanes share a candidate's count (a power of two, so a
+    // group never straddles a warp); every lane runs the same iterations
+    int tpc = 1;
+    while (tpc < 8 && tpc * 2 * cnt <= NT) tpc *= 2;
+    const int sub = tid & (tpc - 1);
+    for (int base = 0; base < cnt * tpc; base += NT) {
+      const int c = (base + tid) / tpc;
+      const uint64_t mine = c < cnt ? sm.keys[lo + c] : ~0ull;
       int rank = 0;
-#pragma unroll 8
-      for (int o = 0; o < cnt; ++o) rank += sm.keys[lo + o] > mine ? 1 : 0;
-      sm.sorted[lo + rank] = mine;
-      sm.lrank[lo + c] = rank;
-      if (level < depth && rank < k) {
-        sm.frontier[rank] = lo + c;
-        sm.cand_row[lo + c] = 1 + (level - 1) * k + rank;
+#pragma unroll 4
+      for (int o = sub; o < cnt; o += tpc) rank += sm.keys[lo + o] > mine ? 1 : 0;
+      for (int m = 1; m < tpc; m <<= 1) rank += __shfl_xor_sync(kFull, rank, m);
+      if (c < cnt && sub == 0) {
+        sm.sorted[lo + rank] = mine;
+        if (level < depth && rank < k) {
+          sm.frontier[rank] = lo + c;
+          sm.cand_row[lo + c] = 1 + (level - 1) * k + rank;
+        }
       }
     }
     __syncthreads();
@@ -135,11 +141,15 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
 
   // 3. rerank: rank among all P = rank in its own level + the larger keys of
   //    every other level (binary search in that level's descending list);
-  //    with per-level widths, the level's rank against its width
-  for (int g = tid; g < P; g += NT) {
-    const uint64_t x = sm.keys[g];
-    const int own = g < k ? 1 : 2 + (g - k) / kk;
-    int rank = sm.lrank[g];
+  //    with per-level widths, the level's rank against its width.  Threads
+  //    take the levels' sorted lists in order, so the lanes of a warp search
+  //    for neighbouring keys (the same or adjacent words) and a warp of ranks
+  //    past n leaves at once.
+  for (int e = tid; e < P; e += NT) {
+    const uint64_t x = sm.sorted[e];
+    const int g = key_gid(x);
+    const int own = e < k ? 1 : 2 + (e - k) / kk;
+    int rank = e - (own == 1 ? 0 : k + (own - 2) * kk);
     if (lw.on) {
       sm.node_of[g] = rank < lw.w[own - 1] ? 1 : 0;
       continue;
@@ -219,7 +229,7 @@ static int build_threads(int P) { return P <= 128 ? 128 : kBuildThreads; }
 size_t tree_build_smem_bytes(int R, int k, int P) {
   const int nt = build_threads(P);
   return sizeof(double) * ((size_t)R * k + P) + 2 * sizeof(uint64_t) * P +
-         sizeof(int) * ((size_t)R * k + 5 * (size_t)P + 32 + nt / 32 + 2 * EAGLE_MAX_NODES);
+         sizeof(int) * ((size_t)R * k + 4 * (size_t)P + 32 + nt / 32 + 2 * EAGLE_MAX_NODES);
 }
 
 // workspace: [chunk stats][chunk keys][row tokens B*R*k int32][row logits B*R*k float]
