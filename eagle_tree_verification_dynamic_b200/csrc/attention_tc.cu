@@ -383,6 +383,12 @@ __device__ bool produce_paged(const TcParams& p, const AttnGeom& a, const Piece&
   return true;
 }
 
+// How long a waiting softmax warp or producer lane may sleep per poll (ns):
+// the MMA warp shares a scheduler with two softmax warps, and a warp that
+// polls in a tight loop takes issue slots from it.
+constexpr uint32_t kSoftmaxSleepNs = 300u;
+constexpr uint32_t kProducerSleepNs = 500u;
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -550,7 +556,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       } else if (lane == 0) {
         for (int t = pc.tb; t < pc.te; ++t) {
           const int st = jg % S;
-          if (jg >= S && !mbar_wait(smem_u32(&bars->empty[st]), ((jg / S) - 1) & 1, abort)) {
+          if (jg >= S && !mbar_wait(smem_u32(&bars->empty[st]), ((jg / S) - 1) & 1, abort, 2000000000ull,
+                                    kProducerSleepNs)) {
             ok = false;
             break;
           }
@@ -736,7 +743,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       float m_used = -INFINITY, l = 0.f;  // reference max (scaled, log2) and row sum of this half
       for (int t = pc.tb; t < pc.te; ++t, ++jg) {
         const int sbuf = jg % 3;
-        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[sbuf]), (uint32_t)(jg / 3) & 1u, abort))) {
+        if (!__all_sync(kFull, mbar_wait(smem_u32(&bars->s_full[sbuf]), (uint32_t)(jg / 3) & 1u, abort, 2000000000ull,
+                                         kSoftmaxSleepNs))) {
           ok = false;
           break;
         }

@@ -541,7 +541,7 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     }
     const int st = j % S;
     // a wait that gives up leaves the data undefined (the status word reports it)
-    mbar_wait(smem_u32(&sh.full[warp][st]), (j / S) & 1, abort);
+    mbar_wait(smem_u32(&sh.full[warp][st]), (j / S) & 1, abort, 2000000000ull, 1000u);
     const int nvec = min(kSwChunkBytes, a.row_bytes - c * kSwChunkBytes) / 16;
     const uint4* sp = reinterpret_cast<const uint4*>(ringp + st * kSwChunkBytes);
     const int idx_base = c * a.chunk_elems;

@@ -73,13 +73,15 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait: gives up after `limit_ns` of wall time or when *abort is set
-// (by any thread of the CTA), setting *abort itself on a timeout.
+// (by any thread of the CTA), setting *abort itself on a timeout.  With
+// sleep_ns > 0 each poll may suspend the thread up to that long (a waiting
+// warp then leaves its scheduler's issue slots to the warps that have work).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit_ns = 2000000000ull) {
+                                          uint64_t limit_ns = 2000000000ull, uint32_t sleep_ns = 0u) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (sleep_ns ? mbar_try_wait_hint(bar, parity, sleep_ns) : mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0) {
       if (*abort) return false;
       if (globaltimer() - t0 > limit_ns) {
