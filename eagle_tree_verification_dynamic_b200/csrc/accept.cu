@@ -29,12 +29,13 @@
 #include <cooperative_groups.h>
 
 #include "eagle_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
 namespace eagle {
 
-constexpr int kAcceptThreads = 512;
+constexpr int kAcceptThreads = 256;
 constexpr int kAcceptWarps = kAcceptThreads / 32;
 constexpr int kCacheBytesPerCta = 64 * 1024;  // both row slices of one CTA
 constexpr int kMaxCluster = 16;
@@ -65,16 +66,19 @@ struct AcceptSmem {
   float u_res[EAGLE_MAX_NODES + 1];
   int first_child[EAGLE_MAX_NODES + 1];  // node j's first child in node order (n + 1: none)
   double warp_part[kAcceptWarps];
-  double red[2][kAcceptWarps];   // block-reduction slots, alternating by call
   double lane_sum[kAcceptThreads];
   double prefix[kAcceptThreads + 1];
-  double cta_total[2];           // cluster-reduction slots, alternating by call
+  // rejection sweeps: every warp's partial of every CTA ([parity][rank * warps + warp]),
+  // and per parity the barrier that completes when all of them have landed
+  double xred[2][kMaxCluster * kAcceptWarps];
+  uint64_t xbar[2];
 };
 
 // Every thread performs the same sequence of reductions, so each keeps its own
 // copy of the slot parities.
 struct Parity {
-  int red = 0, cl = 0;
+  int xs = 0;          // cluster_total / cluster_cta_sum calls so far
+  bool stuck = false;  // a cluster_total wait gave up: later ones do not wait
 };
 
 // This thread's slice [x0, x1) of the current rows, cached in shared memory.
@@ -135,23 +139,6 @@ struct Slice {
       }
     }
   }
-  // A full, 16-byte aligned slice of row src: its loads (issue) and, once
-  // they land, the cached copy (store).  Used to request a row early.
-  __device__ __forceinline__ void issue(const T* src, uint4* v) const {
-#pragma unroll
-    for (int q = 0; q < kMaxLoads; ++q)
-      if (q * kVec < slice) v[q] = __ldg(reinterpret_cast<const uint4*>(src + x0) + q);
-  }
-  __device__ __forceinline__ void store(const uint4* v, T* d, Split2 lse) const {
-#pragma unroll
-    for (int q = 0; q < kMaxLoads; ++q) {
-      if (q * kVec < slice) {
-        const T* e = reinterpret_cast<const T*>(&v[q]);
-#pragma unroll
-        for (int u = 0; u < kVec; ++u) at(d, q * kVec + u) = stored(e[u], lse);
-      }
-    }
-  }
   // tkey / dkey name the rows (target row j, draft row r), lse_t / lse_d their normalisers.
   __device__ void ensure(const T* trow, int tkey, Split2 lse_t, const T* drow, int dkey, Split2 lse_d) {
     const bool lt = cached_t != tkey, ld = drow && cached_d != dkey;
@@ -173,50 +160,83 @@ struct Slice {
   }
 };
 
-// Deterministic block sum; result valid in every thread.  One barrier: the
-// per-warp slots alternate between calls, so a slot is rewritten only after
-// every thread has passed the barrier that follows its last read.
-__device__ double block_sum(double v, AcceptSmem& sm, int& parity) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = warp_sum_d(v);
-  if (lane == 0) sm.red[parity][warp] = v;
-  __syncthreads();
-  double s = 0.0;
-#pragma unroll
-  for (int w = 0; w < kAcceptWarps; ++w) s += sm.red[parity][w];
-  parity ^= 1;
-  return s;
+
+
+__device__ __forceinline__ uint32_t cluster_map(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_async_f64(uint32_t cluster_addr, double v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f64 [%0], %1, [%2];" ::"r"(cluster_addr),
+               "d"(v), "r"(cluster_bar)
+               : "memory");
 }
 
-// Cluster-wide total of one double per CTA, summed in rank order (bit-identical
-// in every CTA).  Each warp reads the ranks' values once (lane r from rank r)
-// and every thread adds them in rank order from registers.  One cluster barrier
-// per call: the slots alternate between calls; a CTA rewrites a slot only after
-// the next call's barrier, which every CTA reaches only after reading that slot.
-__device__ double cluster_sum(double cta_value, AcceptSmem& sm, cg::cluster_group& cluster,
-                              double* prefix_of_rank, int& parity) {
-  if (threadIdx.x == 0) sm.cta_total[parity] = cta_value;
-  cluster.sync();
-  const unsigned nb = cluster.num_blocks();
-  const unsigned me = cluster.block_rank();
-  const unsigned lane = threadIdx.x & 31;
-  const double v_lane = lane < nb ? *cluster.map_shared_rank(&sm.cta_total[parity], lane) : 0.0;
+// Cluster-wide total of one double per warp (the same value in all its
+// lanes), bit-identical in every thread of every CTA.  Lane r of every warp
+// stores the value into rank r's slot [me][warp] with st.async, which counts
+// its bytes on rank r's barrier; a CTA waits until all CL * 16 values have
+// landed, and each warp adds them in a fixed order (lane l: entries l, l + 32,
+// ... in order, then a fixed butterfly).  No cluster barrier: a CTA sends the
+// values of call c + 2 (same slots) only after finishing call c + 1, which
+// needs every CTA's values of c + 1, sent only after each CTA finished reading
+// call c.  A wait that gives up sets *status and the later calls stop waiting.
+__device__ double cluster_total(double wv, AcceptSmem& sm, cg::cluster_group& cluster, Parity& par,
+                                int* status) {
+  const unsigned nb = cluster.num_blocks(), me = cluster.block_rank();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int x = par.xs & 1;
+  const uint32_t phase = (uint32_t)(par.xs >> 1) & 1u;
+  ++par.xs;
+  const uint32_t bar = sm100::smem_u32(&sm.xbar[x]);
+  if (threadIdx.x == 0) sm100::mbar_arrive_expect_tx(bar, nb * kAcceptWarps * (uint32_t)sizeof(double));
+  if ((unsigned)lane < nb)
+    st_async_f64(cluster_map(sm100::smem_u32(&sm.xred[x][me * kAcceptWarps + warp]), lane), wv,
+                 cluster_map(bar, lane));
+  if (!par.stuck && !sm100::mbar_wait_drain(bar, phase, 100000000ull)) {  // 100 ms
+    par.stuck = true;
+    if (status) atomicExch(status, 1);
+  }
+  double acc = 0.0;
+  for (int i = lane; i < (int)nb * kAcceptWarps; i += 32) acc += sm.xred[x][i];
+  return warp_sum_d(acc);
+}
+
+// Cluster-wide total of one double per CTA (the same value in every thread)
+// and the sum of the ranks before this one, both bit-identical in every CTA:
+// thread r stores the value into rank r's slot [me] with st.async; after the
+// barrier every thread adds the CL values in rank order.  Same slots, barriers
+// and call sequence as cluster_total.
+__device__ double cluster_cta_sum(double cta_value, AcceptSmem& sm, cg::cluster_group& cluster, Parity& par,
+                                  int* status, double* prefix_of_rank) {
+  const unsigned nb = cluster.num_blocks(), me = cluster.block_rank();
+  const int x = par.xs & 1;
+  const uint32_t phase = (uint32_t)(par.xs >> 1) & 1u;
+  ++par.xs;
+  const uint32_t bar = sm100::smem_u32(&sm.xbar[x]);
+  if (threadIdx.x == 0) sm100::mbar_arrive_expect_tx(bar, nb * (uint32_t)sizeof(double));
+  if (threadIdx.x < nb)
+    st_async_f64(cluster_map(sm100::smem_u32(&sm.xred[x][me]), threadIdx.x), cta_value,
+                 cluster_map(bar, threadIdx.x));
+  if (!par.stuck && !sm100::mbar_wait_drain(bar, phase, 100000000ull)) {  // 100 ms
+    par.stuck = true;
+    if (status) atomicExch(status, 1);
+  }
   double acc = 0.0;
   for (unsigned r = 0; r < nb; ++r) {
-    const double v = __shfl_sync(kFull, v_lane, r);
-    if (r == me && prefix_of_rank) *prefix_of_rank = acc;
-    acc += v;
+    if (r == me) *prefix_of_rank = acc;
+    acc += sm.xred[x][r];
   }
-  parity ^= 1;
   return acc;
 }
 
 template <typename T>
 __device__ double sweep_total(const Slice<T>& sl, const SweepArgs& a, AcceptSmem& sm, cg::cluster_group& cluster,
-                              Parity& par) {
+                              Parity& par, int* status) {
   float acc = 0.f;  // a slice is <= 32 terms: fp32 within it, fp64 across slices
   for (int i = 0; i < sl.x1 - sl.x0; ++i) acc += sl.weight(a, i);
-  return cluster_sum(block_sum((double)acc, sm, par.red), sm, cluster, nullptr, par.cl);
+  return cluster_total(warp_sum_d((double)acc), sm, cluster, par, status);
 }
 
 // Inverse CDF over the weights: smallest x with cumsum_x > u * total.  Writes
@@ -226,7 +246,7 @@ __device__ double sweep_total(const Slice<T>& sl, const SweepArgs& a, AcceptSmem
 // the crossing lies inside the slice whose interval contains the threshold.
 template <typename T>
 __device__ double sweep_sample(const Slice<T>& sl, const SweepArgs& a, float u, AcceptSmem& sm,
-                               cg::cluster_group& cluster, int32_t* out, Parity& par) {
+                               cg::cluster_group& cluster, int32_t* out, Parity& par, int* status) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int len = sl.x1 - sl.x0;
   float mine_f = 0.f;  // fp32 within the slice; the owner's rescan repeats these additions
@@ -255,7 +275,7 @@ __device__ double sweep_sample(const Slice<T>& sl, const SweepArgs& a, float u, 
   __syncthreads();
   double my_off = 0.0;
   const double cta_total = sm.prefix[kAcceptThreads];
-  const double total = cluster_sum(cta_total, sm, cluster, &my_off, par.cl);
+  const double total = cluster_cta_sum(cta_total, sm, cluster, par, status, &my_off);
   if (total > 0.0) {
     const double thr = (double)u * total;
     const double start = my_off + sm.prefix[tid];
@@ -283,7 +303,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
                    const int32_t* __restrict__ parents, const int32_t* __restrict__ draft_row,
                    const float* __restrict__ uniforms, int32_t* __restrict__ accepted_len,
                    int32_t* __restrict__ path, int32_t* __restrict__ bonus, int slice, bool vec_ok,
-                   bool without_replacement) {
+                   bool without_replacement, int* __restrict__ status) {
   __shared__ AcceptSmem sm;
   extern __shared__ __align__(16) unsigned char cache_raw[];
   griddep_wait();  // the target row statistics come from the previous kernel
@@ -312,12 +332,15 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   // Thread i stages node i and child c = i + 1 (n < kAcceptThreads) in three
   // rounds of dependent loads: the child's parent and token; the parent's
   // rows, log-sum-exp and the token's target logit; the token's draft logit.
-  // The root's row slices (read by the first sweep of any walk that rejects
-  // at the root) are requested with the first two rounds.
   static_assert(EAGLE_MAX_NODES < kAcceptThreads, "one node and one child per thread");
   const size_t trow0 = (size_t)b * (n + 1);
   Parity par;
   for (int i = tid; i <= n; i += kAcceptThreads) sm.first_child[i] = n + 1;
+  if (STOCH && tid == 0) {
+    sm100::mbar_init(sm100::smem_u32(&sm.xbar[0]), 1);
+    sm100::mbar_init(sm100::smem_u32(&sm.xbar[1]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   const int c_me = tid + 1;
   int cpar = -1, ctok = -1;
   if (c_me <= n) {
@@ -337,17 +360,6 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
       nd_ur = uniforms[(size_t)b * 2 * (n + 1) + (n + 1) + tid];
     }
   }
-  constexpr int kML = Slice<T>::kMaxLoads;
-  uint4 pre_t[kML], pre_d[kML];
-  const bool pre = STOCH && sl.vec_ok && sl.x1 - sl.x0 == sl.slice;
-  double lse_t0 = 0.0, lse_d0 = 0.0;
-  int r0 = -1;
-  if (pre) {
-    lse_t0 = row_lse[trow0];
-    const int r = draft_row[trow0];
-    r0 = (r >= 0 && r < R) ? r : -1;
-    sl.issue(tgt + trow0 * (size_t)V, pre_t);
-  }
   // round 2
   const bool cvalid = c_me <= n && cpar >= 0 && cpar <= n && ctok >= 0 && ctok < V;
   double p_logit = 0.0, p_lse = 0.0, nd_lse_d = 0.0;
@@ -360,28 +372,12 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
       p_row = (r >= 0 && r < R) ? r : -1;
     }
     if (tid <= n && nd_r >= 0) nd_lse_d = dlse[(size_t)b * R + nd_r];
-    if (pre && r0 >= 0) {
-      lse_d0 = dlse[(size_t)b * R + r0];
-      sl.issue(dft + ((size_t)b * R + r0) * (size_t)V, pre_d);
-    }
-  }
-  if (pre) {  // the target slice landed with round 1
-    Split2 l2;
-    l2.set(lse_t0);
-    sl.store(pre_t, sl.tc, l2);
-    sl.cached_t = 0;
   }
   // round 3
   double q_logit = 0.0, q_lse = 0.0;
   if (STOCH && cvalid && p_row >= 0) {
     q_logit = (double)load_logit(dft + ((size_t)b * R + p_row) * (size_t)V + ctok);
     q_lse = dlse[(size_t)b * R + p_row];
-  }
-  if (pre && r0 >= 0) {  // the draft slice landed with round 2
-    Split2 l2;
-    l2.set(lse_d0);
-    sl.store(pre_d, sl.dc, l2);
-    sl.cached_d = r0;
   }
   if (c_me <= n) {
     sm.tok[c_me - 1] = ctok;
@@ -408,7 +404,10 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   __syncthreads();  // first_child's initial values and the node arrays
   // each node's first child in node order (siblings follow it, in node order)
   if (c_me <= n && cpar >= 0 && cpar <= n) atomicMin(&sm.first_child[cpar], c_me);
-  __syncthreads();
+  // (with sampling, a cluster barrier: every CTA's sweep barriers are initialised
+  // before any CTA stores into them)
+  if (STOCH) cluster.sync();
+  else __syncthreads();
 
   int j = 0, plen = 0;
   double lse_t = STOCH ? sm.lse_t[0] : 0.0;
@@ -449,7 +448,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
           a.use_q = true;
           a.lse_t.set(lse_t); a.lse_d.set(lse_d); a.t.set(t);
           sl.ensure(trow, j, a.lse_t, drow, r, a.lse_d);
-          F = sweep_total<T>(sl, a, sm, cluster, par);
+          F = sweep_total<T>(sl, a, sm, cluster, par, status);
           if (!(F > 0.0)) break;  // p == q left nothing: keep the walk here
         }
         c = nc;
@@ -489,7 +488,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
   a.t.set(t);
   sl.ensure(tgt + (trow0 + j) * (size_t)V, j, a.lse_t, use_q ? dft + ((size_t)b * R + r) * (size_t)V : nullptr, r,
             a.lse_d);
-  const double total = sweep_sample<T>(sl, a, sm.u_res[j], sm, cluster, bonus + b, par);
+  const double total = sweep_sample<T>(sl, a, sm.u_res[j], sm, cluster, bonus + b, par, status);
   if (!(total > 0.0) && leader) bonus[b] = amax;  // nothing left to sample from
   cluster.sync();  // no CTA leaves while another may still read its shared memory
 }
@@ -512,7 +511,7 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
                                int depth, const int32_t* row_amax, const double* row_lse,
                                const int32_t* tokens, const int32_t* parents, const int32_t* draft_row,
                                const float* uniforms, int B, int32_t* acc_len, int32_t* path,
-                               int32_t* bonus, cudaStream_t s, bool pdl, bool without_replacement) {
+                               int32_t* bonus, cudaStream_t s, bool pdl, bool without_replacement, int* status) {
   int cl = 1, slice = 0;
   size_t dyn = 0;
   const bool vec_ok = (((uintptr_t)tgt | (uintptr_t)dft) % 16 == 0) && ((size_t)V * sizeof(T)) % 16 == 0;
@@ -552,7 +551,7 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
   return cudaLaunchKernelEx(&cfg, accept_walk_kernel<T, STOCH>, static_cast<const T*>(tgt),
                             static_cast<const T*>(dft), dlse, R, V, n, depth, row_amax, row_lse, tokens,
                             parents, draft_row, uniforms, acc_len, path, bonus, slice, vec_ok,
-                            without_replacement);
+                            without_replacement, status);
 }
 
 cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddtype, const double* dlse,
@@ -572,18 +571,24 @@ cudaError_t launch_accept(const void* tgt, int tdtype, const void* dft, int ddty
   cudaError_t e = launch_row_stats(tgt, tdtype, rows, V, 1, stoch, ro, ws, s, zero_tickets, pdl);
   if (e != cudaSuccess) return e;
   (void)ddtype;  // the draft rows share the target's element type (checked by the caller)
+  // the sweep's device status word (after its row tickets): the walk reports a
+  // wait that gave up there too
+  size_t t_off = 0, t_bytes = 0;
+  row_stats_tickets_span(rows, V, dtype_bytes(tdtype), 1, &t_off, &t_bytes);
+  int* status = reinterpret_cast<int*>(static_cast<char*>(ws) + t_off + (size_t)rows * sizeof(int));
   if (tdtype == EAGLE_F32)
     return stoch ? launch_walk<float, true>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens, parents,
                                             draft_row, uniforms, B, accepted_len, path, bonus, s, pdl,
-                                            without_replacement)
+                                            without_replacement, status)
                  : launch_walk<float, false>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
-                                             parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl, false);
+                                             parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl, false,
+                                             status);
   return stoch ? launch_walk<__nv_bfloat16, true>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
                                                   parents, draft_row, uniforms, B, accepted_len, path, bonus, s, pdl,
-                                                  without_replacement)
+                                                  without_replacement, status)
                : launch_walk<__nv_bfloat16, false>(tgt, dft, dlse, R, V, n, depth, row_amax, row_lse, tokens,
                                                    parents, draft_row, uniforms, B, accepted_len, path, bonus, s,
-                                                   pdl, false);
+                                                   pdl, false, status);
 }
 
 }  // namespace eagle

@@ -362,6 +362,16 @@ struct CandBuf {
   }
 };
 
+// Element t of a small register array without dynamic indexing (which would
+// put the array in local memory).
+template <int N>
+__device__ __forceinline__ uint64_t pick(const uint64_t (&v)[N], int t) {
+  uint64_t r = v[0];
+#pragma unroll
+  for (int i = 1; i < N; ++i) r = t == i ? v[i] : r;
+  return r;
+}
+
 // Every warp works alone: its contiguous range of the chunk list streams
 // through a private two-stage ring (lane 0 issues the bulk copies) and each
 // chunk's log-sum-exp partial is a warp reduction written by lane 0.  The
@@ -460,13 +470,19 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
       const int i = lane + 32 * t;
       kv[t] = i < total ? __ldcg(kq + i) : 0ull;
     }
-    uint64_t tk = 0ull;  // k > 1: the best segment list's k-th key bounds the row's from below
+    // k > 1: two lower bounds of the row's k-th key, so that only keys at or
+    // above the larger one are merged: the best segment list's k-th key
+    // (tk), and the k-th largest of the first two keys of the first 64
+    // segment lists (f2: k distinct elements reach it)
+    uint64_t tk = 0ull, f2[4];
     if constexpr (!K1) {
       uint64_t v[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int i = lane + 32 * t;
         v[t] = i < a.ncpr ? __ldcg(kq + (size_t)i * k + (k - 1)) : 0ull;
+        const int i2 = (lane >> 1) + 16 * t;
+        f2[t] = i2 < a.ncpr ? __ldcg(kq + (size_t)i2 * k + (lane & 1)) : 0ull;
       }
       for (int i0 = 128 + lane; i0 < a.ncpr; i0 += 32) tk = umax64(tk, __ldcg(kq + (size_t)i0 * k + (k - 1)));
 #pragma unroll
@@ -506,17 +522,26 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     } else {
       tk = warp_max_u64(tk);
       cb.cnt = 0;
-      cb.tau = tk ? tk - 1ull : 0ull;  // keys at or above tk
+      cb.tau = 0ull;
+      // (the offer loops stay rolled: one copy of offer/select in the code, so
+      // the finalizer, run once per row on a cold instruction cache, is short)
+#pragma unroll 1
+      for (int t = 0; t < 4; ++t) cb.offer(pick(f2, t), k);
+      cb.select(k);
+      const uint64_t bound = umax64(tk, cb.cnt >= k ? cb.buf[k - 1] : 0ull);
+      __syncwarp();
+      cb.cnt = 0;
+      cb.tau = bound ? bound - 1ull : 0ull;  // keys at or above the bound
+      for (int e0 = 0; e0 < total; e0 += 256) {
+        if (e0 > 0) {
 #pragma unroll
-      for (int t = 0; t < 8; ++t) cb.offer(kv[t], k);
-      for (int e0 = 256; e0 < total; e0 += 256) {
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int i = e0 + lane + 32 * t;
-          kv[t] = i < total ? __ldcg(kq + i) : 0ull;
+          for (int t = 0; t < 8; ++t) {
+            const int i = e0 + lane + 32 * t;
+            kv[t] = i < total ? __ldcg(kq + i) : 0ull;
+          }
         }
-#pragma unroll
-        for (int t = 0; t < 8; ++t) cb.offer(kv[t], k);
+#pragma unroll 1
+        for (int t = 0; t < 8; ++t) cb.offer(pick(kv, t), k);
       }
       cb.select(k);
       if (lane < k) {

@@ -10,7 +10,7 @@
 //      the node); their k children each enter the next level with
 //      log V = log V(parent) + lp (log of the product of confidences);
 //   3. rerank: a candidate's rank among all P is its rank in its own level
-//      plus, for every other level, the number of larger keys there (a binary
+//      plus, for every other level, the number of larger keys there (an 8-way
 //      search in that level's sorted list); the n with rank < n are kept;
 //   4. a prefix count renumbers the kept candidates 1..n by ascending id and
 //      the tree arrays are written.
@@ -44,6 +44,31 @@ struct LevelWidths {
   int w[EAGLE_MAX_DEPTH];
   int on;
 };
+
+// The number of keys of the descending list S[0, size) above x: an 8-way
+// search (seven independent probes narrow the range eightfold per round,
+// then at most eight keys are counted), so a list of 100 keys takes three
+// rounds of shared-memory loads instead of a binary search's seven.
+__device__ __forceinline__ int count_greater(const uint64_t* S, int size, uint64_t x) {
+  int lo = 0, n = size;  // the count lies in [lo, lo + n]
+  while (n > 8) {
+    const int step = (n + 7) >> 3;
+    int c = 0;  // S descends: the probes above x form a prefix
+#pragma unroll
+    for (int j = 1; j < 8; ++j) {
+      const int q = step * j;
+      if (q <= n && S[lo + q - 1] > x) ++c;
+    }
+    const int hi = (c < 7 && step * (c + 1) <= n) ? lo + step * (c + 1) - 1 : lo + n;
+    lo += step * c;
+    n = hi - lo;
+  }
+  int c = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < n && S[lo + j] > x) ++c;
+  return lo + c;
+}
 
 // row_tok / row_val: each draft row's top-k tokens and logits (descending),
 // row_lse: each row's log-sum-exp (also the tree's row_lse output).
@@ -110,9 +135,18 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     for (int base = 0; base < cnt * tpc; base += NT) {
       const int c = (base + tid) / tpc;
       const uint64_t mine = c < cnt ? sm.keys[lo + c] : ~0ull;
-      int rank = 0;
-#pragma unroll 4
-      for (int o = sub; o < cnt; o += tpc) rank += sm.keys[lo + o] > mine ? 1 : 0;
+      // this lane's share [o0, o1) of the level, eight independent loads a step
+      const int o0 = sub * cnt / tpc, o1 = (sub + 1) * cnt / tpc;
+      const uint64_t* kp = sm.keys + lo;
+      int rank = 0, o = o0;
+      for (; o + 8 <= o1; o += 8) {
+        uint64_t v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = kp[o + u];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) rank += v[u] > mine ? 1 : 0;
+      }
+      for (; o < o1; ++o) rank += kp[o] > mine ? 1 : 0;
       for (int m = 1; m < tpc; m <<= 1) rank += __shfl_xor_sync(kFull, rank, m);
       if (c < cnt && sub == 0) {
         sm.sorted[lo + rank] = mine;
@@ -140,7 +174,7 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
   }
 
   // 3. rerank: rank among all P = rank in its own level + the larger keys of
-  //    every other level (binary search in that level's descending list);
+  //    every other level (an 8-way search of that level's descending list);
   //    with per-level widths, the level's rank against its width.  Threads
   //    take the levels' sorted lists in order, so the lanes of a warp search
   //    for neighbouring keys (the same or adjacent words) and a warp of ranks
@@ -157,12 +191,7 @@ tree_expand_kernel(const int32_t* __restrict__ row_tok_g, const float* __restric
     for (int level = 1; level <= depth && rank < n; ++level) {
       if (level == own) continue;
       const int lo = level == 1 ? 0 : k + (level - 2) * kk;
-      int a = 0, z = level == 1 ? k : kk;
-      while (a < z) {  // first position whose key is below x
-        const int mid = (a + z) >> 1;
-        if (sm.sorted[lo + mid] > x) a = mid + 1; else z = mid;
-      }
-      rank += a;
+      rank += count_greater(sm.sorted + lo, level == 1 ? k : kk, x);
     }
     sm.node_of[g] = rank < n ? 1 : 0;
   }
