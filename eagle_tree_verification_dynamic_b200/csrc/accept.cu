@@ -519,6 +519,11 @@ static cudaError_t launch_walk(const void* tgt, const void* dft, const double* d
     const int per_cta = kAcceptThreads * slice_max<T>();
     cl = (V + per_cta - 1) / per_cta;
     if (cl < 1) cl = 1;
+    // with few sequences, spread each walk over more CTAs (up to 16, two per
+    // SM): smaller slices load and sweep faster, and the walk is latency-bound
+    const int spare = 2 * device_sm_count() / (B > 0 ? B : 1);
+    const int want = spare < kMaxCluster ? spare : kMaxCluster;
+    if (cl < want) cl = want;
     slice = (V + cl * kAcceptThreads - 1) / (cl * kAcceptThreads);
     constexpr int kVec = 16 / (int)sizeof(T);
     slice = (slice + kVec - 1) / kVec * kVec;  // <= slice_max, itself a multiple of kVec

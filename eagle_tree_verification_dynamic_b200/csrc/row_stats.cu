@@ -769,7 +769,8 @@ template <typename T, bool K1>
 static cudaError_t launch_sweep(const SweepArgs& a, cudaStream_t s, bool pdl) {
   cudaError_t e = ensure_smem_limit((const void*)row_sweep_kernel<T, K1>, kSwSmemBytes);
   if (e != cudaSuccess) return e;
-  // at most three CTAs per SM, and no more warps than chunks
+  // at most three CTAs per SM, and no more warps than chunks (one chunk a
+  // warp beat two: a warp's second chunk waited on the first one's work)
   long long C = (long long)device_sm_count() * kSwCtasPerSm;
   const long long want = (a.nchunks + kSwWarps - 1) / kSwWarps;
   if (C > want) C = want;
