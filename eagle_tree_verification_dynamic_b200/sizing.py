@@ -92,6 +92,21 @@ def default_table() -> CostTable:
     return CostTable.from_json(DEFAULT_TABLE)
 
 
+def table_path(Hq: int, Hkv: int, D: int, V: int, dtype: str) -> str:
+    """Where the shipped B200 table of a verification shape lives (it may not exist)."""
+    return os.path.join(os.path.dirname(DEFAULT_TABLE), f"cost_b200_hq{Hq}_hkv{Hkv}_d{D}_v{V}_{dtype}.json")
+
+
+def table_for(Hq: int, Hkv: int, D: int, V: int, dtype: str) -> CostTable:
+    """The shipped B200 cost table measured for exactly this shape (query / KV heads, head dim,
+    vocabulary, logit storage "bf16" or "f32"); FileNotFoundError when none was measured."""
+    p = table_path(Hq, Hkv, D, V, dtype)
+    if not os.path.exists(p):
+        raise FileNotFoundError(f"no cost table measured for Hq={Hq} Hkv={Hkv} D={D} V={V} {dtype}: run "
+                                f"python -m eagle_tree_verification_dynamic_b200.calibrate --out {p} ...")
+    return CostTable.from_json(p)
+
+
 @dataclass
 class SizedTree:
     tree: Optional[L.Tree]     # None when no level was worth verifying

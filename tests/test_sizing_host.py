@@ -136,3 +136,15 @@ def test_level_widths_match_the_oracle():
             else:
                 assert ratios[j] == pytest.approx(r, rel=1e-12, abs=1e-300)
     assert checked > 250
+
+
+def test_the_shipped_tables_by_shape():
+    from eagle_tree_verification_dynamic_b200.sizing import table_for
+    for shape in [(32, 8, 128, 128256, "bf16"), (32, 32, 128, 32000, "f32")]:
+        t = table_for(*shape)
+        assert t.us.shape == (t.B.size, t.L.size, t.N.size) and np.all(np.isfinite(t.us))
+        assert np.all(t.us[:, :, 0] == 0.0) and np.all(t.us[:, :, 1:] > 0.0)
+        # more candidates never cost less at the largest batch and context
+        assert np.all(np.diff(t.us[-1, -1, :]) >= -0.05 * t.us[-1, -1, 1:])
+    with pytest.raises(FileNotFoundError):
+        table_for(7, 7, 64, 1000, "f32")
