@@ -22,8 +22,12 @@
 // completes a row (nobody waits) merges the row's slots and writes the
 // per-row outputs.  Other rows use row_stats_kernel, one CTA per (row, chunk)
 // with scalar loads.
+#include <cooperative_groups.h>
+
 #include "eagle_internal.h"
 #include "sm100_ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace eagle {
 
@@ -372,6 +376,124 @@ __device__ __forceinline__ uint64_t pick(const uint64_t (&v)[N], int t) {
   return r;
 }
 
+// One 4 KB chunk in shared memory (nvec 16-byte vectors; its first element
+// has index idx_base in the row), whole warp: returns the chunk's log-sum-exp
+// partial (the same in every lane) and folds the chunk into the running top-k
+// of the warp's row segment (k = 1: best / best_v per lane; k > 1: cb, with
+// fresh set while the segment has no threshold yet).
+template <typename T, bool K1>
+__device__ __forceinline__ ChunkStat sweep_chunk(const uint4* sp, int nvec, int idx_base, int k, uint64_t& best,
+                                                 float& best_v, CandBuf& cb, bool& fresh) {
+  using namespace sm100;
+  constexpr int N = Elem<T>::kPerVec;
+  const int lane = threadIdx.x & 31;
+  // pass 1: the lane's vectors into registers (past the chunk's end: -inf),
+  // their maxima and the lane maximum
+  uint4 raw[kSwVecPerLane];
+  float vmx[kSwVecPerLane];
+  float lane_max = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kSwVecPerLane; ++i) {
+    const int v = lane + 32 * i;
+    raw[i] = v < nvec ? sp[v] : Elem<T>::neg_inf_vec();
+    vmx[i] = Elem<T>::vec_max(raw[i]);
+    lane_max = fmaxf(lane_max, vmx[i]);
+  }
+  if constexpr (K1) {
+    if (lane_max >= best_v) {  // rare once the lane holds a large value
+#pragma unroll
+      for (int i = 0; i < kSwVecPerLane; ++i) {
+        if (vmx[i] >= best_v) {
+          float f[N];
+          Elem<T>::unpack(raw[i], f);
+#pragma unroll
+          for (int q = 0; q < N; ++q)
+            if (f[q] > -INFINITY) best = umax64(best, make_key(f[q], idx_base + (lane + 32 * i) * N + q));
+        }
+      }
+      best_v = best ? key_value(best) : -INFINITY;
+    }
+  }
+  // pass 2: sum of 2^(x log2(e) - e_ref) with one reference exponent for
+  // the lane's chunk (every term <= 1; the product x log2(e) formed with
+  // log2(e) as a head/tail pair), each vector's terms in fp32, fp64 across
+  const float e_ref = lane_max > -INFINITY ? ceilf(lane_max * kLog2eHi) : -INFINITY;
+  double acc = 0.0;
+  if (e_ref > -INFINITY) {  // else every term is exp(-inf) = 0
+    const float2 hi2 = make_float2(kLog2eHi, kLog2eHi), lo2 = make_float2(kLog2eLo, kLog2eLo);
+    const float2 ne = make_float2(-e_ref, -e_ref);
+#pragma unroll
+    for (int i = 0; i < kSwVecPerLane; ++i) {
+      float f[N];
+      Elem<T>::unpack(raw[i], f);
+      float2 part = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < N; q += 2) {
+        const float2 xq = make_float2(f[q], f[q + 1]);
+        const float2 z = ffma2(xq, lo2, ffma2(xq, hi2, ne));
+        part = fadd2(part, make_float2(ex2_ftz(z.x), ex2_ftz(z.y)));
+      }
+      acc += (double)(part.x + part.y);
+    }
+  }
+  // this chunk's log-sum-exp partial: a fixed lane order
+  ChunkStat cs;
+  {
+    const float e = warp_max_f(e_ref);
+    double sum = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
+    sum = warp_sum_d(sum);
+    cs.e_ref = e;
+    cs.pad = 0;
+    cs.acc = sum;
+  }
+  if constexpr (!K1) {
+    if (fresh) {
+      // k lanes hold an element at or above the k-th largest lane maximum
+      const float t0 = warp_kth_largest(lane_max, k);
+      cb.tau = t0 > -INFINITY ? ((uint64_t)order_bits(t0) << 32) - 1ull : 0ull;
+      fresh = false;
+    }
+    // offer this lane's elements above tau, one per lane and round, from
+    // the vectors whose maximum reaches tau's value
+    const float tv = cb.tau ? key_value(cb.tau) : -INFINITY;
+    uint32_t fl = 0u;
+#pragma unroll
+    for (int i = 0; i < kSwVecPerLane; ++i)
+      if (lane + 32 * i < nvec && vmx[i] >= tv) fl |= 1u << i;
+    int cq = 0;  // next element of the lowest flagged vector
+    for (;;) {
+      uint64_t key = 0ull;
+      while (fl != 0u) {
+        const int i = __ffs(fl) - 1;
+        const int v = lane + 32 * i;
+        float f[N];
+        Elem<T>::unpack(sp[v], f);
+        int nq = N;
+#pragma unroll
+        for (int q = 0; q < N; ++q) {
+          if (key == 0ull && q >= cq && f[q] > -INFINITY) {
+            const uint64_t x = make_key(f[q], idx_base + v * N + q);
+            if (x > cb.tau) {
+              key = x;
+              nq = q + 1;
+            }
+          }
+        }
+        if (key != 0ull && nq < N) {
+          cq = nq;
+          break;
+        }
+        fl &= fl - 1u;
+        cq = 0;
+        if (key != 0ull) break;
+      }
+      if (!__any_sync(kFull, key != 0ull)) break;
+      cb.offer(key, k);
+    }
+  }
+  return cs;
+}
+
 // Every warp works alone: its contiguous range of the chunk list streams
 // through a private two-stage ring (lane 0 issues the bulk copies) and each
 // chunk's log-sum-exp partial is a warp reduction written by lane 0.  The
@@ -570,113 +692,8 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     const int nvec = min(kSwChunkBytes, a.row_bytes - c * kSwChunkBytes) / 16;
     const uint4* sp = reinterpret_cast<const uint4*>(ringp + st * kSwChunkBytes);
     const int idx_base = c * a.chunk_elems;
-    // pass 1: the lane's vectors into registers (past the chunk's end: -inf),
-    // their maxima and the lane maximum
-    uint4 raw[kSwVecPerLane];
-    float vmx[kSwVecPerLane];
-    float lane_max = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < kSwVecPerLane; ++i) {
-      const int v = lane + 32 * i;
-      raw[i] = v < nvec ? sp[v] : Elem<T>::neg_inf_vec();
-      vmx[i] = Elem<T>::vec_max(raw[i]);
-      lane_max = fmaxf(lane_max, vmx[i]);
-    }
-    if constexpr (K1) {
-      if (lane_max >= best_v) {  // rare once the lane holds a large value
-#pragma unroll
-        for (int i = 0; i < kSwVecPerLane; ++i) {
-          if (vmx[i] >= best_v) {
-            float f[N];
-            Elem<T>::unpack(raw[i], f);
-#pragma unroll
-            for (int q = 0; q < N; ++q)
-              if (f[q] > -INFINITY) best = umax64(best, make_key(f[q], idx_base + (lane + 32 * i) * N + q));
-          }
-        }
-        best_v = best ? key_value(best) : -INFINITY;
-      }
-    }
-    // pass 2: sum of 2^(x log2(e) - e_ref) with one reference exponent for
-    // the lane's chunk (every term <= 1; the product x log2(e) formed with
-    // log2(e) as a head/tail pair), each vector's terms in fp32, fp64 across
-    const float e_ref = lane_max > -INFINITY ? ceilf(lane_max * kLog2eHi) : -INFINITY;
-    double acc = 0.0;
-    if (e_ref > -INFINITY) {  // else every term is exp(-inf) = 0
-      const float2 hi2 = make_float2(kLog2eHi, kLog2eHi), lo2 = make_float2(kLog2eLo, kLog2eLo);
-      const float2 ne = make_float2(-e_ref, -e_ref);
-#pragma unroll
-      for (int i = 0; i < kSwVecPerLane; ++i) {
-        float f[N];
-        Elem<T>::unpack(raw[i], f);
-        float2 part = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < N; q += 2) {
-          const float2 xq = make_float2(f[q], f[q + 1]);
-          const float2 z = ffma2(xq, lo2, ffma2(xq, hi2, ne));
-          part = fadd2(part, make_float2(ex2_ftz(z.x), ex2_ftz(z.y)));
-        }
-        acc += (double)(part.x + part.y);
-      }
-    }
-    // this chunk's log-sum-exp partial: a fixed lane order
-    {
-      const float e = warp_max_f(e_ref);
-      double sum = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
-      sum = warp_sum_d(sum);
-      if (lane == 0) {
-        ChunkStat cs;
-        cs.e_ref = e;
-        cs.pad = 0;
-        cs.acc = sum;
-        a.stats[(size_t)row * a.ncpr + c] = cs;
-      }
-    }
-    if constexpr (!K1) {
-      if (fresh) {
-        // k lanes hold an element at or above the k-th largest lane maximum
-        const float t0 = warp_kth_largest(lane_max, k);
-        cb.tau = t0 > -INFINITY ? ((uint64_t)order_bits(t0) << 32) - 1ull : 0ull;
-        fresh = false;
-      }
-      // offer this lane's elements above tau, one per lane and round, from
-      // the vectors whose maximum reaches tau's value
-      const float tv = cb.tau ? key_value(cb.tau) : -INFINITY;
-      uint32_t fl = 0u;
-#pragma unroll
-      for (int i = 0; i < kSwVecPerLane; ++i)
-        if (lane + 32 * i < nvec && vmx[i] >= tv) fl |= 1u << i;
-      int cq = 0;  // next element of the lowest flagged vector
-      for (;;) {
-        uint64_t key = 0ull;
-        while (fl != 0u) {
-          const int i = __ffs(fl) - 1;
-          const int v = lane + 32 * i;
-          float f[N];
-          Elem<T>::unpack(sp[v], f);
-          int nq = N;
-#pragma unroll
-          for (int q = 0; q < N; ++q) {
-            if (key == 0ull && q >= cq && f[q] > -INFINITY) {
-              const uint64_t x = make_key(f[q], idx_base + v * N + q);
-              if (x > cb.tau) {
-                key = x;
-                nq = q + 1;
-              }
-            }
-          }
-          if (key != 0ull && nq < N) {
-            cq = nq;
-            break;
-          }
-          fl &= fl - 1u;
-          cq = 0;
-          if (key != 0ull) break;
-        }
-        if (!__any_sync(kFull, key != 0ull)) break;
-        cb.offer(key, k);
-      }
-    }
+    const ChunkStat cs = sweep_chunk<T, K1>(sp, nvec, idx_base, k, best, best_v, cb, fresh);
+    if (lane == 0) a.stats[(size_t)row * a.ncpr + c] = cs;
     __syncwarp();
     if (lane == 0 && issued < nj && !*abort) {
       fence_proxy_async_smem();  // this stage's reads come before the copy that overwrites it
@@ -690,6 +707,154 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
     // every copy issued lands before the CTA may exit
     for (int d = issued > S ? issued - S : 0; d < issued; ++d)
       mbar_wait_drain(smem_u32(&sh.full[warp][d % S]), (d / S) & 1, 200000000ull);
+    if (*abort) atomicExch(a.status, 1);
+  }
+}
+
+// ------------------------------------------------- one row per CTA (few rows)
+// When every CTA of the grid is resident at once, each row (or each half of a
+// long row: a cluster of two CTAs) is one CTA's work: every warp requests its
+// four chunks with one bulk copy at the start, folds them with sweep_chunk,
+// and the CTA merges its warps' results in shared memory (the second CTA of a
+// pair hands its chunk partials and lists to the first through distributed
+// shared memory).  No global tickets, no merging warp on another SM.  The
+// chunks and the log-sum-exp combine order are row_sweep_kernel's, so both
+// kernels give bit-identical outputs.
+constexpr int kRcWarps = 8;
+constexpr int kRcThreads = kRcWarps * 32;
+constexpr int kRcChunksPerWarp = 4;
+constexpr int kRcChunks = kRcWarps * kRcChunksPerWarp;  // 128 KB of row per CTA
+constexpr int kRcMaxCluster = 2;
+
+struct RcShared {
+  uint64_t full[kRcWarps];
+  uint64_t cand[kRcWarps][kSwCap];
+  ChunkStat stats[kRcMaxCluster * kRcChunks];               // first CTA: the row's chunk partials
+  uint64_t lists[kRcMaxCluster * kRcWarps][EAGLE_MAX_TOPK];  // first CTA: every warp's list
+  int abort;
+};
+constexpr size_t kRcSmemBytes = (size_t)kRcChunks * kSwChunkBytes + sizeof(RcShared);
+
+template <typename T, bool K1>
+__global__ void __launch_bounds__(kRcThreads, 1) row_cta_kernel(SweepArgs a, int cl) {
+  using namespace sm100;
+  extern __shared__ __align__(1024) unsigned char rc_smem[];
+  RcShared& sh = *reinterpret_cast<RcShared*>(rc_smem + (size_t)kRcChunks * kSwChunkBytes);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int k = K1 ? 1 : a.k;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = cl > 1 ? (int)cluster.block_rank() : 0;
+  const long long row = blockIdx.x / cl;
+  const int wc0 = rank * kRcChunks + warp * kRcChunksPerWarp;  // this warp's first chunk of the row
+  const int nwc = max(0, min(a.ncpr, wc0 + kRcChunksPerWarp) - wc0);
+  const unsigned char* wsm = rc_smem + (size_t)warp * kRcChunksPerWarp * kSwChunkBytes;
+  volatile int* abort = &sh.abort;
+  if (threadIdx.x == 0) sh.abort = 0;
+  if (lane == 0) {
+    mbar_init(smem_u32(&sh.full[warp]), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();  // the logits (and the outputs) may belong to the previous kernel
+  if (lane == 0 && nwc > 0) {
+    const int bytes = min(nwc * kSwChunkBytes, a.row_bytes - wc0 * kSwChunkBytes);
+    const uint32_t fb = smem_u32(&sh.full[warp]);
+    mbar_arrive_expect_tx(fb, (uint32_t)bytes);
+    bulk_load(smem_u32(wsm), a.x + (size_t)row * a.row_bytes + (size_t)wc0 * kSwChunkBytes, (uint32_t)bytes, fb);
+  }
+  // where the first CTA of the row collects the partials and lists
+  ChunkStat* stats = sh.stats;
+  uint64_t* lists = &sh.lists[0][0];
+  if (rank > 0) {
+    stats = cluster.map_shared_rank(stats, 0);
+    lists = cluster.map_shared_rank(lists, 0);
+  }
+  uint64_t best = 0ull;
+  float best_v = -INFINITY;
+  CandBuf cb;
+  cb.buf = sh.cand[warp];
+  cb.cnt = 0;
+  cb.tau = 0ull;
+  bool fresh = true;
+  if (nwc > 0) {
+    // a wait that gives up leaves the data undefined (the status word reports it)
+    mbar_wait(smem_u32(&sh.full[warp]), 0, abort, 2000000000ull, 1000u);
+    for (int j = 0; j < nwc; ++j) {
+      const int c = wc0 + j;
+      const int nvec = min(kSwChunkBytes, a.row_bytes - c * kSwChunkBytes) / 16;
+      const ChunkStat cs = sweep_chunk<T, K1>(reinterpret_cast<const uint4*>(wsm + (size_t)j * kSwChunkBytes), nvec,
+                                              c * a.chunk_elems, k, best, best_v, cb, fresh);
+      if (lane == 0) stats[c] = cs;
+    }
+  }
+  uint64_t* my_list = lists + (size_t)(rank * kRcWarps + warp) * EAGLE_MAX_TOPK;
+  if constexpr (K1) {
+    const uint64_t w = warp_max_u64(best);
+    if (lane == 0) my_list[0] = w;
+  } else {
+    if (nwc > 0) cb.select(k);
+    if (lane < k) my_list[lane] = (nwc > 0 && lane < cb.cnt) ? cb.buf[lane] : 0ull;
+  }
+  griddep_launch_dependents();
+  if (cl > 1) cluster.sync();  // the second CTA's stores land before the first reads them
+  else __syncthreads();
+  if (rank == 0 && warp == 0) {
+    const int nl = cl * kRcWarps;
+    LseAccum la;
+    la.init();
+    for (int c0 = 0; c0 < a.ncpr; c0 += 64) {  // lane l adds chunks l, l + 32, ... in order
+      const int i0 = c0 + lane, i1 = c0 + 32 + lane;
+      float e0 = -INFINITY, e1 = -INFINITY;
+      double s0 = 0.0, s1 = 0.0;
+      if (i0 < a.ncpr) {
+        e0 = sh.stats[i0].e_ref;
+        s0 = sh.stats[i0].acc;
+      }
+      if (i1 < a.ncpr) {
+        e1 = sh.stats[i1].e_ref;
+        s1 = sh.stats[i1].acc;
+      }
+      la.add(e0, s0);
+      la.add(e1, s1);
+    }
+    const float e = warp_max_f(la.e);
+    double sum = la.s > 0.0 ? rescale_pow2(la.s, la.e, e) : 0.0;
+    sum = warp_sum_d(sum);
+    const double lse = sum > 0.0 ? kLn2 * ((double)e + log2(sum)) : -INFINITY;
+    if constexpr (K1) {
+      const uint64_t m = warp_max_u64(lane < nl ? sh.lists[lane][0] : 0ull);
+      if (lane == 0) {
+        if (a.out.tok) a.out.tok[row] = m ? key_index(m) : -1;
+        if (a.out.val) a.out.val[row] = m ? key_value(m) : -INFINITY;
+      }
+    } else {
+      // the same bounds as the segment merge: the best list's k-th key and the
+      // k-th largest of the lists' first two keys; then every key at or above
+      uint64_t tk = warp_max_u64(lane < nl ? sh.lists[lane][k - 1] : 0ull);
+      cb.cnt = 0;
+      cb.tau = 0ull;
+      cb.offer((lane >> 1) < nl ? sh.lists[lane >> 1][lane & 1] : 0ull, k);
+      cb.select(k);
+      const uint64_t bound = umax64(tk, cb.cnt >= k ? cb.buf[k - 1] : 0ull);
+      __syncwarp();
+      cb.cnt = 0;
+      cb.tau = bound ? bound - 1ull : 0ull;
+#pragma unroll 1
+      for (int e0 = 0; e0 < nl * k; e0 += 32) {
+        const int i = e0 + lane;
+        cb.offer(i < nl * k ? sh.lists[i / k][i % k] : 0ull, k);
+      }
+      cb.select(k);
+      if (lane < k) {
+        const uint64_t m = lane < cb.cnt ? cb.buf[lane] : 0ull;
+        if (a.out.tok) a.out.tok[row * k + lane] = m ? key_index(m) : -1;
+        if (a.out.val) a.out.val[row * k + lane] = m ? key_value(m) : -INFINITY;
+      }
+    }
+    if (a.out.lse && lane == 0) a.out.lse[row] = lse;
+  }
+  if (lane == 0) {
+    if (nwc > 0 && *abort) mbar_wait_drain(smem_u32(&sh.full[warp]), 0, 200000000ull);  // the copy lands first
     if (*abort) atomicExch(a.status, 1);
   }
 }
@@ -765,8 +930,43 @@ static cudaError_t launch_t(const void* x, long long rows, int V, int k, bool ls
   return launch_typed<T, false, 4>(x, rows, V, k, p, vec, stats, keys, tickets, out, s, pdl);
 }
 
+// One row per CTA (a pair for rows over 128 KB) when the whole grid fits on
+// the GPU at once and the rows are either short (a row is one warp's work) or
+// long (over 128 KB, so an SM would carry a comparable share in the persistent
+// kernel anyway); returns false (launching nothing) otherwise.  In between
+// (e.g. 51 rows of 32 chunks) the persistent kernel, one chunk a warp over
+// every SM, measured faster in spite of its cross-SM merge.
+template <typename T, bool K1>
+static bool launch_rows(const SweepArgs& a, long long rows, cudaStream_t s, bool pdl, cudaError_t* err) {
+  const int cl = (a.ncpr + kRcChunks - 1) / kRcChunks;
+  if (cl > kRcMaxCluster || rows * cl > device_sm_count()) return false;
+  if (a.ncpr > kRcChunksPerWarp && cl < 2) return false;
+  cudaError_t e = ensure_smem_limit((const void*)row_cta_kernel<T, K1>, kRcSmemBytes);
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * cl));
+    cfg.blockDim = dim3(kRcThreads);
+    cfg.dynamicSmemBytes = kRcSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, row_cta_kernel<T, K1>, a, cl);
+  }
+  *err = e;
+  return true;
+}
+
 template <typename T, bool K1>
 static cudaError_t launch_sweep(const SweepArgs& a, cudaStream_t s, bool pdl) {
+  cudaError_t e0;
+  if (launch_rows<T, K1>(a, a.nchunks / a.ncpr, s, pdl, &e0)) return e0;
   cudaError_t e = ensure_smem_limit((const void*)row_sweep_kernel<T, K1>, kSwSmemBytes);
   if (e != cudaSuccess) return e;
   // at most three CTAs per SM, and no more warps than chunks (one chunk a
