@@ -938,20 +938,22 @@ attn_combine_kernel(const CombParams p) {
   const int u = blockIdx.x, b = u / HR, hr = u % HR;
   const int g = hr / a.RG, rg = hr % a.RG;
   const int G = p.Hq / a.Hkv;
-  __shared__ long long s_T, s_start;
-  __shared__ int s_tiles, s_stat[kCombineWarps];
+  __shared__ long long s_T;
+  __shared__ int s_cfirst, s_clast, s_stat[kCombineWarps];
   if (warp == 0) {  // the schedule depends only on prefix_len, not on the attention kernel
     const long long T = geom_prefix(a, a.B, lane);
     const long long cum = geom_prefix(a, b, lane);
     const int tiles = geom_tiles(a, b);
-    if (lane == 0) {
+    if (lane == 0) {  // (64-bit divisions: done before the wait, while the attention runs)
+      const long long start = cum + (long long)hr * tiles;
       s_T = T;
-      s_start = cum + (long long)hr * tiles;
-      s_tiles = tiles;
+      s_cfirst = cta_of_tile(start, T, a.C);
+      s_clast = cta_of_tile(start + tiles - 1, T, a.C);
     }
   }
   __syncthreads();
   griddep_wait();
+  griddep_launch_dependents();  // the next kernel's prologue may overlap this one
   if (blockIdx.x == 0 && blockIdx.y == 0) {
     int st = 0;
     for (int i = tid; i < a.C; i += kCombineThreads) st = max(st, p.cta_status[i]);
@@ -964,9 +966,9 @@ attn_combine_kernel(const CombParams p) {
       *p.status = st;
     }
   }
-  const long long T = s_T, start = s_start;
-  const int c_first = cta_of_tile(start, T, a.C);
-  const int c_last = cta_of_tile(start + s_tiles - 1, T, a.C);
+  const long long T = s_T;
+  const int c_first = s_cfirst, c_last = s_clast;
+  const bool all_live = T >= a.C;  // with at least one tile per CTA no range is empty
   const int r = blockIdx.y * kCombineWarps + warp;
   const int valid = min(kRowsPerCta, a.n * G - rg * kRowsPerCta);
   if (c_first == c_last || r >= valid) return;
@@ -985,7 +987,7 @@ attn_combine_kernel(const CombParams p) {
       // a CTA with an empty range wrote no partial: read the first piece's
       // (always written, finite) and give it weight 0
       const int s = s0 + j;
-      const bool live = s < nseg && cta_nonempty(c_first + s, T, a.C);
+      const bool live = s < nseg && (all_live || cta_nonempty(c_first + s, T, a.C));
       const size_t sl = live ? slot0 + s : slot0;
       ls[j] = live ? __ldcg(p.part_lse + sl * kRowsPerCta + r) : -INFINITY;
       const float* src = p.part_o + (sl * kRowsPerCta + r) * D + lane * DPL;
