@@ -308,7 +308,14 @@ def attn_source_digest() -> str:
 # workload, valid only for the kernel sources whose digest is the key: after any
 # change to the kernel the entry no longer matches and `traffic` reads null
 # until a new capture is taken.
-ATTN_TRAFFIC_BYTES = {}
+ATTN_TRAFFIC_BYTES = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum -k regex:attn_tc_kernel
+    #     -s 8 -c 1 on `bench.py --config <name> --steps 3 --warmup 3 --no-cpu-baseline --no-per-config`
+    ("7b", 0, "f5510cc048b9f0a0"): 35111936 + 0,
+    ("l3-8b", 0, "f5510cc048b9f0a0"): 204041984 + 5385472,
+    ("serve", 0, "f5510cc048b9f0a0"): 309454080 + 13574400,
+    ("long", 0, "f5510cc048b9f0a0"): 194805504 + 3845632,
+}
 
 
 def load_peaks():

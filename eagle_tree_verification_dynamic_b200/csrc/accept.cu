@@ -360,7 +360,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
       nd_ur = uniforms[(size_t)b * 2 * (n + 1) + (n + 1) + tid];
     }
   }
-  // round 2
+  // second load round: the parent's rows, log-sum-exp and target logit
   const bool cvalid = c_me <= n && cpar >= 0 && cpar <= n && ctok >= 0 && ctok < V;
   double p_logit = 0.0, p_lse = 0.0, nd_lse_d = 0.0;
   int p_row = -1;
@@ -373,7 +373,7 @@ accept_walk_kernel(const T* __restrict__ tgt, const T* __restrict__ dft, const d
     }
     if (tid <= n && nd_r >= 0) nd_lse_d = dlse[(size_t)b * R + nd_r];
   }
-  // round 3
+  // third load round: the draft logit
   double q_logit = 0.0, q_lse = 0.0;
   if (STOCH && cvalid && p_row >= 0) {
     q_logit = (double)load_logit(dft + ((size_t)b * R + p_row) * (size_t)V + ctok);

@@ -20,8 +20,10 @@
 // its maximum.  At a segment's end the warp writes its list into the
 // segment's last chunk slot and takes the row's ticket; the warp that
 // completes a row (nobody waits) merges the row's slots and writes the
-// per-row outputs.  Other rows use row_stats_kernel, one CTA per (row, chunk)
-// with scalar loads.
+// per-row outputs.  Rows that are few and short or long use row_cta_kernel
+// (one row per CTA, no cross-SM merge).  Unaligned rows, and argmax sweeps over
+// many rows, use row_stats_kernel: one CTA per (row, chunk), 16-byte loads
+// when the rows allow them (scalar otherwise), the same ticket merge.
 #include <cooperative_groups.h>
 
 #include "eagle_internal.h"
@@ -996,7 +998,12 @@ cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, in
     if (e != cudaSuccess) return e;
   }
   const bool vec = ((uintptr_t)x % 16 == 0) && (((size_t)V * eb) % 16 == 0);
-  if (vec && (size_t)V * eb <= 0x7fffffffu) {
+  // a large argmax sweep (k = 1 over many rows) goes to the per-(row, chunk)
+  // kernel below: its plain 16-byte loads keep more bytes in flight per SM
+  // than the warps' two-stage rings, 80 against 112 us for the 1056 target
+  // rows of the serving mix
+  const bool wide_argmax = k == 1 && rows >= 4LL * device_sm_count();
+  if (vec && (size_t)V * eb <= 0x7fffffffu && !wide_argmax) {
     // the chunked TMA sweep computes the log-sum-exp always (lse == false only drops the output)
     SweepArgs a;
     a.x = static_cast<const unsigned char*>(x);

@@ -30,7 +30,7 @@ def _ref_topk(x64: np.ndarray, k: int):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("V,k,rows", [(1000, 2, 5), (32000, 10, 51), (128256, 8, 7), (4099, 5, 3),
                                       (777, 32, 4), (20000, 1, 9), (4000, 6, 3), (128256, 1, 5),
-                                      (32000, 1, 200)])
+                                      (32000, 1, 200), (32000, 1, 600)])
 def test_row_stats_topk_and_lse(dtype, V, k, rows):
     rng = np.random.default_rng(V + k)
     x = rng.normal(0, 3, size=(rows, V)).astype(np.float32)
