@@ -594,8 +594,10 @@ def measure(torch, cfg, mode, dev, rank, K, W, barrier, paged=0, e2e=False, comp
 
 
 # the other workloads reported beside the headline, each with its acceptance mode
-PER_CONFIG = [("tiny", "greedy"), ("7b", "greedy"), ("l3-8b", "stochastic"), ("long", "greedy"),
-              ("long-window", "greedy"), ("serve", "stochastic")]
+PER_CONFIG = [("tiny", "greedy", 0), ("7b", "greedy", 0), ("l3-8b", "stochastic", 0), ("long", "greedy", 0),
+              ("long-window", "greedy", 0), ("serve", "stochastic", 0),
+              # the serving mix over a paged prefix cache (page size in keys)
+              ("serve", "stochastic", 64), ("serve", "stochastic", 16)]
 
 
 def main():
@@ -668,19 +670,20 @@ def main():
     if not args.no_per_config and not ps and args.config == "7b" and world == 1:
         per = {}
         Kc = max(20, K // 4)
-        for name, mode in PER_CONFIG:
+        for name, mode, pg in PER_CONFIG:
             c = get_config(name)
-            rc = measure(torch, c, mode, dev, rank, Kc, W, barrier)
+            rc = measure(torch, c, mode, dev, rank, Kc, W, barrier, paged=pg)
             a2, s2, st2, sb2 = rooflines(c, mode, rc["ms"], rc["stage_ms"], hbm_peak, tc_peak, peak_src,
-                                         (name, 0, digest))
-            entry = {"workload": workload_desc(c, mode), "steps": Kc, "l2": rc["l2"],
+                                         (name, pg, digest))
+            desc = workload_desc(c, mode) + (f", paged KV cache ({pg}-key pages)" if pg else "")
+            entry = {"workload": desc, "steps": Kc, "l2": rc["l2"],
                      "ms_per_step": round(rc["ms"], 5), "steps_per_s": round(1000.0 / rc["ms"], 2),
                      "stages_ms": {k: round(v, 5) for k, v in rc["stage_ms"].items()},
                      "roofline": a2, "accept_sweep_roofline": s2, "step_roofline": st2,
                      "accepted_mean": rc["accepted_mean"]}
-            if not args.no_cpu_baseline:
+            if not args.no_cpu_baseline and not pg:  # (the oracle's work does not depend on the paging)
                 entry["cpu_baseline"] = cpu_baseline(c, mode, args.cpu_seconds_per_config)
-            per[f"{name} {mode}"] = entry
+            per[f"{name} {mode}" + (f" paged{pg}" if pg else "")] = entry
         line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
