@@ -14,10 +14,9 @@
 // Per chunk a base-2 scaled fp64 partial of sum exp(logit), reduced over the
 // warp in a fixed order, goes to the chunk's slot (so a row's log-sum-exp does
 // not depend on the grid).  The top-k of the warp's row segment: for k = 1
-// each lane keeps its best (value, id) key; for k > 1 the warp buffers the
-// keys above a threshold and selects by rank when the buffer fills, which
-// raises the threshold, so almost every vector is dismissed by one compare of
-// its maximum.  At a segment's end the warp writes its list into the
+// the warp keeps its best (value, id) key; for k > 1 it buffers the keys
+// above a threshold and selects by rank, which raises the threshold, so
+// almost every chunk is dismissed by one compare of its maximum.  At a segment's end the warp writes its list into the
 // segment's last chunk slot and takes the row's ticket; the warp that
 // completes a row (nobody waits) merges the row's slots and writes the
 // per-row outputs.  Rows that are few and short or long use row_cta_kernel
@@ -381,8 +380,11 @@ __device__ __forceinline__ uint64_t pick(const uint64_t (&v)[N], int t) {
 // One 4 KB chunk in shared memory (nvec 16-byte vectors; its first element
 // has index idx_base in the row), whole warp: returns the chunk's log-sum-exp
 // partial (the same in every lane) and folds the chunk into the running top-k
-// of the warp's row segment (k = 1: best / best_v per lane; k > 1: cb, with
-// fresh set while the segment has no threshold yet).
+// of the warp's row segment (k = 1: best / best_v, the same in every lane;
+// k > 1: cb, with fresh set while the segment has no threshold yet).  Every
+// decision that leaves the common path is taken by the whole warp at once
+// (the chunk maximum against the segment's best or threshold), so the warp
+// never diverges over the vectors that cannot enter the top-k.
 template <typename T, bool K1>
 __device__ __forceinline__ ChunkStat sweep_chunk(const uint4* sp, int nvec, int idx_base, int k, uint64_t& best,
                                                  float& best_v, CandBuf& cb, bool& fresh) {
@@ -390,7 +392,7 @@ __device__ __forceinline__ ChunkStat sweep_chunk(const uint4* sp, int nvec, int 
   constexpr int N = Elem<T>::kPerVec;
   const int lane = threadIdx.x & 31;
   // pass 1: the lane's vectors into registers (past the chunk's end: -inf),
-  // their maxima and the lane maximum
+  // their maxima, the lane maximum and the chunk maximum
   uint4 raw[kSwVecPerLane];
   float vmx[kSwVecPerLane];
   float lane_max = -INFINITY;
@@ -401,25 +403,31 @@ __device__ __forceinline__ ChunkStat sweep_chunk(const uint4* sp, int nvec, int 
     vmx[i] = Elem<T>::vec_max(raw[i]);
     lane_max = fmaxf(lane_max, vmx[i]);
   }
+  const float chunk_max = warp_max_f(lane_max);
   if constexpr (K1) {
-    if (lane_max >= best_v) {  // rare once the lane holds a large value
+    if (chunk_max >= best_v) {  // rare once the segment holds a large value
+      uint64_t kl = 0ull;
+      if (lane_max >= best_v) {
 #pragma unroll
-      for (int i = 0; i < kSwVecPerLane; ++i) {
-        if (vmx[i] >= best_v) {
-          float f[N];
-          Elem<T>::unpack(raw[i], f);
+        for (int i = 0; i < kSwVecPerLane; ++i) {
+          if (vmx[i] >= best_v) {
+            float f[N];
+            Elem<T>::unpack(raw[i], f);
 #pragma unroll
-          for (int q = 0; q < N; ++q)
-            if (f[q] > -INFINITY) best = umax64(best, make_key(f[q], idx_base + (lane + 32 * i) * N + q));
+            for (int q = 0; q < N; ++q)
+              if (f[q] > -INFINITY) kl = umax64(kl, make_key(f[q], idx_base + (lane + 32 * i) * N + q));
+          }
         }
       }
+      best = umax64(best, warp_max_u64(kl));
       best_v = best ? key_value(best) : -INFINITY;
     }
   }
-  // pass 2: sum of 2^(x log2(e) - e_ref) with one reference exponent for
-  // the lane's chunk (every term <= 1; the product x log2(e) formed with
-  // log2(e) as a head/tail pair), each vector's terms in fp32, fp64 across
-  const float e_ref = lane_max > -INFINITY ? ceilf(lane_max * kLog2eHi) : -INFINITY;
+  // pass 2: sum of 2^(x log2(e) - e_ref) with one reference exponent for the
+  // chunk, e_ref = ceil(chunk maximum * log2(e)) (every term <= 1; the
+  // product x log2(e) formed with log2(e) as a head/tail pair), each vector's
+  // terms in fp32, fp64 across vectors and lanes
+  const float e_ref = chunk_max > -INFINITY ? ceilf(chunk_max * kLog2eHi) : -INFINITY;
   double acc = 0.0;
   if (e_ref > -INFINITY) {  // else every term is exp(-inf) = 0
     const float2 hi2 = make_float2(kLog2eHi, kLog2eHi), lo2 = make_float2(kLog2eLo, kLog2eLo);
@@ -440,14 +448,9 @@ __device__ __forceinline__ ChunkStat sweep_chunk(const uint4* sp, int nvec, int 
   }
   // this chunk's log-sum-exp partial: a fixed lane order
   ChunkStat cs;
-  {
-    const float e = warp_max_f(e_ref);
-    double sum = acc > 0.0 ? rescale_pow2(acc, e_ref, e) : 0.0;
-    sum = warp_sum_d(sum);
-    cs.e_ref = e;
-    cs.pad = 0;
-    cs.acc = sum;
-  }
+  cs.e_ref = e_ref;
+  cs.pad = 0;
+  cs.acc = warp_sum_d(acc);
   if constexpr (!K1) {
     if (fresh) {
       // k lanes hold an element at or above the k-th largest lane maximum
@@ -455,42 +458,47 @@ __device__ __forceinline__ ChunkStat sweep_chunk(const uint4* sp, int nvec, int 
       cb.tau = t0 > -INFINITY ? ((uint64_t)order_bits(t0) << 32) - 1ull : 0ull;
       fresh = false;
     }
-    // offer this lane's elements above tau, one per lane and round, from
-    // the vectors whose maximum reaches tau's value
     const float tv = cb.tau ? key_value(cb.tau) : -INFINITY;
-    uint32_t fl = 0u;
+    if (chunk_max >= tv) {
+      // offer this lane's elements above tau, one per lane and round, from
+      // the vectors whose maximum reaches tau's value
+      uint32_t fl = 0u;
 #pragma unroll
-    for (int i = 0; i < kSwVecPerLane; ++i)
-      if (lane + 32 * i < nvec && vmx[i] >= tv) fl |= 1u << i;
-    int cq = 0;  // next element of the lowest flagged vector
-    for (;;) {
-      uint64_t key = 0ull;
-      while (fl != 0u) {
-        const int i = __ffs(fl) - 1;
-        const int v = lane + 32 * i;
-        float f[N];
-        Elem<T>::unpack(sp[v], f);
-        int nq = N;
+      for (int i = 0; i < kSwVecPerLane; ++i)
+        if (lane + 32 * i < nvec && vmx[i] >= tv) fl |= 1u << i;
+      int cq = 0;  // next element of the lowest flagged vector
+      for (;;) {
+        uint64_t key = 0ull;
+        while (fl != 0u) {
+          const int i = __ffs(fl) - 1;
+          const int v = lane + 32 * i;
+          float f[N];
+          Elem<T>::unpack(sp[v], f);
+          int nq = N;
 #pragma unroll
-        for (int q = 0; q < N; ++q) {
-          if (key == 0ull && q >= cq && f[q] > -INFINITY) {
-            const uint64_t x = make_key(f[q], idx_base + v * N + q);
-            if (x > cb.tau) {
-              key = x;
-              nq = q + 1;
+          for (int q = 0; q < N; ++q) {
+            if (key == 0ull && q >= cq && f[q] > -INFINITY) {
+              const uint64_t x = make_key(f[q], idx_base + v * N + q);
+              if (x > cb.tau) {
+                key = x;
+                nq = q + 1;
+              }
             }
           }
+          if (key != 0ull && nq < N) {
+            cq = nq;
+            break;
+          }
+          fl &= fl - 1u;
+          cq = 0;
+          if (key != 0ull) break;
         }
-        if (key != 0ull && nq < N) {
-          cq = nq;
-          break;
-        }
-        fl &= fl - 1u;
-        cq = 0;
-        if (key != 0ull) break;
+        if (!__any_sync(kFull, key != 0ull)) break;
+        cb.offer(key, k);
       }
-      if (!__any_sync(kFull, key != 0ull)) break;
-      cb.offer(key, k);
+      // raise the threshold to the k-th key now, so that later chunks of
+      // the segment flag fewer vectors
+      if (cb.cnt > k) cb.select(k);
     }
   }
   return cs;
@@ -499,12 +507,12 @@ __device__ __forceinline__ ChunkStat sweep_chunk(const uint4* sp, int nvec, int 
 // Every warp works alone: its contiguous range of the chunk list streams
 // through a private two-stage ring (lane 0 issues the bulk copies) and each
 // chunk's log-sum-exp partial is a warp reduction written by lane 0.  The
-// running top-k of the warp's row segment: with k = 1 each lane keeps its best
-// key and the warp takes the maximum at the segment's end; with k > 1 the warp
-// buffers candidate keys above a threshold (from the first chunk, the k-th
-// largest lane maximum: k elements reach it) and selects by rank whenever the
-// buffer fills, which raises the threshold to the k-th key; a vector whose
-// maximum is below the threshold is never looked at again.  At the end of a
+// running top-k of the warp's row segment: with k = 1 the warp keeps its best
+// key, looked at again only when a chunk's maximum reaches it; with k > 1 the
+// warp buffers candidate keys above a threshold (from the first chunk, the
+// k-th largest lane maximum: k elements reach it) and selects by rank after
+// every chunk that offered keys, which raises the threshold to the k-th key; a
+// vector whose maximum is below the threshold is never looked at again.  At the end of a
 // row segment the warp writes its list and takes the row's ticket; the warp
 // that completes a row merges it.  No block barrier.
 template <typename T, bool K1>
@@ -550,7 +558,7 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
   if (lane == 0)
     while (issued < nj && issued < S) issue_next();
 
-  uint64_t best = 0ull;      // k = 1: this lane's best key of the segment
+  uint64_t best = 0ull;      // k = 1: the warp's best key of the segment
   float best_v = -INFINITY;  // and its value
   CandBuf cb;                // k > 1: the warp's candidates of the segment
   cb.buf = sh.cand[warp];
@@ -565,8 +573,7 @@ __global__ void __launch_bounds__(kSwThreads, kSwCtasPerSm) row_sweep_kernel(Swe
   auto finish_segment = [&](int c_last) {
     const size_t slot0 = (size_t)seg_row * a.ncpr;
     if constexpr (K1) {
-      const uint64_t w = warp_max_u64(best);
-      if (lane == 0) a.keys[slot0 + c_last] = w;
+      if (lane == 0) a.keys[slot0 + c_last] = best;
       for (int e = lane; e < c_last - seg_c0; e += 32) a.keys[slot0 + seg_c0 + e] = 0ull;
     } else {
       cb.select(k);
@@ -791,8 +798,7 @@ __global__ void __launch_bounds__(kRcThreads, 1) row_cta_kernel(SweepArgs a, int
   }
   uint64_t* my_list = lists + (size_t)(rank * kRcWarps + warp) * EAGLE_MAX_TOPK;
   if constexpr (K1) {
-    const uint64_t w = warp_max_u64(best);
-    if (lane == 0) my_list[0] = w;
+    if (lane == 0) my_list[0] = best;
   } else {
     if (nwc > 0) cb.select(k);
     if (lane < k) my_list[lane] = (nwc > 0 && lane < cb.cnt) ? cb.buf[lane] : 0ull;
