@@ -20,9 +20,10 @@
 // segment's last chunk slot and takes the row's ticket; the warp that
 // completes a row (nobody waits) merges the row's slots and writes the
 // per-row outputs.  Rows that are few and short or long use row_cta_kernel
-// (one row per CTA, no cross-SM merge).  Unaligned rows, and argmax sweeps over
-// many rows, use row_stats_kernel: one CTA per (row, chunk), 16-byte loads
-// when the rows allow them (scalar otherwise), the same ticket merge.
+// (one row per CTA, no cross-SM merge).  Argmax sweeps over many aligned rows
+// use row_argmax_kernel, unaligned rows row_stats_kernel: one CTA per (row,
+// chunk), 16-byte loads when the rows allow them (scalar otherwise), the same
+// ticket merge.
 #include <cooperative_groups.h>
 
 #include "eagle_internal.h"
@@ -273,6 +274,157 @@ row_stats_kernel(const T* __restrict__ x, int V, int chunk_elems, int k, ChunkSt
     if (out.val) out.val[row * k + lane] = merged ? key_value(merged) : -INFINITY;
   }
   if (LSE && out.lse && lane == 0) out.lse[row] = lse;
+}
+
+// ------------------------------------------------- wide argmax (k = 1) sweep
+// The per-(row, chunk) layout of row_stats_kernel for argmax sweeps over many
+// 16-byte aligned rows, with the streaming loop built for throughput: each
+// thread keeps its next four vectors in flight while it works on the current
+// four, and every decision off the common path is taken by the whole warp at
+// once: a vector is looked at again only when some lane's maximum reaches
+// the warp's best value so far, and the warp's log-sum-exp terms share one
+// reference exponent (the ceiling of that best value times log2(e)), so no
+// lane diverges for a new maximum of its own.
+constexpr int kArgPf = 4;  // vectors a thread keeps in flight
+
+template <typename T>
+__global__ void __launch_bounds__(kStatThreads, 4)
+row_argmax_kernel(const T* __restrict__ x, int V, int chunk_elems, ChunkStat* __restrict__ stats,
+                  uint64_t* __restrict__ keys, int* __restrict__ tickets, RowOut out) {
+  using namespace sm100;
+  constexpr int N = Elem<T>::kPerVec;
+  griddep_wait();  // the logits (and this workspace) may belong to the previous kernel
+  const long long row = blockIdx.x;
+  const int chunk = blockIdx.y, n_chunks = gridDim.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c0 = chunk * chunk_elems;
+  const int c1 = min(V, c0 + chunk_elems);
+  const uint4* vp = reinterpret_cast<const uint4*>(x + (size_t)row * (size_t)V + c0);
+  const int nvec = (c1 - c0) / N;
+
+  uint4 cur[kArgPf], nxt[kArgPf];
+  int base = tid;
+#pragma unroll
+  for (int u = 0; u < kArgPf; ++u) {
+    const int vi = base + u * kStatThreads;
+    cur[u] = vi < nvec ? ld_stream(vp + vi) : Elem<T>::neg_inf_vec();
+  }
+  uint64_t best = 0ull;     // the warp's best key (the same in every lane)
+  float tv = -INFINITY;     // its value
+  float wmax;               // the warp's largest value so far
+  float e_ref;              // the warp's reference exponent
+  {
+    float lm = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kArgPf; ++u) lm = fmaxf(lm, Elem<T>::vec_max(cur[u]));
+    wmax = warp_max_f(lm);
+    e_ref = wmax > -INFINITY ? ceilf(wmax * kLog2eHi) : -INFINITY;
+  }
+  double acc = 0.0;
+  const float2 hi2 = make_float2(kLog2eHi, kLog2eHi), lo2 = make_float2(kLog2eLo, kLog2eLo);
+  // the loop test is the warp's (its first lane's): the warp votes inside,
+  // so no lane may leave early; a lane past the end holds -inf vectors
+  for (; base - lane < nvec; base += kStatThreads * kArgPf) {
+    const int nb = base + kStatThreads * kArgPf;
+#pragma unroll
+    for (int u = 0; u < kArgPf; ++u) {
+      const int vi = nb + u * kStatThreads;
+      nxt[u] = vi < nvec ? ld_stream(vp + vi) : Elem<T>::neg_inf_vec();
+    }
+#pragma unroll
+    for (int u = 0; u < kArgPf; ++u) {
+      const float vmax = Elem<T>::vec_max(cur[u]);
+      float f[N];
+      Elem<T>::unpack(cur[u], f);
+      if (__any_sync(kFull, vmax >= tv)) {  // rare once the warp holds a large value
+        uint64_t kl = 0ull;
+        if (vmax >= tv) {
+          const int idx0 = c0 + (base + u * kStatThreads) * N;
+#pragma unroll
+          for (int q = 0; q < N; ++q)
+            if (f[q] > -INFINITY) kl = umax64(kl, make_key(f[q], idx0 + q));
+        }
+        best = umax64(best, warp_max_u64(kl));
+        if (best) {
+          tv = key_value(best);
+          wmax = fmaxf(wmax, tv);
+          const float e_new = ceilf(wmax * kLog2eHi);
+          if (e_new > e_ref) {
+            acc = rescale_pow2(acc, e_ref, e_new);
+            e_ref = e_new;
+          }
+        }
+      }
+      if (e_ref > -INFINITY) {  // until a finite logit arrives every term is exp(-inf) = 0
+        const float2 ne = make_float2(-e_ref, -e_ref);
+        float2 part = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < N; q += 2) {
+          const float2 xq = make_float2(f[q], f[q + 1]);
+          const float2 z = ffma2(xq, lo2, ffma2(xq, hi2, ne));
+          part = fadd2(part, make_float2(ex2_ftz(z.x), ex2_ftz(z.y)));
+        }
+        acc += (double)(part.x + part.y);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kArgPf; ++u) cur[u] = nxt[u];
+  }
+
+  griddep_launch_dependents();  // every CTA that reaches here has done its streaming
+  __shared__ uint64_t s_best[kStatWarps];
+  __shared__ float s_e[kStatWarps];
+  __shared__ double s_s[kStatWarps];
+  __shared__ int s_last;
+  {
+    const double sacc = warp_sum_d(acc);  // e_ref is the same in every lane
+    if (lane == 0) {
+      s_best[warp] = best;
+      s_e[warp] = sacc > 0.0 ? e_ref : -INFINITY;
+      s_s[warp] = sacc;
+    }
+  }
+  __syncthreads();
+  const size_t slot = (size_t)row * n_chunks + chunk;
+  if (tid == 0) {
+    uint64_t m = 0ull;
+    LseAccum a;
+    a.init();
+    for (int w = 0; w < kStatWarps; ++w) {  // a fixed order
+      m = umax64(m, s_best[w]);
+      a.add(s_e[w], s_s[w]);
+    }
+    keys[slot] = m;
+    ChunkStat cs;
+    cs.e_ref = a.e;
+    cs.pad = 0;
+    cs.acc = a.s;
+    stats[slot] = cs;
+    __threadfence();
+    s_last = atomicAdd(tickets + row, 1) == n_chunks - 1;
+  }
+  __syncthreads();
+  // ---- the CTA that completes the row merges all of its chunks
+  if (!s_last || warp != 0) return;
+  __threadfence();
+  const ChunkStat* st = stats + (size_t)row * n_chunks;
+  const unsigned long long* kk = reinterpret_cast<const unsigned long long*>(keys) + (size_t)row * n_chunks;
+  LseAccum a;
+  a.init();
+  uint64_t m = 0ull;
+  for (int c = lane; c < n_chunks; c += 32) {
+    a.add(__ldcg(&st[c].e_ref), __ldcg(&st[c].acc));
+    m = umax64(m, __ldcg(kk + c));
+  }
+  const float e = warp_max_f(a.e);
+  double sum = a.s > 0.0 ? rescale_pow2(a.s, a.e, e) : 0.0;
+  sum = warp_sum_d(sum);
+  m = warp_max_u64(m);
+  if (lane == 0) {
+    if (out.tok) out.tok[row] = m ? key_index(m) : -1;
+    if (out.val) out.val[row] = m ? key_value(m) : -INFINITY;
+    if (out.lse) out.lse[row] = sum > 0.0 ? kLn2 * ((double)e + log2(sum)) : -INFINITY;
+  }
 }
 
 // ------------------------------------------------------ chunked TMA sweep
@@ -1004,10 +1156,9 @@ cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, in
     if (e != cudaSuccess) return e;
   }
   const bool vec = ((uintptr_t)x % 16 == 0) && (((size_t)V * eb) % 16 == 0);
-  // a large argmax sweep (k = 1 over many rows) goes to the per-(row, chunk)
-  // kernel below: its plain 16-byte loads keep more bytes in flight per SM
-  // than the warps' two-stage rings, 80 against 112 us for the 1056 target
-  // rows of the serving mix
+  // a large argmax sweep (k = 1 over many rows) goes to row_argmax_kernel
+  // (one CTA per (row, chunk), plain 16-byte loads four vectors ahead): it
+  // keeps more bytes in flight per SM than the warps' two-stage rings
   const bool wide_argmax = k == 1 && rows >= 4LL * device_sm_count();
   if (vec && (size_t)V * eb <= 0x7fffffffu && !wide_argmax) {
     // the chunked TMA sweep computes the log-sum-exp always (lse == false only drops the output)
@@ -1029,6 +1180,16 @@ cudaError_t launch_row_stats(const void* x, int dtype, long long rows, int V, in
     return k == 1 ? launch_sweep<__nv_bfloat16, true>(a, s, pdl) : launch_sweep<__nv_bfloat16, false>(a, s, pdl);
   }
   const ChunkPlan p = plan_chunks(plan_rows > 0 ? plan_rows : rows, V, eb);
+  if (wide_argmax && vec) {
+    RowOut o = out;
+    if (!lse) o.lse = nullptr;
+    const dim3 grid((unsigned)rows, (unsigned)p.n_chunks);
+    if (dtype == EAGLE_F32)
+      return launch_kernel(row_argmax_kernel<float>, grid, dim3(kStatThreads), 0, s, pdl,
+                           static_cast<const float*>(x), V, p.chunk_elems, stats, keys, tickets, o);
+    return launch_kernel(row_argmax_kernel<__nv_bfloat16>, grid, dim3(kStatThreads), 0, s, pdl,
+                         static_cast<const __nv_bfloat16*>(x), V, p.chunk_elems, stats, keys, tickets, o);
+  }
   if (dtype == EAGLE_F32) return launch_t<float>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s, pdl);
   return launch_t<__nv_bfloat16>(x, rows, V, k, lse, p, vec, stats, keys, tickets, out, s, pdl);
 }

@@ -30,7 +30,7 @@ def _ref_topk(x64: np.ndarray, k: int):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("V,k,rows", [(1000, 2, 5), (32000, 10, 51), (128256, 8, 7), (4099, 5, 3),
                                       (777, 32, 4), (20000, 1, 9), (4000, 6, 3), (128256, 1, 5),
-                                      (32000, 1, 200), (32000, 1, 600)])
+                                      (32000, 1, 200), (32000, 1, 600), (32008, 1, 600)])
 def test_row_stats_topk_and_lse(dtype, V, k, rows):
     rng = np.random.default_rng(V + k)
     x = rng.normal(0, 3, size=(rows, V)).astype(np.float32)
@@ -60,6 +60,32 @@ def test_row_stats_unaligned_rows_and_neg_inf():
     for r in range(6):
         assert tok[r].cpu().numpy().tolist() == _ref_topk(x64[r], k).tolist()
         assert abs(float(lse[r]) - oracle.logsumexp(x64[r])) <= 5e-7
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_row_stats_wide_argmax_edges(dtype):
+    """Argmax over many rows (the wide per-(row, chunk) kernel): a row of -inf
+    only, rows whose first thousands of logits are -inf, a row rising to its
+    maximum at the end (the best value changes at almost every vector), and a
+    vector count per chunk that ends inside a warp."""
+    rng = np.random.default_rng(11)
+    rows, V = 600, 4104
+    x = rng.normal(0, 3, size=(rows, V)).astype(np.float32)
+    x[3, :] = -np.inf
+    x[4, :3000] = -np.inf
+    x[5, :V - 3] = -np.inf
+    x[6] = np.linspace(-20.0, 20.0, V, dtype=np.float32)
+    x[7, 4000] = x[7, 4001] = x[7].max() + 1.0
+    stored = x if dtype == "f32" else bf16_bits_from_f32(x)
+    x64 = oracle.decode_logits(stored, dtype)
+    tok, val, lse = et.row_stats(to_dev_logits(stored, dtype), 1)
+    tok, val, lse = tok.cpu().numpy(), val.cpu().numpy(), lse.cpu().numpy()
+    assert tok[3, 0] == -1 and val[3, 0] == -np.inf and lse[3] == -np.inf
+    for r in range(rows):
+        if r == 3:
+            continue
+        assert tok[r, 0] == _ref_topk(x64[r], 1)[0], f"row {r}"
+        assert abs(lse[r] - oracle.logsumexp(x64[r])) <= 5e-7, f"row {r}"
 
 
 def _check_trees(cfg, seed, gpu_tree, stored):
