@@ -315,6 +315,10 @@ ATTN_TRAFFIC_BYTES = {
     ("l3-8b", 0, "f5510cc048b9f0a0"): 204041984 + 5385472,
     ("serve", 0, "f5510cc048b9f0a0"): 309454080 + 13574400,
     ("long", 0, "f5510cc048b9f0a0"): 194805504 + 3845632,
+    # the serving mix over a paged cache (`--paged 64` / `--paged 16` added to the command above);
+    # ncu printed these two in MB with two decimals, so they are rounded to 10 kB
+    ("serve", 64, "f5510cc048b9f0a0"): 309370000 + 13850000,
+    ("serve", 16, "f5510cc048b9f0a0"): 309470000 + 13980000,
 }
 
 
